@@ -1,0 +1,188 @@
+"""B200 (sm_100a) Gated DeltaNet chunked prefill: Python binding of the C ABI.
+
+Argument marshalling only. Every step of the operator runs in the CUDA kernels
+of the in-tree library libgdn.so (see include/gdn.h); PyTorch provides device
+memory and streams. There is no CPU path: if the library is missing, importing
+works but every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_bwd", "fwd_workspace_size",
+           "bwd_workspace_size", "read_device_status", "Options", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
+
+GDN_F32, GDN_BF16 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace",
+          4: "CUDA runtime error", 5: "device timeout", 6: "inconsistent device input"}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)} (status {code})")
+        self.code = code
+
+
+class Options(ctypes.Structure):
+    """Mirror of gdn_options."""
+    _fields_ = [("cp_segment_chunks", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgdn.so not built ({LIB_PATH}); run "
+                               "`python -m gated_deltanet_chunked_prefill_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        dims = [i] * 7
+        L.gdn_chunk_fwd_workspace_size.argtypes = dims + [vp]
+        L.gdn_chunk_fwd_workspace_size.restype = sz
+        L.gdn_chunk_bwd_workspace_size.argtypes = dims + [vp]
+        L.gdn_chunk_bwd_workspace_size.restype = sz
+        L.gdn_chunk_fwd.argtypes = [i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp, vp, sz,
+                                                    vp, vp]
+        L.gdn_chunk_fwd.restype = i
+        L.gdn_chunk_bwd.argtypes = [i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp,
+                                                    vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+        L.gdn_chunk_bwd.restype = i
+        L.gdn_read_device_status.argtypes = [vp, vp]
+        L.gdn_read_device_status.restype = i
+        L.gdn_status_string.argtypes = [i]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_version.argtypes = []
+        L.gdn_version.restype = i
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported I/O dtype {t.dtype}")
+
+
+def _opts(cp_segment_chunks: int):
+    o = Options()
+    o.cp_segment_chunks = int(cp_segment_chunks)
+    return o
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dims(q, v, cu_seqlens):
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    return B, T, Hqk, Hv, dk, dv, N
+
+
+def fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0) -> int:
+    o = _opts(cp_segment_chunks)
+    return int(lib().gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
+
+
+def bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0) -> int:
+    o = _opts(cp_segment_chunks)
+    return int(lib().gdn_chunk_bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
+
+
+def _check(t, name, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _workspace(nbytes, workspace, device):
+    if workspace is None:
+        return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+    if workspace.numel() < nbytes:
+        raise ValueError(f"workspace too small: {workspace.numel()} < {nbytes}")
+    return workspace
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
+                  output_final_state=True, cp_segment_chunks=0, workspace=None,
+                  o=None, hT=None, stream=None):
+    """Forward through the C ABI. Returns (o, hT or None)."""
+    io = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, n, io)
+    _check(g, "g", torch.float32)
+    _check(h0, "h0", torch.float32)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
+    scale = dk ** -0.5 if scale is None else float(scale)
+    if o is None:
+        o = torch.empty((B, T, Hv, dv), dtype=io, device=q.device)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    ws_bytes = fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks)
+    ws = _workspace(ws_bytes, workspace, q.device)
+    opt = _opts(cp_segment_chunks)
+    st = lib().gdn_chunk_fwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(o),
+                             _ptr(hT), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream(stream))
+    if st != 0:
+        raise GdnError(st, "gdn_chunk_fwd")
+    return o, hT
+
+
+def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlens=None,
+                  cp_segment_chunks=0, workspace=None, want_dh0=True, stream=None):
+    """Backward through the C ABI. Returns dict dq, dk, dv, dg, dbeta, dh0."""
+    io = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta"), (dO, "dO")):
+        _check(t, n, io)
+    _check(g, "g", torch.float32)
+    _check(h0, "h0", torch.float32)
+    _check(dhT, "dhT", torch.float32)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
+    scale = dk ** -0.5 if scale is None else float(scale)
+    dq = torch.empty_like(q)
+    dkk = torch.empty_like(k)
+    dvv = torch.empty_like(v)
+    dg = torch.empty_like(g)
+    db = torch.empty_like(beta)
+    dh0 = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
+    ws_bytes = bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks)
+    ws = _workspace(ws_bytes, workspace, q.device)
+    opt = _opts(cp_segment_chunks)
+    st = lib().gdn_chunk_bwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(dO),
+                             _ptr(dhT), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db),
+                             _ptr(dh0), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream(stream))
+    if st != 0:
+        raise GdnError(st, "gdn_chunk_bwd")
+    return dict(dq=dq, dk=dkk, dv=dvv, dg=dg, dbeta=db, dh0=dh0)
+
+
+def read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and return (and clear) the workspace's device status word."""
+    return int(lib().gdn_read_device_status(_ptr(workspace), _stream(stream)))

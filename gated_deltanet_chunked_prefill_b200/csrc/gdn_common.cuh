@@ -1,0 +1,72 @@
+// Shared host/device definitions of the GDN chunked-prefill library.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+constexpr int kChunk = 64;             // tokens per chunk
+constexpr size_t kStatusBytes = 256;   // head of every workspace: device status word + padding
+
+// Device-side error codes written into the workspace status word (first error wins).
+enum DeviceError : int {
+  kDevOk = 0,
+  kDevTimeout = 1,       // a bounded mbarrier wait gave up
+  kDevBadSeqlens = 2,    // cu_seqlens not monotone / not ending at T
+};
+
+// Everything a forward kernel needs. Pointers are device pointers.
+struct FwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const void* beta;
+  const float* h0;          // nullable, [N,Hv,dk,dv]
+  const int32_t* cu;        // nullable, [N+1]
+  void* o;
+  float* hT;                // nullable
+  int* status;              // device status word
+  int B, T, Hqk, Hv, dk, dv, N;
+  float scale;
+};
+
+__device__ __forceinline__ void record_error(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Token span [s, e) and batch row of sequence n; returns false (after recording an
+// error) when a packed cu_seqlens entry is out of range.
+__device__ __forceinline__ bool seq_span(const FwdParams& p, int n, int& b, int& s, int& e) {
+  if (p.cu == nullptr) {
+    b = n; s = 0; e = p.T;
+    return true;
+  }
+  b = 0;
+  s = p.cu[n];
+  e = p.cu[n + 1];
+  if (s < 0 || e < s || e > p.T) {
+    record_error(p.status, kDevBadSeqlens);
+    return false;
+  }
+  if ((n == 0 && s != 0) || (n == p.N - 1 && e != p.T)) {
+    record_error(p.status, kDevBadSeqlens);
+    return false;
+  }
+  return true;
+}
+
+}  // namespace gdn

@@ -1,0 +1,143 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated DeltaNet chunked-prefill library.
+ *
+ * The operator (named on the pages "Qwen's FlashQLA targets the expensive bit of
+ * long-context AI", section "What happened", and "FlashQLA resource", section 2,
+ * row "What it serves": forward and backward of GDN chunked prefill) is the
+ * gated delta-rule recurrence, per sequence and value head,
+ *
+ *     S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = scale * S_t q_t,
+ *
+ * with S (dv x dk) carried as its transpose h = S^T (dk x dv) in h0 / hT.
+ * The library evaluates it chunk-parallel (64-token chunks, WY/UT transform)
+ * and, for long sequences with few heads, splits a sequence across SMs
+ * ("gate-driven automatic intra-card context parallelism", "FlashQLA resource",
+ * section 3, first row of the feature table), stitching segments exactly through
+ * their affine state maps h_end = M h_start + b.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *     never allocates device memory; scratch space comes from `workspace`,
+ *     whose size the matching *_workspace_size() returns (at least 256 bytes,
+ *     256-byte aligned).
+ *   - Layouts follow the (batch, seqlen, heads, head_dim) convention with the
+ *     last dimension contiguous ("FA4 SM120 bundle" page, API notes on tensor
+ *     layout; packed sequences via cu_seqlens, same page, "Variable-length"):
+ *       q, k  [B, T, Hqk, dk]      v, o, dO  [B, T, Hv, dv]
+ *       g, beta, dg, dbeta [B, T, Hv]
+ *       h0, hT, dhT, dh0 [N, Hv, dk, dv] fp32, N = B (or num_seqs when packed)
+ *     All arrays are dense and contiguous; base pointers 16-byte aligned.
+ *   - Grouped values: Hv must be a multiple of Hqk; v-head j reads q/k head
+ *     j / (Hv / Hqk). dq / dk of a q/k head sum over the v-heads that read it.
+ *   - Packed variable-length input: cu_seqlens (device int32 [num_seqs + 1],
+ *     0 = cu[0] <= cu[1] <= ... <= cu[num_seqs] = T) requires B == 1. Sequences
+ *     never interact. Chunks restart at every sequence start.
+ *   - dtype: GDN_BF16 = q, k, v, beta, o, dO, dq, dk, dv, dbeta in bfloat16;
+ *     GDN_F32 = those in fp32. g, dg, h0, hT, dhT, dh0 are always fp32.
+ *     Internal state and accumulation are fp32 in both cases.
+ *   - dk, dv in {64, 128}; bf16 with dk = dv = 128 runs the tensor-core
+ *     (tcgen05/TMEM/TMA) kernels; every other supported case runs the fp32
+ *     CUDA-core kernels. Anything else returns GDN_ERR_UNSUPPORTED.
+ *   - Calls are asynchronous on `stream` and never synchronise. Arguments are
+ *     validated on the host before anything is launched; an invalid call
+ *     returns an error status and touches no output. Errors a kernel detects
+ *     (an inconsistent cu_seqlens, a bounded wait that timed out) are recorded
+ *     in the workspace's status word and reported by gdn_read_device_status().
+ *   - Launch failures return GDN_ERR_CUDA.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,     /* bad shape, null required pointer, misaligned pointer, bad cu_seqlens */
+  GDN_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. dk = 96)                             */
+  GDN_ERR_WORKSPACE = 3,       /* workspace null, too small or misaligned                              */
+  GDN_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed                                 */
+  GDN_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait gave up (reported via the status word)       */
+  GDN_ERR_DEVICE_INPUT = 6     /* a kernel found device-side input inconsistent (cu_seqlens)          */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Optional knobs; pass NULL for the defaults (all zero). */
+typedef struct {
+  /* Intra-card context parallelism: 0 = automatic (split long sequences when
+   * (sequences x v-heads) leaves SMs idle), -1 = off, n > 0 = segments of n
+   * chunks (64 tokens each). */
+  int cp_segment_chunks;
+  /* Reserved, must be 0. */
+  int reserved[7];
+} gdn_options;
+
+/* Bytes of device workspace gdn_chunk_fwd needs for these sizes and options. */
+size_t gdn_chunk_fwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv,
+                                    int num_seqs, const gdn_options* opt);
+
+/*
+ * Forward. Computes o [B,T,Hv,dv] (dtype) and, if hT != NULL, the final state
+ * of every (sequence, v-head) in hT [N,Hv,dk,dv] fp32.
+ *   q, k, v, beta : dtype;  g : fp32 raw per-token log-decay (<= 0 in GDN,
+ *                   not required); scale : multiplies S_t q_t (usually dk^-0.5)
+ *   h0            : nullable, [N,Hv,dk,dv] fp32 (NULL = zero initial state)
+ *   cu_seqlens    : nullable device int32 [num_seqs+1] (NULL = B independent
+ *                   sequences of length T; num_seqs is then ignored)
+ *   workspace     : device scratch of >= gdn_chunk_fwd_workspace_size() bytes
+ */
+gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
+                         const void* q, const void* k, const void* v,
+                         const float* g, const void* beta, float scale,
+                         const float* h0, const int32_t* cu_seqlens, int num_seqs,
+                         void* o, float* hT,
+                         void* workspace, size_t workspace_bytes,
+                         const gdn_options* opt, cudaStream_t stream);
+
+/* Bytes of device workspace gdn_chunk_bwd needs for these sizes and options. */
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv,
+                                    int num_seqs, const gdn_options* opt);
+
+/*
+ * Backward ("FlashQLA resource", section 5: backward and its intra-card
+ * sequence parallelism). Given the forward inputs and the incoming gradients
+ * dO [B,T,Hv,dv] (dtype) and dhT (nullable, [N,Hv,dk,dv] fp32), writes
+ *   dq, dk [B,T,Hqk,dk] (dtype; summed over the v-heads sharing a q/k head),
+ *   dv [B,T,Hv,dv] (dtype), dg [B,T,Hv] fp32 (w.r.t. the raw per-token g),
+ *   dbeta [B,T,Hv] (dtype), dh0 (nullable) [N,Hv,dk,dv] fp32.
+ * The forward is recomputed inside the call (nothing is cached between calls).
+ */
+gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
+                         const void* q, const void* k, const void* v,
+                         const float* g, const void* beta, float scale,
+                         const float* h0, const int32_t* cu_seqlens, int num_seqs,
+                         const void* dO, const float* dhT,
+                         void* dq, void* dk_out, void* dv_out, float* dg, void* dbeta,
+                         float* dh0,
+                         void* workspace, size_t workspace_bytes,
+                         const gdn_options* opt, cudaStream_t stream);
+
+/* Synchronises `stream`, then returns (and clears) the status word that the
+ * kernels of earlier calls on this workspace recorded: GDN_OK,
+ * GDN_ERR_DEVICE_TIMEOUT or GDN_ERR_DEVICE_INPUT. GDN_ERR_CUDA if the stream
+ * itself reports an error. */
+gdn_status gdn_read_device_status(void* workspace, cudaStream_t stream);
+
+/* Static, human-readable text of a status code. */
+const char* gdn_status_string(gdn_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

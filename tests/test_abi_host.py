@@ -1,0 +1,82 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+entry point include/gdn.h declares, and rejects invalid calls before launching
+anything. Only calls that fail host validation are made here (no kernel runs).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_deltanet_chunked_prefill_b200 as gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+FAKE = 0x7F0000000000        # 16-byte aligned address that is never dereferenced
+MISALIGNED = FAKE + 8
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = gdn.lib()
+    names = declared_functions()
+    assert "gdn_chunk_fwd" in names and "gdn_chunk_bwd" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version():
+    L = gdn.lib()
+    for code in range(7):
+        assert L.gdn_status_string(code)
+    assert L.gdn_version() >= 100
+
+
+def test_workspace_size_has_status_head():
+    for dims in [(1, 256, 2, 2, 64, 64, 1), (4, 4096, 16, 16, 128, 128, 4),
+                 (1, 32768, 16, 32, 128, 128, 1), (1, 65536, 16, 16, 128, 128, 24)]:
+        assert gdn.fwd_workspace_size(*dims) >= 256
+        assert gdn.bwd_workspace_size(*dims) >= 256
+        assert gdn.fwd_workspace_size(*dims) % 256 == 0
+
+
+def _fwd(dtype=1, B=1, T=64, Hqk=1, Hv=1, dk=128, dv=128, q=FAKE, k=FAKE, v=FAKE, g=FAKE,
+         beta=FAKE, h0=None, cu=None, N=1, o=FAKE, hT=None, ws=FAKE, wsb=1 << 20, opt=None):
+    L = gdn.lib()
+    vp = ctypes.c_void_p
+    o_ = gdn.Options() if opt is None else opt
+    return L.gdn_chunk_fwd(dtype, B, T, Hqk, Hv, dk, dv, vp(q), vp(k), vp(v), vp(g), vp(beta),
+                           0.1, vp(h0) if h0 else None, vp(cu) if cu else None, N, vp(o),
+                           vp(hT) if hT else None, vp(ws) if ws else None, wsb, ctypes.byref(o_),
+                           None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), 1), (dict(T=-1), 1), (dict(Hqk=3, Hv=4), 1), (dict(Hqk=0), 1),
+    (dict(dk=96), 2), (dict(dv=32), 2), (dict(dtype=7), 1),
+    (dict(q=None), 1), (dict(o=None), 1), (dict(g=MISALIGNED), 1), (dict(h0=MISALIGNED), 1),
+    (dict(ws=None), 3), (dict(wsb=16), 3), (dict(ws=MISALIGNED), 3),
+    (dict(cu=FAKE, B=2, N=2), 1), (dict(cu=FAKE, N=0), 1),
+])
+def test_forward_rejects_invalid_arguments(kw, code):
+    assert _fwd(**kw) == code
+
+
+def test_forward_rejects_reserved_options():
+    o = gdn.Options()
+    o.reserved[3] = 1
+    assert _fwd(opt=o) == 1
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
+    g = torch.zeros(1, 64, 1)
+    with pytest.raises(ValueError):
+        gdn.gdn_chunk_fwd(x, x, x, g, torch.zeros(1, 64, 1, dtype=torch.bfloat16))

@@ -1,0 +1,136 @@
+"""GPU parity of gdn_chunk_fwd against the fp64 oracle, through the C ABI."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import gated_deltanet_chunked_prefill_b200 as gdn
+from gated_deltanet_chunked_prefill_b200.workloads import CONFIGS, config_inputs, make_inputs
+from oracle import fwd_chunk, fwd_token
+
+from _helpers import assert_close, oracle_unit_fwd, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # name: (B, T, Hqk, Hv, dk, dv, dtype, h0_std, lengths)
+    "tiny_fp32_full": (1, 256, 2, 2, 64, 64, "f32", None, None),
+    "f32_d128_ragged": (2, 200, 2, 2, 128, 128, "f32", 0.1, None),
+    "f32_d64_gqa_varlen": (1, 0, 1, 2, 64, 64, "f32", 0.1, [1, 63, 64, 65, 130]),
+    "bf16_d128_ragged": (2, 300, 2, 2, 128, 128, "bf16", 0.1, None),
+    "bf16_d128_gqa": (1, 257, 2, 4, 128, 128, "bf16", None, None),
+    "bf16_d128_varlen": (1, 0, 2, 2, 128, 128, "bf16", 0.1, [1, 64, 65, 130, 7, 200]),
+    "bf16_d64": (1, 190, 2, 2, 64, 64, "bf16", 0.1, None),
+    "bf16_d128_long": (1, 1100, 1, 1, 128, 128, "bf16", 0.1, None),
+}
+
+
+def run_gpu(x, **kw):
+    d = to_dev(x)
+    o, hT = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
+                              d["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    return o.cpu(), hT.cpu()
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_fwd_small_parity(name):
+    B, T, Hqk, Hv, dk, dv, dt, h0, lengths = SMALL[name]
+    x = make_inputs(B, T, Hqk, Hv, dk, dv, dt, seed=zlib.crc32(name.encode()) % 1000, h0_std=h0, lengths=lengths)
+    o, hT = run_gpu(x)
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"],
+                       x["cu_seqlens"], chunk=64)
+    assert_close(o, ro, dt, f"{name} o")
+    assert_close(hT, rh, dt, f"{name} hT")
+
+
+@pytest.mark.parametrize("cp", [-1, 1, 2, 3])
+def test_fwd_context_parallel_matches_oracle(cp):
+    """Forced segment lengths (1..3 chunks) against the oracle, odd segment boundaries."""
+    x = make_inputs(1, 0, 2, 4, 128, 128, "bf16", seed=77, h0_std=0.1,
+                    lengths=[700, 64, 1, 333, 129])
+    o, hT = run_gpu(x, cp_segment_chunks=cp)
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"],
+                       x["cu_seqlens"], chunk=64)
+    assert_close(o, ro, "bf16", f"cp={cp} o")
+    assert_close(hT, rh, "bf16", f"cp={cp} hT")
+
+
+def test_fwd_weak_decay_long_sequence():
+    """g close to 0: the state remembers across many chunks (and CP segments)."""
+    x = make_inputs(1, 2000, 1, 2, 128, 128, "bf16", seed=5, h0_std=0.1, g_scale=1.0)
+    x["g"] = (x["g"] * 0.01).contiguous()
+    for cp in (-1, 4):
+        o, hT = run_gpu(x, cp_segment_chunks=cp)
+        ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"],
+                           None, chunk=64)
+        assert_close(o, ro, "bf16", f"weak decay cp={cp} o")
+        assert_close(hT, rh, "bf16", f"weak decay cp={cp} hT")
+
+
+def test_fwd_no_cross_sequence_leakage():
+    lengths = [100, 64, 37, 200]
+    x = make_inputs(1, 0, 2, 2, 128, 128, "bf16", seed=9, h0_std=0.1, lengths=lengths)
+    o1, h1 = run_gpu(x)
+    cu = x["cu_seqlens"].tolist()
+    m = 1                                       # perturb sequence 1 only
+    y = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    s, e = cu[m], cu[m + 1]
+    for name in ("q", "k", "v"):
+        y[name][:, s:e] = -y[name][:, s:e]
+    y["g"][:, s:e] = y["g"][:, s:e] * 0.5
+    y["beta"][:, s:e] = 1 - y["beta"][:, s:e]
+    y["h0"][m] = 3.0
+    o2, h2 = run_gpu(y)
+    for n in range(len(lengths)):
+        if n == m:
+            continue
+        a, b = cu[n], cu[n + 1]
+        assert torch.equal(o1[:, a:b], o2[:, a:b]), n
+        assert torch.equal(h1[n], h2[n]), n
+    assert not torch.equal(o1[:, s:e], o2[:, s:e])
+
+
+def test_fwd_empty_and_zero_length_sequences():
+    x = make_inputs(1, 0, 1, 1, 128, 128, "bf16", seed=3, h0_std=0.1, lengths=[0, 70, 0])
+    o, hT = run_gpu(x)
+    ro, rh = fwd_token(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"],
+                       x["cu_seqlens"])
+    assert_close(o, ro, "bf16", "o")
+    assert torch.equal(hT[0], x["h0"][0]) and torch.equal(hT[2], x["h0"][2])
+
+
+def test_fwd_bad_cu_seqlens_reports_device_status():
+    x = make_inputs(1, 0, 1, 1, 128, 128, "bf16", seed=4, h0_std=None, lengths=[64, 64])
+    d = to_dev(x)
+    d["cu_seqlens"] = torch.tensor([0, 100, 64], dtype=torch.int32, device="cuda")  # not monotone
+    ws = torch.zeros(gdn.fwd_workspace_size(1, 128, 1, 1, 128, 128, 2), dtype=torch.uint8,
+                     device="cuda")
+    gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, d["cu_seqlens"],
+                      workspace=ws)
+    assert gdn.read_device_status(ws) == 6
+    assert gdn.read_device_status(ws) == 0          # reading clears it
+
+
+# ---------------------------------------------------------------- full-size configurations
+FULL = {
+    "dense_bf16": [(0, 0), (3, 15), (1, 7)],
+    "long_gqa_bf16": [(0, 0), (0, 31), (0, 18)],
+    "varlen_bf16": None,   # sampled below: the longest, the shortest, a ragged one
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_fwd_full_size_sampled_units(name):
+    x = config_inputs(name)
+    o, hT = run_gpu(x)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+    units = FULL[name]
+    if units is None:
+        L = np.diff(x["cu_seqlens"].numpy())
+        units = [(int(np.argmax(L)), 3), (int(np.argmin(L)), 11), (5, 0)]
+    for n, j in units:
+        ro, rh, (b, s, e) = oracle_unit_fwd(x, n, j)
+        assert_close(o[b, s:e, j], ro, "bf16", f"{name} unit ({n},{j}) o")
+        assert_close(hT[n, j], rh, "bf16", f"{name} unit ({n},{j}) hT")
