@@ -25,7 +25,10 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "wo
 
 class GdnError(RuntimeError):
     def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {STATUS.get(code, code)} (status {code})")
+        detail = ""
+        if code == 4 and _lib is not None:
+            detail = " -- " + _lib.gdn_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS.get(code, code)} (status {code}){detail}")
         self.code = code
 
 
@@ -61,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_read_device_status.restype = i
         L.gdn_status_string.argtypes = [i]
         L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_last_error.argtypes = []
+        L.gdn_last_error.restype = ctypes.c_char_p
         L.gdn_version.argtypes = []
         L.gdn_version.restype = i
         _lib = L

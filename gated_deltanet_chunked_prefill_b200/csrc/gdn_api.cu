@@ -1,7 +1,9 @@
 // C-ABI entry points: argument validation, workspace layout, planning, launches.
+#include <cstdio>
 #include <cstring>
 
 #include "gdn_common.cuh"
+#include "gdn_tc.cuh"
 
 namespace gdn {
 cudaError_t launch_fwd_simt(const FwdParams& p, bool bf16, cudaStream_t st);
@@ -12,6 +14,13 @@ using namespace gdn;
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
+
+thread_local char g_last_error[256] = "";
+
+gdn_status cuda_fail(const char* where, cudaError_t err) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(err), (int)err);
+  return GDN_ERR_CUDA;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -32,13 +41,14 @@ gdn_status check_shape(int B, int T, int Hqk, int Hv, int dk, int dv, int num_se
   return GDN_OK;
 }
 
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
 extern "C" {
 
 int gdn_version(void) { return kVersion; }
+
+const char* gdn_last_error(void) { return g_last_error; }
 
 const char* gdn_status_string(gdn_status s) {
   switch (s) {
@@ -87,8 +97,19 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   p.B = s.B; p.T = s.T; p.Hqk = s.Hqk; p.Hv = s.Hv; p.dk = s.dk; p.dv = s.dv; p.N = s.N;
   p.scale = scale;
 
-  cudaError_t err = launch_fwd_simt(p, dtype == GDN_BF16, stream);
-  return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  if (s.T == 0) return GDN_OK;
+  cudaError_t err;
+  if (dtype == GDN_BF16 && dk == 128 && dv == 128) {
+    TcPlan plan{};
+    plan.kind = kPlanUnits;
+    const char* what = "";
+    err = launch_fwd_tc(p, plan, s.N * s.Hv, stream, &what);
+    if (err != cudaSuccess) return cuda_fail(what, err);
+  } else {
+    err = launch_fwd_simt(p, dtype == GDN_BF16, stream);
+    if (err != cudaSuccess) return cuda_fail("CUDA-core forward", err);
+  }
+  return GDN_OK;
 }
 
 size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs,

@@ -1,0 +1,628 @@
+// Tensor-core (tcgen05 / TMEM / TMA) forward of the GDN chunked prefill for bf16 I/O,
+// dk = dv = 128, 64-token chunks. One CTA runs the whole chunk sequence of one work
+// item (a (sequence, v-head) unit, or one segment of it under context parallelism).
+//
+// The recurrence is carried as S = h^T (dv x dk, fp32, in the epilogue threads'
+// registers) so that every tensor-core product has M = 128 rows = the dv rows of S
+// (or the 128 stacked K;Q token rows of the Gram product). Per chunk (gam = chunk-local
+// inclusive cumsum of g, E_ij = exp(gam_i - gam_j)):
+//
+//   prep warpgroup (state independent, overlaps the previous chunk's chain):
+//     G  = [K;Q] K^T                               tcgen05, M=128 N=64 K=128
+//     L  = strict_lower(diag(beta) KK^T * E),  A = (I + L)^-1      (fp32, CUDA cores)
+//     A2 = A diag(beta) -> bf16;   P = lower_incl(QK^T * E) -> bf16;  Q <- diag(exp(gam)) Q
+//   epilogue warpgroups (the sequential chain):
+//     (a) D1 = S_bf16 [K ; Q~]^T                   tcgen05, M=128 N=128 K=128
+//     (b) Y^T = V^T - D1[:, K part] diag(exp(gam))  -> bf16
+//     (c) Dl  = Y^T A2^T                           tcgen05, M=128 N=64 K=64   (= Delta^T)
+//     (d) Delta^T -> bf16, Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
+//     (e) D1[:, Q part] += Delta^T P^T;  DS = Delta~^T K   (K read MN-major from the TMA tile)
+//     (f) S = exp(gam_n) S + DS (fp32);  O = scale * D1[:, Q part]
+// i.e. O = scale[diag(e^gam) Q h + (QK^T*E*M) Delta], Delta = A diag(beta)(V - diag(e^gam) K h),
+// h' = e^gam_n h + (diag(e^(gam_n-gam)) K)^T Delta: the WY/UT chunk form of the gated delta
+// rule ("FlashQLA resource", section 3: fused warp-specialised kernels that overlap data
+// movement, tensor-core and CUDA-core work).
+#include <cudaTypedefs.h>
+
+#include "gdn_common.cuh"
+#include "gdn_tc.cuh"
+#include "tc_ptx.cuh"
+
+namespace gdn {
+using namespace tc;
+
+namespace {
+
+constexpr int kThreads = 384;             // 12 warps
+constexpr int kPrepWarp0 = 0;             // warps 0-3: prep (TMEM lane quadrants 0..3)
+constexpr int kEpiWarp0 = 4;              // warps 4-11: epilogue (2 x 4 quadrants); its first
+                                          // thread also issues the TMA loads and the chain MMAs
+constexpr int kNumPrep = 128, kNumEpi = 256;
+constexpr int kBarPrep = 1, kBarEpi = 2;  // named barrier ids
+
+// shared memory layout (bytes from a 1024-aligned base)
+constexpr uint32_t kStageBytes = 48u * 1024u;   // [K0 Q0 K1 Q1] (8KB each) + [V0 V1]
+constexpr uint32_t kOffV = 32u * 1024u;         // within a stage
+constexpr uint32_t kOffA2 = 96u * 1024u;        // 2 x 8KB  A diag(beta), bf16, SW128 rows
+constexpr uint32_t kOffP = 112u * 1024u;        // 2 x 8KB  masked decayed QK^T, bf16
+constexpr uint32_t kOffSb = 128u * 1024u;       // 32KB     S in bf16 (two 64-col sub-tiles)
+constexpr uint32_t kOffYt = 160u * 1024u;       // 16KB     Y^T, then Delta^T
+constexpr uint32_t kOffDt = 176u * 1024u;       // 16KB     Delta~^T, then O staging
+constexpr uint32_t kOffLf = 192u * 1024u;       // fp32 [64][65] L, inverted in place
+constexpr int kLd = 65;
+constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
+
+struct Small {
+  float gam[2][64];
+  float eg[2][64];    // exp(gam)
+  float egd[2][64];   // exp(gam_n - gam)
+  float bet[2][64];
+  float egn[2];       // exp(gam_n)
+  int nv[2];
+  float Xf[16 * 49];  // inverse scratch
+  uint64_t full[2], prep_full[2], gdone, mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small) + 1024;  // + alignment slack
+
+// TMEM columns (fp32, 128 lanes)
+constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T
+constexpr uint32_t kColD1 = 64;   // 128: S [K;Q~]^T, Q part accumulates Delta^T P^T
+constexpr uint32_t kColDd = 192;  // 64: Delta^T
+constexpr uint32_t kColDS = 256;  // 128: Delta~^T K
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kIdG = idesc_bf16(128, 64, false, false);
+constexpr uint32_t kIdA = idesc_bf16(128, 128, false, false);
+constexpr uint32_t kIdC = idesc_bf16(128, 64, false, false);
+constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);
+
+__device__ __forceinline__ float bf16_at(const uint8_t* p) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+}
+
+// 16-byte chunk of 8 bf16 values, scaled
+__device__ __forceinline__ uint4 scale_chunk(uint4 v, float f) {
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 x = __bfloat1622float2(h[i]);
+    h[i] = __floats2bfloat162_rn(x.x * f, x.y * f);
+  }
+  return v;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p, const TcPlan plan) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Small* ss = reinterpret_cast<Small*>(sm + kOffSmall);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  WorkItem it;
+  if (!get_work_item(p, plan, blockIdx.x, it)) return;   // uniform over the CTA
+  const int nchunks = (it.e - it.s + kChunk - 1) / kChunk;
+  const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ss->full[s], 1);
+      mbar_init(&ss->prep_full[s], 1);
+    }
+    mbar_init(&ss->gdone, 1);
+    mbar_init(&ss->mma_done, 1);
+    ss->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kPrepWarp0) {
+    tmem_alloc(&ss->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == kEpiWarp0 * 32) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ss->tmem_base;
+  volatile int* abort_flag = &ss->abort_flag;
+  const uint32_t sbase = smem_u32(sm);
+
+  // Every role keeps executing its loop (and its named barriers) after an aborted
+  // wait, with the work skipped: a role never leaves its peers stuck at a barrier.
+  // TMA loads of chunk c into stage c % 2 (issued by the epilogue's first thread: chunks
+  // 0 and 1 at the start, chunk c + 2 as soon as chunk c has released its stage).
+  const uint32_t stage_bytes = it.zero_v ? 32u * 1024u : kStageBytes;
+  auto load_chunk = [&](int c) {
+    const int s = c & 1;
+    const int row = it.b * p.T + it.s + c * kChunk;
+    uint8_t* st = sm + s * kStageBytes;
+    mbar_arrive_expect_tx(&ss->full[s], stage_bytes);
+    tma_load_3d(st + 0, &tm_k, &ss->full[s], 0, it.hq, row);
+    tma_load_3d(st + 8192, &tm_q, &ss->full[s], 0, it.hq, row);
+    tma_load_3d(st + 16384, &tm_k, &ss->full[s], 64, it.hq, row);
+    tma_load_3d(st + 24576, &tm_q, &ss->full[s], 64, it.hq, row);
+    if (!it.zero_v) {
+      tma_load_3d(st + kOffV, &tm_v, &ss->full[s], 0, it.j, row);
+      tma_load_3d(st + kOffV + 8192, &tm_v, &ss->full[s], 64, it.j, row);
+    }
+  };
+
+  if (warp < kEpiWarp0) {
+    // ------------------------------------------------------------ prep warpgroup
+    const int pt = threadIdx.x;            // 0..127
+    const int pw = warp;                   // TMEM lane quadrant
+    float* Lf = reinterpret_cast<float*>(sm + kOffLf);
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      const int t0 = it.s + c * kChunk;
+      const int nv = min(kChunk, it.e - t0);
+      uint8_t* st = sm + s * kStageBytes;
+      // g, beta of the chunk (masked beyond the sequence end)
+      float gv = 0.f, bv = 0.f;
+      if (pt < kChunk && pt < nv) {
+        const size_t gi = (size_t)(it.b * p.T + t0 + pt) * p.Hv + it.j;
+        gv = p.g[gi];
+        bv = __bfloat162float(beta[gi]);
+      }
+      ok = ok && mbar_wait(&ss->full[s], (c >> 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (pt < kChunk) {
+        ss->gam[s][pt] = gv;
+        ss->bet[s][pt] = bv;
+      }
+      if (nv < kChunk) {
+        // rows past the sequence end hold the next sequence's tokens: clear them
+        const int tiles = it.zero_v ? 4 : 6;
+        for (int idx = pt; idx < (kChunk - nv) * tiles * 8; idx += kNumPrep) {
+          const int r = nv + idx / (tiles * 8), rem = idx % (tiles * 8), tile = rem / 8, ch = rem % 8;
+          const uint32_t off = (tile < 4 ? tile * 8192u : kOffV + (tile - 4) * 8192u) + r * 128u + ch * 16u;
+          *reinterpret_cast<uint4*>(st + off) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(kBarPrep, kNumPrep);
+      if (pt == 0 && ok) {
+        tc_fence_after();
+        const uint32_t a0 = sbase + s * kStageBytes;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+          umma_f16(tmem + kColG, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off, 16, 1024), kIdG, ks > 0);
+        }
+        umma_commit(&ss->gdone);
+      }
+      if (pw == 0) {  // inclusive cumsum of g (two values per lane)
+        const float a0 = ss->gam[s][2 * lane], a1 = ss->gam[s][2 * lane + 1];
+        const float pair = a0 + a1;
+        float run = pair;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, run, off);
+          if (lane >= off) run += y;
+        }
+        ss->gam[s][2 * lane] = run - pair + a0;
+        ss->gam[s][2 * lane + 1] = run;
+      }
+      named_bar_sync(kBarPrep, kNumPrep);
+      const float gn = ss->gam[s][kChunk - 1];
+      if (pt < kChunk) {
+        ss->eg[s][pt] = __expf(ss->gam[s][pt]);
+        ss->egd[s][pt] = __expf(gn - ss->gam[s][pt]);
+      }
+      if (pt == 0) {
+        ss->egn[s] = __expf(gn);
+        ss->nv[s] = nv;
+      }
+      ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      {
+        // rows 0..63 of G: K K^T -> L (fp32);  rows 64..127: Q K^T -> P (bf16)
+        const int rr = 32 * pw + lane;
+        float vals[64];
+        if (ok) {
+          tmem_ld32_sync(tmem + ((uint32_t)(32 * pw) << 16) + kColG, vals);
+          tmem_ld32_sync(tmem + ((uint32_t)(32 * pw) << 16) + kColG + 32, vals + 32);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) vals[j] = 0.f;
+        }
+        const float* gam = ss->gam[s];
+        if (rr < kChunk) {
+          const int i = rr;
+          const float gi = gam[i], bi = ss->bet[s][i];
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j)
+            Lf[i * kLd + j] = (j < i) ? bi * vals[j] * __expf(gi - gam[j]) : 0.f;
+        } else {
+          const int i = rr - kChunk;
+          const float gi = gam[i];
+          const uint32_t prow = sbase + kOffP + s * 8192u;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int j0 = ch * 8 + 2 * u, j1 = j0 + 1;
+              const float p0 = (j0 <= i) ? vals[j0] * __expf(gi - gam[j0]) : 0.f;
+              const float p1 = (j1 <= i) ? vals[j1] * __expf(gi - gam[j1]) : 0.f;
+              w[u] = pack_bf16(p0, p1);
+            }
+            st_shared_v4(prow + sw128(i, ch), w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      named_bar_sync(kBarPrep, kNumPrep);
+      // Q <- diag(exp(gam)) Q, in place (the Gram product has consumed Q)
+      {
+        const int i = pt >> 1, half = pt & 1;
+        uint8_t* row = st + 8192 + half * 16384 + i * 128;
+        const float f = ss->eg[s][i];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4* q16 = reinterpret_cast<uint4*>(row + ch * 16);
+          *q16 = scale_chunk(*q16, f);
+        }
+      }
+      // A = (I + L)^-1: 16x16 diagonal blocks by forward substitution (one warp each) ...
+      {
+        const int R = pw, col = lane & 15;
+        float a[16];
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) {
+          float acc = (ii == col) ? 1.f : 0.f;
+#pragma unroll
+          for (int jj = 0; jj < ii; ++jj) acc -= Lf[(16 * R + ii) * kLd + 16 * R + jj] * a[jj];
+          a[ii] = (ii < col) ? 0.f : acc;
+        }
+        __syncwarp();
+        if (lane < 16) {
+#pragma unroll
+          for (int ii = 0; ii < 16; ++ii) Lf[(16 * R + ii) * kLd + 16 * R + col] = a[ii];
+        }
+      }
+      named_bar_sync(kBarPrep, kNumPrep);
+      // ... then block rows R = 1..3: A[R, <R] = -D_R (L[R, <R] A[<R, <R])
+      {
+        const int r = pt & 15, cg = pt >> 4;
+        float* Xf = ss->Xf;
+#pragma unroll
+        for (int R = 1; R < 4; ++R) {
+          const int ncol = 16 * R;
+          float acc[6];
+#pragma unroll
+          for (int m = 0; m < 6; ++m) acc[m] = 0.f;
+          const float* lrow = Lf + (16 * R + r) * kLd;
+          for (int kk = 0; kk < ncol; ++kk) {
+            const float l = lrow[kk];
+            const float* arow = Lf + kk * kLd + cg;
+#pragma unroll
+            for (int m = 0; m < 6; ++m)
+              if (m < 2 * R) acc[m] += l * arow[8 * m];
+          }
+#pragma unroll
+          for (int m = 0; m < 6; ++m)
+            if (m < 2 * R) Xf[r * 49 + cg + 8 * m] = acc[m];
+          named_bar_sync(kBarPrep, kNumPrep);
+          const float* drow = Lf + (16 * R + r) * kLd + 16 * R;
+#pragma unroll
+          for (int m = 0; m < 6; ++m) acc[m] = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < 16; ++kk) {
+            const float d = drow[kk];
+#pragma unroll
+            for (int m = 0; m < 6; ++m)
+              if (m < 2 * R) acc[m] += d * Xf[kk * 49 + cg + 8 * m];
+          }
+#pragma unroll
+          for (int m = 0; m < 6; ++m)
+            if (m < 2 * R) Lf[(16 * R + r) * kLd + cg + 8 * m] = -acc[m];
+          named_bar_sync(kBarPrep, kNumPrep);
+        }
+      }
+      // A2 = A diag(beta) -> bf16, 128B-swizzled rows
+      {
+        const int i = pt >> 1, half = pt & 1;
+        const uint32_t arow = sbase + kOffA2 + s * 8192u;
+        const float* bet = ss->bet[s];
+#pragma unroll
+        for (int ch4 = 0; ch4 < 4; ++ch4) {
+          const int ch = half * 4 + ch4;
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j0 = ch * 8 + 2 * u;
+            w[u] = pack_bf16(Lf[i * kLd + j0] * bet[j0], Lf[i * kLd + j0 + 1] * bet[j0 + 1]);
+          }
+          st_shared_v4(arow + sw128(i, ch), w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(kBarPrep, kNumPrep);
+      if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: the state chain
+    const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..255
+    const int ew = et >> 5;
+    const int qd = ew & 3, hh = ew >> 2;
+    const int r = 32 * qd + lane;                 // dv row of S (= TMEM lane)
+    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+    float S[64];                                  // S[r][hh*64 + d]
+    if (it.init_mode == kInitPtr) {
+#pragma unroll
+      for (int d = 0; d < 64; ++d) S[d] = it.init[(size_t)(hh * 64 + d) * 128 + r];
+    } else if (it.init_mode == kInitIdentity) {
+#pragma unroll
+      for (int d = 0; d < 64; ++d) S[d] = (hh * 64 + d == r) ? 1.f : 0.f;
+    } else {
+#pragma unroll
+      for (int d = 0; d < 64; ++d) S[d] = 0.f;
+    }
+    auto write_sb = [&]() {
+      const uint32_t base = sbase + kOffSb + hh * 16384u;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        st_shared_v4(base + sw128(r, ch), pack_bf16(S[ch * 8 + 0], S[ch * 8 + 1]),
+                     pack_bf16(S[ch * 8 + 2], S[ch * 8 + 3]), pack_bf16(S[ch * 8 + 4], S[ch * 8 + 5]),
+                     pack_bf16(S[ch * 8 + 6], S[ch * 8 + 7]));
+    };
+    write_sb();
+    fence_proxy_async_smem();
+    named_bar_sync(kBarEpi, kNumEpi);
+    uint32_t mph = 0;
+    auto issue_a = [&](int c) {
+      tc_fence_after();
+      const uint32_t a0 = sbase + kOffSb, b0 = sbase + (c & 1) * kStageBytes;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+        umma_f16(tmem + kColD1, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024), kIdA, ks > 0);
+      }
+      umma_commit(&ss->mma_done);
+    };
+    bool ok = true;
+    int loaded = 0;                               // chunks whose loads were issued (et == 0)
+    if (et == 0) {
+      for (; loaded < 2 && loaded < nchunks; ++loaded) load_chunk(loaded);
+    }
+    if (nchunks > 0 && et == 0) {
+      ok = mbar_wait(&ss->prep_full[0], 0, abort_flag);
+      if (ok) issue_a(0);
+    }
+    auto wait_mma = [&]() {
+      ok = ok && mbar_wait(&ss->mma_done, mph, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      mph ^= 1;
+      tc_fence_after();
+    };
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      ok = ok && mbar_wait(&ss->prep_full[s], (c >> 1) & 1, abort_flag);
+      wait_mma();
+      const uint8_t* st = sm + s * kStageBytes;
+      // (b) Y^T = V^T - (S K^T) diag(exp(gam))
+      {
+        float y[32];
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColD1 + hh * 32, y);
+        else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) y[u] = 0.f;
+        }
+        const uint8_t* vt = st + kOffV + (r >> 6) * 8192;
+        const int rc = (r & 63) >> 3, rb = (r & 7) * 2;
+        const float* eg = ss->eg[s];
+        uint32_t w[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j0 = hh * 32 + 2 * u, j1 = j0 + 1;
+          float v0 = 0.f, v1 = 0.f;
+          if (!it.zero_v) {
+            v0 = bf16_at(vt + j0 * 128 + ((rc ^ (j0 & 7)) << 4) + rb);
+            v1 = bf16_at(vt + j1 * 128 + ((rc ^ (j1 & 7)) << 4) + rb);
+          }
+          w[u] = pack_bf16(v0 - eg[j0] * y[2 * u], v1 - eg[j1] * y[2 * u + 1]);
+        }
+        const uint32_t yrow = sbase + kOffYt;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          st_shared_v4(yrow + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarEpi, kNumEpi);
+      // (c) Delta^T = Y^T (A diag(beta))^T
+      if (et == 0 && ok) {
+        tc_fence_after();
+        const uint32_t a0 = sbase + kOffYt, b0 = sbase + kOffA2 + s * 8192u;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          umma_f16(tmem + kColDd, sdesc_sw128(a0 + ks * 32, 16, 1024), sdesc_sw128(b0 + ks * 32, 16, 1024), kIdC,
+                   ks > 0);
+        umma_commit(&ss->mma_done);
+      }
+      wait_mma();
+      // (d) Delta^T and Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
+      {
+        float dd[32];
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColDd + hh * 32, dd);
+        else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) dd[u] = 0.f;
+        }
+        const float* egd = ss->egd[s];
+        uint32_t w[16], x[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j0 = hh * 32 + 2 * u;
+          w[u] = pack_bf16(dd[2 * u], dd[2 * u + 1]);
+          x[u] = pack_bf16(dd[2 * u] * egd[j0], dd[2 * u + 1] * egd[j0 + 1]);
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          st_shared_v4(sbase + kOffYt + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+          st_shared_v4(sbase + kOffDt + sw128(r, hh * 4 + c4), x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarEpi, kNumEpi);
+      // (e) O part += Delta^T P^T;  DS = Delta~^T K
+      if (et == 0 && ok) {
+        tc_fence_after();
+        const uint32_t ya = sbase + kOffYt, pb = sbase + kOffP + s * 8192u;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          umma_f16(tmem + kColD1 + 64, sdesc_sw128(ya + ks * 32, 16, 1024), sdesc_sw128(pb + ks * 32, 16, 1024), kIdC,
+                   1);
+        const uint32_t da = sbase + kOffDt, kb = sbase + s * kStageBytes;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          umma_f16(tmem + kColDS, sdesc_sw128(da + ks * 32, 16, 1024), sdesc_sw128(kb + ks * 2048, 16384, 1024),
+                   kIdE2, ks > 0);
+        umma_commit(&ss->mma_done);
+      }
+      wait_mma();
+      // (f) S = exp(gam_n) S + DS;  O = scale * (Q part)
+      float oo[32];
+      const int nv = ss->nv[s];
+      {
+        const float egn = ss->egn[s];
+        float ds[32];
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColDS + hh * 64, ds);
+        else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) ds[u] = 0.f;
+        }
+#pragma unroll
+        for (int d = 0; d < 32; ++d) S[d] = fmaf(egn, S[d], ds[d]);
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColDS + hh * 64 + 32, ds);
+#pragma unroll
+        for (int d = 0; d < 32; ++d) S[32 + d] = fmaf(egn, S[32 + d], ds[d]);
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColD1 + 64 + hh * 32, oo);
+        else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) oo[u] = 0.f;
+        }
+      }
+      write_sb();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarEpi, kNumEpi);
+      if (et == 0) {
+        if (c + 2 < nchunks && ok) {                // stage s fully consumed: refill it
+          load_chunk(c + 2);
+          loaded = c + 3;
+        }
+        if (c + 1 < nchunks && ok) {
+          ok = mbar_wait(&ss->prep_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag);
+          if (ok) issue_a(c + 1);
+        }
+      }
+      // O staging (row j = token, 256 B per row) then coalesced 16-byte stores
+      if (it.write_o) {
+        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sm + kOffDt);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) stg[(hh * 32 + jj) * 128 + r] = __float2bfloat16_rn(p.scale * oo[jj]);
+      }
+      named_bar_sync(kBarEpi, kNumEpi);
+      if (it.write_o && ok) {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.o);
+        const int t0 = it.s + c * kChunk;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int idx = et + k4 * kNumEpi;
+          const int j = idx >> 4, ch = idx & 15;
+          if (j < nv) {
+            const uint4 val = *reinterpret_cast<const uint4*>(sm + kOffDt + j * 256 + ch * 16);
+            *reinterpret_cast<uint4*>(o + ((size_t)(it.b * p.T + t0 + j) * p.Hv + it.j) * 128 + ch * 8) = val;
+          }
+        }
+      }
+      named_bar_sync(kBarEpi, kNumEpi);
+    }
+    if (ok && it.fin != nullptr) {
+#pragma unroll
+      for (int d = 0; d < 64; ++d) it.fin[(size_t)(hh * 64 + d) * 128 + r] = S[d];
+    }
+    if (et == 0 && !ok) {
+      // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
+      for (int c = (loaded >= 2 ? loaded - 2 : 0); c < loaded; ++c) {
+        volatile int never = 0;
+        mbar_wait(&ss->full[c & 1], (c >> 1) & 1, &never);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kPrepWarp0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) record_error(p.status, kDevTimeout);
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [rows, heads, 128] bf16 tensor, boxes of 64 rows x 64 elements of one head, 128B swizzle
+bool make_map(CUtensorMap* m, const void* base, int heads, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)heads * 128 * 2};
+  cuuint32_t box[3] = {64, 1, 64};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st,
+                          const char** what) {
+  if (num_items <= 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv;
+  const long long rows = (long long)p.B * p.T;
+  *what = "tensor map encode";
+  if (!encode_fn()) return cudaErrorSymbolNotFound;
+  if (!make_map(&mq, p.q, p.Hqk, rows) || !make_map(&mk, p.k, p.Hqk, rows) || !make_map(&mv, p.v, p.Hv, rows))
+    return cudaErrorInvalidValue;
+  *what = "shared memory attribute";
+  cudaError_t err = cudaFuncSetAttribute(gdn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+  if (err != cudaSuccess) return err;
+  *what = "tensor-core forward launch";
+  gdn_fwd_tc_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, p, plan);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn

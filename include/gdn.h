@@ -133,6 +133,10 @@ gdn_status gdn_read_device_status(void* workspace, cudaStream_t stream);
 /* Static, human-readable text of a status code. */
 const char* gdn_status_string(gdn_status s);
 
+/* Detail of the last GDN_ERR_CUDA returned on the calling host thread (which call
+ * failed and the CUDA error text); empty if none. Static storage, not to be freed. */
+const char* gdn_last_error(void);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int gdn_version(void);
 
