@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet chunked-prefill operator on B200.
+
+One step = one pass of the operator over one batch of the dense bf16 workload
+(B=4, T=4096, H=16, dk=dv=128): gdn_chunk_fwd, and with STEP = "fwdbwd" also
+gdn_chunk_bwd on the same inputs with incoming gradients dO, dhT (the backward
+recomputes the forward internally). Inputs are synthetic (seeded, see the workloads module)
+and resident in HBM when the timed region starts; the working set is larger
+than the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--mode fwd]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own replica
+(the operator shards by independent (sequence, head) units; no collective on
+the data path) and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_chunked_prefill_b200.workloads import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "GDN chunk fwd/bwd tokens/s and TFLOP/s on 1 B200; % of roofline"
+WORKLOAD = "dense_bf16"
+STEP = "fwd"          # what one step runs: "fwd" or "fwdbwd"
+C = 64
+
+
+def flops(w, fwd=True, bwd=True):
+    """Chunked-algorithm FLOPs: dense GEMMs at 2 flop/MAC, triangular inverse C^3/3 MAC/chunk."""
+    ntok = w.B * w.T
+    gemm_v = 6 * w.dk * w.dv + 2 * C * (w.dk + 2 * w.dv)      # per token per v-head
+    gram = 4 * C * w.dk                                       # per token per q/k head
+    inv = (2.0 / 3.0) * C * C                                 # per token per v-head
+    f = ntok * (w.Hv * (gemm_v + inv) + w.Hqk * gram)
+    b = ntok * (2 * (w.Hv * gemm_v + w.Hqk * gram) + w.Hv * 4 * C * C)
+    return (f if fwd else 0.0) + (b if bwd else 0.0)
+
+
+def alg_bytes(w, fwd=True, bwd=True):
+    """Algorithmic minimum bytes: every input read once, every output written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    ntok = w.B * w.T
+    qk = ntok * w.Hqk * w.dk * es
+    vv = ntok * w.Hv * w.dv * es
+    gb = ntok * w.Hv * (4 + es)
+    st = w.num_seqs * w.Hv * w.dk * w.dv * 4
+    h0 = st if w.h0_std is not None else 0
+    f = 2 * qk + vv + gb + h0 + vv + st                       # q k v g beta h0 | o hT
+    b = 2 * qk + vv + gb + h0 + vv + st + 2 * qk + vv + gb + h0   # + dO dhT | dq dk dv dg dbeta dh0
+    return (f if fwd else 0) + (b if bwd else 0)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) every 20 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.time(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if not inside:
+            inside, window = self.samples, "warmup+timed"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = float(np.median([s[1] for s in inside]))
+        bits = 0
+        for s in inside:
+            bits |= int(s[2])
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(inside), "window": window}
+
+
+def traffic_record(kernel_name, workload):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if its source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        recs = json.load(fh)
+    for r in recs:
+        if r.get("kernel") == kernel_name and r.get("workload") == workload:
+            src = os.path.join(ROOT, r["source"])
+            if not os.path.exists(src):
+                return None
+            with open(src, "rb") as fh:
+                if hashlib.sha256(fh.read()).hexdigest()[:16] != r.get("source_sha256_16"):
+                    return None
+            return float(r["bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------------------------- oracle arm
+def oracle_sample(w, x, mode, budget_s):
+    """Time the fp64 oracle on whole (sequence, head) units of the workload until `budget_s`."""
+    from oracle import bwd_token, fwd_chunk  # the CPU baseline is the oracle as it stands
+    hq_of = lambda j: j // (w.Hv // w.Hqk)
+    units, tok, t0 = 0, 0, time.perf_counter()
+    order = [(n, j) for n in range(w.B) for j in range(w.Hv)]
+    for n, j in order:
+        sl = lambda a, h: a[n:n + 1, :, h:h + 1]
+        q, k, v = sl(x["q"], hq_of(j)), sl(x["k"], hq_of(j)), sl(x["v"], j)
+        g, b = sl(x["g"], j), sl(x["beta"], j)
+        h0 = None if x["h0"] is None else x["h0"][n:n + 1, j:j + 1]
+        fwd_chunk(q, k, v, g, b, x["scale"], h0, chunk=C)
+        if mode == "fwdbwd":
+            bwd_token(q, k, v, g, b, x["scale"], sl(x["dO"], j), h0, x["dhT"][n:n + 1, j:j + 1])
+        units += 1
+        tok += w.T
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    # one workload token carries all Hv heads: unit-tokens / Hv = workload tokens
+    return (tok / w.Hv) / el, el, units
+
+
+def run_reference(args, w, x):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cores = 1
+    per_step = []
+    for _ in range(args.warmup):
+        oracle_sample(w, x, args.mode, budget_s=0.0)
+    for _ in range(args.steps):
+        v, el, units = oracle_sample(w, x, args.mode, budget_s=0.0)
+        per_step.append(el)
+    tok = w.T / w.Hv
+    value = tok * len(per_step) / sum(per_step)
+    sample = f"one (sequence, head) unit of {w.T} tokens per step ({args.mode}), fp64 numpy oracle"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": 1e3 * sum(per_step) / len(per_step), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.description + f"; step = {args.mode}", "mode": args.mode},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--mode", default=STEP, choices=["fwd", "fwdbwd"])
+    ap.add_argument("--single", action="store_true",
+                    help="only warm-up steps plus one step, no report (for profiler launch lists)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=list(CONFIGS))
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
+    ap.add_argument("--cp", type=int, default=0, help="cp_segment_chunks option (0 = automatic)")
+    args = ap.parse_args()
+
+    w = CONFIGS[args.workload]
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed, h0_std=w.h0_std,
+                        backward=True)
+        run_reference(args, w, x)
+        return
+
+    import gated_deltanet_chunked_prefill_b200 as gdn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed + 17 * rank, h0_std=w.h0_std,
+                    backward=True)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    stream = torch.cuda.current_stream(dev)
+
+    mode = args.mode
+
+    ws_f = torch.zeros(gdn.fwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp),
+                       dtype=torch.uint8, device=dev)
+    ws_b = torch.zeros(gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp),
+                       dtype=torch.uint8, device=dev)
+    o = torch.empty_like(d["v"])
+    hT = torch.empty((w.num_seqs, w.Hv, w.dk, w.dv), dtype=torch.float32, device=dev)
+
+    def step(dd):
+        gdn.gdn_chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["scale"], dd["h0"],
+                          cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT)
+        if mode == "fwdbwd":
+            return gdn.gdn_chunk_bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["dO"], dd["scale"],
+                                     dd["h0"], dd["dhT"], cp_segment_chunks=args.cp, workspace=ws_b)
+        return None
+
+    # ---- device-resident timing
+    for _ in range(max(args.warmup, 3)):
+        step(d)
+    torch.cuda.synchronize()
+    if args.single:
+        step(d)
+        torch.cuda.synchronize()
+        return
+    if dist:
+        dist.barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    n0 = gdn.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    tw0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(d)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    tw1 = time.time()
+    if dist:
+        dist.barrier()
+    sampler.stop()
+    launches = gdn.launch_count() - n0
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    tokens = w.B * w.T * world
+    value = tokens / (ms_step / 1e3)
+
+    # ---- per-kernel times (CUDA events on the launch stream, library-recorded)
+    per_kernel = {}
+    with gdn.KernelTrace(capacity=64) as tr:
+        for _ in range(5):
+            step(d)
+    for name, t in tr.launches:
+        per_kernel.setdefault(name, []).append(t)
+    fwd_ms = bwd_ms = None
+    with gdn.KernelTrace(capacity=64) as trf:
+        for _ in range(5):
+            gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
+                              cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT)
+    fwd_ms = sum(t for _, t in trf.launches) / 5
+    if mode == "fwdbwd":
+        bwd_ms = sum(t for _, t in tr.launches) / 5 - fwd_ms
+
+    hbm, tc_peak, src = peaks()
+    dom = max(per_kernel, key=lambda k: sum(per_kernel[k]))
+    dom_ms = float(np.mean(per_kernel[dom]))
+    fwd_only_dom = dom in ("gdn_fwd_tc_kernel", "gdn_fwd_simt_kernel")
+    if fwd_only_dom and len(trf.launches) == 5:
+        dom_bytes = alg_bytes(w, fwd=True, bwd=False)
+    else:
+        dom_bytes = alg_bytes(w, fwd=True, bwd=mode == "fwdbwd") / max(1, len(tr.launches) // 5)
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_source": src,
+                "traffic": traffic_record(dom, args.workload),
+                "alg_bytes_per_launch": dom_bytes, "avg_launch_ms": dom_ms}
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    host_in = {k: x[k].pin_memory() for k in ("q", "k", "v", "g", "beta", "h0", "dO", "dhT")
+               if x.get(k) is not None}
+    dev_in = {k: torch.empty_like(d[k]) for k in host_in}
+    dev_in["scale"] = d["scale"]
+    h2d = sum(t.numel() * t.element_size() for k, t in host_in.items()
+              if mode == "fwdbwd" or k not in ("dO", "dhT"))
+    out_host = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                "hT": torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)}
+
+    def e2e_step():
+        for k, t in host_in.items():
+            if mode == "fwdbwd" or k not in ("dO", "dhT"):
+                dev_in[k].copy_(t, non_blocking=True)
+        gr = step(dev_in)
+        out_host["o"].copy_(o, non_blocking=True)
+        out_host["hT"].copy_(hT, non_blocking=True)
+        nbytes = o.numel() * o.element_size() + hT.numel() * 4
+        if gr is not None:
+            for k2, t2 in gr.items():
+                if t2 is None:
+                    continue
+                if k2 not in out_host:
+                    out_host[k2] = torch.empty(t2.shape, dtype=t2.dtype, pin_memory=True)
+                out_host[k2].copy_(t2, non_blocking=True)
+                nbytes += t2.numel() * t2.element_size()
+        return nbytes
+
+    for _ in range(2):
+        d2h = e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 20))
+    if dist:
+        dist.barrier()
+    ev0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e = {"value": tokens / (e_ms / e_steps / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_budget > 0:
+        v_cpu, el, units = oracle_sample(w, x, mode, args.cpu_budget)
+        cpu = {"value": v_cpu, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{units} (sequence, head) units x {w.T} tokens of the same workload "
+                         f"({mode}), fp64 numpy oracle, {el:.1f} s"}
+
+    fl = flops(w, fwd=True, bwd=mode == "fwdbwd") * world
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": w.description, "step": mode, "global_batch": w.B * world,
+                      "seq_len": w.T, "heads_qk": w.Hqk, "heads_v": w.Hv, "dk": w.dk, "dv": w.dv,
+                      "chunk": C, "parallelism": f"replicas x{world}" if world > 1 else "single",
+                      "l2": "working set larger than the 126 MB L2; no flush",
+                      "cp_segment_chunks": args.cp},
+           "tflops": fl / (ms_step / 1e3) / 1e12,
+           "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+           "per_kernel_ms": {k: float(np.mean(v)) for k, v in per_kernel.items()},
+           "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+           "clocks": sampler.summary(tw0, tw1)}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

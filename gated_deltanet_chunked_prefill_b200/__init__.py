@@ -14,7 +14,8 @@ from typing import Optional
 import torch
 
 __all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_bwd", "fwd_workspace_size",
-           "bwd_workspace_size", "read_device_status", "Options", "LIB_PATH"]
+           "bwd_workspace_size", "read_device_status", "Options", "LIB_PATH", "KernelTrace",
+           "launch_count"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
@@ -34,7 +35,8 @@ class GdnError(RuntimeError):
 
 class Options(ctypes.Structure):
     """Mirror of gdn_options."""
-    _fields_ = [("cp_segment_chunks", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+    _fields_ = [("cp_segment_chunks", ctypes.c_int), ("cp_exact", ctypes.c_int),
+                ("reserved", ctypes.c_int * 6)]
 
 
 _lib = None
@@ -66,6 +68,14 @@ def lib() -> ctypes.CDLL:
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_last_error.argtypes = []
         L.gdn_last_error.restype = ctypes.c_char_p
+        L.gdn_trace_begin.argtypes = [i]
+        L.gdn_trace_begin.restype = i
+        L.gdn_trace_end.argtypes = [vp, vp]
+        L.gdn_trace_end.restype = i
+        L.gdn_kernel_name.argtypes = [i]
+        L.gdn_kernel_name.restype = ctypes.c_char_p
+        L.gdn_launch_count.argtypes = []
+        L.gdn_launch_count.restype = ctypes.c_longlong
         L.gdn_version.argtypes = []
         L.gdn_version.restype = i
         _lib = L
@@ -84,9 +94,10 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported I/O dtype {t.dtype}")
 
 
-def _opts(cp_segment_chunks: int):
+def _opts(cp_segment_chunks: int, cp_exact: bool = False):
     o = Options()
     o.cp_segment_chunks = int(cp_segment_chunks)
+    o.cp_exact = int(bool(cp_exact))
     return o
 
 
@@ -102,13 +113,13 @@ def _dims(q, v, cu_seqlens):
     return B, T, Hqk, Hv, dk, dv, N
 
 
-def fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0) -> int:
-    o = _opts(cp_segment_chunks)
+def fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False) -> int:
+    o = _opts(cp_segment_chunks, cp_exact)
     return int(lib().gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
 
 
-def bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0) -> int:
-    o = _opts(cp_segment_chunks)
+def bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False) -> int:
+    o = _opts(cp_segment_chunks, cp_exact)
     return int(lib().gdn_chunk_bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
 
 
@@ -132,7 +143,7 @@ def _workspace(nbytes, workspace, device):
 
 
 def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
-                  output_final_state=True, cp_segment_chunks=0, workspace=None,
+                  output_final_state=True, cp_segment_chunks=0, cp_exact=False, workspace=None,
                   o=None, hT=None, stream=None):
     """Forward through the C ABI. Returns (o, hT or None)."""
     io = q.dtype
@@ -147,9 +158,9 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
         o = torch.empty((B, T, Hv, dv), dtype=io, device=q.device)
     if hT is None and output_final_state:
         hT = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
-    ws_bytes = fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks)
+    ws_bytes = fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact)
     ws = _workspace(ws_bytes, workspace, q.device)
-    opt = _opts(cp_segment_chunks)
+    opt = _opts(cp_segment_chunks, cp_exact)
     st = lib().gdn_chunk_fwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                              _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(o),
                              _ptr(hT), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream(stream))
@@ -159,7 +170,7 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
 
 
 def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlens=None,
-                  cp_segment_chunks=0, workspace=None, want_dh0=True, stream=None):
+                  cp_segment_chunks=0, cp_exact=False, workspace=None, want_dh0=True, stream=None):
     """Backward through the C ABI. Returns dict dq, dk, dv, dg, dbeta, dh0."""
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta"), (dO, "dO")):
@@ -176,9 +187,9 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
     dg = torch.empty_like(g)
     db = torch.empty_like(beta)
     dh0 = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
-    ws_bytes = bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks)
+    ws_bytes = bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact)
     ws = _workspace(ws_bytes, workspace, q.device)
-    opt = _opts(cp_segment_chunks)
+    opt = _opts(cp_segment_chunks, cp_exact)
     st = lib().gdn_chunk_bwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                              _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(dO),
                              _ptr(dhT), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db),
@@ -186,6 +197,38 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
     if st != 0:
         raise GdnError(st, "gdn_chunk_bwd")
     return dict(dq=dq, dk=dkk, dv=dvv, dg=dg, dbeta=db, dh0=dh0)
+
+
+class KernelTrace:
+    """Context manager: device time of every kernel the library launches inside it.
+
+    After exit, `launches` holds (kernel name, milliseconds) per launch, in order.
+    The library records the CUDA events itself, on each kernel's launch stream.
+    """
+
+    def __init__(self, capacity: int = 256):
+        self.capacity = capacity
+        self.launches = []
+
+    def __enter__(self):
+        st = lib().gdn_trace_begin(self.capacity)
+        if st != 0:
+            raise GdnError(st, "gdn_trace_begin")
+        return self
+
+    def __exit__(self, *exc):
+        ms = (ctypes.c_float * self.capacity)()
+        ids = (ctypes.c_int * self.capacity)()
+        n = lib().gdn_trace_end(ms, ids)
+        if n < 0:
+            raise GdnError(4, "gdn_trace_end")
+        self.launches = [(lib().gdn_kernel_name(ids[i]).decode(), float(ms[i])) for i in range(n)]
+        return False
+
+
+def launch_count() -> int:
+    """Kernels launched by the library from this host thread so far."""
+    return int(lib().gdn_launch_count())
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:

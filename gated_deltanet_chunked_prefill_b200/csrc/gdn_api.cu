@@ -42,9 +42,151 @@ gdn_status check_shape(int B, int T, int Hqk, int Hv, int dk, int dv, int num_se
 }
 
 
+constexpr int kTraceMax = 4096;
+struct Trace {
+  cudaEvent_t events[2 * kTraceMax];
+  int capacity = 0;   // > 0 while a trace is active
+  int count = 0;
+  int ids[kTraceMax];
+};
+thread_local Trace g_trace;
+thread_local long long g_launches = 0;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+bool uses_tc(gdn_dtype dtype, const Shape& s) { return dtype == GDN_BF16 && s.dk == 128 && s.dv == 128; }
+
+// Segment length (chunks) for automatic context parallelism, 0 = none. Independent
+// sequences: the segment count minimising waves x (segment chunks + 1 warm-up chunk),
+// with one CTA per SM per wave. Packed sequences (lengths unknown on the host): segments
+// of 32 chunks once the batch holds at least 128 chunks.
+int auto_segment(const Shape& s, int nch) {
+  const int sms = num_sms();
+  if (s.packed) return nch >= 128 ? 32 : 0;
+  const long long units = (long long)s.N * s.Hv;
+  long long best_cost = -1;
+  int best = 1;
+  for (int nseg = 1; nseg <= 64 && nseg <= nch; ++nseg) {
+    const long long waves = (units * nseg + sms - 1) / sms;
+    const long long cost = waves * ((nch + nseg - 1) / nseg + (nseg > 1 ? 1 : 0));
+    if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = nseg; }
+  }
+  return best > 1 ? (nch + best - 1) / best : 0;
+}
+
+struct FwdPlan {
+  int kind = kPlanUnits;
+  int seg_chunks = 0, max_segs = 0, max_pairs = 0;
+  bool table = false, exact = false;
+  size_t off_table = 0, off_count = 0, off_first = 0, off_state = 0, off_trans = 0, total = kStatusBytes;
+};
+
+FwdPlan plan_forward(gdn_dtype dtype, const Shape& s, const gdn_options* opt) {
+  FwdPlan f;
+  if (!uses_tc(dtype, s) || s.T == 0) return f;
+  const int mode = opt ? opt->cp_segment_chunks : 0;
+  if (mode < 0) return f;
+  const int nch = (s.T + kChunk - 1) / kChunk;
+  const int seg = mode > 0 ? mode : auto_segment(s, nch);
+  if (seg <= 0 || (!s.packed && seg >= nch)) return f;
+  f.seg_chunks = seg;
+  f.exact = opt && opt->cp_exact;
+  f.kind = f.exact ? kPlanCpP3 : kPlanGate;
+  if (s.packed) {
+    f.table = true;
+    f.max_pairs = (nch + s.N + seg - 1) / seg + s.N;
+  } else {
+    f.max_segs = (nch + seg - 1) / seg;
+    f.max_pairs = s.N * f.max_segs;
+  }
+  size_t off = kStatusBytes;
+  if (f.table) {
+    f.off_table = off; off = align256(off + (size_t)f.max_pairs * sizeof(int2));
+    f.off_count = off; off = align256(off + sizeof(int));
+    f.off_first = off; off = align256(off + (size_t)s.N * sizeof(int));
+  }
+  if (f.exact) {
+    const size_t per = (size_t)f.max_pairs * s.Hv * s.dk * s.dv * sizeof(float);
+    f.off_state = off; off = align256(off + per);
+    f.off_trans = off; off = align256(off + per);
+  }
+  f.total = off;
+  return f;
+}
+
 }  // namespace
 
+namespace gdn {
+void trace_pre(int kernel_id, cudaStream_t st) {
+  ++g_launches;
+  Trace& t = g_trace;
+  if (t.count < t.capacity) {
+    t.ids[t.count] = kernel_id;
+    cudaEventRecord(t.events[2 * t.count], st);
+  }
+}
+void trace_post(cudaStream_t st) {
+  Trace& t = g_trace;
+  if (t.count < t.capacity) {
+    cudaEventRecord(t.events[2 * t.count + 1], st);
+    ++t.count;
+  }
+}
+}  // namespace gdn
+
 extern "C" {
+
+gdn_status gdn_trace_begin(int capacity) {
+  Trace& t = g_trace;
+  if (t.capacity > 0 || capacity <= 0 || capacity > kTraceMax) return GDN_ERR_INVALID_ARG;
+  for (int i = 0; i < 2 * capacity; ++i) {
+    cudaError_t err = cudaEventCreate(&t.events[i]);
+    if (err != cudaSuccess) {
+      for (int k = 0; k < i; ++k) cudaEventDestroy(t.events[k]);
+      return cuda_fail("trace event create", err);
+    }
+  }
+  t.capacity = capacity;
+  t.count = 0;
+  return GDN_OK;
+}
+
+int gdn_trace_end(float* ms, int* kernel_ids) {
+  Trace& t = g_trace;
+  const int n = t.count;
+  int ret = n;
+  for (int i = 0; i < n; ++i) {
+    float v = 0.f;
+    if (cudaEventSynchronize(t.events[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&v, t.events[2 * i], t.events[2 * i + 1]) != cudaSuccess)
+      ret = -1;
+    if (ms) ms[i] = v;
+    if (kernel_ids) kernel_ids[i] = t.ids[i];
+  }
+  for (int i = 0; i < 2 * t.capacity; ++i) cudaEventDestroy(t.events[i]);
+  t.capacity = 0;
+  t.count = 0;
+  return ret;
+}
+
+const char* gdn_kernel_name(int kernel_id) {
+  static const char* names[kKernCount] = {"gdn_fwd_tc_kernel",   "gdn_fwd_simt_kernel", "gdn_cp_stitch_kernel",
+                                          "gdn_bwd_tc_kernel",   "gdn_bwd_simt_kernel", "gdn_bwd_reduce_kernel",
+                                          "gdn_cp_plan_kernel"};
+  return (kernel_id >= 0 && kernel_id < kKernCount) ? names[kernel_id] : "unknown";
+}
+
+long long gdn_launch_count(void) { return g_launches; }
 
 int gdn_version(void) { return kVersion; }
 
@@ -65,8 +207,11 @@ const char* gdn_status_string(gdn_status s) {
 
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs,
                                     const gdn_options* opt) {
-  (void)B; (void)T; (void)Hqk; (void)Hv; (void)dk; (void)dv; (void)num_seqs; (void)opt;
-  return kStatusBytes;
+  // sized for both the bf16 tensor-core plan (the larger) and the fp32 path
+  Shape s;
+  const bool packed = num_seqs > 0 && B == 1;
+  if (check_shape(B, T, Hqk, Hv, dk, dv, packed ? num_seqs : 0, packed, s) != GDN_OK) return kStatusBytes;
+  return plan_forward(GDN_BF16, s, opt).total;
 }
 
 gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
@@ -99,11 +244,47 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
 
   if (s.T == 0) return GDN_OK;
   cudaError_t err;
-  if (dtype == GDN_BF16 && dk == 128 && dv == 128) {
+  if (uses_tc(dtype, s)) {
+    const FwdPlan f = plan_forward(dtype, s, opt);
+    if (workspace_bytes < f.total) return GDN_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
     TcPlan plan{};
     plan.kind = kPlanUnits;
+    plan.roles = 1;
     const char* what = "";
-    err = launch_fwd_tc(p, plan, s.N * s.Hv, stream, &what);
+    if (f.kind == kPlanUnits) {
+      err = launch_fwd_tc(p, plan, s.N * s.Hv, stream, &what);
+      if (err != cudaSuccess) return cuda_fail(what, err);
+      return GDN_OK;
+    }
+    plan.seg_chunks = f.seg_chunks;
+    plan.max_segs = f.max_segs;
+    int* first = nullptr;
+    if (f.table) {
+      plan.table = reinterpret_cast<int2*>(ws + f.off_table);
+      plan.table_count = reinterpret_cast<int*>(ws + f.off_count);
+      first = reinterpret_cast<int*>(ws + f.off_first);
+      err = launch_cp_plan(p, f.seg_chunks, f.max_pairs, const_cast<int2*>(plan.table),
+                           const_cast<int*>(plan.table_count), first, stream);
+      if (err != cudaSuccess) return cuda_fail("segment table", err);
+    }
+    if (!f.exact) {
+      plan.kind = kPlanGate;
+      err = launch_fwd_tc(p, plan, f.max_pairs * s.Hv, stream, &what);
+      if (err != cudaSuccess) return cuda_fail(what, err);
+      return GDN_OK;
+    }
+    plan.seg_state = reinterpret_cast<float*>(ws + f.off_state);
+    plan.seg_trans = reinterpret_cast<float*>(ws + f.off_trans);
+    plan.kind = kPlanCpP1;
+    plan.roles = 2;
+    err = launch_fwd_tc(p, plan, f.max_pairs * 2 * s.Hv, stream, &what);
+    if (err != cudaSuccess) return cuda_fail(what, err);
+    plan.roles = 1;
+    err = launch_cp_stitch(p, plan, first, stream);
+    if (err != cudaSuccess) return cuda_fail("segment stitch", err);
+    plan.kind = kPlanCpP3;
+    err = launch_fwd_tc(p, plan, f.max_pairs * s.Hv, stream, &what);
     if (err != cudaSuccess) return cuda_fail(what, err);
   } else {
     err = launch_fwd_simt(p, dtype == GDN_BF16, stream);

@@ -69,4 +69,10 @@ __device__ __forceinline__ bool seq_span(const FwdParams& p, int n, int& b, int&
   return true;
 }
 
+// ---- host-side launch instrumentation (gdn_api.cu)
+enum KernelId : int { kKernFwdTc = 0, kKernFwdSimt = 1, kKernCpStitch = 2, kKernBwdTc = 3,
+                      kKernBwdSimt = 4, kKernBwdReduce = 5, kKernCpPlan = 6, kKernCount = 7 };
+void trace_pre(int kernel_id, cudaStream_t st);
+void trace_post(cudaStream_t st);
+
 }  // namespace gdn

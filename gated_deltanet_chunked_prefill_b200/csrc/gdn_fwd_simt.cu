@@ -185,8 +185,11 @@ static cudaError_t launch_simt_t(const FwdParams& p, cudaStream_t st) {
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid(p.dv / kSimtSlice, p.Hv, p.N);
+  trace_pre(kKernFwdSimt, st);
   kern<<<grid, kSimtThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  err = cudaGetLastError();
+  trace_post(st);
+  return err;
 }
 
 cudaError_t launch_fwd_simt(const FwdParams& p, bool bf16, cudaStream_t st) {

@@ -33,11 +33,11 @@ using namespace tc;
 
 namespace {
 
-constexpr int kThreads = 384;             // 12 warps
-constexpr int kPrepWarp0 = 0;             // warps 0-3: prep (TMEM lane quadrants 0..3)
-constexpr int kEpiWarp0 = 4;              // warps 4-11: epilogue (2 x 4 quadrants); its first
+constexpr int kThreads = 512;             // 16 warps
+constexpr int kEpiWarp0 = 8;              // warps 0-7: prep (TMEM lane quadrant w % 4, column half w / 4)
+                                          // warps 8-15: epilogue (same split); the epilogue's first
                                           // thread also issues the TMA loads and the chain MMAs
-constexpr int kNumPrep = 128, kNumEpi = 256;
+constexpr int kNumPrep = 256, kNumEpi = 256;
 constexpr int kBarPrep = 1, kBarEpi = 2;  // named barrier ids
 
 // shared memory layout (bytes from a 1024-aligned base)
@@ -54,23 +54,26 @@ constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 
 struct Small {
   float gam[2][64];
+  float egt[2][64];   // exp(g_t) of each token (1 past the sequence end)
   float eg[2][64];    // exp(gam)
   float egd[2][64];   // exp(gam_n - gam)
   float bet[2][64];
   float egn[2];       // exp(gam_n)
   int nv[2];
-  float Xf[16 * 49];  // inverse scratch
+  float Xf[8 * 128];      // inverse scratch: one 16 x 8 tile per prep warp
+  float wsum[16];         // warm-up window search: per-warp partial sums
+  int ws;                 // warm-up start token (context parallelism)
   uint64_t full[2], prep_full[2], gdone, mma_done;
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small) + 1024;  // + alignment slack
+constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T
 constexpr uint32_t kColD1 = 64;   // 128: S [K;Q~]^T, Q part accumulates Delta^T P^T
 constexpr uint32_t kColDd = 192;  // 64: Delta^T
-constexpr uint32_t kColDS = 256;  // 128: Delta~^T K
+constexpr uint32_t kColS = 256;   // 128: the fp32 state S (dv x dk), updated in place
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdG = idesc_bf16(128, 64, false, false);
@@ -103,15 +106,22 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p, const TcPlan plan) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Dynamic shared memory starts at the (1024-aligned) base of the CTA's window: the
+  // kernel has no static shared variables. Used directly so every access stays a
+  // shared-space access.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
   Small* ss = reinterpret_cast<Small*>(sm + kOffSmall);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  if ((smem_u32(sm) & 1023u) != 0) {                     // 128B-swizzled tiles need 1024B alignment
+    if (threadIdx.x == 0) record_error(p.status, kDevTimeout);
+    return;
+  }
   WorkItem it;
   if (!get_work_item(p, plan, blockIdx.x, it)) return;   // uniform over the CTA
-  const int nchunks = (it.e - it.s + kChunk - 1) / kChunk;
   const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -121,9 +131,10 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(&ss->gdone, 1);
     mbar_init(&ss->mma_done, 1);
     ss->abort_flag = 0;
+    ss->ws = it.s;
     fence_mbar_init();
   }
-  if (warp == kPrepWarp0) {
+  if (warp == 0) {
     tmem_alloc(&ss->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -135,18 +146,72 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+
+  // Gate-driven warm-up (context parallelism): a segment that starts inside a sequence
+  // begins from a zero state at the start of a window of earlier chunks whose transition
+  // has spectral norm <= prod_t exp(g_t) max(1, |1 - beta_t |k_t|^2|) <= 2^-64: the state
+  // it drops is then below fp32 resolution. Each token's factor is the exact norm of
+  // exp(g)(I - beta k k^T); the window walks back chunk by chunk (at most kMaxWarm chunks,
+  // otherwise the segment starts at the sequence start with h0: the exact recurrence).
+  if (it.gate && it.s > it.seq_s) {
+    const int tok = threadIdx.x >> 3, part = threadIdx.x & 7;   // 64 tokens x 8 threads
+    float logb = 0.f;
+    int start = it.seq_s;
+    for (int m = 1; m <= kMaxWarm; ++m) {
+      const int cs = it.s - m * kChunk;
+      if (cs < it.seq_s) break;
+      const size_t row = (size_t)(it.b * p.T + cs + tok);
+      const uint4* kr = reinterpret_cast<const uint4*>(kg + (row * p.Hqk + it.hq) * 128 + part * 16);
+      float sq = 0.f;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint4 v = kr[u];
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h[e]);
+          sq = fmaf(f.x, f.x, fmaf(f.y, f.y, sq));
+        }
+      }
+      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+      float lt = 0.f;
+      if (part == 0) {
+        const size_t gi = row * p.Hv + it.j;
+        const float bt = __bfloat162float(beta[gi]);
+        lt = p.g[gi] + __logf(fmaxf(1.f, fabsf(1.f - bt * sq)));
+      }
+      lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+      lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+      if (lane == 0) ss->wsum[warp] = lt;           // warp w covers tokens 4w .. 4w + 3
+      __syncthreads();
+      float tot = 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) tot += ss->wsum[u];
+      __syncthreads();
+      logb += tot;
+      if (logb <= kLogWarmBound) { start = cs; break; }
+    }
+    if (threadIdx.x == 0) ss->ws = start;
+    __syncthreads();
+  }
+  const int ws = ss->ws;                          // first token processed (warm-up start)
+  const int nchunks = (it.e - ws + kChunk - 1) / kChunk;
+  const bool from_seq_start = (ws == it.seq_s);
+  const int init_mode = (ws == it.s) ? it.init_mode : (from_seq_start && p.h0 ? (int)kInitPtr : (int)kInitZero);
+  const float* init_ptr = (ws == it.s) ? it.init : p.h0 + ((size_t)it.n * p.Hv + it.j) * (size_t)(128 * 128);
+
   const uint32_t tmem = ss->tmem_base;
   volatile int* abort_flag = &ss->abort_flag;
   const uint32_t sbase = smem_u32(sm);
 
-  // Every role keeps executing its loop (and its named barriers) after an aborted
-  // wait, with the work skipped: a role never leaves its peers stuck at a barrier.
   // TMA loads of chunk c into stage c % 2 (issued by the epilogue's first thread: chunks
   // 0 and 1 at the start, chunk c + 2 as soon as chunk c has released its stage).
   const uint32_t stage_bytes = it.zero_v ? 32u * 1024u : kStageBytes;
   auto load_chunk = [&](int c) {
     const int s = c & 1;
-    const int row = it.b * p.T + it.s + c * kChunk;
+    const int row = it.b * p.T + ws + c * kChunk;
     uint8_t* st = sm + s * kStageBytes;
     mbar_arrive_expect_tx(&ss->full[s], stage_bytes);
     tma_load_3d(st + 0, &tm_k, &ss->full[s], 0, it.hq, row);
@@ -159,15 +224,18 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   };
 
+  // Every role keeps executing its loop (and its named barriers) after an aborted
+  // wait, with the work skipped: a role never leaves its peers stuck at a barrier.
   if (warp < kEpiWarp0) {
-    // ------------------------------------------------------------ prep warpgroup
-    const int pt = threadIdx.x;            // 0..127
-    const int pw = warp;                   // TMEM lane quadrant
+    // ------------------------------------------------------------ prep (8 warps)
+    const int pt = threadIdx.x;            // 0..255
+    const int pw = warp;                   // 0..7
+    const int qd = pw & 3, hc = pw >> 2;   // TMEM lane quadrant, column half
     float* Lf = reinterpret_cast<float*>(sm + kOffLf);
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
-      const int t0 = it.s + c * kChunk;
+      const int t0 = ws + c * kChunk;
       const int nv = min(kChunk, it.e - t0);
       uint8_t* st = sm + s * kStageBytes;
       // g, beta of the chunk (masked beyond the sequence end)
@@ -182,6 +250,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (pt < kChunk) {
         ss->gam[s][pt] = gv;
         ss->bet[s][pt] = bv;
+        ss->egt[s][pt] = fast_exp(gv);
       }
       if (nv < kChunk) {
         // rows past the sequence end hold the next sequence's tokens: clear them
@@ -219,67 +288,90 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       named_bar_sync(kBarPrep, kNumPrep);
       const float gn = ss->gam[s][kChunk - 1];
       if (pt < kChunk) {
-        ss->eg[s][pt] = __expf(ss->gam[s][pt]);
-        ss->egd[s][pt] = __expf(gn - ss->gam[s][pt]);
+        ss->eg[s][pt] = fast_exp(ss->gam[s][pt]);
+        ss->egd[s][pt] = fast_exp(gn - ss->gam[s][pt]);
       }
       if (pt == 0) {
-        ss->egn[s] = __expf(gn);
+        ss->egn[s] = fast_exp(gn);
         ss->nv[s] = nv;
       }
       ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       {
-        // rows 0..63 of G: K K^T -> L (fp32);  rows 64..127: Q K^T -> P (bf16)
-        const int rr = 32 * pw + lane;
-        float vals[64];
+        // G row rr (TMEM lane), columns j0..j0+31. Rows 0..63: K K^T -> L (fp32);
+        // rows 64..127: Q K^T -> P (bf16). E_ij = exp(gam_i - gam_j) (j <= i) is the running
+        // product of exp(g_t) over t = j+1..i, walking j down: one exponential per row
+        // segment instead of one per entry, no overflow, monotone underflow to 0.
+        const int rr = 32 * qd + lane;
+        const int j0 = 32 * hc;
+        float vals[32];
         if (ok) {
-          tmem_ld32_sync(tmem + ((uint32_t)(32 * pw) << 16) + kColG, vals);
-          tmem_ld32_sync(tmem + ((uint32_t)(32 * pw) << 16) + kColG + 32, vals + 32);
+          tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + kColG + j0, vals);
         } else {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) vals[j] = 0.f;
+          for (int j = 0; j < 32; ++j) vals[j] = 0.f;
         }
-        const float* gam = ss->gam[s];
-        if (rr < kChunk) {
-          const int i = rr;
-          const float gi = gam[i], bi = ss->bet[s][i];
+        float et[32];
+        {
+          const float4* e4 = reinterpret_cast<const float4*>(ss->egt[s] + j0);
 #pragma unroll
-          for (int j = 0; j < kChunk; ++j)
-            Lf[i * kLd + j] = (j < i) ? bi * vals[j] * __expf(gi - gam[j]) : 0.f;
+          for (int u = 0; u < 8; ++u) {
+            const float4 t = e4[u];
+            et[4 * u] = t.x; et[4 * u + 1] = t.y; et[4 * u + 2] = t.z; et[4 * u + 3] = t.w;
+          }
+        }
+        const int i = rr & 63;
+        const float gi = ss->gam[s][i];
+        const float glast = ss->gam[s][j0 + 31];
+        float run = 1.f;
+        if (rr < kChunk) {
+          const float bi = ss->bet[s][i];
+#pragma unroll
+          for (int jj = 31; jj >= 0; --jj) {
+            const int j = j0 + jj;
+            if (jj == 31) run = (j >= i) ? 1.f : fast_exp(gi - glast);
+            else run = (j >= i) ? 1.f : run * et[jj + 1];
+            vals[jj] = (j < i) ? bi * vals[jj] * run : 0.f;
+          }
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) Lf[i * kLd + j0 + jj] = vals[jj];
         } else {
-          const int i = rr - kChunk;
-          const float gi = gam[i];
+#pragma unroll
+          for (int jj = 31; jj >= 0; --jj) {
+            const int j = j0 + jj;
+            if (jj == 31) run = (j >= i) ? 1.f : fast_exp(gi - glast);
+            else run = (j >= i) ? 1.f : run * et[jj + 1];
+            vals[jj] = (j <= i) ? vals[jj] * run : 0.f;
+          }
           const uint32_t prow = sbase + kOffP + s * 8192u;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint32_t w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int j0 = ch * 8 + 2 * u, j1 = j0 + 1;
-              const float p0 = (j0 <= i) ? vals[j0] * __expf(gi - gam[j0]) : 0.f;
-              const float p1 = (j1 <= i) ? vals[j1] * __expf(gi - gam[j1]) : 0.f;
-              w[u] = pack_bf16(p0, p1);
-            }
-            st_shared_v4(prow + sw128(i, ch), w[0], w[1], w[2], w[3]);
-          }
+          for (int c4 = 0; c4 < 4; ++c4)
+            st_shared_v4(prow + sw128(i, 4 * hc + c4), pack_bf16(vals[c4 * 8 + 0], vals[c4 * 8 + 1]),
+                         pack_bf16(vals[c4 * 8 + 2], vals[c4 * 8 + 3]), pack_bf16(vals[c4 * 8 + 4], vals[c4 * 8 + 5]),
+                         pack_bf16(vals[c4 * 8 + 6], vals[c4 * 8 + 7]));
         }
       }
       tc_fence_before();
       named_bar_sync(kBarPrep, kNumPrep);
-      // Q <- diag(exp(gam)) Q, in place (the Gram product has consumed Q)
+      // Q <- diag(exp(gam)) Q, in place (the Gram product has consumed Q): 4 x 16 bytes per thread
       {
-        const int i = pt >> 1, half = pt & 1;
-        uint8_t* row = st + 8192 + half * 16384 + i * 128;
-        const float f = ss->eg[s][i];
+        uint4 qv[4];
+        uint8_t* qa[4];
+        float f[4];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4* q16 = reinterpret_cast<uint4*>(row + ch * 16);
-          *q16 = scale_chunk(*q16, f);
+        for (int m = 0; m < 4; ++m) {
+          const int idx = pt + kNumPrep * m;                 // 0..1023
+          const int row = idx >> 4, half = (idx >> 3) & 1, ch = idx & 7;
+          qa[m] = st + 8192 + half * 16384 + row * 128 + ch * 16;
+          f[m] = ss->eg[s][row];
+          qv[m] = *reinterpret_cast<const uint4*>(qa[m]);
         }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(qa[m]) = scale_chunk(qv[m], f[m]);
       }
-      // A = (I + L)^-1: 16x16 diagonal blocks by forward substitution (one warp each) ...
-      {
+      // A = (I + L)^-1: 16x16 diagonal blocks by forward substitution (warps 0..3, one each) ...
+      if (pw < 4) {
         const int R = pw, col = lane & 15;
         float a[16];
 #pragma unroll
@@ -296,60 +388,73 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
       }
       named_bar_sync(kBarPrep, kNumPrep);
-      // ... then block rows R = 1..3: A[R, <R] = -D_R (L[R, <R] A[<R, <R])
+      // ... then block rows R = 1..3: A[R, <R] = -D_R (L[R, <R] A[<R, <R]) in 16 x 8 output
+      // tiles of m16n8k8 tf32 products (warp w takes tile w of each row block).
       {
-        const int r = pt & 15, cg = pt >> 4;
-        float* Xf = ss->Xf;
+        const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
         for (int R = 1; R < 4; ++R) {
-          const int ncol = 16 * R;
-          float acc[6];
+          const int K = 16 * R;
+          const int tile = pw;
+          float y[4] = {0.f, 0.f, 0.f, 0.f};
+          if (tile < 2 * R) {
+            const int n0 = 8 * tile;
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            const float* lr = Lf + (16 * R) * kLd;
 #pragma unroll
-          for (int m = 0; m < 6; ++m) acc[m] = 0.f;
-          const float* lrow = Lf + (16 * R + r) * kLd;
-          for (int kk = 0; kk < ncol; ++kk) {
-            const float l = lrow[kk];
-            const float* arow = Lf + kk * kLd + cg;
+            for (int k0 = 0; k0 < K; k0 += 8) {
+              uint32_t af[4], bf[2];
+              af[0] = to_tf32(lr[gid * kLd + k0 + tig]);
+              af[1] = to_tf32(lr[(gid + 8) * kLd + k0 + tig]);
+              af[2] = to_tf32(lr[gid * kLd + k0 + tig + 4]);
+              af[3] = to_tf32(lr[(gid + 8) * kLd + k0 + tig + 4]);
+              bf[0] = to_tf32(Lf[(k0 + tig) * kLd + n0 + gid]);
+              bf[1] = to_tf32(Lf[(k0 + tig + 4) * kLd + n0 + gid]);
+              mma_tf32_16x8x8(x, af, bf);
+            }
+            float* xw = ss->Xf + pw * 128;
+            xw[gid * 8 + 2 * tig] = x[0];
+            xw[gid * 8 + 2 * tig + 1] = x[1];
+            xw[(gid + 8) * 8 + 2 * tig] = x[2];
+            xw[(gid + 8) * 8 + 2 * tig + 1] = x[3];
+            __syncwarp();
+            const float* dr = Lf + (16 * R) * kLd + 16 * R;
 #pragma unroll
-            for (int m = 0; m < 6; ++m)
-              if (m < 2 * R) acc[m] += l * arow[8 * m];
+            for (int k0 = 0; k0 < 16; k0 += 8) {
+              uint32_t af[4], bf[2];
+              af[0] = to_tf32(dr[gid * kLd + k0 + tig]);
+              af[1] = to_tf32(dr[(gid + 8) * kLd + k0 + tig]);
+              af[2] = to_tf32(dr[gid * kLd + k0 + tig + 4]);
+              af[3] = to_tf32(dr[(gid + 8) * kLd + k0 + tig + 4]);
+              bf[0] = to_tf32(xw[(k0 + tig) * 8 + gid]);
+              bf[1] = to_tf32(xw[(k0 + tig + 4) * 8 + gid]);
+              mma_tf32_16x8x8(y, af, bf);
+            }
           }
-#pragma unroll
-          for (int m = 0; m < 6; ++m)
-            if (m < 2 * R) Xf[r * 49 + cg + 8 * m] = acc[m];
-          named_bar_sync(kBarPrep, kNumPrep);
-          const float* drow = Lf + (16 * R + r) * kLd + 16 * R;
-#pragma unroll
-          for (int m = 0; m < 6; ++m) acc[m] = 0.f;
-#pragma unroll
-          for (int kk = 0; kk < 16; ++kk) {
-            const float d = drow[kk];
-#pragma unroll
-            for (int m = 0; m < 6; ++m)
-              if (m < 2 * R) acc[m] += d * Xf[kk * 49 + cg + 8 * m];
+          named_bar_sync(kBarPrep, kNumPrep);         // every warp is done reading L[R, <R]
+          if (tile < 2 * R) {
+            float* ar = Lf + (16 * R) * kLd + 8 * tile;
+            ar[gid * kLd + 2 * tig] = -y[0];
+            ar[gid * kLd + 2 * tig + 1] = -y[1];
+            ar[(gid + 8) * kLd + 2 * tig] = -y[2];
+            ar[(gid + 8) * kLd + 2 * tig + 1] = -y[3];
           }
-#pragma unroll
-          for (int m = 0; m < 6; ++m)
-            if (m < 2 * R) Lf[(16 * R + r) * kLd + cg + 8 * m] = -acc[m];
           named_bar_sync(kBarPrep, kNumPrep);
         }
       }
-      // A2 = A diag(beta) -> bf16, 128B-swizzled rows
+      // A2 = A diag(beta) -> bf16, 128B-swizzled rows (thread: 16 columns of one row)
       {
-        const int i = pt >> 1, half = pt & 1;
+        const int i = pt >> 2, qq = pt & 3;
         const uint32_t arow = sbase + kOffA2 + s * 8192u;
         const float* bet = ss->bet[s];
+        uint32_t w[8];
 #pragma unroll
-        for (int ch4 = 0; ch4 < 4; ++ch4) {
-          const int ch = half * 4 + ch4;
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j0 = ch * 8 + 2 * u;
-            w[u] = pack_bf16(Lf[i * kLd + j0] * bet[j0], Lf[i * kLd + j0 + 1] * bet[j0 + 1]);
-          }
-          st_shared_v4(arow + sw128(i, ch), w[0], w[1], w[2], w[3]);
+        for (int u = 0; u < 8; ++u) {
+          const int j0 = qq * 16 + 2 * u;
+          w[u] = pack_bf16(Lf[i * kLd + j0] * bet[j0], Lf[i * kLd + j0 + 1] * bet[j0 + 1]);
         }
+        st_shared_v4(arow + sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+        st_shared_v4(arow + sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
       }
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
@@ -362,27 +467,33 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int qd = ew & 3, hh = ew >> 2;
     const int r = 32 * qd + lane;                 // dv row of S (= TMEM lane)
     const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-    float S[64];                                  // S[r][hh*64 + d]
-    if (it.init_mode == kInitPtr) {
-#pragma unroll
-      for (int d = 0; d < 64; ++d) S[d] = it.init[(size_t)(hh * 64 + d) * 128 + r];
-    } else if (it.init_mode == kInitIdentity) {
-#pragma unroll
-      for (int d = 0; d < 64; ++d) S[d] = (hh * 64 + d == r) ? 1.f : 0.f;
-    } else {
-#pragma unroll
-      for (int d = 0; d < 64; ++d) S[d] = 0.f;
-    }
-    auto write_sb = [&]() {
+    const uint32_t s_addr = tmem + lane_base + kColS + hh * 64;   // this thread's 64 columns of S
+    // initial state -> TMEM (fp32) and Sb (bf16)
+    auto write_sb = [&](const float* v, int half32) {
       const uint32_t base = sbase + kOffSb + hh * 16384u;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        st_shared_v4(base + sw128(r, ch), pack_bf16(S[ch * 8 + 0], S[ch * 8 + 1]),
-                     pack_bf16(S[ch * 8 + 2], S[ch * 8 + 3]), pack_bf16(S[ch * 8 + 4], S[ch * 8 + 5]),
-                     pack_bf16(S[ch * 8 + 6], S[ch * 8 + 7]));
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int ch = half32 * 4 + c4;
+        st_shared_v4(base + sw128(r, ch), pack_bf16(v[c4 * 8 + 0], v[c4 * 8 + 1]),
+                     pack_bf16(v[c4 * 8 + 2], v[c4 * 8 + 3]), pack_bf16(v[c4 * 8 + 4], v[c4 * 8 + 5]),
+                     pack_bf16(v[c4 * 8 + 6], v[c4 * 8 + 7]));
+      }
     };
-    write_sb();
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      float v[32];
+#pragma unroll
+      for (int d = 0; d < 32; ++d) {
+        const int col = hh * 64 + h2 * 32 + d;
+        if (init_mode == kInitPtr) v[d] = init_ptr[(size_t)col * 128 + r];
+        else if (init_mode == kInitIdentity) v[d] = (col == r) ? 1.f : 0.f;
+        else v[d] = 0.f;
+      }
+      tmem_st32_sync(s_addr + h2 * 32, v);
+      write_sb(v, h2);
+    }
     fence_proxy_async_smem();
+    tc_fence_before();
     named_bar_sync(kBarEpi, kNumEpi);
     uint32_t mph = 0;
     auto issue_a = [&](int c) {
@@ -395,14 +506,29 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       umma_commit(&ss->mma_done);
     };
+    // S <- exp(gam_n) S in TMEM (before the chunk's update accumulates onto it)
+    auto prescale = [&](int s) {
+      const float egn = ss->egn[s];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float v[32];
+        tmem_ld32_sync(s_addr + h2 * 32, v);
+#pragma unroll
+        for (int d = 0; d < 32; ++d) v[d] *= egn;
+        tmem_st32_sync(s_addr + h2 * 32, v);
+      }
+    };
     bool ok = true;
     int loaded = 0;                               // chunks whose loads were issued (et == 0)
     if (et == 0) {
       for (; loaded < 2 && loaded < nchunks; ++loaded) load_chunk(loaded);
     }
-    if (nchunks > 0 && et == 0) {
+    if (nchunks > 0) {
       ok = mbar_wait(&ss->prep_full[0], 0, abort_flag);
-      if (ok) issue_a(0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (et == 0 && ok) issue_a(0);
+      if (ok) prescale(0);
+      tc_fence_before();
     }
     auto wait_mma = [&]() {
       ok = ok && mbar_wait(&ss->mma_done, mph, abort_flag);
@@ -412,7 +538,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     };
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
-      ok = ok && mbar_wait(&ss->prep_full[s], (c >> 1) & 1, abort_flag);
+      const int t0 = ws + c * kChunk;
       wait_mma();
       const uint8_t* st = sm + s * kStageBytes;
       // (b) Y^T = V^T - (S K^T) diag(exp(gam))
@@ -481,7 +607,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
-      // (e) O part += Delta^T P^T;  DS = Delta~^T K
+      // (e) O part += Delta^T P^T;  S += Delta~^T K   (S was pre-scaled by exp(gam_n))
       if (et == 0 && ok) {
         tc_fence_after();
         const uint32_t ya = sbase + kOffYt, pb = sbase + kOffP + s * 8192u;
@@ -492,57 +618,59 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t da = sbase + kOffDt, kb = sbase + s * kStageBytes;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          umma_f16(tmem + kColDS, sdesc_sw128(da + ks * 32, 16, 1024), sdesc_sw128(kb + ks * 2048, 16384, 1024),
-                   kIdE2, ks > 0);
+          umma_f16(tmem + kColS, sdesc_sw128(da + ks * 32, 16, 1024), sdesc_sw128(kb + ks * 2048, 16384, 1024),
+                   kIdE2, 1);
         umma_commit(&ss->mma_done);
       }
       wait_mma();
-      // (f) S = exp(gam_n) S + DS;  O = scale * (Q part)
+      // (f) S -> bf16 copy for the next chunk's product;  O = scale * (Q part) -> registers
       float oo[32];
       const int nv = ss->nv[s];
       {
-        const float egn = ss->egn[s];
-        float ds[32];
-        if (ok) tmem_ld32_sync(tmem + lane_base + kColDS + hh * 64, ds);
-        else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) ds[u] = 0.f;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          float v[32];
+          if (ok) tmem_ld32_sync(s_addr + h2 * 32, v);
+          else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] = 0.f;
+          }
+          write_sb(v, h2);
         }
-#pragma unroll
-        for (int d = 0; d < 32; ++d) S[d] = fmaf(egn, S[d], ds[d]);
-        if (ok) tmem_ld32_sync(tmem + lane_base + kColDS + hh * 64 + 32, ds);
-#pragma unroll
-        for (int d = 0; d < 32; ++d) S[32 + d] = fmaf(egn, S[32 + d], ds[d]);
         if (ok) tmem_ld32_sync(tmem + lane_base + kColD1 + 64 + hh * 32, oo);
         else {
 #pragma unroll
           for (int u = 0; u < 32; ++u) oo[u] = 0.f;
         }
       }
-      write_sb();
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
-      if (et == 0) {
-        if (c + 2 < nchunks && ok) {                // stage s fully consumed: refill it
+      const bool next = c + 1 < nchunks;
+      if (et == 0 && ok) {
+        if (c + 2 < nchunks) {                      // stage s fully consumed: refill it
           load_chunk(c + 2);
           loaded = c + 3;
         }
-        if (c + 1 < nchunks && ok) {
-          ok = mbar_wait(&ss->prep_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag);
-          if (ok) issue_a(c + 1);
-        }
       }
-      // O staging (row j = token, 256 B per row) then coalesced 16-byte stores
-      if (it.write_o) {
+      if (next) {
+        ok = ok && mbar_wait(&ss->prep_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (et == 0 && ok) issue_a(c + 1);
+      }
+      // O staging (row j = token, 256 B per row) then coalesced 16-byte stores; the
+      // prescale of S for the next chunk overlaps its first product
+      const bool write_o = it.write_o && t0 >= it.s;
+      if (write_o) {
         __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sm + kOffDt);
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) stg[(hh * 32 + jj) * 128 + r] = __float2bfloat16_rn(p.scale * oo[jj]);
       }
+      if (next && ok) prescale((c + 1) & 1);
+      tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
-      if (it.write_o && ok) {
+      if (write_o && ok) {
         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.o);
-        const int t0 = it.s + c * kChunk;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int idx = et + k4 * kNumEpi;
@@ -556,8 +684,14 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       named_bar_sync(kBarEpi, kNumEpi);
     }
     if (ok && it.fin != nullptr) {
+      tc_fence_after();
 #pragma unroll
-      for (int d = 0; d < 64; ++d) it.fin[(size_t)(hh * 64 + d) * 128 + r] = S[d];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float v[32];
+        tmem_ld32_sync(s_addr + h2 * 32, v);
+#pragma unroll
+        for (int d = 0; d < 32; ++d) it.fin[(size_t)(hh * 64 + h2 * 32 + d) * 128 + r] = v[d];
+      }
     }
     if (et == 0 && !ok) {
       // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
@@ -570,7 +704,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kPrepWarp0) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -621,8 +755,11 @@ cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items,
                                          (int)kSmemBytes);
   if (err != cudaSuccess) return err;
   *what = "tensor-core forward launch";
+  trace_pre(kKernFwdTc, st);
   gdn_fwd_tc_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, p, plan);
-  return cudaGetLastError();
+  err = cudaGetLastError();
+  trace_post(st);
+  return err;
 }
 
 }  // namespace gdn

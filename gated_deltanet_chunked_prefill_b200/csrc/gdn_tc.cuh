@@ -17,18 +17,34 @@ enum InitMode : int { kInitZero = 0, kInitPtr = 1, kInitIdentity = 2 };
 //                identity with v = 0 and stores the segment's transition M_s.
 //   kPlanCpP3:   phase 3: per (sequence, v-head, segment) one CTA runs the segment from
 //                its stitched start state and writes o (and hT for the last segment).
-enum PlanKind : int { kPlanUnits = 0, kPlanCpP1 = 1, kPlanCpP3 = 2 };
+//   kPlanGate:   gate-driven context parallelism in one launch: per (sequence, v-head,
+//                segment) one CTA writes o for its segment; it reconstructs its start state
+//                by running, from a zero state, a window of earlier chunks whose decay bound
+//                is below 2^-64 (or from the sequence start when no such window exists
+//                within kMaxWarm chunks).
+enum PlanKind : int { kPlanUnits = 0, kPlanCpP1 = 1, kPlanCpP3 = 2, kPlanGate = 3 };
 
+constexpr int kMaxWarm = 16;                      // longest warm-up window, in chunks
+constexpr float kLogWarmBound = -44.3614195558f;  // ln(2^-64)
+
+// A segment is named by its pair index pi: pi = n * max_segs + seg for B independent
+// sequences, or the position of (n, seg) in a table the plan kernel builds for packed
+// sequences (ordered by n, then seg, so that segment seg + 1 of n is pi + 1).
 struct TcPlan {
   int kind;
   int seg_chunks;        // chunks per segment (CP)
-  int max_segs;          // segment slots per sequence in the workspace
-  float* seg_state;      // [N][Hv][max_segs][dk][dv] fp32: start state of segment s (s >= 1)
-  float* seg_trans;      // [N][Hv][max_segs][dk][dk] fp32: transition M_s of segment s (s >= 1)
+  int max_segs;          // segment slots per sequence (B independent sequences)
+  int roles;             // 2 in phase 1 of the exact stitch, else 1
+  const int2* table;     // nullable: (sequence, segment) per pair index (packed sequences)
+  const int* table_count;
+  float* seg_state;      // [pairs][Hv][dk][dv] fp32: start state of segment pi (exact stitch)
+  float* seg_trans;      // [pairs][Hv][dk][dk] fp32: transition of segment pi (exact stitch)
 };
 
 struct WorkItem {
   int n, j, hq, b, s, e;  // sequence, v-head, q/k head, batch row, token range [s, e)
+  int seq_s;              // first token of the sequence
+  bool gate;              // may start earlier than s with a warm-up window (kPlanGate)
   int init_mode;
   const float* init;      // [dk][dv] fp32 when init_mode == kInitPtr
   float* fin;             // [dk][dv] fp32 destination of the end state, or nullptr
@@ -43,24 +59,35 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
   w.fin = nullptr;
   w.init = nullptr;
   w.init_mode = kInitZero;
+  w.gate = false;
   if (plan.kind == kPlanUnits) {
     w.j = item % p.Hv;
     w.n = item / p.Hv;
     if (!seq_span(p, w.n, w.b, w.s, w.e)) return false;
+    w.seq_s = w.s;
     w.hq = w.j / (p.Hv / p.Hqk);
     if (p.h0) { w.init_mode = kInitPtr; w.init = p.h0 + ((size_t)w.n * p.Hv + w.j) * hsz; }
     if (p.hT) w.fin = p.hT + ((size_t)w.n * p.Hv + w.j) * hsz;
     w.write_o = true;
     return true;
   }
-  // context-parallel plans: item = ((n * Hv + j) * max_segs + seg) * roles + role
-  const int roles = plan.kind == kPlanCpP1 ? 2 : 1;
-  const int role = item % roles;
-  int rest = item / roles;
-  const int seg = rest % plan.max_segs;
-  rest /= plan.max_segs;
-  w.j = rest % p.Hv;
-  w.n = rest / p.Hv;
+  // context-parallel plans: item = (pi * roles + role) * Hv + j (consecutive items are the
+  // v-heads of one segment, so heads that share q/k read the same tiles close in time)
+  w.j = item % p.Hv;
+  const int rest = item / p.Hv;
+  const int role = rest % plan.roles;
+  const int pi = rest / plan.roles;
+  int seg;
+  if (plan.table) {
+    if (pi >= *plan.table_count) return false;
+    const int2 e = plan.table[pi];
+    w.n = e.x;
+    seg = e.y;
+  } else {
+    w.n = pi / plan.max_segs;
+    seg = pi % plan.max_segs;
+    if (w.n >= p.N) return false;
+  }
   int b, s, e;
   if (!seq_span(p, w.n, b, s, e)) return false;
   const int nchunks = (e - s + kChunk - 1) / kChunk;
@@ -68,30 +95,32 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
   const int segs_used = nseg > 0 ? nseg : 1;
   if (seg >= segs_used) return false;
   w.b = b;
+  w.seq_s = s;
   w.hq = w.j / (p.Hv / p.Hqk);
   w.s = s + seg * plan.seg_chunks * kChunk;
   w.e = min(e, w.s + plan.seg_chunks * kChunk);
-  if (w.s > e) w.s = e;
-  const size_t slot = ((size_t)w.n * p.Hv + w.j) * plan.max_segs;
+  const float* h0u = p.h0 ? p.h0 + ((size_t)w.n * p.Hv + w.j) * hsz : nullptr;
   if (plan.kind == kPlanCpP1) {
-    if (seg + 1 >= segs_used) return false;                 // last segment: no transition needed
+    if (seg + 1 >= segs_used) return false;                 // last segment: no map needed
     if (role == 0) {
-      if (seg == 0 && p.h0) { w.init_mode = kInitPtr; w.init = p.h0 + ((size_t)w.n * p.Hv + w.j) * hsz; }
-      w.fin = plan.seg_state + (slot + seg + 1) * hsz;      // b_s lands in the next segment's slot
+      if (seg == 0 && h0u) { w.init_mode = kInitPtr; w.init = h0u; }
+      w.fin = plan.seg_state + ((size_t)(pi + 1) * p.Hv + w.j) * hsz;   // b_seg -> slot of seg + 1
     } else {
       if (seg == 0) return false;                           // segment 0 starts from the known h0
       w.init_mode = kInitIdentity;
       w.zero_v = true;
-      w.fin = plan.seg_trans + (slot + seg) * (size_t)p.dk * p.dk;
+      w.fin = plan.seg_trans + ((size_t)pi * p.Hv + w.j) * (size_t)p.dk * p.dk;
     }
     return true;
   }
-  // phase 3
+  // phase 3 of the exact stitch, or the single launch of the gate-driven plan
+  if (role != 0) return false;
+  w.gate = plan.kind == kPlanGate;
   if (seg == 0) {
-    if (p.h0) { w.init_mode = kInitPtr; w.init = p.h0 + ((size_t)w.n * p.Hv + w.j) * hsz; }
-  } else {
+    if (h0u) { w.init_mode = kInitPtr; w.init = h0u; }
+  } else if (plan.kind == kPlanCpP3) {
     w.init_mode = kInitPtr;
-    w.init = plan.seg_state + (slot + seg) * hsz;
+    w.init = plan.seg_state + ((size_t)pi * p.Hv + w.j) * hsz;
   }
   if (seg + 1 == segs_used && p.hT) w.fin = p.hT + ((size_t)w.n * p.Hv + w.j) * hsz;
   w.write_o = true;
@@ -100,5 +129,10 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
 
 cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st,
                           const char** what);
+// Packed sequences: build the (sequence, segment) table of a segmented plan.
+cudaError_t launch_cp_plan(const FwdParams& p, int seg_chunks, int max_pairs, int2* table, int* count,
+                           int* first_pair, cudaStream_t st);
+// Exact stitch, phase 2: chain the segment maps h_{s+1} = M_s h_s + b_s in place.
+cudaError_t launch_cp_stitch(const FwdParams& p, const TcPlan& plan, const int* first_pair, cudaStream_t st);
 
 }  // namespace gdn

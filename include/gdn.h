@@ -71,12 +71,22 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /* Optional knobs; pass NULL for the defaults (all zero). */
 typedef struct {
-  /* Intra-card context parallelism: 0 = automatic (split long sequences when
-   * (sequences x v-heads) leaves SMs idle), -1 = off, n > 0 = segments of n
-   * chunks (64 tokens each). */
+  /* Intra-card context parallelism (tensor-core path): 0 = automatic (split a
+   * sequence into segments when (sequences x v-heads) leaves SMs idle), -1 = off,
+   * n > 0 = segments of n chunks (64 tokens each). */
   int cp_segment_chunks;
+  /* How a segment obtains its start state.
+   * 0 (default): gate-driven. The segment's CTA runs, from a zero state, the
+   *   shortest window of preceding chunks whose transition has spectral norm
+   *   <= 2^-64 (each token's factor exp(g) max(1, |1 - beta |k|^2|) is exact), so
+   *   the dropped part is below fp32 resolution; with no such window within 16
+   *   chunks it starts at the sequence start (the plain recurrence).
+   * 1: exact affine stitch. Phase 1 computes every segment's map
+   *   h_end = M h_start + b, phase 2 chains the maps, phase 3 reruns each segment
+   *   from its stitched start state. */
+  int cp_exact;
   /* Reserved, must be 0. */
-  int reserved[7];
+  int reserved[6];
 } gdn_options;
 
 /* Bytes of device workspace gdn_chunk_fwd needs for these sizes and options. */
@@ -136,6 +146,22 @@ const char* gdn_status_string(gdn_status s);
 /* Detail of the last GDN_ERR_CUDA returned on the calling host thread (which call
  * failed and the CUDA error text); empty if none. Static storage, not to be freed. */
 const char* gdn_last_error(void);
+
+/*
+ * Instrumentation (host-thread local). gdn_trace_begin() creates 2 * capacity
+ * timing events; while the trace is active every kernel the library launches
+ * from this thread is bracketed by cudaEventRecord on its launch stream (launches
+ * beyond `capacity` are not recorded). gdn_trace_end() waits for the recorded
+ * events, writes each launch's device time in milliseconds to ms[i] and its kernel
+ * id to kernel_ids[i] (both nullable, capacity entries), destroys the events and
+ * returns the number of launches recorded (-1 on a CUDA error).
+ * gdn_kernel_name() names a kernel id; gdn_launch_count() counts every kernel
+ * launched from this thread since the library was loaded.
+ */
+gdn_status gdn_trace_begin(int capacity);
+int gdn_trace_end(float* ms, int* kernel_ids);
+const char* gdn_kernel_name(int kernel_id);
+long long gdn_launch_count(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int gdn_version(void);

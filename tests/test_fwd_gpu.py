@@ -45,12 +45,15 @@ def test_fwd_small_parity(name):
     assert_close(hT, rh, dt, f"{name} hT")
 
 
+@pytest.mark.parametrize("exact", [False, True])
 @pytest.mark.parametrize("cp", [-1, 1, 2, 3])
-def test_fwd_context_parallel_matches_oracle(cp):
-    """Forced segment lengths (1..3 chunks) against the oracle, odd segment boundaries."""
+def test_fwd_context_parallel_matches_oracle(cp, exact):
+    """Forced segment lengths (1..3 chunks), both ways of obtaining a segment's start state
+    (gate-driven window, exact affine stitch), against the oracle; packed sequences put the
+    segment boundaries at odd token positions."""
     x = make_inputs(1, 0, 2, 4, 128, 128, "bf16", seed=77, h0_std=0.1,
                     lengths=[700, 64, 1, 333, 129])
-    o, hT = run_gpu(x, cp_segment_chunks=cp)
+    o, hT = run_gpu(x, cp_segment_chunks=cp, cp_exact=exact)
     ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"],
                        x["cu_seqlens"], chunk=64)
     assert_close(o, ro, "bf16", f"cp={cp} o")
@@ -58,15 +61,40 @@ def test_fwd_context_parallel_matches_oracle(cp):
 
 
 def test_fwd_weak_decay_long_sequence():
-    """g close to 0: the state remembers across many chunks (and CP segments)."""
-    x = make_inputs(1, 2000, 1, 2, 128, 128, "bf16", seed=5, h0_std=0.1, g_scale=1.0)
+    """g close to 0: the state remembers across many chunks (and CP segments); the
+    gate-driven window cannot close, so those segments start at the sequence start."""
+    x = make_inputs(2, 2000, 1, 2, 128, 128, "bf16", seed=5, h0_std=0.1, g_scale=1.0)
     x["g"] = (x["g"] * 0.01).contiguous()
-    for cp in (-1, 4):
-        o, hT = run_gpu(x, cp_segment_chunks=cp)
+    for cp, exact in ((-1, False), (4, False), (4, True), (7, True)):
+        o, hT = run_gpu(x, cp_segment_chunks=cp, cp_exact=exact)
         ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"],
                            None, chunk=64)
-        assert_close(o, ro, "bf16", f"weak decay cp={cp} o")
-        assert_close(hT, rh, "bf16", f"weak decay cp={cp} hT")
+        assert_close(o, ro, "bf16", f"weak decay cp={cp} exact={exact} o")
+        assert_close(hT, rh, "bf16", f"weak decay cp={cp} exact={exact} hT")
+
+
+@pytest.mark.parametrize("exact", [False, True])
+def test_fwd_context_parallel_dense_unit_norm_violation(exact):
+    """Keys far from unit norm (beta |k|^2 > 2): the per-token bound grows instead of
+    decaying, the gate-driven window falls back to the sequence start; still exact."""
+    x = make_inputs(1, 900, 1, 1, 128, 128, "bf16", seed=8, h0_std=0.1)
+    x["k"] = (x["k"].float() * 1.8).to(torch.bfloat16)
+    x["g"] = (x["g"] * 0.2).contiguous()
+    o, hT = run_gpu(x, cp_segment_chunks=3, cp_exact=exact)
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"], None, chunk=64)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(hT, rh, "bf16", "hT")
+
+
+def test_fwd_cp_bit_identical_when_segments_decay():
+    """Strong decay: the gate-driven start state equals the exact one to fp32 resolution."""
+    x = make_inputs(1, 1500, 2, 2, 128, 128, "bf16", seed=12, h0_std=0.1)
+    o0, h0 = run_gpu(x, cp_segment_chunks=-1)
+    o1, h1 = run_gpu(x, cp_segment_chunks=5)
+    o2, h2 = run_gpu(x, cp_segment_chunks=5, cp_exact=True)
+    from _helpers import rel_l2
+    assert rel_l2(o1, o0) < 2e-3 and rel_l2(o2, o0) < 2e-3
+    assert rel_l2(h1, h0) < 2e-3 and rel_l2(h2, h0) < 2e-3
 
 
 def test_fwd_no_cross_sequence_leakage():
