@@ -330,6 +330,8 @@ def main():
                if x.get(k) is not None}
     dev_in = {k: torch.empty_like(d[k]) for k in host_in}
     dev_in["scale"] = d["scale"]
+    for k in ("h0", "dO", "dhT"):
+        dev_in.setdefault(k, None)
     h2d = sum(t.numel() * t.element_size() for k, t in host_in.items()
               if mode == "fwdbwd" or k not in ("dO", "dhT"))
     out_host = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),

@@ -124,6 +124,36 @@ FwdPlan plan_forward(gdn_dtype dtype, const Shape& s, const gdn_options* opt) {
   return f;
 }
 
+struct BwdPlan {
+  FwdPlan chain;                 // gate-driven segments (or none) for the two sequential passes
+  long long total_chunks = 0;    // chunk slots (upper bound for packed sequences)
+  bool grouped = false;
+  size_t off_chunk_off = 0, off_states = 0, off_dstates = 0, off_dq = 0, off_dk = 0, total = kStatusBytes;
+};
+
+BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
+  BwdPlan b;
+  gdn_options o{};
+  if (opt) o = *opt;
+  if (o.cp_exact) o.cp_segment_chunks = -1;   // exact: the sequential passes run unsplit
+  b.chain = plan_forward(GDN_BF16, s, &o);
+  const int nch = (s.T + kChunk - 1) / kChunk;
+  b.total_chunks = s.packed ? (long long)nch + s.N : (long long)s.N * nch;
+  b.grouped = s.Hv != s.Hqk;
+  size_t off = b.chain.total;
+  if (s.packed) { b.off_chunk_off = off; off = align256(off + (size_t)(s.N + 1) * sizeof(int)); }
+  const size_t st = (size_t)b.total_chunks * s.Hv * s.dk * s.dv * 2;
+  b.off_states = off; off = align256(off + st);
+  b.off_dstates = off; off = align256(off + st);
+  if (b.grouped) {
+    const size_t part = (size_t)s.B * s.T * s.Hv * s.dk * sizeof(float);
+    b.off_dq = off; off = align256(off + part);
+    b.off_dk = off; off = align256(off + part);
+  }
+  b.total = off;
+  return b;
+}
+
 }  // namespace
 
 namespace gdn {
@@ -181,8 +211,8 @@ int gdn_trace_end(float* ms, int* kernel_ids) {
 
 const char* gdn_kernel_name(int kernel_id) {
   static const char* names[kKernCount] = {"gdn_fwd_tc_kernel",   "gdn_fwd_simt_kernel", "gdn_cp_stitch_kernel",
-                                          "gdn_bwd_tc_kernel",   "gdn_bwd_simt_kernel", "gdn_bwd_reduce_kernel",
-                                          "gdn_cp_plan_kernel"};
+                                          "gdn_bwd_grad_kernel", "gdn_bwd_simt_kernel", "gdn_bwd_reduce_kernel",
+                                          "gdn_cp_plan_kernel",  "gdn_bwd_chain_kernel"};
   return (kernel_id >= 0 && kernel_id < kKernCount) ? names[kernel_id] : "unknown";
 }
 
@@ -265,7 +295,7 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
       plan.table_count = reinterpret_cast<int*>(ws + f.off_count);
       first = reinterpret_cast<int*>(ws + f.off_first);
       err = launch_cp_plan(p, f.seg_chunks, f.max_pairs, const_cast<int2*>(plan.table),
-                           const_cast<int*>(plan.table_count), first, stream);
+                           const_cast<int*>(plan.table_count), first, nullptr, stream);
       if (err != cudaSuccess) return cuda_fail("segment table", err);
     }
     if (!f.exact) {
@@ -295,8 +325,10 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
 
 size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs,
                                     const gdn_options* opt) {
-  (void)B; (void)T; (void)Hqk; (void)Hv; (void)dk; (void)dv; (void)num_seqs; (void)opt;
-  return kStatusBytes;
+  Shape s;
+  const bool packed = num_seqs > 0 && B == 1;
+  if (check_shape(B, T, Hqk, Hv, dk, dv, packed ? num_seqs : 0, packed, s) != GDN_OK) return kStatusBytes;
+  return plan_backward(s, opt).total;
 }
 
 gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
@@ -305,11 +337,81 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
                          int num_seqs, const void* dO, const float* dhT, void* dq, void* dk_out,
                          void* dv_out, float* dg, void* dbeta, float* dh0, void* workspace,
                          size_t workspace_bytes, const gdn_options* opt, cudaStream_t stream) {
-  (void)dtype; (void)B; (void)T; (void)Hqk; (void)Hv; (void)dk; (void)dv; (void)q; (void)k;
-  (void)v; (void)g; (void)beta; (void)scale; (void)h0; (void)cu_seqlens; (void)num_seqs;
-  (void)dO; (void)dhT; (void)dq; (void)dk_out; (void)dv_out; (void)dg; (void)dbeta; (void)dh0;
-  (void)workspace; (void)workspace_bytes; (void)opt; (void)stream;
-  return GDN_ERR_UNSUPPORTED;
+  if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+  Shape s;
+  gdn_status st = check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, cu_seqlens != nullptr, s);
+  if (st != GDN_OK) return st;
+  if (opt) {
+    for (int r : opt->reserved)
+      if (r != 0) return GDN_ERR_INVALID_ARG;
+  }
+  if (T > 0 && (!q || !k || !v || !g || !beta || !dO || !dq || !dk_out || !dv_out || !dg || !dbeta))
+    return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, dO, dhT, dq, dk_out, dv_out, dg, dbeta, dh0};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (!uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;   // backward: bf16, dk = dv = 128
+  const BwdPlan bp = plan_backward(s, opt);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < bp.total) return GDN_ERR_WORKSPACE;
+  if (s.T == 0) return GDN_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  FwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.h0 = h0; p.cu = cu_seqlens;
+  p.o = nullptr; p.hT = nullptr;
+  p.status = static_cast<int*>(workspace);
+  p.B = s.B; p.T = s.T; p.Hqk = s.Hqk; p.Hv = s.Hv; p.dk = s.dk; p.dv = s.dv; p.N = s.N;
+  p.scale = scale;
+  p.states = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_states);
+  p.chunk_off = s.packed ? reinterpret_cast<int*>(ws + bp.off_chunk_off) : nullptr;
+  __nv_bfloat16* dstates = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_dstates);
+
+  const FwdPlan& f = bp.chain;
+  TcPlan plan{};
+  plan.kind = kPlanUnits;
+  plan.roles = 1;
+  plan.seg_chunks = f.seg_chunks;
+  plan.max_segs = f.max_segs;
+  int items = s.N * s.Hv;
+  cudaError_t err;
+  const char* what = "";
+  if (s.packed || f.kind != kPlanUnits) {
+    int2* table = f.table ? reinterpret_cast<int2*>(ws + f.off_table) : nullptr;
+    int* count = f.table ? reinterpret_cast<int*>(ws + f.off_count) : nullptr;
+    int* first = f.table ? reinterpret_cast<int*>(ws + f.off_first) : nullptr;
+    if (s.packed) {
+      err = launch_cp_plan(p, f.seg_chunks > 0 ? f.seg_chunks : 1, f.max_pairs, table, count, first,
+                           const_cast<int*>(p.chunk_off), stream);
+      if (err != cudaSuccess) return cuda_fail("backward plan", err);
+    }
+    if (f.kind != kPlanUnits) {
+      plan.kind = kPlanGate;
+      plan.table = table;
+      plan.table_count = count;
+      items = f.max_pairs * s.Hv;
+    }
+  }
+  // 1) forward recompute: the bf16 start state of every chunk
+  err = launch_fwd_tc(p, plan, items, stream, &what);
+  if (err != cudaSuccess) return cuda_fail(what, err);
+  // 2) reverse chain: the state gradient at every chunk end, and dh0
+  FwdParams pc = p;
+  pc.v = dO;
+  pc.h0 = dhT;
+  pc.hT = dh0;
+  pc.states = dstates;
+  err = launch_bwd_chain(pc, plan, items, stream, &what);
+  if (err != cudaSuccess) return cuda_fail(what, err);
+  // 3) per-chunk gradients
+  BwdOut out{};
+  out.dq = dq; out.dk = dk_out; out.dv = dv_out; out.dg = dg; out.dbeta = dbeta; out.dO = dO;
+  out.dstates = dstates;
+  out.qk_partial = bp.grouped ? 1 : 0;
+  out.dq_part = bp.grouped ? reinterpret_cast<float*>(ws + bp.off_dq) : nullptr;
+  out.dk_part = bp.grouped ? reinterpret_cast<float*>(ws + bp.off_dk) : nullptr;
+  err = launch_bwd_grad(p, out, bp.total_chunks, stream, &what);
+  if (err != cudaSuccess) return cuda_fail(what, err);
+  return GDN_OK;
 }
 
 gdn_status gdn_read_device_status(void* workspace, cudaStream_t stream) {

@@ -1,0 +1,726 @@
+// Backward, part 2 of 2 (tensor cores): the gradients of one 64-token chunk of one
+// (sequence, v-head), given the chunk's start state S and the state gradient dS' at its
+// end (both bf16, dv x dk, written by the state pass and the reverse chain). Chunks are
+// independent here, so the grid covers every (chunk, v-head) at once.
+//
+// Forward of the chunk (S-form, gam = inclusive cumsum of g, E_ij = exp(gam_i - gam_j)):
+//   L = strict_lower(diag(beta) KK^T * E), A = (I + L)^-1, A2 = A diag(beta)
+//   Y^T = V^T - S K^T diag(e^gam),  Delta^T = Y^T A2^T
+//   O^T = scale (S Q^T diag(e^gam) + Delta^T P^T),  P = lower_incl(QK^T * E)
+//   S'  = e^gam_n S + Delta^T diag(e^(gam_n - gam)) K
+// Adjoint (dO, dS' given; dP = scale dO Delta^T, dPm = dP * E * lower_incl):
+//   dDelta^T = dS' K^T diag(e^(gam_n - gam)) + dO^T (scale P);   dY^T = dDelta^T A2
+//   dV = dY;  dA2 = dDelta Y^T;  dbeta_j += sum_i dA2_ij A_ij;  dA = dA2 diag(beta)
+//   dL = -A^T dA A^T (strictly lower);  dG = dL * beta_i E (i > j);  dbeta_i += sum_j dL_ij KK_ij E_ij
+//   dQ = scale diag(e^gam) dO S + dPm K
+//   dK = dPm^T Q + (dG + dG^T) K - diag(e^gam) dY S + diag(e^(gam_n - gam)) Delta dS'
+//   dgam_i += scale e^gam_i sum_r dO_ir (S Q^T)_ri - e^gam_i sum_r dY_ir (S K^T)_ri
+//            + sum_j (F_ij - F_ji),  F = dP * P + dL * L
+//   dgam_j -= s_j,  dgam_{n} += sum_j s_j + e^gam_n <S, dS'>,  s_j = e^(gam_n - gam_j) sum_r Delta_jr (dS' K^T)_rj
+//   dg = reverse cumsum of dgam within the chunk.
+// (The oracle's token adjoint is the reference semantics; this is its chunked form.)
+//
+// All products are tcgen05 MMAs with 128 TMEM lanes: a product with 64 meaningful rows reads
+// 64 further rows of whatever follows in shared memory and ignores those lanes.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "gdn_chunk_prep.cuh"
+#include "gdn_common.cuh"
+#include "gdn_tc.cuh"
+#include "tc_ptx.cuh"
+
+namespace gdn {
+using namespace tc;
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBar = 1;
+
+// shared memory (bytes from the 1024-aligned base)
+constexpr uint32_t kOffKQ = 0;            // [K0 Q0 K1 Q1]
+constexpr uint32_t kOffVDO = 32u * 1024;  // [V0 dO0 V1 dO1]; V0/V1 become dD0/dD1 (dDelta, token-major)
+constexpr uint32_t kOffS = 64u * 1024;    // S  [r][d] bf16, two 16KB column halves
+constexpr uint32_t kOffDS = 96u * 1024;   // dS'
+constexpr uint32_t kOffYt = 128u * 1024;  // Y^T [r][j]; then -e^gam dY^T
+constexpr uint32_t kOffDt = 144u * 1024;  // Delta^T [r][j]; then e^(gam_n - gam) Delta^T
+constexpr uint32_t kOffA2 = 160u * 1024;  // A diag(beta)
+constexpr uint32_t kOffP = 168u * 1024;   // scale P; then dPm
+constexpr uint32_t kOffA = 176u * 1024;   // A; then dG + dG^T
+constexpr uint32_t kOffDA = 184u * 1024;  // dA; then X = dA A^T
+constexpr uint32_t kOffLf = 192u * 1024;  // fp32 64 x 65: L -> A; then dG
+constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
+
+struct Small {
+  ChunkScalars cs;
+  float dgam[64];
+  float dbeta[64];
+  float dgn;
+  uint64_t tma_bar, mma_bar;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
+
+// TMEM columns
+constexpr uint32_t kColG = 0;     // [K;Q] K^T (64)
+constexpr uint32_t kColY = 64;    // S K^T (64)
+constexpr uint32_t kColD = 128;   // Delta^T (64); later [dDelta;dO][Y^T|Delta^T] (128): dA2 | dP
+constexpr uint32_t kColSQ = 192;  // S Q^T (64)
+constexpr uint32_t kColDa = 256;  // dS' K^T (64); later X (64)
+constexpr uint32_t kColDb = 320;  // dO^T scale P (64); later dY^T (64); later dL (64)
+constexpr uint32_t kColQ = 384;   // dQ (128)
+constexpr uint32_t kColK = 128;   // dK (128), after dA2/dP are consumed
+constexpr uint32_t kTmemCols = 512;
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t a) { return sdesc_sw128(a, 16, 1024); }
+__device__ __forceinline__ uint64_t mdesc(uint32_t a, uint32_t lbo) { return sdesc_sw128(a, lbo, 1024); }
+
+// 32 values per lane -> lane l gets the sum over the warp's 32 lanes of value l.
+__device__ __forceinline__ float warp_transpose_sum(float* v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = upper ? v[i] : v[i + w];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, w);
+      v[i] = (upper ? v[i + w] : v[i]) + recv;
+    }
+  }
+  return v[0];
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_ds,
+                    const FwdParams p, const BwdOut out) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
+  Small* ss = reinterpret_cast<Small*>(sm + kOffSmall);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hh = warp >> 2;
+  if ((smem_u32(sm) & 1023u) != 0) {
+    if (tid == 0) record_error(p.status, kDevTimeout);
+    return;
+  }
+  // ---- which chunk: item = chunk_index * Hv + j
+  const int j = blockIdx.x % p.Hv;
+  const int gc = blockIdx.x / p.Hv;
+  int n, c;
+  if (p.chunk_off) {                          // packed sequences: last n with chunk_off[n] <= gc
+    int lo = 0, hi = p.N - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
+    }
+    n = lo;
+    c = gc - p.chunk_off[n];
+  } else {
+    const int nch = (p.T + kChunk - 1) / kChunk;
+    n = gc / nch;
+    c = gc % nch;
+  }
+  if (n >= p.N) return;
+  int b, s0, e0;
+  if (!seq_span(p, n, b, s0, e0)) return;
+  const int t0 = s0 + c * kChunk;
+  if (c < 0 || t0 >= e0) return;
+  const int nv = min(kChunk, e0 - t0);
+  const int hq = j / (p.Hv / p.Hqk);
+  const size_t slot = chunk_slot(p, n, c) * p.Hv + j;
+  const int row = b * p.T + t0;
+  const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
+
+  if (tid == 0) {
+    mbar_init(&ss->tma_bar, 1);
+    mbar_init(&ss->mma_bar, 1);
+    ss->abort_flag = 0;
+    ss->dgn = 0.f;
+    fence_mbar_init();
+  }
+  if (tid < 64) {
+    ss->dgam[tid] = 0.f;
+    ss->dbeta[tid] = 0.f;
+  }
+  if (warp == 0) {
+    tmem_alloc(&ss->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ss->tmem_base;
+  volatile int* abort_flag = &ss->abort_flag;
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+  const int r = 32 * qd + lane;               // TMEM lane of this thread (M = 128 layouts)
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&ss->tma_bar, 128u * 1024u);
+    tma_load_3d(sm + kOffKQ + 0, &tm_k, &ss->tma_bar, 0, hq, row);
+    tma_load_3d(sm + kOffKQ + 8192, &tm_q, &ss->tma_bar, 0, hq, row);
+    tma_load_3d(sm + kOffKQ + 16384, &tm_k, &ss->tma_bar, 64, hq, row);
+    tma_load_3d(sm + kOffKQ + 24576, &tm_q, &ss->tma_bar, 64, hq, row);
+    tma_load_3d(sm + kOffVDO + 0, &tm_v, &ss->tma_bar, 0, j, row);
+    tma_load_3d(sm + kOffVDO + 8192, &tm_do, &ss->tma_bar, 0, j, row);
+    tma_load_3d(sm + kOffVDO + 16384, &tm_v, &ss->tma_bar, 64, j, row);
+    tma_load_3d(sm + kOffVDO + 24576, &tm_do, &ss->tma_bar, 64, j, row);
+    const int srow = (int)(slot * 128);
+    tma_load_3d(sm + kOffS, &tm_s, &ss->tma_bar, 0, 0, srow);
+    tma_load_3d(sm + kOffS + 16384, &tm_s, &ss->tma_bar, 64, 0, srow);
+    tma_load_3d(sm + kOffDS, &tm_ds, &ss->tma_bar, 0, 0, srow);
+    tma_load_3d(sm + kOffDS + 16384, &tm_ds, &ss->tma_bar, 64, 0, srow);
+  }
+  PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), reinterpret_cast<float*>(sm + kOffYt), &ss->cs,
+             tmem, kColG, tid, warp, lane, kBar};
+  float gv = 0.f, bv = 0.f;
+  if (tid < nv) {
+    const size_t gi = (size_t)row * p.Hv + j + (size_t)tid * p.Hv;
+    gv = p.g[gi];
+    bv = __bfloat162float(beta[gi]);
+  }
+  prep_store_gb(pc, 0, gv, bv);
+  bool ok = mbar_wait(&ss->tma_bar, 0, abort_flag);
+  ok = __syncthreads_and(ok);
+  if (nv < kChunk) {                          // rows past the sequence end: zero
+    for (int idx = tid; idx < (kChunk - nv) * 64; idx += kThreads) {
+      const int rr = nv + idx / 64, rem = idx % 64, tile = rem / 8, ch = rem % 8;
+      *reinterpret_cast<uint4*>(sm + tile * 8192u + rr * 128u + ch * 16u) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  uint32_t mph = 0;
+  auto commit_wait = [&]() {
+    if (tid == 0 && ok) umma_commit(&ss->mma_bar);
+    ok = ok && mbar_wait(&ss->mma_bar, mph, abort_flag);
+    ok = __syncthreads_and(ok);
+    mph ^= 1;
+    tc_fence_after();
+  };
+  // ---- prep: G, gam, masks (scale * P), inverse, A2 and A
+  if (tid == 0 && ok) issue_gram(tmem + kColG, sbase + kOffKQ, &ss->mma_bar);
+  prep_scan(pc, 0);
+  __syncthreads();
+  prep_decays(pc, 0, nv);
+  // products that need only the loaded tiles: S K^T, S Q^T, dS' K^T, dO^T (scale P) comes later
+  ok = ok && mbar_wait(&ss->mma_bar, mph, abort_flag);
+  ok = __syncthreads_and(ok);
+  mph ^= 1;
+  tc_fence_after();
+  prep_masks(pc, 0, sbase + kOffP, p.scale, ok);
+  fence_proxy_async_smem();                   // scale * P is an operand of the next products
+  __syncthreads();
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t id64 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+      umma_f16(tmem + kColY, kdesc(sbase + kOffS + off), kdesc(sbase + kOffKQ + off), id64, ks > 0);
+      umma_f16(tmem + kColSQ, kdesc(sbase + kOffS + off), kdesc(sbase + kOffKQ + 8192 + off), id64, ks > 0);
+      umma_f16(tmem + kColDa, kdesc(sbase + kOffDS + off), kdesc(sbase + kOffKQ + off), id64, ks > 0);
+    }
+    // dO^T (scale P): A = dO MN-major (dv halves 16KB apart), B = scale P MN-major
+    constexpr uint32_t idmm = idesc_bf16(128, 64, true, true);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      umma_f16(tmem + kColDb, mdesc(sbase + kOffVDO + 8192 + ks * 2048, 16384), mdesc(sbase + kOffP + ks * 2048, 8192),
+               idmm, ks > 0);
+  }
+  prep_inverse(pc);
+  prep_write_a(pc, 0, sbase + kOffA2, sbase + kOffA);
+  fence_proxy_async_smem();
+  commit_wait();
+  const float* eg = ss->cs.eg[0];
+  const float* egd = ss->cs.egd[0];
+  // ---- Y^T = V^T - (S K^T) diag(e^gam);  dDelta = dS' K^T diag(e^(gam_n - gam)) + dO^T scale P
+  float yv[32], ddv[32];
+  {
+    float sk[32], da[32], db[32];
+    if (ok) {
+      tmem_ld32_sync(tmem + lane_base + kColY + hh * 32, sk);
+      tmem_ld32_sync(tmem + lane_base + kColDa + hh * 32, da);
+      tmem_ld32_sync(tmem + lane_base + kColDb + hh * 32, db);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 32; ++u) sk[u] = da[u] = db[u] = 0.f;
+    }
+    const uint8_t* vt = sm + kOffVDO + (r >> 6) * 16384;
+    const int rc = (r & 63) >> 3, rb = (r & 7) * 2;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int jj = hh * 32 + u;
+      const float vv = bf16_at(vt + jj * 128 + ((rc ^ (jj & 7)) << 4) + rb);
+      yv[u] = vv - eg[jj] * sk[u];
+      ddv[u] = fmaf(da[u], egd[jj], db[u]);
+    }
+  }
+  __syncthreads();                            // every V read is done: dD may overwrite V
+  {
+    uint32_t w[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) w[u] = pack_bf16(yv[2 * u], yv[2 * u + 1]);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+      st_shared_v4(sbase + kOffYt + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+    // dDelta token-major [i][r] in the V slots (dv half r / 64)
+    uint8_t* dd = sm + kOffVDO + (r >> 6) * 16384;
+    const int rc = (r & 63) >> 3, rb = (r & 7) * 2;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int ii = hh * 32 + u;
+      *reinterpret_cast<__nv_bfloat16*>(dd + ii * 128 + ((rc ^ (ii & 7)) << 4) + rb) = __float2bfloat16_rn(ddv[u]);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---- Delta^T = Y^T A2^T ;  dY^T = dDelta^T A2 ;  [dDelta; dO] [Y^T | Delta^T] needs Delta^T: later
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t id64 = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t idmm = idesc_bf16(128, 64, true, true);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      umma_f16(tmem + kColD, kdesc(sbase + kOffYt + ks * 32), kdesc(sbase + kOffA2 + ks * 32), id64, ks > 0);
+      // A[m=r][k=i] = dDelta[i][r]: token-major dD tile read MN-major (dv halves 16KB apart)
+      umma_f16(tmem + kColDb, mdesc(sbase + kOffVDO + ks * 2048, 16384), mdesc(sbase + kOffA2 + ks * 2048, 8192), idmm,
+               ks > 0);
+    }
+  }
+  commit_wait();
+  // ---- Delta^T -> bf16; dY^T -> dv (output) and -e^gam dY^T (bf16); dgam terms (1)-(4)
+  float dgpart[32];
+  {
+    float dl[32], dy[32], sk[32], sq[32], da[32];
+    if (ok) {
+      tmem_ld32_sync(tmem + lane_base + kColD + hh * 32, dl);
+      tmem_ld32_sync(tmem + lane_base + kColDb + hh * 32, dy);
+      tmem_ld32_sync(tmem + lane_base + kColY + hh * 32, sk);
+      tmem_ld32_sync(tmem + lane_base + kColSQ + hh * 32, sq);
+      tmem_ld32_sync(tmem + lane_base + kColDa + hh * 32, da);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 32; ++u) dl[u] = dy[u] = sk[u] = sq[u] = da[u] = 0.f;
+    }
+    const uint8_t* dot = sm + kOffVDO + 8192 + (r >> 6) * 16384;   // dO, token-major
+    const int rc = (r & 63) >> 3, rb = (r & 7) * 2;
+    float sj[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int jj = hh * 32 + u;
+      const float dov = bf16_at(dot + jj * 128 + ((rc ^ (jj & 7)) << 4) + rb);
+      // (1) + (2): scale e^gam_j dO_jr (S Q^T)_rj - e^gam_j dY_jr (S K^T)_rj
+      dgpart[u] = eg[jj] * (p.scale * dov * sq[u] - dy[u] * sk[u]);
+      sj[u] = egd[jj] * dl[u] * da[u];                 // (3) s_j partial
+    }
+    uint32_t w[16], x[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      w[u] = pack_bf16(dl[2 * u], dl[2 * u + 1]);
+      const int j0 = hh * 32 + 2 * u;
+      x[u] = pack_bf16(-dy[2 * u] * eg[j0], -dy[2 * u + 1] * eg[j0 + 1]);
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      st_shared_v4(sbase + kOffDt + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+    }
+    // the stacked product below still reads Y^T: -e^gam dY^T goes in after it
+    // dv (token-major) from dY^T: stage through registers of this thread: dv[jj][r]
+    if (ok) {
+      __nv_bfloat16* dvo = static_cast<__nv_bfloat16*>(out.dv);
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int jj = hh * 32 + u;
+        if (jj < nv) dvo[((size_t)(row + jj) * p.Hv + j) * 128 + r] = __float2bfloat16_rn(dy[u]);
+      }
+    }
+    // reductions over r (the 128 TMEM lanes = 4 warps x 32 lanes) into per-token sums
+    const float tot1 = warp_transpose_sum(dgpart);       // lane l: token hh*32 + l
+    const float tot3 = warp_transpose_sum(sj);
+    atomicAdd(&ss->dgam[hh * 32 + lane], tot1 - tot3);
+    float sred = tot3;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) sred += __shfl_xor_sync(0xffffffffu, sred, off);
+    if (lane == 0) atomicAdd(&ss->dgn, sred);            // (3): sum_j s_j -> gam_n
+    // keep -e^gam dY^T for later (registers -> written after the stacked product)
+#pragma unroll
+    for (int u = 0; u < 16; ++u) dgpart[u] = __uint_as_float(x[u]);
+  }
+  // (4) e^gam_n <S, dS'> over this thread's 64 entries (row r, half hh)
+  {
+    const uint8_t* sr = sm + kOffS + hh * 16384;
+    const uint8_t* dsr = sm + kOffDS + hh * 16384;
+    float acc = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint4 a = *reinterpret_cast<const uint4*>(sr + sw128(r, ch));
+      const uint4 d = *reinterpret_cast<const uint4*>(dsr + sw128(r, ch));
+      const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* dh = reinterpret_cast<const __nv_bfloat162*>(&d);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 af = __bfloat1622float2(ah[e]), df = __bfloat1622float2(dh[e]);
+        acc = fmaf(af.x, df.x, fmaf(af.y, df.y, acc));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) atomicAdd(&ss->dgn, ss->cs.egn[0] * acc);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---- [dDelta; dO] [Y^T | Delta^T]: rows 0..63 x cols 0..63 = dA2, rows 64..127 x cols 64..127 = dP / scale
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+      // B[k=r][n]: Y^T (n < 64) and Delta^T (n >= 64), tiles 16KB apart; k-step = 16 rows r
+      umma_f16(tmem + kColD, kdesc(sbase + kOffVDO + off), mdesc(sbase + kOffYt + ks * 2048, 16384), id, ks > 0);
+    }
+  }
+  commit_wait();
+  // Y^T is free: -e^gam dY^T; Delta^T -> e^(gam_n - gam) Delta^T in place (dP has consumed it)
+  {
+    uint32_t x[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) x[u] = __float_as_uint(dgpart[u]);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+      st_shared_v4(sbase + kOffYt + sw128(r, hh * 4 + c4), x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
+    uint8_t* dtr = sm + kOffDt;
+    uint4 q4[4];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) q4[c4] = *reinterpret_cast<const uint4*>(dtr + sw128(r, hh * 4 + c4));
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q4[c4]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int jj = hh * 32 + c4 * 8 + 2 * e;
+        const float2 f = __bfloat1622float2(h[e]);
+        h[e] = __floats2bfloat162_rn(f.x * egd[jj], f.y * egd[jj + 1]);
+      }
+      *reinterpret_cast<uint4*>(dtr + sw128(r, hh * 4 + c4)) = q4[c4];
+    }
+  }
+  // ---- C x C step. Lanes 0..63 (quadrants 0, 1): row i of dA2 (cols 0..63) and of K K^T (G);
+  //      lanes 64..127 (quadrants 2, 3): row i of dP (cols 64..127) and of Q K^T (G).
+  {
+    const int i = r & 63;
+    float gvals[32], mvals[32];
+    if (ok) {
+      tmem_ld32_sync(tmem + lane_base + kColG + hh * 32, gvals);
+      tmem_ld32_sync(tmem + lane_base + kColD + (r >= 64 ? 64 : 0) + hh * 32, mvals);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 32; ++u) gvals[u] = mvals[u] = 0.f;
+    }
+    // E_ij for this row's 32 columns by running products (as in the prep)
+    const int j0 = hh * 32;
+    float e[32];
+    {
+      const float gi = ss->cs.gam[0][i], glast = ss->cs.gam[0][j0 + 31];
+      float run = 1.f;
+#pragma unroll
+      for (int jj = 31; jj >= 0; --jj) {
+        const int jx = j0 + jj;
+        if (jj == 31) run = (jx >= i) ? 1.f : fast_exp(gi - glast);
+        else run = (jx >= i) ? 1.f : run * ss->cs.egt[0][jx + 1];
+        e[jj] = run;
+      }
+    }
+    const float* Lf = reinterpret_cast<const float*>(sm + kOffLf);   // A (fp32)
+    float rowsum = 0.f;
+    float colv[32];
+    if (r < 64) {
+      // dbeta_j += sum_i dA2_ij A_ij ;  dA = dA2 diag(beta) -> bf16
+      const float* bet = ss->cs.bet[0];
+      uint32_t w[16];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) colv[u] = mvals[u] * Lf[i * kLd + j0 + u];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        w[u] = pack_bf16(mvals[2 * u] * bet[j0 + 2 * u], mvals[2 * u + 1] * bet[j0 + 2 * u + 1]);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        st_shared_v4(sbase + kOffDA + sw128(i, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+      const float cs_ = warp_transpose_sum(colv);
+      atomicAdd(&ss->dbeta[j0 + lane], cs_);
+    } else {
+      // dP = scale * mvals;  P = QK^T * E (j <= i);  F = dP * P -> dgam_i += row sum, dgam_j -= col sum
+      // dPm = dP * E (j <= i) -> bf16
+      uint32_t w[16];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int jx = j0 + u;
+        const bool m = jx <= i;
+        const float dp = p.scale * mvals[u];
+        const float pv = m ? gvals[u] * e[u] : 0.f;
+        const float f = dp * pv;
+        rowsum += f;
+        colv[u] = f;
+        mvals[u] = m ? dp * e[u] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) w[u] = pack_bf16(mvals[2 * u], mvals[2 * u + 1]);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        st_shared_v4(sbase + kOffP + sw128(i, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+      const float cs_ = warp_transpose_sum(colv);
+      atomicAdd(&ss->dgam[j0 + lane], -cs_);
+      atomicAdd(&ss->dgam[i], rowsum);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---- X = dA A^T (rows i < 64 valid)
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      umma_f16(tmem + kColDa, kdesc(sbase + kOffDA + ks * 32), kdesc(sbase + kOffA + ks * 32), id, ks > 0);
+  }
+  commit_wait();
+  if (r < 64) {
+    float xv[32];
+    if (ok) tmem_ld32_sync(tmem + lane_base + kColDa + hh * 32, xv);
+    else {
+#pragma unroll
+      for (int u = 0; u < 32; ++u) xv[u] = 0.f;
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) w[u] = pack_bf16(xv[2 * u], xv[2 * u + 1]);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+      st_shared_v4(sbase + kOffDA + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---- dL = -A^T X  (A read MN-major: A^T[i][k] = A[k][i])
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      umma_f16(tmem + kColDb, mdesc(sbase + kOffA + ks * 2048, 8192), mdesc(sbase + kOffDA + ks * 2048, 8192), id,
+               ks > 0);
+  }
+  commit_wait();
+  // ---- dL (rows i < 64): strictly lower part. F += dL * L, dbeta_i += sum_j dL_ij KK_ij E_ij,
+  //      dG = dL beta_i E (fp32 to Lf), then dGs = dG + dG^T -> bf16 (A's slot)
+  {
+    const int i = r & 63;
+    const int j0 = hh * 32;
+    float* Lf = reinterpret_cast<float*>(sm + kOffLf);
+    if (r < 64) {
+      float dlv[32], gvals[32];
+      if (ok) {
+        tmem_ld32_sync(tmem + lane_base + kColDb + hh * 32, dlv);
+        tmem_ld32_sync(tmem + lane_base + kColG + hh * 32, gvals);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) dlv[u] = gvals[u] = 0.f;
+      }
+      const float gi = ss->cs.gam[0][i], glast = ss->cs.gam[0][j0 + 31];
+      const float bi = ss->cs.bet[0][i];
+      float run = 1.f, rowsum = 0.f, bsum = 0.f;
+      float colv[32], dg[32];
+#pragma unroll
+      for (int jj = 31; jj >= 0; --jj) {
+        const int jx = j0 + jj;
+        if (jj == 31) run = (jx >= i) ? 1.f : fast_exp(gi - glast);
+        else run = (jx >= i) ? 1.f : run * ss->cs.egt[0][jx + 1];
+        const bool m = jx < i;
+        const float dl = m ? -dlv[jj] : 0.f;
+        const float ke = gvals[jj] * run;
+        const float f = dl * bi * ke;            // dL * L
+        rowsum += f;
+        colv[jj] = f;
+        bsum += dl * ke;
+        dg[jj] = dl * bi * run;
+      }
+      // A (fp32) in Lf has no readers left: dG takes its place
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) Lf[i * kLd + j0 + jj] = dg[jj];
+      const float cs_ = warp_transpose_sum(colv);
+      atomicAdd(&ss->dgam[j0 + lane], -cs_);
+      atomicAdd(&ss->dgam[i], rowsum);
+      // bsum: this thread's half of row i; the other half is in warp qd + 4
+      atomicAdd(&ss->dbeta[i], bsum);
+    }
+  }
+  __syncthreads();
+  if (r < 64) {
+    const int i = r, j0 = hh * 32;
+    const float* Lf = reinterpret_cast<const float*>(sm + kOffLf);
+    uint32_t w[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int ja = j0 + 2 * u;
+      w[u] = pack_bf16(Lf[i * kLd + ja] + Lf[ja * kLd + i], Lf[i * kLd + ja + 1] + Lf[(ja + 1) * kLd + i]);
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+      st_shared_v4(sbase + kOffA + sw128(i, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+  }
+  // dO <- scale diag(e^gam) dO in place (for dQ); its other uses have completed
+  scale_rows_tile(pc, sm + kOffVDO + 8192, 16384, eg, p.scale);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---- dQ = (scale e^gam dO) S + dPm K ;  dK = dPm^T Q + dGs K + (-e^gam dY) S + (e^(gam_n-gam) Delta) dS'
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    constexpr uint32_t idkm = idesc_bf16(128, 128, false, true);   // A K-major, B MN-major
+    constexpr uint32_t idmm = idesc_bf16(128, 128, true, true);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;   // dO rows (K = r), 16 per step
+      umma_f16(tmem + kColQ, kdesc(sbase + kOffVDO + 8192 + off), mdesc(sbase + kOffS + ks * 2048, 16384), idkm,
+               ks > 0);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      umma_f16(tmem + kColQ, kdesc(sbase + kOffP + ks * 32), mdesc(sbase + kOffKQ + ks * 2048, 16384), idkm, 1);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      umma_f16(tmem + kColK, mdesc(sbase + kOffP + ks * 2048, 8192), mdesc(sbase + kOffKQ + 8192 + ks * 2048, 16384),
+               idmm, ks > 0);
+      umma_f16(tmem + kColK, kdesc(sbase + kOffA + ks * 32), mdesc(sbase + kOffKQ + ks * 2048, 16384), idkm, 1);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      umma_f16(tmem + kColK, mdesc(sbase + kOffYt + ks * 2048, 16384), mdesc(sbase + kOffS + ks * 2048, 16384), idmm, 1);
+      umma_f16(tmem + kColK, mdesc(sbase + kOffDt + ks * 2048, 16384), mdesc(sbase + kOffDS + ks * 2048, 16384), idmm,
+               1);
+    }
+  }
+  commit_wait();
+  // ---- outputs: dq, dk (rows i < nv), dbeta, dg
+  if (r < 64) {
+    const int i = r;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      float v[64];
+      const uint32_t col = which == 0 ? kColQ : kColK;
+      if (ok) {
+        tmem_ld32_sync(tmem + lane_base + col + hh * 64, v);
+        tmem_ld32_sync(tmem + lane_base + col + hh * 64 + 32, v + 32);
+      }
+      if (ok && i < nv) {
+        if (out.qk_partial) {                  // grouped values: fp32 per v-head, summed later
+          float* dst = (which == 0 ? out.dq_part : out.dk_part) + ((size_t)(row + i) * p.Hv + j) * 128 + hh * 64;
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            reinterpret_cast<float4*>(dst)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        } else {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(which == 0 ? out.dq : out.dk) +
+                               ((size_t)(row + i) * p.Hqk + hq) * 128 + hh * 64;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            reinterpret_cast<uint4*>(dst)[u] =
+                make_uint4(pack_bf16(v[8 * u], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+                           pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // dgam_{63} += dgn; dg = reverse cumsum of dgam over the chunk (two values per lane)
+    float a0 = ss->dgam[2 * lane], a1 = ss->dgam[2 * lane + 1];
+    if (lane == 31) a1 += ss->dgn;
+    // reverse inclusive scan: dg_t = sum_{i >= t} dgam_i
+    const float pair = a0 + a1;
+    float run = pair;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_down_sync(0xffffffffu, run, off);
+      if (lane + off < 32) run += y;
+    }
+    const float dg1 = run - a0;              // sum from 2*lane+1 up
+    const float dg0 = run;                   // sum from 2*lane up
+    if (ok) {
+      const size_t gi = (size_t)(row + 2 * lane) * p.Hv + j;
+      if (2 * lane < nv) out.dg[gi] = dg0;
+      if (2 * lane + 1 < nv) out.dg[gi + p.Hv] = dg1;
+      __nv_bfloat16* db = static_cast<__nv_bfloat16*>(out.dbeta);
+      if (2 * lane < nv) db[gi] = __float2bfloat16_rn(ss->dbeta[2 * lane]);
+      if (2 * lane + 1 < nv) db[gi + p.Hv] = __float2bfloat16_rn(ss->dbeta[2 * lane + 1]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (tid == 0 && *abort_flag) record_error(p.status, kDevTimeout);
+}
+
+// fp32 per-v-head partials of dq / dk -> the sum over the v-heads of each q/k head (fixed order)
+__global__ void gdn_bwd_reduce_kernel(const float* part, __nv_bfloat16* dst, int rows, int Hv, int Hqk) {
+  const int group = Hv / Hqk;
+  const size_t total = (size_t)rows * Hqk * 128;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
+    const size_t d = idx % 128;
+    const size_t h = (idx / 128) % Hqk;
+    const size_t t = idx / (128 * Hqk);
+    float acc = 0.f;
+    for (int g = 0; g < group; ++g) acc += part[(t * Hv + h * group + g) * 128 + d];
+    dst[idx] = __float2bfloat16_rn(acc);
+  }
+}
+
+// [slots * 128, 128] bf16 state array: boxes of 128 rows x 64 columns, 128B swizzle
+static bool make_state_map(CUtensorMap* m, const void* base, long long slots) {
+  return make_tile_map(m, base, 1, slots * 128, 128);
+}
+
+cudaError_t launch_bwd_grad(const FwdParams& p, const BwdOut& out, long long total_chunks, cudaStream_t st,
+                            const char** what) {
+  if (total_chunks <= 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv, mdo, ms, mds;
+  const long long rows = (long long)p.B * p.T;
+  *what = "tensor map encode";
+  if (!make_tile_map(&mq, p.q, p.Hqk, rows) || !make_tile_map(&mk, p.k, p.Hqk, rows) ||
+      !make_tile_map(&mv, p.v, p.Hv, rows) || !make_tile_map(&mdo, out.dO, p.Hv, rows) ||
+      !make_state_map(&ms, p.states, total_chunks * p.Hv) || !make_state_map(&mds, out.dstates, total_chunks * p.Hv))
+    return cudaErrorInvalidValue;
+  *what = "shared memory attribute";
+  cudaError_t err = cudaFuncSetAttribute(gdn_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+  if (err != cudaSuccess) return err;
+  *what = "backward gradient launch";
+  trace_pre(kKernBwdTc, st);
+  gdn_bwd_grad_kernel<<<(unsigned)(total_chunks * p.Hv), kThreads, kSmemBytes, st>>>(mq, mk, mv, mdo, ms, mds, p, out);
+  err = cudaGetLastError();
+  trace_post(st);
+  if (err != cudaSuccess || !out.qk_partial) return err;
+  *what = "backward dq/dk reduction";
+  const int rows_i = p.B * p.T;
+  const int blocks = (int)std::min<long long>(4096, ((long long)rows_i * p.Hqk * 128 + 255) / 256);
+  trace_pre(kKernBwdReduce, st);
+  gdn_bwd_reduce_kernel<<<blocks, 256, 0, st>>>(out.dq_part, static_cast<__nv_bfloat16*>(out.dq), rows_i, p.Hv, p.Hqk);
+  gdn_bwd_reduce_kernel<<<blocks, 256, 0, st>>>(out.dk_part, static_cast<__nv_bfloat16*>(out.dk), rows_i, p.Hv, p.Hqk);
+  err = cudaGetLastError();
+  trace_post(st);
+  return err;
+}
+
+}  // namespace gdn

@@ -1,0 +1,292 @@
+// State-independent per-chunk work shared by the tensor-core kernels (forward, the
+// backward's reverse state-gradient chain, the backward's gradient kernel), for one
+// 64-token chunk of one (sequence, v-head), run by a group of 256 threads (8 warps;
+// warp w reads TMEM lane quadrant w % 4 and column half w / 4):
+//
+//   gam = inclusive cumsum of g,  E_ij = exp(gam_i - gam_j)
+//   G = [K;Q] K^T   (one tcgen05 product, rows 0..63 = K K^T, rows 64..127 = Q K^T)
+//   L = strict_lower(diag(beta) K K^T * E)  -> fp32, inverted in place: A = (I + L)^-1
+//   P = lower_incl(Q K^T * E) * p_scale     -> bf16
+//   A2 = A diag(beta) -> bf16 (and A itself -> bf16 when asked)
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "gdn_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace gdn {
+
+constexpr int kLd = 65;           // row stride (floats) of the fp32 64 x 64 scratch
+constexpr int kPrepThreads = 256;
+
+// per-chunk scalars, double-buffered by chunk parity
+struct ChunkScalars {
+  float gam[2][64];   // chunk-local inclusive cumsum of g
+  float egt[2][64];   // exp(g_t) (1 past the sequence end)
+  float eg[2][64];    // exp(gam)
+  float egd[2][64];   // exp(gam_n - gam)
+  float bet[2][64];   // beta (0 past the sequence end)
+  float egn[2];       // exp(gam_n)
+  int nv[2];          // valid tokens in the chunk
+};
+
+__device__ __forceinline__ float bf16_at(const uint8_t* p) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+}
+
+// 16-byte chunk of 8 bf16 values, scaled
+__device__ __forceinline__ uint4 scale_chunk(uint4 v, float f) {
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 x = __bfloat1622float2(h[i]);
+    h[i] = __floats2bfloat162_rn(x.x * f, x.y * f);
+  }
+  return v;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+struct PrepCtx {
+  uint32_t sbase;     // shared address of the 1024-aligned smem base
+  float* Lf;          // fp32 [64][kLd] scratch
+  float* Xf;          // fp32 8 x 128 scratch
+  ChunkScalars* cs;
+  uint32_t tmem;      // TMEM base
+  uint32_t colG;      // TMEM column of G
+  int pt, pw, lane;   // thread index in the group, warp in the group, lane
+  int bar;            // named barrier id of the group
+};
+
+// g, beta of the chunk -> scalars (step 1: before the scan). gv, bv are this thread's
+// values (0 past the sequence end), loaded by the caller.
+__device__ __forceinline__ void prep_store_gb(const PrepCtx& c, int s, float gv, float bv) {
+  if (c.pt < kChunk) {
+    c.cs->gam[s][c.pt] = gv;
+    c.cs->bet[s][c.pt] = bv;
+    c.cs->egt[s][c.pt] = tc::fast_exp(gv);
+  }
+}
+
+// inclusive cumsum (warp 0) -- the caller separates this from prep_store_gb with a barrier
+__device__ __forceinline__ void prep_scan(const PrepCtx& c, int s) {
+  if (c.pw == 0) {
+    const float a0 = c.cs->gam[s][2 * c.lane], a1 = c.cs->gam[s][2 * c.lane + 1];
+    const float pair = a0 + a1;
+    float run = pair;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, run, off);
+      if (c.lane >= off) run += y;
+    }
+    c.cs->gam[s][2 * c.lane] = run - pair + a0;
+    c.cs->gam[s][2 * c.lane + 1] = run;
+  }
+}
+
+// decay factors (after the scan and a barrier)
+__device__ __forceinline__ void prep_decays(const PrepCtx& c, int s, int nv) {
+  const float gn = c.cs->gam[s][kChunk - 1];
+  if (c.pt < kChunk) {
+    c.cs->eg[s][c.pt] = tc::fast_exp(c.cs->gam[s][c.pt]);
+    c.cs->egd[s][c.pt] = tc::fast_exp(gn - c.cs->gam[s][c.pt]);
+  }
+  if (c.pt == 0) {
+    c.cs->egn[s] = tc::fast_exp(gn);
+    c.cs->nv[s] = nv;
+  }
+}
+
+// Issue G = [K;Q] K^T (K at kq_addr: [K0 Q0 K1 Q1] 8KB sub-tiles) and commit to `bar`.
+__device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, uint64_t* bar) {
+  constexpr uint32_t id = tc::idesc_bf16(128, 64, false, false);
+  tc::tc_fence_after();
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+    tc::umma_f16(tmem_g, tc::sdesc_sw128(kq_addr + off, 16, 1024), tc::sdesc_sw128(kq_addr + off, 16, 1024), id,
+                 ks > 0);
+  }
+  tc::umma_commit(bar);
+}
+
+// G (TMEM) -> L (fp32 in Lf, strictly lower) and P = p_scale * lower_incl(QK^T * E) (bf16,
+// 128B-swizzled rows at p_addr). E_ij = exp(gam_i - gam_j) (j <= i) is the running product
+// of exp(g_t) over t = j+1..i, walking j down: one exponential per row segment instead of
+// one per entry, no overflow, monotone underflow to 0. `ok` false: G treated as 0.
+// Ends with tcgen05 fence + group barrier.
+__device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_addr, float p_scale, bool ok) {
+  const int qd = c.pw & 3, hc = c.pw >> 2;
+  const int rr = 32 * qd + c.lane;
+  const int j0 = 32 * hc;
+  float vals[32];
+  if (ok) {
+    tc::tmem_ld32_sync(c.tmem + ((uint32_t)(32 * qd) << 16) + c.colG + j0, vals);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) vals[j] = 0.f;
+  }
+  float et[32];
+  {
+    const float4* e4 = reinterpret_cast<const float4*>(c.cs->egt[s] + j0);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 t = e4[u];
+      et[4 * u] = t.x; et[4 * u + 1] = t.y; et[4 * u + 2] = t.z; et[4 * u + 3] = t.w;
+    }
+  }
+  const int i = rr & 63;
+  const float gi = c.cs->gam[s][i];
+  const float glast = c.cs->gam[s][j0 + 31];
+  float run = 1.f;
+  if (rr < kChunk) {
+    const float bi = c.cs->bet[s][i];
+#pragma unroll
+    for (int jj = 31; jj >= 0; --jj) {
+      const int j = j0 + jj;
+      if (jj == 31) run = (j >= i) ? 1.f : tc::fast_exp(gi - glast);
+      else run = (j >= i) ? 1.f : run * et[jj + 1];
+      vals[jj] = (j < i) ? bi * vals[jj] * run : 0.f;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) c.Lf[i * kLd + j0 + jj] = vals[jj];
+  } else {
+#pragma unroll
+    for (int jj = 31; jj >= 0; --jj) {
+      const int j = j0 + jj;
+      if (jj == 31) run = (j >= i) ? 1.f : tc::fast_exp(gi - glast);
+      else run = (j >= i) ? 1.f : run * et[jj + 1];
+      vals[jj] = (j <= i) ? vals[jj] * run * p_scale : 0.f;
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+      st_shared_v4(p_addr + tc::sw128(i, 4 * hc + c4), tc::pack_bf16(vals[c4 * 8 + 0], vals[c4 * 8 + 1]),
+                   tc::pack_bf16(vals[c4 * 8 + 2], vals[c4 * 8 + 3]), tc::pack_bf16(vals[c4 * 8 + 4], vals[c4 * 8 + 5]),
+                   tc::pack_bf16(vals[c4 * 8 + 6], vals[c4 * 8 + 7]));
+  }
+  tc::tc_fence_before();
+  tc::named_bar_sync(c.bar, kPrepThreads);
+}
+
+// Scale the 64 rows of a [64 x 128] bf16 tile held as two 8KB 128B-swizzled sub-tiles
+// (sub-tile 1 at +sub_stride) by f[row] * mult, in place.
+__device__ __forceinline__ void scale_rows_tile(const PrepCtx& c, uint8_t* tile, uint32_t sub_stride,
+                                                const float* f, float mult) {
+  uint4 qv[4];
+  uint8_t* qa[4];
+  float fs[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int idx = c.pt + kPrepThreads * m;       // 0..1023
+    const int row = idx >> 4, half = (idx >> 3) & 1, ch = idx & 7;
+    qa[m] = tile + half * sub_stride + row * 128 + ch * 16;
+    fs[m] = f[row] * mult;
+    qv[m] = *reinterpret_cast<const uint4*>(qa[m]);
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(qa[m]) = scale_chunk(qv[m], fs[m]);
+}
+
+// A = (I + L)^-1 in place in Lf: 16x16 diagonal blocks by forward substitution (warps
+// 0..3), then block rows R = 1..3: A[R,<R] = -D_R (L[R,<R] A[<R,<R]) as 16 x 8 tiles of
+// m16n8k8 tf32 products (warp w: tile w). Starts and ends with a group barrier.
+__device__ __forceinline__ void prep_inverse(const PrepCtx& c) {
+  float* Lf = c.Lf;
+  if (c.pw < 4) {
+    const int R = c.pw, col = c.lane & 15;
+    float a[16];
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) {
+      float acc = (ii == col) ? 1.f : 0.f;
+#pragma unroll
+      for (int jj = 0; jj < ii; ++jj) acc -= Lf[(16 * R + ii) * kLd + 16 * R + jj] * a[jj];
+      a[ii] = (ii < col) ? 0.f : acc;
+    }
+    __syncwarp();
+    if (c.lane < 16) {
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) Lf[(16 * R + ii) * kLd + 16 * R + col] = a[ii];
+    }
+  }
+  tc::named_bar_sync(c.bar, kPrepThreads);
+  const int gid = c.lane >> 2, tig = c.lane & 3;
+#pragma unroll
+  for (int R = 1; R < 4; ++R) {
+    const int K = 16 * R;
+    const int tile = c.pw;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    if (tile < 2 * R) {
+      const int n0 = 8 * tile;
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      const float* lr = Lf + (16 * R) * kLd;
+#pragma unroll
+      for (int k0 = 0; k0 < K; k0 += 8) {
+        uint32_t af[4], bf[2];
+        af[0] = tc::to_tf32(lr[gid * kLd + k0 + tig]);
+        af[1] = tc::to_tf32(lr[(gid + 8) * kLd + k0 + tig]);
+        af[2] = tc::to_tf32(lr[gid * kLd + k0 + tig + 4]);
+        af[3] = tc::to_tf32(lr[(gid + 8) * kLd + k0 + tig + 4]);
+        bf[0] = tc::to_tf32(Lf[(k0 + tig) * kLd + n0 + gid]);
+        bf[1] = tc::to_tf32(Lf[(k0 + tig + 4) * kLd + n0 + gid]);
+        tc::mma_tf32_16x8x8(x, af, bf);
+      }
+      float* xw = c.Xf + c.pw * 128;
+      xw[gid * 8 + 2 * tig] = x[0];
+      xw[gid * 8 + 2 * tig + 1] = x[1];
+      xw[(gid + 8) * 8 + 2 * tig] = x[2];
+      xw[(gid + 8) * 8 + 2 * tig + 1] = x[3];
+      __syncwarp();
+      const float* dr = Lf + (16 * R) * kLd + 16 * R;
+#pragma unroll
+      for (int k0 = 0; k0 < 16; k0 += 8) {
+        uint32_t af[4], bf[2];
+        af[0] = tc::to_tf32(dr[gid * kLd + k0 + tig]);
+        af[1] = tc::to_tf32(dr[(gid + 8) * kLd + k0 + tig]);
+        af[2] = tc::to_tf32(dr[gid * kLd + k0 + tig + 4]);
+        af[3] = tc::to_tf32(dr[(gid + 8) * kLd + k0 + tig + 4]);
+        bf[0] = tc::to_tf32(xw[(k0 + tig) * 8 + gid]);
+        bf[1] = tc::to_tf32(xw[(k0 + tig + 4) * 8 + gid]);
+        tc::mma_tf32_16x8x8(y, af, bf);
+      }
+    }
+    tc::named_bar_sync(c.bar, kPrepThreads);       // every warp is done reading L[R, <R]
+    if (tile < 2 * R) {
+      float* ar = Lf + (16 * R) * kLd + 8 * tile;
+      ar[gid * kLd + 2 * tig] = -y[0];
+      ar[gid * kLd + 2 * tig + 1] = -y[1];
+      ar[(gid + 8) * kLd + 2 * tig] = -y[2];
+      ar[(gid + 8) * kLd + 2 * tig + 1] = -y[3];
+    }
+    tc::named_bar_sync(c.bar, kPrepThreads);
+  }
+}
+
+// A2 = A diag(beta) -> bf16 rows at a2_addr; with a_addr != 0 also A -> bf16 (thread: 16
+// columns of one row).
+__device__ __forceinline__ void prep_write_a(const PrepCtx& c, int s, uint32_t a2_addr, uint32_t a_addr) {
+  const int i = c.pt >> 2, qq = c.pt & 3;
+  const float* bet = c.cs->bet[s];
+  float a[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) a[u] = c.Lf[i * kLd + qq * 16 + u];
+  uint32_t w[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int j0 = qq * 16 + 2 * u;
+    w[u] = tc::pack_bf16(a[2 * u] * bet[j0], a[2 * u + 1] * bet[j0 + 1]);
+  }
+  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  if (a_addr) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) w[u] = tc::pack_bf16(a[2 * u], a[2 * u + 1]);
+    st_shared_v4(a_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+    st_shared_v4(a_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  }
+}
+
+}  // namespace gdn

@@ -29,9 +29,13 @@ struct FwdParams {
   const void* beta;
   const float* h0;          // nullable, [N,Hv,dk,dv]
   const int32_t* cu;        // nullable, [N+1]
-  void* o;
+  void* o;                  // nullable (no output written)
   float* hT;                // nullable
   int* status;              // device status word
+  // backward support: bf16 start state S (dv x dk, row-major) of every chunk, at
+  // states + ((chunk_off[n] + chunk) * Hv + j) * dv * dk; chunk_off nullable -> n * ceil(T/64)
+  __nv_bfloat16* states;    // nullable
+  const int* chunk_off;     // nullable
   int B, T, Hqk, Hv, dk, dv, N;
   float scale;
 };
@@ -46,6 +50,11 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ size_t chunk_slot(const FwdParams& p, int n, int chunk) {
+  const int base = p.chunk_off ? p.chunk_off[n] : n * ((p.T + kChunk - 1) / kChunk);
+  return (size_t)(base + chunk);
 }
 
 // Token span [s, e) and batch row of sequence n; returns false (after recording an
@@ -71,7 +80,8 @@ __device__ __forceinline__ bool seq_span(const FwdParams& p, int n, int& b, int&
 
 // ---- host-side launch instrumentation (gdn_api.cu)
 enum KernelId : int { kKernFwdTc = 0, kKernFwdSimt = 1, kKernCpStitch = 2, kKernBwdTc = 3,
-                      kKernBwdSimt = 4, kKernBwdReduce = 5, kKernCpPlan = 6, kKernCount = 7 };
+                      kKernBwdSimt = 4, kKernBwdReduce = 5, kKernCpPlan = 6, kKernBwdChain = 7,
+                      kKernCount = 8 };
 void trace_pre(int kernel_id, cudaStream_t st);
 void trace_post(cudaStream_t st);
 

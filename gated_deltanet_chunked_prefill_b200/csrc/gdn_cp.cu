@@ -18,7 +18,8 @@ constexpr int kPlanThreads = 1024;
 // exclusive scan gives the first pair index of each sequence; the table lists
 // (n, seg) for every pair. Inconsistent cu_seqlens are reported in the status word.
 __global__ void __launch_bounds__(kPlanThreads)
-gdn_cp_plan_kernel(const FwdParams p, int seg_chunks, int max_pairs, int2* table, int* count, int* first_pair) {
+gdn_cp_plan_kernel(const FwdParams p, int seg_chunks, int max_pairs, int2* table, int* count, int* first_pair,
+                   int* chunk_off) {
   __shared__ int part[kPlanThreads];
   const int tid = threadIdx.x;
   const int per = (p.N + kPlanThreads - 1) / kPlanThreads;
@@ -32,6 +33,32 @@ gdn_cp_plan_kernel(const FwdParams p, int seg_chunks, int max_pairs, int2* table
     }
     const int ch = (hi - lo + kChunk - 1) / kChunk;
     mine += max(1, (ch + seg_chunks - 1) / seg_chunks);
+  }
+  // chunk offsets (exclusive scan of ceil(len / 64)), when asked
+  if (chunk_off) {
+    int chunks = 0;
+    for (int n = n0; n < n1; ++n) {
+      int lo = p.cu[n], hi = p.cu[n + 1];
+      if (lo < 0 || hi < lo || hi > p.T) hi = lo = 0;
+      chunks += (hi - lo + kChunk - 1) / kChunk;
+    }
+    part[tid] = chunks;
+    __syncthreads();
+    for (int off = 1; off < kPlanThreads; off <<= 1) {
+      const int v = tid >= off ? part[tid - off] : 0;
+      __syncthreads();
+      part[tid] += v;
+      __syncthreads();
+    }
+    int base = part[tid] - chunks;
+    for (int n = n0; n < n1; ++n) {
+      chunk_off[n] = base;
+      int lo = p.cu[n], hi = p.cu[n + 1];
+      if (lo < 0 || hi < lo || hi > p.T) hi = lo = 0;
+      base += (hi - lo + kChunk - 1) / kChunk;
+    }
+    if (tid == kPlanThreads - 1) chunk_off[p.N] = part[tid];
+    __syncthreads();
   }
   part[tid] = mine;
   __syncthreads();
@@ -47,15 +74,16 @@ gdn_cp_plan_kernel(const FwdParams p, int seg_chunks, int max_pairs, int2* table
     if (lo < 0 || hi < lo || hi > p.T) hi = lo = 0;
     const int ch = (hi - lo + kChunk - 1) / kChunk;
     const int segs = max(1, (ch + seg_chunks - 1) / seg_chunks);
-    first_pair[n] = base;
-    for (int sgi = 0; sgi < segs; ++sgi)
-      if (base + sgi < max_pairs) table[base + sgi] = make_int2(n, sgi);
+    if (first_pair) first_pair[n] = base;
+    if (table)
+      for (int sgi = 0; sgi < segs; ++sgi)
+        if (base + sgi < max_pairs) table[base + sgi] = make_int2(n, sgi);
     base += segs;
   }
   if (tid == kPlanThreads - 1) {
     const int total = part[tid];
-    *count = min(total, max_pairs);
-    if (total > max_pairs || p.cu[0] != 0 || p.cu[p.N] != p.T) record_error(p.status, kDevBadSeqlens);
+    if (count) *count = min(total, max_pairs);
+    if ((table && total > max_pairs) || p.cu[0] != 0 || p.cu[p.N] != p.T) record_error(p.status, kDevBadSeqlens);
   }
 }
 
@@ -116,9 +144,9 @@ gdn_cp_stitch_kernel(const FwdParams p, const TcPlan plan, const int* first_pair
 }
 
 cudaError_t launch_cp_plan(const FwdParams& p, int seg_chunks, int max_pairs, int2* table, int* count,
-                           int* first_pair, cudaStream_t st) {
+                           int* first_pair, int* chunk_off, cudaStream_t st) {
   trace_pre(kKernCpPlan, st);
-  gdn_cp_plan_kernel<<<1, kPlanThreads, 0, st>>>(p, seg_chunks, max_pairs, table, count, first_pair);
+  gdn_cp_plan_kernel<<<1, kPlanThreads, 0, st>>>(p, seg_chunks, max_pairs, table, count, first_pair, chunk_off);
   cudaError_t err = cudaGetLastError();
   trace_post(st);
   return err;

@@ -24,6 +24,7 @@
 // movement, tensor-core and CUDA-core work).
 #include <cudaTypedefs.h>
 
+#include "gdn_chunk_prep.cuh"
 #include "gdn_common.cuh"
 #include "gdn_tc.cuh"
 #include "tc_ptx.cuh"
@@ -49,17 +50,10 @@ constexpr uint32_t kOffSb = 128u * 1024u;       // 32KB     S in bf16 (two 64-co
 constexpr uint32_t kOffYt = 160u * 1024u;       // 16KB     Y^T, then Delta^T
 constexpr uint32_t kOffDt = 176u * 1024u;       // 16KB     Delta~^T, then O staging
 constexpr uint32_t kOffLf = 192u * 1024u;       // fp32 [64][65] L, inverted in place
-constexpr int kLd = 65;
 constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 
 struct Small {
-  float gam[2][64];
-  float egt[2][64];   // exp(g_t) of each token (1 past the sequence end)
-  float eg[2][64];    // exp(gam)
-  float egd[2][64];   // exp(gam_n - gam)
-  float bet[2][64];
-  float egn[2];       // exp(gam_n)
-  int nv[2];
+  ChunkScalars cs;
   float Xf[8 * 128];      // inverse scratch: one 16 x 8 tile per prep warp
   float wsum[16];         // warm-up window search: per-warp partial sums
   int ws;                 // warm-up start token (context parallelism)
@@ -81,25 +75,6 @@ constexpr uint32_t kIdA = idesc_bf16(128, 128, false, false);
 constexpr uint32_t kIdC = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);
 
-__device__ __forceinline__ float bf16_at(const uint8_t* p) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
-}
-
-// 16-byte chunk of 8 bf16 values, scaled
-__device__ __forceinline__ uint4 scale_chunk(uint4 v, float f) {
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 x = __bfloat1622float2(h[i]);
-    h[i] = __floats2bfloat162_rn(x.x * f, x.y * f);
-  }
-  return v;
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
 
 }  // namespace
 
@@ -121,7 +96,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   WorkItem it;
   if (!get_work_item(p, plan, blockIdx.x, it)) return;   // uniform over the CTA
   const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -154,43 +128,12 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // exp(g)(I - beta k k^T); the window walks back chunk by chunk (at most kMaxWarm chunks,
   // otherwise the segment starts at the sequence start with h0: the exact recurrence).
   if (it.gate && it.s > it.seq_s) {
-    const int tok = threadIdx.x >> 3, part = threadIdx.x & 7;   // 64 tokens x 8 threads
     float logb = 0.f;
     int start = it.seq_s;
     for (int m = 1; m <= kMaxWarm; ++m) {
       const int cs = it.s - m * kChunk;
       if (cs < it.seq_s) break;
-      const size_t row = (size_t)(it.b * p.T + cs + tok);
-      const uint4* kr = reinterpret_cast<const uint4*>(kg + (row * p.Hqk + it.hq) * 128 + part * 16);
-      float sq = 0.f;
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const uint4 v = kr[u];
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(h[e]);
-          sq = fmaf(f.x, f.x, fmaf(f.y, f.y, sq));
-        }
-      }
-      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-      sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-      sq += __shfl_xor_sync(0xffffffffu, sq, 4);
-      float lt = 0.f;
-      if (part == 0) {
-        const size_t gi = row * p.Hv + it.j;
-        const float bt = __bfloat162float(beta[gi]);
-        lt = p.g[gi] + __logf(fmaxf(1.f, fabsf(1.f - bt * sq)));
-      }
-      lt += __shfl_xor_sync(0xffffffffu, lt, 8);
-      lt += __shfl_xor_sync(0xffffffffu, lt, 16);
-      if (lane == 0) ss->wsum[warp] = lt;           // warp w covers tokens 4w .. 4w + 3
-      __syncthreads();
-      float tot = 0.f;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) tot += ss->wsum[u];
-      __syncthreads();
-      logb += tot;
+      logb += chunk_log_bound(p, it, cs, kChunk, ss->wsum);
       if (logb <= kLogWarmBound) { start = cs; break; }
     }
     if (threadIdx.x == 0) ss->ws = start;
@@ -229,9 +172,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ prep (8 warps)
     const int pt = threadIdx.x;            // 0..255
-    const int pw = warp;                   // 0..7
-    const int qd = pw & 3, hc = pw >> 2;   // TMEM lane quadrant, column half
-    float* Lf = reinterpret_cast<float*>(sm + kOffLf);
+    PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), ss->Xf, &ss->cs, tmem, kColG, pt, warp, lane, kBarPrep};
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
@@ -247,11 +188,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       ok = ok && mbar_wait(&ss->full[s], (c >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
-      if (pt < kChunk) {
-        ss->gam[s][pt] = gv;
-        ss->bet[s][pt] = bv;
-        ss->egt[s][pt] = fast_exp(gv);
-      }
+      prep_store_gb(pc, s, gv, bv);
       if (nv < kChunk) {
         // rows past the sequence end hold the next sequence's tokens: clear them
         const int tiles = it.zero_v ? 4 : 6;
@@ -263,199 +200,18 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         fence_proxy_async_smem();
       }
       named_bar_sync(kBarPrep, kNumPrep);
-      if (pt == 0 && ok) {
-        tc_fence_after();
-        const uint32_t a0 = sbase + s * kStageBytes;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
-          umma_f16(tmem + kColG, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off, 16, 1024), kIdG, ks > 0);
-        }
-        umma_commit(&ss->gdone);
-      }
-      if (pw == 0) {  // inclusive cumsum of g (two values per lane)
-        const float a0 = ss->gam[s][2 * lane], a1 = ss->gam[s][2 * lane + 1];
-        const float pair = a0 + a1;
-        float run = pair;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, run, off);
-          if (lane >= off) run += y;
-        }
-        ss->gam[s][2 * lane] = run - pair + a0;
-        ss->gam[s][2 * lane + 1] = run;
-      }
+      if (pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
+      prep_scan(pc, s);
       named_bar_sync(kBarPrep, kNumPrep);
-      const float gn = ss->gam[s][kChunk - 1];
-      if (pt < kChunk) {
-        ss->eg[s][pt] = fast_exp(ss->gam[s][pt]);
-        ss->egd[s][pt] = fast_exp(gn - ss->gam[s][pt]);
-      }
-      if (pt == 0) {
-        ss->egn[s] = fast_exp(gn);
-        ss->nv[s] = nv;
-      }
+      prep_decays(pc, s, nv);
       ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      {
-        // G row rr (TMEM lane), columns j0..j0+31. Rows 0..63: K K^T -> L (fp32);
-        // rows 64..127: Q K^T -> P (bf16). E_ij = exp(gam_i - gam_j) (j <= i) is the running
-        // product of exp(g_t) over t = j+1..i, walking j down: one exponential per row
-        // segment instead of one per entry, no overflow, monotone underflow to 0.
-        const int rr = 32 * qd + lane;
-        const int j0 = 32 * hc;
-        float vals[32];
-        if (ok) {
-          tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + kColG + j0, vals);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) vals[j] = 0.f;
-        }
-        float et[32];
-        {
-          const float4* e4 = reinterpret_cast<const float4*>(ss->egt[s] + j0);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 t = e4[u];
-            et[4 * u] = t.x; et[4 * u + 1] = t.y; et[4 * u + 2] = t.z; et[4 * u + 3] = t.w;
-          }
-        }
-        const int i = rr & 63;
-        const float gi = ss->gam[s][i];
-        const float glast = ss->gam[s][j0 + 31];
-        float run = 1.f;
-        if (rr < kChunk) {
-          const float bi = ss->bet[s][i];
-#pragma unroll
-          for (int jj = 31; jj >= 0; --jj) {
-            const int j = j0 + jj;
-            if (jj == 31) run = (j >= i) ? 1.f : fast_exp(gi - glast);
-            else run = (j >= i) ? 1.f : run * et[jj + 1];
-            vals[jj] = (j < i) ? bi * vals[jj] * run : 0.f;
-          }
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) Lf[i * kLd + j0 + jj] = vals[jj];
-        } else {
-#pragma unroll
-          for (int jj = 31; jj >= 0; --jj) {
-            const int j = j0 + jj;
-            if (jj == 31) run = (j >= i) ? 1.f : fast_exp(gi - glast);
-            else run = (j >= i) ? 1.f : run * et[jj + 1];
-            vals[jj] = (j <= i) ? vals[jj] * run : 0.f;
-          }
-          const uint32_t prow = sbase + kOffP + s * 8192u;
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-            st_shared_v4(prow + sw128(i, 4 * hc + c4), pack_bf16(vals[c4 * 8 + 0], vals[c4 * 8 + 1]),
-                         pack_bf16(vals[c4 * 8 + 2], vals[c4 * 8 + 3]), pack_bf16(vals[c4 * 8 + 4], vals[c4 * 8 + 5]),
-                         pack_bf16(vals[c4 * 8 + 6], vals[c4 * 8 + 7]));
-        }
-      }
-      tc_fence_before();
-      named_bar_sync(kBarPrep, kNumPrep);
-      // Q <- diag(exp(gam)) Q, in place (the Gram product has consumed Q): 4 x 16 bytes per thread
-      {
-        uint4 qv[4];
-        uint8_t* qa[4];
-        float f[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int idx = pt + kNumPrep * m;                 // 0..1023
-          const int row = idx >> 4, half = (idx >> 3) & 1, ch = idx & 7;
-          qa[m] = st + 8192 + half * 16384 + row * 128 + ch * 16;
-          f[m] = ss->eg[s][row];
-          qv[m] = *reinterpret_cast<const uint4*>(qa[m]);
-        }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(qa[m]) = scale_chunk(qv[m], f[m]);
-      }
-      // A = (I + L)^-1: 16x16 diagonal blocks by forward substitution (warps 0..3, one each) ...
-      if (pw < 4) {
-        const int R = pw, col = lane & 15;
-        float a[16];
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          float acc = (ii == col) ? 1.f : 0.f;
-#pragma unroll
-          for (int jj = 0; jj < ii; ++jj) acc -= Lf[(16 * R + ii) * kLd + 16 * R + jj] * a[jj];
-          a[ii] = (ii < col) ? 0.f : acc;
-        }
-        __syncwarp();
-        if (lane < 16) {
-#pragma unroll
-          for (int ii = 0; ii < 16; ++ii) Lf[(16 * R + ii) * kLd + 16 * R + col] = a[ii];
-        }
-      }
-      named_bar_sync(kBarPrep, kNumPrep);
-      // ... then block rows R = 1..3: A[R, <R] = -D_R (L[R, <R] A[<R, <R]) in 16 x 8 output
-      // tiles of m16n8k8 tf32 products (warp w takes tile w of each row block).
-      {
-        const int gid = lane >> 2, tig = lane & 3;
-#pragma unroll
-        for (int R = 1; R < 4; ++R) {
-          const int K = 16 * R;
-          const int tile = pw;
-          float y[4] = {0.f, 0.f, 0.f, 0.f};
-          if (tile < 2 * R) {
-            const int n0 = 8 * tile;
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-            const float* lr = Lf + (16 * R) * kLd;
-#pragma unroll
-            for (int k0 = 0; k0 < K; k0 += 8) {
-              uint32_t af[4], bf[2];
-              af[0] = to_tf32(lr[gid * kLd + k0 + tig]);
-              af[1] = to_tf32(lr[(gid + 8) * kLd + k0 + tig]);
-              af[2] = to_tf32(lr[gid * kLd + k0 + tig + 4]);
-              af[3] = to_tf32(lr[(gid + 8) * kLd + k0 + tig + 4]);
-              bf[0] = to_tf32(Lf[(k0 + tig) * kLd + n0 + gid]);
-              bf[1] = to_tf32(Lf[(k0 + tig + 4) * kLd + n0 + gid]);
-              mma_tf32_16x8x8(x, af, bf);
-            }
-            float* xw = ss->Xf + pw * 128;
-            xw[gid * 8 + 2 * tig] = x[0];
-            xw[gid * 8 + 2 * tig + 1] = x[1];
-            xw[(gid + 8) * 8 + 2 * tig] = x[2];
-            xw[(gid + 8) * 8 + 2 * tig + 1] = x[3];
-            __syncwarp();
-            const float* dr = Lf + (16 * R) * kLd + 16 * R;
-#pragma unroll
-            for (int k0 = 0; k0 < 16; k0 += 8) {
-              uint32_t af[4], bf[2];
-              af[0] = to_tf32(dr[gid * kLd + k0 + tig]);
-              af[1] = to_tf32(dr[(gid + 8) * kLd + k0 + tig]);
-              af[2] = to_tf32(dr[gid * kLd + k0 + tig + 4]);
-              af[3] = to_tf32(dr[(gid + 8) * kLd + k0 + tig + 4]);
-              bf[0] = to_tf32(xw[(k0 + tig) * 8 + gid]);
-              bf[1] = to_tf32(xw[(k0 + tig + 4) * 8 + gid]);
-              mma_tf32_16x8x8(y, af, bf);
-            }
-          }
-          named_bar_sync(kBarPrep, kNumPrep);         // every warp is done reading L[R, <R]
-          if (tile < 2 * R) {
-            float* ar = Lf + (16 * R) * kLd + 8 * tile;
-            ar[gid * kLd + 2 * tig] = -y[0];
-            ar[gid * kLd + 2 * tig + 1] = -y[1];
-            ar[(gid + 8) * kLd + 2 * tig] = -y[2];
-            ar[(gid + 8) * kLd + 2 * tig + 1] = -y[3];
-          }
-          named_bar_sync(kBarPrep, kNumPrep);
-        }
-      }
-      // A2 = A diag(beta) -> bf16, 128B-swizzled rows (thread: 16 columns of one row)
-      {
-        const int i = pt >> 2, qq = pt & 3;
-        const uint32_t arow = sbase + kOffA2 + s * 8192u;
-        const float* bet = ss->bet[s];
-        uint32_t w[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j0 = qq * 16 + 2 * u;
-          w[u] = pack_bf16(Lf[i * kLd + j0] * bet[j0], Lf[i * kLd + j0 + 1] * bet[j0 + 1]);
-        }
-        st_shared_v4(arow + sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
-        st_shared_v4(arow + sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
-      }
+      prep_masks(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
+      // Q <- diag(exp(gam)) Q, in place (the Gram product has consumed Q)
+      scale_rows_tile(pc, st + 8192, 16384, ss->cs.eg[s], 1.f);
+      prep_inverse(pc);
+      prep_write_a(pc, s, sbase + kOffA2 + s * 8192u, 0);
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);
@@ -508,7 +264,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     };
     // S <- exp(gam_n) S in TMEM (before the chunk's update accumulates onto it)
     auto prescale = [&](int s) {
-      const float egn = ss->egn[s];
+      const float egn = ss->cs.egn[s];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         float v[32];
@@ -541,6 +297,14 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int t0 = ws + c * kChunk;
       wait_mma();
       const uint8_t* st = sm + s * kStageBytes;
+      if (p.states != nullptr && t0 >= it.s && ok) {
+        // backward support: this chunk's start state (the bf16 copy its products use)
+        const uint8_t* srow = sm + kOffSb + hh * 16384u;
+        uint4* dst = reinterpret_cast<uint4*>(p.states + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
+                                                             (size_t)(128 * 128) + (size_t)r * 128 + hh * 64);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) dst[ch] = *reinterpret_cast<const uint4*>(srow + sw128(r, ch));
+      }
       // (b) Y^T = V^T - (S K^T) diag(exp(gam))
       {
         float y[32];
@@ -551,7 +315,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         const uint8_t* vt = st + kOffV + (r >> 6) * 8192;
         const int rc = (r & 63) >> 3, rb = (r & 7) * 2;
-        const float* eg = ss->eg[s];
+        const float* eg = ss->cs.eg[s];
         uint32_t w[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
@@ -590,7 +354,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
           for (int u = 0; u < 32; ++u) dd[u] = 0.f;
         }
-        const float* egd = ss->egd[s];
+        const float* egd = ss->cs.egd[s];
         uint32_t w[16], x[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
@@ -625,7 +389,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       wait_mma();
       // (f) S -> bf16 copy for the next chunk's product;  O = scale * (Q part) -> registers
       float oo[32];
-      const int nv = ss->nv[s];
+      const int nv = ss->cs.nv[s];
       {
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -660,7 +424,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       // O staging (row j = token, 256 B per row) then coalesced 16-byte stores; the
       // prescale of S for the next chunk overlaps its first product
-      const bool write_o = it.write_o && t0 >= it.s;
+      const bool write_o = it.write_o && t0 >= it.s && p.o != nullptr;
       if (write_o) {
         __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sm + kOffDt);
 #pragma unroll
@@ -714,31 +478,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // ---------------------------------------------------------------- host side
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// [rows, heads, 128] bf16 tensor, boxes of 64 rows x 64 elements of one head, 128B swizzle
-bool make_map(CUtensorMap* m, const void* base, int heads, long long rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)heads * 128 * 2};
-  cuuint32_t box[3] = {64, 1, 64};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st,
@@ -747,8 +486,8 @@ cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items,
   CUtensorMap mq, mk, mv;
   const long long rows = (long long)p.B * p.T;
   *what = "tensor map encode";
-  if (!encode_fn()) return cudaErrorSymbolNotFound;
-  if (!make_map(&mq, p.q, p.Hqk, rows) || !make_map(&mk, p.k, p.Hqk, rows) || !make_map(&mv, p.v, p.Hv, rows))
+  if (!make_tile_map(&mq, p.q, p.Hqk, rows) || !make_tile_map(&mk, p.k, p.Hqk, rows) ||
+      !make_tile_map(&mv, p.v, p.Hv, rows))
     return cudaErrorInvalidValue;
   *what = "shared memory attribute";
   cudaError_t err = cudaFuncSetAttribute(gdn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

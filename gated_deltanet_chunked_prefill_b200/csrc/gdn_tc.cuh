@@ -3,9 +3,31 @@
 // final state goes.
 #pragma once
 
+#include <cuda.h>
+
 #include "gdn_common.cuh"
 
 namespace gdn {
+
+// TMA map of a [rows, heads, 128] bf16 tensor: boxes of box_rows rows x 64 elements of one
+// head, 128-byte swizzle (rows = B * T tokens; boxes past the last row read zeros).
+bool make_tile_map(CUtensorMap* m, const void* base, int heads, long long rows, int box_rows = 64);
+
+// Outputs and scratch of the backward's gradient kernel.
+struct BwdOut {
+  void* dq;                  // [B,T,Hqk,dk] bf16
+  void* dk;                  // [B,T,Hqk,dk] bf16
+  void* dv;                  // [B,T,Hv,dv] bf16
+  float* dg;                 // [B,T,Hv]
+  void* dbeta;               // [B,T,Hv] bf16
+  const void* dO;            // [B,T,Hv,dv] bf16
+  const __nv_bfloat16* dstates;   // per-chunk dS' (bf16, dv x dk)
+  int qk_partial;            // grouped values: dq/dk go through fp32 per-v-head partials
+  float* dq_part;            // [B,T,Hv,dk] fp32
+  float* dk_part;            // [B,T,Hv,dk] fp32
+};
+cudaError_t launch_bwd_grad(const FwdParams& p, const BwdOut& out, long long total_chunks, cudaStream_t st,
+                            const char** what);
 
 enum InitMode : int { kInitZero = 0, kInitPtr = 1, kInitIdentity = 2 };
 
@@ -43,7 +65,7 @@ struct TcPlan {
 
 struct WorkItem {
   int n, j, hq, b, s, e;  // sequence, v-head, q/k head, batch row, token range [s, e)
-  int seq_s;              // first token of the sequence
+  int seq_s, seq_e;       // token range of the whole sequence
   bool gate;              // may start earlier than s with a warm-up window (kPlanGate)
   int init_mode;
   const float* init;      // [dk][dv] fp32 when init_mode == kInitPtr
@@ -65,6 +87,7 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
     w.n = item / p.Hv;
     if (!seq_span(p, w.n, w.b, w.s, w.e)) return false;
     w.seq_s = w.s;
+    w.seq_e = w.e;
     w.hq = w.j / (p.Hv / p.Hqk);
     if (p.h0) { w.init_mode = kInitPtr; w.init = p.h0 + ((size_t)w.n * p.Hv + w.j) * hsz; }
     if (p.hT) w.fin = p.hT + ((size_t)w.n * p.Hv + w.j) * hsz;
@@ -96,6 +119,7 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
   if (seg >= segs_used) return false;
   w.b = b;
   w.seq_s = s;
+  w.seq_e = e;
   w.hq = w.j / (p.Hv / p.Hqk);
   w.s = s + seg * plan.seg_chunks * kChunk;
   w.e = min(e, w.s + plan.seg_chunks * kChunk);
@@ -127,11 +151,58 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
   return true;
 }
 
+// Sum over the tokens [cs, cs + n) (n <= 64) of log(exp(g_t) max(1, |1 - beta_t |k_t|^2|)),
+// the log of the exact spectral norm of each token's state transition exp(g)(I - beta k k^T)
+// (eigenvalues exp(g) and exp(g)(1 - beta |k|^2)). All 512 threads of the CTA call it and
+// get the same value; wsum is 16 floats of shared scratch.
+__device__ __forceinline__ float chunk_log_bound(const FwdParams& p, const WorkItem& it, int cs, int n,
+                                                 float* wsum) {
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
+  const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
+  const int tok = threadIdx.x >> 3, part = threadIdx.x & 7;   // 64 tokens x 8 threads
+  float sq = 0.f;
+  const size_t row = (size_t)(it.b * p.T + cs + tok);
+  if (tok < n) {
+    const uint4* kr = reinterpret_cast<const uint4*>(kg + (row * p.Hqk + it.hq) * 128 + part * 16);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint4 v = kr[u];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        sq = fmaf(f.x, f.x, fmaf(f.y, f.y, sq));
+      }
+    }
+  }
+  sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+  float lt = 0.f;
+  if (part == 0 && tok < n) {
+    const size_t gi = row * p.Hv + it.j;
+    const float bt = __bfloat162float(beta[gi]);
+    lt = p.g[gi] + __logf(fmaxf(1.f, fabsf(1.f - bt * sq)));
+  }
+  lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+  lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = lt;   // warp w covers tokens 4w .. 4w + 3
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) tot += wsum[u];
+  __syncthreads();
+  return tot;
+}
+
 cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st,
                           const char** what);
+// Backward, reverse state-gradient chain (see gdn_bwd_chain.cu for the parameter mapping).
+cudaError_t launch_bwd_chain(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st,
+                             const char** what);
 // Packed sequences: build the (sequence, segment) table of a segmented plan.
 cudaError_t launch_cp_plan(const FwdParams& p, int seg_chunks, int max_pairs, int2* table, int* count,
-                           int* first_pair, cudaStream_t st);
+                           int* first_pair, int* chunk_off, cudaStream_t st);
 // Exact stitch, phase 2: chain the segment maps h_{s+1} = M_s h_s + b_s in place.
 cudaError_t launch_cp_stitch(const FwdParams& p, const TcPlan& plan, const int* first_pair, cudaStream_t st);
 
