@@ -34,7 +34,7 @@ from gated_deltanet_chunked_prefill_b200.workloads import CONFIGS, make_inputs  
 
 METRIC = "GDN chunk fwd/bwd tokens/s and TFLOP/s on 1 B200; % of roofline"
 WORKLOAD = "dense_bf16"
-STEP = "fwd"          # what one step runs: "fwd" or "fwdbwd"
+STEP = "fwdbwd"       # what one step runs: "fwd" or "fwdbwd"
 C = 64
 
 

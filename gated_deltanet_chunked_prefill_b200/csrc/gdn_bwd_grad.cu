@@ -53,11 +53,16 @@ constexpr uint32_t kOffDA = 184u * 1024;  // dA; then X = dA A^T
 constexpr uint32_t kOffLf = 192u * 1024;  // fp32 64 x 65: L -> A; then dG
 constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 
+// Per-token partial sums, one slot per producer so that every slot entry is written exactly
+// once and the final sums run in a fixed order (bit-reproducible results).
+enum : int { kSlotTok = 0, kSlotFP = 4, kSlotFPRow = 6, kSlotFL = 8, kSlotFLRow = 10, kNumGamSlots = 12 };
+enum : int { kSlotBetaA = 0, kSlotBetaL = 2, kNumBetaSlots = 4 };
+
 struct Small {
   ChunkScalars cs;
-  float dgam[64];
-  float dbeta[64];
-  float dgn;
+  float dgam[kNumGamSlots][64];
+  float dbeta[kNumBetaSlots][64];
+  float dgn[16];
   uint64_t tma_bar, mma_bar;
   uint32_t tmem_base;
   int abort_flag;
@@ -142,12 +147,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(&ss->tma_bar, 1);
     mbar_init(&ss->mma_bar, 1);
     ss->abort_flag = 0;
-    ss->dgn = 0.f;
     fence_mbar_init();
-  }
-  if (tid < 64) {
-    ss->dgam[tid] = 0.f;
-    ss->dbeta[tid] = 0.f;
   }
   if (warp == 0) {
     tmem_alloc(&ss->tmem_base, kTmemCols);
@@ -345,11 +345,11 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // reductions over r (the 128 TMEM lanes = 4 warps x 32 lanes) into per-token sums
     const float tot1 = warp_transpose_sum(dgpart);       // lane l: token hh*32 + l
     const float tot3 = warp_transpose_sum(sj);
-    atomicAdd(&ss->dgam[hh * 32 + lane], tot1 - tot3);
+    ss->dgam[kSlotTok + qd][hh * 32 + lane] = tot1 - tot3;
     float sred = tot3;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) sred += __shfl_xor_sync(0xffffffffu, sred, off);
-    if (lane == 0) atomicAdd(&ss->dgn, sred);            // (3): sum_j s_j -> gam_n
+    if (lane == 0) ss->dgn[warp] = sred;                 // (3): sum_j s_j -> gam_n
     // keep -e^gam dY^T for later (registers -> written after the stacked product)
 #pragma unroll
     for (int u = 0; u < 16; ++u) dgpart[u] = __uint_as_float(x[u]);
@@ -373,7 +373,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) atomicAdd(&ss->dgn, ss->cs.egn[0] * acc);
+    if (lane == 0) ss->dgn[8 + warp] = ss->cs.egn[0] * acc;
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -456,7 +456,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int c4 = 0; c4 < 4; ++c4)
         st_shared_v4(sbase + kOffDA + sw128(i, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
       const float cs_ = warp_transpose_sum(colv);
-      atomicAdd(&ss->dbeta[j0 + lane], cs_);
+      ss->dbeta[kSlotBetaA + qd][j0 + lane] = cs_;       // qd in {0, 1}
     } else {
       // dP = scale * mvals;  P = QK^T * E (j <= i);  F = dP * P -> dgam_i += row sum, dgam_j -= col sum
       // dPm = dP * E (j <= i) -> bf16
@@ -478,8 +478,8 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int c4 = 0; c4 < 4; ++c4)
         st_shared_v4(sbase + kOffP + sw128(i, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
       const float cs_ = warp_transpose_sum(colv);
-      atomicAdd(&ss->dgam[j0 + lane], -cs_);
-      atomicAdd(&ss->dgam[i], rowsum);
+      ss->dgam[kSlotFP + (qd - 2)][j0 + lane] = -cs_;   // qd in {2, 3}
+      ss->dgam[kSlotFPRow + hh][i] = rowsum;
     }
   }
   fence_proxy_async_smem();
@@ -558,10 +558,10 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) Lf[i * kLd + j0 + jj] = dg[jj];
       const float cs_ = warp_transpose_sum(colv);
-      atomicAdd(&ss->dgam[j0 + lane], -cs_);
-      atomicAdd(&ss->dgam[i], rowsum);
+      ss->dgam[kSlotFL + qd][j0 + lane] = -cs_;         // qd in {0, 1}
+      ss->dgam[kSlotFLRow + hh][i] = rowsum;
       // bsum: this thread's half of row i; the other half is in warp qd + 4
-      atomicAdd(&ss->dbeta[i], bsum);
+      ss->dbeta[kSlotBetaL + hh][i] = bsum;
     }
   }
   __syncthreads();
@@ -643,8 +643,24 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __syncthreads();
   if (warp == 0) {
     // dgam_{63} += dgn; dg = reverse cumsum of dgam over the chunk (two values per lane)
-    float a0 = ss->dgam[2 * lane], a1 = ss->dgam[2 * lane + 1];
-    if (lane == 31) a1 += ss->dgn;
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < kNumGamSlots; ++sl) {
+      a0 += ss->dgam[sl][2 * lane];
+      a1 += ss->dgam[sl][2 * lane + 1];
+    }
+    if (lane == 31) {
+      float gn = 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) gn += ss->dgn[u];
+      a1 += gn;
+    }
+    float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < kNumBetaSlots; ++sl) {
+      b0 += ss->dbeta[sl][2 * lane];
+      b1 += ss->dbeta[sl][2 * lane + 1];
+    }
     // reverse inclusive scan: dg_t = sum_{i >= t} dgam_i
     const float pair = a0 + a1;
     float run = pair;
@@ -660,8 +676,8 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (2 * lane < nv) out.dg[gi] = dg0;
       if (2 * lane + 1 < nv) out.dg[gi + p.Hv] = dg1;
       __nv_bfloat16* db = static_cast<__nv_bfloat16*>(out.dbeta);
-      if (2 * lane < nv) db[gi] = __float2bfloat16_rn(ss->dbeta[2 * lane]);
-      if (2 * lane + 1 < nv) db[gi + p.Hv] = __float2bfloat16_rn(ss->dbeta[2 * lane + 1]);
+      if (2 * lane < nv) db[gi] = __float2bfloat16_rn(b0);
+      if (2 * lane + 1 < nv) db[gi + p.Hv] = __float2bfloat16_rn(b1);
     }
   }
   tc_fence_before();
