@@ -63,6 +63,26 @@ def alg_bytes(w, fwd=True, bwd=True):
     return (f if fwd else 0) + (b if bwd else 0)
 
 
+def kernel_alg_bytes(w):
+    """Algorithmic bytes of one launch of each kernel (inputs read once, outputs written once;
+    scratch such as the per-chunk states is not counted), per the workload."""
+    es = 2 if w.dtype == "bf16" else 4
+    ntok = w.B * w.T
+    qk = ntok * w.Hqk * w.dk * es            # q or k (or dq, dk)
+    vv = ntok * w.Hv * w.dv * es             # v, o, dO or dv
+    gb = ntok * w.Hv * (4 + es)              # g and beta (or dg, dbeta)
+    st = w.num_seqs * w.Hv * w.dk * w.dv * 4
+    h0 = st if w.h0_std is not None else 0
+    return {
+        # forward call: q k v g beta h0 -> o hT ; the backward's state pass reads the same inputs
+        "gdn_fwd_tc_kernel": [2 * qk + vv + gb + h0 + vv + st, 2 * qk + vv + gb + h0],
+        # reverse chain: q k dO g beta dhT -> dh0
+        "gdn_bwd_chain_kernel": [2 * qk + vv + gb + st + st],
+        # gradients: q k v dO g beta -> dq dk dv dg dbeta
+        "gdn_bwd_grad_kernel": [2 * qk + 2 * vv + gb + 2 * qk + vv + gb],
+    }
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -148,6 +168,20 @@ def traffic_record(kernel_name, workload):
                     return None
             return float(r["bytes_per_launch"])
     return None
+
+
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """The largest value of x over all ranks (the step time of the slowest rank)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank times its own replica of the workload, drawn from its own seed."""
+    return base + 17 * rank
 
 
 # ------------------------------------------------------------------------------------- oracle arm
@@ -236,7 +270,7 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed + 17 * rank, h0_std=w.h0_std,
+    x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, rank_seed(w.seed, rank), h0_std=w.h0_std,
                     backward=True)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     stream = torch.cuda.current_stream(dev)
@@ -286,11 +320,7 @@ def main():
         dist.barrier()
     sampler.stop()
     launches = gdn.launch_count() - n0
-    ms = ev0.elapsed_time(ev1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     ms_step = ms / args.steps
     tokens = w.B * w.T * world
     value = tokens / (ms_step / 1e3)
@@ -312,18 +342,29 @@ def main():
         bwd_ms = sum(t for _, t in tr.launches) / 5 - fwd_ms
 
     hbm, tc_peak, src = peaks()
+    # per-launch algorithmic bytes, matched to the launches of one step in order
+    kb = kernel_alg_bytes(w)
+    seen = {}
+    per_kernel_bytes = {}
+    for name, t in tr.launches[: len(tr.launches) // 5]:
+        k = seen.get(name, 0)
+        seen[name] = k + 1
+        opts = kb.get(name)
+        if opts:
+            per_kernel_bytes.setdefault(name, []).append(opts[min(k, len(opts) - 1)])
     dom = max(per_kernel, key=lambda k: sum(per_kernel[k]))
     dom_ms = float(np.mean(per_kernel[dom]))
-    fwd_only_dom = dom in ("gdn_fwd_tc_kernel", "gdn_fwd_simt_kernel")
-    if fwd_only_dom and len(trf.launches) == 5:
-        dom_bytes = alg_bytes(w, fwd=True, bwd=False)
-    else:
-        dom_bytes = alg_bytes(w, fwd=True, bwd=mode == "fwdbwd") / max(1, len(tr.launches) // 5)
+    dom_bytes = float(np.mean(per_kernel_bytes.get(dom, [0])))
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "peak_source": src,
                 "traffic": traffic_record(dom, args.workload),
                 "alg_bytes_per_launch": dom_bytes, "avg_launch_ms": dom_ms}
+    step_bytes = alg_bytes(w, fwd=True, bwd=mode == "fwdbwd")
+    step_roofline = {"alg_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                     "frac_hbm": step_bytes / (ms_step / 1e3) / 1e9 / hbm,
+                     "tflops": flops(w, fwd=True, bwd=mode == "fwdbwd") / (ms_step / 1e3) / 1e12,
+                     "frac_tensor": flops(w, fwd=True, bwd=mode == "fwdbwd") / (ms_step / 1e3) / 1e12 / tc_peak}
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     host_in = {k: x[k].pin_memory() for k in ("q", "k", "v", "g", "beta", "h0", "dO", "dhT")
@@ -366,11 +407,7 @@ def main():
         e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    e_ms = ev0.elapsed_time(ev1)
-    if dist:
-        t = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     e2e = {"value": tokens / (e_ms / e_steps / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
@@ -394,7 +431,8 @@ def main():
            "tflops": fl / (ms_step / 1e3) / 1e12,
            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
            "per_kernel_ms": {k: float(np.mean(v)) for k, v in per_kernel.items()},
-           "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+           "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
+           "gpu_launches": int(launches),
            "clocks": sampler.summary(tw0, tw1)}
     if rank == 0:
         print(json.dumps(out), flush=True)
