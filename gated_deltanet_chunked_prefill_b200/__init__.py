@@ -13,7 +13,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_bwd", "fwd_workspace_size",
+__all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd", "fwd_workspace_size",
            "bwd_workspace_size", "read_device_status", "Options", "LIB_PATH", "KernelTrace",
            "launch_count"]
 
@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_bwd.argtypes = [i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp,
                                                     vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
         L.gdn_chunk_bwd.restype = i
+        L.gdn_chunk_fwd_noalloc.argtypes = [i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp,
+                                                            vp, vp]
+        L.gdn_chunk_fwd_noalloc.restype = i
         L.gdn_read_device_status.argtypes = [vp, vp]
         L.gdn_read_device_status.restype = i
         L.gdn_status_string.argtypes = [i]
@@ -166,6 +169,30 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
                              _ptr(hT), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream(stream))
     if st != 0:
         raise GdnError(st, "gdn_chunk_fwd")
+    return o, hT
+
+
+def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
+                          output_final_state=True, cp_segment_chunks=0, o=None, hT=None, stream=None):
+    """Forward through the allocation-free entry point (library-held 1 MiB scratch; see gdn.h)."""
+    io = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, n, io)
+    _check(g, "g", torch.float32)
+    _check(h0, "h0", torch.float32)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
+    scale = dk ** -0.5 if scale is None else float(scale)
+    if o is None:
+        o = torch.empty((B, T, Hv, dv), dtype=io, device=q.device)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    opt = _opts(cp_segment_chunks)
+    st = lib().gdn_chunk_fwd_noalloc(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N,
+                                     _ptr(o), _ptr(hT), ctypes.byref(opt), _stream(stream))
+    if st != 0:
+        raise GdnError(st, "gdn_chunk_fwd_noalloc")
     return o, hT
 
 

@@ -157,6 +157,8 @@ BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
 }  // namespace
 
 namespace gdn {
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 void trace_pre(int kernel_id, cudaStream_t st) {
   ++g_launches;
   Trace& t = g_trace;

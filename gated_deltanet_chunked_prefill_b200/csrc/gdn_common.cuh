@@ -83,6 +83,7 @@ enum KernelId : int { kKernFwdTc = 0, kKernFwdSimt = 1, kKernCpStitch = 2, kKern
                       kKernBwdSimt = 4, kKernBwdReduce = 5, kKernCpPlan = 6, kKernBwdChain = 7,
                       kKernCount = 8 };
 void trace_pre(int kernel_id, cudaStream_t st);
+void set_last_error(const char* msg);   // text returned by gdn_last_error() on this thread
 void trace_post(cudaStream_t st);
 
 }  // namespace gdn

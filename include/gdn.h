@@ -134,6 +134,31 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
                          void* workspace, size_t workspace_bytes,
                          const gdn_options* opt, cudaStream_t stream);
 
+/*
+ * Forward without a workspace, for callers that cannot allocate device memory where
+ * they run the operator (inside a framework's memory pool, or a runtime that forbids
+ * allocation on its hot path). The pages have no counterpart: this is a library
+ * convenience, not part of the method.
+ *
+ * Same arguments and results as gdn_chunk_fwd, minus the workspace. Scratch comes from
+ * a 1 MiB array in the library's device memory that every GPU loading the library holds
+ * until the process exits; the call allocates nothing (no cudaMalloc, no library
+ * allocator). Calls whose scratch need (gdn_chunk_fwd_workspace_size) exceeds 1 MiB,
+ * e.g. the exact affine stitch (cp_exact) on large inputs, return GDN_ERR_WORKSPACE
+ * with the sizes in gdn_last_error(). The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress, once per device); make that first call before
+ * any stream capture. All calls share the one array: calls that overlap on the GPU
+ * (concurrent streams) race and must not be issued. Each call clears the status word;
+ * device-side findings (inconsistent cu_seqlens, a timed-out wait) are not reported
+ * back through this entry point.
+ */
+gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
+                                 const void* q, const void* k, const void* v,
+                                 const float* g, const void* beta, float scale,
+                                 const float* h0, const int32_t* cu_seqlens, int num_seqs,
+                                 void* o, float* hT,
+                                 const gdn_options* opt, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns (and clears) the status word that the
  * kernels of earlier calls on this workspace recorded: GDN_OK,
  * GDN_ERR_DEVICE_TIMEOUT or GDN_ERR_DEVICE_INPUT. GDN_ERR_CUDA if the stream
