@@ -175,6 +175,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       ok = ok && mbar_wait(&ss->full[s], (k >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
+      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
       prep_store_gb(pc, s, gv, bv);
       if (nv < kChunk) {
         for (int idx = pt; idx < (kChunk - nv) * 48; idx += kNumPrep) {
@@ -185,7 +186,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         fence_proxy_async_smem();
       }
       named_bar_sync(kBarPrep, kNumPrep);
-      if (pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
+      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
       prep_scan(pc, s);
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays(pc, s, nv);

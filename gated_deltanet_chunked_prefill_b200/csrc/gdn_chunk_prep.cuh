@@ -201,10 +201,14 @@ __device__ __forceinline__ void prep_inverse(const PrepCtx& c) {
     float a[16];
 #pragma unroll
     for (int ii = 0; ii < 16; ++ii) {
-      float acc = (ii == col) ? 1.f : 0.f;
+      // two independent accumulation chains (even / odd jj) halve the dependent latency
+      float acc0 = (ii == col) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < ii; ++jj) acc -= Lf[(16 * R + ii) * kLd + 16 * R + jj] * a[jj];
-      a[ii] = (ii < col) ? 0.f : acc;
+      for (int jj = 0; jj < ii; jj += 2) {
+        acc0 -= Lf[(16 * R + ii) * kLd + 16 * R + jj] * a[jj];
+        if (jj + 1 < ii) acc1 -= Lf[(16 * R + ii) * kLd + 16 * R + jj + 1] * a[jj + 1];
+      }
+      a[ii] = (ii < col) ? 0.f : acc0 + acc1;
     }
     __syncwarp();
     if (c.lane < 16) {
@@ -221,7 +225,8 @@ __device__ __forceinline__ void prep_inverse(const PrepCtx& c) {
     float y[4] = {0.f, 0.f, 0.f, 0.f};
     if (tile < 2 * R) {
       const int n0 = 8 * tile;
-      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      // two accumulator chains over alternate k-steps, summed at the end
+      float x[4] = {0.f, 0.f, 0.f, 0.f}, x2[4] = {0.f, 0.f, 0.f, 0.f};
       const float* lr = Lf + (16 * R) * kLd;
 #pragma unroll
       for (int k0 = 0; k0 < K; k0 += 8) {
@@ -232,8 +237,11 @@ __device__ __forceinline__ void prep_inverse(const PrepCtx& c) {
         af[3] = tc::to_tf32(lr[(gid + 8) * kLd + k0 + tig + 4]);
         bf[0] = tc::to_tf32(Lf[(k0 + tig) * kLd + n0 + gid]);
         bf[1] = tc::to_tf32(Lf[(k0 + tig + 4) * kLd + n0 + gid]);
-        tc::mma_tf32_16x8x8(x, af, bf);
+        if ((k0 >> 3) & 1) tc::mma_tf32_16x8x8(x2, af, bf);
+        else tc::mma_tf32_16x8x8(x, af, bf);
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] += x2[u];
       float* xw = c.Xf + c.pw * 128;
       xw[gid * 8 + 2 * tig] = x[0];
       xw[gid * 8 + 2 * tig + 1] = x[1];

@@ -188,6 +188,8 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       ok = ok && mbar_wait(&ss->full[s], (c >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
+      // full chunk: the Gram product can start at once (a partial one waits for its zeroed rows)
+      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
       prep_store_gb(pc, s, gv, bv);
       if (nv < kChunk) {
         // rows past the sequence end hold the next sequence's tokens: clear them
@@ -200,7 +202,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         fence_proxy_async_smem();
       }
       named_bar_sync(kBarPrep, kNumPrep);
-      if (pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
+      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
       prep_scan(pc, s);
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays(pc, s, nv);
