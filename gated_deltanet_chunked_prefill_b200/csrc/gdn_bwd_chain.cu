@@ -58,6 +58,7 @@ struct Small {
   int abort_flag;
 };
 constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a block can opt into");
 
 constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T
 constexpr uint32_t kColDa = 64;   // 64: dS' K^T

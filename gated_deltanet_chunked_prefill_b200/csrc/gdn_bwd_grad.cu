@@ -50,7 +50,7 @@ constexpr uint32_t kOffA2 = 160u * 1024;  // A diag(beta)
 constexpr uint32_t kOffP = 168u * 1024;   // scale P; then dPm
 constexpr uint32_t kOffA = 176u * 1024;   // A; then dG + dG^T
 constexpr uint32_t kOffDA = 184u * 1024;  // dA; then X = dA A^T
-constexpr uint32_t kOffLf = 192u * 1024;  // fp32 64 x 65: L -> A; then dG
+constexpr uint32_t kOffLf = 192u * 1024;  // fp32 64 x kLd: L -> A; then dG
 constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 
 // Per-token partial sums, one slot per producer so that every slot entry is written exactly
@@ -68,6 +68,7 @@ struct Small {
   int abort_flag;
 };
 constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a block can opt into");
 
 // TMEM columns
 constexpr uint32_t kColG = 0;     // [K;Q] K^T (64)
@@ -447,8 +448,17 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // dbeta_j += sum_i dA2_ij A_ij ;  dA = dA2 diag(beta) -> bf16
       const float* bet = ss->cs.bet[0];
       uint32_t w[16];
+      {
+        const float4* src = reinterpret_cast<const float4*>(Lf + i * kLd + j0);
 #pragma unroll
-      for (int u = 0; u < 32; ++u) colv[u] = mvals[u] * Lf[i * kLd + j0 + u];
+        for (int u = 0; u < 8; ++u) {
+          const float4 t = src[u];
+          colv[4 * u] = mvals[4 * u] * t.x;
+          colv[4 * u + 1] = mvals[4 * u + 1] * t.y;
+          colv[4 * u + 2] = mvals[4 * u + 2] * t.z;
+          colv[4 * u + 3] = mvals[4 * u + 3] * t.w;
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         w[u] = pack_bf16(mvals[2 * u] * bet[j0 + 2 * u], mvals[2 * u + 1] * bet[j0 + 2 * u + 1]);
@@ -555,8 +565,11 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         dg[jj] = dl * bi * run;
       }
       // A (fp32) in Lf has no readers left: dG takes its place
+      {
+        float4* dst = reinterpret_cast<float4*>(Lf + i * kLd + j0);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) Lf[i * kLd + j0 + jj] = dg[jj];
+        for (int u = 0; u < 8; ++u) dst[u] = make_float4(dg[4 * u], dg[4 * u + 1], dg[4 * u + 2], dg[4 * u + 3]);
+      }
       const float cs_ = warp_transpose_sum(colv);
       ss->dgam[kSlotFL + qd][j0 + lane] = -cs_;         // qd in {0, 1}
       ss->dgam[kSlotFLRow + hh][i] = rowsum;
@@ -569,10 +582,13 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int i = r, j0 = hh * 32;
     const float* Lf = reinterpret_cast<const float*>(sm + kOffLf);
     uint32_t w[16];
+    const float4* rowv = reinterpret_cast<const float4*>(Lf + i * kLd + j0);
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int ja = j0 + 2 * u;
-      w[u] = pack_bf16(Lf[i * kLd + ja] + Lf[ja * kLd + i], Lf[i * kLd + ja + 1] + Lf[(ja + 1) * kLd + i]);
+    for (int u = 0; u < 8; ++u) {
+      const float4 t = rowv[u];
+      const int ja = j0 + 4 * u;
+      w[2 * u] = pack_bf16(t.x + Lf[ja * kLd + i], t.y + Lf[(ja + 1) * kLd + i]);
+      w[2 * u + 1] = pack_bf16(t.z + Lf[(ja + 2) * kLd + i], t.w + Lf[(ja + 3) * kLd + i]);
     }
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4)

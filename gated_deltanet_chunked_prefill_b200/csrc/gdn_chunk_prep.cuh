@@ -17,7 +17,11 @@
 
 namespace gdn {
 
-constexpr int kLd = 65;           // row stride (floats) of the fp32 64 x 64 scratch
+// Row stride (floats) of the fp32 64 x 64 scratch. 68 = 4 mod 32 makes the m16n8k8 A
+// fragments (row gid, column tig) hit 32 distinct banks; row-per-thread accesses go through
+// 16-byte vectors (8 threads per phase, rows 4 banks apart: conflict-free) and
+// column-per-thread accesses stay scalar (consecutive rows, distinct banks).
+constexpr int kLd = 68;
 constexpr int kPrepThreads = 256;
 
 // per-chunk scalars, double-buffered by chunk parity
@@ -152,8 +156,9 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
       else run = (j >= i) ? 1.f : run * et[jj + 1];
       vals[jj] = (j < i) ? bi * vals[jj] * run : 0.f;
     }
+    float4* dst = reinterpret_cast<float4*>(c.Lf + i * kLd + j0);
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) c.Lf[i * kLd + j0 + jj] = vals[jj];
+    for (int u = 0; u < 8; ++u) dst[u] = make_float4(vals[4 * u], vals[4 * u + 1], vals[4 * u + 2], vals[4 * u + 3]);
   } else {
 #pragma unroll
     for (int jj = 31; jj >= 0; --jj) {
@@ -189,6 +194,171 @@ __device__ __forceinline__ void scale_rows_tile(const PrepCtx& c, uint8_t* tile,
   }
 #pragma unroll
   for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(qa[m]) = scale_chunk(qv[m], fs[m]);
+}
+
+// Scale rows of a [64 x 128] bf16 tile (two 8KB 128B-swizzled sub-tiles, sub-tile 1 at
+// +sub_stride) by f[row] * mult, in place, with nt threads (t = this thread's index).
+__device__ __forceinline__ void scale_rows_tile_part(uint8_t* tile, uint32_t sub_stride, const float* f, float mult,
+                                                     int t, int nt) {
+  for (int idx = t; idx < 1024; idx += nt) {
+    const int row = idx >> 4, half = (idx >> 3) & 1, ch = idx & 7;
+    uint4* q = reinterpret_cast<uint4*>(tile + half * sub_stride + row * 128 + ch * 16);
+    *q = scale_chunk(*q, f[row] * mult);
+  }
+}
+
+// 16 x 16 unit-lower diagonal blocks of (I + L) inverted in place in Lf by forward
+// substitution. Called by warps 0..3 of the group: warp R inverts block R, lane = column
+// (lanes 16..31 mirror 0..15). Rows are read as 16-byte broadcasts. No group barrier.
+__device__ __forceinline__ void prep_diag_inverse(const PrepCtx& c) {
+  float* Lf = c.Lf;
+  const int R = c.pw, col = c.lane & 15;
+  float a[16];
+#pragma unroll
+  for (int ii = 0; ii < 16; ++ii) {
+    float l[16];
+    const float4* row = reinterpret_cast<const float4*>(Lf + (16 * R + ii) * kLd + 16 * R);
+#pragma unroll
+    for (int q4 = 0; q4 < (ii + 3) / 4; ++q4) {
+      const float4 t = row[q4];
+      l[4 * q4] = t.x; l[4 * q4 + 1] = t.y; l[4 * q4 + 2] = t.z; l[4 * q4 + 3] = t.w;
+    }
+    // two accumulation chains (even / odd jj) halve the dependent latency
+    float acc0 = (ii == col) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < ii; jj += 2) {
+      acc0 -= l[jj] * a[jj];
+      if (jj + 1 < ii) acc1 -= l[jj + 1] * a[jj + 1];
+    }
+    a[ii] = (ii < col) ? 0.f : acc0 + acc1;
+  }
+  __syncwarp();
+  if (c.lane < 16) {
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) Lf[(16 * R + ii) * kLd + 16 * R + col] = a[ii];
+  }
+}
+
+// m16n8k8 tf32 product without the volatile qualifier (a pure register operation, so the
+// compiler may interleave independent products)
+__device__ __forceinline__ void mma_tf32_free(float* d, const uint32_t* a, const uint32_t* b) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// A fragment (16 x 8 at rows r0.., columns k0..) of the fp32 row-major scratch
+__device__ __forceinline__ void lf_afrag(const float* Lf, int r0, int k0, int gid, int tig, uint32_t* af) {
+  af[0] = tc::to_tf32(Lf[(r0 + gid) * kLd + k0 + tig]);
+  af[1] = tc::to_tf32(Lf[(r0 + gid + 8) * kLd + k0 + tig]);
+  af[2] = tc::to_tf32(Lf[(r0 + gid) * kLd + k0 + tig + 4]);
+  af[3] = tc::to_tf32(Lf[(r0 + gid + 8) * kLd + k0 + tig + 4]);
+}
+
+// B fragments (k rows 0..7 -> bf[0..1], rows 8..15 -> bf[2..3]) of a 16 x 8 tile held in
+// accumulator layout (lane 4 r + c / 2 holds rows r, r + 8 at columns c, c + 1), by shuffles
+__device__ __forceinline__ void acc_to_bfrag(const float* x, int lane, uint32_t* bf) {
+  const int gid = lane >> 2, tig = lane & 3;
+  const int s0 = tig * 4 + (gid >> 1), s1 = s0 + 16;
+  const bool odd = gid & 1;
+#pragma unroll
+  for (int kk = 0; kk < 2; ++kk) {
+    const float e0 = __shfl_sync(0xffffffffu, x[2 * kk], s0), o0 = __shfl_sync(0xffffffffu, x[2 * kk + 1], s0);
+    const float e1 = __shfl_sync(0xffffffffu, x[2 * kk], s1), o1 = __shfl_sync(0xffffffffu, x[2 * kk + 1], s1);
+    bf[2 * kk] = tc::to_tf32(odd ? o0 : e0);
+    bf[2 * kk + 1] = tc::to_tf32(odd ? o1 : e1);
+  }
+}
+
+// A = (I + L)^-1 from the inverted diagonal blocks D_R (prep_diag_inverse) and the strictly
+// lower blocks L_{R,R'} of Lf, which it only reads: one 8-column strip per warp of the
+// group, no group barrier. Warp w owns columns 8w .. 8w+7, whose first nonzero block row
+// is R0 = w / 2:
+//   X_R0 = D_R0 (its columns),   X_R = -D_R sum_{R0 <= R' < R} L_{R,R'} X_R'   (R > R0)
+// as m16n8k8 tf32 products. Each solved block adds its term to every later block row at
+// once, so the dependent path is one (L, D) product pair per block row.
+// Out: x[R] = rows 16R + gid (+8) at columns 8w + 2 tig (+1), accumulator layout.
+// R0 is a template parameter so that each warp's path is straight-line code and the
+// compiler can issue every fragment load ahead of the dependent products.
+template <int R0>
+__device__ __forceinline__ void prep_solve_strip_t(const PrepCtx& c, float (&x)[4][4]) {
+  const float* Lf = c.Lf;
+  const int gid = c.lane >> 2, tig = c.lane & 3;
+  const int n0 = 8 * c.pw;
+  float t[4][4];
+#pragma unroll
+  for (int R = 0; R < 4; ++R)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) t[R][u] = 0.f;
+#pragma unroll
+  for (int R = 0; R < R0; ++R)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[R][u] = 0.f;
+  {
+    const float* d = Lf + (16 * R0 + gid) * kLd + n0 + 2 * tig;
+    x[R0][0] = d[0];
+    x[R0][1] = d[1];
+    x[R0][2] = d[8 * kLd];
+    x[R0][3] = d[8 * kLd + 1];
+  }
+#pragma unroll
+  for (int R = R0; R < 4; ++R) {
+    if (R > R0) {
+      uint32_t bt[4];
+      acc_to_bfrag(t[R], c.lane, bt);
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        uint32_t af[4];
+        lf_afrag(Lf, 16 * R, 16 * R + 8 * kk, gid, tig, af);
+        mma_tf32_free(y, af, bt + 2 * kk);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[R][u] = -y[u];
+    }
+    if (R < 3) {
+      uint32_t bx[4];
+      acc_to_bfrag(x[R], c.lane, bx);
+#pragma unroll
+      for (int R2 = R + 1; R2 < 4; ++R2) {
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          uint32_t af[4];
+          lf_afrag(Lf, 16 * R2, 16 * R + 8 * kk, gid, tig, af);
+          mma_tf32_free(t[R2], af, bx + 2 * kk);
+        }
+      }
+    }
+  }
+}
+__device__ __forceinline__ void prep_solve_strip(const PrepCtx& c, float (&x)[4][4]) {
+  switch (c.pw >> 1) {                       // uniform over the warp
+    case 0: prep_solve_strip_t<0>(c, x); break;
+    case 1: prep_solve_strip_t<1>(c, x); break;
+    case 2: prep_solve_strip_t<2>(c, x); break;
+    default: prep_solve_strip_t<3>(c, x); break;
+  }
+}
+
+// A2 = A diag(beta) and B2 = A diag(beta exp(gam)) -> bf16 (128B-swizzled rows at a2_addr,
+// b2_addr) straight from prep_solve_strip's fragments.
+__device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const float (&x)[4][4], uint32_t a2_addr,
+                                                 uint32_t b2_addr) {
+  const int w = c.pw, gid = c.lane >> 2, tig = c.lane & 3;
+  const int j = 8 * w + 2 * tig;
+  const float b0 = c.cs->bet[s][j], b1 = c.cs->bet[s][j + 1];
+  const float e0 = b0 * c.cs->eg[s][j], e1 = b1 * c.cs->eg[s][j + 1];
+#pragma unroll
+  for (int R = 0; R < 4; ++R) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 16 * R + gid + 8 * h;
+      const uint32_t off = tc::sw128(i, w) + 4 * tig;
+      const float v0 = x[R][2 * h], v1 = x[R][2 * h + 1];
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2_addr + off), "r"(tc::pack_bf16(v0 * b0, v1 * b1)) : "memory");
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(b2_addr + off), "r"(tc::pack_bf16(v0 * e0, v1 * e1)) : "memory");
+    }
+  }
 }
 
 // A = (I + L)^-1 in place in Lf: 16x16 diagonal blocks by forward substitution (warps
@@ -243,10 +413,8 @@ __device__ __forceinline__ void prep_inverse(const PrepCtx& c) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) x[u] += x2[u];
       float* xw = c.Xf + c.pw * 128;
-      xw[gid * 8 + 2 * tig] = x[0];
-      xw[gid * 8 + 2 * tig + 1] = x[1];
-      xw[(gid + 8) * 8 + 2 * tig] = x[2];
-      xw[(gid + 8) * 8 + 2 * tig + 1] = x[3];
+      *reinterpret_cast<float2*>(xw + gid * 8 + 2 * tig) = make_float2(x[0], x[1]);
+      *reinterpret_cast<float2*>(xw + (gid + 8) * 8 + 2 * tig) = make_float2(x[2], x[3]);
       __syncwarp();
       const float* dr = Lf + (16 * R) * kLd + 16 * R;
 #pragma unroll
@@ -273,14 +441,20 @@ __device__ __forceinline__ void prep_inverse(const PrepCtx& c) {
   }
 }
 
-// A2 = A diag(beta) -> bf16 rows at a2_addr; with a_addr != 0 also A -> bf16 (thread: 16
-// columns of one row).
-__device__ __forceinline__ void prep_write_a(const PrepCtx& c, int s, uint32_t a2_addr, uint32_t a_addr) {
-  const int i = c.pt >> 2, qq = c.pt & 3;
+// A2 = A diag(beta) -> bf16 rows at a2_addr; with a_addr != 0 also A -> bf16, with
+// b2_addr != 0 also B2 = A diag(beta exp(gam)) -> bf16 (thread: 16 columns of one row; a
+// warp covers 32 consecutive rows of one 16-column quarter).
+__device__ __forceinline__ void prep_write_a(const PrepCtx& c, int s, uint32_t a2_addr, uint32_t a_addr,
+                                             uint32_t b2_addr = 0) {
+  const int i = c.pt & 63, qq = c.pt >> 6;
   const float* bet = c.cs->bet[s];
   float a[16];
+  const float4* src = reinterpret_cast<const float4*>(c.Lf + i * kLd + qq * 16);
 #pragma unroll
-  for (int u = 0; u < 16; ++u) a[u] = c.Lf[i * kLd + qq * 16 + u];
+  for (int u = 0; u < 4; ++u) {
+    const float4 t = src[u];
+    a[4 * u] = t.x; a[4 * u + 1] = t.y; a[4 * u + 2] = t.z; a[4 * u + 3] = t.w;
+  }
   uint32_t w[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
@@ -289,6 +463,16 @@ __device__ __forceinline__ void prep_write_a(const PrepCtx& c, int s, uint32_t a
   }
   st_shared_v4(a2_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
   st_shared_v4(a2_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  if (b2_addr) {
+    const float* eg = c.cs->eg[s];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j0 = qq * 16 + 2 * u;
+      w[u] = tc::pack_bf16(a[2 * u] * (bet[j0] * eg[j0]), a[2 * u + 1] * (bet[j0 + 1] * eg[j0 + 1]));
+    }
+    st_shared_v4(b2_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+    st_shared_v4(b2_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  }
   if (a_addr) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) w[u] = tc::pack_bf16(a[2 * u], a[2 * u + 1]);

@@ -2,26 +2,28 @@
 // dk = dv = 128, 64-token chunks. One CTA runs the whole chunk sequence of one work
 // item (a (sequence, v-head) unit, or one segment of it under context parallelism).
 //
-// The recurrence is carried as S = h^T (dv x dk, fp32, in the epilogue threads'
-// registers) so that every tensor-core product has M = 128 rows = the dv rows of S
-// (or the 128 stacked K;Q token rows of the Gram product). Per chunk (gam = chunk-local
-// inclusive cumsum of g, E_ij = exp(gam_i - gam_j)):
+// The recurrence is carried as S = h^T (dv x dk, fp32, in TMEM) so that every
+// tensor-core product has M = 128 rows = the dv rows of S (or the dk rows of W^T, or the
+// 128 stacked K;Q token rows of the Gram product). Per chunk (gam = chunk-local inclusive
+// cumsum of g, E_ij = exp(gam_i - gam_j)):
 //
-//   prep warpgroup (state independent, overlaps the previous chunk's chain):
+//   prep warps (state independent, overlap the previous chunk's chain):
 //     G  = [K;Q] K^T                               tcgen05, M=128 N=64 K=128
 //     L  = strict_lower(diag(beta) KK^T * E),  A = (I + L)^-1      (fp32, CUDA cores)
-//     A2 = A diag(beta) -> bf16;   P = lower_incl(QK^T * E) -> bf16;  Q <- diag(exp(gam)) Q
-//   epilogue warpgroups (the sequential chain):
-//     (a) D1 = S_bf16 [K ; Q~]^T                   tcgen05, M=128 N=128 K=128
-//     (b) Y^T = V^T - D1[:, K part] diag(exp(gam))  -> bf16
-//     (c) Dl  = Y^T A2^T                           tcgen05, M=128 N=64 K=64   (= Delta^T)
-//     (d) Delta^T -> bf16, Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
-//     (e) D1[:, Q part] += Delta^T P^T;  DS = Delta~^T K   (K read MN-major from the TMA tile)
-//     (f) S = exp(gam_n) S + DS (fp32);  O = scale * D1[:, Q part]
-// i.e. O = scale[diag(e^gam) Q h + (QK^T*E*M) Delta], Delta = A diag(beta)(V - diag(e^gam) K h),
-// h' = e^gam_n h + (diag(e^(gam_n-gam)) K)^T Delta: the WY/UT chunk form of the gated delta
-// rule ("FlashQLA resource", section 3: fused warp-specialised kernels that overlap data
-// movement, tensor-core and CUDA-core work).
+//     A2 = A diag(beta), B2 = A diag(beta exp(gam)) -> bf16;  P = lower_incl(QK^T * E) -> bf16
+//     Q <- diag(exp(gam)) Q  (Q~)
+//     U^T = V^T A2^T   into the chunk's Delta accumulator          tcgen05, M=128 N=64 K=64
+//     W^T = K^T B2^T   -> -W^T in bf16 over the V tile              tcgen05, M=128 N=64 K=64
+//   epilogue warps (the sequential chain, two tensor-core round trips per chunk):
+//     (a) Delta^T = U^T - S_bf16 W^T;  D_Q = S_bf16 Q~^T             tcgen05, M=128 N=64 K=128
+//     (b) Delta^T -> bf16, Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
+//     (c) D_Q += Delta^T P^T;  S += Delta~^T K   (K read MN-major from the TMA tile)
+//     (d) S -> bf16 for the next chunk's products;  O = scale * D_Q
+// i.e. Delta = U - W h with U = A diag(beta) V and W = A diag(beta e^gam) K,
+// O = scale[diag(e^gam) Q h + (QK^T*E*M) Delta], h' = e^gam_n h + (diag(e^(gam_n-gam)) K)^T Delta:
+// the WY/UT chunk form of the gated delta rule ("Gated Delta Networks" paper, section 3.3,
+// hardware-efficient chunkwise training; "FlashQLA resource", section 3: fused
+// warp-specialised kernels that overlap data movement, tensor-core and CUDA-core work).
 #include <cudaTypedefs.h>
 
 #include "gdn_chunk_prep.cuh"
@@ -43,13 +45,14 @@ constexpr int kBarPrep = 1, kBarEpi = 2;  // named barrier ids
 
 // shared memory layout (bytes from a 1024-aligned base)
 constexpr uint32_t kStageBytes = 48u * 1024u;   // [K0 Q0 K1 Q1] (8KB each) + [V0 V1]
-constexpr uint32_t kOffV = 32u * 1024u;         // within a stage
-constexpr uint32_t kOffA2 = 96u * 1024u;        // 2 x 8KB  A diag(beta), bf16, SW128 rows
+constexpr uint32_t kOffV = 32u * 1024u;         // within a stage: V, then -W^T ([dk][token] rows)
+constexpr uint32_t kOffA2 = 96u * 1024u;        // 8KB      A diag(beta), bf16, SW128 rows
+constexpr uint32_t kOffB2 = 104u * 1024u;       // 8KB      A diag(beta exp(gam)), bf16
 constexpr uint32_t kOffP = 112u * 1024u;        // 2 x 8KB  masked decayed QK^T, bf16
 constexpr uint32_t kOffSb = 128u * 1024u;       // 32KB     S in bf16 (two 64-col sub-tiles)
-constexpr uint32_t kOffYt = 160u * 1024u;       // 16KB     Y^T, then Delta^T
+constexpr uint32_t kOffYt = 160u * 1024u;       // 16KB     Delta^T, bf16 [dv][token]
 constexpr uint32_t kOffDt = 176u * 1024u;       // 16KB     Delta~^T, then O staging
-constexpr uint32_t kOffLf = 192u * 1024u;       // fp32 [64][65] L, inverted in place
+constexpr uint32_t kOffLf = 192u * 1024u;       // fp32 [64][kLd] L, inverted in place
 constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 
 struct Small {
@@ -57,22 +60,23 @@ struct Small {
   float Xf[8 * 128];      // inverse scratch: one 16 x 8 tile per prep warp
   float wsum[16];         // warm-up window search: per-warp partial sums
   int ws;                 // warm-up start token (context parallelism)
-  uint64_t full[2], prep_full[2], gdone, mma_done;
+  uint64_t full[2], prep_full[2], gdone, wdone, mma_done;
   uint32_t tmem_base;
   int abort_flag;
 };
 constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a block can opt into");
 
 // TMEM columns (fp32, 128 lanes)
-constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T
-constexpr uint32_t kColD1 = 64;   // 128: S [K;Q~]^T, Q part accumulates Delta^T P^T
-constexpr uint32_t kColDd = 192;  // 64: Delta^T
+constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T, then W^T (prep)
+constexpr uint32_t kColDQ = 64;   // 64: S Q~^T, accumulates Delta^T P^T
+constexpr uint32_t kColDd = 128;  // 2 x 64: U^T - S W^T = Delta^T, by chunk parity
 constexpr uint32_t kColS = 256;   // 128: the fp32 state S (dv x dk), updated in place
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kIdG = idesc_bf16(128, 64, false, false);
-constexpr uint32_t kIdA = idesc_bf16(128, 128, false, false);
-constexpr uint32_t kIdC = idesc_bf16(128, 64, false, false);
+constexpr uint32_t kId64 = idesc_bf16(128, 64, false, false);    // A, B K-major
+constexpr uint32_t kId64km = idesc_bf16(128, 64, false, true);   // B MN-major
+constexpr uint32_t kId64mk = idesc_bf16(128, 64, true, false);   // A MN-major
 constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);
 
 
@@ -103,6 +107,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(&ss->prep_full[s], 1);
     }
     mbar_init(&ss->gdone, 1);
+    mbar_init(&ss->wdone, 1);
     mbar_init(&ss->mma_done, 1);
     ss->abort_flag = 0;
     ss->ws = it.s;
@@ -174,22 +179,31 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int pt = threadIdx.x;            // 0..255
     PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), ss->Xf, &ss->cs, tmem, kColG, pt, warp, lane, kBarPrep};
     bool ok = true;
+    // g, beta of a chunk (0 past the sequence end); loaded one chunk ahead
+    auto load_gb = [&](int c, float& gv, float& bv) {
+      const int t0 = ws + c * kChunk;
+      gv = 0.f;
+      bv = 0.f;
+      if (pt < kChunk && t0 + pt < it.e) {
+        const size_t gi = (size_t)(it.b * p.T + t0 + pt) * p.Hv + it.j;
+        gv = p.g[gi];
+        bv = __bfloat162float(beta[gi]);
+      }
+    };
+    float gv_next = 0.f, bv_next = 0.f;
+    if (nchunks > 0) load_gb(0, gv_next, bv_next);
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       const int t0 = ws + c * kChunk;
       const int nv = min(kChunk, it.e - t0);
       uint8_t* st = sm + s * kStageBytes;
-      // g, beta of the chunk (masked beyond the sequence end)
-      float gv = 0.f, bv = 0.f;
-      if (pt < kChunk && pt < nv) {
-        const size_t gi = (size_t)(it.b * p.T + t0 + pt) * p.Hv + it.j;
-        gv = p.g[gi];
-        bv = __bfloat162float(beta[gi]);
-      }
+      const uint32_t st_addr = sbase + s * kStageBytes;
+      const float gv = gv_next, bv = bv_next;
+      if (c + 1 < nchunks) load_gb(c + 1, gv_next, bv_next);
       ok = ok && mbar_wait(&ss->full[s], (c >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       // full chunk: the Gram product can start at once (a partial one waits for its zeroed rows)
-      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
+      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColG, st_addr, &ss->gdone);
       prep_store_gb(pc, s, gv, bv);
       if (nv < kChunk) {
         // rows past the sequence end hold the next sequence's tokens: clear them
@@ -202,7 +216,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         fence_proxy_async_smem();
       }
       named_bar_sync(kBarPrep, kNumPrep);
-      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
+      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColG, st_addr, &ss->gdone);
       prep_scan(pc, s);
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays(pc, s, nv);
@@ -210,11 +224,53 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       prep_masks(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
-      // Q <- diag(exp(gam)) Q, in place (the Gram product has consumed Q)
-      scale_rows_tile(pc, st + 8192, 16384, ss->cs.eg[s], 1.f);
-      prep_inverse(pc);
-      prep_write_a(pc, s, sbase + kOffA2 + s * 8192u, 0);
+      // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- diag(exp(gam)) Q
+      // in place (the Gram product has consumed Q); then one column strip of A per warp
+      if (warp < 4) prep_diag_inverse(pc);
+      else scale_rows_tile_part(st + 8192, 16384, ss->cs.eg[s], 1.f, pt - 128, 128);
+      named_bar_sync(kBarPrep, kNumPrep);
+      {
+        float x[4][4];
+        prep_solve_strip(pc, x);
+        prep_store_strip(pc, s, x, sbase + kOffA2, sbase + kOffB2);
+      }
       fence_proxy_async_smem();
+      named_bar_sync(kBarPrep, kNumPrep);
+      // U^T = V^T A2^T (A = V tile read MN-major, dv halves 8KB apart) into this chunk's
+      // Delta accumulator; W^T = K^T B2^T (A = K tile read MN-major) over G
+      if (pt == 0 && ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          if (!it.zero_v)
+            umma_f16(tmem + kColDd + 64u * s, sdesc_sw128(st_addr + kOffV + ks * 2048, 8192, 1024),
+                     sdesc_sw128(sbase + kOffA2 + ks * 32, 16, 1024), kId64mk, ks > 0);
+          umma_f16(tmem + kColG, sdesc_sw128(st_addr + ks * 2048, 16384, 1024),
+                   sdesc_sw128(sbase + kOffB2 + ks * 32, 16, 1024), kId64mk, ks > 0);
+        }
+        umma_commit(&ss->wdone);
+      }
+      ok = ok && mbar_wait(&ss->wdone, c & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      // -W^T -> bf16 rows [dk][token] over the V tile (consumed by the U^T product)
+      {
+        const int qd = warp & 3, hc = warp >> 2;
+        const int r = 32 * qd + lane;
+        float v[32];
+        if (ok) tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + kColG + 32 * hc, v);
+        else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = 0.f;
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          st_shared_v4(st_addr + kOffV + sw128(r, 4 * hc + c4), pack_bf16(-v[8 * c4], -v[8 * c4 + 1]),
+                       pack_bf16(-v[8 * c4 + 2], -v[8 * c4 + 3]), pack_bf16(-v[8 * c4 + 4], -v[8 * c4 + 5]),
+                       pack_bf16(-v[8 * c4 + 6], -v[8 * c4 + 7]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);
     }
@@ -254,13 +310,18 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_before();
     named_bar_sync(kBarEpi, kNumEpi);
     uint32_t mph = 0;
+    // (a) Delta^T = U^T + S_bf16 (-W^T) (onto the prep's U^T; from zero when V is zero)
+    //     and D_Q = S_bf16 Q~^T
     auto issue_a = [&](int c) {
       tc_fence_after();
-      const uint32_t a0 = sbase + kOffSb, b0 = sbase + (c & 1) * kStageBytes;
+      const uint32_t a0 = sbase + kOffSb, st_addr = sbase + (c & 1) * kStageBytes;
+      const uint32_t dd = tmem + kColDd + 64u * (c & 1);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
-        umma_f16(tmem + kColD1, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024), kIdA, ks > 0);
+        const uint64_t sa = sdesc_sw128(a0 + off, 16, 1024);
+        umma_f16(dd, sa, sdesc_sw128(st_addr + kOffV + ks * 2048, 8192, 1024), kId64km, !it.zero_v || ks > 0);
+        umma_f16(tmem + kColDQ, sa, sdesc_sw128(st_addr + 8192 + off, 16, 1024), kId64, ks > 0);
       }
       umma_commit(&ss->mma_done);
     };
@@ -298,7 +359,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int s = c & 1;
       const int t0 = ws + c * kChunk;
       wait_mma();
-      const uint8_t* st = sm + s * kStageBytes;
       if (p.states != nullptr && t0 >= it.s && ok) {
         // backward support: this chunk's start state (the bf16 copy its products use)
         const uint8_t* srow = sm + kOffSb + hh * 16384u;
@@ -307,51 +367,10 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) dst[ch] = *reinterpret_cast<const uint4*>(srow + sw128(r, ch));
       }
-      // (b) Y^T = V^T - (S K^T) diag(exp(gam))
-      {
-        float y[32];
-        if (ok) tmem_ld32_sync(tmem + lane_base + kColD1 + hh * 32, y);
-        else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) y[u] = 0.f;
-        }
-        const uint8_t* vt = st + kOffV + (r >> 6) * 8192;
-        const int rc = (r & 63) >> 3, rb = (r & 7) * 2;
-        const float* eg = ss->cs.eg[s];
-        uint32_t w[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int j0 = hh * 32 + 2 * u, j1 = j0 + 1;
-          float v0 = 0.f, v1 = 0.f;
-          if (!it.zero_v) {
-            v0 = bf16_at(vt + j0 * 128 + ((rc ^ (j0 & 7)) << 4) + rb);
-            v1 = bf16_at(vt + j1 * 128 + ((rc ^ (j1 & 7)) << 4) + rb);
-          }
-          w[u] = pack_bf16(v0 - eg[j0] * y[2 * u], v1 - eg[j1] * y[2 * u + 1]);
-        }
-        const uint32_t yrow = sbase + kOffYt;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          st_shared_v4(yrow + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      named_bar_sync(kBarEpi, kNumEpi);
-      // (c) Delta^T = Y^T (A diag(beta))^T
-      if (et == 0 && ok) {
-        tc_fence_after();
-        const uint32_t a0 = sbase + kOffYt, b0 = sbase + kOffA2 + s * 8192u;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          umma_f16(tmem + kColDd, sdesc_sw128(a0 + ks * 32, 16, 1024), sdesc_sw128(b0 + ks * 32, 16, 1024), kIdC,
-                   ks > 0);
-        umma_commit(&ss->mma_done);
-      }
-      wait_mma();
-      // (d) Delta^T and Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
+      // (b) Delta^T and Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
       {
         float dd[32];
-        if (ok) tmem_ld32_sync(tmem + lane_base + kColDd + hh * 32, dd);
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColDd + 64u * s + hh * 32, dd);
         else {
 #pragma unroll
           for (int u = 0; u < 32; ++u) dd[u] = 0.f;
@@ -373,13 +392,13 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
-      // (e) O part += Delta^T P^T;  S += Delta~^T K   (S was pre-scaled by exp(gam_n))
+      // (c) D_Q += Delta^T P^T;  S += Delta~^T K   (S was pre-scaled by exp(gam_n))
       if (et == 0 && ok) {
         tc_fence_after();
         const uint32_t ya = sbase + kOffYt, pb = sbase + kOffP + s * 8192u;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          umma_f16(tmem + kColD1 + 64, sdesc_sw128(ya + ks * 32, 16, 1024), sdesc_sw128(pb + ks * 32, 16, 1024), kIdC,
+          umma_f16(tmem + kColDQ, sdesc_sw128(ya + ks * 32, 16, 1024), sdesc_sw128(pb + ks * 32, 16, 1024), kId64,
                    1);
         const uint32_t da = sbase + kOffDt, kb = sbase + s * kStageBytes;
 #pragma unroll
@@ -389,7 +408,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         umma_commit(&ss->mma_done);
       }
       wait_mma();
-      // (f) S -> bf16 copy for the next chunk's product;  O = scale * (Q part) -> registers
+      // (d) S -> bf16 copy for the next chunk's products;  O = scale * D_Q -> registers
       float oo[32];
       const int nv = ss->cs.nv[s];
       {
@@ -403,7 +422,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           }
           write_sb(v, h2);
         }
-        if (ok) tmem_ld32_sync(tmem + lane_base + kColD1 + 64 + hh * 32, oo);
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColDQ + hh * 32, oo);
         else {
 #pragma unroll
           for (int u = 0; u < 32; ++u) oo[u] = 0.f;
