@@ -11,6 +11,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "gdn_common.cuh"
 #include "tc_ptx.cuh"
@@ -22,6 +23,9 @@ namespace gdn {
 // 16-byte vectors (8 threads per phase, rows 4 banks apart: conflict-free) and
 // column-per-thread accesses stay scalar (consecutive rows, distinct banks).
 constexpr int kLd = 68;
+// Row stride (halves) of the fp16 64 x 64 variant of the scratch: 36 words = 4 mod 32, so
+// the m16n8k16 A fragments (row gid, word tig) hit 32 distinct banks.
+constexpr int kLdh = 72;
 constexpr int kPrepThreads = 256;
 
 // per-chunk scalars, double-buffered by chunk parity
@@ -48,6 +52,11 @@ __device__ __forceinline__ uint4 scale_chunk(uint4 v, float f) {
     h[i] = __floats2bfloat162_rn(x.x * f, x.y * f);
   }
   return v;
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -105,13 +114,15 @@ __device__ __forceinline__ void prep_decays(const PrepCtx& c, int s, int nv) {
   }
 }
 
-// Issue G = [K;Q] K^T (K at kq_addr: [K0 Q0 K1 Q1] 8KB sub-tiles) and commit to `bar`.
-__device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, uint64_t* bar) {
+// Issue G = [K;Q] K^T and commit to `bar`. K0, Q0 (8KB sub-tiles, dk 0..63) are adjacent
+// at kq_addr; K1, Q1 (dk 64..127) follow at kq_addr + half_stride.
+__device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, uint64_t* bar,
+                                           uint32_t half_stride = 16384u) {
   constexpr uint32_t id = tc::idesc_bf16(128, 64, false, false);
   tc::tc_fence_after();
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
-    const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+    const uint32_t off = (ks >> 2) * half_stride + (ks & 3) * 32u;
     tc::umma_f16(tmem_g, tc::sdesc_sw128(kq_addr + off, 16, 1024), tc::sdesc_sw128(kq_addr + off, 16, 1024), id,
                  ks > 0);
   }
@@ -123,6 +134,8 @@ __device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, ui
 // of exp(g_t) over t = j+1..i, walking j down: one exponential per row segment instead of
 // one per entry, no overflow, monotone underflow to 0. `ok` false: G treated as 0.
 // Ends with tcgen05 fence + group barrier.
+// kHalfL: L goes to the scratch as fp16 rows of stride kLdh instead of fp32 rows of kLd.
+template <bool kHalfL = false>
 __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_addr, float p_scale, bool ok) {
   const int qd = c.pw & 3, hc = c.pw >> 2;
   const int rr = 32 * qd + c.lane;
@@ -156,9 +169,17 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
       else run = (j >= i) ? 1.f : run * et[jj + 1];
       vals[jj] = (j < i) ? bi * vals[jj] * run : 0.f;
     }
-    float4* dst = reinterpret_cast<float4*>(c.Lf + i * kLd + j0);
+    if (kHalfL) {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(c.Lf) + i * kLdh + j0);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) dst[u] = make_float4(vals[4 * u], vals[4 * u + 1], vals[4 * u + 2], vals[4 * u + 3]);
+      for (int u = 0; u < 4; ++u)
+        dst[u] = make_uint4(pack_h2(vals[8 * u], vals[8 * u + 1]), pack_h2(vals[8 * u + 2], vals[8 * u + 3]),
+                            pack_h2(vals[8 * u + 4], vals[8 * u + 5]), pack_h2(vals[8 * u + 6], vals[8 * u + 7]));
+    } else {
+      float4* dst = reinterpret_cast<float4*>(c.Lf + i * kLd + j0);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) dst[u] = make_float4(vals[4 * u], vals[4 * u + 1], vals[4 * u + 2], vals[4 * u + 3]);
+    }
   } else {
 #pragma unroll
     for (int jj = 31; jj >= 0; --jj) {
@@ -337,6 +358,132 @@ __device__ __forceinline__ void prep_solve_strip(const PrepCtx& c, float (&x)[4]
     case 1: prep_solve_strip_t<1>(c, x); break;
     case 2: prep_solve_strip_t<2>(c, x); break;
     default: prep_solve_strip_t<3>(c, x); break;
+  }
+}
+
+// ---- fp16 variant of the inverse: L and the diagonal-block inverses D_R held as fp16
+// rows of stride kLdh (11-bit significand, as the tf32 products it replaces), the strip
+// products on m16n8k16 f16 tensor instructions (one per 16 x 16 block instead of two).
+
+// Diagonal 16 x 16 blocks, inverted in place (fp32 arithmetic, fp16 storage). Warps 0..3.
+__device__ __forceinline__ void prep_diag_inverse_h(const PrepCtx& c) {
+  __half* Lh = reinterpret_cast<__half*>(c.Lf);
+  const int R = c.pw, col = c.lane & 15;
+  float a[16];
+#pragma unroll
+  for (int ii = 0; ii < 16; ++ii) {
+    float l[16];
+    const uint4* row = reinterpret_cast<const uint4*>(Lh + (16 * R + ii) * kLdh + 16 * R);
+#pragma unroll
+    for (int q8 = 0; q8 < (ii + 7) / 8; ++q8) {
+      const uint4 t = row[q8];
+      const __half2* h = reinterpret_cast<const __half2*>(&t);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        l[8 * q8 + 2 * e] = f.x;
+        l[8 * q8 + 2 * e + 1] = f.y;
+      }
+    }
+    float acc0 = (ii == col) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < ii; jj += 2) {
+      acc0 -= l[jj] * a[jj];
+      if (jj + 1 < ii) acc1 -= l[jj + 1] * a[jj + 1];
+    }
+    a[ii] = (ii < col) ? 0.f : acc0 + acc1;
+  }
+  __syncwarp();
+  if (c.lane < 16) {
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) Lh[(16 * R + ii) * kLdh + 16 * R + col] = __float2half_rn(a[ii]);
+  }
+}
+
+__device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, const uint32_t* b) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// A fragment (16 x 16 at rows r0.., columns k0..) of the fp16 scratch: half pairs
+__device__ __forceinline__ void lh_afrag(const __half* Lh, int r0, int k0, int gid, int tig, uint32_t* af) {
+  const uint32_t* w0 = reinterpret_cast<const uint32_t*>(Lh + (r0 + gid) * kLdh + k0) + tig;
+  const uint32_t* w1 = reinterpret_cast<const uint32_t*>(Lh + (r0 + gid + 8) * kLdh + k0) + tig;
+  af[0] = w0[0];
+  af[1] = w1[0];
+  af[2] = w0[4];
+  af[3] = w1[4];
+}
+
+// B fragment (k rows 0..15 of a 16 x 8 tile in accumulator layout) as fp16 pairs, by
+// shuffles: b0 = rows 2 tig, 2 tig + 1 and b1 = rows 2 tig + 8, 2 tig + 9, at column gid.
+__device__ __forceinline__ void acc_to_bfrag_h(const float* x, int lane, uint32_t* bf) {
+  const int gid = lane >> 2, tig = lane & 3;
+  const int sa = 8 * tig + (gid >> 1), sb = sa + 4;
+  const bool odd = gid & 1;
+  const float a0 = __shfl_sync(0xffffffffu, x[0], sa), a1 = __shfl_sync(0xffffffffu, x[1], sa);
+  const float a2 = __shfl_sync(0xffffffffu, x[2], sa), a3 = __shfl_sync(0xffffffffu, x[3], sa);
+  const float b0 = __shfl_sync(0xffffffffu, x[0], sb), b1 = __shfl_sync(0xffffffffu, x[1], sb);
+  const float b2 = __shfl_sync(0xffffffffu, x[2], sb), b3 = __shfl_sync(0xffffffffu, x[3], sb);
+  bf[0] = pack_h2(odd ? a1 : a0, odd ? b1 : b0);
+  bf[1] = pack_h2(odd ? a3 : a2, odd ? b3 : b2);
+}
+
+// Column strip of A = (I + L)^-1 for warp w (columns 8w..8w+7, first block row R0 = w/2),
+// as prep_solve_strip_t, on the fp16 scratch.
+template <int R0>
+__device__ __forceinline__ void prep_solve_strip_h_t(const PrepCtx& c, float (&x)[4][4]) {
+  const __half* Lh = reinterpret_cast<const __half*>(c.Lf);
+  const int gid = c.lane >> 2, tig = c.lane & 3;
+  const int n0 = 8 * c.pw;
+  float t[4][4];
+#pragma unroll
+  for (int R = 0; R < 4; ++R)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) t[R][u] = 0.f;
+#pragma unroll
+  for (int R = 0; R < R0; ++R)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[R][u] = 0.f;
+  {
+    const __half2* d0 = reinterpret_cast<const __half2*>(Lh + (16 * R0 + gid) * kLdh + n0 + 2 * tig);
+    const __half2* d1 = reinterpret_cast<const __half2*>(Lh + (16 * R0 + gid + 8) * kLdh + n0 + 2 * tig);
+    const float2 f0 = __half22float2(*d0), f1 = __half22float2(*d1);
+    x[R0][0] = f0.x;
+    x[R0][1] = f0.y;
+    x[R0][2] = f1.x;
+    x[R0][3] = f1.y;
+  }
+#pragma unroll
+  for (int R = R0; R < 4; ++R) {
+    if (R > R0) {
+      uint32_t bt[2], af[4];
+      acc_to_bfrag_h(t[R], c.lane, bt);
+      lh_afrag(Lh, 16 * R, 16 * R, gid, tig, af);
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16_16816(y, af, bt);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[R][u] = -y[u];
+    }
+    if (R < 3) {
+      uint32_t bx[2];
+      acc_to_bfrag_h(x[R], c.lane, bx);
+#pragma unroll
+      for (int R2 = R + 1; R2 < 4; ++R2) {
+        uint32_t af[4];
+        lh_afrag(Lh, 16 * R2, 16 * R, gid, tig, af);
+        mma_f16_16816(t[R2], af, bx);
+      }
+    }
+  }
+}
+__device__ __forceinline__ void prep_solve_strip_h(const PrepCtx& c, float (&x)[4][4]) {
+  switch (c.pw >> 1) {                       // uniform over the warp
+    case 0: prep_solve_strip_h_t<0>(c, x); break;
+    case 1: prep_solve_strip_h_t<1>(c, x); break;
+    case 2: prep_solve_strip_h_t<2>(c, x); break;
+    default: prep_solve_strip_h_t<3>(c, x); break;
   }
 }
 

@@ -9,13 +9,15 @@
 //
 //   prep warps (state independent, overlap the previous chunk's chain):
 //     G  = [K;Q] K^T                               tcgen05, M=128 N=64 K=128
-//     L  = strict_lower(diag(beta) KK^T * E),  A = (I + L)^-1      (fp32, CUDA cores)
+//     L  = strict_lower(diag(beta) KK^T * E) (fp16),  A = (I + L)^-1: 16 x 16 diagonal blocks
+//          by substitution (CUDA cores), one column strip per warp on m16n8k16 f16 products
 //     A2 = A diag(beta), B2 = A diag(beta exp(gam)) -> bf16;  P = lower_incl(QK^T * E) -> bf16
 //     Q <- diag(exp(gam)) Q  (Q~)
 //     U^T = V^T A2^T   into the chunk's Delta accumulator          tcgen05, M=128 N=64 K=64
-//     W^T = K^T B2^T   -> -W^T in bf16 over the V tile              tcgen05, M=128 N=64 K=64
+//     W   = B2 K       -> -W in bf16 over the V tile (token rows)   tcgen05, M=64 N=128 K=64
 //   epilogue warps (the sequential chain, two tensor-core round trips per chunk):
-//     (a) Delta^T = U^T - S_bf16 W^T;  D_Q = S_bf16 Q~^T             tcgen05, M=128 N=64 K=128
+//     (a) [D_Q | Delta^T] += S_bf16 [Q~ ; -W]^T  (D_Q from zero, Delta^T onto U^T)
+//                                                                  tcgen05, M=128 N=128 K=128
 //     (b) Delta^T -> bf16, Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
 //     (c) D_Q += Delta^T P^T;  S += Delta~^T K   (K read MN-major from the TMA tile)
 //     (d) S -> bf16 for the next chunk's products;  O = scale * D_Q
@@ -44,23 +46,25 @@ constexpr int kNumPrep = 256, kNumEpi = 256;
 constexpr int kBarPrep = 1, kBarEpi = 2;  // named barrier ids
 
 // shared memory layout (bytes from a 1024-aligned base)
-constexpr uint32_t kStageBytes = 48u * 1024u;   // [K0 Q0 K1 Q1] (8KB each) + [V0 V1]
-constexpr uint32_t kOffV = 32u * 1024u;         // within a stage: V, then -W^T ([dk][token] rows)
+constexpr uint32_t kStageBytes = 48u * 1024u;   // [K0 Q0 V0 | K1 Q1 V1], 8KB 128B-swizzled sub-tiles
+constexpr uint32_t kHalf = 24u * 1024u;         // feature columns 64..127 of K, Q, V
+constexpr uint32_t kOffQ = 8u * 1024u;          // within a half
+constexpr uint32_t kOffV = 16u * 1024u;         // within a half: V, then -W (token rows)
 constexpr uint32_t kOffA2 = 96u * 1024u;        // 8KB      A diag(beta), bf16, SW128 rows
 constexpr uint32_t kOffB2 = 104u * 1024u;       // 8KB      A diag(beta exp(gam)), bf16
 constexpr uint32_t kOffP = 112u * 1024u;        // 2 x 8KB  masked decayed QK^T, bf16
 constexpr uint32_t kOffSb = 128u * 1024u;       // 32KB     S in bf16 (two 64-col sub-tiles)
 constexpr uint32_t kOffYt = 160u * 1024u;       // 16KB     Delta^T, bf16 [dv][token]
 constexpr uint32_t kOffDt = 176u * 1024u;       // 16KB     Delta~^T, then O staging
-constexpr uint32_t kOffLf = 192u * 1024u;       // fp32 [64][kLd] L, inverted in place
-constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
+constexpr uint32_t kOffLf = 192u * 1024u;       // fp16 [64][kLdh] L, diagonal blocks inverted in place
+constexpr uint32_t kOffSmall = kOffLf + 64u * kLdh * 2u;
 
 struct Small {
   ChunkScalars cs;
   float Xf[8 * 128];      // inverse scratch: one 16 x 8 tile per prep warp
   float wsum[16];         // warm-up window search: per-warp partial sums
   int ws;                 // warm-up start token (context parallelism)
-  uint64_t full[2], prep_full[2], gdone, wdone, mma_done;
+  uint64_t full[2], prep_full[2], gdone, wdone, mma_done, dd_free;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -68,16 +72,19 @@ constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a block can opt into");
 
 // TMEM columns (fp32, 128 lanes)
-constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T, then W^T (prep)
-constexpr uint32_t kColDQ = 64;   // 64: S Q~^T, accumulates Delta^T P^T
-constexpr uint32_t kColDd = 128;  // 2 x 64: U^T - S W^T = Delta^T, by chunk parity
-constexpr uint32_t kColS = 256;   // 128: the fp32 state S (dv x dk), updated in place
+constexpr uint32_t kColGW = 0;      // 2 x 128 by chunk parity: [K;Q] K^T (64 cols); then
+                                    //   W (M=64 layout: row m in lane m%16 + 32(m/16), 128 cols)
+constexpr uint32_t kColPair = 256;  // 128: [D_Q | Delta^T]
+                                    //   D_Q = S Q~^T + Delta^T P^T,  Delta^T = U^T - S W^T
+constexpr uint32_t kColDd = kColPair + 64;
+constexpr uint32_t kColS = 384;     // 128: the fp32 state S (dv x dk), updated in place
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kId64 = idesc_bf16(128, 64, false, false);    // A, B K-major
-constexpr uint32_t kId64km = idesc_bf16(128, 64, false, true);   // B MN-major
-constexpr uint32_t kId64mk = idesc_bf16(128, 64, true, false);   // A MN-major
-constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);
+constexpr uint32_t kId64 = idesc_bf16(128, 64, false, false);     // A, B K-major
+constexpr uint32_t kId128 = idesc_bf16(128, 128, false, false);   // A, B K-major
+constexpr uint32_t kIdU = idesc_bf16(128, 64, true, false);       // A MN-major
+constexpr uint32_t kIdW = idesc_bf16(64, 128, false, true);       // B MN-major, M = 64
+constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);     // B MN-major
 
 
 }  // namespace
@@ -108,6 +115,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     mbar_init(&ss->gdone, 1);
     mbar_init(&ss->wdone, 1);
+    mbar_init(&ss->dd_free, 1);
     mbar_init(&ss->mma_done, 1);
     ss->abort_flag = 0;
     ss->ws = it.s;
@@ -162,13 +170,13 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int row = it.b * p.T + ws + c * kChunk;
     uint8_t* st = sm + s * kStageBytes;
     mbar_arrive_expect_tx(&ss->full[s], stage_bytes);
-    tma_load_3d(st + 0, &tm_k, &ss->full[s], 0, it.hq, row);
-    tma_load_3d(st + 8192, &tm_q, &ss->full[s], 0, it.hq, row);
-    tma_load_3d(st + 16384, &tm_k, &ss->full[s], 64, it.hq, row);
-    tma_load_3d(st + 24576, &tm_q, &ss->full[s], 64, it.hq, row);
+    tma_load_3d(st, &tm_k, &ss->full[s], 0, it.hq, row);
+    tma_load_3d(st + kOffQ, &tm_q, &ss->full[s], 0, it.hq, row);
+    tma_load_3d(st + kHalf, &tm_k, &ss->full[s], 64, it.hq, row);
+    tma_load_3d(st + kHalf + kOffQ, &tm_q, &ss->full[s], 64, it.hq, row);
     if (!it.zero_v) {
       tma_load_3d(st + kOffV, &tm_v, &ss->full[s], 0, it.j, row);
-      tma_load_3d(st + kOffV + 8192, &tm_v, &ss->full[s], 64, it.j, row);
+      tma_load_3d(st + kHalf + kOffV, &tm_v, &ss->full[s], 64, it.j, row);
     }
   };
 
@@ -177,9 +185,10 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ prep (8 warps)
     const int pt = threadIdx.x;            // 0..255
-    PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), ss->Xf, &ss->cs, tmem, kColG, pt, warp, lane, kBarPrep};
+    PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), ss->Xf, &ss->cs, tmem, kColGW, pt, warp, lane, kBarPrep};
     bool ok = true;
-    // g, beta of a chunk (0 past the sequence end); loaded one chunk ahead
+    const int qd = warp & 3, hc = warp >> 2;
+    // g, beta of a chunk (0 past the sequence end), loaded one chunk ahead
     auto load_gb = [&](int c, float& gv, float& bv) {
       const int t0 = ws + c * kChunk;
       gv = 0.f;
@@ -190,89 +199,124 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bv = __bfloat162float(beta[gi]);
       }
     };
-    float gv_next = 0.f, bv_next = 0.f;
-    if (nchunks > 0) load_gb(0, gv_next, bv_next);
-    for (int c = 0; c < nchunks; ++c) {
+    // Start of chunk c: wait for its tiles, clear rows past the sequence end, issue
+    // G = [K;Q] K^T into G/W buffer c % 2 and form the chunk's decay scalars.
+    auto chunk_start = [&](int c, float gv, float bv) {
       const int s = c & 1;
-      const int t0 = ws + c * kChunk;
-      const int nv = min(kChunk, it.e - t0);
+      const int nv = min(kChunk, it.e - (ws + c * kChunk));
       uint8_t* st = sm + s * kStageBytes;
       const uint32_t st_addr = sbase + s * kStageBytes;
-      const float gv = gv_next, bv = bv_next;
-      if (c + 1 < nchunks) load_gb(c + 1, gv_next, bv_next);
       ok = ok && mbar_wait(&ss->full[s], (c >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       // full chunk: the Gram product can start at once (a partial one waits for its zeroed rows)
-      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColG, st_addr, &ss->gdone);
+      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
       prep_store_gb(pc, s, gv, bv);
       if (nv < kChunk) {
         // rows past the sequence end hold the next sequence's tokens: clear them
         const int tiles = it.zero_v ? 4 : 6;
         for (int idx = pt; idx < (kChunk - nv) * tiles * 8; idx += kNumPrep) {
           const int r = nv + idx / (tiles * 8), rem = idx % (tiles * 8), tile = rem / 8, ch = rem % 8;
-          const uint32_t off = (tile < 4 ? tile * 8192u : kOffV + (tile - 4) * 8192u) + r * 128u + ch * 16u;
-          *reinterpret_cast<uint4*>(st + off) = make_uint4(0, 0, 0, 0);
+          // tiles 0..3: K0 Q0 K1 Q1; 4, 5: V0 V1
+          const uint32_t toff = tile < 4 ? (tile >> 1) * kHalf + (tile & 1) * kOffQ : (tile - 4) * kHalf + kOffV;
+          *reinterpret_cast<uint4*>(st + toff + r * 128u + ch * 16u) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
       named_bar_sync(kBarPrep, kNumPrep);
-      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColG, st_addr, &ss->gdone);
+      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
       prep_scan(pc, s);
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays(pc, s, nv);
+    };
+    if (nchunks > 0) {
+      float gv0, bv0;
+      load_gb(0, gv0, bv0);
+      chunk_start(0, gv0, bv0);
+    }
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      uint8_t* st = sm + s * kStageBytes;
+      const uint32_t st_addr = sbase + s * kStageBytes;
+      const uint32_t gw_col = kColGW + 128u * s;
+      float gv1 = 0.f, bv1 = 0.f;
+      if (c + 1 < nchunks) load_gb(c + 1, gv1, bv1);
       ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      prep_masks(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
+      pc.colG = gw_col;
+      prep_masks<true>(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
       // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- diag(exp(gam)) Q
       // in place (the Gram product has consumed Q); then one column strip of A per warp
-      if (warp < 4) prep_diag_inverse(pc);
-      else scale_rows_tile_part(st + 8192, 16384, ss->cs.eg[s], 1.f, pt - 128, 128);
+      if (warp < 4) prep_diag_inverse_h(pc);
+      else scale_rows_tile_part(st + kOffQ, kHalf, ss->cs.eg[s], 1.f, pt - 128, 128);
       named_bar_sync(kBarPrep, kNumPrep);
       {
         float x[4][4];
-        prep_solve_strip(pc, x);
+        prep_solve_strip_h(pc, x);
         prep_store_strip(pc, s, x, sbase + kOffA2, sbase + kOffB2);
       }
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
-      // U^T = V^T A2^T (A = V tile read MN-major, dv halves 8KB apart) into this chunk's
-      // Delta accumulator; W^T = K^T B2^T (A = K tile read MN-major) over G
+      // the Delta accumulator is free once the chain has read chunk c - 1's
+      if (c > 0) {
+        ok = ok && mbar_wait(&ss->dd_free, (c - 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      // U^T = V^T A2^T (A = the V tile read MN-major) into the Delta accumulator;
+      // W = B2 K (B = the K tile read MN-major, M = 64) over this chunk's G
       if (pt == 0 && ok) {
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           if (!it.zero_v)
-            umma_f16(tmem + kColDd + 64u * s, sdesc_sw128(st_addr + kOffV + ks * 2048, 8192, 1024),
-                     sdesc_sw128(sbase + kOffA2 + ks * 32, 16, 1024), kId64mk, ks > 0);
-          umma_f16(tmem + kColG, sdesc_sw128(st_addr + ks * 2048, 16384, 1024),
-                   sdesc_sw128(sbase + kOffB2 + ks * 32, 16, 1024), kId64mk, ks > 0);
+            umma_f16(tmem + kColDd, sdesc_sw128(st_addr + kOffV + ks * 2048, kHalf, 1024),
+                     sdesc_sw128(sbase + kOffA2 + ks * 32, 16, 1024), kIdU, ks > 0);
+          umma_f16(tmem + gw_col, sdesc_sw128(sbase + kOffB2 + ks * 32, 16, 1024),
+                   sdesc_sw128(st_addr + ks * 2048, kHalf, 1024), kIdW, ks > 0);
         }
         umma_commit(&ss->wdone);
+      }
+      if (it.zero_v && ok) {                    // V = 0: the Delta accumulator starts from zero
+        tc_fence_after();
+        float z[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) z[u] = 0.f;
+        tmem_st32_sync(tmem + ((uint32_t)(32 * qd) << 16) + kColDd + 32 * hc, z);
       }
       ok = ok && mbar_wait(&ss->wdone, c & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      // -W^T -> bf16 rows [dk][token] over the V tile (consumed by the U^T product)
+      // -W -> bf16 token rows over the V tile (consumed by the U^T product): warp (qd, hc)
+      // holds tokens 16 qd + lane (lanes 0..15) at features 64 hc .. 64 hc + 63
       {
-        const int qd = warp & 3, hc = warp >> 2;
-        const int r = 32 * qd + lane;
-        float v[32];
-        if (ok) tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + kColG + 32 * hc, v);
-        else {
+        float v[32], v2[32];
+        if (ok) {
+          tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + gw_col + 64 * hc, v);
+          tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + gw_col + 64 * hc + 32, v2);
+        } else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] = 0.f;
+          for (int u = 0; u < 32; ++u) v[u] = v2[u] = 0.f;
         }
+        if (lane < 16) {
+          const int jr = 16 * qd + lane;
+          const uint32_t wb = st_addr + hc * kHalf + kOffV;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          st_shared_v4(st_addr + kOffV + sw128(r, 4 * hc + c4), pack_bf16(-v[8 * c4], -v[8 * c4 + 1]),
-                       pack_bf16(-v[8 * c4 + 2], -v[8 * c4 + 3]), pack_bf16(-v[8 * c4 + 4], -v[8 * c4 + 5]),
-                       pack_bf16(-v[8 * c4 + 6], -v[8 * c4 + 7]));
+          for (int c4 = 0; c4 < 4; ++c4) {
+            st_shared_v4(wb + sw128(jr, c4), pack_bf16(-v[8 * c4], -v[8 * c4 + 1]),
+                         pack_bf16(-v[8 * c4 + 2], -v[8 * c4 + 3]), pack_bf16(-v[8 * c4 + 4], -v[8 * c4 + 5]),
+                         pack_bf16(-v[8 * c4 + 6], -v[8 * c4 + 7]));
+            st_shared_v4(wb + sw128(jr, 4 + c4), pack_bf16(-v2[8 * c4], -v2[8 * c4 + 1]),
+                         pack_bf16(-v2[8 * c4 + 2], -v2[8 * c4 + 3]), pack_bf16(-v2[8 * c4 + 4], -v2[8 * c4 + 5]),
+                         pack_bf16(-v2[8 * c4 + 6], -v2[8 * c4 + 7]));
+          }
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);
+      // the next chunk's start (its Gram product goes to the other G/W buffer)
+      if (c + 1 < nchunks) chunk_start(c + 1, gv1, bv1);
     }
   } else {
     // ------------------------------------------------------------ epilogue: the state chain
@@ -306,23 +350,25 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tmem_st32_sync(s_addr + h2 * 32, v);
       write_sb(v, h2);
     }
+    {
+      float z[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) z[u] = 0.f;
+      tmem_st32_sync(tmem + lane_base + kColPair + hh * 32, z);          // D_Q starts at 0
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar_sync(kBarEpi, kNumEpi);
     uint32_t mph = 0;
-    // (a) Delta^T = U^T + S_bf16 (-W^T) (onto the prep's U^T; from zero when V is zero)
-    //     and D_Q = S_bf16 Q~^T
+    // (a) [D_Q | Delta^T] += S_bf16 [Q~ ; -W]^T: B = rows Q~ then -W, adjacent in each half of
+    //     the stage. D_Q was zeroed after its last read; Delta^T holds the prep's U^T (or 0).
     auto issue_a = [&](int c) {
       tc_fence_after();
-      const uint32_t a0 = sbase + kOffSb, st_addr = sbase + (c & 1) * kStageBytes;
-      const uint32_t dd = tmem + kColDd + 64u * (c & 1);
+      const uint32_t a0 = sbase + kOffSb, b0 = sbase + (c & 1) * kStageBytes + kOffQ;
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
-        const uint64_t sa = sdesc_sw128(a0 + off, 16, 1024);
-        umma_f16(dd, sa, sdesc_sw128(st_addr + kOffV + ks * 2048, 8192, 1024), kId64km, !it.zero_v || ks > 0);
-        umma_f16(tmem + kColDQ, sa, sdesc_sw128(st_addr + 8192 + off, 16, 1024), kId64, ks > 0);
-      }
+      for (int ks = 0; ks < 8; ++ks)
+        umma_f16(tmem + kColPair, sdesc_sw128(a0 + (ks >> 2) * 16384u + (ks & 3) * 32u, 16, 1024),
+                 sdesc_sw128(b0 + (ks >> 2) * kHalf + (ks & 3) * 32u, 16, 1024), kId128, 1);
       umma_commit(&ss->mma_done);
     };
     // S <- exp(gam_n) S in TMEM (before the chunk's update accumulates onto it)
@@ -370,7 +416,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // (b) Delta^T and Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
       {
         float dd[32];
-        if (ok) tmem_ld32_sync(tmem + lane_base + kColDd + 64u * s + hh * 32, dd);
+        if (ok) tmem_ld32_sync(tmem + lane_base + kColDd + hh * 32, dd);
         else {
 #pragma unroll
           for (int u = 0; u < 32; ++u) dd[u] = 0.f;
@@ -394,16 +440,17 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       named_bar_sync(kBarEpi, kNumEpi);
       // (c) D_Q += Delta^T P^T;  S += Delta~^T K   (S was pre-scaled by exp(gam_n))
       if (et == 0 && ok) {
+        mbar_arrive(&ss->dd_free);                // every Delta^T read is done: the prep may refill it
         tc_fence_after();
         const uint32_t ya = sbase + kOffYt, pb = sbase + kOffP + s * 8192u;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          umma_f16(tmem + kColDQ, sdesc_sw128(ya + ks * 32, 16, 1024), sdesc_sw128(pb + ks * 32, 16, 1024), kId64,
-                   1);
+          umma_f16(tmem + kColPair, sdesc_sw128(ya + ks * 32, 16, 1024),
+                   sdesc_sw128(pb + ks * 32, 16, 1024), kId64, 1);
         const uint32_t da = sbase + kOffDt, kb = sbase + s * kStageBytes;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          umma_f16(tmem + kColS, sdesc_sw128(da + ks * 32, 16, 1024), sdesc_sw128(kb + ks * 2048, 16384, 1024),
+          umma_f16(tmem + kColS, sdesc_sw128(da + ks * 32, 16, 1024), sdesc_sw128(kb + ks * 2048, kHalf, 1024),
                    kIdE2, 1);
         umma_commit(&ss->mma_done);
       }
@@ -422,8 +469,13 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           }
           write_sb(v, h2);
         }
-        if (ok) tmem_ld32_sync(tmem + lane_base + kColDQ + hh * 32, oo);
-        else {
+        if (ok) {
+          tmem_ld32_sync(tmem + lane_base + kColPair + hh * 32, oo);
+          float z[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) z[u] = 0.f;
+          tmem_st32_sync(tmem + lane_base + kColPair + hh * 32, z);   // D_Q of chunk c + 1 starts at 0
+        } else {
 #pragma unroll
           for (int u = 0; u < 32; ++u) oo[u] = 0.f;
         }
