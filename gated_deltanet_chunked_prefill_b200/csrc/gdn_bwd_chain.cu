@@ -194,10 +194,17 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ok = ok && mbar_wait(&ss->gdone, k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      prep_masks(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P
-      scale_rows_tile(pc, st + 8192, 16384, ss->cs.eg[s], p.scale);  // Q <- scale diag(exp(gam)) Q
-      prep_inverse(pc);
-      prep_write_a(pc, s, sbase + kOffA2 + s * 8192u, 0);
+      prep_masks<true>(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P; L as fp16
+      // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- scale diag(exp(gam)) Q;
+      // then one column strip of A per warp -> A diag(beta)
+      if (warp < 4) prep_diag_inverse_h(pc);
+      else scale_rows_tile_part(st + 8192, 16384, ss->cs.eg[s], p.scale, pt - 128, 128);
+      named_bar_sync(kBarPrep, kNumPrep);
+      {
+        float x[4][4];
+        prep_solve_strip_h(pc, x);
+        prep_store_strip(pc, s, x, sbase + kOffA2 + s * 8192u, 0);
+      }
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);

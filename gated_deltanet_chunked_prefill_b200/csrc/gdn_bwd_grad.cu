@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_ds,
-                    const FwdParams p, const BwdOut out) {
+                    const FwdParams p, const BwdOut out, const int num_items) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw;
   Small* ss = reinterpret_cast<Small*>(sm + kOffSmall);
@@ -116,34 +116,6 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (tid == 0) record_error(p.status, kDevTimeout);
     return;
   }
-  // ---- which chunk: item = chunk_index * Hv + j
-  const int j = blockIdx.x % p.Hv;
-  const int gc = blockIdx.x / p.Hv;
-  int n, c;
-  if (p.chunk_off) {                          // packed sequences: last n with chunk_off[n] <= gc
-    int lo = 0, hi = p.N - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (p.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
-    }
-    n = lo;
-    c = gc - p.chunk_off[n];
-  } else {
-    const int nch = (p.T + kChunk - 1) / kChunk;
-    n = gc / nch;
-    c = gc % nch;
-  }
-  if (n >= p.N) return;
-  int b, s0, e0;
-  if (!seq_span(p, n, b, s0, e0)) return;
-  const int t0 = s0 + c * kChunk;
-  if (c < 0 || t0 >= e0) return;
-  const int nv = min(kChunk, e0 - t0);
-  const int hq = j / (p.Hv / p.Hqk);
-  const size_t slot = chunk_slot(p, n, c) * p.Hv + j;
-  const int row = b * p.T + t0;
-  const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
-
   if (tid == 0) {
     mbar_init(&ss->tma_bar, 1);
     mbar_init(&ss->mma_bar, 1);
@@ -162,6 +134,51 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint32_t sbase = smem_u32(sm);
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
   const int r = 32 * qd + lane;               // TMEM lane of this thread (M = 128 layouts)
+  const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
+  // item = chunk_index * Hv + j -> (sequence n, chunk c of it, v-head j) and its token span
+  struct Pos {
+    int n, c, j, b, s0, e0;
+  };
+  auto decode = [&](int item, Pos& q) -> bool {
+    q.j = item % p.Hv;
+    const int gc = item / p.Hv;
+    if (p.chunk_off) {                        // packed sequences: last n with chunk_off[n] <= gc
+      int lo = 0, hi = p.N - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
+      }
+      q.n = lo;
+      q.c = gc - p.chunk_off[q.n];
+    } else {
+      const int nch = (p.T + kChunk - 1) / kChunk;
+      q.n = gc / nch;
+      q.c = gc % nch;
+    }
+    if (q.n >= p.N || q.c < 0) return false;
+    if (!seq_span(p, q.n, q.b, q.s0, q.e0)) return false;
+    return q.s0 + q.c * kChunk < q.e0;
+  };
+  // tiles of an item: K, Q (q/k head), V, dO (v-head) token rows; S, dS' state rows
+  auto item_rows = [&](const Pos& q, int& row, int& hq, int& srow) {
+    row = q.b * p.T + q.s0 + q.c * kChunk;
+    hq = q.j / (p.Hv / p.Hqk);
+    srow = (int)((chunk_slot(p, q.n, q.c) * p.Hv + q.j) * 128);
+  };
+  uint32_t mph = 0, tph = 0;
+  // Persistent: this CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ... (setup and
+  // TMEM allocation once per CTA).
+  for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
+  Pos pos;
+  if (!decode(item, pos)) continue;           // uniform over the CTA
+  if (__syncthreads_or(*abort_flag)) break;
+  const int j = pos.j, n = pos.n, c = pos.c, b = pos.b, e0 = pos.e0;
+  int row, hq, srow;
+  item_rows(pos, row, hq, srow);
+  const int t0 = pos.s0 + c * kChunk;
+  const int nv = min(kChunk, e0 - t0);
+  (void)n;
+  (void)b;
   if (tid == 0) {
     mbar_arrive_expect_tx(&ss->tma_bar, 128u * 1024u);
     tma_load_3d(sm + kOffKQ + 0, &tm_k, &ss->tma_bar, 0, hq, row);
@@ -172,7 +189,6 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_load_3d(sm + kOffVDO + 8192, &tm_do, &ss->tma_bar, 0, j, row);
     tma_load_3d(sm + kOffVDO + 16384, &tm_v, &ss->tma_bar, 64, j, row);
     tma_load_3d(sm + kOffVDO + 24576, &tm_do, &ss->tma_bar, 64, j, row);
-    const int srow = (int)(slot * 128);
     tma_load_3d(sm + kOffS, &tm_s, &ss->tma_bar, 0, 0, srow);
     tma_load_3d(sm + kOffS + 16384, &tm_s, &ss->tma_bar, 64, 0, srow);
     tma_load_3d(sm + kOffDS, &tm_ds, &ss->tma_bar, 0, 0, srow);
@@ -187,7 +203,8 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bv = __bfloat162float(beta[gi]);
   }
   prep_store_gb(pc, 0, gv, bv);
-  bool ok = mbar_wait(&ss->tma_bar, 0, abort_flag);
+  bool ok = mbar_wait(&ss->tma_bar, tph, abort_flag);
+  tph ^= 1;
   ok = __syncthreads_and(ok);
   if (nv < kChunk) {                          // rows past the sequence end: zero
     for (int idx = tid; idx < (kChunk - nv) * 64; idx += kThreads) {
@@ -197,7 +214,6 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
   fence_proxy_async_smem();
   __syncthreads();
-  uint32_t mph = 0;
   auto commit_wait = [&]() {
     if (tid == 0 && ok) umma_commit(&ss->mma_bar);
     ok = ok && mbar_wait(&ss->mma_bar, mph, abort_flag);
@@ -215,7 +231,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   ok = __syncthreads_and(ok);
   mph ^= 1;
   tc_fence_after();
-  prep_masks(pc, 0, sbase + kOffP, p.scale, ok);
+  prep_masks<true>(pc, 0, sbase + kOffP, p.scale, ok);
   fence_proxy_async_smem();                   // scale * P is an operand of the next products
   __syncthreads();
   if (tid == 0 && ok) {
@@ -235,8 +251,16 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       umma_f16(tmem + kColDb, mdesc(sbase + kOffVDO + 8192 + ks * 2048, 16384), mdesc(sbase + kOffP + ks * 2048, 8192),
                idmm, ks > 0);
   }
-  prep_inverse(pc);
-  prep_write_a(pc, 0, sbase + kOffA2, sbase + kOffA);
+  // A = (I + L)^-1: diagonal blocks (warps 0-3), then one column strip per warp; the
+  // fp32 A rows replace the fp16 L once every strip is solved
+  if (warp < 4) prep_diag_inverse_h(pc);
+  __syncthreads();
+  {
+    float xs[4][4];
+    prep_solve_strip_h(pc, xs);
+    __syncthreads();
+    prep_store_strip_a(pc, 0, xs, sbase + kOffA2, sbase + kOffA);
+  }
   fence_proxy_async_smem();
   commit_wait();
   const float* eg = ss->cs.eg[0];
@@ -696,13 +720,23 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (2 * lane + 1 < nv) db[gi + p.Hv] = __float2bfloat16_rn(b1);
     }
   }
+  // the next item's loads overwrite every tile and TMEM column this one used
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  }
+  if (tid == 0 && *abort_flag) {
+    // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
+    volatile int never = 0;
+    mbar_wait(&ss->tma_bar, tph ^ 1, &never);
+    record_error(p.status, kDevTimeout);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (tid == 0 && *abort_flag) record_error(p.status, kDevTimeout);
 }
 
 // fp32 per-v-head partials of dq / dk -> the sum over the v-heads of each q/k head (fixed order)
@@ -738,9 +772,18 @@ cudaError_t launch_bwd_grad(const FwdParams& p, const BwdOut& out, long long tot
   cudaError_t err = cudaFuncSetAttribute(gdn_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
   if (err != cudaSuccess) return err;
+  // persistent: one CTA per SM (the shared-memory footprint allows one), items strided over CTAs
+  const long long items = total_chunks * p.Hv;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  *what = "device query";
+  err = cudaGetDevice(&dev);
+  if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (err != cudaSuccess) return err;
+  const unsigned grid = (unsigned)std::min<long long>(items, std::max(sms, 1));
   *what = "backward gradient launch";
   trace_pre(kKernBwdTc, st);
-  gdn_bwd_grad_kernel<<<(unsigned)(total_chunks * p.Hv), kThreads, kSmemBytes, st>>>(mq, mk, mv, mdo, ms, mds, p, out);
+  gdn_bwd_grad_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, mdo, ms, mds, p, out, (int)items);
   err = cudaGetLastError();
   trace_post(st);
   if (err != cudaSuccess || !out.qk_partial) return err;

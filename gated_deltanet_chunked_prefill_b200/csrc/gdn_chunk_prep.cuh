@@ -487,8 +487,8 @@ __device__ __forceinline__ void prep_solve_strip_h(const PrepCtx& c, float (&x)[
   }
 }
 
-// A2 = A diag(beta) and B2 = A diag(beta exp(gam)) -> bf16 (128B-swizzled rows at a2_addr,
-// b2_addr) straight from prep_solve_strip's fragments.
+// A2 = A diag(beta) and (b2_addr != 0) B2 = A diag(beta exp(gam)) -> bf16 (128B-swizzled
+// rows at a2_addr, b2_addr) straight from a strip solve's fragments.
 __device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const float (&x)[4][4], uint32_t a2_addr,
                                                  uint32_t b2_addr) {
   const int w = c.pw, gid = c.lane >> 2, tig = c.lane & 3;
@@ -503,7 +503,8 @@ __device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const 
       const uint32_t off = tc::sw128(i, w) + 4 * tig;
       const float v0 = x[R][2 * h], v1 = x[R][2 * h + 1];
       asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2_addr + off), "r"(tc::pack_bf16(v0 * b0, v1 * b1)) : "memory");
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(b2_addr + off), "r"(tc::pack_bf16(v0 * e0, v1 * e1)) : "memory");
+      if (b2_addr)
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(b2_addr + off), "r"(tc::pack_bf16(v0 * e0, v1 * e1)) : "memory");
     }
   }
 }
@@ -625,6 +626,28 @@ __device__ __forceinline__ void prep_write_a(const PrepCtx& c, int s, uint32_t a
     for (int u = 0; u < 8; ++u) w[u] = tc::pack_bf16(a[2 * u], a[2 * u + 1]);
     st_shared_v4(a_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
     st_shared_v4(a_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  }
+}
+
+// A2 = A diag(beta) and A -> bf16 (128B-swizzled rows at a2_addr, a_addr), and A -> fp32
+// rows of stride kLd in the scratch, from prep_solve_strip_h's fragments. The caller
+// separates this from the solve with a group barrier (the fp32 rows overwrite the fp16 L).
+__device__ __forceinline__ void prep_store_strip_a(const PrepCtx& c, int s, const float (&x)[4][4], uint32_t a2_addr,
+                                                   uint32_t a_addr) {
+  const int w = c.pw, gid = c.lane >> 2, tig = c.lane & 3;
+  const int j = 8 * w + 2 * tig;
+  const float b0 = c.cs->bet[s][j], b1 = c.cs->bet[s][j + 1];
+#pragma unroll
+  for (int R = 0; R < 4; ++R) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 16 * R + gid + 8 * h;
+      const uint32_t off = tc::sw128(i, w) + 4 * tig;
+      const float v0 = x[R][2 * h], v1 = x[R][2 * h + 1];
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2_addr + off), "r"(tc::pack_bf16(v0 * b0, v1 * b1)) : "memory");
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a_addr + off), "r"(tc::pack_bf16(v0, v1)) : "memory");
+      *reinterpret_cast<float2*>(c.Lf + i * kLd + j) = make_float2(v0, v1);
+    }
   }
 }
 
