@@ -14,7 +14,7 @@ from typing import Optional
 import torch
 
 __all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd", "fwd_workspace_size",
-           "bwd_workspace_size", "read_device_status", "Options", "LIB_PATH", "KernelTrace",
+           "bwd_workspace_size", "chunk_states", "read_device_status", "Options", "LIB_PATH", "KernelTrace",
            "launch_count"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
@@ -36,7 +36,7 @@ class GdnError(RuntimeError):
 class Options(ctypes.Structure):
     """Mirror of gdn_options."""
     _fields_ = [("cp_segment_chunks", ctypes.c_int), ("cp_exact", ctypes.c_int),
-                ("reserved", ctypes.c_int * 6)]
+                ("states", ctypes.c_void_p), ("reserved", ctypes.c_int * 4)]
 
 
 _lib = None
@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_fwd_workspace_size.restype = sz
         L.gdn_chunk_bwd_workspace_size.argtypes = dims + [vp]
         L.gdn_chunk_bwd_workspace_size.restype = sz
+        L.gdn_chunk_states_size.argtypes = dims
+        L.gdn_chunk_states_size.restype = sz
         L.gdn_chunk_fwd.argtypes = [i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp, vp, sz,
                                                     vp, vp]
         L.gdn_chunk_fwd.restype = i
@@ -97,10 +99,14 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported I/O dtype {t.dtype}")
 
 
-def _opts(cp_segment_chunks: int, cp_exact: bool = False):
+def _opts(cp_segment_chunks: int, cp_exact: bool = False, states=None):
     o = Options()
     o.cp_segment_chunks = int(cp_segment_chunks)
     o.cp_exact = int(bool(cp_exact))
+    if states is not None:
+        if states.dtype != torch.bfloat16 or not states.is_cuda or not states.is_contiguous():
+            raise ValueError("states: a contiguous bf16 CUDA tensor from chunk_states()")
+        o.states = states.data_ptr()
     return o
 
 
@@ -121,9 +127,17 @@ def fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=F
     return int(lib().gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
 
 
-def bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False) -> int:
-    o = _opts(cp_segment_chunks, cp_exact)
+def bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False, states=None) -> int:
+    o = _opts(cp_segment_chunks, cp_exact, states)
     return int(lib().gdn_chunk_bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
+
+
+def chunk_states(q, v, cu_seqlens=None):
+    """A chunk-start-state cache (gdn_options.states) for these inputs: pass it as
+    `states=` to gdn_chunk_fwd, then to gdn_chunk_bwd, which then skips its forward pass."""
+    B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
+    nbytes = int(lib().gdn_chunk_states_size(B, T, Hqk, Hv, dk, dv, N))
+    return torch.empty(max(nbytes // 2, 1), dtype=torch.bfloat16, device=q.device)
 
 
 def _check(t, name, dtype=None):
@@ -147,8 +161,9 @@ def _workspace(nbytes, workspace, device):
 
 def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
                   output_final_state=True, cp_segment_chunks=0, cp_exact=False, workspace=None,
-                  o=None, hT=None, stream=None):
-    """Forward through the C ABI. Returns (o, hT or None)."""
+                  o=None, hT=None, stream=None, states=None):
+    """Forward through the C ABI. Returns (o, hT or None). With `states` (from
+    chunk_states()) it also writes every chunk's start state for a later backward."""
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
         _check(t, n, io)
@@ -163,7 +178,7 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
         hT = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
     ws_bytes = fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact)
     ws = _workspace(ws_bytes, workspace, q.device)
-    opt = _opts(cp_segment_chunks, cp_exact)
+    opt = _opts(cp_segment_chunks, cp_exact, states)
     st = lib().gdn_chunk_fwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                              _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(o),
                              _ptr(hT), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream(stream))
@@ -197,8 +212,10 @@ def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None
 
 
 def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlens=None,
-                  cp_segment_chunks=0, cp_exact=False, workspace=None, want_dh0=True, stream=None):
-    """Backward through the C ABI. Returns dict dq, dk, dv, dg, dbeta, dh0."""
+                  cp_segment_chunks=0, cp_exact=False, workspace=None, want_dh0=True, stream=None,
+                  states=None):
+    """Backward through the C ABI. Returns dict dq, dk, dv, dg, dbeta, dh0. With `states`
+    written by the matching gdn_chunk_fwd call, the forward pass is not recomputed."""
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta"), (dO, "dO")):
         _check(t, n, io)
@@ -214,9 +231,9 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
     dg = torch.empty_like(g)
     db = torch.empty_like(beta)
     dh0 = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
-    ws_bytes = bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact)
+    ws_bytes = bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact, states)
     ws = _workspace(ws_bytes, workspace, q.device)
-    opt = _opts(cp_segment_chunks, cp_exact)
+    opt = _opts(cp_segment_chunks, cp_exact, states)
     st = lib().gdn_chunk_bwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                              _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(dO),
                              _ptr(dhT), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db),

@@ -89,11 +89,16 @@ struct FwdPlan {
   int seg_chunks = 0, max_segs = 0, max_pairs = 0;
   bool table = false, exact = false;
   size_t off_table = 0, off_count = 0, off_first = 0, off_state = 0, off_trans = 0, total = kStatusBytes;
+  size_t off_chunk_off = 0;     // packed sequences: per-sequence first chunk slot (state cache)
 };
 
 FwdPlan plan_forward(gdn_dtype dtype, const Shape& s, const gdn_options* opt) {
   FwdPlan f;
   if (!uses_tc(dtype, s) || s.T == 0) return f;
+  if (s.packed) {
+    f.off_chunk_off = f.total;
+    f.total = align256(f.total + (size_t)(s.N + 1) * sizeof(int));
+  }
   const int mode = opt ? opt->cp_segment_chunks : 0;
   if (mode < 0) return f;
   const int nch = (s.T + kChunk - 1) / kChunk;
@@ -109,7 +114,7 @@ FwdPlan plan_forward(gdn_dtype dtype, const Shape& s, const gdn_options* opt) {
     f.max_segs = (nch + seg - 1) / seg;
     f.max_pairs = s.N * f.max_segs;
   }
-  size_t off = kStatusBytes;
+  size_t off = f.total;
   if (f.table) {
     f.off_table = off; off = align256(off + (size_t)f.max_pairs * sizeof(int2));
     f.off_count = off; off = align256(off + sizeof(int));
@@ -141,9 +146,9 @@ BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
   b.total_chunks = s.packed ? (long long)nch + s.N : (long long)s.N * nch;
   b.grouped = s.Hv != s.Hqk;
   size_t off = b.chain.total;
-  if (s.packed) { b.off_chunk_off = off; off = align256(off + (size_t)(s.N + 1) * sizeof(int)); }
+  if (s.packed) b.off_chunk_off = b.chain.off_chunk_off;
   const size_t st = (size_t)b.total_chunks * s.Hv * s.dk * s.dv * 2;
-  b.off_states = off; off = align256(off + st);
+  if (!(opt && opt->states)) { b.off_states = off; off = align256(off + st); }
   b.off_dstates = off; off = align256(off + st);
   if (b.grouped) {
     const size_t part = (size_t)s.B * s.T * s.Hv * s.dk * sizeof(float);
@@ -260,7 +265,9 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
       if (r != 0) return GDN_ERR_INVALID_ARG;
   }
   if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, o, hT};
+  void* save_states = opt ? opt->states : nullptr;
+  if (save_states && !uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, o, hT, save_states};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
   if (!workspace || !aligned16(workspace) ||
@@ -284,8 +291,20 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
     plan.kind = kPlanUnits;
     plan.roles = 1;
     const char* what = "";
+    // the launch that produces o also writes the chunk start states, when asked
+    FwdParams pf = p;
+    pf.states = static_cast<__nv_bfloat16*>(save_states);
+    int* chunk_off = nullptr;
+    if (save_states && s.packed) {           // packed: per-sequence first slot, from cu_seqlens
+      chunk_off = reinterpret_cast<int*>(ws + f.off_chunk_off);
+      pf.chunk_off = chunk_off;
+      if (!f.table) {
+        err = launch_cp_plan(p, 1, 0, nullptr, nullptr, nullptr, chunk_off, stream);
+        if (err != cudaSuccess) return cuda_fail("chunk offsets", err);
+      }
+    }
     if (f.kind == kPlanUnits) {
-      err = launch_fwd_tc(p, plan, s.N * s.Hv, stream, &what);
+      err = launch_fwd_tc(pf, plan, s.N * s.Hv, stream, &what);
       if (err != cudaSuccess) return cuda_fail(what, err);
       return GDN_OK;
     }
@@ -297,12 +316,12 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
       plan.table_count = reinterpret_cast<int*>(ws + f.off_count);
       first = reinterpret_cast<int*>(ws + f.off_first);
       err = launch_cp_plan(p, f.seg_chunks, f.max_pairs, const_cast<int2*>(plan.table),
-                           const_cast<int*>(plan.table_count), first, nullptr, stream);
+                           const_cast<int*>(plan.table_count), first, chunk_off, stream);
       if (err != cudaSuccess) return cuda_fail("segment table", err);
     }
     if (!f.exact) {
       plan.kind = kPlanGate;
-      err = launch_fwd_tc(p, plan, f.max_pairs * s.Hv, stream, &what);
+      err = launch_fwd_tc(pf, plan, f.max_pairs * s.Hv, stream, &what);
       if (err != cudaSuccess) return cuda_fail(what, err);
       return GDN_OK;
     }
@@ -316,13 +335,22 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
     err = launch_cp_stitch(p, plan, first, stream);
     if (err != cudaSuccess) return cuda_fail("segment stitch", err);
     plan.kind = kPlanCpP3;
-    err = launch_fwd_tc(p, plan, f.max_pairs * s.Hv, stream, &what);
+    err = launch_fwd_tc(pf, plan, f.max_pairs * s.Hv, stream, &what);
     if (err != cudaSuccess) return cuda_fail(what, err);
   } else {
     err = launch_fwd_simt(p, dtype == GDN_BF16, stream);
     if (err != cudaSuccess) return cuda_fail("CUDA-core forward", err);
   }
   return GDN_OK;
+}
+
+size_t gdn_chunk_states_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs) {
+  Shape s;
+  const bool packed = num_seqs > 0 && B == 1;
+  if (check_shape(B, T, Hqk, Hv, dk, dv, packed ? num_seqs : 0, packed, s) != GDN_OK) return 0;
+  const long long nch = (s.T + kChunk - 1) / kChunk;
+  const long long slots = s.packed ? nch + s.N : (long long)s.N * nch;   // as the backward's slots
+  return (size_t)slots * s.Hv * s.dk * s.dv * 2;
 }
 
 size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs,
@@ -349,7 +377,8 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   }
   if (T > 0 && (!q || !k || !v || !g || !beta || !dO || !dq || !dk_out || !dv_out || !dg || !dbeta))
     return GDN_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, dO, dhT, dq, dk_out, dv_out, dg, dbeta, dh0};
+  const void* cached = opt ? opt->states : nullptr;
+  const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, dO, dhT, dq, dk_out, dv_out, dg, dbeta, dh0, cached};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
   if (!uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;   // backward: bf16, dk = dv = 128
@@ -364,7 +393,8 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   p.status = static_cast<int*>(workspace);
   p.B = s.B; p.T = s.T; p.Hqk = s.Hqk; p.Hv = s.Hv; p.dk = s.dk; p.dv = s.dv; p.N = s.N;
   p.scale = scale;
-  p.states = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_states);
+  p.states = cached ? static_cast<__nv_bfloat16*>(const_cast<void*>(cached))
+                    : reinterpret_cast<__nv_bfloat16*>(ws + bp.off_states);
   p.chunk_off = s.packed ? reinterpret_cast<int*>(ws + bp.off_chunk_off) : nullptr;
   __nv_bfloat16* dstates = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_dstates);
 
@@ -393,9 +423,11 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
       items = f.max_pairs * s.Hv;
     }
   }
-  // 1) forward recompute: the bf16 start state of every chunk
-  err = launch_fwd_tc(p, plan, items, stream, &what);
-  if (err != cudaSuccess) return cuda_fail(what, err);
+  // 1) forward recompute: the bf16 start state of every chunk (unless the caller cached them)
+  if (!cached) {
+    err = launch_fwd_tc(p, plan, items, stream, &what);
+    if (err != cudaSuccess) return cuda_fail(what, err);
+  }
   // 2) reverse chain: the state gradient at every chunk end, and dh0
   FwdParams pc = p;
   pc.v = dO;

@@ -85,9 +85,24 @@ typedef struct {
    *   h_end = M h_start + b, phase 2 chains the maps, phase 3 reruns each segment
    *   from its stitched start state. */
   int cp_exact;
+  /* Chunk start states cached between a forward and its backward (tensor-core path:
+   * bf16, dk = dv = 128), device memory of gdn_chunk_states_size() bytes, 16-byte
+   * aligned, owned by the caller. NULL (default): nothing is cached and the backward
+   * recomputes the states itself.
+   *   gdn_chunk_fwd writes, for every chunk c of every sequence n and v-head j, the
+   *     state at the chunk's first token in bf16, transposed: states[slot][j][r][d] =
+   *     h[d][r] (r < dv, d < dk), slot = n * ceil(T/64) + c for independent sequences,
+   *     or (sum over m < n of ceil(len_m / 64)) + c for packed ones.
+   *   gdn_chunk_bwd reads them instead of running its forward pass; they must come
+   *     from gdn_chunk_fwd on the same q, k, v, g, beta, h0 and cu_seqlens.
+   * Set on another path: GDN_ERR_UNSUPPORTED; not 16-byte aligned: GDN_ERR_INVALID_ARG. */
+  void* states;
   /* Reserved, must be 0. */
-  int reserved[6];
+  int reserved[4];
 } gdn_options;
+
+/* Bytes of the chunk-state cache (gdn_options.states) for these sizes. */
+size_t gdn_chunk_states_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs);
 
 /* Bytes of device workspace gdn_chunk_fwd needs for these sizes and options. */
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv,
@@ -122,7 +137,8 @@ size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int d
  *   dq, dk [B,T,Hqk,dk] (dtype; summed over the v-heads sharing a q/k head),
  *   dv [B,T,Hv,dv] (dtype), dg [B,T,Hv] fp32 (w.r.t. the raw per-token g),
  *   dbeta [B,T,Hv] (dtype), dh0 (nullable) [N,Hv,dk,dv] fp32.
- * The forward is recomputed inside the call (nothing is cached between calls).
+ * Unless opt->states holds the chunk start states of the matching forward call
+ * (see gdn_options.states), the forward pass is recomputed inside the call.
  */
 gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
                          const void* q, const void* k, const void* v,

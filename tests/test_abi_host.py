@@ -80,3 +80,27 @@ def test_python_binding_refuses_cpu_tensors():
     g = torch.zeros(1, 64, 1)
     with pytest.raises(ValueError):
         gdn.gdn_chunk_fwd(x, x, x, g, torch.zeros(1, 64, 1, dtype=torch.bfloat16))
+
+
+def test_options_struct_layout():
+    # int, int, pointer, int[4]: 32 bytes with the pointer at offset 8
+    assert ctypes.sizeof(gdn.Options) == 32
+    assert gdn.Options.states.offset == 8
+
+
+def test_chunk_states_size():
+    L = gdn.lib()
+    # independent sequences: N * ceil(T / 64) slots of Hv * dk * dv bf16
+    assert L.gdn_chunk_states_size(2, 8192, 16, 16, 128, 128, 0) == 2 * 128 * 16 * 128 * 128 * 2
+    assert L.gdn_chunk_states_size(3, 100, 2, 4, 128, 128, 0) == 3 * 2 * 4 * 128 * 128 * 2
+    # packed: ceil(T / 64) + N slots bound the chunks of any split of T tokens into N sequences
+    assert L.gdn_chunk_states_size(1, 65536, 16, 16, 128, 128, 24) == (1024 + 24) * 16 * 128 * 128 * 2
+    assert L.gdn_chunk_states_size(0, 64, 1, 1, 128, 128, 0) == 0
+
+
+def test_states_option_checks():
+    o = gdn.Options()
+    o.states = FAKE
+    assert _fwd(dtype=0, dk=64, dv=64, opt=o) == 2        # fp32 / CUDA-core path: unsupported
+    o.states = MISALIGNED
+    assert _fwd(opt=o) == 1

@@ -106,3 +106,55 @@ def test_bwd_full_size_sampled_units():
         assert_close(gr["dg"][b, s:e, j], ref["dg"][0, :, 0], "bf16", f"unit ({n},{j}) dg")
         assert_close(gr["dbeta"][b, s:e, j], ref["dbeta"][0, :, 0], "bf16", f"unit ({n},{j}) dbeta")
         assert_close(gr["dh0"][n, j], ref["dh0"][0, 0], "bf16", f"unit ({n},{j}) dh0")
+
+
+def _fwd_states(d, **kw):
+    states = gdn.chunk_states(d["q"], d["v"], d["cu_seqlens"])
+    gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"], d["cu_seqlens"],
+                      states=states, **kw)
+    return states
+
+
+def _bwd(d, **kw):
+    gr = gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["scale"], d["h0"],
+                           d["dhT"], d["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    return {k: (v.cpu() if v is not None else None) for k, v in gr.items()}
+
+
+@pytest.mark.parametrize("name,cp", [("ragged", 0), ("gqa", 0), ("varlen", 0), ("varlen", 2), ("long", 3)])
+def test_bwd_cached_states_match_recompute(name, cp):
+    """States written by the forward give the same gradients, bit for bit, as the backward's
+    own forward pass (same segmentation on both sides), and match the oracle."""
+    B, T, Hqk, Hv, h0, lengths = SMALL[name]
+    x = make_inputs(B, T, Hqk, Hv, 128, 128, "bf16", seed=zlib.crc32(name.encode()) % 1000 + 7, h0_std=h0,
+                    lengths=lengths, backward=True)
+    d = to_dev(x)
+    states = _fwd_states(d, cp_segment_chunks=cp)
+    cached = _bwd(d, cp_segment_chunks=cp, states=states)
+    recomputed = _bwd(d, cp_segment_chunks=cp)
+    ref = oracle_bwd(x)
+    for n in GRADS:
+        assert torch.equal(cached[n], recomputed[n]), n
+        assert_close(cached[n], ref[n], "bf16", f"{name} cached {n}")
+
+
+def test_bwd_cached_states_from_exact_stitch():
+    """Forward with the exact affine stitch writes its states from the final pass."""
+    x = make_inputs(1, 0, 2, 2, 128, 128, "bf16", seed=41, h0_std=0.1, backward=True, lengths=[700, 64, 333])
+    d = to_dev(x)
+    states = _fwd_states(d, cp_segment_chunks=2, cp_exact=True)
+    cached = _bwd(d, states=states)
+    ref = oracle_bwd(x)
+    for n in GRADS:
+        assert_close(cached[n], ref[n], "bf16", f"exact-stitch cached {n}")
+
+
+def test_bwd_cached_states_full_size():
+    x = config_inputs("bwd_bf16")
+    d = to_dev(x)
+    states = _fwd_states(d)
+    cached = _bwd(d, states=states)
+    recomputed = _bwd(d)
+    for n in GRADS:
+        assert torch.equal(cached[n], recomputed[n]), n
