@@ -152,23 +152,32 @@ class ClockSampler:
                 "samples": len(inside), "window": window}
 
 
-def traffic_record(kernel_name, workload):
-    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if its source is unchanged."""
+def traffic_record(kernel_name, workload, mode):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary of the same workload and
+    step, if its sources are unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
         recs = json.load(fh)
     for r in recs:
-        if r.get("kernel") == kernel_name and r.get("workload") == workload:
-            src = os.path.join(ROOT, r["source"])
-            if not os.path.exists(src):
-                return None
-            with open(src, "rb") as fh:
-                if hashlib.sha256(fh.read()).hexdigest()[:16] != r.get("source_sha256_16"):
-                    return None
+        if r.get("kernel") == kernel_name and r.get("workload") == workload and r.get("step") == mode:
+            if sources_sha(r["sources"]) != r.get("sources_sha256_16"):
+                return None                      # the kernel changed since the capture
             return float(r["bytes_per_launch"])
     return None
+
+
+def sources_sha(paths):
+    """First 16 hex digits of the SHA-256 of the concatenated files (None if one is missing)."""
+    h = hashlib.sha256()
+    for rel in paths:
+        path = os.path.join(ROOT, rel)
+        if not os.path.exists(path):
+            return None
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def max_over_ranks(x: float, dist=None, device="cpu") -> float:
@@ -361,7 +370,7 @@ def main():
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "peak_source": src,
-                "traffic": traffic_record(dom, args.workload),
+                "traffic": traffic_record(dom, args.workload, mode),
                 "alg_bytes_per_launch": dom_bytes, "avg_launch_ms": dom_ms}
     step_bytes = alg_bytes(w, fwd=True, bwd=mode == "fwdbwd")
     step_roofline = {"alg_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,

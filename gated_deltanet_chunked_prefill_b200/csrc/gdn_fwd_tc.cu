@@ -23,8 +23,7 @@
 //     (d) S -> bf16 for the next chunk's products;  O = scale * D_Q
 // i.e. Delta = U - W h with U = A diag(beta) V and W = A diag(beta e^gam) K,
 // O = scale[diag(e^gam) Q h + (QK^T*E*M) Delta], h' = e^gam_n h + (diag(e^(gam_n-gam)) K)^T Delta:
-// the WY/UT chunk form of the gated delta rule ("Gated Delta Networks" paper, section 3.3,
-// hardware-efficient chunkwise training; "FlashQLA resource", section 3: fused
+// the WY/UT chunkwise form of the gated delta rule ("FlashQLA resource", section 3: fused
 // warp-specialised kernels that overlap data movement, tensor-core and CUDA-core work).
 #include <cudaTypedefs.h>
 
