@@ -350,8 +350,18 @@ def main():
             gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
                               cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT, states=states)
     fwd_ms = sum(t for _, t in trf.launches) / 5
+    bwd_recompute_ms = None
     if mode == "fwdbwd":
         bwd_ms = sum(t for _, t in tr.launches) / 5 - fwd_ms
+        # the backward alone once more, recomputing the chunk states itself (no cache)
+        ws_r = torch.zeros(gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp),
+                           dtype=torch.uint8, device=dev)
+        with gdn.KernelTrace(capacity=64) as trb:
+            for _ in range(5):
+                gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["scale"], d["h0"],
+                                  d["dhT"], cp_segment_chunks=args.cp, workspace=ws_r)
+        bwd_recompute_ms = sum(t for _, t in trb.launches) / 5
+        del ws_r
 
     hbm, tc_peak, src = peaks()
     # per-launch algorithmic bytes, matched to the launches of one step in order
@@ -442,7 +452,7 @@ def main():
                       "bwd_states": "cached by the forward (bf16 chunk start states)" if mode == "fwdbwd" else None,
                       "cp_segment_chunks": args.cp},
            "tflops": fl / (ms_step / 1e3) / 1e12,
-           "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+           "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "bwd_recompute_ms": bwd_recompute_ms,
            "per_kernel_ms": {k: float(np.mean(v)) for k, v in per_kernel.items()},
            "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
            "gpu_launches": int(launches),
