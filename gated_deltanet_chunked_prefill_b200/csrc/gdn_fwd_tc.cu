@@ -63,7 +63,7 @@ struct Small {
   float Xf[8 * 128];      // inverse scratch: one 16 x 8 tile per prep warp
   float wsum[16];         // warm-up window search: per-warp partial sums
   int ws;                 // warm-up start token (context parallelism)
-  uint64_t full[2], prep_full[2], gdone, wdone, mma_done, dd_free;
+  uint64_t full_k[2], full_qv[2], prep_full[2], gdone, wdone, mma_done, dd_free;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -109,7 +109,8 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&ss->full[s], 1);
+      mbar_init(&ss->full_k[s], 1);
+      mbar_init(&ss->full_qv[s], 1);
       mbar_init(&ss->prep_full[s], 1);
     }
     mbar_init(&ss->gdone, 1);
@@ -161,21 +162,27 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   volatile int* abort_flag = &ss->abort_flag;
   const uint32_t sbase = smem_u32(sm);
 
-  // TMA loads of chunk c into stage c % 2 (issued by the epilogue's first thread: chunks
-  // 0 and 1 at the start, chunk c + 2 as soon as chunk c has released its stage).
-  const uint32_t stage_bytes = it.zero_v ? 32u * 1024u : kStageBytes;
-  auto load_chunk = [&](int c) {
+  // TMA loads of chunk c into stage c % 2, issued by the epilogue's first thread: chunks 0
+  // and 1 at the start; for chunk c + 2, the Q and V tiles as soon as chunk c's state product
+  // has read Q~ and -W, the K tiles once its update product has read K.
+  auto load_k = [&](int c) {
     const int s = c & 1;
     const int row = it.b * p.T + ws + c * kChunk;
     uint8_t* st = sm + s * kStageBytes;
-    mbar_arrive_expect_tx(&ss->full[s], stage_bytes);
-    tma_load_3d(st, &tm_k, &ss->full[s], 0, it.hq, row);
-    tma_load_3d(st + kOffQ, &tm_q, &ss->full[s], 0, it.hq, row);
-    tma_load_3d(st + kHalf, &tm_k, &ss->full[s], 64, it.hq, row);
-    tma_load_3d(st + kHalf + kOffQ, &tm_q, &ss->full[s], 64, it.hq, row);
+    mbar_arrive_expect_tx(&ss->full_k[s], 16u * 1024u);
+    tma_load_3d(st, &tm_k, &ss->full_k[s], 0, it.hq, row);
+    tma_load_3d(st + kHalf, &tm_k, &ss->full_k[s], 64, it.hq, row);
+  };
+  auto load_qv = [&](int c) {
+    const int s = c & 1;
+    const int row = it.b * p.T + ws + c * kChunk;
+    uint8_t* st = sm + s * kStageBytes;
+    mbar_arrive_expect_tx(&ss->full_qv[s], it.zero_v ? 16u * 1024u : 32u * 1024u);
+    tma_load_3d(st + kOffQ, &tm_q, &ss->full_qv[s], 0, it.hq, row);
+    tma_load_3d(st + kHalf + kOffQ, &tm_q, &ss->full_qv[s], 64, it.hq, row);
     if (!it.zero_v) {
-      tma_load_3d(st + kOffV, &tm_v, &ss->full[s], 0, it.j, row);
-      tma_load_3d(st + kHalf + kOffV, &tm_v, &ss->full[s], 64, it.j, row);
+      tma_load_3d(st + kOffV, &tm_v, &ss->full_qv[s], 0, it.j, row);
+      tma_load_3d(st + kHalf + kOffV, &tm_v, &ss->full_qv[s], 64, it.j, row);
     }
   };
 
@@ -205,7 +212,8 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int nv = min(kChunk, it.e - (ws + c * kChunk));
       uint8_t* st = sm + s * kStageBytes;
       const uint32_t st_addr = sbase + s * kStageBytes;
-      ok = ok && mbar_wait(&ss->full[s], (c >> 1) & 1, abort_flag);
+      ok = ok && mbar_wait(&ss->full_k[s], (c >> 1) & 1, abort_flag);
+      ok = ok && mbar_wait(&ss->full_qv[s], (c >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       // full chunk: the Gram product can start at once (a partial one waits for its zeroed rows)
       if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
@@ -252,6 +260,12 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       {
         float x[4][4];
         prep_solve_strip_h(pc, x);
+        // the previous chunk's U / W products have read A2, B2 (their completion is almost
+        // always past by now)
+        if (c > 0) {
+          ok = ok && mbar_wait(&ss->wdone, (c - 1) & 1, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+        }
         prep_store_strip(pc, s, x, sbase + kOffA2, sbase + kOffB2);
       }
       fence_proxy_async_smem();
@@ -282,34 +296,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int u = 0; u < 32; ++u) z[u] = 0.f;
         tmem_st32_sync(tmem + ((uint32_t)(32 * qd) << 16) + kColDd + 32 * hc, z);
       }
-      ok = ok && mbar_wait(&ss->wdone, c & 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-      // -W -> bf16 token rows over the V tile (consumed by the U^T product): warp (qd, hc)
-      // holds tokens 16 qd + lane (lanes 0..15) at features 64 hc .. 64 hc + 63
-      {
-        float v[32], v2[32];
-        if (ok) {
-          tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + gw_col + 64 * hc, v);
-          tmem_ld32_sync(tmem + ((uint32_t)(32 * qd) << 16) + gw_col + 64 * hc + 32, v2);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] = v2[u] = 0.f;
-        }
-        if (lane < 16) {
-          const int jr = 16 * qd + lane;
-          const uint32_t wb = st_addr + hc * kHalf + kOffV;
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            st_shared_v4(wb + sw128(jr, c4), pack_bf16(-v[8 * c4], -v[8 * c4 + 1]),
-                         pack_bf16(-v[8 * c4 + 2], -v[8 * c4 + 3]), pack_bf16(-v[8 * c4 + 4], -v[8 * c4 + 5]),
-                         pack_bf16(-v[8 * c4 + 6], -v[8 * c4 + 7]));
-            st_shared_v4(wb + sw128(jr, 4 + c4), pack_bf16(-v2[8 * c4], -v2[8 * c4 + 1]),
-                         pack_bf16(-v2[8 * c4 + 2], -v2[8 * c4 + 3]), pack_bf16(-v2[8 * c4 + 4], -v2[8 * c4 + 5]),
-                         pack_bf16(-v2[8 * c4 + 6], -v2[8 * c4 + 7]));
-          }
-        }
-      }
+      // the chain waits for these products and moves -W into the stage itself
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarPrep, kNumPrep);
@@ -383,13 +370,52 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     };
     bool ok = true;
-    int loaded = 0;                               // chunks whose loads were issued (et == 0)
+    int loaded_k = 0, loaded_qv = 0;              // chunks whose K / Q,V loads were issued (et == 0)
+    // Chunk c's W (the prep's product, M = 64 layout in G/W buffer c % 2) -> -W in bf16 token
+    // rows over the stage's V tile, which the U^T product has consumed: warp (qd, hh) holds
+    // tokens 16 qd + lane (lanes 0..15) at features 64 hh .. 64 hh + 63. Ends with the
+    // epilogue barrier.
+    auto store_w = [&](int c) {
+      ok = ok && mbar_wait(&ss->wdone, c & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      float v[32], v2[32];
+      const uint32_t gw = tmem + lane_base + kColGW + 128u * (c & 1) + 64 * hh;
+      if (ok) {
+        tmem_ld32_sync(gw, v);
+        tmem_ld32_sync(gw + 32, v2);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = v2[u] = 0.f;
+      }
+      if (lane < 16) {
+        const int jr = 16 * qd + lane;
+        const uint32_t wb = sbase + (c & 1) * kStageBytes + hh * kHalf + kOffV;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          st_shared_v4(wb + sw128(jr, c4), pack_bf16(-v[8 * c4], -v[8 * c4 + 1]),
+                       pack_bf16(-v[8 * c4 + 2], -v[8 * c4 + 3]), pack_bf16(-v[8 * c4 + 4], -v[8 * c4 + 5]),
+                       pack_bf16(-v[8 * c4 + 6], -v[8 * c4 + 7]));
+          st_shared_v4(wb + sw128(jr, 4 + c4), pack_bf16(-v2[8 * c4], -v2[8 * c4 + 1]),
+                       pack_bf16(-v2[8 * c4 + 2], -v2[8 * c4 + 3]), pack_bf16(-v2[8 * c4 + 4], -v2[8 * c4 + 5]),
+                       pack_bf16(-v2[8 * c4 + 6], -v2[8 * c4 + 7]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarEpi, kNumEpi);
+    };
     if (et == 0) {
-      for (; loaded < 2 && loaded < nchunks; ++loaded) load_chunk(loaded);
+      for (; loaded_k < 2 && loaded_k < nchunks; ++loaded_k) {
+        load_k(loaded_k);
+        load_qv(loaded_k);
+      }
+      loaded_qv = loaded_k;
     }
     if (nchunks > 0) {
       ok = mbar_wait(&ss->prep_full[0], 0, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
+      store_w(0);
       if (et == 0 && ok) issue_a(0);
       if (ok) prescale(0);
       tc_fence_before();
@@ -404,6 +430,10 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int s = c & 1;
       const int t0 = ws + c * kChunk;
       wait_mma();
+      if (et == 0 && ok && c + 2 < nchunks) {     // Q~ and -W of stage s are consumed
+        load_qv(c + 2);
+        loaded_qv = c + 3;
+      }
       if (p.states != nullptr && t0 >= it.s && ok) {
         // backward support: this chunk's start state (the bf16 copy its products use)
         const uint8_t* srow = sm + kOffSb + hh * 16384u;
@@ -454,6 +484,10 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         umma_commit(&ss->mma_done);
       }
       wait_mma();
+      if (et == 0 && ok && c + 2 < nchunks) {     // K of stage s is consumed
+        load_k(c + 2);
+        loaded_k = c + 3;
+      }
       // (d) S -> bf16 copy for the next chunk's products;  O = scale * D_Q -> registers
       float oo[32];
       const int nv = ss->cs.nv[s];
@@ -483,17 +517,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
       const bool next = c + 1 < nchunks;
-      if (et == 0 && ok) {
-        if (c + 2 < nchunks) {                      // stage s fully consumed: refill it
-          load_chunk(c + 2);
-          loaded = c + 3;
-        }
-      }
-      if (next) {
-        ok = ok && mbar_wait(&ss->prep_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (et == 0 && ok) issue_a(c + 1);
-      }
       // O staging (row j = token, 256 B per row) then coalesced 16-byte stores; the
       // prescale of S for the next chunk overlaps its first product
       const bool write_o = it.write_o && t0 >= it.s && p.o != nullptr;
@@ -501,6 +524,12 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sm + kOffDt);
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) stg[(hh * 32 + jj) * 128 + r] = __float2bfloat16_rn(p.scale * oo[jj]);
+      }
+      if (next) {
+        ok = ok && mbar_wait(&ss->prep_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        store_w(c + 1);
+        if (et == 0 && ok) issue_a(c + 1);
       }
       if (next && ok) prescale((c + 1) & 1);
       tc_fence_before();
@@ -531,10 +560,11 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (et == 0 && !ok) {
       // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
-      for (int c = (loaded >= 2 ? loaded - 2 : 0); c < loaded; ++c) {
-        volatile int never = 0;
-        mbar_wait(&ss->full[c & 1], (c >> 1) & 1, &never);
-      }
+      volatile int never = 0;
+      for (int c = (loaded_k >= 2 ? loaded_k - 2 : 0); c < loaded_k; ++c)
+        mbar_wait(&ss->full_k[c & 1], (c >> 1) & 1, &never);
+      for (int c = (loaded_qv >= 2 ? loaded_qv - 2 : 0); c < loaded_qv; ++c)
+        mbar_wait(&ss->full_qv[c & 1], (c >> 1) & 1, &never);
     }
   }
 
