@@ -50,7 +50,6 @@ constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 
 struct Small {
   ChunkScalars cs;
-  float Xf[8 * 128];
   float wsum[16];
   int we;                 // end of the processed range (warm-up window end)
   uint64_t full[2], prep_full[2], gdone, mma_done;
@@ -161,7 +160,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ prep (8 warps)
     const int pt = threadIdx.x;
-    PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), ss->Xf, &ss->cs, tmem, kColG, pt, warp, lane, kBarPrep};
+    PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColG, pt, warp, lane, kBarPrep};
     bool ok = true;
     for (int k = 0; k < nchunks; ++k) {
       const int s = k & 1;
@@ -194,7 +193,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ok = ok && mbar_wait(&ss->gdone, k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      prep_masks<true>(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P; L as fp16
+      prep_masks(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P; L as fp16
       // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- scale diag(exp(gam)) Q;
       // then one column strip of A per warp -> A diag(beta)
       if (warp < 4) prep_diag_inverse_h(pc);

@@ -194,8 +194,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_load_3d(sm + kOffDS, &tm_ds, &ss->tma_bar, 0, 0, srow);
     tma_load_3d(sm + kOffDS + 16384, &tm_ds, &ss->tma_bar, 64, 0, srow);
   }
-  PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), reinterpret_cast<float*>(sm + kOffYt), &ss->cs,
-             tmem, kColG, tid, warp, lane, kBar};
+  PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColG, tid, warp, lane, kBar};
   float gv = 0.f, bv = 0.f;
   if (tid < nv) {
     const size_t gi = (size_t)row * p.Hv + j + (size_t)tid * p.Hv;
@@ -231,7 +230,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   ok = __syncthreads_and(ok);
   mph ^= 1;
   tc_fence_after();
-  prep_masks<true>(pc, 0, sbase + kOffP, p.scale, ok);
+  prep_masks(pc, 0, sbase + kOffP, p.scale, ok);
   fence_proxy_async_smem();                   // scale * P is an operand of the next products
   __syncthreads();
   if (tid == 0 && ok) {

@@ -5,9 +5,10 @@
 //
 //   gam = inclusive cumsum of g,  E_ij = exp(gam_i - gam_j)
 //   G = [K;Q] K^T   (one tcgen05 product, rows 0..63 = K K^T, rows 64..127 = Q K^T)
-//   L = strict_lower(diag(beta) K K^T * E)  -> fp32, inverted in place: A = (I + L)^-1
+//   L = strict_lower(diag(beta) K K^T * E)  -> fp16;  A = (I + L)^-1: 16 x 16 diagonal
+//       blocks by substitution, then one 8-column strip of A per warp (m16n8k16 products)
 //   P = lower_incl(Q K^T * E) * p_scale     -> bf16
-//   A2 = A diag(beta) -> bf16 (and A itself -> bf16 when asked)
+//   A2 = A diag(beta) -> bf16 (with B2 = A diag(beta exp(gam)), or A in bf16 and fp32)
 #pragma once
 
 #include <cuda_bf16.h>
@@ -18,10 +19,10 @@
 
 namespace gdn {
 
-// Row stride (floats) of the fp32 64 x 64 scratch. 68 = 4 mod 32 makes the m16n8k8 A
-// fragments (row gid, column tig) hit 32 distinct banks; row-per-thread accesses go through
-// 16-byte vectors (8 threads per phase, rows 4 banks apart: conflict-free) and
-// column-per-thread accesses stay scalar (consecutive rows, distinct banks).
+// Row stride (floats) of the fp32 64 x 64 scratch rows (A and dG in the gradient kernel).
+// 68: row-per-thread accesses go through 16-byte vectors (8 threads per phase, rows 4 banks
+// apart: conflict-free) and column-per-thread accesses stay scalar (consecutive rows,
+// distinct banks).
 constexpr int kLd = 68;
 // Row stride (halves) of the fp16 64 x 64 variant of the scratch: 36 words = 4 mod 32, so
 // the m16n8k16 A fragments (row gid, word tig) hit 32 distinct banks.
@@ -66,8 +67,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 
 struct PrepCtx {
   uint32_t sbase;     // shared address of the 1024-aligned smem base
-  float* Lf;          // fp32 [64][kLd] scratch
-  float* Xf;          // fp32 8 x 128 scratch
+  float* Lf;          // scratch: fp16 L [64][kLdh]; fp32 rows [64][kLd] where a kernel asks
   ChunkScalars* cs;
   uint32_t tmem;      // TMEM base
   uint32_t colG;      // TMEM column of G
@@ -129,13 +129,11 @@ __device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, ui
   tc::umma_commit(bar);
 }
 
-// G (TMEM) -> L (fp32 in Lf, strictly lower) and P = p_scale * lower_incl(QK^T * E) (bf16,
+// G (TMEM) -> L (fp16 rows of stride kLdh in Lf, strictly lower) and P = p_scale * lower_incl(QK^T * E) (bf16,
 // 128B-swizzled rows at p_addr). E_ij = exp(gam_i - gam_j) (j <= i) is the running product
 // of exp(g_t) over t = j+1..i, walking j down: one exponential per row segment instead of
 // one per entry, no overflow, monotone underflow to 0. `ok` false: G treated as 0.
 // Ends with tcgen05 fence + group barrier.
-// kHalfL: L goes to the scratch as fp16 rows of stride kLdh instead of fp32 rows of kLd.
-template <bool kHalfL = false>
 __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_addr, float p_scale, bool ok) {
   const int qd = c.pw & 3, hc = c.pw >> 2;
   const int rr = 32 * qd + c.lane;
@@ -169,17 +167,11 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
       else run = (j >= i) ? 1.f : run * et[jj + 1];
       vals[jj] = (j < i) ? bi * vals[jj] * run : 0.f;
     }
-    if (kHalfL) {
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(c.Lf) + i * kLdh + j0);
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(c.Lf) + i * kLdh + j0);
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        dst[u] = make_uint4(pack_h2(vals[8 * u], vals[8 * u + 1]), pack_h2(vals[8 * u + 2], vals[8 * u + 3]),
-                            pack_h2(vals[8 * u + 4], vals[8 * u + 5]), pack_h2(vals[8 * u + 6], vals[8 * u + 7]));
-    } else {
-      float4* dst = reinterpret_cast<float4*>(c.Lf + i * kLd + j0);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) dst[u] = make_float4(vals[4 * u], vals[4 * u + 1], vals[4 * u + 2], vals[4 * u + 3]);
-    }
+    for (int u = 0; u < 4; ++u)
+      dst[u] = make_uint4(pack_h2(vals[8 * u], vals[8 * u + 1]), pack_h2(vals[8 * u + 2], vals[8 * u + 3]),
+                          pack_h2(vals[8 * u + 4], vals[8 * u + 5]), pack_h2(vals[8 * u + 6], vals[8 * u + 7]));
   } else {
 #pragma unroll
     for (int jj = 31; jj >= 0; --jj) {
@@ -225,139 +217,6 @@ __device__ __forceinline__ void scale_rows_tile_part(uint8_t* tile, uint32_t sub
     const int row = idx >> 4, half = (idx >> 3) & 1, ch = idx & 7;
     uint4* q = reinterpret_cast<uint4*>(tile + half * sub_stride + row * 128 + ch * 16);
     *q = scale_chunk(*q, f[row] * mult);
-  }
-}
-
-// 16 x 16 unit-lower diagonal blocks of (I + L) inverted in place in Lf by forward
-// substitution. Called by warps 0..3 of the group: warp R inverts block R, lane = column
-// (lanes 16..31 mirror 0..15). Rows are read as 16-byte broadcasts. No group barrier.
-__device__ __forceinline__ void prep_diag_inverse(const PrepCtx& c) {
-  float* Lf = c.Lf;
-  const int R = c.pw, col = c.lane & 15;
-  float a[16];
-#pragma unroll
-  for (int ii = 0; ii < 16; ++ii) {
-    float l[16];
-    const float4* row = reinterpret_cast<const float4*>(Lf + (16 * R + ii) * kLd + 16 * R);
-#pragma unroll
-    for (int q4 = 0; q4 < (ii + 3) / 4; ++q4) {
-      const float4 t = row[q4];
-      l[4 * q4] = t.x; l[4 * q4 + 1] = t.y; l[4 * q4 + 2] = t.z; l[4 * q4 + 3] = t.w;
-    }
-    // two accumulation chains (even / odd jj) halve the dependent latency
-    float acc0 = (ii == col) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int jj = 0; jj < ii; jj += 2) {
-      acc0 -= l[jj] * a[jj];
-      if (jj + 1 < ii) acc1 -= l[jj + 1] * a[jj + 1];
-    }
-    a[ii] = (ii < col) ? 0.f : acc0 + acc1;
-  }
-  __syncwarp();
-  if (c.lane < 16) {
-#pragma unroll
-    for (int ii = 0; ii < 16; ++ii) Lf[(16 * R + ii) * kLd + 16 * R + col] = a[ii];
-  }
-}
-
-// m16n8k8 tf32 product without the volatile qualifier (a pure register operation, so the
-// compiler may interleave independent products)
-__device__ __forceinline__ void mma_tf32_free(float* d, const uint32_t* a, const uint32_t* b) {
-  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// A fragment (16 x 8 at rows r0.., columns k0..) of the fp32 row-major scratch
-__device__ __forceinline__ void lf_afrag(const float* Lf, int r0, int k0, int gid, int tig, uint32_t* af) {
-  af[0] = tc::to_tf32(Lf[(r0 + gid) * kLd + k0 + tig]);
-  af[1] = tc::to_tf32(Lf[(r0 + gid + 8) * kLd + k0 + tig]);
-  af[2] = tc::to_tf32(Lf[(r0 + gid) * kLd + k0 + tig + 4]);
-  af[3] = tc::to_tf32(Lf[(r0 + gid + 8) * kLd + k0 + tig + 4]);
-}
-
-// B fragments (k rows 0..7 -> bf[0..1], rows 8..15 -> bf[2..3]) of a 16 x 8 tile held in
-// accumulator layout (lane 4 r + c / 2 holds rows r, r + 8 at columns c, c + 1), by shuffles
-__device__ __forceinline__ void acc_to_bfrag(const float* x, int lane, uint32_t* bf) {
-  const int gid = lane >> 2, tig = lane & 3;
-  const int s0 = tig * 4 + (gid >> 1), s1 = s0 + 16;
-  const bool odd = gid & 1;
-#pragma unroll
-  for (int kk = 0; kk < 2; ++kk) {
-    const float e0 = __shfl_sync(0xffffffffu, x[2 * kk], s0), o0 = __shfl_sync(0xffffffffu, x[2 * kk + 1], s0);
-    const float e1 = __shfl_sync(0xffffffffu, x[2 * kk], s1), o1 = __shfl_sync(0xffffffffu, x[2 * kk + 1], s1);
-    bf[2 * kk] = tc::to_tf32(odd ? o0 : e0);
-    bf[2 * kk + 1] = tc::to_tf32(odd ? o1 : e1);
-  }
-}
-
-// A = (I + L)^-1 from the inverted diagonal blocks D_R (prep_diag_inverse) and the strictly
-// lower blocks L_{R,R'} of Lf, which it only reads: one 8-column strip per warp of the
-// group, no group barrier. Warp w owns columns 8w .. 8w+7, whose first nonzero block row
-// is R0 = w / 2:
-//   X_R0 = D_R0 (its columns),   X_R = -D_R sum_{R0 <= R' < R} L_{R,R'} X_R'   (R > R0)
-// as m16n8k8 tf32 products. Each solved block adds its term to every later block row at
-// once, so the dependent path is one (L, D) product pair per block row.
-// Out: x[R] = rows 16R + gid (+8) at columns 8w + 2 tig (+1), accumulator layout.
-// R0 is a template parameter so that each warp's path is straight-line code and the
-// compiler can issue every fragment load ahead of the dependent products.
-template <int R0>
-__device__ __forceinline__ void prep_solve_strip_t(const PrepCtx& c, float (&x)[4][4]) {
-  const float* Lf = c.Lf;
-  const int gid = c.lane >> 2, tig = c.lane & 3;
-  const int n0 = 8 * c.pw;
-  float t[4][4];
-#pragma unroll
-  for (int R = 0; R < 4; ++R)
-#pragma unroll
-    for (int u = 0; u < 4; ++u) t[R][u] = 0.f;
-#pragma unroll
-  for (int R = 0; R < R0; ++R)
-#pragma unroll
-    for (int u = 0; u < 4; ++u) x[R][u] = 0.f;
-  {
-    const float* d = Lf + (16 * R0 + gid) * kLd + n0 + 2 * tig;
-    x[R0][0] = d[0];
-    x[R0][1] = d[1];
-    x[R0][2] = d[8 * kLd];
-    x[R0][3] = d[8 * kLd + 1];
-  }
-#pragma unroll
-  for (int R = R0; R < 4; ++R) {
-    if (R > R0) {
-      uint32_t bt[4];
-      acc_to_bfrag(t[R], c.lane, bt);
-      float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        uint32_t af[4];
-        lf_afrag(Lf, 16 * R, 16 * R + 8 * kk, gid, tig, af);
-        mma_tf32_free(y, af, bt + 2 * kk);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) x[R][u] = -y[u];
-    }
-    if (R < 3) {
-      uint32_t bx[4];
-      acc_to_bfrag(x[R], c.lane, bx);
-#pragma unroll
-      for (int R2 = R + 1; R2 < 4; ++R2) {
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          uint32_t af[4];
-          lf_afrag(Lf, 16 * R2, 16 * R + 8 * kk, gid, tig, af);
-          mma_tf32_free(t[R2], af, bx + 2 * kk);
-        }
-      }
-    }
-  }
-}
-__device__ __forceinline__ void prep_solve_strip(const PrepCtx& c, float (&x)[4][4]) {
-  switch (c.pw >> 1) {                       // uniform over the warp
-    case 0: prep_solve_strip_t<0>(c, x); break;
-    case 1: prep_solve_strip_t<1>(c, x); break;
-    case 2: prep_solve_strip_t<2>(c, x); break;
-    default: prep_solve_strip_t<3>(c, x); break;
   }
 }
 
@@ -506,126 +365,6 @@ __device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const 
       if (b2_addr)
         asm volatile("st.shared.b32 [%0], %1;" ::"r"(b2_addr + off), "r"(tc::pack_bf16(v0 * e0, v1 * e1)) : "memory");
     }
-  }
-}
-
-// A = (I + L)^-1 in place in Lf: 16x16 diagonal blocks by forward substitution (warps
-// 0..3), then block rows R = 1..3: A[R,<R] = -D_R (L[R,<R] A[<R,<R]) as 16 x 8 tiles of
-// m16n8k8 tf32 products (warp w: tile w). Starts and ends with a group barrier.
-__device__ __forceinline__ void prep_inverse(const PrepCtx& c) {
-  float* Lf = c.Lf;
-  if (c.pw < 4) {
-    const int R = c.pw, col = c.lane & 15;
-    float a[16];
-#pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      // two independent accumulation chains (even / odd jj) halve the dependent latency
-      float acc0 = (ii == col) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < ii; jj += 2) {
-        acc0 -= Lf[(16 * R + ii) * kLd + 16 * R + jj] * a[jj];
-        if (jj + 1 < ii) acc1 -= Lf[(16 * R + ii) * kLd + 16 * R + jj + 1] * a[jj + 1];
-      }
-      a[ii] = (ii < col) ? 0.f : acc0 + acc1;
-    }
-    __syncwarp();
-    if (c.lane < 16) {
-#pragma unroll
-      for (int ii = 0; ii < 16; ++ii) Lf[(16 * R + ii) * kLd + 16 * R + col] = a[ii];
-    }
-  }
-  tc::named_bar_sync(c.bar, kPrepThreads);
-  const int gid = c.lane >> 2, tig = c.lane & 3;
-#pragma unroll
-  for (int R = 1; R < 4; ++R) {
-    const int K = 16 * R;
-    const int tile = c.pw;
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
-    if (tile < 2 * R) {
-      const int n0 = 8 * tile;
-      // two accumulator chains over alternate k-steps, summed at the end
-      float x[4] = {0.f, 0.f, 0.f, 0.f}, x2[4] = {0.f, 0.f, 0.f, 0.f};
-      const float* lr = Lf + (16 * R) * kLd;
-#pragma unroll
-      for (int k0 = 0; k0 < K; k0 += 8) {
-        uint32_t af[4], bf[2];
-        af[0] = tc::to_tf32(lr[gid * kLd + k0 + tig]);
-        af[1] = tc::to_tf32(lr[(gid + 8) * kLd + k0 + tig]);
-        af[2] = tc::to_tf32(lr[gid * kLd + k0 + tig + 4]);
-        af[3] = tc::to_tf32(lr[(gid + 8) * kLd + k0 + tig + 4]);
-        bf[0] = tc::to_tf32(Lf[(k0 + tig) * kLd + n0 + gid]);
-        bf[1] = tc::to_tf32(Lf[(k0 + tig + 4) * kLd + n0 + gid]);
-        if ((k0 >> 3) & 1) tc::mma_tf32_16x8x8(x2, af, bf);
-        else tc::mma_tf32_16x8x8(x, af, bf);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) x[u] += x2[u];
-      float* xw = c.Xf + c.pw * 128;
-      *reinterpret_cast<float2*>(xw + gid * 8 + 2 * tig) = make_float2(x[0], x[1]);
-      *reinterpret_cast<float2*>(xw + (gid + 8) * 8 + 2 * tig) = make_float2(x[2], x[3]);
-      __syncwarp();
-      const float* dr = Lf + (16 * R) * kLd + 16 * R;
-#pragma unroll
-      for (int k0 = 0; k0 < 16; k0 += 8) {
-        uint32_t af[4], bf[2];
-        af[0] = tc::to_tf32(dr[gid * kLd + k0 + tig]);
-        af[1] = tc::to_tf32(dr[(gid + 8) * kLd + k0 + tig]);
-        af[2] = tc::to_tf32(dr[gid * kLd + k0 + tig + 4]);
-        af[3] = tc::to_tf32(dr[(gid + 8) * kLd + k0 + tig + 4]);
-        bf[0] = tc::to_tf32(xw[(k0 + tig) * 8 + gid]);
-        bf[1] = tc::to_tf32(xw[(k0 + tig + 4) * 8 + gid]);
-        tc::mma_tf32_16x8x8(y, af, bf);
-      }
-    }
-    tc::named_bar_sync(c.bar, kPrepThreads);       // every warp is done reading L[R, <R]
-    if (tile < 2 * R) {
-      float* ar = Lf + (16 * R) * kLd + 8 * tile;
-      ar[gid * kLd + 2 * tig] = -y[0];
-      ar[gid * kLd + 2 * tig + 1] = -y[1];
-      ar[(gid + 8) * kLd + 2 * tig] = -y[2];
-      ar[(gid + 8) * kLd + 2 * tig + 1] = -y[3];
-    }
-    tc::named_bar_sync(c.bar, kPrepThreads);
-  }
-}
-
-// A2 = A diag(beta) -> bf16 rows at a2_addr; with a_addr != 0 also A -> bf16, with
-// b2_addr != 0 also B2 = A diag(beta exp(gam)) -> bf16 (thread: 16 columns of one row; a
-// warp covers 32 consecutive rows of one 16-column quarter).
-__device__ __forceinline__ void prep_write_a(const PrepCtx& c, int s, uint32_t a2_addr, uint32_t a_addr,
-                                             uint32_t b2_addr = 0) {
-  const int i = c.pt & 63, qq = c.pt >> 6;
-  const float* bet = c.cs->bet[s];
-  float a[16];
-  const float4* src = reinterpret_cast<const float4*>(c.Lf + i * kLd + qq * 16);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float4 t = src[u];
-    a[4 * u] = t.x; a[4 * u + 1] = t.y; a[4 * u + 2] = t.z; a[4 * u + 3] = t.w;
-  }
-  uint32_t w[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int j0 = qq * 16 + 2 * u;
-    w[u] = tc::pack_bf16(a[2 * u] * bet[j0], a[2 * u + 1] * bet[j0 + 1]);
-  }
-  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
-  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
-  if (b2_addr) {
-    const float* eg = c.cs->eg[s];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j0 = qq * 16 + 2 * u;
-      w[u] = tc::pack_bf16(a[2 * u] * (bet[j0] * eg[j0]), a[2 * u + 1] * (bet[j0 + 1] * eg[j0 + 1]));
-    }
-    st_shared_v4(b2_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
-    st_shared_v4(b2_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
-  }
-  if (a_addr) {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) w[u] = tc::pack_bf16(a[2 * u], a[2 * u + 1]);
-    st_shared_v4(a_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
-    st_shared_v4(a_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
   }
 }
 

@@ -60,7 +60,6 @@ constexpr uint32_t kOffSmall = kOffLf + 64u * kLdh * 2u;
 
 struct Small {
   ChunkScalars cs;
-  float Xf[8 * 128];      // inverse scratch: one 16 x 8 tile per prep warp
   float wsum[16];         // warm-up window search: per-warp partial sums
   int ws;                 // warm-up start token (context parallelism)
   uint64_t full_k[2], full_qv[2], prep_full[2], gdone, wdone, mma_done, dd_free;
@@ -191,7 +190,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ prep (8 warps)
     const int pt = threadIdx.x;            // 0..255
-    PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), ss->Xf, &ss->cs, tmem, kColGW, pt, warp, lane, kBarPrep};
+    PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColGW, pt, warp, lane, kBarPrep};
     bool ok = true;
     const int qd = warp & 3, hc = warp >> 2;
     // g, beta of a chunk (0 past the sequence end), loaded one chunk ahead
@@ -251,7 +250,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       pc.colG = gw_col;
-      prep_masks<true>(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
+      prep_masks(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
       // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- diag(exp(gam)) Q
       // in place (the Gram product has consumed Q); then one column strip of A per warp
       if (warp < 4) prep_diag_inverse_h(pc);
