@@ -203,6 +203,9 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         float x[4][4];
         prep_solve_strip_h(pc, x);
         prep_store_strip(pc, s, x, sbase + kOffA2 + s * 8192u, 0);
+        if (p.chunk_a != nullptr && t0 < it.e && ok)   // the gradient kernel's copy of A
+          prep_store_strip_global(pc, x, p.chunk_a + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
+                                                         (size_t)(kChunk * kChunk));
       }
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);

@@ -195,6 +195,16 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_load_3d(sm + kOffDS + 16384, &tm_ds, &ss->tma_bar, 64, 0, srow);
   }
   PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColG, tid, warp, lane, kBar};
+  // A = (I + L)^-1 of this chunk, as the reverse chain computed it: fp32 rows into the scratch
+  {
+    const float* ag = out.chunk_a + (size_t)srow / 128 * (kChunk * kChunk);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = tid + kThreads * m, ar = idx >> 4, c16 = idx & 15;
+      cp_async_16(sbase + kOffLf + (uint32_t)(ar * kLd + c16 * 4) * 4u, ag + ar * kChunk + c16 * 4);
+    }
+    cp_async_commit();
+  }
   float gv = 0.f, bv = 0.f;
   if (tid < nv) {
     const size_t gi = (size_t)row * p.Hv + j + (size_t)tid * p.Hv;
@@ -230,7 +240,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   ok = __syncthreads_and(ok);
   mph ^= 1;
   tc_fence_after();
-  prep_masks(pc, 0, sbase + kOffP, p.scale, ok);
+  prep_masks<false>(pc, 0, sbase + kOffP, p.scale, ok);
   fence_proxy_async_smem();                   // scale * P is an operand of the next products
   __syncthreads();
   if (tid == 0 && ok) {
@@ -250,16 +260,10 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       umma_f16(tmem + kColDb, mdesc(sbase + kOffVDO + 8192 + ks * 2048, 16384), mdesc(sbase + kOffP + ks * 2048, 8192),
                idmm, ks > 0);
   }
-  // A = (I + L)^-1: diagonal blocks (warps 0-3), then one column strip per warp; the
-  // fp32 A rows replace the fp16 L once every strip is solved
-  if (warp < 4) prep_diag_inverse_h(pc);
+  // A (fp32 rows, from the reverse chain) -> A diag(beta) and A in bf16
+  cp_async_wait_all();
   __syncthreads();
-  {
-    float xs[4][4];
-    prep_solve_strip_h(pc, xs);
-    __syncthreads();
-    prep_store_strip_a(pc, 0, xs, sbase + kOffA2, sbase + kOffA);
-  }
+  prep_write_a_rows(pc, 0, sbase + kOffA2, sbase + kOffA);
   fence_proxy_async_smem();
   commit_wait();
   const float* eg = ss->cs.eg[0];

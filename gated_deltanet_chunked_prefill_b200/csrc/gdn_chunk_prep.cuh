@@ -134,6 +134,8 @@ __device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, ui
 // of exp(g_t) over t = j+1..i, walking j down: one exponential per row segment instead of
 // one per entry, no overflow, monotone underflow to 0. `ok` false: G treated as 0.
 // Ends with tcgen05 fence + group barrier.
+// kWriteL false: only P is produced (the caller has A from elsewhere).
+template <bool kWriteL = true>
 __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_addr, float p_scale, bool ok) {
   const int qd = c.pw & 3, hc = c.pw >> 2;
   const int rr = 32 * qd + c.lane;
@@ -158,7 +160,9 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
   const float gi = c.cs->gam[s][i];
   const float glast = c.cs->gam[s][j0 + 31];
   float run = 1.f;
-  if (rr < kChunk) {
+  if (rr < kChunk && !kWriteL) {
+    // no L wanted
+  } else if (rr < kChunk) {
     const float bi = c.cs->bet[s][i];
 #pragma unroll
     for (int jj = 31; jj >= 0; --jj) {
@@ -366,6 +370,44 @@ __device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const 
         asm volatile("st.shared.b32 [%0], %1;" ::"r"(b2_addr + off), "r"(tc::pack_bf16(v0 * e0, v1 * e1)) : "memory");
     }
   }
+}
+
+// A2 = A diag(beta) and A -> bf16 (128B-swizzled rows at a2_addr, a_addr) from the fp32 rows
+// of A (stride kLd) in the scratch (thread: 16 columns of one row; a warp covers 32
+// consecutive rows of one 16-column quarter).
+__device__ __forceinline__ void prep_write_a_rows(const PrepCtx& c, int s, uint32_t a2_addr, uint32_t a_addr) {
+  const int i = c.pt & 63, qq = c.pt >> 6;
+  const float* bet = c.cs->bet[s];
+  float a[16];
+  const float4* src = reinterpret_cast<const float4*>(c.Lf + i * kLd + qq * 16);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 t = src[u];
+    a[4 * u] = t.x; a[4 * u + 1] = t.y; a[4 * u + 2] = t.z; a[4 * u + 3] = t.w;
+  }
+  uint32_t w[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int j0 = qq * 16 + 2 * u;
+    w[u] = tc::pack_bf16(a[2 * u] * bet[j0], a[2 * u + 1] * bet[j0 + 1]);
+  }
+  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) w[u] = tc::pack_bf16(a[2 * u], a[2 * u + 1]);
+  st_shared_v4(a_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+  st_shared_v4(a_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+}
+
+// A strip's fragments (prep_solve_strip_h) -> fp32 rows of a global 64 x 64 matrix.
+__device__ __forceinline__ void prep_store_strip_global(const PrepCtx& c, const float (&x)[4][4], float* a_g) {
+  const int gid = c.lane >> 2, tig = c.lane & 3;
+  const int j = 8 * c.pw + 2 * tig;
+#pragma unroll
+  for (int R = 0; R < 4; ++R)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      *reinterpret_cast<float2*>(a_g + (16 * R + gid + 8 * h) * kChunk + j) = make_float2(x[R][2 * h], x[R][2 * h + 1]);
 }
 
 // A2 = A diag(beta) and A -> bf16 (128B-swizzled rows at a2_addr, a_addr), and A -> fp32

@@ -36,6 +36,9 @@ struct FwdParams {
   // states + ((chunk_off[n] + chunk) * Hv + j) * dv * dk; chunk_off nullable -> n * ceil(T/64)
   __nv_bfloat16* states;    // nullable
   const int* chunk_off;     // nullable
+  // backward support: A = (I + L)^-1 (fp32, 64 x 64 row-major) of every chunk, written by the
+  // reverse chain at chunk_a + (slot * Hv + j) * 4096 (slot as for states); nullable
+  float* chunk_a;
   int B, T, Hqk, Hv, dk, dv, N;
   float scale;
 };
