@@ -133,7 +133,8 @@ struct BwdPlan {
   FwdPlan chain;                 // gate-driven segments (or none) for the two sequential passes
   long long total_chunks = 0;    // chunk slots (upper bound for packed sequences)
   bool grouped = false;
-  size_t off_chunk_off = 0, off_states = 0, off_dstates = 0, off_a = 0, off_dq = 0, off_dk = 0, total = kStatusBytes;
+  size_t off_chunk_off = 0, off_states = 0, off_dstates = 0, off_a = 0, off_p = 0, off_dq = 0, off_dk = 0;
+  size_t total = kStatusBytes;
 };
 
 BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
@@ -151,6 +152,7 @@ BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
   if (!(opt && opt->states)) { b.off_states = off; off = align256(off + st); }
   b.off_dstates = off; off = align256(off + st);
   b.off_a = off; off = align256(off + (size_t)b.total_chunks * s.Hv * kChunk * kChunk * sizeof(float));
+  b.off_p = off; off = align256(off + (size_t)b.total_chunks * s.Hv * kChunk * kChunk * 2);
   if (b.grouped) {
     const size_t part = (size_t)s.B * s.T * s.Hv * s.dk * sizeof(float);
     b.off_dq = off; off = align256(off + part);
@@ -436,6 +438,7 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   pc.hT = dh0;
   pc.states = dstates;
   pc.chunk_a = reinterpret_cast<float*>(ws + bp.off_a);
+  pc.chunk_p = ws + bp.off_p;
   err = launch_bwd_chain(pc, plan, items, stream, &what);
   if (err != cudaSuccess) return cuda_fail(what, err);
   // 3) per-chunk gradients
@@ -443,6 +446,7 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   out.dq = dq; out.dk = dk_out; out.dv = dv_out; out.dg = dg; out.dbeta = dbeta; out.dO = dO;
   out.dstates = dstates;
   out.chunk_a = reinterpret_cast<const float*>(ws + bp.off_a);
+  out.chunk_p = ws + bp.off_p;
   out.qk_partial = bp.grouped ? 1 : 0;
   out.dq_part = bp.grouped ? reinterpret_cast<float*>(ws + bp.off_dq) : nullptr;
   out.dk_part = bp.grouped ? reinterpret_cast<float*>(ws + bp.off_dk) : nullptr;

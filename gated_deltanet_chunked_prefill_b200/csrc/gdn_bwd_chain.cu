@@ -194,6 +194,13 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       prep_masks(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P; L as fp16
+      if (p.chunk_p != nullptr && t0 < it.e && ok) {      // the gradient kernel's copy of scale * P
+        uint4* dst = reinterpret_cast<uint4*>(p.chunk_p + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
+                                                              (size_t)8192);
+        const uint4* src = reinterpret_cast<const uint4*>(sm + kOffP + s * 8192u);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) dst[pt + kNumPrep * m] = src[pt + kNumPrep * m];
+      }
       // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- scale diag(exp(gam)) Q;
       // then one column strip of A per warp -> A diag(beta)
       if (warp < 4) prep_diag_inverse_h(pc);

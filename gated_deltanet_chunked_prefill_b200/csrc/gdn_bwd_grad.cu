@@ -203,6 +203,13 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int idx = tid + kThreads * m, ar = idx >> 4, c16 = idx & 15;
       cp_async_16(sbase + kOffLf + (uint32_t)(ar * kLd + c16 * 4) * 4u, ag + ar * kChunk + c16 * 4);
     }
+    // and scale * P (the swizzled bf16 tile, byte for byte)
+    const uint8_t* pg = out.chunk_p + (size_t)srow / 128 * 8192;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int idx = tid + kThreads * m;
+      cp_async_16(sbase + kOffP + idx * 16u, pg + idx * 16);
+    }
     cp_async_commit();
   }
   float gv = 0.f, bv = 0.f;
@@ -240,7 +247,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   ok = __syncthreads_and(ok);
   mph ^= 1;
   tc_fence_after();
-  prep_masks<false>(pc, 0, sbase + kOffP, p.scale, ok);
+  cp_async_wait_all();                        // A and scale * P from the reverse chain
   fence_proxy_async_smem();                   // scale * P is an operand of the next products
   __syncthreads();
   if (tid == 0 && ok) {
@@ -261,8 +268,6 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                idmm, ks > 0);
   }
   // A (fp32 rows, from the reverse chain) -> A diag(beta) and A in bf16
-  cp_async_wait_all();
-  __syncthreads();
   prep_write_a_rows(pc, 0, sbase + kOffA2, sbase + kOffA);
   fence_proxy_async_smem();
   commit_wait();

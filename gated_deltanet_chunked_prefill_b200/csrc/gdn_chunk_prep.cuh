@@ -134,8 +134,6 @@ __device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, ui
 // of exp(g_t) over t = j+1..i, walking j down: one exponential per row segment instead of
 // one per entry, no overflow, monotone underflow to 0. `ok` false: G treated as 0.
 // Ends with tcgen05 fence + group barrier.
-// kWriteL false: only P is produced (the caller has A from elsewhere).
-template <bool kWriteL = true>
 __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_addr, float p_scale, bool ok) {
   const int qd = c.pw & 3, hc = c.pw >> 2;
   const int rr = 32 * qd + c.lane;
@@ -160,9 +158,7 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
   const float gi = c.cs->gam[s][i];
   const float glast = c.cs->gam[s][j0 + 31];
   float run = 1.f;
-  if (rr < kChunk && !kWriteL) {
-    // no L wanted
-  } else if (rr < kChunk) {
+  if (rr < kChunk) {
     const float bi = c.cs->bet[s][i];
 #pragma unroll
     for (int jj = 31; jj >= 0; --jj) {
