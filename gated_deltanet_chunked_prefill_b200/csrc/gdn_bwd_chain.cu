@@ -167,6 +167,9 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int t0 = it.s + chunk_of(k) * kChunk;
       const int nv = min(kChunk, we - t0);
       uint8_t* st = sm + s * kStageBytes;
+      // A = (I + L)^-1 of this chunk, as the forward pass computed it (same arithmetic)
+      prep_fetch_a(pc, p.chunk_a + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
+                                       (size_t)(kChunk * kChunk));
       float gv = 0.f, bv = 0.f;
       if (pt < kChunk && pt < nv) {
         const size_t gi = (size_t)(it.b * p.T + t0 + pt) * p.Hv + it.j;
@@ -193,7 +196,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ok = ok && mbar_wait(&ss->gdone, k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      prep_masks(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P; L as fp16
+      prep_masks<false>(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P
       if (p.chunk_p != nullptr && t0 < it.e && ok) {      // the gradient kernel's copy of scale * P
         uint4* dst = reinterpret_cast<uint4*>(p.chunk_p + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
                                                               (size_t)8192);
@@ -201,19 +204,10 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
         for (int m = 0; m < 2; ++m) dst[pt + kNumPrep * m] = src[pt + kNumPrep * m];
       }
-      // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- scale diag(exp(gam)) Q;
-      // then one column strip of A per warp -> A diag(beta)
-      if (warp < 4) prep_diag_inverse_h(pc);
-      else scale_rows_tile_part(st + 8192, 16384, ss->cs.eg[s], p.scale, pt - 128, 128);
+      scale_rows_tile_part(st + 8192, 16384, ss->cs.eg[s], p.scale, pt, kNumPrep);   // Q <- scale diag(exp(gam)) Q
+      tc::cp_async_wait_all();
       named_bar_sync(kBarPrep, kNumPrep);
-      {
-        float x[4][4];
-        prep_solve_strip_h(pc, x);
-        prep_store_strip(pc, s, x, sbase + kOffA2 + s * 8192u, 0);
-        if (p.chunk_a != nullptr && t0 < it.e && ok)   // the gradient kernel's copy of A
-          prep_store_strip_global(pc, x, p.chunk_a + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
-                                                         (size_t)(kChunk * kChunk));
-      }
+      prep_write_a_rows(pc, s, sbase + kOffA2 + s * 8192u, 0);                       // A diag(beta)
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);

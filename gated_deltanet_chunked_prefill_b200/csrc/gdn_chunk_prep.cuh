@@ -134,6 +134,8 @@ __device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, ui
 // of exp(g_t) over t = j+1..i, walking j down: one exponential per row segment instead of
 // one per entry, no overflow, monotone underflow to 0. `ok` false: G treated as 0.
 // Ends with tcgen05 fence + group barrier.
+// kWriteL false: only P is produced (the caller takes A from elsewhere).
+template <bool kWriteL = true>
 __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_addr, float p_scale, bool ok) {
   const int qd = c.pw & 3, hc = c.pw >> 2;
   const int rr = 32 * qd + c.lane;
@@ -158,7 +160,9 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
   const float gi = c.cs->gam[s][i];
   const float glast = c.cs->gam[s][j0 + 31];
   float run = 1.f;
-  if (rr < kChunk) {
+  if (rr < kChunk && !kWriteL) {
+    // L not wanted
+  } else if (rr < kChunk) {
     const float bi = c.cs->bet[s][i];
 #pragma unroll
     for (int jj = 31; jj >= 0; --jj) {
@@ -371,6 +375,7 @@ __device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const 
 // A2 = A diag(beta) and A -> bf16 (128B-swizzled rows at a2_addr, a_addr) from the fp32 rows
 // of A (stride kLd) in the scratch (thread: 16 columns of one row; a warp covers 32
 // consecutive rows of one 16-column quarter).
+// (a_addr == 0: A2 only)
 __device__ __forceinline__ void prep_write_a_rows(const PrepCtx& c, int s, uint32_t a2_addr, uint32_t a_addr) {
   const int i = c.pt & 63, qq = c.pt >> 6;
   const float* bet = c.cs->bet[s];
@@ -389,10 +394,23 @@ __device__ __forceinline__ void prep_write_a_rows(const PrepCtx& c, int s, uint3
   }
   st_shared_v4(a2_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
   st_shared_v4(a2_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  if (a_addr) {
 #pragma unroll
-  for (int u = 0; u < 8; ++u) w[u] = tc::pack_bf16(a[2 * u], a[2 * u + 1]);
-  st_shared_v4(a_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
-  st_shared_v4(a_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+    for (int u = 0; u < 8; ++u) w[u] = tc::pack_bf16(a[2 * u], a[2 * u + 1]);
+    st_shared_v4(a_addr + tc::sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+    st_shared_v4(a_addr + tc::sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  }
+}
+
+// Start fetching a chunk's A (fp32 64 x 64 rows in global memory) into the scratch as rows of
+// stride kLd, 4 x 16 bytes per thread of a 256-thread group (completion: cp_async_wait_all).
+__device__ __forceinline__ void prep_fetch_a(const PrepCtx& c, const float* a_g) {
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int idx = c.pt + kPrepThreads * m, ar = idx >> 4, c16 = idx & 15;
+    tc::cp_async_16(tc::smem_u32(c.Lf + ar * kLd + c16 * 4), a_g + ar * kChunk + c16 * 4);
+  }
+  tc::cp_async_commit();
 }
 
 // A strip's fragments (prep_solve_strip_h) -> fp32 rows of a global 64 x 64 matrix.

@@ -259,6 +259,10 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       {
         float x[4][4];
         prep_solve_strip_h(pc, x);
+        const int t0 = ws + c * kChunk;
+        if (p.states != nullptr && p.chunk_a != nullptr && t0 >= it.s && ok)   // A for the backward
+          prep_store_strip_global(pc, x, p.chunk_a + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
+                                                         (size_t)(kChunk * kChunk));
         // the previous chunk's U / W products have read A2, B2 (their completion is almost
         // always past by now)
         if (c > 0) {

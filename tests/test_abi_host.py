@@ -90,11 +90,12 @@ def test_options_struct_layout():
 
 def test_chunk_states_size():
     L = gdn.lib()
-    # independent sequences: N * ceil(T / 64) slots of Hv * dk * dv bf16
-    assert L.gdn_chunk_states_size(2, 8192, 16, 16, 128, 128, 0) == 2 * 128 * 16 * 128 * 128 * 2
-    assert L.gdn_chunk_states_size(3, 100, 2, 4, 128, 128, 0) == 3 * 2 * 4 * 128 * 128 * 2
+    per = 128 * 128 * 2 + 64 * 64 * 4      # bf16 start state and fp32 A = (I + L)^-1 per chunk slot
+    # independent sequences: N * ceil(T / 64) slots per v-head
+    assert L.gdn_chunk_states_size(2, 8192, 16, 16, 128, 128, 0) == 2 * 128 * 16 * per
+    assert L.gdn_chunk_states_size(3, 100, 2, 4, 128, 128, 0) == 3 * 2 * 4 * per
     # packed: ceil(T / 64) + N slots bound the chunks of any split of T tokens into N sequences
-    assert L.gdn_chunk_states_size(1, 65536, 16, 16, 128, 128, 24) == (1024 + 24) * 16 * 128 * 128 * 2
+    assert L.gdn_chunk_states_size(1, 65536, 16, 16, 128, 128, 24) == (1024 + 24) * 16 * per
     assert L.gdn_chunk_states_size(0, 64, 1, 1, 128, 128, 0) == 0
 
 
