@@ -63,7 +63,8 @@ struct Small {
   float dgam[kNumGamSlots][64];
   float dbeta[kNumBetaSlots][64];
   float dgn[16];
-  uint64_t tma_bar, mma_bar;
+  uint64_t tma_bar, mma_bar, gram_bar;   // gram_bar: the Gram product's own commit (its
+                                         // completion is implied by the next mma_bar phase)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -119,6 +120,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (tid == 0) {
     mbar_init(&ss->tma_bar, 1);
     mbar_init(&ss->mma_bar, 1);
+    mbar_init(&ss->gram_bar, 1);
     ss->abort_flag = 0;
     fence_mbar_init();
   }
@@ -238,15 +240,12 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_after();
   };
   // ---- prep: G, gam, masks (scale * P), inverse, A2 and A
-  if (tid == 0 && ok) issue_gram(tmem + kColG, sbase + kOffKQ, &ss->mma_bar);
+  if (tid == 0 && ok) issue_gram(tmem + kColG, sbase + kOffKQ, &ss->gram_bar);
   prep_scan(pc, 0);
   __syncthreads();
   prep_decays(pc, 0, nv);
-  // products that need only the loaded tiles: S K^T, S Q^T, dS' K^T, dO^T (scale P) comes later
-  ok = ok && mbar_wait(&ss->mma_bar, mph, abort_flag);
-  ok = __syncthreads_and(ok);
-  mph ^= 1;
-  tc_fence_after();
+  // products that need only the loaded tiles: S K^T, S Q^T, dS' K^T, dO^T (scale P). G is
+  // first read after their commit, which also covers the Gram product issued before them.
   cp_async_wait_all();                        // A and scale * P from the reverse chain
   fence_proxy_async_smem();                   // scale * P is an operand of the next products
   __syncthreads();
@@ -688,8 +687,9 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
     }
   }
-  __syncthreads();
-  if (warp == 0) {
+  // warp 2 (no dq / dk rows above) turns the per-token slots into dg, dbeta while the
+  // others store dq, dk; every slot was written before the last product's barrier
+  if (warp == 2) {
     // dgam_{63} += dgn; dg = reverse cumsum of dgam over the chunk (two values per lane)
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
