@@ -137,6 +137,8 @@ long long state_slots(const Shape& s) {
 }
 size_t cache_states_bytes(const Shape& s) { return (size_t)state_slots(s) * s.Hv * s.dk * s.dv * 2; }
 size_t cache_a_bytes(const Shape& s) { return (size_t)state_slots(s) * s.Hv * kChunk * kChunk * sizeof(float); }
+// then the bf16 P = lower_incl(Q K^T * E) tile of every chunk slot (8 KB, swizzled as the operand)
+size_t cache_p_bytes(const Shape& s) { return (size_t)state_slots(s) * s.Hv * kChunk * kChunk * 2; }
 
 struct BwdPlan {
   FwdPlan chain;                 // gate-driven segments (or none) for the two sequential passes
@@ -161,9 +163,10 @@ BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
   if (!(opt && opt->states)) {                  // states and A are in the caller's cache otherwise
     b.off_states = off; off = align256(off + st);
     b.off_a = off; off = align256(off + (size_t)b.total_chunks * s.Hv * kChunk * kChunk * sizeof(float));
+    b.off_p = off; off = align256(off + (size_t)b.total_chunks * s.Hv * kChunk * kChunk * 2);
   }
   b.off_dstates = off; off = align256(off + st);
-  b.off_p = off; off = align256(off + (size_t)b.total_chunks * s.Hv * kChunk * kChunk * 2);
+
   if (b.grouped) {
     const size_t part = (size_t)s.B * s.T * s.Hv * s.dk * sizeof(float);
     b.off_dq = off; off = align256(off + part);
@@ -308,7 +311,10 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
     // the launch that produces o also writes the chunk start states, when asked
     FwdParams pf = p;
     pf.states = static_cast<__nv_bfloat16*>(save_states);
-    if (save_states) pf.chunk_a = reinterpret_cast<float*>(static_cast<uint8_t*>(save_states) + cache_states_bytes(s));
+    if (save_states) {
+      pf.chunk_a = reinterpret_cast<float*>(static_cast<uint8_t*>(save_states) + cache_states_bytes(s));
+      pf.chunk_p = static_cast<uint8_t*>(save_states) + cache_states_bytes(s) + cache_a_bytes(s);
+    }
     int* chunk_off = nullptr;
     if (save_states && s.packed) {           // packed: per-sequence first slot, from cu_seqlens
       chunk_off = reinterpret_cast<int*>(ws + f.off_chunk_off);
@@ -363,7 +369,7 @@ size_t gdn_chunk_states_size(int B, int T, int Hqk, int Hv, int dk, int dv, int 
   Shape s;
   const bool packed = num_seqs > 0 && B == 1;
   if (check_shape(B, T, Hqk, Hv, dk, dv, packed ? num_seqs : 0, packed, s) != GDN_OK) return 0;
-  return cache_states_bytes(s) + cache_a_bytes(s);
+  return cache_states_bytes(s) + cache_a_bytes(s) + cache_p_bytes(s);
 }
 
 size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs,
@@ -410,8 +416,9 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
                     : reinterpret_cast<__nv_bfloat16*>(ws + bp.off_states);
   p.chunk_off = s.packed ? reinterpret_cast<int*>(ws + bp.off_chunk_off) : nullptr;
   // per-chunk A, written by the forward pass with the states, read by the chain and the gradients
-  p.chunk_a = cached ? reinterpret_cast<float*>(static_cast<uint8_t*>(const_cast<void*>(cached)) + cache_states_bytes(s))
-                     : reinterpret_cast<float*>(ws + bp.off_a);
+  uint8_t* cache = static_cast<uint8_t*>(const_cast<void*>(cached));
+  p.chunk_a = cached ? reinterpret_cast<float*>(cache + cache_states_bytes(s)) : reinterpret_cast<float*>(ws + bp.off_a);
+  p.chunk_p = cached ? cache + cache_states_bytes(s) + cache_a_bytes(s) : ws + bp.off_p;
   __nv_bfloat16* dstates = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_dstates);
 
   const FwdPlan& f = bp.chain;
@@ -451,7 +458,7 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   pc.hT = dh0;
   pc.states = dstates;
 
-  pc.chunk_p = ws + bp.off_p;
+
   err = launch_bwd_chain(pc, plan, items, stream, &what);
   if (err != cudaSuccess) return cuda_fail(what, err);
   // 3) per-chunk gradients
@@ -459,7 +466,7 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   out.dq = dq; out.dk = dk_out; out.dv = dv_out; out.dg = dg; out.dbeta = dbeta; out.dO = dO;
   out.dstates = dstates;
   out.chunk_a = p.chunk_a;
-  out.chunk_p = ws + bp.off_p;
+  out.chunk_p = p.chunk_p;
   out.qk_partial = bp.grouped ? 1 : 0;
   out.dq_part = bp.grouped ? reinterpret_cast<float*>(ws + bp.off_dq) : nullptr;
   out.dk_part = bp.grouped ? reinterpret_cast<float*>(ws + bp.off_dk) : nullptr;

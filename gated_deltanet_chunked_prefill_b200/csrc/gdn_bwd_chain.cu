@@ -41,7 +41,7 @@ constexpr int kBarPrep = 1, kBarEpi = 2;
 constexpr uint32_t kStageBytes = 48u * 1024u;   // [K0 Q0 K1 Q1] + [dO0 dO1]
 constexpr uint32_t kOffDO = 32u * 1024u;        // within a stage
 constexpr uint32_t kOffA2 = 96u * 1024u;        // 2 x 8KB
-constexpr uint32_t kOffP = 112u * 1024u;        // 2 x 8KB  scale * P
+constexpr uint32_t kOffP = 112u * 1024u;        // 2 x 8KB  P (from the forward pass)
 constexpr uint32_t kOffSb = 128u * 1024u;       // 32KB  dS in bf16
 constexpr uint32_t kOffDD = 160u * 1024u;       // 16KB  dDelta^T, bf16 [r][j]
 constexpr uint32_t kOffDY = 176u * 1024u;       // 16KB  -dY^T diag(exp(gam)), bf16 [r][j]
@@ -61,7 +61,7 @@ static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a bl
 
 constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T
 constexpr uint32_t kColDa = 64;   // 64: dS' K^T
-constexpr uint32_t kColDb = 128;  // 64: dO^T (scale P)
+constexpr uint32_t kColDb = 128;  // 64: dO^T P (scale applied when combined)
 constexpr uint32_t kColDY = 192;  // 64: dDelta^T A2
 constexpr uint32_t kColS = 256;   // 128: dS (dv x dk) fp32, updated in place
 constexpr uint32_t kTmemCols = 512;
@@ -178,7 +178,17 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       ok = ok && mbar_wait(&ss->full[s], (k >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
-      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
+      // P = lower_incl(Q K^T * E) of this chunk from the forward pass (bf16 operand tile); its
+      // slot was last read by chunk k - 2's first product, complete once these tiles landed
+      {
+        const uint8_t* pg = p.chunk_p + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) * (size_t)8192;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const int idx = pt + kNumPrep * m;
+          tc::cp_async_16(sbase + kOffP + s * 8192u + idx * 16u, pg + idx * 16);
+        }
+        tc::cp_async_commit();
+      }
       prep_store_gb(pc, s, gv, bv);
       if (nv < kChunk) {
         for (int idx = pt; idx < (kChunk - nv) * 48; idx += kNumPrep) {
@@ -189,21 +199,10 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         fence_proxy_async_smem();
       }
       named_bar_sync(kBarPrep, kNumPrep);
-      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColG, sbase + s * kStageBytes, &ss->gdone);
       prep_scan(pc, s);
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays(pc, s, nv);
-      ok = ok && mbar_wait(&ss->gdone, k & 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-      prep_masks<false>(pc, s, sbase + kOffP + s * 8192u, p.scale, ok);   // scale * P
-      if (p.chunk_p != nullptr && t0 < it.e && ok) {      // the gradient kernel's copy of scale * P
-        uint4* dst = reinterpret_cast<uint4*>(p.chunk_p + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
-                                                              (size_t)8192);
-        const uint4* src = reinterpret_cast<const uint4*>(sm + kOffP + s * 8192u);
-#pragma unroll
-        for (int m = 0; m < 2; ++m) dst[pt + kNumPrep * m] = src[pt + kNumPrep * m];
-      }
+      named_bar_sync(kBarPrep, kNumPrep);
       scale_rows_tile_part(st + 8192, 16384, ss->cs.eg[s], p.scale, pt, kNumPrep);   // Q <- scale diag(exp(gam)) Q
       tc::cp_async_wait_all();
       named_bar_sync(kBarPrep, kNumPrep);
@@ -246,7 +245,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc_fence_before();
     named_bar_sync(kBarEpi, kNumEpi);
     uint32_t mph = 0;
-    // (1) Da = dS' K^T ;  Db = dO^T (scale P)
+    // (1) Da = dS' K^T ;  Db = dO^T P
     auto issue_1 = [&](int k) {
       tc_fence_after();
       const uint32_t a0 = sbase + kOffSb, st = sbase + (k & 1) * kStageBytes;
@@ -319,7 +318,8 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int j0 = hh * 32 + 2 * u;
-          w[u] = pack_bf16(fmaf(da[2 * u], egd[j0], db[2 * u]), fmaf(da[2 * u + 1], egd[j0 + 1], db[2 * u + 1]));
+          w[u] = pack_bf16(fmaf(da[2 * u], egd[j0], p.scale * db[2 * u]),
+                           fmaf(da[2 * u + 1], egd[j0 + 1], p.scale * db[2 * u + 1]));
         }
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)

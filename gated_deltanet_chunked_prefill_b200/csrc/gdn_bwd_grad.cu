@@ -47,7 +47,7 @@ constexpr uint32_t kOffDS = 96u * 1024;   // dS'
 constexpr uint32_t kOffYt = 128u * 1024;  // Y^T [r][j]; then -e^gam dY^T
 constexpr uint32_t kOffDt = 144u * 1024;  // Delta^T [r][j]; then e^(gam_n - gam) Delta^T
 constexpr uint32_t kOffA2 = 160u * 1024;  // A diag(beta)
-constexpr uint32_t kOffP = 168u * 1024;   // scale P; then dPm
+constexpr uint32_t kOffP = 168u * 1024;   // P (from the forward pass); then dPm
 constexpr uint32_t kOffA = 176u * 1024;   // A; then dG + dG^T
 constexpr uint32_t kOffDA = 184u * 1024;  // dA; then X = dA A^T
 constexpr uint32_t kOffLf = 192u * 1024;  // fp32 64 x kLd: L -> A; then dG
@@ -77,7 +77,7 @@ constexpr uint32_t kColY = 64;    // S K^T (64)
 constexpr uint32_t kColD = 128;   // Delta^T (64); later [dDelta;dO][Y^T|Delta^T] (128): dA2 | dP
 constexpr uint32_t kColSQ = 192;  // S Q^T (64)
 constexpr uint32_t kColDa = 256;  // dS' K^T (64); later X (64)
-constexpr uint32_t kColDb = 320;  // dO^T scale P (64); later dY^T (64); later dL (64)
+constexpr uint32_t kColDb = 320;  // dO^T P (64); later dY^T (64); later dL (64)
 constexpr uint32_t kColQ = 384;   // dQ (128)
 constexpr uint32_t kColK = 128;   // dK (128), after dA2/dP are consumed
 constexpr uint32_t kTmemCols = 512;
@@ -197,7 +197,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_load_3d(sm + kOffDS + 16384, &tm_ds, &ss->tma_bar, 64, 0, srow);
   }
   PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColG, tid, warp, lane, kBar};
-  // A = (I + L)^-1 of this chunk, as the reverse chain computed it: fp32 rows into the scratch
+  // A = (I + L)^-1 of this chunk, as the forward pass computed it: fp32 rows into the scratch
   {
     const float* ag = out.chunk_a + (size_t)srow / 128 * (kChunk * kChunk);
 #pragma unroll
@@ -205,7 +205,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int idx = tid + kThreads * m, ar = idx >> 4, c16 = idx & 15;
       cp_async_16(sbase + kOffLf + (uint32_t)(ar * kLd + c16 * 4) * 4u, ag + ar * kChunk + c16 * 4);
     }
-    // and scale * P (the swizzled bf16 tile, byte for byte)
+    // and P (the swizzled bf16 tile, byte for byte)
     const uint8_t* pg = out.chunk_p + (size_t)srow / 128 * 8192;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
@@ -239,14 +239,14 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mph ^= 1;
     tc_fence_after();
   };
-  // ---- prep: G, gam, masks (scale * P), inverse, A2 and A
+  // ---- prep: G, gam; A and P come from the forward pass
   if (tid == 0 && ok) issue_gram(tmem + kColG, sbase + kOffKQ, &ss->gram_bar);
   prep_scan(pc, 0);
   __syncthreads();
   prep_decays(pc, 0, nv);
-  // products that need only the loaded tiles: S K^T, S Q^T, dS' K^T, dO^T (scale P). G is
+  // products that need only the loaded tiles: S K^T, S Q^T, dS' K^T, dO^T P. G is
   // first read after their commit, which also covers the Gram product issued before them.
-  cp_async_wait_all();                        // A and scale * P from the reverse chain
+  cp_async_wait_all();                        // A and P from the forward pass
   fence_proxy_async_smem();                   // scale * P is an operand of the next products
   __syncthreads();
   if (tid == 0 && ok) {
@@ -266,7 +266,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       umma_f16(tmem + kColDb, mdesc(sbase + kOffVDO + 8192 + ks * 2048, 16384), mdesc(sbase + kOffP + ks * 2048, 8192),
                idmm, ks > 0);
   }
-  // A (fp32 rows, from the reverse chain) -> A diag(beta) and A in bf16
+  // A (fp32 rows, from the forward pass) -> A diag(beta) and A in bf16
   prep_write_a_rows(pc, 0, sbase + kOffA2, sbase + kOffA);
   fence_proxy_async_smem();
   commit_wait();
@@ -291,7 +291,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int jj = hh * 32 + u;
       const float vv = bf16_at(vt + jj * 128 + ((rc ^ (jj & 7)) << 4) + rb);
       yv[u] = vv - eg[jj] * sk[u];
-      ddv[u] = fmaf(da[u], egd[jj], db[u]);
+      ddv[u] = fmaf(da[u], egd[jj], p.scale * db[u]);      // P is unscaled
     }
   }
   __syncthreads();                            // every V read is done: dD may overwrite V

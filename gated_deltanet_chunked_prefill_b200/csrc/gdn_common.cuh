@@ -37,10 +37,11 @@ struct FwdParams {
   __nv_bfloat16* states;    // nullable
   const int* chunk_off;     // nullable
   // backward support: A = (I + L)^-1 (fp32, 64 x 64 row-major) of every chunk, written by the
-  // reverse chain at chunk_a + (slot * Hv + j) * 4096 (slot as for states); nullable
+  // forward pass (state-store mode) at chunk_a + (slot * Hv + j) * 4096 (slot as for states); nullable
   float* chunk_a;
-  // backward support: scale * P (bf16, the 8 KB 128B-swizzled tile of the tensor-core
-  // operand) of every chunk, at chunk_p + (slot * Hv + j) * 8192 bytes; nullable
+  // backward support: P = lower_incl(Q K^T * E) (bf16, the 8 KB 128B-swizzled tile of the
+  // tensor-core operand) of every chunk, written by the forward pass, at
+  // chunk_p + (slot * Hv + j) * 8192 bytes; nullable
   uint8_t* chunk_p;
   int B, T, Hqk, Hv, dk, dv, N;
   float scale;

@@ -251,6 +251,13 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_after();
       pc.colG = gw_col;
       prep_masks(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
+      if (p.states != nullptr && p.chunk_p != nullptr && ws + c * kChunk >= it.s && ok) {   // P for the backward
+        uint4* dst = reinterpret_cast<uint4*>(
+            p.chunk_p + (chunk_slot(p, it.n, (ws + c * kChunk - it.seq_s) / kChunk) * p.Hv + it.j) * (size_t)8192);
+        const uint4* src = reinterpret_cast<const uint4*>(sm + kOffP + s * 8192u);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) dst[pt + kNumPrep * m] = src[pt + kNumPrep * m];
+      }
       // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- diag(exp(gam)) Q
       // in place (the Gram product has consumed Q); then one column strip of A per warp
       if (warp < 4) prep_diag_inverse_h(pc);

@@ -22,8 +22,8 @@ struct BwdOut {
   void* dbeta;               // [B,T,Hv] bf16
   const void* dO;            // [B,T,Hv,dv] bf16
   const __nv_bfloat16* dstates;   // per-chunk dS' (bf16, dv x dk)
-  const float* chunk_a;           // per-chunk A = (I + L)^-1 (fp32, 64 x 64), from the reverse chain
-  const uint8_t* chunk_p;         // per-chunk scale * P (bf16 swizzled 8 KB tile), from the reverse chain
+  const float* chunk_a;           // per-chunk A = (I + L)^-1 (fp32, 64 x 64), from the forward pass
+  const uint8_t* chunk_p;         // per-chunk P (bf16 swizzled 8 KB tile), from the forward pass
   int qk_partial;            // grouped values: dq/dk go through fp32 per-v-head partials
   float* dq_part;            // [B,T,Hv,dk] fp32
   float* dk_part;            // [B,T,Hv,dk] fp32

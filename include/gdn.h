@@ -93,7 +93,8 @@ typedef struct {
    *     state at the chunk's first token in bf16, transposed: states[slot][j][r][d] =
    *     h[d][r] (r < dv, d < dk), slot = n * ceil(T/64) + c for independent sequences,
    *     or (sum over m < n of ceil(len_m / 64)) + c for packed ones; after all slots, the
-   *     chunk's A = (I + L)^-1 (fp32, 64 x 64 row-major) in the same slot order.
+   *     chunk's A = (I + L)^-1 (fp32, 64 x 64 row-major), then its P = lower_incl(Q K^T * E)
+   *     (bf16, 64 x 64, 128-byte-swizzled rows), both in the same slot order.
    *   gdn_chunk_bwd reads them instead of running its forward pass; they must come
    *     from gdn_chunk_fwd on the same q, k, v, g, beta, h0 and cu_seqlens.
    * Set on another path: GDN_ERR_UNSUPPORTED; not 16-byte aligned: GDN_ERR_INVALID_ARG. */

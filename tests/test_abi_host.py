@@ -90,7 +90,7 @@ def test_options_struct_layout():
 
 def test_chunk_states_size():
     L = gdn.lib()
-    per = 128 * 128 * 2 + 64 * 64 * 4      # bf16 start state and fp32 A = (I + L)^-1 per chunk slot
+    per = 128 * 128 * 2 + 64 * 64 * 4 + 64 * 64 * 2   # bf16 start state, fp32 A, bf16 P per chunk slot
     # independent sequences: N * ceil(T / 64) slots per v-head
     assert L.gdn_chunk_states_size(2, 8192, 16, 16, 128, 128, 0) == 2 * 128 * 16 * per
     assert L.gdn_chunk_states_size(3, 100, 2, 4, 128, 128, 0) == 3 * 2 * 4 * per
