@@ -89,7 +89,8 @@ constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);     // B MN-major
 
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p, const TcPlan plan) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
+                  const FwdParams p, const TcPlan plan) {
   // Dynamic shared memory starts at the (1024-aligned) base of the CTA's window: the
   // kernel has no static shared variables. Used directly so every access stays a
   // shared-space access.
@@ -231,6 +232,8 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       named_bar_sync(kBarPrep, kNumPrep);
       if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
       prep_scan(pc, s);
+      // the bulk copies of earlier P tiles have read their slots (this chunk's masks rewrite one)
+      if (pt == 0 && p.chunk_p != nullptr) bulk_wait_read();
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays(pc, s, nv);
     };
@@ -251,13 +254,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_after();
       pc.colG = gw_col;
       prep_masks(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
-      if (p.states != nullptr && p.chunk_p != nullptr && ws + c * kChunk >= it.s && ok) {   // P for the backward
-        uint4* dst = reinterpret_cast<uint4*>(
-            p.chunk_p + (chunk_slot(p, it.n, (ws + c * kChunk - it.seq_s) / kChunk) * p.Hv + it.j) * (size_t)8192);
-        const uint4* src = reinterpret_cast<const uint4*>(sm + kOffP + s * 8192u);
-#pragma unroll
-        for (int m = 0; m < 2; ++m) dst[pt + kNumPrep * m] = src[pt + kNumPrep * m];
-      }
       // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- diag(exp(gam)) Q
       // in place (the Gram product has consumed Q); then one column strip of A per warp
       if (warp < 4) prep_diag_inverse_h(pc);
@@ -280,6 +276,13 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
+      if (pt == 0 && p.states != nullptr && p.chunk_p != nullptr && ws + c * kChunk >= it.s && ok) {
+        // P for the backward: one bulk copy of the operand tile (fenced above); its reads are
+        // waited for before the tile's slot is rewritten two chunks later
+        bulk_store(p.chunk_p + (chunk_slot(p, it.n, (ws + c * kChunk - it.seq_s) / kChunk) * p.Hv + it.j) * (size_t)8192,
+                   sbase + kOffP + s * 8192u, 8192u);
+        bulk_commit();
+      }
       // the Delta accumulator is free once the chain has read chunk c - 1's
       if (c > 0) {
         ok = ok && mbar_wait(&ss->dd_free, (c - 1) & 1, abort_flag);
@@ -314,6 +317,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // the next chunk's start (its Gram product goes to the other G/W buffer)
       if (c + 1 < nchunks) chunk_start(c + 1, gv1, bv1);
     }
+    if (pt == 0 && p.chunk_p != nullptr) bulk_wait_all();
   } else {
     // ------------------------------------------------------------ epilogue: the state chain
     const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..255
@@ -444,13 +448,13 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         load_qv(c + 2);
         loaded_qv = c + 3;
       }
-      if (p.states != nullptr && t0 >= it.s && ok) {
-        // backward support: this chunk's start state (the bf16 copy its products use)
-        const uint8_t* srow = sm + kOffSb + hh * 16384u;
-        uint4* dst = reinterpret_cast<uint4*>(p.states + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
-                                                             (size_t)(128 * 128) + (size_t)r * 128 + hh * 64);
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) dst[ch] = *reinterpret_cast<const uint4*>(srow + sw128(r, ch));
+      if (et == 0 && p.states != nullptr && t0 >= it.s && ok) {
+        // backward support: this chunk's start state (the bf16 copy its products use), two TMA
+        // tile stores from the swizzled copy; waited for (reads) before the copy is rewritten
+        const int srow = (int)((chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) * 128);
+        tma_store_3d(&tm_s, sbase + kOffSb, 0, 0, srow);
+        tma_store_3d(&tm_s, sbase + kOffSb + 16384u, 64, 0, srow);
+        bulk_commit();
       }
       // (b) Delta^T and Delta~^T = Delta^T diag(exp(gam_n - gam)) -> bf16
       {
@@ -474,6 +478,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           st_shared_v4(sbase + kOffDt + sw128(r, hh * 4 + c4), x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
         }
       }
+      if (et == 0 && p.states != nullptr) bulk_wait_read();   // Sb is rewritten after this barrier
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
@@ -568,6 +573,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int d = 0; d < 32; ++d) it.fin[(size_t)(hh * 64 + h2 * 32 + d) * 128 + r] = v[d];
       }
     }
+    if (et == 0 && p.states != nullptr) bulk_wait_all();
     if (et == 0 && !ok) {
       // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
       volatile int never = 0;
@@ -601,13 +607,20 @@ cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items,
   if (!make_tile_map(&mq, p.q, p.Hqk, rows) || !make_tile_map(&mk, p.k, p.Hqk, rows) ||
       !make_tile_map(&mv, p.v, p.Hv, rows))
     return cudaErrorInvalidValue;
+  // chunk start states (bf16 [slots * Hv * 128 rows][128]): 128-row x 64-column boxes
+  CUtensorMap ms = mq;                       // unused unless states are stored
+  if (p.states != nullptr) {
+    const long long nch = (p.T + kChunk - 1) / kChunk;
+    const long long slots = p.cu != nullptr ? nch + p.N : (long long)p.N * nch;
+    if (!make_tile_map(&ms, p.states, 1, slots * p.Hv * 128, 128)) return cudaErrorInvalidValue;
+  }
   *what = "shared memory attribute";
   cudaError_t err = cudaFuncSetAttribute(gdn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
   if (err != cudaSuccess) return err;
   *what = "tensor-core forward launch";
   trace_pre(kKernFwdTc, st);
-  gdn_fwd_tc_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, p, plan);
+  gdn_fwd_tc_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, ms, p, plan);
   err = cudaGetLastError();
   trace_post(st);
   return err;
