@@ -76,7 +76,8 @@ constexpr uint32_t kId128km = idesc_bf16(128, 128, false, true);
 
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_do, const FwdParams p, const TcPlan plan) {
+                     const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_s,
+                     const FwdParams p, const TcPlan plan) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw;
   Small* ss = reinterpret_cast<Small*>(sm + kOffSmall);
@@ -295,13 +296,13 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int c = chunk_of(k);
       const int t0 = it.s + c * kChunk;
       wait_mma();
-      if (t0 < it.e && ok) {
-        // dS' of this chunk (its end gradient) for the gradient kernel
-        const uint8_t* srow = sm + kOffSb + hh * 16384u;
-        uint4* dst = reinterpret_cast<uint4*>(p.states + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
-                                                             (size_t)(128 * 128) + (size_t)r * 128 + hh * 64);
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) dst[ch] = *reinterpret_cast<const uint4*>(srow + sw128(r, ch));
+      if (et == 0 && t0 < it.e && ok) {
+        // dS' of this chunk (its end gradient) for the gradient kernel: two TMA tile stores
+        // from the swizzled bf16 copy, waited for (reads) before the copy is rewritten
+        const int srow = (int)((chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) * 128);
+        tma_store_3d(&tm_s, sbase + kOffSb, 0, 0, srow);
+        tma_store_3d(&tm_s, sbase + kOffSb + 16384u, 64, 0, srow);
+        bulk_commit();
       }
       // dDelta^T = Da diag(exp(gam_n - gam)) + Db  -> bf16
       {
@@ -358,6 +359,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int c4 = 0; c4 < 4; ++c4)
           st_shared_v4(sbase + kOffDY + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
       }
+      if (et == 0) bulk_wait_read();                // the dS' copy is rewritten after this barrier
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
@@ -414,6 +416,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int d = 0; d < 32; ++d) dh0[(size_t)(hh * 64 + h2 * 32 + d) * 128 + r] = v[d];
       }
     }
+    if (et == 0) bulk_wait_all();
     if (et == 0 && !ok) {
       for (int k = (loaded >= 2 ? loaded - 2 : 0); k < loaded; ++k) {
         volatile int never = 0;
@@ -440,13 +443,20 @@ cudaError_t launch_bwd_chain(const FwdParams& p, const TcPlan& plan, int num_ite
   if (!make_tile_map(&mq, p.q, p.Hqk, rows) || !make_tile_map(&mk, p.k, p.Hqk, rows) ||
       !make_tile_map(&mdo, p.v, p.Hv, rows))
     return cudaErrorInvalidValue;
+  // per-chunk dS' (bf16 [slots * Hv * 128 rows][128]): 128-row x 64-column boxes
+  CUtensorMap ms;
+  {
+    const long long nch = (p.T + kChunk - 1) / kChunk;
+    const long long slots = p.cu != nullptr ? nch + p.N : (long long)p.N * nch;
+    if (!make_tile_map(&ms, p.states, 1, slots * p.Hv * 128, 128)) return cudaErrorInvalidValue;
+  }
   *what = "shared memory attribute";
   cudaError_t err = cudaFuncSetAttribute(gdn_bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
   if (err != cudaSuccess) return err;
   *what = "backward chain launch";
   trace_pre(kKernBwdChain, st);
-  gdn_bwd_chain_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mdo, p, plan);
+  gdn_bwd_chain_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mdo, ms, p, plan);
   err = cudaGetLastError();
   trace_post(st);
   return err;
