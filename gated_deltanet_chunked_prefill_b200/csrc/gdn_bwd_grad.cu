@@ -203,7 +203,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int idx = tid + kThreads * m, ar = idx >> 4, c16 = idx & 15;
-      cp_async_16(sbase + kOffLf + (uint32_t)(ar * kLd + c16 * 4) * 4u, ag + ar * kChunk + c16 * 4);
+      cp_async_16(sbase + kOffLf + (uint32_t)(ar * kLd + c16 * 4) * 4u, ag + ar * kChunk + a_chunk(ar, c16) * 4);
     }
     // and P (the swizzled bf16 tile, byte for byte)
     const uint8_t* pg = out.chunk_p + (size_t)srow / 128 * 8192;

@@ -29,6 +29,10 @@ constexpr int kLd = 68;
 constexpr int kLdh = 72;
 constexpr int kPrepThreads = 256;
 
+// Layout of a stored A (fp32 64 x 64): row i, 16-byte chunk k of the row at chunk k ^ (i % 16),
+// so that a strip's fragment writes hit distinct banks; the whole 16 KB moves as one copy.
+__device__ __forceinline__ int a_chunk(int row, int k) { return k ^ (row & 15); }
+
 // per-chunk scalars, double-buffered by chunk parity
 struct ChunkScalars {
   float gam[2][64];   // chunk-local inclusive cumsum of g
@@ -408,20 +412,23 @@ __device__ __forceinline__ void prep_fetch_a(const PrepCtx& c, const float* a_g)
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const int idx = c.pt + kPrepThreads * m, ar = idx >> 4, c16 = idx & 15;
-    tc::cp_async_16(tc::smem_u32(c.Lf + ar * kLd + c16 * 4), a_g + ar * kChunk + c16 * 4);
+    tc::cp_async_16(tc::smem_u32(c.Lf + ar * kLd + c16 * 4), a_g + ar * kChunk + a_chunk(ar, c16) * 4);
   }
   tc::cp_async_commit();
 }
 
-// A strip's fragments (prep_solve_strip_h) -> fp32 rows of a global 64 x 64 matrix.
-__device__ __forceinline__ void prep_store_strip_global(const PrepCtx& c, const float (&x)[4][4], float* a_g) {
+// A strip's fragments (prep_solve_strip_h) -> the stored-A layout at a_s (shared memory).
+__device__ __forceinline__ void prep_stage_strip_a(const PrepCtx& c, const float (&x)[4][4], float* a_s) {
   const int gid = c.lane >> 2, tig = c.lane & 3;
   const int j = 8 * c.pw + 2 * tig;
 #pragma unroll
   for (int R = 0; R < 4; ++R)
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-      *reinterpret_cast<float2*>(a_g + (16 * R + gid + 8 * h) * kChunk + j) = make_float2(x[R][2 * h], x[R][2 * h + 1]);
+    for (int h = 0; h < 2; ++h) {
+      const int i = 16 * R + gid + 8 * h;
+      *reinterpret_cast<float2*>(a_s + i * kChunk + a_chunk(i, j >> 2) * 4 + (j & 3)) =
+          make_float2(x[R][2 * h], x[R][2 * h + 1]);
+    }
 }
 
 // A2 = A diag(beta) and A -> bf16 (128B-swizzled rows at a2_addr, a_addr), and A -> fp32

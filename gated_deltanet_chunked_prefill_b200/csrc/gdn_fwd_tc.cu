@@ -54,9 +54,10 @@ constexpr uint32_t kOffB2 = 104u * 1024u;       // 8KB      A diag(beta exp(gam)
 constexpr uint32_t kOffP = 112u * 1024u;        // 2 x 8KB  masked decayed QK^T, bf16
 constexpr uint32_t kOffSb = 128u * 1024u;       // 32KB     S in bf16 (two 64-col sub-tiles)
 constexpr uint32_t kOffYt = 160u * 1024u;       // 16KB     Delta^T, bf16 [dv][token]
-constexpr uint32_t kOffDt = 176u * 1024u;       // 16KB     Delta~^T, then O staging
+constexpr uint32_t kOffDt = 176u * 1024u;       // 16KB     Delta~^T, then O staging (two swizzled 64-column halves)
 constexpr uint32_t kOffLf = 192u * 1024u;       // fp16 [64][kLdh] L, diagonal blocks inverted in place
-constexpr uint32_t kOffSmall = kOffLf + 64u * kLdh * 2u;
+constexpr uint32_t kOffAst = kOffLf + 64u * kLdh * 2u;   // 16KB  A staged for its bulk copy (state-store mode)
+constexpr uint32_t kOffSmall = kOffAst + 16384u;
 
 struct Small {
   ChunkScalars cs;
@@ -90,7 +91,7 @@ constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);     // B MN-major
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
-                  const FwdParams p, const TcPlan plan) {
+                  const __grid_constant__ CUtensorMap tm_o, const FwdParams p, const TcPlan plan) {
   // Dynamic shared memory starts at the (1024-aligned) base of the CTA's window: the
   // kernel has no static shared variables. Used directly so every access stays a
   // shared-space access.
@@ -233,7 +234,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
       prep_scan(pc, s);
       // the bulk copies of earlier P tiles have read their slots (this chunk's masks rewrite one)
-      if (pt == 0 && p.chunk_p != nullptr) bulk_wait_read();
+      if (pt == 0) bulk_wait_read();
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays(pc, s, nv);
     };
@@ -263,9 +264,8 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         float x[4][4];
         prep_solve_strip_h(pc, x);
         const int t0 = ws + c * kChunk;
-        if (p.states != nullptr && p.chunk_a != nullptr && t0 >= it.s && ok)   // A for the backward
-          prep_store_strip_global(pc, x, p.chunk_a + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
-                                                         (size_t)(kChunk * kChunk));
+        if (p.states != nullptr && p.chunk_a != nullptr && t0 >= it.s)   // A for the backward (copied below)
+          prep_stage_strip_a(pc, x, reinterpret_cast<float*>(sm + kOffAst));
         // the previous chunk's U / W products have read A2, B2 (their completion is almost
         // always past by now)
         if (c > 0) {
@@ -279,8 +279,9 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (pt == 0 && p.states != nullptr && p.chunk_p != nullptr && ws + c * kChunk >= it.s && ok) {
         // P for the backward: one bulk copy of the operand tile (fenced above); its reads are
         // waited for before the tile's slot is rewritten two chunks later
-        bulk_store(p.chunk_p + (chunk_slot(p, it.n, (ws + c * kChunk - it.seq_s) / kChunk) * p.Hv + it.j) * (size_t)8192,
-                   sbase + kOffP + s * 8192u, 8192u);
+        const size_t slot = chunk_slot(p, it.n, (ws + c * kChunk - it.seq_s) / kChunk) * p.Hv + it.j;
+        bulk_store(p.chunk_p + slot * 8192, sbase + kOffP + s * 8192u, 8192u);
+        if (p.chunk_a != nullptr) bulk_store(p.chunk_a + slot * (kChunk * kChunk), sbase + kOffAst, 16384u);
         bulk_commit();
       }
       // the Delta accumulator is free once the chain has read chunk c - 1's
@@ -317,7 +318,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // the next chunk's start (its Gram product goes to the other G/W buffer)
       if (c + 1 < nchunks) chunk_start(c + 1, gv1, bv1);
     }
-    if (pt == 0 && p.chunk_p != nullptr) bulk_wait_all();
+    if (pt == 0) bulk_wait_all();
   } else {
     // ------------------------------------------------------------ epilogue: the state chain
     const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..255
@@ -478,7 +479,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           st_shared_v4(sbase + kOffDt + sw128(r, hh * 4 + c4), x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
         }
       }
-      if (et == 0 && p.states != nullptr) bulk_wait_read();   // Sb is rewritten after this barrier
+      if (et == 0) bulk_wait_read();                // Sb is rewritten after this barrier
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
@@ -536,31 +537,53 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // prescale of S for the next chunk overlaps its first product
       const bool write_o = it.write_o && t0 >= it.s && p.o != nullptr;
       if (write_o) {
-        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sm + kOffDt);
+        // token rows, two 64-column halves, 128B-swizzled (the layout of the TMA tile store)
+        uint8_t* stg = sm + kOffDt + (r >> 6) * 8192 + (r & 7) * 2;
+        const int rc = (r & 63) >> 3;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) stg[(hh * 32 + jj) * 128 + r] = __float2bfloat16_rn(p.scale * oo[jj]);
+        for (int jj = 0; jj < 32; ++jj) {
+          const int i = hh * 32 + jj;
+          *reinterpret_cast<__nv_bfloat16*>(stg + i * 128 + ((rc ^ (i & 7)) << 4)) = __float2bfloat16_rn(p.scale * oo[jj]);
+        }
       }
+      // a full chunk's O leaves through two TMA tile stores as soon as the staging is fenced
+      // (inside store_w when a chunk follows); their reads are waited for before this
+      // iteration's last barrier, since the next chunk's step (b) rewrites the staging
+      const bool o_tma = write_o && nv == kChunk;
+      auto store_o = [&]() {
+        tma_store_3d(&tm_o, sbase + kOffDt, 0, it.j, it.b * p.T + t0);
+        tma_store_3d(&tm_o, sbase + kOffDt + 8192u, 64, it.j, it.b * p.T + t0);
+        bulk_commit();
+      };
       if (next) {
         ok = ok && mbar_wait(&ss->prep_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         store_w(c + 1);
+        if (et == 0 && ok && o_tma) store_o();
         if (et == 0 && ok) issue_a(c + 1);
       }
       if (next && ok) prescale((c + 1) & 1);
+      fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
       if (write_o && ok) {
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.o);
+        if (o_tma) {
+          if (et == 0 && !next) store_o();          // the last chunk
+        } else {                                    // rows past the end belong to other data
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.o);
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int idx = et + k4 * kNumEpi;
-          const int j = idx >> 4, ch = idx & 15;
-          if (j < nv) {
-            const uint4 val = *reinterpret_cast<const uint4*>(sm + kOffDt + j * 256 + ch * 16);
-            *reinterpret_cast<uint4*>(o + ((size_t)(it.b * p.T + t0 + j) * p.Hv + it.j) * 128 + ch * 8) = val;
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int idx = et + k4 * kNumEpi;
+            const int j = idx >> 4, ch = idx & 15;
+            if (j < nv) {
+              const uint4 val =
+                  *reinterpret_cast<const uint4*>(sm + kOffDt + (ch >> 3) * 8192 + j * 128 + (((ch & 7) ^ (j & 7)) << 4));
+              *reinterpret_cast<uint4*>(o + ((size_t)(it.b * p.T + t0 + j) * p.Hv + it.j) * 128 + ch * 8) = val;
+            }
           }
         }
       }
+      if (et == 0) bulk_wait_read();                // the next chunk's step (b) rewrites the O staging
       named_bar_sync(kBarEpi, kNumEpi);
     }
     if (ok && it.fin != nullptr) {
@@ -573,7 +596,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int d = 0; d < 32; ++d) it.fin[(size_t)(hh * 64 + h2 * 32 + d) * 128 + r] = v[d];
       }
     }
-    if (et == 0 && p.states != nullptr) bulk_wait_all();
+    if (et == 0) bulk_wait_all();
     if (et == 0 && !ok) {
       // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
       volatile int never = 0;
@@ -607,6 +630,8 @@ cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items,
   if (!make_tile_map(&mq, p.q, p.Hqk, rows) || !make_tile_map(&mk, p.k, p.Hqk, rows) ||
       !make_tile_map(&mv, p.v, p.Hv, rows))
     return cudaErrorInvalidValue;
+  CUtensorMap mo = mq;                       // o, same tiling as v (unused without o)
+  if (p.o != nullptr && !make_tile_map(&mo, p.o, p.Hv, rows)) return cudaErrorInvalidValue;
   // chunk start states (bf16 [slots * Hv * 128 rows][128]): 128-row x 64-column boxes
   CUtensorMap ms = mq;                       // unused unless states are stored
   if (p.states != nullptr) {
@@ -620,7 +645,7 @@ cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items,
   if (err != cudaSuccess) return err;
   *what = "tensor-core forward launch";
   trace_pre(kKernFwdTc, st);
-  gdn_fwd_tc_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, ms, p, plan);
+  gdn_fwd_tc_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, ms, mo, p, plan);
   err = cudaGetLastError();
   trace_post(st);
   return err;
