@@ -107,7 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_ds,
-                    const FwdParams p, const BwdOut out, const int num_items) {
+                    const __grid_constant__ CUtensorMap tm_dv, const __grid_constant__ CUtensorMap tm_dq,
+                    const __grid_constant__ CUtensorMap tm_dk, const FwdParams p, const BwdOut out,
+                    const int num_items) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw;
   Small* ss = reinterpret_cast<Small*>(sm + kOffSmall);
@@ -173,6 +175,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
   Pos pos;
   if (!decode(item, pos)) continue;           // uniform over the CTA
+  if (tid == 0) bulk_wait_read();             // the previous item's output tiles have been read
   if (__syncthreads_or(*abort_flag)) break;
   const int j = pos.j, n = pos.n, c = pos.c, b = pos.b, e0 = pos.e0;
   int row, hq, srow;
@@ -365,8 +368,18 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       st_shared_v4(sbase + kOffDt + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
     }
     // the stacked product below still reads Y^T: -e^gam dY^T goes in after it
-    // dv (token-major) from dY^T: stage through registers of this thread: dv[jj][r]
-    if (ok) {
+    // dv (token-major) from dY^T. A full chunk is staged as two 128B-swizzled 64-column halves
+    // in the A2 / P slots (their products have completed) for two TMA tile stores after the
+    // barrier below; a partial one is stored per thread (rows past the end are other data).
+    if (nv == kChunk) {
+      uint8_t* stg = sm + kOffA2 + (r >> 6) * 8192 + (r & 7) * 2;
+      const int rc = (r & 63) >> 3;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int i = hh * 32 + u;
+        *reinterpret_cast<__nv_bfloat16*>(stg + i * 128 + ((rc ^ (i & 7)) << 4)) = __float2bfloat16_rn(dy[u]);
+      }
+    } else if (ok) {
       __nv_bfloat16* dvo = static_cast<__nv_bfloat16*>(out.dv);
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
@@ -411,6 +424,11 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   tc_fence_before();
   __syncthreads();
   // ---- [dDelta; dO] [Y^T | Delta^T]: rows 0..63 x cols 0..63 = dA2, rows 64..127 x cols 64..127 = dP / scale
+  if (tid == 0 && ok && nv == kChunk) {       // dv tile stores (the staging is fenced above)
+    tma_store_3d(&tm_dv, sbase + kOffA2, 0, j, row);
+    tma_store_3d(&tm_dv, sbase + kOffA2 + 8192u, 64, j, row);
+    bulk_commit();
+  }
   if (tid == 0 && ok) {
     tc_fence_after();
     constexpr uint32_t id = idesc_bf16(128, 128, false, true);
@@ -421,6 +439,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       umma_f16(tmem + kColD, kdesc(sbase + kOffVDO + off), mdesc(sbase + kOffYt + ks * 2048, 16384), id, ks > 0);
     }
   }
+  if (tid == 0) bulk_wait_read();             // the P slot is rewritten (dPm) after this barrier
   commit_wait();
   // Y^T is free: -e^gam dY^T; Delta^T -> e^(gam_n - gam) Delta^T in place (dP has consumed it)
   {
@@ -658,7 +677,9 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   }
   commit_wait();
-  // ---- outputs: dq, dk (rows i < nv), dbeta, dg
+  // ---- outputs: dq, dk (rows i < nv), dbeta, dg. A full chunk's bf16 dq, dk leave through TMA
+  //      tile stores from staging (every operand tile is free now), otherwise per thread.
+  const bool qk_tma = !out.qk_partial && nv == kChunk;
   if (r < 64) {
     const int i = r;
 #pragma unroll
@@ -669,7 +690,14 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_ld32_sync(tmem + lane_base + col + hh * 64, v);
         tmem_ld32_sync(tmem + lane_base + col + hh * 64 + 32, v + 32);
       }
-      if (ok && i < nv) {
+      if (qk_tma) {                            // staged: Yt (dq) / Dt (dk), 128B-swizzled halves
+        uint8_t* srow = sm + (which == 0 ? kOffYt : kOffDt) + hh * 8192 + i * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(srow + ((u ^ (i & 7)) << 4)) =
+              make_uint4(pack_bf16(v[8 * u], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+                         pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+      } else if (ok && i < nv) {
         if (out.qk_partial) {                  // grouped values: fp32 per v-head, summed later
           float* dst = (which == 0 ? out.dq_part : out.dk_part) + ((size_t)(row + i) * p.Hv + j) * 128 + hh * 64;
 #pragma unroll
@@ -685,6 +713,17 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                            pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
         }
       }
+    }
+  }
+  if (qk_tma) {
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0 && ok) {
+      tma_store_3d(&tm_dq, sbase + kOffYt, 0, hq, row);
+      tma_store_3d(&tm_dq, sbase + kOffYt + 8192u, 64, hq, row);
+      tma_store_3d(&tm_dk, sbase + kOffDt, 0, hq, row);
+      tma_store_3d(&tm_dk, sbase + kOffDt + 8192u, 64, hq, row);
+      bulk_commit();
     }
   }
   // warp 2 (no dq / dk rows above) turns the per-token slots into dg, dbeta while the
@@ -733,6 +772,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   tc_fence_before();
   __syncthreads();
   }
+  if (tid == 0) bulk_wait_all();
   if (tid == 0 && *abort_flag) {
     // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
     volatile int never = 0;
@@ -776,6 +816,10 @@ cudaError_t launch_bwd_grad(const FwdParams& p, const BwdOut& out, long long tot
       !make_tile_map(&mv, p.v, p.Hv, rows) || !make_tile_map(&mdo, out.dO, p.Hv, rows) ||
       !make_state_map(&ms, p.states, total_chunks * p.Hv) || !make_state_map(&mds, out.dstates, total_chunks * p.Hv))
     return cudaErrorInvalidValue;
+  CUtensorMap mdv, mdq = mq, mdk = mq;       // dq, dk maps only for the bf16 (non-grouped) outputs
+  if (!make_tile_map(&mdv, out.dv, p.Hv, rows)) return cudaErrorInvalidValue;
+  if (!out.qk_partial && (!make_tile_map(&mdq, out.dq, p.Hqk, rows) || !make_tile_map(&mdk, out.dk, p.Hqk, rows)))
+    return cudaErrorInvalidValue;
   *what = "shared memory attribute";
   cudaError_t err = cudaFuncSetAttribute(gdn_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
@@ -791,7 +835,8 @@ cudaError_t launch_bwd_grad(const FwdParams& p, const BwdOut& out, long long tot
   const unsigned grid = (unsigned)std::min<long long>(items, std::max(sms, 1));
   *what = "backward gradient launch";
   trace_pre(kKernBwdTc, st);
-  gdn_bwd_grad_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, mdo, ms, mds, p, out, (int)items);
+  gdn_bwd_grad_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, mdo, ms, mds, mdv, mdq, mdk, p, out,
+                                                          (int)items);
   err = cudaGetLastError();
   trace_post(st);
   if (err != cudaSuccess || !out.qk_partial) return err;
