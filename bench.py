@@ -21,6 +21,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import sys
 import threading
 import time
@@ -169,14 +170,20 @@ def traffic_record(kernel_name, workload, mode):
 
 
 def sources_sha(paths):
-    """First 16 hex digits of the SHA-256 of the concatenated files (None if one is missing)."""
+    """First 16 hex digits of the SHA-256 of the concatenated files' code (None if one is missing).
+    Comments, trailing blanks and empty lines are dropped first, so that only a change of code
+    invalidates a capture."""
     h = hashlib.sha256()
     for rel in paths:
         path = os.path.join(ROOT, rel)
         if not os.path.exists(path):
             return None
-        with open(path, "rb") as fh:
-            h.update(fh.read())
+        with open(path) as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        for line in text.splitlines():
+            line = re.sub(r"//.*$", "", line).rstrip()
+            if line:
+                h.update(line.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -59,7 +59,7 @@ struct Small {
 constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a block can opt into");
 
-constexpr uint32_t kColG = 0;     // 64: [K;Q] K^T
+constexpr uint32_t kColG = 0;     // 64: unused (the Gram product of the prep runs in the forward)
 constexpr uint32_t kColDa = 64;   // 64: dS' K^T
 constexpr uint32_t kColDb = 128;  // 64: dO^T P (scale applied when combined)
 constexpr uint32_t kColDY = 192;  // 64: dDelta^T A2
