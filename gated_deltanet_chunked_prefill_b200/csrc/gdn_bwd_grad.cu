@@ -38,6 +38,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kBar = 1;
+constexpr int kLateIssuer = 64;   // lane 0 of warp 2 (TMEM lanes 64..95: no rows in the dL phase)
 
 // shared memory (bytes from the 1024-aligned base)
 constexpr uint32_t kOffKQ = 0;            // [K0 Q0 K1 Q1]
@@ -224,36 +225,35 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bv = __bfloat162float(beta[gi]);
   }
   prep_store_gb(pc, 0, gv, bv);
+  // gam and the decay factors need only g: they run while the tiles are in flight
+  __syncthreads();
+  prep_scan(pc, 0);
+  __syncthreads();
+  prep_decays(pc, 0, nv);
+  cp_async_wait_all();                        // A and P from the forward pass
   bool ok = mbar_wait(&ss->tma_bar, tph, abort_flag);
   tph ^= 1;
-  ok = __syncthreads_and(ok);
   if (nv < kChunk) {                          // rows past the sequence end: zero
+    ok = __syncthreads_and(ok);
     for (int idx = tid; idx < (kChunk - nv) * 64; idx += kThreads) {
       const int rr = nv + idx / 64, rem = idx % 64, tile = rem / 8, ch = rem % 8;
       *reinterpret_cast<uint4*>(sm + tile * 8192u + rr * 128u + ch * 16u) = make_uint4(0, 0, 0, 0);
     }
   }
-  fence_proxy_async_smem();
-  __syncthreads();
-  auto commit_wait = [&]() {
-    if (tid == 0 && ok) umma_commit(&ss->mma_bar);
+  fence_proxy_async_smem();                   // zeroed rows and P (cp.async) are operands below
+  ok = __syncthreads_and(ok);
+  auto commit_wait = [&](int issuer = 0) {
+    if (tid == issuer && ok) umma_commit(&ss->mma_bar);
     ok = ok && mbar_wait(&ss->mma_bar, mph, abort_flag);
     ok = __syncthreads_and(ok);
     mph ^= 1;
     tc_fence_after();
   };
-  // ---- prep: G, gam; A and P come from the forward pass
-  if (tid == 0 && ok) issue_gram(tmem + kColG, sbase + kOffKQ, &ss->gram_bar);
-  prep_scan(pc, 0);
-  __syncthreads();
-  prep_decays(pc, 0, nv);
-  // products that need only the loaded tiles: S K^T, S Q^T, dS' K^T, dO^T P. G is
-  // first read after their commit, which also covers the Gram product issued before them.
-  cp_async_wait_all();                        // A and P from the forward pass
-  fence_proxy_async_smem();                   // scale * P is an operand of the next products
-  __syncthreads();
+  // ---- G = [K;Q] K^T and the products that need only the loaded tiles: S K^T, S Q^T,
+  //      dS' K^T, dO^T P. G is first read after their commit, which also covers the Gram
+  //      product issued before them.
   if (tid == 0 && ok) {
-    tc_fence_after();
+    issue_gram(tmem + kColG, sbase + kOffKQ, &ss->gram_bar);
     constexpr uint32_t id64 = idesc_bf16(128, 64, false, false);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -567,20 +567,53 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4)
       st_shared_v4(sbase + kOffDA + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+  } else {
+    // dO <- scale diag(e^gam) dO in place (an operand of dQ); its other uses have completed
+    scale_rows_tile_part(sm + kOffVDO + 8192, 16384, eg, p.scale, (r - 64) + 64 * hh, 128);
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
-  // ---- dL = -A^T X  (A read MN-major: A^T[i][k] = A[k][i])
-  if (tid == 0 && ok) {
+  // ---- dL = -A^T X  (A read MN-major: A^T[i][k] = A[k][i]), then, behind it, every product of
+  //      dQ = (scale e^gam dO) S + dPm K  and  dK = dPm^T Q + (-e^gam dY) S + (e^(gam_n-gam) Delta) dS'
+  //      whose operands are ready (dK's dGs K term follows once dGs is written). They are issued by
+  //      warp 2, which has no rows in the dL phase, so that the issue and the tensor-core time
+  //      overlap that phase; only the threads of rows i < 64 wait for dL.
+  if (tid == kLateIssuer && ok) {
     tc_fence_after();
     constexpr uint32_t id = idesc_bf16(128, 64, true, true);
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks)
       umma_f16(tmem + kColDb, mdesc(sbase + kOffA + ks * 2048, 8192), mdesc(sbase + kOffDA + ks * 2048, 8192), id,
                ks > 0);
+    umma_commit(&ss->mma_bar);
+    constexpr uint32_t idkm = idesc_bf16(128, 128, false, true);   // A K-major, B MN-major
+    constexpr uint32_t idmm = idesc_bf16(128, 128, true, true);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;   // dO rows (K = r), 16 per step
+      umma_f16(tmem + kColQ, kdesc(sbase + kOffVDO + 8192 + off), mdesc(sbase + kOffS + ks * 2048, 16384), idkm,
+               ks > 0);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      umma_f16(tmem + kColQ, kdesc(sbase + kOffP + ks * 32), mdesc(sbase + kOffKQ + ks * 2048, 16384), idkm, 1);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      umma_f16(tmem + kColK, mdesc(sbase + kOffP + ks * 2048, 8192), mdesc(sbase + kOffKQ + 8192 + ks * 2048, 16384),
+               idmm, ks > 0);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      umma_f16(tmem + kColK, mdesc(sbase + kOffYt + ks * 2048, 16384), mdesc(sbase + kOffS + ks * 2048, 16384), idmm, 1);
+      umma_f16(tmem + kColK, mdesc(sbase + kOffDt + ks * 2048, 16384), mdesc(sbase + kOffDS + ks * 2048, 16384), idmm,
+               1);
+    }
   }
-  commit_wait();
+  if (r < 64) {
+    ok = ok && mbar_wait(&ss->mma_bar, mph, abort_flag);
+    tc_fence_after();
+  }
+  mph ^= 1;
   // ---- dL (rows i < 64): strictly lower part. F += dL * L, dbeta_i += sum_j dL_ij KK_ij E_ij,
   //      dG = dL beta_i E (fp32 to Lf), then dGs = dG + dG^T -> bf16 (A's slot)
   {
@@ -644,39 +677,18 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int c4 = 0; c4 < 4; ++c4)
       st_shared_v4(sbase + kOffA + sw128(i, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
   }
-  // dO <- scale diag(e^gam) dO in place (for dQ); its other uses have completed
-  scale_rows_tile(pc, sm + kOffVDO + 8192, 16384, eg, p.scale);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
-  // ---- dQ = (scale e^gam dO) S + dPm K ;  dK = dPm^T Q + dGs K + (-e^gam dY) S + (e^(gam_n-gam) Delta) dS'
-  if (tid == 0 && ok) {
+  // ---- dK += dGs K (same issuing thread as the rest of dK)
+  if (tid == kLateIssuer && ok) {
     tc_fence_after();
-    constexpr uint32_t idkm = idesc_bf16(128, 128, false, true);   // A K-major, B MN-major
-    constexpr uint32_t idmm = idesc_bf16(128, 128, true, true);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;   // dO rows (K = r), 16 per step
-      umma_f16(tmem + kColQ, kdesc(sbase + kOffVDO + 8192 + off), mdesc(sbase + kOffS + ks * 2048, 16384), idkm,
-               ks > 0);
-    }
+    constexpr uint32_t idkm = idesc_bf16(128, 128, false, true);
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks)
-      umma_f16(tmem + kColQ, kdesc(sbase + kOffP + ks * 32), mdesc(sbase + kOffKQ + ks * 2048, 16384), idkm, 1);
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      umma_f16(tmem + kColK, mdesc(sbase + kOffP + ks * 2048, 8192), mdesc(sbase + kOffKQ + 8192 + ks * 2048, 16384),
-               idmm, ks > 0);
       umma_f16(tmem + kColK, kdesc(sbase + kOffA + ks * 32), mdesc(sbase + kOffKQ + ks * 2048, 16384), idkm, 1);
-    }
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      umma_f16(tmem + kColK, mdesc(sbase + kOffYt + ks * 2048, 16384), mdesc(sbase + kOffS + ks * 2048, 16384), idmm, 1);
-      umma_f16(tmem + kColK, mdesc(sbase + kOffDt + ks * 2048, 16384), mdesc(sbase + kOffDS + ks * 2048, 16384), idmm,
-               1);
-    }
   }
-  commit_wait();
+  commit_wait(kLateIssuer);
   // ---- outputs: dq, dk (rows i < nv), dbeta, dg. A full chunk's bf16 dq, dk leave through TMA
   //      tile stores from staging (every operand tile is free now), otherwise per thread.
   const bool qk_tma = !out.qk_partial && nv == kChunk;
