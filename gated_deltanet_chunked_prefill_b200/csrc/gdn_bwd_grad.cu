@@ -74,9 +74,10 @@ static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a bl
 
 // TMEM columns
 constexpr uint32_t kColG = 0;     // [K;Q] K^T (64)
-constexpr uint32_t kColY = 64;    // S K^T (64)
-constexpr uint32_t kColD = 128;   // Delta^T (64); later [dDelta;dO][Y^T|Delta^T] (128): dA2 | dP
-constexpr uint32_t kColSQ = 192;  // S Q^T (64)
+constexpr uint32_t kColY = 64;    // S K^T (64), with S Q^T next to it: one S [K;Q]^T product
+constexpr uint32_t kColSQ = 128;  // S Q^T (64)
+constexpr uint32_t kColDt = 192;  // Delta^T (64)
+constexpr uint32_t kColD = 128;   // [dDelta;dO][Y^T|Delta^T] (128): dA2 | dP, after S Q^T and Delta^T are read
 constexpr uint32_t kColDa = 256;  // dS' K^T (64); later X (64)
 constexpr uint32_t kColDb = 320;  // dO^T P (64); later dY^T (64); later dL (64)
 constexpr uint32_t kColQ = 384;   // dQ (128)
@@ -255,11 +256,12 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (tid == 0 && ok) {
     issue_gram(tmem + kColG, sbase + kOffKQ, &ss->gram_bar);
     constexpr uint32_t id64 = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t id128 = idesc_bf16(128, 128, false, false);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
-      umma_f16(tmem + kColY, kdesc(sbase + kOffS + off), kdesc(sbase + kOffKQ + off), id64, ks > 0);
-      umma_f16(tmem + kColSQ, kdesc(sbase + kOffS + off), kdesc(sbase + kOffKQ + 8192 + off), id64, ks > 0);
+      // B = [K;Q] (K then Q, 8KB apart): N = 128 gives S K^T and S Q^T in one series
+      umma_f16(tmem + kColY, kdesc(sbase + kOffS + off), kdesc(sbase + kOffKQ + off), id128, ks > 0);
       umma_f16(tmem + kColDa, kdesc(sbase + kOffDS + off), kdesc(sbase + kOffKQ + off), id64, ks > 0);
     }
     // dO^T (scale P): A = dO MN-major (dv halves 16KB apart), B = scale P MN-major
@@ -324,7 +326,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     constexpr uint32_t idmm = idesc_bf16(128, 64, true, true);
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      umma_f16(tmem + kColD, kdesc(sbase + kOffYt + ks * 32), kdesc(sbase + kOffA2 + ks * 32), id64, ks > 0);
+      umma_f16(tmem + kColDt, kdesc(sbase + kOffYt + ks * 32), kdesc(sbase + kOffA2 + ks * 32), id64, ks > 0);
       // A[m=r][k=i] = dDelta[i][r]: token-major dD tile read MN-major (dv halves 16KB apart)
       umma_f16(tmem + kColDb, mdesc(sbase + kOffVDO + ks * 2048, 16384), mdesc(sbase + kOffA2 + ks * 2048, 8192), idmm,
                ks > 0);
@@ -336,7 +338,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   {
     float dl[32], dy[32], sk[32], sq[32], da[32];
     if (ok) {
-      tmem_ld32_sync(tmem + lane_base + kColD + hh * 32, dl);
+      tmem_ld32_sync(tmem + lane_base + kColDt + hh * 32, dl);
       tmem_ld32_sync(tmem + lane_base + kColDb + hh * 32, dy);
       tmem_ld32_sync(tmem + lane_base + kColY + hh * 32, sk);
       tmem_ld32_sync(tmem + lane_base + kColSQ + hh * 32, sq);
