@@ -15,7 +15,7 @@ import torch
 
 __all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd", "fwd_workspace_size",
            "bwd_workspace_size", "chunk_states", "read_device_status", "Options", "LIB_PATH", "KernelTrace",
-           "launch_count"]
+           "launch_count", "chunk_gated_delta_rule"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
@@ -278,3 +278,6 @@ def launch_count() -> int:
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise and return (and clear) the workspace's device status word."""
     return int(lib().gdn_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+from .autograd import chunk_gated_delta_rule  # noqa: E402  (uses the functions above)

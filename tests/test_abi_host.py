@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import gated_deltanet_chunked_prefill_b200 as gdn
 
@@ -105,3 +106,17 @@ def test_states_option_checks():
     assert _fwd(dtype=0, dk=64, dv=64, opt=o) == 2        # fp32 / CUDA-core path: unsupported
     o.states = MISALIGNED
     assert _fwd(opt=o) == 1
+
+
+def test_autograd_entry_host_checks():
+    """The autograd entry point refuses what it does not do before touching the GPU."""
+    x = torch.zeros(1, 64, 1, 128)
+    g = torch.zeros(1, 64, 1)
+    with pytest.raises(NotImplementedError):
+        gdn.chunk_gated_delta_rule(x, x, x, g, g, use_qk_l2norm_in_kernel=True)
+    with pytest.raises(ValueError):
+        gdn.chunk_gated_delta_rule(x, x, x, g, g)
+    from gated_deltanet_chunked_prefill_b200.autograd import backward_supported
+    assert backward_supported(x.to(torch.bfloat16), x)
+    assert not backward_supported(x, x)                                   # fp32
+    assert not backward_supported(torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), x)   # dk = 64
