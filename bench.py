@@ -251,13 +251,128 @@ def run_reference(args, w, x):
 
 
 # ------------------------------------------------------------------------------------- GPU arm
+# Decode step workload: a serving batch whose fp32 states (268 MB) exceed the 126 MB L2.
+DECODE = dict(N=256, Hqk=16, Hv=16, dk=128, dv=128)
+
+
+def decode_bytes(N, Hqk, Hv, dk, dv):
+    """Algorithmic bytes of one decode step (bf16 I/O): each state read and written once (fp32),
+    v, o, g, beta per v-head and q, k per q/k head once."""
+    return N * Hv * (2 * dk * dv * 4 + 2 * dv * 2 + 4 + 2) + N * Hqk * 2 * dk * 2
+
+
+def decode_oracle_sample(x, Hv, budget_s):
+    """The fp64 oracle's token form, one token of 8 sequences per repetition, for `budget_s`."""
+    from oracle import fwd_token  # the CPU baseline is the oracle as it stands
+    n_s = 8
+    t0 = time.time()
+    reps = 0
+    while reps == 0 or time.time() - t0 < budget_s:
+        fwd_token(x["q"][:n_s], x["k"][:n_s], x["v"][:n_s], x["g"][:n_s], x["beta"][:n_s], x["scale"],
+                  x["h0"][:n_s])
+        reps += 1
+    el = time.time() - t0
+    return {"value": n_s * reps / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_s} sequences x {Hv} heads, one token each, fp64 numpy oracle, {reps} reps, {el:.1f} s"}
+
+
+def run_decode(args):
+    """One step = gdn_recurrent_step over every sequence of the batch (one token each). With
+    --impl reference the oracle's token form alone is timed (rank 0)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    c = DECODE
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        x = make_inputs(c["N"], 1, c["Hqk"], c["Hv"], c["dk"], c["dv"], "bf16", 2000, h0_std=0.1)
+        cpu = decode_oracle_sample(x, c["Hv"], 5.0)
+        print(json.dumps({"impl": "reference", "metric": "GDN recurrent decode step tokens/s on 1 B200; % of HBM "
+                          "roofline", "value": cpu["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+                          "steps": 1, "warmup": 0, "higher_is_better": True, "scaling": "weak",
+                          "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": "decode step (oracle sample)", "step": "decode"},
+                          "cpu_baseline": cpu, "e2e": {"value": cpu["value"], "unit": "tokens/s",
+                                                       "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return
+    import gated_deltanet_chunked_prefill_b200 as gdn
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    N, Hqk, Hv, dk, dv = c["N"], c["Hqk"], c["Hv"], c["dk"], c["dv"]
+    x = make_inputs(N, 1, Hqk, Hv, dk, dv, "bf16", rank_seed(2000, rank), h0_std=0.1)
+    tok = {n: x[n][:, 0].contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")}
+    state = x["h0"].to(dev)
+    o = torch.empty((N, Hv, dv), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.gdn_recurrent_step(tok["q"], tok["k"], tok["v"], tok["g"], tok["beta"], state, x["scale"], o=o)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if args.single:
+        step()
+        torch.cuda.synchronize()
+        return
+    sampler = ClockSampler(local)
+    sampler.start()
+    n0 = gdn.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    tw0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    tw1 = time.time()
+    if dist:
+        dist.barrier()
+    sampler.stop()
+    launches = gdn.launch_count() - n0
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / args.steps
+    hbm, _, src = peaks()
+    nbytes = decode_bytes(N, Hqk, Hv, dk, dv)
+    gbs = nbytes / (ms_step / 1e3) / 1e9
+    # the oracle's token form on a bounded sample of the same batch (rank 0, N = 1 only)
+    cpu = decode_oracle_sample(x, Hv, min(args.cpu_budget, 5.0)) \
+        if rank == 0 and world == 1 and args.cpu_budget > 0 else None
+    if rank == 0:
+        line = {"metric": "GDN recurrent decode step tokens/s on 1 B200; % of HBM roofline",
+                "value": N * world / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"decode step: {N} sequences, Hqk={Hqk} Hv={Hv}, dk=dv={dk}, bf16 I/O, "
+                                       f"fp32 state", "step": "decode", "parallelism": "single" if world == 1
+                           else f"replicas{world}", "l2": "states (268 MB) larger than the 126 MB L2; no flush"},
+                "roofline": {"bound": "hbm", "kernel": "gdn_step_kernel", "achieved": gbs, "peak": hbm,
+                             "unit": "GB/s", "frac": gbs / hbm, "peak_source": src,
+                             "traffic": traffic_record("gdn_step_kernel", "decode", "decode"),
+                             "alg_bytes_per_launch": nbytes, "avg_launch_ms": ms_step},
+                "cpu_baseline": cpu, "gpu_launches": launches, "clocks": sampler.summary(tw0, tw1)}
+        print(json.dumps(line))
+    if dist:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--mode", default=STEP, choices=["fwd", "fwdbwd"])
+    ap.add_argument("--mode", default=STEP, choices=["fwd", "fwdbwd", "decode"],
+                    help="decode: the recurrent decode step on its own batch (a separate line)")
     ap.add_argument("--single", action="store_true",
                     help="only warm-up steps plus one step, no report (for profiler launch lists)")
     ap.add_argument("--workload", default=WORKLOAD, choices=list(CONFIGS))
@@ -266,6 +381,9 @@ def main():
     args = ap.parse_args()
 
     w = CONFIGS[args.workload]
+    if args.mode == "decode":
+        run_decode(args)
+        return
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return

@@ -15,7 +15,7 @@ import torch
 
 __all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd", "fwd_workspace_size",
            "bwd_workspace_size", "chunk_states", "read_device_status", "Options", "LIB_PATH", "KernelTrace",
-           "launch_count", "chunk_gated_delta_rule"]
+           "launch_count", "gdn_recurrent_step", "chunk_gated_delta_rule"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_fwd_noalloc.argtypes = [i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp,
                                                             vp, vp]
         L.gdn_chunk_fwd_noalloc.restype = i
+        L.gdn_recurrent_step.argtypes = [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, vp]
+        L.gdn_recurrent_step.restype = i
         L.gdn_read_device_status.argtypes = [vp, vp]
         L.gdn_read_device_status.restype = i
         L.gdn_status_string.argtypes = [i]
@@ -241,6 +243,29 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
     if st != 0:
         raise GdnError(st, "gdn_chunk_bwd")
     return dict(dq=dq, dk=dkk, dv=dvv, dg=dg, dbeta=db, dh0=dh0)
+
+
+def gdn_recurrent_step(q, k, v, g, beta, state, scale=None, o=None, stream=None):
+    """One decode step through the C ABI: q, k [N,Hqk,dk], v [N,Hv,dv], beta [N,Hv] (one dtype),
+    g [N,Hv] fp32; `state` [N,Hv,dk,dv] fp32 (e.g. a prefill's hT) is advanced in place.
+    Returns o [N,Hv,dv]."""
+    io = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, n, io)
+    _check(g, "g", torch.float32)
+    _check(state, "state", torch.float32)
+    N, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if tuple(state.shape) != (N, Hv, dk, dv):
+        raise ValueError(f"state must be [{N},{Hv},{dk},{dv}], got {tuple(state.shape)}")
+    scale = dk ** -0.5 if scale is None else float(scale)
+    if o is None:
+        o = torch.empty((N, Hv, dv), dtype=io, device=q.device)
+    st = lib().gdn_recurrent_step(_dtype_code(q), N, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                  _ptr(beta), scale, _ptr(state), _ptr(o), _stream(stream))
+    if st != 0:
+        raise GdnError(st, "gdn_recurrent_step")
+    return o
 
 
 class KernelTrace:

@@ -236,7 +236,7 @@ int gdn_trace_end(float* ms, int* kernel_ids) {
 const char* gdn_kernel_name(int kernel_id) {
   static const char* names[kKernCount] = {"gdn_fwd_tc_kernel",   "gdn_fwd_simt_kernel", "gdn_cp_stitch_kernel",
                                           "gdn_bwd_grad_kernel", "gdn_bwd_simt_kernel", "gdn_bwd_reduce_kernel",
-                                          "gdn_cp_plan_kernel",  "gdn_bwd_chain_kernel"};
+                                          "gdn_cp_plan_kernel",  "gdn_bwd_chain_kernel", "gdn_step_kernel"};
   return (kernel_id >= 0 && kernel_id < kKernCount) ? names[kernel_id] : "unknown";
 }
 

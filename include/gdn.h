@@ -153,6 +153,27 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
                          const gdn_options* opt, cudaStream_t stream);
 
 /*
+ * One recurrent (decode) step per sequence and v-head, continuing a prefill: with
+ * h = S^T the current state (for instance the hT of gdn_chunk_fwd),
+ *     h <- exp(g) h;   r = v - h^T k;   h <- h + beta k r^T;   o = scale h^T q,
+ * i.e. the recurrence above for a single token. The pages list on-device agentic
+ * inference among the scenarios ("FlashQLA resource", section 4, table of the
+ * authors' stated results); generation after a prefill runs this step.
+ *   q, k  [N, Hqk, dk] (dtype)     v, o [N, Hv, dv] (dtype)
+ *   g     [N, Hv] fp32 (raw log-decay)   beta [N, Hv] (dtype)
+ *   state [N, Hv, dk, dv] fp32, read and overwritten in place (the caller's h0/hT
+ *         layout); it must not overlap the other arrays.
+ * dk, dv in {64, 128}; dtype GDN_BF16 or GDN_F32 (fp32 arithmetic in both).
+ * N = 0 is a no-op. Null or misaligned pointers, Hv not a multiple of Hqk:
+ * GDN_ERR_INVALID_ARG; other head dims: GDN_ERR_UNSUPPORTED; launch failure:
+ * GDN_ERR_CUDA. Asynchronous on `stream`; needs no workspace.
+ */
+gdn_status gdn_recurrent_step(gdn_dtype dtype, int N, int Hqk, int Hv, int dk, int dv,
+                              const void* q, const void* k, const void* v,
+                              const float* g, const void* beta, float scale,
+                              float* state, void* o, cudaStream_t stream);
+
+/*
  * Forward without a workspace, for callers that cannot allocate device memory where
  * they run the operator (inside a framework's memory pool, or a runtime that forbids
  * allocation on its hot path). The pages have no counterpart: this is a library

@@ -120,3 +120,18 @@ def test_autograd_entry_host_checks():
     assert backward_supported(x.to(torch.bfloat16), x)
     assert not backward_supported(x, x)                                   # fp32
     assert not backward_supported(torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), x)   # dk = 64
+
+
+def test_recurrent_step_host_validation():
+    """gdn_recurrent_step rejects bad arguments on the host (no GPU call is reached)."""
+    L = gdn.lib()
+    p = ctypes.c_void_p(16)                   # never dereferenced: validation fails first
+    call = lambda dtype, N, Hqk, Hv, dk, dv, ptr: L.gdn_recurrent_step(dtype, N, Hqk, Hv, dk, dv, ptr, ptr, ptr,
+                                                                        ptr, ptr, 1.0, ptr, ptr, None)
+    assert call(7, 1, 1, 1, 128, 128, p) == 1                # unknown dtype
+    assert call(1, 1, 2, 3, 128, 128, p) == 1                # Hv not a multiple of Hqk
+    assert call(1, -1, 1, 1, 128, 128, p) == 1               # negative N
+    assert call(1, 1, 1, 1, 96, 128, p) == 2                 # unsupported head dim
+    assert call(1, 1, 1, 1, 128, 128, None) == 1             # null pointers
+    assert call(1, 1, 1, 1, 128, 128, ctypes.c_void_p(24)) == 1   # misaligned
+    assert call(1, 0, 1, 1, 128, 128, None) == 0             # N = 0: nothing to do

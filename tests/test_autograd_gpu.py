@@ -25,14 +25,15 @@ def _autograd(d, leaves, cu=None, final_state=True):
     o, hT = gdn.chunk_gated_delta_rule(leaves["q"], leaves["k"], leaves["v"], leaves["g"], leaves["beta"],
                                        scale=d["scale"], initial_state=leaves["h0"],
                                        output_final_state=final_state, cu_seqlens=cu)
-    wrt = [leaves[n] for n in INPUTS] + ([leaves["h0"]] if leaves["h0"] is not None else [])
+    with_h0 = leaves["h0"] is not None and leaves["h0"].requires_grad
+    wrt = [leaves[n] for n in INPUTS] + ([leaves["h0"]] if with_h0 else [])
     outs, grads_out = [o], [d["dO"]]
     if final_state:
         outs.append(hT)
         grads_out.append(d["dhT"])
     gr = torch.autograd.grad(outs, wrt, grads_out)
     torch.cuda.synchronize()
-    names = list(INPUTS) + (["h0"] if leaves["h0"] is not None else [])
+    names = list(INPUTS) + (["h0"] if with_h0 else [])
     return o, hT, dict(zip(names, gr))
 
 
