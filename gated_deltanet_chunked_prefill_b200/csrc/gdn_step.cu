@@ -6,9 +6,11 @@
 // With h = S^T (dk x dv, fp32) the step is the token form of the recurrence:
 //   h <- exp(g) h;   r = v - h^T k;   h <- h + beta k r^T;   o = scale h^T q.
 // It moves the state once each way (2 dk dv fp32 per v-head) and does O(dk dv) flops, so it
-// is HBM-bound: one CTA per (sequence, v-head), threads over the dv columns of h (rows of h
-// are coalesced) and kRows thread rows over dk, with the two dot products over dk reduced
-// through shared memory in a fixed order (bit-reproducible).
+// is HBM-bound. The dv columns of h are independent, so a CTA takes kCols of them for one
+// (sequence, v-head): threads over those columns (rows of h are coalesced) and kRows thread
+// rows over dk, with the two dot products over dk reduced through shared memory in a fixed
+// order (bit-reproducible). Two CTAs fit on an SM, so one's loads overlap the other's
+// reductions and stores.
 #include <cstdio>
 
 #include "gdn_common.cuh"
@@ -17,6 +19,7 @@ namespace gdn {
 namespace {
 
 constexpr int kRows = 4;   // thread rows splitting dk
+constexpr int kCols = 64;  // columns of h per CTA
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -24,20 +27,22 @@ __device__ __forceinline__ void from_f(float* p, float x) { *p = x; }
 __device__ __forceinline__ void from_f(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(DV * kRows)
+__global__ void __launch_bounds__(kCols * kRows, 2)
 gdn_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const float* __restrict__ g, const T* __restrict__ beta, float scale,
                 float* __restrict__ state, T* __restrict__ o, int Hqk, int Hv) {
   constexpr int kPer = DK / kRows;            // dk entries of one column per thread
   __shared__ float ks[DK], qs[DK];
-  __shared__ float part_k[kRows][DV], part_q[kRows][DV];
-  const int unit = blockIdx.x;                // n * Hv + j
+  constexpr int kSplit = DV / kCols;          // CTAs per (sequence, v-head)
+  __shared__ float part_k[kRows][kCols], part_q[kRows][kCols];
+  const int unit = blockIdx.x / kSplit;       // n * Hv + j
   const int j = unit % Hv, n = unit / Hv;
   const int hq = j / (Hv / Hqk);
-  const int c = threadIdx.x, w = threadIdx.y;  // column c of h (dv), row block w (dk)
-  const int tid = w * DV + c;
+  const int x = threadIdx.x, w = threadIdx.y;  // column slot x, row block w (dk)
+  const int c = (blockIdx.x % kSplit) * kCols + x;   // column of h (dv)
+  const int tid = w * kCols + x;
   const size_t qk_off = ((size_t)n * Hqk + hq) * DK;
-  for (int d = tid; d < DK; d += DV * kRows) {
+  for (int d = tid; d < DK; d += kCols * kRows) {
     ks[d] = to_f(k[qk_off + d]);
     qs[d] = to_f(q[qk_off + d]);
   }
@@ -51,13 +56,13 @@ gdn_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     hc[i] = h[(size_t)d * DV];
     acc = fmaf(hc[i], ks[d], acc);
   }
-  part_k[w][c] = acc;
+  part_k[w][x] = acc;
   __syncthreads();
   const float decay = expf(g[unit]);
   const float b = to_f(beta[unit]);
   float hk = 0.f;                             // (h^T k)_c of the old state, same order in every row
 #pragma unroll
-  for (int x = 0; x < kRows; ++x) hk += part_k[x][c];
+  for (int y = 0; y < kRows; ++y) hk += part_k[y][x];
   const float rc = to_f(v[(size_t)unit * DV + c]) - decay * hk;   // v - (exp(g) h)^T k
   const float brc = b * rc;
   float acc2 = 0.f;
@@ -68,12 +73,12 @@ gdn_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     h[(size_t)d * DV] = hn;
     acc2 = fmaf(hn, qs[d], acc2);
   }
-  part_q[w][c] = acc2;
+  part_q[w][x] = acc2;
   __syncthreads();
   if (w == 0) {
     float ov = 0.f;
 #pragma unroll
-    for (int x = 0; x < kRows; ++x) ov += part_q[x][c];
+    for (int y = 0; y < kRows; ++y) ov += part_q[y][x];
     from_f(o + (size_t)unit * DV + c, scale * ov);
   }
 }
@@ -82,7 +87,7 @@ template <typename T, int DK, int DV>
 cudaError_t launch_step(const void* q, const void* k, const void* v, const float* g, const void* beta,
                         float scale, float* state, void* o, int N, int Hqk, int Hv, cudaStream_t st) {
   trace_pre(kKernStep, st);
-  gdn_step_kernel<T, DK, DV><<<(unsigned)N * (unsigned)Hv, dim3(DV, kRows), 0, st>>>(
+  gdn_step_kernel<T, DK, DV><<<(unsigned)N * (unsigned)Hv * (DV / kCols), dim3(kCols, kRows), 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, static_cast<const T*>(beta),
       scale, state, static_cast<T*>(o), Hqk, Hv);
   const cudaError_t err = cudaGetLastError();
@@ -111,7 +116,7 @@ extern "C" gdn_status gdn_recurrent_step(gdn_dtype dtype, int N, int Hqk, int Hv
                                          cudaStream_t stream) {
   if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
   if (N < 0 || Hqk < 1 || Hv < 1 || Hv % Hqk != 0) return GDN_ERR_INVALID_ARG;
-  if ((long long)N * Hv >= (1LL << 31)) return GDN_ERR_UNSUPPORTED;
+  if ((long long)N * Hv >= (1LL << 30)) return GDN_ERR_UNSUPPORTED;   // grid: N Hv dv / 64 blocks
   if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED;
   if (N == 0) return GDN_OK;
   const void* ptrs[] = {q, k, v, g, beta, state, o};

@@ -165,8 +165,8 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
  *         layout); it must not overlap the other arrays.
  * dk, dv in {64, 128}; dtype GDN_BF16 or GDN_F32 (fp32 arithmetic in both).
  * N = 0 is a no-op. Null or misaligned pointers, Hv not a multiple of Hqk:
- * GDN_ERR_INVALID_ARG; other head dims: GDN_ERR_UNSUPPORTED; launch failure:
- * GDN_ERR_CUDA. Asynchronous on `stream`; needs no workspace.
+ * GDN_ERR_INVALID_ARG; other head dims or N * Hv >= 2^30: GDN_ERR_UNSUPPORTED;
+ * launch failure: GDN_ERR_CUDA. Asynchronous on `stream`; needs no workspace.
  */
 gdn_status gdn_recurrent_step(gdn_dtype dtype, int N, int Hqk, int Hv, int dk, int dv,
                               const void* q, const void* k, const void* v,
