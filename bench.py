@@ -207,9 +207,15 @@ def oracle_sample(w, x, mode, budget_s):
     from oracle import bwd_token, fwd_chunk  # the CPU baseline is the oracle as it stands
     hq_of = lambda j: j // (w.Hv // w.Hqk)
     units, tok, t0 = 0, 0, time.perf_counter()
-    order = [(n, j) for n in range(w.B) for j in range(w.Hv)]
+    if x["cu_seqlens"] is not None:         # packed: sequence n is tokens cu[n]..cu[n+1] of batch row 0
+        cu = x["cu_seqlens"].tolist()
+        spans = [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
+    else:
+        spans = [(n, 0, w.T) for n in range(w.B)]
+    order = [(n, j) for n in range(len(spans)) for j in range(w.Hv)]
     for n, j in order:
-        sl = lambda a, h: a[n:n + 1, :, h:h + 1]
+        bi, s0, e0 = spans[n]
+        sl = lambda a, h: a[bi:bi + 1, s0:e0, h:h + 1]
         q, k, v = sl(x["q"], hq_of(j)), sl(x["k"], hq_of(j)), sl(x["v"], j)
         g, b = sl(x["g"], j), sl(x["beta"], j)
         h0 = None if x["h0"] is None else x["h0"][n:n + 1, j:j + 1]
@@ -217,12 +223,12 @@ def oracle_sample(w, x, mode, budget_s):
         if mode == "fwdbwd":
             bwd_token(q, k, v, g, b, x["scale"], sl(x["dO"], j), h0, x["dhT"][n:n + 1, j:j + 1])
         units += 1
-        tok += w.T
+        tok += e0 - s0
         if time.perf_counter() - t0 >= budget_s:
             break
     el = time.perf_counter() - t0
     # one workload token carries all Hv heads: unit-tokens / Hv = workload tokens
-    return (tok / w.Hv) / el, el, units
+    return (tok / w.Hv) / el, el, units, tok
 
 
 def run_reference(args, w, x):
@@ -234,11 +240,11 @@ def run_reference(args, w, x):
     for _ in range(args.warmup):
         oracle_sample(w, x, args.mode, budget_s=0.0)
     for _ in range(args.steps):
-        v, el, units = oracle_sample(w, x, args.mode, budget_s=0.0)
+        v, el, units, unit_tok = oracle_sample(w, x, args.mode, budget_s=0.0)
         per_step.append(el)
-    tok = w.T / w.Hv
+    tok = unit_tok / w.Hv
     value = tok * len(per_step) / sum(per_step)
-    sample = f"one (sequence, head) unit of {w.T} tokens per step ({args.mode}), fp64 numpy oracle"
+    sample = f"one (sequence, head) unit of {unit_tok} tokens per step ({args.mode}), fp64 numpy oracle"
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": 1e3 * sum(per_step) / len(per_step), "higher_is_better": True,
@@ -387,7 +393,7 @@ def main():
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return
-        x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed, h0_std=w.h0_std,
+        x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed, h0_std=w.h0_std, lengths=w.lengths,
                         backward=True)
         run_reference(args, w, x)
         return
@@ -406,6 +412,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, rank_seed(w.seed, rank), h0_std=w.h0_std,
+                    lengths=w.lengths,
                     backward=True)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     stream = torch.cuda.current_stream(dev)
@@ -414,7 +421,7 @@ def main():
 
     ws_f = torch.zeros(gdn.fwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp),
                        dtype=torch.uint8, device=dev)
-    states = gdn.chunk_states(d["q"], d["v"]) if mode == "fwdbwd" else None
+    states = gdn.chunk_states(d["q"], d["v"], d["cu_seqlens"]) if mode == "fwdbwd" else None
     ws_b = torch.zeros(gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp,
                                               states=states), dtype=torch.uint8, device=dev)
     o = torch.empty_like(d["v"])
@@ -422,11 +429,11 @@ def main():
 
     def step(dd):
         gdn.gdn_chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["scale"], dd["h0"],
-                          cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT, states=states)
+                          dd["cu_seqlens"], cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT, states=states)
         if mode == "fwdbwd":
             return gdn.gdn_chunk_bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["dO"], dd["scale"],
-                                     dd["h0"], dd["dhT"], cp_segment_chunks=args.cp, workspace=ws_b,
-                                     states=states)
+                                     dd["h0"], dd["dhT"], dd["cu_seqlens"], cp_segment_chunks=args.cp,
+                                     workspace=ws_b, states=states)
         return None
 
     # ---- device-resident timing
@@ -473,7 +480,7 @@ def main():
     with gdn.KernelTrace(capacity=64) as trf:
         for _ in range(5):
             gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
-                              cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT, states=states)
+                              d["cu_seqlens"], cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT, states=states)
     fwd_ms = sum(t for _, t in trf.launches) / 5
     bwd_recompute_ms = None
     if mode == "fwdbwd":
@@ -484,7 +491,7 @@ def main():
         with gdn.KernelTrace(capacity=64) as trb:
             for _ in range(5):
                 gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["scale"], d["h0"],
-                                  d["dhT"], cp_segment_chunks=args.cp, workspace=ws_r)
+                                  d["dhT"], d["cu_seqlens"], cp_segment_chunks=args.cp, workspace=ws_r)
         bwd_recompute_ms = sum(t for _, t in trb.launches) / 5
         del ws_r
 
@@ -514,11 +521,11 @@ def main():
                      "frac_tensor": flops(w, fwd=True, bwd=mode == "fwdbwd") / (ms_step / 1e3) / 1e12 / tc_peak}
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
-    host_in = {k: x[k].pin_memory() for k in ("q", "k", "v", "g", "beta", "h0", "dO", "dhT")
+    host_in = {k: x[k].pin_memory() for k in ("q", "k", "v", "g", "beta", "h0", "dO", "dhT", "cu_seqlens")
                if x.get(k) is not None}
     dev_in = {k: torch.empty_like(d[k]) for k in host_in}
     dev_in["scale"] = d["scale"]
-    for k in ("h0", "dO", "dhT"):
+    for k in ("h0", "dO", "dhT", "cu_seqlens"):
         dev_in.setdefault(k, None)
     h2d = sum(t.numel() * t.element_size() for k, t in host_in.items()
               if mode == "fwdbwd" or k not in ("dO", "dhT"))
@@ -561,9 +568,9 @@ def main():
     # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and args.cpu_budget > 0:
-        v_cpu, el, units = oracle_sample(w, x, mode, args.cpu_budget)
+        v_cpu, el, units, unit_tok = oracle_sample(w, x, mode, args.cpu_budget)
         cpu = {"value": v_cpu, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"{units} (sequence, head) units x {w.T} tokens of the same workload "
+               "sample": f"{units} (sequence, head) units, {unit_tok} unit-tokens of the same workload "
                          f"({mode}), fp64 numpy oracle, {el:.1f} s"}
 
     fl = flops(w, fwd=True, bwd=mode == "fwdbwd") * world

@@ -147,7 +147,7 @@ CONFIGS = {
         seed=1002, description="long-context grouped-value GDN forward, bf16: T=32768 Hqk=16 Hv=32"),
     "varlen_bf16": Workload(
         "varlen_bf16", B=1, T=65536, Hqk=16, Hv=16, dk=128, dv=128, dtype="bf16", h0_std=0.1,
-        seed=1003, lengths=None,
+        seed=1003, lengths=_varlen_c3(),
         description="packed variable-length GDN forward, bf16: 24 seqs, 65536 tokens, H=16"),
     "bwd_bf16": Workload(
         "bwd_bf16", B=2, T=8192, Hqk=16, Hv=16, dk=128, dv=128, dtype="bf16", h0_std=0.1,
@@ -159,8 +159,5 @@ CONFIGS = {
 def config_inputs(name: str) -> dict:
     """Inputs of one named workload (full size)."""
     w = CONFIGS[name]
-    lengths = w.lengths
-    if name == "varlen_bf16":
-        lengths = _varlen_c3()
     return make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed,
-                       h0_std=w.h0_std, lengths=lengths, backward=w.backward)
+                       h0_std=w.h0_std, lengths=w.lengths, backward=w.backward)

@@ -1,0 +1,64 @@
+"""Host-side pieces of bench.py: the algorithmic FLOP and byte counts against the figures worked
+out by hand for the named workloads, the packed workload's sequence table, and the source hash
+that keeps a DRAM traffic record valid only for unchanged kernel code."""
+import os
+
+import pytest
+
+import bench
+from gated_deltanet_chunked_prefill_b200.workloads import CONFIGS
+
+# (workload, forward GFLOP, forward MB, backward GFLOP, backward MB), from the chunked-algorithm
+# convention (dense GEMMs at 2 flop/MAC, the inverse at C^3/3 MAC per chunk, every input read once
+# and every output written once), computed by hand per configuration.
+TABLE = [
+    ("dense_bf16", 47.96, 278.4, None, None),
+    ("long_gqa_bf16", 174.66, 813.7, None, None),
+    ("varlen_bf16", 191.84, 1130.4, None, None),
+    ("bwd_bf16", None, None, 98.78, 479.2),
+]
+
+
+@pytest.mark.parametrize("name,fg,fmb,bg,bmb", TABLE)
+def test_algorithmic_counts(name, fg, fmb, bg, bmb):
+    w = CONFIGS[name]
+    if fg is not None:
+        assert bench.flops(w, True, False) / 1e9 == pytest.approx(fg, abs=0.01)
+        assert bench.alg_bytes(w, True, False) / 1e6 == pytest.approx(fmb, abs=0.1)
+    if bg is not None:
+        assert bench.flops(w, False, True) / 1e9 == pytest.approx(bg, abs=0.01)
+        assert bench.alg_bytes(w, False, True) / 1e6 == pytest.approx(bmb, abs=0.1)
+
+
+def test_per_token_flops():
+    """182,955 flop per token and v-head forward, 376,832 backward (d = 128, MHA)."""
+    w = CONFIGS["dense_bf16"]
+    units = w.B * w.T * w.Hv
+    assert bench.flops(w, True, False) / units == pytest.approx(182955, abs=1)
+    assert bench.flops(w, False, True) / units == pytest.approx(376832, abs=1)
+
+
+def test_packed_workload_is_packed():
+    """The packed workload carries its 24 sequence lengths, so the bench passes cu_seqlens."""
+    w = CONFIGS["varlen_bf16"]
+    assert w.num_seqs == 24 and sum(w.lengths) == w.T == 65536 and w.B == 1
+    assert any(n % 64 for n in w.lengths)           # at least one ragged last chunk
+
+
+def test_decode_bytes():
+    """State in and out (fp32), v, o, g, beta per v-head, q, k per q/k head."""
+    assert bench.decode_bytes(1, 1, 1, 128, 128) == 2 * 128 * 128 * 4 + 2 * 128 * 2 + 6 + 2 * 128 * 2
+    assert bench.decode_bytes(256, 16, 16, 128, 128) == 541089792
+
+
+def test_source_hash_ignores_comments(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    src = tmp_path / "k.cu"
+    src.write_text("int f() { return 1; }  // one\n/* block\n comment */\n")
+    h1 = bench.sources_sha(["k.cu"])
+    src.write_text("// a new note\nint f() { return 1; }  // changed comment\n\n")
+    assert bench.sources_sha(["k.cu"]) == h1
+    src.write_text("int f() { return 2; }\n")
+    assert bench.sources_sha(["k.cu"]) != h1
+    assert bench.sources_sha(["missing.cu"]) is None
+    assert os.path.exists(src)
