@@ -142,6 +142,31 @@ def chunk_states(q, v, cu_seqlens=None):
     return torch.empty(max(nbytes // 2, 1), dtype=torch.bfloat16, device=q.device)
 
 
+def _check_shapes(q, k, v, g, beta, h0=None, cu_seqlens=None, dO=None, dhT=None, o=None, hT=None):
+    """The C ABI takes its sizes from q and v and trusts every other array to match them, so a
+    mismatch is refused here, on the host, before anything reaches the GPU (tensor shapes only)."""
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k must be [B,T,Hqk,dk] and v [B,T,Hv,dv]")
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if tuple(k.shape) != tuple(q.shape):
+        raise ValueError(f"k must have q's shape {tuple(q.shape)}, got {tuple(k.shape)}")
+    if tuple(v.shape[:2]) != (B, T):
+        raise ValueError(f"v must be [{B},{T},Hv,dv], got {tuple(v.shape)}")
+    for t, n in ((g, "g"), (beta, "beta")):
+        if tuple(t.shape) != (B, T, Hv):
+            raise ValueError(f"{n} must be [{B},{T},{Hv}], got {tuple(t.shape)}")
+    if cu_seqlens is not None and (cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1):
+        raise ValueError("cu_seqlens must be 1-D [N+1]")
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for t, n in ((h0, "h0"), (dhT, "dhT"), (hT, "hT")):
+        if t is not None and tuple(t.shape) != (N, Hv, dk, dv):
+            raise ValueError(f"{n} must be [{N},{Hv},{dk},{dv}], got {tuple(t.shape)}")
+    for t, n in ((dO, "dO"), (o, "o")):
+        if t is not None and tuple(t.shape) != tuple(v.shape):
+            raise ValueError(f"{n} must have v's shape {tuple(v.shape)}, got {tuple(t.shape)}")
+
+
 def _check(t, name, dtype=None):
     if t is None:
         return
@@ -166,6 +191,7 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
                   o=None, hT=None, stream=None, states=None):
     """Forward through the C ABI. Returns (o, hT or None). With `states` (from
     chunk_states()) it also writes every chunk's start state for a later backward."""
+    _check_shapes(q, k, v, g, beta, h0, cu_seqlens, o=o, hT=hT)
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
         _check(t, n, io)
@@ -192,6 +218,7 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
 def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
                           output_final_state=True, cp_segment_chunks=0, o=None, hT=None, stream=None):
     """Forward through the allocation-free entry point (library-held 1 MiB scratch; see gdn.h)."""
+    _check_shapes(q, k, v, g, beta, h0, cu_seqlens, o=o, hT=hT)
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
         _check(t, n, io)
@@ -218,6 +245,7 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
                   states=None):
     """Backward through the C ABI. Returns dict dq, dk, dv, dg, dbeta, dh0. With `states`
     written by the matching gdn_chunk_fwd call, the forward pass is not recomputed."""
+    _check_shapes(q, k, v, g, beta, h0, cu_seqlens, dO=dO, dhT=dhT)
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta"), (dO, "dO")):
         _check(t, n, io)
@@ -249,15 +277,25 @@ def gdn_recurrent_step(q, k, v, g, beta, state, scale=None, o=None, stream=None)
     """One decode step through the C ABI: q, k [N,Hqk,dk], v [N,Hv,dv], beta [N,Hv] (one dtype),
     g [N,Hv] fp32; `state` [N,Hv,dk,dv] fp32 (e.g. a prefill's hT) is advanced in place.
     Returns o [N,Hv,dv]."""
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k must be [N,Hqk,dk] and v [N,Hv,dv]")
+    N, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if tuple(k.shape) != tuple(q.shape) or v.shape[0] != N:
+        raise ValueError(f"k must have q's shape {tuple(q.shape)} and v must be [{N},Hv,dv]")
+    for t, n in ((g, "g"), (beta, "beta")):
+        if tuple(t.shape) != (N, Hv):
+            raise ValueError(f"{n} must be [{N},{Hv}], got {tuple(t.shape)}")
+    if tuple(state.shape) != (N, Hv, dk, dv):
+        raise ValueError(f"state must be [{N},{Hv},{dk},{dv}], got {tuple(state.shape)}")
+    if o is not None and tuple(o.shape) != (N, Hv, dv):
+        raise ValueError(f"o must be [{N},{Hv},{dv}], got {tuple(o.shape)}")
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
         _check(t, n, io)
     _check(g, "g", torch.float32)
     _check(state, "state", torch.float32)
-    N, Hqk, dk = q.shape
-    Hv, dv = v.shape[1], v.shape[2]
-    if tuple(state.shape) != (N, Hv, dk, dv):
-        raise ValueError(f"state must be [{N},{Hv},{dk},{dv}], got {tuple(state.shape)}")
+    _check(o, "o", io)
     scale = dk ** -0.5 if scale is None else float(scale)
     if o is None:
         o = torch.empty((N, Hv, dv), dtype=io, device=q.device)

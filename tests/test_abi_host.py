@@ -135,3 +135,30 @@ def test_recurrent_step_host_validation():
     assert call(1, 1, 1, 1, 128, 128, None) == 1             # null pointers
     assert call(1, 1, 1, 1, 128, 128, ctypes.c_void_p(24)) == 1   # misaligned
     assert call(1, 0, 1, 1, 128, 128, None) == 0             # N = 0: nothing to do
+
+
+def test_binding_refuses_mismatched_shapes():
+    """Shapes that disagree with q and v are refused on the host (the C ABI would trust them)."""
+    from gated_deltanet_chunked_prefill_b200.workloads import make_inputs
+    x = make_inputs(2, 70, 2, 4, 64, 64, "f32", seed=3, h0_std=0.1, backward=True)
+    args = lambda **kw: {**{n: x[n] for n in ("q", "k", "v", "g", "beta")}, "h0": x["h0"], **kw}
+    fwd = lambda a: gdn.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], None, a["h0"])
+    with pytest.raises(ValueError, match="CUDA"):           # consistent shapes reach the device check
+        fwd(args())
+    bad = {"k": x["k"][:, :, :1], "g": x["g"][:, :, :2], "beta": x["beta"][:1], "h0": x["h0"][:1],
+           "v": x["v"][:, :69]}
+    for name, t in bad.items():
+        with pytest.raises(ValueError, match=name):
+            fwd(args(**{name: t}))
+    with pytest.raises(ValueError, match="dO"):
+        gdn.gdn_chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["dO"][:, :, :1], None, x["h0"], x["dhT"])
+    with pytest.raises(ValueError, match="dhT"):
+        gdn.gdn_chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["dO"], None, x["h0"], x["dhT"][:1])
+    # the decode step: q, k [N,Hqk,dk], v [N,Hv,dv], g, beta [N,Hv], state [N,Hv,dk,dv]
+    t = {n: x[n][:, 0].contiguous() for n in ("q", "k", "v", "g", "beta")}
+    step = lambda **kw: gdn.gdn_recurrent_step(**{**t, "state": x["h0"], **kw})
+    with pytest.raises(ValueError, match="CUDA"):
+        step()
+    for name, bad_t in (("state", x["h0"][:, :1]), ("g", t["g"][:, :1]), ("k", t["k"][:1])):
+        with pytest.raises(ValueError, match=name):
+            step(**{name: bad_t})
