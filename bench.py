@@ -1,19 +1,25 @@
 #!/usr/bin/env python
 """Benchmark of the Gated DeltaNet chunked-prefill operator on B200.
 
-One step = one pass of the operator over one batch of the dense bf16 workload
-(B=4, T=4096, H=16, dk=dv=128): gdn_chunk_fwd, and with STEP = "fwdbwd" also
-gdn_chunk_bwd on the same inputs with incoming gradients dO, dhT. In the fwd+bwd step the
-forward also writes the bf16 chunk start states (gdn_options.states) and the backward
-reads them instead of recomputing its forward pass. Inputs are synthetic (seeded, see the workloads module)
-and resident in HBM when the timed region starts; the working set is larger
-than the 126 MB L2, so no flush is needed between steps.
+Headline step: one pass of the whole operator -- gdn_chunk_fwd then gdn_chunk_bwd -- over the
+packed variable-length workload (24 sequences, 65536 tokens, H=16, dk=dv=128, bf16), the largest
+single-GPU configuration. The forward writes the chunk-state cache (gdn_options.states) and the
+backward reads it. Inputs are synthetic (seeded, see the workloads module) and resident in HBM
+when the timed region starts; the working set is larger than the 126 MB L2.
 
-  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--mode fwd]
+The same JSON line carries, under "per_config", every named workload measured the same way:
+the tiny fp32 forward, the dense forward, the long grouped-value forward (context parallelism),
+the packed forward, the backward configuration (backward alone, reading the forward's cache;
+its forward is timed separately) and the recurrent decode step. Each entry has its roofline
+fraction (the slower of bf16 tensor peak and HBM bytes, against the measured peaks), the
+dominant kernel's achieved bandwidth, an end-to-end number through the public API with host
+buffers, and the fp64 oracle timed on a bounded sample on all host cores.
 
-Prints one JSON line (rank 0). Under torchrun each rank runs its own replica
-(the operator shards by independent (sequence, head) units; no collective on
-the data path) and the time is the max over ranks.
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--only NAME]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own replica (the operator
+shards by independent (sequence, head) units; no collective on the data path) and the time is
+the max over ranks.
 """
 from __future__ import annotations
 
@@ -35,9 +41,14 @@ sys.path.insert(0, ROOT)
 from gated_deltanet_chunked_prefill_b200.workloads import CONFIGS, make_inputs  # noqa: E402
 
 METRIC = "GDN chunk fwd/bwd tokens/s and TFLOP/s on 1 B200; % of roofline"
-WORKLOAD = "dense_bf16"
-STEP = "fwdbwd"       # what one step runs: "fwd" or "fwdbwd"
+HEADLINE = ("varlen_bf16", "fwdbwd")
+# (workload, step) of the per-configuration entries; "bwd" = backward alone with the cache
+SUBS = [("tiny_fp32", "fwd"), ("dense_bf16", "fwd"), ("long_gqa_bf16", "fwd"), ("varlen_bf16", "fwd"),
+        ("bwd_bf16", "bwd")]
 C = 64
+L2_BYTES = 126 * 1024 * 1024
+# datasheet peaks of a B200 (HGX), reported beside the measured ones
+DATASHEET_HBM_GBS, DATASHEET_BF16_TFLOPS = 7700.0, 2250.0
 
 
 def flops(w, fwd=True, bwd=True):
@@ -75,9 +86,11 @@ def kernel_alg_bytes(w):
     gb = ntok * w.Hv * (4 + es)              # g and beta (or dg, dbeta)
     st = w.num_seqs * w.Hv * w.dk * w.dv * 4
     h0 = st if w.h0_std is not None else 0
+    fwd_call = 2 * qk + vv + gb + h0 + vv + st
     return {
         # forward call: q k v g beta h0 -> o hT ; the backward's state pass reads the same inputs
-        "gdn_fwd_tc_kernel": [2 * qk + vv + gb + h0 + vv + st, 2 * qk + vv + gb + h0],
+        "gdn_fwd_tc_kernel": [fwd_call, 2 * qk + vv + gb + h0],
+        "gdn_fwd_simt_kernel": [fwd_call],
         # reverse chain: q k dO g beta dhT -> dh0
         "gdn_bwd_chain_kernel": [2 * qk + vv + gb + st + st],
         # gradients: q k v dO g beta -> dq dk dv dg dbeta
@@ -92,6 +105,23 @@ def peaks():
             d = json.load(fh)
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     return 6650.0, 1590.0, "fallback"
+
+
+def roofline_fraction(w, step, ms):
+    """Fraction of the roofline time (the slower of bf16 tensor peak and HBM bytes) that one step
+    of `ms` milliseconds reaches, against the measured peaks and against the datasheet ones."""
+    fwd, bwd = step in ("fwd", "fwdbwd"), step in ("bwd", "fwdbwd")
+    fl, by = flops(w, fwd, bwd), alg_bytes(w, fwd, bwd)
+    hbm, tc, src = peaks()
+    fp32_tc = w.dtype == "f32"       # fp32 I/O runs on CUDA cores; its flops are still counted on bf16 peak
+    t_hbm, t_tc = by / (hbm * 1e9), fl / (tc * 1e12)
+    t_dhbm, t_dtc = by / (DATASHEET_HBM_GBS * 1e9), fl / (DATASHEET_BF16_TFLOPS * 1e12)
+    t = ms / 1e3
+    return {"alg_bytes": by, "alg_flop": fl, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "roofline_ms": 1e3 * max(t_hbm, t_tc), "frac": max(t_hbm, t_tc) / t,
+            "frac_datasheet": max(t_dhbm, t_dtc) / t, "achieved_gbs": by / t / 1e9,
+            "achieved_tflops": fl / t / 1e12, "peak_source": src,
+            "note": "fp32 I/O on CUDA cores" if fp32_tc else None}
 
 
 class ClockSampler:
@@ -201,55 +231,142 @@ def rank_seed(base: int, rank: int) -> int:
     return base + 17 * rank
 
 
-# ------------------------------------------------------------------------------------- oracle arm
-def oracle_sample(w, x, mode, budget_s):
-    """Time the fp64 oracle on whole (sequence, head) units of the workload until `budget_s`."""
-    from oracle import bwd_token, fwd_chunk  # the CPU baseline is the oracle as it stands
+# ------------------------------------------------------------------------------ oracle (CPU) legs
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _pool_init():
+    # one BLAS thread per worker: the pool itself spreads the units over the cores
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:
+        pass
+
+
+def make_pool(cores: int):
+    """Worker processes for the oracle, forked before this process touches CUDA (a pool forked
+    after the first GPU call is not safe)."""
+    import multiprocessing as mp
+    return mp.get_context("fork").Pool(cores, initializer=_pool_init)
+
+
+def _oracle_unit(task):
+    """One (sequence, v-head) unit through the oracle as it stands; returns its token count."""
+    from oracle import bwd_token, fwd_chunk, fwd_token  # the CPU baseline is the oracle as it stands
+    kind, a = task
+    if kind == "decode":
+        fwd_token(a["q"], a["k"], a["v"], a["g"], a["beta"], a["scale"], a["h0"])
+        return a["q"].shape[0]
+    ex = lambda t: None if t is None else t[None, :, None]
+    q, k, v, g, b = ex(a["q"]), ex(a["k"]), ex(a["v"]), ex(a["g"]), ex(a["beta"])
+    h0 = None if a["h0"] is None else a["h0"][None, None]
+    if kind in ("fwd", "fwdbwd"):
+        fwd_chunk(q, k, v, g, b, a["scale"], h0, chunk=C)
+    if kind in ("bwd", "fwdbwd"):
+        bwd_token(q, k, v, g, b, a["scale"], ex(a["dO"]), h0, a["dhT"][None, None])
+    return a["q"].shape[0]
+
+
+def unit_tasks(w, x, mode, order_seed=0, by_sequence=False):
+    """Oracle tasks, one per (sequence, v-head) unit of the workload, in a fixed shuffled order
+    (a bounded sample then covers short and long packed sequences alike). by_sequence: the
+    sequences in shuffled order, each with its v-heads in order (consecutive units have equal
+    lengths)."""
+    f32 = lambda t: None if t is None else t.float().numpy()
     hq_of = lambda j: j // (w.Hv // w.Hqk)
-    units, tok, t0 = 0, 0, time.perf_counter()
-    if x["cu_seqlens"] is not None:         # packed: sequence n is tokens cu[n]..cu[n+1] of batch row 0
+    if x["cu_seqlens"] is not None:
         cu = x["cu_seqlens"].tolist()
         spans = [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
     else:
         spans = [(n, 0, w.T) for n in range(w.B)]
-    order = [(n, j) for n in range(len(spans)) for j in range(w.Hv)]
-    for n, j in order:
+    if by_sequence:
+        seqs = list(range(len(spans)))
+        np.random.default_rng(order_seed).shuffle(seqs)
+        units = [(n, j) for n in seqs for j in range(w.Hv)]
+    else:
+        units = [(n, j) for n in range(len(spans)) for j in range(w.Hv)]
+        np.random.default_rng(order_seed).shuffle(units)
+    for n, j in units:
         bi, s0, e0 = spans[n]
-        sl = lambda a, h: a[bi:bi + 1, s0:e0, h:h + 1]
-        q, k, v = sl(x["q"], hq_of(j)), sl(x["k"], hq_of(j)), sl(x["v"], j)
-        g, b = sl(x["g"], j), sl(x["beta"], j)
-        h0 = None if x["h0"] is None else x["h0"][n:n + 1, j:j + 1]
-        fwd_chunk(q, k, v, g, b, x["scale"], h0, chunk=C)
-        if mode == "fwdbwd":
-            bwd_token(q, k, v, g, b, x["scale"], sl(x["dO"], j), h0, x["dhT"][n:n + 1, j:j + 1])
-        units += 1
-        tok += e0 - s0
-        if time.perf_counter() - t0 >= budget_s:
+        a = {"q": f32(x["q"][bi, s0:e0, hq_of(j)]), "k": f32(x["k"][bi, s0:e0, hq_of(j)]),
+             "v": f32(x["v"][bi, s0:e0, j]), "g": f32(x["g"][bi, s0:e0, j]),
+             "beta": f32(x["beta"][bi, s0:e0, j]), "scale": x["scale"],
+             "h0": None if x["h0"] is None else f32(x["h0"][n, j])}
+        if mode in ("bwd", "fwdbwd"):
+            a["dO"] = f32(x["dO"][bi, s0:e0, j])
+            a["dhT"] = f32(x["dhT"][n, j])
+        yield (mode, a)
+
+
+def oracle_run(pool, tasks, budget_s, max_units=None):
+    """Run oracle tasks on the pool, at most one per worker in flight, submitting until
+    `budget_s` seconds have passed (or `max_units` were submitted); waits for those in flight.
+    Returns (unit-tokens, seconds, units)."""
+    cores = pool._processes
+    t0 = time.perf_counter()
+    inflight, done_tok, units, submitted = [], 0, 0, 0
+    it = iter(tasks)
+    exhausted = False
+    while True:
+        while (not exhausted and len(inflight) < cores and time.perf_counter() - t0 < budget_s
+               and (max_units is None or submitted < max_units)):
+            try:
+                task = next(it)
+            except StopIteration:
+                exhausted = True
+                break
+            inflight.append(pool.apply_async(_oracle_unit, (task,)))
+            submitted += 1
+        if not inflight:
             break
-    el = time.perf_counter() - t0
-    # one workload token carries all Hv heads: unit-tokens / Hv = workload tokens
-    return (tok / w.Hv) / el, el, units, tok
+        ready = [r for r in inflight if r.ready()]
+        if not ready:
+            time.sleep(0.002)
+            continue
+        for r in ready:
+            done_tok += r.get()
+            units += 1
+            inflight.remove(r)
+    return done_tok, time.perf_counter() - t0, units
 
 
-def run_reference(args, w, x):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return
-    cores = 1
-    per_step = []
+def cpu_baseline(pool, w, x, mode, budget_s):
+    tok, el, units = oracle_run(pool, unit_tasks(w, x, mode), budget_s)
+    return {"value": (tok / w.Hv) / el, "unit": "tokens/s", "cores": pool._processes, "kind": "oracle",
+            "sample": f"{units} (sequence, v-head) units, {tok} unit-tokens of this workload ({mode}), "
+                      f"fp64 numpy oracle, {pool._processes} processes, {el:.1f} s; tokens/s counts a "
+                      f"workload token as all {w.Hv} v-heads"}
+
+
+def run_reference(args, pool):
+    """The oracle as it stands on the host cores, on the headline workload: each step runs one
+    (sequence, v-head) unit per core, v-heads of one sequence together (equal lengths), the
+    sequences in a fixed shuffled order."""
+    name, mode = HEADLINE
+    w = CONFIGS[name]
+    x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed, h0_std=w.h0_std, lengths=w.lengths,
+                    backward=True)
+    cores = pool._processes
+    tasks = iter(unit_tasks(w, x, mode, by_sequence=True))
     for _ in range(args.warmup):
-        oracle_sample(w, x, args.mode, budget_s=0.0)
+        oracle_run(pool, tasks, 1e9, max_units=cores)
+    tok_all, t_all, units_all = 0, 0.0, 0
     for _ in range(args.steps):
-        v, el, units, unit_tok = oracle_sample(w, x, args.mode, budget_s=0.0)
-        per_step.append(el)
-    tok = unit_tok / w.Hv
-    value = tok * len(per_step) / sum(per_step)
-    sample = f"one (sequence, head) unit of {unit_tok} tokens per step ({args.mode}), fp64 numpy oracle"
+        tok, el, units = oracle_run(pool, tasks, 1e9, max_units=cores)
+        tok_all, t_all, units_all = tok_all + tok, t_all + el, units_all + units
+    value = (tok_all / w.Hv) / t_all
+    sample = (f"{units_all} (sequence, v-head) units ({tok_all} unit-tokens) of the packed workload, "
+              f"{cores} v-heads of one sequence per step on {cores} processes ({mode}), fp64 numpy oracle")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": 1e3 * sum(per_step) / len(per_step), "higher_is_better": True,
+           "ms_per_step": 1e3 * t_all / args.steps, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": w.description + f"; step = {args.mode}", "mode": args.mode},
+           "config": {"workload": w.description + f"; step = {mode}", "step": mode},
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -257,8 +374,9 @@ def run_reference(args, w, x):
 
 
 # ------------------------------------------------------------------------------------- GPU arm
-# Decode step workload: a serving batch whose fp32 states (268 MB) exceed the 126 MB L2.
+# Decode step workloads: serving batches whose fp32 states (268 MB) exceed the 126 MB L2.
 DECODE = dict(N=256, Hqk=16, Hv=16, dk=128, dv=128)
+DECODE_256 = dict(N=64, Hqk=16, Hv=16, dk=256, dv=256)
 
 
 def decode_bytes(N, Hqk, Hv, dk, dv):
@@ -267,56 +385,227 @@ def decode_bytes(N, Hqk, Hv, dk, dv):
     return N * Hv * (2 * dk * dv * 4 + 2 * dv * 2 + 4 + 2) + N * Hqk * 2 * dk * 2
 
 
-def decode_oracle_sample(x, Hv, budget_s):
-    """The fp64 oracle's token form, one token of 8 sequences per repetition, for `budget_s`."""
-    from oracle import fwd_token  # the CPU baseline is the oracle as it stands
-    n_s = 8
-    t0 = time.time()
-    reps = 0
-    while reps == 0 or time.time() - t0 < budget_s:
-        fwd_token(x["q"][:n_s], x["k"][:n_s], x["v"][:n_s], x["g"][:n_s], x["beta"][:n_s], x["scale"],
-                  x["h0"][:n_s])
-        reps += 1
-    el = time.time() - t0
-    return {"value": n_s * reps / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n_s} sequences x {Hv} heads, one token each, fp64 numpy oracle, {reps} reps, {el:.1f} s"}
+def time_steps(step, steps, stream, flush=None):
+    """Device time of `steps` calls of step() in ms per step: one event pair around all of them,
+    or, with `flush` (a buffer larger than L2), one pair per step with the buffer rewritten between
+    steps (outside the pairs)."""
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+    pairs = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        pairs.append((e0, e1))
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in pairs]))
 
 
-def run_decode(args):
-    """One step = gdn_recurrent_step over every sequence of the batch (one token each). With
-    --impl reference the oracle's token form alone is timed (rank 0)."""
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    c = DECODE
-    if args.impl == "reference":
-        if rank != 0:
-            return
-        x = make_inputs(c["N"], 1, c["Hqk"], c["Hv"], c["dk"], c["dv"], "bf16", 2000, h0_std=0.1)
-        cpu = decode_oracle_sample(x, c["Hv"], 5.0)
-        print(json.dumps({"impl": "reference", "metric": "GDN recurrent decode step tokens/s on 1 B200; % of HBM "
-                          "roofline", "value": cpu["value"], "unit": "tokens/s", "n_gpus": args.gpus,
-                          "steps": 1, "warmup": 0, "higher_is_better": True, "scaling": "weak",
-                          "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                          "config": {"workload": "decode step (oracle sample)", "step": "decode"},
-                          "cpu_baseline": cpu, "e2e": {"value": cpu["value"], "unit": "tokens/s",
-                                                       "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
-        return
-    import gated_deltanet_chunked_prefill_b200 as gdn
+class Case:
+    """One workload on the device: its inputs, the step a measurement times, and the same step
+    end to end from pinned host buffers."""
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    def __init__(self, gdn, name, mode, dev, rank, cp):
+        self.gdn, self.name, self.mode, self.dev, self.cp = gdn, name, mode, dev, cp
+        self.w = w = CONFIGS[name]
+        self.x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, rank_seed(w.seed, rank),
+                             h0_std=w.h0_std, lengths=w.lengths, backward=mode != "fwd")
+        self.d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.x.items()}
+        d = self.d
+        self.o = torch.empty_like(d["v"])
+        self.hT = torch.empty((w.num_seqs, w.Hv, w.dk, w.dv), dtype=torch.float32, device=dev)
+        self.ws_f = torch.zeros(gdn.fwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, cp),
+                                dtype=torch.uint8, device=dev)
+        self.states = gdn.chunk_states(d["q"], d["v"], d["cu_seqlens"]) if mode != "fwd" else None
+        self.ws_b = None
+        if mode != "fwd":
+            self.ws_b = torch.zeros(gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, cp,
+                                                           states=self.states), dtype=torch.uint8, device=dev)
+            if mode == "bwd":                   # the cache the timed backward reads
+                self.fwd(d)
+        self.flush = (torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+                      if alg_bytes(w, mode != "bwd", mode != "fwd") < 2 * L2_BYTES else None)
+
+    def fwd(self, dd):
+        self.gdn.gdn_chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["scale"], dd["h0"],
+                               dd["cu_seqlens"], cp_segment_chunks=self.cp, workspace=self.ws_f, o=self.o,
+                               hT=self.hT, states=self.states, check_status=False)
+
+    def bwd(self, dd, states=True, ws=None):
+        return self.gdn.gdn_chunk_bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["dO"], dd["scale"],
+                                      dd["h0"], dd["dhT"], dd["cu_seqlens"], cp_segment_chunks=self.cp,
+                                      workspace=self.ws_b if ws is None else ws,
+                                      states=self.states if states else None, check_status=False)
+
+    def step(self, dd=None):
+        dd = self.d if dd is None else dd
+        if self.mode == "fwd":
+            self.fwd(dd)
+            return None
+        if self.mode == "fwdbwd":
+            self.fwd(dd)
+        return self.bwd(dd)
+
+    def measure(self, steps, warmup, stream):
+        for _ in range(max(warmup, 3)):
+            self.step()
+        torch.cuda.synchronize()
+        ms = time_steps(self.step, steps, stream, self.flush)
+        per_kernel, launches_one = {}, []
+        with self.gdn.KernelTrace(capacity=256) as tr:
+            for _ in range(3):
+                if self.flush is not None:
+                    self.flush.zero_()
+                self.step()
+        for name, t in tr.launches:
+            per_kernel.setdefault(name, []).append(t)
+        launches_one = tr.launches[: len(tr.launches) // 3]
+        return ms, per_kernel, launches_one
+
+    def extra_times(self, stream):
+        """The forward call alone, and (with a backward) the backward that recomputes its forward
+        pass instead of reading the cache."""
+        out = {}
+        if self.mode == "fwd":
+            return out
+        with self.gdn.KernelTrace(capacity=256) as trf:
+            for _ in range(3):
+                self.fwd(self.d)
+        out["fwd_ms"] = sum(t for _, t in trf.launches) / 3
+        ws_r = torch.zeros(self.gdn.bwd_workspace_size(self.w.B, self.w.T, self.w.Hqk, self.w.Hv, self.w.dk,
+                                                       self.w.dv, self.w.num_seqs, self.cp),
+                           dtype=torch.uint8, device=self.dev)
+        with self.gdn.KernelTrace(capacity=256) as trb:
+            for _ in range(3):
+                self.bwd(self.d, states=False, ws=ws_r)
+        out["bwd_recompute_ms"] = sum(t for _, t in trb.launches) / 3
+        with self.gdn.KernelTrace(capacity=256) as trc:
+            for _ in range(3):
+                self.bwd(self.d)
+        out["bwd_ms"] = sum(t for _, t in trc.launches) / 3
+        return out
+
+    def e2e(self, steps, stream, dist):
+        """The step through the public API from pinned host inputs, every output copied back to
+        pinned host memory, all inside the timed region. The backward-alone workload recomputes its
+        forward pass (the host holds no chunk-state cache)."""
+        mode = self.mode
+        need = ["q", "k", "v", "g", "beta", "h0", "cu_seqlens"] + (["dO", "dhT"] if mode != "fwd" else [])
+        host = {k: self.x[k].pin_memory() for k in need if self.x.get(k) is not None}
+        dev_in = {k: torch.empty_like(self.d[k]) for k in host}
+        dev_in["scale"] = self.d["scale"]
+        for k in ("h0", "dO", "dhT", "cu_seqlens"):
+            dev_in.setdefault(k, None)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        out_host = {}
+
+        def back(name, t):
+            if name not in out_host:
+                out_host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            out_host[name].copy_(t, non_blocking=True)
+            return t.numel() * t.element_size()
+
+        def one():
+            for k, t in host.items():
+                dev_in[k].copy_(t, non_blocking=True)
+            nbytes = 0
+            if mode in ("fwd", "fwdbwd"):
+                self.fwd(dev_in)
+                nbytes += back("o", self.o) + back("hT", self.hT)
+            if mode != "fwd":
+                gr = self.bwd(dev_in, states=mode == "fwdbwd", ws=None if mode == "fwdbwd" else self._ws_recompute())
+                for k2, t2 in gr.items():
+                    if t2 is not None:
+                        nbytes += back(k2, t2)
+            return nbytes
+
+        for _ in range(2):
+            d2h = one()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, self.dev) / steps
+        return e_ms, int(h2d), int(d2h)
+
+    def _ws_recompute(self):
+        if getattr(self, "_wsr", None) is None:
+            w = self.w
+            self._wsr = torch.zeros(self.gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs,
+                                                                self.cp), dtype=torch.uint8, device=self.dev)
+        return self._wsr
+
+
+def dominant_roofline(case, per_kernel, launches_one, step_label):
+    """The roofline object of the kernel with the largest total time in one step: its algorithmic
+    bytes per launch over its average CUDA-event launch time."""
+    hbm, _, src = peaks()
+    kb = kernel_alg_bytes(case.w)
+    seen, per_kernel_bytes = {}, {}
+    for name, _t in launches_one:
+        k = seen.get(name, 0)
+        seen[name] = k + 1
+        opts = kb.get(name)
+        if opts:
+            # the backward's state pass is the second forward-kernel launch only in a recompute
+            idx = min(k, len(opts) - 1) if case.mode == "fwdbwd" or case.states is None else 0
+            per_kernel_bytes.setdefault(name, []).append(opts[idx])
+    dom = max(per_kernel, key=lambda k: sum(per_kernel[k]))
+    dom_ms = float(np.mean(per_kernel[dom]))
+    dom_bytes = float(np.mean(per_kernel_bytes.get(dom, [0])))
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "frac_datasheet": achieved / DATASHEET_HBM_GBS, "peak_source": src,
+            "traffic": traffic_record(dom, case.name, step_label),
+            "alg_bytes_per_launch": dom_bytes, "avg_launch_ms": dom_ms}
+
+
+def measure_case(gdn, name, mode, args, dev, rank, world, dist, stream, pool, budget, e2e_steps):
+    case = Case(gdn, name, mode, dev, rank, args.cp)
+    w = case.w
+    ms, per_kernel, launches_one = case.measure(args.steps, args.warmup, stream)
+    ms = max_over_ranks(ms, dist, dev)
+    tokens = w.B * w.T
+    fwd, bwd = mode in ("fwd", "fwdbwd"), mode in ("bwd", "fwdbwd")
+    res = {"workload": name, "description": w.description, "step": mode, "ms_per_step": ms,
+           "tokens_per_s": tokens * world / (ms / 1e3),
+           "tflops": flops(w, fwd, bwd) * world / (ms / 1e3) / 1e12,
+           "step_roofline": roofline_fraction(w, mode, ms),
+           "roofline": dominant_roofline(case, per_kernel, launches_one, mode),
+           "per_kernel_ms": {k: float(np.mean(v)) for k, v in per_kernel.items()},
+           "l2": ("inputs larger than the 126 MB L2; no flush" if case.flush is None else
+                  "working set below 2x L2: a 252 MB buffer is rewritten between timed steps")}
+    res.update(case.extra_times(stream))
+    e_ms, h2d, d2h = case.e2e(e2e_steps, stream, dist)
+    res["e2e"] = {"value": tokens * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    res["cpu_baseline"] = (cpu_baseline(pool, w, case.x, mode, budget)
+                           if pool is not None and rank == 0 and world == 1 else None)
+    del case
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_decode(gdn, args, dev, rank, world, dist, stream, pool, budget, c=DECODE):
+    """One step = gdn_recurrent_step over every sequence of the batch (one token each)."""
     N, Hqk, Hv, dk, dv = c["N"], c["Hqk"], c["Hv"], c["dk"], c["dv"]
     x = make_inputs(N, 1, Hqk, Hv, dk, dv, "bf16", rank_seed(2000, rank), h0_std=0.1)
     tok = {n: x[n][:, 0].contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")}
     state = x["h0"].to(dev)
     o = torch.empty((N, Hv, dv), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def step():
         gdn.gdn_recurrent_step(tok["q"], tok["k"], tok["v"], tok["g"], tok["beta"], state, x["scale"], o=o)
@@ -324,85 +613,65 @@ def run_decode(args):
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
-    if args.single:
-        step()
-        torch.cuda.synchronize()
-        return
-    sampler = ClockSampler(local)
-    sampler.start()
-    n0 = gdn.launch_count()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    tw0 = time.time()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    tw1 = time.time()
-    if dist:
-        dist.barrier()
-    sampler.stop()
-    launches = gdn.launch_count() - n0
-    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dist, dev) / args.steps
+    ms = max_over_ranks(time_steps(step, args.steps, stream), dist, dev)
     hbm, _, src = peaks()
     nbytes = decode_bytes(N, Hqk, Hv, dk, dv)
-    gbs = nbytes / (ms_step / 1e3) / 1e9
-    # the oracle's token form on a bounded sample of the same batch (rank 0, N = 1 only)
-    cpu = decode_oracle_sample(x, Hv, min(args.cpu_budget, 5.0)) \
-        if rank == 0 and world == 1 and args.cpu_budget > 0 else None
-    if rank == 0:
-        line = {"metric": "GDN recurrent decode step tokens/s on 1 B200; % of HBM roofline",
-                "value": N * world / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": f"decode step: {N} sequences, Hqk={Hqk} Hv={Hv}, dk=dv={dk}, bf16 I/O, "
-                                       f"fp32 state", "step": "decode", "parallelism": "single" if world == 1
-                           else f"replicas{world}", "l2": "states (268 MB) larger than the 126 MB L2; no flush"},
-                "roofline": {"bound": "hbm", "kernel": "gdn_step_kernel", "achieved": gbs, "peak": hbm,
-                             "unit": "GB/s", "frac": gbs / hbm, "peak_source": src,
-                             "traffic": traffic_record("gdn_step_kernel", "decode", "decode"),
-                             "alg_bytes_per_launch": nbytes, "avg_launch_ms": ms_step},
-                "cpu_baseline": cpu, "gpu_launches": launches, "clocks": sampler.summary(tw0, tw1)}
-        print(json.dumps(line))
-    if dist:
-        dist.destroy_process_group()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    cpu = None
+    if pool is not None and rank == 0 and world == 1:
+        def tasks():
+            for s0 in range(0, N, 8):
+                yield ("decode", {n: x[n][s0:s0 + 8].float().numpy() for n in ("q", "k", "v", "g", "beta", "h0")}
+                       | {"scale": x["scale"]})
+        tk, el, units = oracle_run(pool, tasks(), budget)
+        cpu = {"value": tk / el, "unit": "tokens/s", "cores": pool._processes, "kind": "oracle",
+               "sample": f"{units} groups of 8 sequences x {Hv} heads, one token each, fp64 numpy oracle "
+                         f"(token form), {pool._processes} processes, {el:.1f} s"}
+    return {"workload": f"decode step: {N} sequences, Hqk={Hqk} Hv={Hv}, dk=dv={dk}, bf16 I/O, fp32 state",
+            "step": "decode", "ms_per_step": ms, "tokens_per_s": N * world / (ms / 1e3),
+            "roofline": {"bound": "hbm", "kernel": "gdn_step_kernel", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "frac_datasheet": gbs / DATASHEET_HBM_GBS, "peak_source": src,
+                         "traffic": traffic_record("gdn_step_kernel", "decode", "decode"),
+                         "alg_bytes_per_launch": nbytes, "avg_launch_ms": ms},
+            "l2": f"states ({N * Hv * dk * dv * 4 / 1e6:.0f} MB) larger than the 126 MB L2; no flush",
+            "cpu_baseline": cpu}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--mode", default=STEP, choices=["fwd", "fwdbwd", "decode"],
-                    help="decode: the recurrent decode step on its own batch (a separate line)")
+    ap.add_argument("--only", default=None,
+                    help="time only this workload (name from the workloads module, or 'decode') as the line")
+    ap.add_argument("--mode", default=None, choices=["fwd", "fwdbwd", "bwd"], help="step of --only")
+    ap.add_argument("--no-sub", action="store_true", help="skip the per-configuration entries")
     ap.add_argument("--single", action="store_true",
-                    help="only warm-up steps plus one step, no report (for profiler launch lists)")
-    ap.add_argument("--workload", default=WORKLOAD, choices=list(CONFIGS))
-    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
+                    help="only warm-up steps plus one step of the headline, no report (profiler launch lists)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline (headline)")
     ap.add_argument("--cp", type=int, default=0, help="cp_segment_chunks option (0 = automatic)")
     args = ap.parse_args()
-
-    w = CONFIGS[args.workload]
-    if args.mode == "decode":
-        run_decode(args)
-        return
-    if args.impl == "reference":
-        if int(os.environ.get("RANK", "0")) != 0:
-            return
-        x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.seed, h0_std=w.h0_std, lengths=w.lengths,
-                        backward=True)
-        run_reference(args, w, x)
-        return
-
-    import gated_deltanet_chunked_prefill_b200 as gdn
+    assert args.warmup >= 0 and args.steps > 0
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    # the oracle's process pool is forked before anything touches CUDA
+    want_cpu = rank == 0 and world == 1 and args.cpu_budget > 0 and not args.single
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        pool = make_pool(host_cores())
+        try:
+            run_reference(args, pool)
+        finally:
+            pool.terminate()
+        return
+    pool = make_pool(host_cores()) if want_cpu else None
+
+    import gated_deltanet_chunked_prefill_b200 as gdn
+
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = None
@@ -410,185 +679,87 @@ def main():
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, rank_seed(w.seed, rank), h0_std=w.h0_std,
-                    lengths=w.lengths,
-                    backward=True)
-    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     stream = torch.cuda.current_stream(dev)
 
-    mode = args.mode
-
-    ws_f = torch.zeros(gdn.fwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp),
-                       dtype=torch.uint8, device=dev)
-    states = gdn.chunk_states(d["q"], d["v"], d["cu_seqlens"]) if mode == "fwdbwd" else None
-    ws_b = torch.zeros(gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp,
-                                              states=states), dtype=torch.uint8, device=dev)
-    o = torch.empty_like(d["v"])
-    hT = torch.empty((w.num_seqs, w.Hv, w.dk, w.dv), dtype=torch.float32, device=dev)
-
-    def step(dd):
-        gdn.gdn_chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["scale"], dd["h0"],
-                          dd["cu_seqlens"], cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT, states=states)
-        if mode == "fwdbwd":
-            return gdn.gdn_chunk_bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["dO"], dd["scale"],
-                                     dd["h0"], dd["dhT"], dd["cu_seqlens"], cp_segment_chunks=args.cp,
-                                     workspace=ws_b, states=states)
-        return None
-
-    # ---- device-resident timing
-    for _ in range(max(args.warmup, 3)):
-        step(d)
-    torch.cuda.synchronize()
+    name, mode = HEADLINE
+    if args.only:
+        name, mode = args.only, args.mode or ("fwd" if args.only != "bwd_bf16" else "bwd")
     if args.single:
-        step(d)
+        case = Case(gdn, name, mode, dev, rank, args.cp)
+        for _ in range(max(args.warmup, 3)):
+            case.step()
+        case.step()
         torch.cuda.synchronize()
         return
-    if dist:
-        dist.barrier()
+
+    # ---- the headline step, device-resident, with clocks sampled during the timed region
     sampler = ClockSampler(local)
     sampler.start()
-    n0 = gdn.launch_count()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    case = Case(gdn, name, mode, dev, rank, args.cp)
+    w = case.w
+    for _ in range(max(args.warmup, 3)):
+        case.step()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
+    n0 = gdn.launch_count()
     tw0 = time.time()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step(d)
-    ev1.record(stream)
-    torch.cuda.synchronize()
+    ms = time_steps(case.step, args.steps, stream, case.flush)
     tw1 = time.time()
+    launches = gdn.launch_count() - n0
     if dist:
         dist.barrier()
     sampler.stop()
-    launches = gdn.launch_count() - n0
-    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
-    ms_step = ms / args.steps
-    tokens = w.B * w.T * world
-    value = tokens / (ms_step / 1e3)
-
-    # ---- per-kernel times (CUDA events on the launch stream, library-recorded)
+    ms = max_over_ranks(ms, dist, dev)
+    tokens = w.B * w.T
+    fwd, bwd = mode in ("fwd", "fwdbwd"), mode in ("bwd", "fwdbwd")
     per_kernel = {}
-    with gdn.KernelTrace(capacity=64) as tr:
-        for _ in range(5):
-            step(d)
-    for name, t in tr.launches:
-        per_kernel.setdefault(name, []).append(t)
-    fwd_ms = bwd_ms = None
-    with gdn.KernelTrace(capacity=64) as trf:
-        for _ in range(5):
-            gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"],
-                              d["cu_seqlens"], cp_segment_chunks=args.cp, workspace=ws_f, o=o, hT=hT, states=states)
-    fwd_ms = sum(t for _, t in trf.launches) / 5
-    bwd_recompute_ms = None
-    if mode == "fwdbwd":
-        bwd_ms = sum(t for _, t in tr.launches) / 5 - fwd_ms
-        # the backward alone once more, recomputing the chunk states itself (no cache)
-        ws_r = torch.zeros(gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, args.cp),
-                           dtype=torch.uint8, device=dev)
-        with gdn.KernelTrace(capacity=64) as trb:
-            for _ in range(5):
-                gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["scale"], d["h0"],
-                                  d["dhT"], d["cu_seqlens"], cp_segment_chunks=args.cp, workspace=ws_r)
-        bwd_recompute_ms = sum(t for _, t in trb.launches) / 5
-        del ws_r
+    with gdn.KernelTrace(capacity=256) as tr:
+        for _ in range(3):
+            case.step()
+    for kname, t in tr.launches:
+        per_kernel.setdefault(kname, []).append(t)
+    roofline = dominant_roofline(case, per_kernel, tr.launches[: len(tr.launches) // 3], mode)
+    extra = case.extra_times(stream)
+    e_ms, h2d, d2h = case.e2e(max(3, min(args.steps, 10)), stream, dist)
+    head_x = case.x
+    del case
+    torch.cuda.empty_cache()
 
-    hbm, tc_peak, src = peaks()
-    # per-launch algorithmic bytes, matched to the launches of one step in order
-    kb = kernel_alg_bytes(w)
-    seen = {}
-    per_kernel_bytes = {}
-    for name, t in tr.launches[: len(tr.launches) // 5]:
-        k = seen.get(name, 0)
-        seen[name] = k + 1
-        opts = kb.get(name)
-        if opts:
-            per_kernel_bytes.setdefault(name, []).append(opts[min(k, len(opts) - 1)])
-    dom = max(per_kernel, key=lambda k: sum(per_kernel[k]))
-    dom_ms = float(np.mean(per_kernel[dom]))
-    dom_bytes = float(np.mean(per_kernel_bytes.get(dom, [0])))
-    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "peak_source": src,
-                "traffic": traffic_record(dom, args.workload, mode),
-                "alg_bytes_per_launch": dom_bytes, "avg_launch_ms": dom_ms}
-    step_bytes = alg_bytes(w, fwd=True, bwd=mode == "fwdbwd")
-    step_roofline = {"alg_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
-                     "frac_hbm": step_bytes / (ms_step / 1e3) / 1e9 / hbm,
-                     "tflops": flops(w, fwd=True, bwd=mode == "fwdbwd") / (ms_step / 1e3) / 1e12,
-                     "frac_tensor": flops(w, fwd=True, bwd=mode == "fwdbwd") / (ms_step / 1e3) / 1e12 / tc_peak}
-
-    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
-    host_in = {k: x[k].pin_memory() for k in ("q", "k", "v", "g", "beta", "h0", "dO", "dhT", "cu_seqlens")
-               if x.get(k) is not None}
-    dev_in = {k: torch.empty_like(d[k]) for k in host_in}
-    dev_in["scale"] = d["scale"]
-    for k in ("h0", "dO", "dhT", "cu_seqlens"):
-        dev_in.setdefault(k, None)
-    h2d = sum(t.numel() * t.element_size() for k, t in host_in.items()
-              if mode == "fwdbwd" or k not in ("dO", "dhT"))
-    out_host = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
-                "hT": torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)}
-
-    def e2e_step():
-        for k, t in host_in.items():
-            if mode == "fwdbwd" or k not in ("dO", "dhT"):
-                dev_in[k].copy_(t, non_blocking=True)
-        gr = step(dev_in)
-        out_host["o"].copy_(o, non_blocking=True)
-        out_host["hT"].copy_(hT, non_blocking=True)
-        nbytes = o.numel() * o.element_size() + hT.numel() * 4
-        if gr is not None:
-            for k2, t2 in gr.items():
-                if t2 is None:
-                    continue
-                if k2 not in out_host:
-                    out_host[k2] = torch.empty(t2.shape, dtype=t2.dtype, pin_memory=True)
-                out_host[k2].copy_(t2, non_blocking=True)
-                nbytes += t2.numel() * t2.element_size()
-        return nbytes
-
-    for _ in range(2):
-        d2h = e2e_step()
-    torch.cuda.synchronize()
-    e_steps = max(3, min(args.steps, 20))
-    if dist:
-        dist.barrier()
-    ev0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
-    e2e = {"value": tokens / (e_ms / e_steps / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
-
-    # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
-    cpu = None
-    if rank == 0 and world == 1 and args.cpu_budget > 0:
-        v_cpu, el, units, unit_tok = oracle_sample(w, x, mode, args.cpu_budget)
-        cpu = {"value": v_cpu, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"{units} (sequence, head) units, {unit_tok} unit-tokens of the same workload "
-                         f"({mode}), fp64 numpy oracle, {el:.1f} s"}
-
-    fl = flops(w, fwd=True, bwd=mode == "fwdbwd") * world
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": w.description, "step": mode, "global_batch": w.B * world,
-                      "seq_len": w.T, "heads_qk": w.Hqk, "heads_v": w.Hv, "dk": w.dk, "dv": w.dv,
-                      "chunk": C, "parallelism": f"replicas x{world}" if world > 1 else "single",
+    out = {"metric": METRIC, "value": tokens * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+           "data": "synthetic",
+           "config": {"workload": w.description + f"; step = {mode}", "name": name, "step": mode,
+                      "global_batch": w.B * world, "seq_len": w.T, "num_seqs": w.num_seqs, "heads_qk": w.Hqk,
+                      "heads_v": w.Hv, "dk": w.dk, "dv": w.dv, "chunk": C,
+                      "parallelism": f"replicas x{world}" if world > 1 else "single",
                       "l2": "working set larger than the 126 MB L2; no flush",
                       "bwd_states": "cached by the forward (bf16 chunk start states)" if mode == "fwdbwd" else None,
                       "cp_segment_chunks": args.cp},
-           "tflops": fl / (ms_step / 1e3) / 1e12,
-           "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "bwd_recompute_ms": bwd_recompute_ms,
+           "tflops": flops(w, fwd, bwd) * world / (ms / 1e3) / 1e12,
+           **extra,
            "per_kernel_ms": {k: float(np.mean(v)) for k, v in per_kernel.items()},
-           "roofline": roofline, "step_roofline": step_roofline, "cpu_baseline": cpu, "e2e": e2e,
-           "gpu_launches": int(launches),
-           "clocks": sampler.summary(tw0, tw1)}
+           "roofline": roofline, "step_roofline": roofline_fraction(w, mode, ms),
+           "e2e": {"value": tokens * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
+           "gpu_launches": int(launches), "clocks": sampler.summary(tw0, tw1)}
+    out["cpu_baseline"] = cpu_baseline(pool, w, head_x, mode, args.cpu_budget) if pool is not None else None
+    del head_x
+
+    # ---- every named workload, measured the same way
+    if not args.no_sub and not args.only:
+        sub_budget = max(2.0, args.cpu_budget / 3)
+        per = {}
+        for sname, smode in SUBS:
+            per[f"{sname}:{smode}"] = measure_case(gdn, sname, smode, args, dev, rank, world, dist, stream, pool,
+                                                   sub_budget, max(3, min(args.steps, 5)))
+        per["decode"] = measure_decode(gdn, args, dev, rank, world, dist, stream, pool, sub_budget)
+        per["decode_d256"] = measure_decode(gdn, args, dev, rank, world, dist, stream, pool, sub_budget / 2,
+                                            DECODE_256)
+        out["per_config"] = per
+    if pool is not None:
+        pool.terminate()
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist:

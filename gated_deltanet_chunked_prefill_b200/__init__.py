@@ -14,29 +14,39 @@ from typing import Optional
 import torch
 
 __all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd", "fwd_workspace_size",
-           "bwd_workspace_size", "chunk_states", "read_device_status", "Options", "LIB_PATH", "KernelTrace",
-           "launch_count", "gdn_recurrent_step", "chunk_gated_delta_rule"]
+           "bwd_workspace_size", "chunk_states", "read_device_status", "check_device_error", "Options",
+           "LIB_PATH", "KernelTrace", "launch_count", "gdn_recurrent_step", "chunk_gated_delta_rule"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
 GDN_F32, GDN_BF16 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace",
-          4: "CUDA runtime error", 5: "device timeout", 6: "inconsistent device input"}
+          4: "CUDA runtime error", 5: "device timeout", 6: "inconsistent device input",
+          7: "unusable kernel launch"}
+
+
+def _check_default() -> bool:
+    """Whether calls read back the device status word by default (environment GDN_CHECK_STATUS=1)."""
+    return os.environ.get("GDN_CHECK_STATUS", "0") not in ("", "0")
 
 
 class GdnError(RuntimeError):
     def __init__(self, code: int, where: str):
         detail = ""
-        if code == 4 and _lib is not None:
-            detail = " -- " + _lib.gdn_last_error().decode(errors="replace")
+        if code in (3, 4) and _lib is not None:
+            text = _lib.gdn_last_error().decode(errors="replace")
+            if text:
+                detail = " -- " + text
         super().__init__(f"{where}: {STATUS.get(code, code)} (status {code}){detail}")
         self.code = code
 
 
 class Options(ctypes.Structure):
-    """Mirror of gdn_options."""
-    _fields_ = [("cp_segment_chunks", ctypes.c_int), ("cp_exact", ctypes.c_int),
-                ("states", ctypes.c_void_p), ("reserved", ctypes.c_int * 4)]
+    """Mirror of gdn_options (include/gdn.h)."""
+    _fields_ = [("cp_mode", ctypes.c_int), ("deterministic", ctypes.c_int),
+                ("cp_segment_chunks", ctypes.c_int), ("cp_exact", ctypes.c_int),
+                ("states", ctypes.c_void_p), ("qk_l2norm", ctypes.c_int), ("test_stall", ctypes.c_int),
+                ("reserved", ctypes.c_int * 2)]
 
 
 _lib = None
@@ -71,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_recurrent_step.restype = i
         L.gdn_read_device_status.argtypes = [vp, vp]
         L.gdn_read_device_status.restype = i
+        L.gdn_check_device_error.argtypes = [vp]
+        L.gdn_check_device_error.restype = i
         L.gdn_status_string.argtypes = [i]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_last_error.argtypes = []
@@ -101,15 +113,34 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported I/O dtype {t.dtype}")
 
 
-def _opts(cp_segment_chunks: int, cp_exact: bool = False, states=None):
+def _opts(cp_segment_chunks: int = 0, cp_exact: bool = False, states=None, cp_mode: int = 0,
+          qk_l2norm: bool = False, deterministic: bool = False, test_stall: bool = False):
     o = Options()
+    o.cp_mode = int(cp_mode)
+    o.deterministic = int(bool(deterministic))
     o.cp_segment_chunks = int(cp_segment_chunks)
     o.cp_exact = int(bool(cp_exact))
+    o.qk_l2norm = int(bool(qk_l2norm))
+    o.test_stall = int(bool(test_stall))
     if states is not None:
         if states.dtype != torch.bfloat16 or not states.is_cuda or not states.is_contiguous():
             raise ValueError("states: a contiguous bf16 CUDA tensor from chunk_states()")
         o.states = states.data_ptr()
     return o
+
+
+def _check_states(states, q, v, cu_seqlens):
+    """The C ABI takes the chunk-state cache as a bare pointer: refuse one that is too small for
+    these sizes or lives on another device before the kernels write or read it."""
+    if states is None:
+        return
+    if states.device != q.device:
+        raise ValueError(f"states is on device {states.device}, the inputs on {q.device}")
+    B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
+    need = int(lib().gdn_chunk_states_size(B, T, Hqk, Hv, dk, dv, N))
+    if states.numel() * states.element_size() < need:
+        raise ValueError(f"states holds {states.numel() * states.element_size()} bytes; these sizes need {need} "
+                         "(make it with chunk_states() on the same inputs)")
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -124,13 +155,14 @@ def _dims(q, v, cu_seqlens):
     return B, T, Hqk, Hv, dk, dv, N
 
 
-def fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False) -> int:
-    o = _opts(cp_segment_chunks, cp_exact)
+def fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False, cp_mode=0) -> int:
+    o = _opts(cp_segment_chunks, cp_exact, cp_mode=cp_mode)
     return int(lib().gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
 
 
-def bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False, states=None) -> int:
-    o = _opts(cp_segment_chunks, cp_exact, states)
+def bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False, states=None,
+                       cp_mode=0) -> int:
+    o = _opts(cp_segment_chunks, cp_exact, states, cp_mode=cp_mode)
     return int(lib().gdn_chunk_bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
 
 
@@ -186,11 +218,24 @@ def _workspace(nbytes, workspace, device):
     return workspace
 
 
+def _status_after(ws, stream, where):
+    """Synchronise and raise if the call's kernels recorded a device-side finding in `ws`."""
+    code = read_device_status(ws, stream)
+    if code != 0:
+        raise GdnError(code, where + " (device status)")
+
+
 def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
                   output_final_state=True, cp_segment_chunks=0, cp_exact=False, workspace=None,
-                  o=None, hT=None, stream=None, states=None):
+                  o=None, hT=None, stream=None, states=None, cp_mode=0, qk_l2norm=False,
+                  deterministic=False, check_status=None, test_stall=False):
     """Forward through the C ABI. Returns (o, hT or None). With `states` (from
-    chunk_states()) it also writes every chunk's start state for a later backward."""
+    chunk_states()) it also writes every chunk's start state for a later backward.
+
+    Device-side findings (inconsistent cu_seqlens, a timed-out wait) leave o / hT unspecified and
+    are only visible through the workspace's status word: with check_status=True (default: the
+    environment variable GDN_CHECK_STATUS=1) the call synchronises, reads it and raises GdnError.
+    Otherwise read it with read_device_status(workspace) or check_device_error()."""
     _check_shapes(q, k, v, g, beta, h0, cu_seqlens, o=o, hT=hT)
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
@@ -198,26 +243,32 @@ def gdn_chunk_fwd(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
     _check(g, "g", torch.float32)
     _check(h0, "h0", torch.float32)
     _check(cu_seqlens, "cu_seqlens", torch.int32)
+    _check_states(states, q, v, cu_seqlens)
     B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
     scale = dk ** -0.5 if scale is None else float(scale)
     if o is None:
         o = torch.empty((B, T, Hv, dv), dtype=io, device=q.device)
     if hT is None and output_final_state:
         hT = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
-    ws_bytes = fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact)
+    ws_bytes = fwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact, cp_mode)
     ws = _workspace(ws_bytes, workspace, q.device)
-    opt = _opts(cp_segment_chunks, cp_exact, states)
+    opt = _opts(cp_segment_chunks, cp_exact, states, cp_mode, qk_l2norm, deterministic, test_stall)
     st = lib().gdn_chunk_fwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                              _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(o),
                              _ptr(hT), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream(stream))
     if st != 0:
         raise GdnError(st, "gdn_chunk_fwd")
+    if _check_default() if check_status is None else check_status:
+        _status_after(ws, stream, "gdn_chunk_fwd")
     return o, hT
 
 
 def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None,
-                          output_final_state=True, cp_segment_chunks=0, o=None, hT=None, stream=None):
-    """Forward through the allocation-free entry point (library-held 1 MiB scratch; see gdn.h)."""
+                          output_final_state=True, cp_segment_chunks=0, o=None, hT=None, stream=None,
+                          cp_mode=0, check_status=None):
+    """Forward through the allocation-free entry point (library-held 1 MiB scratch; see gdn.h).
+    With check_status (as in gdn_chunk_fwd) the device-side findings are read through
+    check_device_error(), the per-device status word."""
     _check_shapes(q, k, v, g, beta, h0, cu_seqlens, o=o, hT=hT)
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
@@ -231,20 +282,26 @@ def gdn_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None
         o = torch.empty((B, T, Hv, dv), dtype=io, device=q.device)
     if hT is None and output_final_state:
         hT = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
-    opt = _opts(cp_segment_chunks)
+    opt = _opts(cp_segment_chunks, cp_mode=cp_mode)
     st = lib().gdn_chunk_fwd_noalloc(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                                      _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N,
                                      _ptr(o), _ptr(hT), ctypes.byref(opt), _stream(stream))
     if st != 0:
         raise GdnError(st, "gdn_chunk_fwd_noalloc")
+    if _check_default() if check_status is None else check_status:
+        code = check_device_error(stream)
+        if code != 0:
+            raise GdnError(code, "gdn_chunk_fwd_noalloc (device status)")
     return o, hT
 
 
 def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlens=None,
                   cp_segment_chunks=0, cp_exact=False, workspace=None, want_dh0=True, stream=None,
-                  states=None):
+                  states=None, cp_mode=0, qk_l2norm=False, deterministic=False, check_status=None):
     """Backward through the C ABI. Returns dict dq, dk, dv, dg, dbeta, dh0. With `states`
-    written by the matching gdn_chunk_fwd call, the forward pass is not recomputed."""
+    written by the matching gdn_chunk_fwd call, the forward pass is not recomputed.
+    check_status: as in gdn_chunk_fwd (device-side findings otherwise leave the gradients
+    unspecified without an exception)."""
     _check_shapes(q, k, v, g, beta, h0, cu_seqlens, dO=dO, dhT=dhT)
     io = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta"), (dO, "dO")):
@@ -253,6 +310,7 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
     _check(h0, "h0", torch.float32)
     _check(dhT, "dhT", torch.float32)
     _check(cu_seqlens, "cu_seqlens", torch.int32)
+    _check_states(states, q, v, cu_seqlens)
     B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
     scale = dk ** -0.5 if scale is None else float(scale)
     dq = torch.empty_like(q)
@@ -261,15 +319,17 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
     dg = torch.empty_like(g)
     db = torch.empty_like(beta)
     dh0 = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
-    ws_bytes = bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact, states)
+    ws_bytes = bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact, states, cp_mode)
     ws = _workspace(ws_bytes, workspace, q.device)
-    opt = _opts(cp_segment_chunks, cp_exact, states)
+    opt = _opts(cp_segment_chunks, cp_exact, states, cp_mode, qk_l2norm, deterministic)
     st = lib().gdn_chunk_bwd(_dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                              _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N, _ptr(dO),
                              _ptr(dhT), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db),
                              _ptr(dh0), _ptr(ws), ws.numel(), ctypes.byref(opt), _stream(stream))
     if st != 0:
         raise GdnError(st, "gdn_chunk_bwd")
+    if _check_default() if check_status is None else check_status:
+        _status_after(ws, stream, "gdn_chunk_bwd")
     return dict(dq=dq, dk=dkk, dv=dvv, dg=dg, dbeta=db, dh0=dh0)
 
 
@@ -341,6 +401,12 @@ def launch_count() -> int:
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise and return (and clear) the workspace's device status word."""
     return int(lib().gdn_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+def check_device_error(stream=None) -> int:
+    """Synchronise `stream` and return (and clear) the library's per-device status word: the first
+    device-side finding of any call on the current device since the last check (0 = none)."""
+    return int(lib().gdn_check_device_error(_stream(stream)))
 
 
 from .autograd import chunk_gated_delta_rule  # noqa: E402  (uses the functions above)

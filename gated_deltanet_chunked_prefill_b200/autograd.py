@@ -30,13 +30,14 @@ def backward_supported(q: torch.Tensor, v: torch.Tensor) -> bool:
 class _ChunkGatedDeltaRule(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, g, beta, scale, initial_state, output_final_state, cu_seqlens,
-                cp_segment_chunks, needs_grad):
+                cp_segment_chunks, needs_grad, qk_l2norm):
         states = chunk_states(q, v, cu_seqlens) if needs_grad else None
         o, hT = gdn_chunk_fwd(q, k, v, g, beta, scale, initial_state, cu_seqlens,
                               output_final_state=output_final_state,
-                              cp_segment_chunks=cp_segment_chunks, states=states)
+                              cp_segment_chunks=cp_segment_chunks, states=states, qk_l2norm=qk_l2norm)
         ctx.set_materialize_grads(False)
         ctx.scale = scale
+        ctx.qk_l2norm = qk_l2norm
         ctx.cp_segment_chunks = cp_segment_chunks
         ctx.want_dh0 = initial_state is not None and ctx.needs_input_grad[6]
         ctx.save_for_backward(q, k, v, g, beta, initial_state, cu_seqlens, states)
@@ -50,9 +51,17 @@ class _ChunkGatedDeltaRule(torch.autograd.Function):
         gr = gdn_chunk_bwd(q, k, v, g, beta, do.contiguous(), ctx.scale, h0,
                            None if dht is None else dht.contiguous(), cu_seqlens,
                            cp_segment_chunks=ctx.cp_segment_chunks, want_dh0=ctx.want_dh0,
-                           states=states)
+                           states=states, qk_l2norm=ctx.qk_l2norm)
         return (gr["dq"], gr["dk"], gr["dv"], gr["dg"], gr["dbeta"], None, gr["dh0"], None, None,
-                None, None)
+                None, None, None)
+
+
+def _host_cu_seqlens(cu: torch.Tensor, T: int) -> None:
+    """Check a host-side cu_seqlens before it goes to the device: the kernels only report an
+    inconsistent one through their status word, after the fact."""
+    c = cu.tolist()
+    if not c or c[0] != 0 or c[-1] != T or any(b < a for a, b in zip(c, c[1:])):
+        raise ValueError(f"cu_seqlens must rise from 0 to T={T} without decreasing, got {c[:8]}...")
 
 
 def chunk_gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
@@ -73,21 +82,24 @@ def chunk_gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g:
     [N,Hv,dk,dv] fp32, else None.
 
     Gradients flow to q, k, v, g, beta and initial_state; the backward supports bf16 with
-    dk = dv = 128 (the forward supports dk, dv in {64, 128} in bf16 and fp32). q/k L2
-    normalisation inside the op is not implemented: normalise before the call.
+    dk = dv = 128 (the forward supports dk, dv in {64, 128} in bf16 and fp32).
+    use_qk_l2norm_in_kernel: q and k rows are divided by sqrt(|x|^2 + 1e-6) inside the kernels
+    (bf16, dk = dv = 128), and their gradients are taken through that normalisation. A cu_seqlens
+    on the host is checked before it is copied to the device; one already on the device is not
+    (the kernels report an inconsistent one only through their status word).
     """
-    if use_qk_l2norm_in_kernel:
-        raise NotImplementedError("use_qk_l2norm_in_kernel: normalise q and k before the call")
     for t, name in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta")):
         if not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
     q, k, v, g, beta = (t.contiguous() for t in (q, k, v, g, beta))
     if initial_state is not None:
         initial_state = initial_state.contiguous()
-    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
-        if cu_seqlens.dtype != torch.int64:
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype not in (torch.int32, torch.int64):
             raise TypeError("cu_seqlens must be int32 or int64")
-        cu_seqlens = cu_seqlens.to(torch.int32)
+        if not cu_seqlens.is_cuda:
+            _host_cu_seqlens(cu_seqlens, q.shape[1])
+        cu_seqlens = cu_seqlens.to(device=q.device, dtype=torch.int32).contiguous()
     scale = q.shape[-1] ** -0.5 if scale is None else float(scale)
     needs_grad = torch.is_grad_enabled() and (
         any(t.requires_grad for t in (q, k, v, g, beta))
@@ -95,4 +107,5 @@ def chunk_gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g:
     if needs_grad and not backward_supported(q, v):
         raise NotImplementedError("backward: bf16 with dk = dv = 128 only")
     return _ChunkGatedDeltaRule.apply(q, k, v, g, beta, scale, initial_state, output_final_state,
-                                      cu_seqlens, int(cp_segment_chunks), needs_grad)
+                                      cu_seqlens, int(cp_segment_chunks), needs_grad,
+                                      bool(use_qk_l2norm_in_kernel))

@@ -66,6 +66,47 @@ int num_sms() {
 
 bool uses_tc(gdn_dtype dtype, const Shape& s) { return dtype == GDN_BF16 && s.dk == 128 && s.dv == 128; }
 
+// The caller's options with the defaults (all zero) filled in; GDN_ERR_INVALID_ARG for a value
+// outside its range.
+gdn_status read_options(const gdn_options* opt, gdn_options& o) {
+  o = gdn_options{};
+  if (opt) o = *opt;
+  for (int r : o.reserved)
+    if (r != 0) return GDN_ERR_INVALID_ARG;
+  if (o.deterministic != 0 && o.deterministic != 1) return GDN_ERR_INVALID_ARG;
+  if (o.qk_l2norm != 0 && o.qk_l2norm != 1) return GDN_ERR_INVALID_ARG;
+  if (o.test_stall != 0 && o.test_stall != 1) return GDN_ERR_INVALID_ARG;
+  if (o.cp_mode < -1) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+// Segment length (chunks) the options ask for: n > 0 segments of n chunks, -1 off, 0 automatic.
+// cp_segment_chunks, when nonzero, wins; cp_mode = n > 0 gives at most n segments per sequence.
+int segment_option(const Shape& s, const gdn_options* opt) {
+  if (!opt) return 0;
+  if (opt->cp_segment_chunks != 0) return opt->cp_segment_chunks < 0 ? -1 : opt->cp_segment_chunks;
+  if (opt->cp_mode < 0) return -1;
+  if (opt->cp_mode > 0) {
+    const int nch = (s.T + kChunk - 1) / kChunk;
+    return nch > 0 ? (nch + opt->cp_mode - 1) / opt->cp_mode : -1;
+  }
+  return 0;
+}
+
+// Status of a device status word's code.
+gdn_status device_code_status(int code) {
+  switch (code) {
+    case kDevOk: return GDN_OK;
+    case kDevTimeout: return GDN_ERR_DEVICE_TIMEOUT;
+    case kDevMisaligned: return GDN_ERR_DEVICE_LAUNCH;
+    default: return GDN_ERR_DEVICE_INPUT;
+  }
+}
+
+// Row coordinates of the per-chunk state arrays (slots x Hv x 128 rows) are 32-bit TMA
+// coordinates: refuse sizes whose last row does not fit.
+bool state_rows_fit(long long slots, int Hv) { return slots * Hv * 128LL < (1LL << 31); }
+
 // Segment length (chunks) for automatic context parallelism, 0 = none. Independent
 // sequences: the segment count minimising waves x (segment chunks + 1 warm-up chunk),
 // with one CTA per SM per wave. Packed sequences (lengths unknown on the host): segments
@@ -99,7 +140,7 @@ FwdPlan plan_forward(gdn_dtype dtype, const Shape& s, const gdn_options* opt) {
     f.off_chunk_off = f.total;
     f.total = align256(f.total + (size_t)(s.N + 1) * sizeof(int));
   }
-  const int mode = opt ? opt->cp_segment_chunks : 0;
+  const int mode = segment_option(s, opt);
   if (mode < 0) return f;
   const int nch = (s.T + kChunk - 1) / kChunk;
   const int seg = mode > 0 ? mode : auto_segment(s, nch);
@@ -176,6 +217,25 @@ BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
   return b;
 }
 
+}  // namespace
+
+// The library's per-device status word (gdn_check_device_error): kernels record their first
+// finding here as well as in the call's workspace.
+__device__ int g_device_status;
+
+namespace {
+// Device address of the per-device status word on the current device, or nullptr when it cannot
+// be found (the call then records in its workspace only). Looked up on every call: the host-side
+// name of a __device__ variable is not a device address, and an address cached across a
+// cudaDeviceReset would be stale.
+int* device_status_word() {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return static_cast<int*>(ptr);
+}
 }  // namespace
 
 namespace gdn {
@@ -255,6 +315,7 @@ const char* gdn_status_string(gdn_status s) {
     case GDN_ERR_CUDA: return "CUDA runtime error";
     case GDN_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait timed out";
     case GDN_ERR_DEVICE_INPUT: return "a kernel found inconsistent device input (cu_seqlens)";
+    case GDN_ERR_DEVICE_LAUNCH: return "a kernel found its launch unusable (shared memory misaligned)";
   }
   return "unknown status";
 }
@@ -277,13 +338,15 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   Shape s;
   gdn_status st = check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, cu_seqlens != nullptr, s);
   if (st != GDN_OK) return st;
-  if (opt) {
-    for (int r : opt->reserved)
-      if (r != 0) return GDN_ERR_INVALID_ARG;
-  }
+  gdn_options op;
+  st = read_options(opt, op);
+  if (st != GDN_OK) return st;
+  opt = &op;
   if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
-  void* save_states = opt ? opt->states : nullptr;
-  if (save_states && !uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;
+  void* save_states = op.states;
+  if ((save_states || op.qk_l2norm) && !uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;
+  if (op.qk_l2norm) return GDN_ERR_UNSUPPORTED;   // NORM-TODO
+  if (save_states && !state_rows_fit(state_slots(s), s.Hv)) return GDN_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, o, hT, save_states};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
@@ -297,8 +360,11 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   p.status = static_cast<int*>(workspace);
   p.B = s.B; p.T = s.T; p.Hqk = s.Hqk; p.Hv = s.Hv; p.dk = s.dk; p.dv = s.dv; p.N = s.N;
   p.scale = scale;
+  p.qk_l2norm = op.qk_l2norm;
+  p.test_stall = op.test_stall;
 
   if (s.T == 0) return GDN_OK;
+  p.status_dev = device_status_word();
   cudaError_t err;
   if (uses_tc(dtype, s)) {
     const FwdPlan f = plan_forward(dtype, s, opt);
@@ -390,17 +456,19 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   Shape s;
   gdn_status st = check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, cu_seqlens != nullptr, s);
   if (st != GDN_OK) return st;
-  if (opt) {
-    for (int r : opt->reserved)
-      if (r != 0) return GDN_ERR_INVALID_ARG;
-  }
+  gdn_options op;
+  st = read_options(opt, op);
+  if (st != GDN_OK) return st;
+  opt = &op;
   if (T > 0 && (!q || !k || !v || !g || !beta || !dO || !dq || !dk_out || !dv_out || !dg || !dbeta))
     return GDN_ERR_INVALID_ARG;
-  const void* cached = opt ? opt->states : nullptr;
+  const void* cached = op.states;
   const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, dO, dhT, dq, dk_out, dv_out, dg, dbeta, dh0, cached};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
   if (!uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;   // backward: bf16, dk = dv = 128
+  if (op.qk_l2norm) return GDN_ERR_UNSUPPORTED;   // NORM-TODO
+  if (!state_rows_fit(state_slots(s), s.Hv)) return GDN_ERR_UNSUPPORTED;
   const BwdPlan bp = plan_backward(s, opt);
   if (!workspace || !aligned16(workspace) || workspace_bytes < bp.total) return GDN_ERR_WORKSPACE;
   if (s.T == 0) return GDN_OK;
@@ -410,8 +478,10 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.h0 = h0; p.cu = cu_seqlens;
   p.o = nullptr; p.hT = nullptr;
   p.status = static_cast<int*>(workspace);
+  p.status_dev = device_status_word();
   p.B = s.B; p.T = s.T; p.Hqk = s.Hqk; p.Hv = s.Hv; p.dk = s.dk; p.dv = s.dv; p.N = s.N;
   p.scale = scale;
+  p.qk_l2norm = op.qk_l2norm;
   p.states = cached ? static_cast<__nv_bfloat16*>(const_cast<void*>(cached))
                     : reinterpret_cast<__nv_bfloat16*>(ws + bp.off_states);
   p.chunk_off = s.packed ? reinterpret_cast<int*>(ws + bp.off_chunk_off) : nullptr;
@@ -484,11 +554,21 @@ gdn_status gdn_read_device_status(void* workspace, cudaStream_t stream) {
   const int zero = 0;
   if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return GDN_ERR_CUDA;
-  switch (code) {
-    case kDevOk: return GDN_OK;
-    case kDevTimeout: return GDN_ERR_DEVICE_TIMEOUT;
-    default: return GDN_ERR_DEVICE_INPUT;
+  return device_code_status(code);
+}
+
+gdn_status gdn_check_device_error(cudaStream_t stream) {
+  cudaError_t err = cudaStreamSynchronize(stream);
+  if (err != cudaSuccess) return cuda_fail("gdn_check_device_error: stream", err);
+  int code = 0;
+  err = cudaMemcpyFromSymbol(&code, g_device_status, sizeof(int));
+  if (err != cudaSuccess) return cuda_fail("gdn_check_device_error: read", err);
+  if (code != 0) {
+    const int zero = 0;
+    err = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    if (err != cudaSuccess) return cuda_fail("gdn_check_device_error: clear", err);
   }
+  return device_code_status(code);
 }
 
 }  // extern "C"

@@ -83,7 +83,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   Small* ss = reinterpret_cast<Small*>(sm + kOffSmall);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if ((smem_u32(sm) & 1023u) != 0) {
-    if (threadIdx.x == 0) record_error(p.status, kDevTimeout);
+    if (threadIdx.x == 0) report_error(p, kDevMisaligned);
     return;
   }
   // decode the work item with h0/hT hidden: dhT / dh0 belong to the other ends here
@@ -431,7 +431,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) record_error(p.status, kDevTimeout);
+  if (threadIdx.x == 0 && *abort_flag) report_error(p, kDevTimeout);
 }
 
 cudaError_t launch_bwd_chain(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st,

@@ -118,7 +118,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, hh = warp >> 2;
   if ((smem_u32(sm) & 1023u) != 0) {
-    if (tid == 0) record_error(p.status, kDevTimeout);
+    if (tid == 0) report_error(p, kDevMisaligned);
     return;
   }
   if (tid == 0) {
@@ -791,7 +791,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
     volatile int never = 0;
     mbar_wait(&ss->tma_bar, tph ^ 1, &never);
-    record_error(p.status, kDevTimeout);
+    report_error(p, kDevTimeout);
   }
   tc_fence_before();
   __syncthreads();

@@ -18,6 +18,7 @@ enum DeviceError : int {
   kDevOk = 0,
   kDevTimeout = 1,       // a bounded mbarrier wait gave up
   kDevBadSeqlens = 2,    // cu_seqlens not monotone / not ending at T
+  kDevMisaligned = 3,    // dynamic shared memory not at the 1024-byte alignment the swizzled tiles need
 };
 
 // Everything a forward kernel needs. Pointers are device pointers.
@@ -31,7 +32,10 @@ struct FwdParams {
   const int32_t* cu;        // nullable, [N+1]
   void* o;                  // nullable (no output written)
   float* hT;                // nullable
-  int* status;              // device status word
+  int* status;              // device status word (head of the caller's workspace)
+  int* status_dev;          // nullable: the library's per-device status word (gdn_check_device_error)
+  int qk_l2norm;            // q, k rows divided by sqrt(|x|^2 + eps) inside the kernels
+  int test_stall;           // testing only: the tensor-core forward's CTAs wait once on a barrier nothing completes
   // backward support: bf16 start state S (dv x dk, row-major) of every chunk, at
   // states + ((chunk_off[n] + chunk) * Hv + j) * dv * dk; chunk_off nullable -> n * ceil(T/64)
   __nv_bfloat16* states;    // nullable
@@ -49,6 +53,12 @@ struct FwdParams {
 
 __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+// Record a device-side finding in the call's workspace status word and in the library's
+// per-device word (first error wins in each).
+__device__ __forceinline__ void report_error(const FwdParams& p, int code) {
+  record_error(p.status, code);
+  record_error(p.status_dev, code);
 }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
@@ -75,11 +85,11 @@ __device__ __forceinline__ bool seq_span(const FwdParams& p, int n, int& b, int&
   s = p.cu[n];
   e = p.cu[n + 1];
   if (s < 0 || e < s || e > p.T) {
-    record_error(p.status, kDevBadSeqlens);
+    report_error(p, kDevBadSeqlens);
     return false;
   }
   if ((n == 0 && s != 0) || (n == p.N - 1 && e != p.T)) {
-    record_error(p.status, kDevBadSeqlens);
+    report_error(p, kDevBadSeqlens);
     return false;
   }
   return true;

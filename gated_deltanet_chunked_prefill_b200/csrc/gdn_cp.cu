@@ -28,7 +28,7 @@ gdn_cp_plan_kernel(const FwdParams p, int seg_chunks, int max_pairs, int2* table
   for (int n = n0; n < n1; ++n) {
     int lo = p.cu[n], hi = p.cu[n + 1];
     if (lo < 0 || hi < lo || hi > p.T) {
-      record_error(p.status, kDevBadSeqlens);
+      report_error(p, kDevBadSeqlens);
       hi = lo = 0;
     }
     const int ch = (hi - lo + kChunk - 1) / kChunk;
@@ -83,7 +83,7 @@ gdn_cp_plan_kernel(const FwdParams p, int seg_chunks, int max_pairs, int2* table
   if (tid == kPlanThreads - 1) {
     const int total = part[tid];
     if (count) *count = min(total, max_pairs);
-    if ((table && total > max_pairs) || p.cu[0] != 0 || p.cu[p.N] != p.T) record_error(p.status, kDevBadSeqlens);
+    if ((table && total > max_pairs) || p.cu[0] != 0 || p.cu[p.N] != p.T) report_error(p, kDevBadSeqlens);
   }
 }
 

@@ -64,11 +64,13 @@ struct Small {
   float wsum[16];         // warm-up window search: per-warp partial sums
   int ws;                 // warm-up start token (context parallelism)
   uint64_t full_k[2], full_qv[2], prep_full[2], gdone, wdone, mma_done, dd_free;
+  uint64_t stall;         // testing only: a barrier that nothing completes
   uint32_t tmem_base;
   int abort_flag;
 };
 constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a block can opt into");
+constexpr long long kStallCycles = 1LL << 21;   // ~1 ms: limit of the testing hook's wait
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t kColGW = 0;      // 2 x 128 by chunk parity: [K;Q] K^T (64 cols); then
@@ -101,7 +103,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if ((smem_u32(sm) & 1023u) != 0) {                     // 128B-swizzled tiles need 1024B alignment
-    if (threadIdx.x == 0) record_error(p.status, kDevTimeout);
+    if (threadIdx.x == 0) report_error(p, kDevMisaligned);
     return;
   }
   WorkItem it;
@@ -118,6 +120,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(&ss->wdone, 1);
     mbar_init(&ss->dd_free, 1);
     mbar_init(&ss->mma_done, 1);
+    mbar_init(&ss->stall, 1);
     ss->abort_flag = 0;
     ss->ws = it.s;
     fence_mbar_init();
@@ -134,6 +137,17 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+
+  // Testing hook: one thread waits on a barrier that nothing completes. The wait gives up
+  // after ~1 ms and the CTA reports a timed-out wait; the chunk work below then runs as usual
+  // (its own waits keep their normal limit), so the context stays usable.
+  if (p.test_stall) {
+    if (threadIdx.x == 0) {
+      volatile int stall_flag = 0;
+      if (!mbar_wait_limit(&ss->stall, 0, &stall_flag, kStallCycles)) report_error(p, kDevTimeout);
+    }
+    __syncthreads();
+  }
 
   // Gate-driven warm-up (context parallelism): a segment that starts inside a sequence
   // begins from a zero state at the start of a window of earlier chunks whose transition
@@ -613,7 +627,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) record_error(p.status, kDevTimeout);
+  if (threadIdx.x == 0 && *abort_flag) report_error(p, kDevTimeout);
 }
 
 // ---------------------------------------------------------------- host side

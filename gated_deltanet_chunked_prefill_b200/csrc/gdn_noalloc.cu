@@ -25,7 +25,17 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // a device address, so it is looked up once per device (with that device current).
 gdn_status scratch_address(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
+  const cudaError_t derr = cudaGetDevice(&dev);
+  if (derr != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    char msg[160];
+    if (derr != cudaSuccess)
+      snprintf(msg, sizeof(msg), "gdn_chunk_fwd_noalloc: cudaGetDevice: %s", cudaGetErrorString(derr));
+    else
+      snprintf(msg, sizeof(msg), "gdn_chunk_fwd_noalloc: device index %d beyond the %d the library tracks", dev,
+               kMaxDevices);
+    gdn::set_last_error(msg);
+    return GDN_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
@@ -61,7 +71,13 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int H
   gdn_status st = scratch_address(&scratch);
   if (st != GDN_OK) return st;
   // the status word must start at zero; the rest of the scratch is rewritten by every call
-  if (cudaMemsetAsync(scratch, 0, gdn::kStatusBytes, stream) != cudaSuccess) return GDN_ERR_CUDA;
+  const cudaError_t merr = cudaMemsetAsync(scratch, 0, gdn::kStatusBytes, stream);
+  if (merr != cudaSuccess) {
+    char msg[160];
+    snprintf(msg, sizeof(msg), "gdn_chunk_fwd_noalloc: clearing the status word: %s", cudaGetErrorString(merr));
+    gdn::set_last_error(msg);
+    return GDN_ERR_CUDA;
+  }
   return gdn_chunk_fwd(dtype, B, T, Hqk, Hv, dk, dv, q, k, v, g, beta, scale, h0, cu_seqlens, num_seqs, o, hT,
                        scratch, kNoAllocScratchBytes, opt, stream);
 }

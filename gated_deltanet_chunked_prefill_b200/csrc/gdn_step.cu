@@ -18,8 +18,10 @@
 namespace gdn {
 namespace {
 
-constexpr int kRows = 4;   // thread rows splitting dk
-constexpr int kCols = 64;  // columns of h per CTA
+// Columns of h per CTA (64, or 32 at dk = 256) and thread rows splitting dk (4, or 8 at dk = 256):
+// 256 threads per CTA, each holding at most 32 entries of its column, two CTAs per SM.
+template <int DK> constexpr int cols_for() { return DK == 256 ? 32 : 64; }
+template <int DK> constexpr int rows_for() { return DK == 256 ? 8 : 4; }
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -27,10 +29,12 @@ __device__ __forceinline__ void from_f(float* p, float x) { *p = x; }
 __device__ __forceinline__ void from_f(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kCols * kRows, 2)
+__global__ void __launch_bounds__(cols_for<DK>() * rows_for<DK>(), 2)
 gdn_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const float* __restrict__ g, const T* __restrict__ beta, float scale,
                 float* __restrict__ state, T* __restrict__ o, int Hqk, int Hv) {
+  constexpr int kRows = rows_for<DK>();
+  constexpr int kCols = cols_for<DK>();
   constexpr int kPer = DK / kRows;            // dk entries of one column per thread
   __shared__ float ks[DK], qs[DK];
   constexpr int kSplit = DV / kCols;          // CTAs per (sequence, v-head)
@@ -87,7 +91,8 @@ template <typename T, int DK, int DV>
 cudaError_t launch_step(const void* q, const void* k, const void* v, const float* g, const void* beta,
                         float scale, float* state, void* o, int N, int Hqk, int Hv, cudaStream_t st) {
   trace_pre(kKernStep, st);
-  gdn_step_kernel<T, DK, DV><<<(unsigned)N * (unsigned)Hv * (DV / kCols), dim3(kCols, kRows), 0, st>>>(
+  constexpr int kCols = cols_for<DK>();
+  gdn_step_kernel<T, DK, DV><<<(unsigned)N * (unsigned)Hv * (DV / kCols), dim3(kCols, rows_for<DK>()), 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, static_cast<const T*>(beta),
       scale, state, static_cast<T*>(o), Hqk, Hv);
   const cudaError_t err = cudaGetLastError();
@@ -95,15 +100,24 @@ cudaError_t launch_step(const void* q, const void* k, const void* v, const float
   return err;
 }
 
+template <typename T, int DK>
+cudaError_t launch_step_dv(int dv, const void* q, const void* k, const void* v, const float* g, const void* beta,
+                           float scale, float* state, void* o, int N, int Hqk, int Hv, cudaStream_t st) {
+  if (dv == 256) return launch_step<T, DK, 256>(q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
+  if (dv == 128) return launch_step<T, DK, 128>(q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
+  return launch_step<T, DK, 64>(q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
+}
+
 template <typename T>
 cudaError_t launch_step_dims(int dk, int dv, const void* q, const void* k, const void* v, const float* g,
                              const void* beta, float scale, float* state, void* o, int N, int Hqk, int Hv,
                              cudaStream_t st) {
-  if (dk == 128 && dv == 128) return launch_step<T, 128, 128>(q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
-  if (dk == 128 && dv == 64) return launch_step<T, 128, 64>(q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
-  if (dk == 64 && dv == 128) return launch_step<T, 64, 128>(q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
-  return launch_step<T, 64, 64>(q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
+  if (dk == 256) return launch_step_dv<T, 256>(dv, q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
+  if (dk == 128) return launch_step_dv<T, 128>(dv, q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
+  return launch_step_dv<T, 64>(dv, q, k, v, g, beta, scale, state, o, N, Hqk, Hv, st);
 }
+
+bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
 
 bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -116,8 +130,9 @@ extern "C" gdn_status gdn_recurrent_step(gdn_dtype dtype, int N, int Hqk, int Hv
                                          cudaStream_t stream) {
   if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
   if (N < 0 || Hqk < 1 || Hv < 1 || Hv % Hqk != 0) return GDN_ERR_INVALID_ARG;
-  if ((long long)N * Hv >= (1LL << 30)) return GDN_ERR_UNSUPPORTED;   // grid: N Hv dv / 64 blocks
-  if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED;
+  if (!gdn::head_dim_ok(dk) || !gdn::head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+  // grid: N Hv dv / (64, or 32 at dk = 256) blocks
+  if ((long long)N * Hv * (dv / (dk == 256 ? 32 : 64)) >= (1LL << 31)) return GDN_ERR_UNSUPPORTED;
   if (N == 0) return GDN_OK;
   const void* ptrs[] = {q, k, v, g, beta, state, o};
   for (const void* p : ptrs)

@@ -43,7 +43,9 @@
  *     validated on the host before anything is launched; an invalid call
  *     returns an error status and touches no output. Errors a kernel detects
  *     (an inconsistent cu_seqlens, a bounded wait that timed out) are recorded
- *     in the workspace's status word and reported by gdn_read_device_status().
+ *     in the workspace's status word, reported by gdn_read_device_status(), and
+ *     in a per-device word, reported by gdn_check_device_error(). Outputs of a
+ *     call whose kernels recorded an error are unspecified.
  *   - Launch failures return GDN_ERR_CUDA.
  */
 #ifndef GDN_H_
@@ -64,16 +66,27 @@ typedef enum {
   GDN_ERR_WORKSPACE = 3,       /* workspace null, too small or misaligned                              */
   GDN_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed                                 */
   GDN_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait gave up (reported via the status word)       */
-  GDN_ERR_DEVICE_INPUT = 6     /* a kernel found device-side input inconsistent (cu_seqlens)          */
+  GDN_ERR_DEVICE_INPUT = 6,    /* a kernel found device-side input inconsistent (cu_seqlens)          */
+  GDN_ERR_DEVICE_LAUNCH = 7    /* a kernel found its launch unusable (dynamic shared memory misaligned) */
 } gdn_status;
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /* Optional knobs; pass NULL for the defaults (all zero). */
 typedef struct {
-  /* Intra-card context parallelism (tensor-core path): 0 = automatic (split a
-   * sequence into segments when (sequences x v-heads) leaves SMs idle), -1 = off,
-   * n > 0 = segments of n chunks (64 tokens each). */
+  /* Intra-card context parallelism on the tensor-core path ("FlashQLA resource", section 3,
+   * "Gate-driven automatic intra-card context parallelism"):
+   *   0 = automatic: sequences are split into segments when (sequences x v-heads) leaves SMs
+   *       idle; -1 = off; n > 0 = at most n segments per sequence, each of ceil(ceil(T / 64) / n)
+   *       chunks (T = B's sequence length, or the packed total). */
+  int cp_mode;
+  /* 0 or 1 (anything else: GDN_ERR_INVALID_ARG). Every kernel of this library reduces in a
+   * fixed order (no floating-point atomics, fixed per-producer slots), so results are
+   * bit-reproducible from run to run whatever the value; 1 is accepted for callers that ask
+   * for determinism explicitly and changes nothing. */
+  int deterministic;
+  /* Finer control of the segment length, overriding cp_mode when nonzero: n > 0 = segments
+   * of n chunks (64 tokens each), -1 = off. */
   int cp_segment_chunks;
   /* How a segment obtains its start state.
    * 0 (default): gate-driven. The segment's CTA runs, from a zero state, the
@@ -83,7 +96,8 @@ typedef struct {
    *   chunks it starts at the sequence start (the plain recurrence).
    * 1: exact affine stitch. Phase 1 computes every segment's map
    *   h_end = M h_start + b, phase 2 chains the maps, phase 3 reruns each segment
-   *   from its stitched start state. */
+   *   from its stitched start state. The backward mirrors it on the state gradient:
+   *   dh_start = M'^T dh_end + c, chained from the sequence end. */
   int cp_exact;
   /* Chunk start states cached between a forward and its backward (tensor-core path:
    * bf16, dk = dv = 128), device memory of gdn_chunk_states_size() bytes, 16-byte
@@ -96,11 +110,22 @@ typedef struct {
    *     chunk's A = (I + L)^-1 (fp32, 64 x 64 row-major), then its P = lower_incl(Q K^T * E)
    *     (bf16, 64 x 64, 128-byte-swizzled rows), both in the same slot order.
    *   gdn_chunk_bwd reads them instead of running its forward pass; they must come
-   *     from gdn_chunk_fwd on the same q, k, v, g, beta, h0 and cu_seqlens.
+   *     from gdn_chunk_fwd on the same q, k, v, g, beta, h0, cu_seqlens and qk_l2norm.
    * Set on another path: GDN_ERR_UNSUPPORTED; not 16-byte aligned: GDN_ERR_INVALID_ARG. */
   void* states;
+  /* 1: every q and k row is L2-normalised inside the kernels, x / sqrt(|x|^2 + 1e-6), and the
+   * backward returns the gradients with respect to the raw (unnormalised) q and k. 0: q and k
+   * are used as given. Tensor-core path only (bf16, dk = dv = 128); elsewhere
+   * GDN_ERR_UNSUPPORTED. */
+  int qk_l2norm;
+  /* Testing only; must be 0 in production. 1: every CTA of the forward's tensor-core kernel
+   * first waits on a barrier that nothing completes; the wait gives up after about 1 ms and
+   * records GDN_ERR_DEVICE_TIMEOUT (in the workspace's status word and the per-device word),
+   * then the call completes its work as usual. It lets a test see a bounded wait run out
+   * without faulting or hanging the GPU. */
+  int test_stall;
   /* Reserved, must be 0. */
-  int reserved[4];
+  int reserved[2];
 } gdn_options;
 
 /* Bytes of the chunk-state cache (gdn_options.states) for these sizes. */
@@ -163,9 +188,9 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
  *   g     [N, Hv] fp32 (raw log-decay)   beta [N, Hv] (dtype)
  *   state [N, Hv, dk, dv] fp32, read and overwritten in place (the caller's h0/hT
  *         layout); it must not overlap the other arrays.
- * dk, dv in {64, 128}; dtype GDN_BF16 or GDN_F32 (fp32 arithmetic in both).
+ * dk, dv in {64, 128, 256} (any pair); dtype GDN_BF16 or GDN_F32 (fp32 arithmetic in both).
  * N = 0 is a no-op. Null or misaligned pointers, Hv not a multiple of Hqk:
- * GDN_ERR_INVALID_ARG; other head dims or N * Hv >= 2^30: GDN_ERR_UNSUPPORTED;
+ * GDN_ERR_INVALID_ARG; other head dims or N * Hv * dv / 64 >= 2^31: GDN_ERR_UNSUPPORTED;
  * launch failure: GDN_ERR_CUDA. Asynchronous on `stream`; needs no workspace.
  */
 gdn_status gdn_recurrent_step(gdn_dtype dtype, int N, int Hqk, int Hv, int dk, int dv,
@@ -186,7 +211,9 @@ gdn_status gdn_recurrent_step(gdn_dtype dtype, int N, int Hqk, int Hv, int dk, i
  * e.g. the exact affine stitch (cp_exact) on large inputs, return GDN_ERR_WORKSPACE
  * with the sizes in gdn_last_error(). The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress, once per device); make that first call before
- * any stream capture. All calls share the one array: calls that overlap on the GPU
+ * any stream capture. The address is kept for the life of the process: after a
+ * cudaDeviceReset the array is reloaded elsewhere, so do not use this entry point on a
+ * device that was reset. All calls share the one array: calls that overlap on the GPU
  * (concurrent streams) race and must not be issued. Each call clears the status word;
  * device-side findings (inconsistent cu_seqlens, a timed-out wait) are not reported
  * back through this entry point.
@@ -200,9 +227,18 @@ gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int Hqk, int Hv,
 
 /* Synchronises `stream`, then returns (and clears) the status word that the
  * kernels of earlier calls on this workspace recorded: GDN_OK,
- * GDN_ERR_DEVICE_TIMEOUT or GDN_ERR_DEVICE_INPUT. GDN_ERR_CUDA if the stream
- * itself reports an error. */
+ * GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_DEVICE_INPUT or GDN_ERR_DEVICE_LAUNCH.
+ * GDN_ERR_CUDA if the stream itself reports an error. */
 gdn_status gdn_read_device_status(void* workspace, cudaStream_t stream);
+
+/* Synchronises `stream`, then returns (and clears) the library's status word of the current
+ * device: the first device-side finding (GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_DEVICE_INPUT,
+ * GDN_ERR_DEVICE_LAUNCH) of any gdn_chunk_fwd / gdn_chunk_bwd / gdn_chunk_fwd_noalloc call on
+ * this device since the last check, whatever its workspace; GDN_OK if none. The word is found
+ * with cudaGetSymbolAddress on every call; a call that cannot find it (for instance the very
+ * first library call of a process made under stream capture) records only in its workspace.
+ * GDN_ERR_CUDA if the stream or a copy fails (detail in gdn_last_error()). */
+gdn_status gdn_check_device_error(cudaStream_t stream);
 
 /* Static, human-readable text of a status code. */
 const char* gdn_status_string(gdn_status s);

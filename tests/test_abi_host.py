@@ -71,8 +71,81 @@ def test_forward_rejects_invalid_arguments(kw, code):
 
 def test_forward_rejects_reserved_options():
     o = gdn.Options()
-    o.reserved[3] = 1
+    o.reserved[1] = 1
     assert _fwd(opt=o) == 1
+
+
+@pytest.mark.parametrize("field,value", [("deterministic", 2), ("qk_l2norm", -1), ("test_stall", 3),
+                                         ("cp_mode", -2)])
+def test_forward_rejects_option_values_out_of_range(field, value):
+    o = gdn.Options()
+    setattr(o, field, value)
+    assert _fwd(opt=o) == 1
+
+
+def test_deterministic_option_accepted():
+    """deterministic = 1 is accepted (every path already reduces in a fixed order): the call gets
+    past option validation to the workspace check."""
+    o = gdn.Options()
+    o.deterministic = 1
+    assert _fwd(opt=o, ws=None) == 3
+
+
+def test_cp_mode_gives_the_segment_count():
+    """cp_mode = n asks for at most n segments: the plan matches cp_segment_chunks of
+    ceil(chunks / n) (visible in the exact stitch's workspace, which holds per-segment maps)."""
+    dims = (1, 4096, 1, 1, 128, 128, 1)           # 64 chunks
+    for n, seg in ((4, 16), (3, 22), (64, 1)):
+        assert gdn.fwd_workspace_size(*dims, cp_mode=n, cp_exact=True) == \
+            gdn.fwd_workspace_size(*dims, cp_segment_chunks=seg, cp_exact=True)
+    assert gdn.fwd_workspace_size(*dims, cp_mode=-1, cp_exact=True) == \
+        gdn.fwd_workspace_size(*dims, cp_segment_chunks=-1, cp_exact=True) < \
+        gdn.fwd_workspace_size(*dims, cp_mode=2, cp_exact=True)
+    # cp_segment_chunks, when set, wins over cp_mode
+    assert gdn.fwd_workspace_size(*dims, cp_mode=4, cp_segment_chunks=8, cp_exact=True) == \
+        gdn.fwd_workspace_size(*dims, cp_segment_chunks=8, cp_exact=True)
+
+
+def test_interface_names():
+    """The calls and option fields of the interface exist under their names."""
+    L = gdn.lib()
+    for name in ("gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_chunk_fwd_workspace_size", "gdn_chunk_bwd_workspace_size",
+                 "gdn_status_string", "gdn_check_device_error", "gdn_read_device_status"):
+        assert hasattr(L, name), name
+    fields = [f[0] for f in gdn.Options._fields_]
+    assert fields[:2] == ["cp_mode", "deterministic"]
+    for code in range(8):
+        assert L.gdn_status_string(code) != b"unknown status"
+
+
+def test_state_rows_beyond_32_bit_coordinates_refused():
+    """Chunk-state rows (slots x Hv x 128) are 32-bit TMA coordinates: sizes whose rows do not fit
+    are refused on the host, for a forward that caches states and for the backward."""
+    T = 1 << 26                                   # B * T * H = 2^30 fits; 2^20 slots * 16 * 128 = 2^31 does not
+    o = gdn.Options()
+    o.states = FAKE
+    assert _fwd(T=T, Hqk=16, Hv=16, opt=o) == 2
+    assert _fwd(T=T, Hqk=16, Hv=16, opt=o, ws=None) == 2     # refused before the workspace check
+    L = gdn.lib()
+    vp = ctypes.c_void_p
+    f = vp(FAKE)
+    st = L.gdn_chunk_bwd(1, 1, T, 16, 16, 128, 128, f, f, f, f, f, 0.1, None, None, 1, f, None, f, f, f, f, f,
+                         None, f, 1 << 40, ctypes.byref(gdn.Options()), None)
+    assert st == 2
+
+
+def test_binding_refuses_a_states_cache_that_does_not_fit():
+    """The C ABI takes the chunk-state cache as a bare pointer; the binding checks its size and
+    device against the inputs first."""
+    from gated_deltanet_chunked_prefill_b200 import _check_states
+    q = torch.zeros(1, 256, 2, 128, dtype=torch.bfloat16)
+    v = torch.zeros(1, 256, 2, 128, dtype=torch.bfloat16)
+    need = gdn.lib().gdn_chunk_states_size(1, 256, 2, 2, 128, 128, 1)
+    _check_states(torch.zeros(need // 2, dtype=torch.bfloat16), q, v, None)
+    with pytest.raises(ValueError, match="bytes"):
+        _check_states(torch.zeros(need // 2 - 1, dtype=torch.bfloat16), q, v, None)
+    with pytest.raises(ValueError, match="device"):
+        _check_states(torch.zeros(need // 2, dtype=torch.bfloat16, device="meta"), q, v, None)
 
 
 def test_python_binding_refuses_cpu_tensors():
@@ -84,9 +157,11 @@ def test_python_binding_refuses_cpu_tensors():
 
 
 def test_options_struct_layout():
-    # int, int, pointer, int[4]: 32 bytes with the pointer at offset 8
-    assert ctypes.sizeof(gdn.Options) == 32
-    assert gdn.Options.states.offset == 8
+    # int cp_mode, deterministic, cp_segment_chunks, cp_exact; pointer; int qk_l2norm, test_stall,
+    # reserved[2]: 40 bytes with the pointer at offset 16
+    assert ctypes.sizeof(gdn.Options) == 40
+    assert gdn.Options.states.offset == 16
+    assert gdn.Options.qk_l2norm.offset == 24
 
 
 def test_chunk_states_size():
@@ -112,10 +187,13 @@ def test_autograd_entry_host_checks():
     """The autograd entry point refuses what it does not do before touching the GPU."""
     x = torch.zeros(1, 64, 1, 128)
     g = torch.zeros(1, 64, 1)
-    with pytest.raises(NotImplementedError):
-        gdn.chunk_gated_delta_rule(x, x, x, g, g, use_qk_l2norm_in_kernel=True)
     with pytest.raises(ValueError):
         gdn.chunk_gated_delta_rule(x, x, x, g, g)
+    from gated_deltanet_chunked_prefill_b200.autograd import _host_cu_seqlens
+    _host_cu_seqlens(torch.tensor([0, 3, 3, 10]), 10)
+    for bad in ([0, 5, 3, 10], [1, 10], [0, 9]):
+        with pytest.raises(ValueError, match="cu_seqlens"):
+            _host_cu_seqlens(torch.tensor(bad), 10)
     from gated_deltanet_chunked_prefill_b200.autograd import backward_supported
     assert backward_supported(x.to(torch.bfloat16), x)
     assert not backward_supported(x, x)                                   # fp32
@@ -132,6 +210,8 @@ def test_recurrent_step_host_validation():
     assert call(1, 1, 2, 3, 128, 128, p) == 1                # Hv not a multiple of Hqk
     assert call(1, -1, 1, 1, 128, 128, p) == 1               # negative N
     assert call(1, 1, 1, 1, 96, 128, p) == 2                 # unsupported head dim
+    assert call(1, 1, 1, 1, 128, 512, p) == 2
+    assert call(1, 1 << 28, 1, 2, 256, 256, p) == 2          # grid of N * Hv * dv / 64 blocks beyond 2^31 - 1
     assert call(1, 1, 1, 1, 128, 128, None) == 1             # null pointers
     assert call(1, 1, 1, 1, 128, 128, ctypes.c_void_p(24)) == 1   # misaligned
     assert call(1, 0, 1, 1, 128, 128, None) == 0             # N = 0: nothing to do

@@ -135,10 +135,51 @@ def test_fwd_bad_cu_seqlens_reports_device_status():
     d["cu_seqlens"] = torch.tensor([0, 100, 64], dtype=torch.int32, device="cuda")  # not monotone
     ws = torch.zeros(gdn.fwd_workspace_size(1, 128, 1, 1, 128, 128, 2), dtype=torch.uint8,
                      device="cuda")
+    gdn.check_device_error()                        # start from a clear per-device word
     gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, d["cu_seqlens"],
-                      workspace=ws)
+                      workspace=ws, check_status=False)
     assert gdn.read_device_status(ws) == 6
     assert gdn.read_device_status(ws) == 0          # reading clears it
+    assert gdn.check_device_error() == 6            # the per-device word saw it too
+    assert gdn.check_device_error() == 0
+    with pytest.raises(gdn.GdnError, match="inconsistent device input"):
+        gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, d["cu_seqlens"],
+                          workspace=ws, check_status=True)
+    gdn.check_device_error()
+
+
+def test_fwd_bounded_wait_times_out_and_context_stays_usable():
+    """The testing hook makes one thread of every CTA wait on a barrier that nothing completes:
+    the wait gives up after ~1 ms, the call reports GDN_ERR_DEVICE_TIMEOUT through the workspace
+    and the per-device status word, and the next call on the same context works."""
+    x = make_inputs(1, 300, 2, 2, 128, 128, "bf16", seed=21, h0_std=0.1)
+    d = to_dev(x)
+    ws = torch.zeros(gdn.fwd_workspace_size(1, 300, 2, 2, 128, 128, 1), dtype=torch.uint8, device="cuda")
+    gdn.check_device_error()
+    gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"], workspace=ws,
+                      test_stall=True, check_status=False)
+    assert gdn.read_device_status(ws) == 5
+    assert gdn.check_device_error() == 5
+    assert gdn.check_device_error() == 0
+    o, hT = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"], workspace=ws,
+                              check_status=True)
+    torch.cuda.synchronize()
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"], None, chunk=64)
+    assert_close(o.cpu(), ro, "bf16", "o after a timed-out call")
+    assert_close(hT.cpu(), rh, "bf16", "hT after a timed-out call")
+    assert gdn.check_device_error() == 0
+
+
+def test_fwd_cp_mode_segments_and_deterministic_flag():
+    """cp_mode = n (at most n segments per sequence) and deterministic = 1 give the oracle's
+    result; with the same segmentation the output is bit-identical to cp_segment_chunks."""
+    x = make_inputs(1, 1500, 2, 2, 128, 128, "bf16", seed=13, h0_std=0.1)
+    o1, h1 = run_gpu(x, cp_mode=4, deterministic=True)
+    o2, h2 = run_gpu(x, cp_segment_chunks=6)         # 24 chunks / 4 segments
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"], None, chunk=64)
+    assert_close(o1, ro, "bf16", "o")
+    assert_close(h1, rh, "bf16", "hT")
 
 
 # ---------------------------------------------------------------- full-size configurations

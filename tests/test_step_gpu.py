@@ -20,6 +20,10 @@ CASES = {
     "f32_d64": (4, 1, 2, 64, 64, "f32"),
     "f32_dk128_dv64": (2, 1, 1, 128, 64, "f32"),
     "f32_dk64_dv128": (2, 1, 1, 64, 128, "f32"),
+    "bf16_d256": (3, 1, 2, 256, 256, "bf16"),
+    "f32_d256": (2, 1, 1, 256, 256, "f32"),
+    "f32_dk256_dv64": (2, 1, 1, 256, 64, "f32"),
+    "bf16_dk64_dv256_gqa": (2, 1, 2, 64, 256, "bf16"),
 }
 
 
