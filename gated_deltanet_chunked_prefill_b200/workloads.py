@@ -91,13 +91,14 @@ def _l2norm(x: np.ndarray) -> np.ndarray:
 
 def make_inputs(B: int, T: int, Hqk: int, Hv: int, dk: int, dv: int, dtype: str,
                 seed: int, h0_std: Optional[float] = None, lengths=None,
-                backward: bool = False, g_scale: float = 1.0) -> dict:
+                backward: bool = False, g_scale: float = 1.0, qk_unit: bool = True) -> dict:
     """Draw one seeded input set (CPU tensors).
 
     Returns a dict with q, k [B,T,Hqk,dk], v [B,T,Hv,dv], beta [B,T,Hv] in the I/O
     dtype; g [B,T,Hv] fp32; h0 [N,Hv,dk,dv] fp32 or None; cu_seqlens int32 [N+1]
     or None; and, when backward, dO [B,T,Hv,dv] (I/O dtype) and dhT [N,Hv,dk,dv]
     fp32. `g_scale` multiplies the N(0,1) draw inside logsigmoid (1.0 = recipe).
+    qk_unit=False leaves q and k as drawn, N(0, 1) (for the operator's own normalisation).
     """
     rng = np.random.default_rng(seed)
     if lengths is not None:
@@ -112,8 +113,9 @@ def make_inputs(B: int, T: int, Hqk: int, Hv: int, dk: int, dv: int, dtype: str,
     else:
         N = B
         cu_seqlens = None
-    q = _l2norm(rng.standard_normal((B, T, Hqk, dk)))
-    k = _l2norm(rng.standard_normal((B, T, Hqk, dk)))
+    unit = _l2norm if qk_unit else (lambda a: a)
+    q = unit(rng.standard_normal((B, T, Hqk, dk)))
+    k = unit(rng.standard_normal((B, T, Hqk, dk)))
     v = rng.standard_normal((B, T, Hv, dv))
     xg = rng.standard_normal((B, T, Hv)) * g_scale
     g = -np.logaddexp(0.0, -xg)                      # logsigmoid, <= 0

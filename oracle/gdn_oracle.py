@@ -23,7 +23,8 @@ layout of the h0 / hT tensors [N, Hv, dk, dv]. With h = S^T one token step is
 Readings taken where the operator definition leaves a step open (each is the
 plainest one the formula supports):
   * g is the raw per-token log-decay; the operator forms the cumulative sums.
-  * q and k are used as given (normalisation belongs to the input recipe).
+  * q and k are used as given (normalisation belongs to the input recipe), unless
+    qk_l2norm asks for the in-operator normalisation below.
   * grouped values: v-head j reads q/k head j // (Hv // Hqk).
   * packed sequences: cu_seqlens = [0, cumsum(lengths)], B == 1; h0 / hT are
     per sequence. Sequences never interact.
@@ -36,12 +37,19 @@ Three independent forms:
                  substitution; chunk size is a parameter
   bwd_token   -- the exact adjoint of fwd_token, token by token in reverse
 
+Optional q/k normalisation (qk_l2norm=True on every form): rows of q and k become
+x / sqrt(|x|^2 + 1e-6) before the recurrence, and the backward maps the gradients back
+through that normalisation to the raw q and k.
+
 Pins (tests/test_oracle.py): the token and chunked forms agree to 1e-10 for
 every chunk size; beta=0, g=0, h0=0 gives zero; a single unit-norm write is
 retrieved exactly; decay-only inputs follow the closed form; tiny cases match
 exact rational brute force of the S-form with explicit matrices; the affine
 map in h0, linearity, resume, packed-vs-alone, a hand-derived worked example,
-and the backward against central finite differences and closed forms.
+and the backward against central finite differences and closed forms. The
+normalisation: the squared row norm s / (s + eps) in closed form, invariance of
+the outputs to a positive rescaling of each row, the gradients orthogonal to
+their rows, and central finite differences through it.
 """
 from __future__ import annotations
 
@@ -49,8 +57,20 @@ import numpy as np
 
 __all__ = [
     "as_f64", "sequences", "qk_head_of", "fwd_token", "fwd_chunk", "bwd_token",
-    "unit_lower_inverse",
+    "unit_lower_inverse", "l2norm", "L2NORM_EPS",
 ]
+
+# Optional normalisation of q and k inside the operator (the flash-linear-attention entry point's
+# use_qk_l2norm_in_kernel, which the pages say the library's entry signature follows): every
+# row x (one token of one q/k head) becomes x / sqrt(|x|^2 + eps). The pages fix no eps; 1e-6
+# keeps an all-zero row at zero instead of dividing by zero.
+L2NORM_EPS = 1e-6
+
+
+def l2norm(x, eps=L2NORM_EPS):
+    """Rows of x (last axis) divided by sqrt(sum of squares + eps), in fp64."""
+    x = as_f64(x)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
 
 
 def as_f64(x):
@@ -87,14 +107,17 @@ def _unpack(q, k, v, g, beta, h0):
 # --------------------------------------------------------------------------
 # token recurrence
 # --------------------------------------------------------------------------
-def fwd_token(q, k, v, g, beta, scale, h0=None, cu_seqlens=None):
+def fwd_token(q, k, v, g, beta, scale, h0=None, cu_seqlens=None, qk_l2norm=False):
     """Token-by-token recurrence.
 
     q, k: [B,T,Hqk,dk]; v: [B,T,Hv,dv]; g, beta: [B,T,Hv]; h0: [N,Hv,dk,dv] or None.
     Returns (o [B,T,Hv,dv], hT [N,Hv,dk,dv]) in fp64. Vectorised over heads only;
-    every token is one step of the recurrence in the module docstring.
+    every token is one step of the recurrence in the module docstring. qk_l2norm: q and k
+    rows are normalised first (l2norm).
     """
     q, k, v, g, beta, h0 = _unpack(q, k, v, g, beta, h0)
+    if qk_l2norm:
+        q, k = l2norm(q), l2norm(k)
     B, T, Hqk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     hm = qk_head_of(Hqk, Hv)
@@ -131,7 +154,7 @@ def unit_lower_inverse(L):
     return A
 
 
-def fwd_chunk(q, k, v, g, beta, scale, h0=None, cu_seqlens=None, chunk=64):
+def fwd_chunk(q, k, v, g, beta, scale, h0=None, cu_seqlens=None, chunk=64, qk_l2norm=False):
     """Chunk-parallel form of the same recurrence.
 
     For each sequence, v-head and chunk of n <= `chunk` tokens, with h the state
@@ -144,9 +167,12 @@ def fwd_chunk(q, k, v, g, beta, scale, h0=None, cu_seqlens=None, chunk=64):
         D     = U - W h                            (per-token residuals times beta)
         O     = scale [ diag(exp(gam)) Q h + (Q K^T * E * lower_incl) D ]
         h'    = exp(gam_n) h + (diag(exp(gam_n - gam)) K)^T D
-    Chunks never cross a sequence boundary; the last chunk may be partial.
+    Chunks never cross a sequence boundary; the last chunk may be partial. qk_l2norm: q and k
+    rows are normalised first (l2norm).
     """
     q, k, v, g, beta, h0 = _unpack(q, k, v, g, beta, h0)
+    if qk_l2norm:
+        q, k = l2norm(q), l2norm(k)
     B, T, Hqk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     hm = qk_head_of(Hqk, Hv)
@@ -196,7 +222,16 @@ def _head_forward_states(qh, kh, vh, gh, bh, h_init, ckpt):
     return saved, h
 
 
-def bwd_token(q, k, v, g, beta, scale, dO, h0=None, dhT=None, cu_seqlens=None, ckpt=64):
+def _l2norm_adjoint(x, dxn, eps=L2NORM_EPS):
+    """Gradient with respect to the raw rows x of a function of xn = l2norm(x), given its
+    gradient dxn with respect to xn: with r = (|x|^2 + eps)^(-1/2), xn = r x and
+    d xn / d x = r (I - xn xn^T), so dx = r (dxn - xn <xn, dxn>), row by row."""
+    r = 1.0 / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+    xn = r * x
+    return r * (dxn - xn * np.sum(xn * dxn, axis=-1, keepdims=True))
+
+
+def bwd_token(q, k, v, g, beta, scale, dO, h0=None, dhT=None, cu_seqlens=None, ckpt=64, qk_l2norm=False):
     """Exact adjoint of fwd_token, in reverse token order.
 
     Per token, with dh the adjoint of h_t carried from later tokens:
@@ -208,9 +243,13 @@ def bwd_token(q, k, v, g, beta, scale, dO, h0=None, dhT=None, cu_seqlens=None, c
     head are the sums over the v-heads that read it. Forward states are kept at
     every `ckpt` tokens and recomputed in between (memory, not arithmetic).
     Returns dict dq, dk [B,T,Hqk,dk]; dv [B,T,Hv,dv]; dg, dbeta [B,T,Hv];
-    dh0 [N,Hv,dk,dv] (fp64).
+    dh0 [N,Hv,dk,dv] (fp64). qk_l2norm: the recurrence runs on l2norm(q), l2norm(k), and the
+    returned dq, dk are taken with respect to the raw q, k through that normalisation.
     """
     q, k, v, g, beta, h0 = _unpack(q, k, v, g, beta, h0)
+    if qk_l2norm:
+        q_raw, k_raw = q, k
+        q, k = l2norm(q), l2norm(k)
     dO = as_f64(dO)
     dhT = as_f64(dhT)
     B, T, Hqk, dk = q.shape
@@ -260,4 +299,6 @@ def bwd_token(q, k, v, g, beta, scale, dO, h0=None, dhT=None, cu_seqlens=None, c
                     dg[b, s + t, j] = np.sum(dht * ht)
                     dh = np.exp(gh[t]) * dht
             dh0[n_seq, j] = dh
+    if qk_l2norm:
+        dq, dkk = _l2norm_adjoint(q_raw, dq), _l2norm_adjoint(k_raw, dkk)
     return dict(dq=dq, dk=dkk, dv=dvv, dg=dg, dbeta=db, dh0=dh0)

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import bwd_token, fwd_chunk, fwd_token, unit_lower_inverse
+from oracle import L2NORM_EPS, bwd_token, fwd_chunk, fwd_token, l2norm, unit_lower_inverse
 from gated_deltanet_chunked_prefill_b200.workloads import make_inputs
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -361,3 +361,129 @@ def test_pins_reject_planted_mistakes(fn_name, old, new):
     o1, h1 = call_fwd(fwd_token, x)
     o2, h2 = call_fwd(m["fwd_chunk"], x, chunk=16)
     assert rel(o2, o1) > 1e-6 or rel(h2, h1) > 1e-6
+
+
+# ---------------------------------------------------------------- q/k normalisation
+def test_l2norm_closed_form():
+    """|x / sqrt(s + eps)|^2 = s / (s + eps), the direction is kept, a zero row stays zero."""
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((5, 3, 16)) * rng.uniform(0.01, 10.0, (5, 3, 1))
+    y = l2norm(x)
+    s = np.sum(x * x, -1)
+    np.testing.assert_allclose(np.sum(y * y, -1), s / (s + L2NORM_EPS), rtol=1e-14)
+    np.testing.assert_allclose(y * np.sqrt(s + L2NORM_EPS)[..., None], x, rtol=1e-13)
+    assert np.all(l2norm(np.zeros((2, 4))) == 0.0)
+
+
+def _rescaled_rows(x, lo, hi, seed):
+    """q and k with every (token, head) row multiplied by its own factor in [lo, hi] (fp64)."""
+    rng = np.random.default_rng(seed)
+    out = dict(x)
+    for n in ("q", "k"):
+        a = x[n].double().numpy() if hasattr(x[n], "double") else np.asarray(x[n], dtype=np.float64)
+        out[n] = a * rng.uniform(lo, hi, a.shape[:-1] + (1,))
+    return out
+
+
+@pytest.mark.parametrize("form", [fwd_token, fwd_chunk])
+def test_l2norm_forward_row_scale_invariance(form):
+    """With the normalisation the outputs depend on each q/k row's direction only: rescaling every
+    row by its own positive factor (norms 10..90, where eps moves the result by < 1e-8) leaves o
+    and hT unchanged, and with unit rows the result is the plain one up to eps / 2."""
+    x = small(B=1, Hqk=1, Hv=2, dk=6, dv=5, seed=61, lengths=[20, 9, 33])
+    a = _rescaled_rows(x, 10.0, 30.0, 1)
+    b = _rescaled_rows(x, 40.0, 90.0, 2)
+    oa, ha = call_fwd(form, a, qk_l2norm=True)
+    ob, hb = call_fwd(form, b, qk_l2norm=True)
+    assert rel(oa, ob) < 1e-7 and rel(ha, hb) < 1e-7
+    o0, h0 = call_fwd(form, x)                  # rows already of unit norm
+    assert rel(oa, o0) < 2e-6 and rel(ha, h0) < 2e-6
+    assert rel(call_fwd(form, a)[0], o0) > 1.0  # without it the rescaling shows
+
+
+def test_l2norm_forms_agree():
+    x = small(B=2, T=45, Hqk=1, Hv=2, dk=6, dv=4, seed=62)
+    a = _rescaled_rows(x, 0.3, 5.0, 3)
+    o1, h1 = call_fwd(fwd_token, a, qk_l2norm=True)
+    o2, h2 = call_fwd(fwd_chunk, a, qk_l2norm=True, chunk=16)
+    assert rel(o2, o1) < 1e-10 and rel(h2, h1) < 1e-10
+
+
+def _loss_raw(x, dO, dhT, **over):
+    a = {n: x[n] for n in ("q", "k", "v", "g", "beta", "h0")}
+    a.update(over)
+    o, hT = fwd_token(a["q"], a["k"], a["v"], a["g"], a["beta"], x["scale"], a["h0"], x["cu_seqlens"],
+                      qk_l2norm=True)
+    return float(np.sum(o * dO) + np.sum(hT * dhT))
+
+
+def test_l2norm_backward_central_differences():
+    """Gradients with respect to the raw q and k, through the normalisation, against central
+    differences of <o, dO> + <hT, dhT> (grouped values: dq, dk sum over the v-heads)."""
+    x = small(B=1, T=7, Hqk=1, Hv=2, dk=3, dv=2, seed=83, backward=True, h0=0.5)
+    x = _rescaled_rows(x, 0.5, 3.0, 4)
+    dO = x["dO"].double().numpy(); dhT = x["dhT"].double().numpy()
+    gr = bwd_token(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["dO"], x["h0"], x["dhT"],
+                   ckpt=3, qk_l2norm=True)
+    eps = 1e-6
+    for n, gname in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("beta", "dbeta"), ("h0", "dh0")):
+        base = x[n].double().numpy() if hasattr(x[n], "double") else np.asarray(x[n], dtype=np.float64)
+        fd = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            p = base.copy(); p[idx] += eps
+            m = base.copy(); m[idx] -= eps
+            fd[idx] = (_loss_raw(x, dO, dhT, **{n: p}) - _loss_raw(x, dO, dhT, **{n: m})) / (2 * eps)
+        np.testing.assert_allclose(gr[gname], fd, rtol=1e-6, atol=1e-8, err_msg=n)
+
+
+def test_l2norm_gradients_orthogonal_to_rows():
+    """A function of x / |x| does not change along x: each raw row's gradient is orthogonal to the
+    row (up to the eps term, relative eps / |x|^2)."""
+    x = small(B=1, T=40, Hqk=1, Hv=2, dk=8, dv=4, seed=84, backward=True)
+    x = _rescaled_rows(x, 2.0, 5.0, 5)
+    gr = bwd_token(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["dO"], x["h0"], x["dhT"],
+                   qk_l2norm=True)
+    for n, gname in (("q", "dq"), ("k", "dk")):
+        a = np.asarray(x[n])
+        dot = np.abs(np.sum(a * gr[gname], -1))
+        scale_ = np.linalg.norm(a, axis=-1) * np.linalg.norm(gr[gname], axis=-1)
+        assert np.all(dot <= 1e-6 * scale_ + 1e-15), n
+        assert np.max(scale_) > 0
+
+
+L2_MUTATIONS = [
+    ("_l2norm_adjoint", "return r * (dxn - xn * np.sum(xn * dxn, axis=-1, keepdims=True))",
+     "return r * dxn"),                                                       # drops the projection
+    ("_l2norm_adjoint", "return r * (dxn - xn * np.sum(xn * dxn, axis=-1, keepdims=True))",
+     "return dxn - xn * np.sum(xn * dxn, axis=-1, keepdims=True)"),           # drops the 1 / |x|
+    ("fwd_chunk", "    if qk_l2norm:\n        q, k = l2norm(q), l2norm(k)\n    B, T, Hqk, dk = q.shape\n"
+                  "    Hv, dv = v.shape[2], v.shape[3]\n    hm = qk_head_of(Hqk, Hv)\n"
+                  "    spans = sequences(B, T, cu_seqlens)\n    o = np.zeros((B, T, Hv, dv))\n"
+                  "    hT = np.zeros((len(spans), Hv, dk, dv))\n    for n_seq",
+     "    if qk_l2norm:\n        q = l2norm(q)\n    B, T, Hqk, dk = q.shape\n"
+     "    Hv, dv = v.shape[2], v.shape[3]\n    hm = qk_head_of(Hqk, Hv)\n"
+     "    spans = sequences(B, T, cu_seqlens)\n    o = np.zeros((B, T, Hv, dv))\n"
+     "    hT = np.zeros((len(spans), Hv, dk, dv))\n    for n_seq"),           # k left unnormalised
+    ("l2norm", "return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)",
+     "return x / np.sqrt(np.sum(x * x, axis=-2, keepdims=True) + eps)"),      # wrong axis
+]
+
+
+@pytest.mark.parametrize("fn_name,old,new", L2_MUTATIONS)
+def test_l2norm_pins_reject_planted_mistakes(fn_name, old, new):
+    m = _mutant(fn_name, old, new)
+    if fn_name == "_l2norm_adjoint":
+        x = _rescaled_rows(small(B=1, T=30, Hqk=1, Hv=2, dk=4, dv=4, seed=98, backward=True), 0.5, 3.0, 6)
+        args = (x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["dO"], x["h0"], x["dhT"])
+        gr = m["bwd_token"](*args, qk_l2norm=True)
+        ok = bwd_token(*args, qk_l2norm=True)         # pinned by the finite differences above
+        assert max(rel(gr[n], ok[n]) for n in ("dq", "dk")) > 1e-6
+        return
+    x = small(B=1, Hqk=1, Hv=2, dk=6, dv=5, seed=61, lengths=[20, 9, 33])
+    a = _rescaled_rows(x, 10.0, 30.0, 1)
+    b = _rescaled_rows(x, 40.0, 90.0, 2)
+    oa, ha = call_fwd(m["fwd_chunk"], a, qk_l2norm=True)
+    ob, hb = call_fwd(m["fwd_chunk"], b, qk_l2norm=True)
+    assert rel(oa, ob) > 1e-6 or rel(ha, hb) > 1e-6   # the row-scale invariance pin rejects it
