@@ -345,7 +345,6 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
   void* save_states = op.states;
   if ((save_states || op.qk_l2norm) && !uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;
-  if (op.qk_l2norm) return GDN_ERR_UNSUPPORTED;   // NORM-TODO
   if (save_states && !state_rows_fit(state_slots(s), s.Hv)) return GDN_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, o, hT, save_states};
   for (const void* p : ptrs)
@@ -467,7 +466,6 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
   if (!uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;   // backward: bf16, dk = dv = 128
-  if (op.qk_l2norm) return GDN_ERR_UNSUPPORTED;   // NORM-TODO
   if (!state_rows_fit(state_slots(s), s.Hv)) return GDN_ERR_UNSUPPORTED;
   const BwdPlan bp = plan_backward(s, opt);
   if (!workspace || !aligned16(workspace) || workspace_bytes < bp.total) return GDN_ERR_WORKSPACE;

@@ -74,6 +74,9 @@ constexpr uint32_t kId128km = idesc_bf16(128, 128, false, true);
 
 }  // namespace
 
+// kNorm: q and k rows are L2-normalised in the kernel (their inverse norms folded into the
+// per-token factors: egd and egk carry rk, the scaled Q tile carries rq).
+template <bool kNorm>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_s,
@@ -200,11 +203,13 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         fence_proxy_async_smem();
       }
       named_bar_sync(kBarPrep, kNumPrep);
+      if (kNorm) row_inv_norms(st, st + 16384, st + 8192, st + 24576, ss->cs.rk[s], ss->cs.rq[s], pt);
       prep_scan(pc, s);
       named_bar_sync(kBarPrep, kNumPrep);
-      prep_decays(pc, s, nv);
+      prep_decays<kNorm>(pc, s, nv);
       named_bar_sync(kBarPrep, kNumPrep);
-      scale_rows_tile_part(st + 8192, 16384, ss->cs.eg[s], p.scale, pt, kNumPrep);   // Q <- scale diag(exp(gam)) Q
+      // Q <- scale diag(exp(gam)) Q (times rq under the normalisation)
+      scale_rows_tile_part(st + 8192, 16384, kNorm ? ss->cs.egq[s] : ss->cs.eg[s], p.scale, pt, kNumPrep);
       tc::cp_async_wait_all();
       named_bar_sync(kBarPrep, kNumPrep);
       prep_write_a_rows(pc, s, sbase + kOffA2 + s * 8192u, 0);                       // A diag(beta)
@@ -340,7 +345,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         umma_commit(&ss->mma_done);
       }
       wait_mma();
-      // -dY^T diag(exp(gam)) -> bf16
+      // -dY^T diag(exp(gam)) -> bf16 (times rk under the normalisation: it multiplies the raw K)
       {
         float dy[32];
         if (ok) tmem_ld32_sync(tmem + lane_base + kColDY + hh * 32, dy);
@@ -348,7 +353,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
           for (int u = 0; u < 32; ++u) dy[u] = 0.f;
         }
-        const float* eg = ss->cs.eg[s];
+        const float* eg = kNorm ? ss->cs.egk[s] : ss->cs.eg[s];
         uint32_t w[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
@@ -451,12 +456,12 @@ cudaError_t launch_bwd_chain(const FwdParams& p, const TcPlan& plan, int num_ite
     if (!make_tile_map(&ms, p.states, 1, slots * p.Hv * 128, 128)) return cudaErrorInvalidValue;
   }
   *what = "shared memory attribute";
-  cudaError_t err = cudaFuncSetAttribute(gdn_bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+  auto kernel = p.qk_l2norm ? gdn_bwd_chain_kernel<true> : gdn_bwd_chain_kernel<false>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (err != cudaSuccess) return err;
   *what = "backward chain launch";
   trace_pre(kKernBwdChain, st);
-  gdn_bwd_chain_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mdo, ms, p, plan);
+  kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mdo, ms, p, plan);
   err = cudaGetLastError();
   trace_post(st);
   return err;

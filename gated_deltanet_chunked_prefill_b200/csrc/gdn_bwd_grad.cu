@@ -64,6 +64,7 @@ struct Small {
   float dgam[kNumGamSlots][64];
   float dbeta[kNumBetaSlots][64];
   float dgn[16];
+  float pdot[2][2][64];   // q/k normalisation: per (dq | dk, column half, row) partial dot products
   uint64_t tma_bar, mma_bar, gram_bar;   // gram_bar: the Gram product's own commit (its
                                          // completion is implied by the next mma_bar phase)
   uint32_t tmem_base;
@@ -105,6 +106,11 @@ __device__ __forceinline__ float warp_transpose_sum(float* v) {
 
 }  // namespace
 
+// kNorm: q and k rows are L2-normalised in the kernel. The products run on the raw tiles with the
+// inverse row norms rk, rq folded into per-token factors: the dQ accumulator holds rq * dQn and the
+// dK accumulator rk * dKn (dQn, dKn: gradients w.r.t. the normalised rows), and the raw-row
+// gradients are x - xn (xn . x) of those, with xn the normalised row.
+template <bool kNorm>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -273,10 +279,24 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
   // A (fp32 rows, from the forward pass) -> A diag(beta) and A in bf16
   prep_write_a_rows(pc, 0, sbase + kOffA2, sbase + kOffA);
+  if (kNorm) {
+    // inverse row norms of K and Q, folded into the decay factors (egd, egk carry rk; egq rq)
+    row_inv_norms(sm + kOffKQ, sm + kOffKQ + 16384, sm + kOffKQ + 8192, sm + kOffKQ + 24576, ss->cs.rk[0],
+                  ss->cs.rq[0], tid);
+    __syncthreads();
+    if (tid < kChunk) {
+      const float rk = ss->cs.rk[0][tid], e = ss->cs.eg[0][tid];
+      ss->cs.egd[0][tid] *= rk;
+      ss->cs.egk[0][tid] = e * rk;
+      ss->cs.egq[0][tid] = e * ss->cs.rq[0][tid];
+    }
+  }
   fence_proxy_async_smem();
   commit_wait();
   const float* eg = ss->cs.eg[0];
   const float* egd = ss->cs.egd[0];
+  const float* egk = kNorm ? ss->cs.egk[0] : eg;   // exp(gam), times rk under the normalisation
+  const float* egq = kNorm ? ss->cs.egq[0] : eg;   // exp(gam), times rq under the normalisation
   // ---- Y^T = V^T - (S K^T) diag(e^gam);  dDelta = dS' K^T diag(e^(gam_n - gam)) + dO^T scale P
   float yv[32], ddv[32];
   {
@@ -295,7 +315,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int u = 0; u < 32; ++u) {
       const int jj = hh * 32 + u;
       const float vv = bf16_at(vt + jj * 128 + ((rc ^ (jj & 7)) << 4) + rb);
-      yv[u] = vv - eg[jj] * sk[u];
+      yv[u] = vv - egk[jj] * sk[u];
       ddv[u] = fmaf(da[u], egd[jj], p.scale * db[u]);      // P is unscaled
     }
   }
@@ -355,7 +375,8 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int jj = hh * 32 + u;
       const float dov = bf16_at(dot + jj * 128 + ((rc ^ (jj & 7)) << 4) + rb);
       // (1) + (2): scale e^gam_j dO_jr (S Q^T)_rj - e^gam_j dY_jr (S K^T)_rj
-      dgpart[u] = eg[jj] * (p.scale * dov * sq[u] - dy[u] * sk[u]);
+      if (kNorm) dgpart[u] = p.scale * dov * sq[u] * egq[jj] - dy[u] * sk[u] * egk[jj];
+      else dgpart[u] = eg[jj] * (p.scale * dov * sq[u] - dy[u] * sk[u]);
       sj[u] = egd[jj] * dl[u] * da[u];                 // (3) s_j partial
     }
     uint32_t w[16], x[16];
@@ -363,7 +384,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int u = 0; u < 16; ++u) {
       w[u] = pack_bf16(dl[2 * u], dl[2 * u + 1]);
       const int j0 = hh * 32 + 2 * u;
-      x[u] = pack_bf16(-dy[2 * u] * eg[j0], -dy[2 * u + 1] * eg[j0 + 1]);
+      x[u] = pack_bf16(-dy[2 * u] * egk[j0], -dy[2 * u + 1] * egk[j0 + 1]);
     }
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) {
@@ -523,6 +544,11 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // dP = scale * mvals;  P = QK^T * E (j <= i);  F = dP * P -> dgam_i += row sum, dgam_j -= col sum
       // dPm = dP * E (j <= i) -> bf16
       uint32_t w[16];
+      if (kNorm) {                            // normalised P and dPm: rows times rq_i, columns times rk_j
+        const float rqi = ss->cs.rq[0][i];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) e[u] *= rqi * ss->cs.rk[0][j0 + u];
+      }
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
         const int jx = j0 + u;
@@ -570,8 +596,9 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int c4 = 0; c4 < 4; ++c4)
       st_shared_v4(sbase + kOffDA + sw128(r, hh * 4 + c4), w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
   } else {
-    // dO <- scale diag(e^gam) dO in place (an operand of dQ); its other uses have completed
-    scale_rows_tile_part(sm + kOffVDO + 8192, 16384, eg, p.scale, (r - 64) + 64 * hh, 128);
+    // dO <- scale diag(e^gam) dO in place (an operand of dQ; times rq under the normalisation);
+    // its other uses have completed
+    scale_rows_tile_part(sm + kOffVDO + 8192, 16384, egq, p.scale, (r - 64) + 64 * hh, 128);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -633,6 +660,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       const float gi = ss->cs.gam[0][i], glast = ss->cs.gam[0][j0 + 31];
       const float bi = ss->cs.bet[0][i];
+      const float rki = kNorm ? ss->cs.rk[0][i] : 1.f;
       float run = 1.f, rowsum = 0.f, bsum = 0.f;
       float colv[32], dg[32];
 #pragma unroll
@@ -642,7 +670,8 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         else run = (jx >= i) ? 1.f : run * ss->cs.egt[0][jx + 1];
         const bool m = jx < i;
         const float dl = m ? -dlv[jj] : 0.f;
-        const float ke = gvals[jj] * run;
+        // (K K^T)_ij E_ij of the normalised rows under the normalisation
+        const float ke = kNorm ? gvals[jj] * run * (rki * ss->cs.rk[0][jx]) : gvals[jj] * run;
         const float f = dl * bi * ke;            // dL * L
         rowsum += f;
         colv[jj] = f;
@@ -668,12 +697,25 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const float* Lf = reinterpret_cast<const float*>(sm + kOffLf);
     uint32_t w[16];
     const float4* rowv = reinterpret_cast<const float4*>(Lf + i * kLd + j0);
+    if (kNorm) {                              // dGs multiplies the raw K: rk_i (dG + dG^T)_ij rk_j
+      const float rki = ss->cs.rk[0][i];
+      const float* rk = ss->cs.rk[0];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 t = rowv[u];
-      const int ja = j0 + 4 * u;
-      w[2 * u] = pack_bf16(t.x + Lf[ja * kLd + i], t.y + Lf[(ja + 1) * kLd + i]);
-      w[2 * u + 1] = pack_bf16(t.z + Lf[(ja + 2) * kLd + i], t.w + Lf[(ja + 3) * kLd + i]);
+      for (int u = 0; u < 8; ++u) {
+        const float4 t = rowv[u];
+        const int ja = j0 + 4 * u;
+        w[2 * u] = pack_bf16((t.x + Lf[ja * kLd + i]) * rki * rk[ja], (t.y + Lf[(ja + 1) * kLd + i]) * rki * rk[ja + 1]);
+        w[2 * u + 1] = pack_bf16((t.z + Lf[(ja + 2) * kLd + i]) * rki * rk[ja + 2],
+                                 (t.w + Lf[(ja + 3) * kLd + i]) * rki * rk[ja + 3]);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4 t = rowv[u];
+        const int ja = j0 + 4 * u;
+        w[2 * u] = pack_bf16(t.x + Lf[ja * kLd + i], t.y + Lf[(ja + 1) * kLd + i]);
+        w[2 * u + 1] = pack_bf16(t.z + Lf[(ja + 2) * kLd + i], t.w + Lf[(ja + 3) * kLd + i]);
+      }
     }
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4)
@@ -694,6 +736,44 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   // ---- outputs: dq, dk (rows i < nv), dbeta, dg. A full chunk's bf16 dq, dk leave through TMA
   //      tile stores from staging (every operand tile is free now), otherwise per thread.
   const bool qk_tma = !out.qk_partial && nv == kChunk;
+  // Under the normalisation the accumulators hold x = r * (gradient w.r.t. the normalised row); the
+  // gradient w.r.t. the raw row is x - xn (xn . x), xn = r * (raw row). This thread holds 64 of
+  // the row's 128 columns (the other half is in warp qd + 4): partial dot products through smem.
+  // raw_half: row i, column half hh of the Q (which = 0) or K (which = 1) tile (bf16, swizzled)
+  auto raw_half = [&](int which, int i) -> const uint8_t* {
+    return sm + kOffKQ + (which == 0 ? 8192 : 0) + hh * 16384 + i * 128;
+  };
+  if (kNorm) {
+    if (r < 64) {
+      const int i = r;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        float v[64];
+        const uint32_t col = which == 0 ? kColQ : kColK;
+        if (ok) {
+          tmem_ld32_sync(tmem + lane_base + col + hh * 64, v);
+          tmem_ld32_sync(tmem + lane_base + col + hh * 64 + 32, v + 32);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 64; ++u) v[u] = 0.f;
+        }
+        const uint8_t* xr = raw_half(which, i);
+        float acc = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xr + ((ch ^ (i & 7)) << 4));
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = __bfloat1622float2(h2[e2]);
+            acc = fmaf(f.x, v[8 * ch + 2 * e2], fmaf(f.y, v[8 * ch + 2 * e2 + 1], acc));
+          }
+        }
+        ss->pdot[which][hh][i] = acc;
+      }
+    }
+    __syncthreads();
+  }
   if (r < 64) {
     const int i = r;
 #pragma unroll
@@ -703,6 +783,23 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (ok) {
         tmem_ld32_sync(tmem + lane_base + col + hh * 64, v);
         tmem_ld32_sync(tmem + lane_base + col + hh * 64 + 32, v + 32);
+      }
+      if (kNorm && ok) {
+        // v -= xn (xn . v) = raw * (r^2 (raw . v)), both halves summed in a fixed order
+        const float ri = which == 0 ? ss->cs.rq[0][i] : ss->cs.rk[0][i];
+        const float coef = ri * ri * (ss->pdot[which][0][i] + ss->pdot[which][1][i]);
+        const uint8_t* xr = raw_half(which, i);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xr + ((ch ^ (i & 7)) << 4));
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = __bfloat1622float2(h2[e2]);
+            v[8 * ch + 2 * e2] = fmaf(-coef, f.x, v[8 * ch + 2 * e2]);
+            v[8 * ch + 2 * e2 + 1] = fmaf(-coef, f.y, v[8 * ch + 2 * e2 + 1]);
+          }
+        }
       }
       if (qk_tma) {                            // staged: Yt (dq) / Dt (dk), 128B-swizzled halves
         uint8_t* srow = sm + (which == 0 ? kOffYt : kOffDt) + hh * 8192 + i * 128;
@@ -835,8 +932,8 @@ cudaError_t launch_bwd_grad(const FwdParams& p, const BwdOut& out, long long tot
   if (!out.qk_partial && (!make_tile_map(&mdq, out.dq, p.Hqk, rows) || !make_tile_map(&mdk, out.dk, p.Hqk, rows)))
     return cudaErrorInvalidValue;
   *what = "shared memory attribute";
-  cudaError_t err = cudaFuncSetAttribute(gdn_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+  auto kernel = p.qk_l2norm ? gdn_bwd_grad_kernel<true> : gdn_bwd_grad_kernel<false>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (err != cudaSuccess) return err;
   // persistent: one CTA per SM (the shared-memory footprint allows one), items strided over CTAs
   const long long items = total_chunks * p.Hv;
@@ -849,8 +946,7 @@ cudaError_t launch_bwd_grad(const FwdParams& p, const BwdOut& out, long long tot
   const unsigned grid = (unsigned)std::min<long long>(items, std::max(sms, 1));
   *what = "backward gradient launch";
   trace_pre(kKernBwdTc, st);
-  gdn_bwd_grad_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, mdo, ms, mds, mdv, mdq, mdk, p, out,
-                                                          (int)items);
+  kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, mdo, ms, mds, mdv, mdq, mdk, p, out, (int)items);
   err = cudaGetLastError();
   trace_post(st);
   if (err != cudaSuccess || !out.qk_partial) return err;

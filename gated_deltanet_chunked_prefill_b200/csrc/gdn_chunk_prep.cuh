@@ -38,11 +38,43 @@ struct ChunkScalars {
   float gam[2][64];   // chunk-local inclusive cumsum of g
   float egt[2][64];   // exp(g_t) (1 past the sequence end)
   float eg[2][64];    // exp(gam)
-  float egd[2][64];   // exp(gam_n - gam)
+  float egd[2][64];   // exp(gam_n - gam), times rk under the q/k normalisation
   float bet[2][64];   // beta (0 past the sequence end)
   float egn[2];       // exp(gam_n)
   int nv[2];          // valid tokens in the chunk
+  // q/k normalisation only: the inverse row norms (|x|^2 + eps)^(-1/2) of the chunk's K and Q
+  // rows, and exp(gam) times them. A normalised row is r * (raw row), so every product with a
+  // normalised K or Q row is the raw tile's product with r folded into a per-token factor.
+  float rk[2][64], rq[2][64];
+  float egk[2][64];   // exp(gam) rk
+  float egq[2][64];   // exp(gam) rq
 };
+
+// eps of the in-kernel q/k normalisation x / sqrt(|x|^2 + eps)
+constexpr float kL2NormEps = 1e-6f;
+
+// Inverse row norms of a chunk's K and Q tiles in shared memory (64 rows x 128 bf16 each, held
+// as two 64-column halves of 128-byte rows; the swizzle only permutes a row's 16-byte pieces).
+// 256 threads, two per row: threads 0..127 take K rows, 128..255 Q rows.
+__device__ __forceinline__ void row_inv_norms(const uint8_t* k0, const uint8_t* k1, const uint8_t* q0,
+                                              const uint8_t* q1, float* rk, float* rq, int t) {
+  const int row = (t >> 1) & 63, half = t & 1;
+  const bool isq = t >= 128;
+  const uint8_t* base = (isq ? (half ? q1 : q0) : (half ? k1 : k0)) + row * 128;
+  float ssq = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {
+    const uint4 v = *reinterpret_cast<const uint4*>(base + ch * 16);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      ssq = fmaf(f.x, f.x, fmaf(f.y, f.y, ssq));
+    }
+  }
+  ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
+  if (half == 0) (isq ? rq : rk)[row] = rsqrtf(ssq + kL2NormEps);
+}
 
 __device__ __forceinline__ float bf16_at(const uint8_t* p) {
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
@@ -105,12 +137,23 @@ __device__ __forceinline__ void prep_scan(const PrepCtx& c, int s) {
   }
 }
 
-// decay factors (after the scan and a barrier)
+// decay factors (after the scan and a barrier; under the q/k normalisation also after the
+// inverse row norms): eg, egd (times rk when kNorm), and with kNorm egk, egq
+template <bool kNorm = false>
 __device__ __forceinline__ void prep_decays(const PrepCtx& c, int s, int nv) {
   const float gn = c.cs->gam[s][kChunk - 1];
   if (c.pt < kChunk) {
-    c.cs->eg[s][c.pt] = tc::fast_exp(c.cs->gam[s][c.pt]);
-    c.cs->egd[s][c.pt] = tc::fast_exp(gn - c.cs->gam[s][c.pt]);
+    const float e = tc::fast_exp(c.cs->gam[s][c.pt]);
+    const float ed = tc::fast_exp(gn - c.cs->gam[s][c.pt]);
+    c.cs->eg[s][c.pt] = e;
+    if (kNorm) {
+      const float rk = c.cs->rk[s][c.pt];
+      c.cs->egd[s][c.pt] = ed * rk;
+      c.cs->egk[s][c.pt] = e * rk;
+      c.cs->egq[s][c.pt] = e * c.cs->rq[s][c.pt];
+    } else {
+      c.cs->egd[s][c.pt] = ed;
+    }
   }
   if (c.pt == 0) {
     c.cs->egn[s] = tc::fast_exp(gn);
@@ -139,7 +182,9 @@ __device__ __forceinline__ void issue_gram(uint32_t tmem_g, uint32_t kq_addr, ui
 // one per entry, no overflow, monotone underflow to 0. `ok` false: G treated as 0.
 // Ends with tcgen05 fence + group barrier.
 // kWriteL false: only P is produced (the caller takes A from elsewhere).
-template <bool kWriteL = true>
+// kNorm: G holds raw-row products; the normalised ones are rk_i rk_j (KK^T)_ij and
+// rq_i rk_j (QK^T)_ij, so the rows take rk_i (L) or rq_i (P) and the columns rk_j.
+template <bool kWriteL = true, bool kNorm = false>
 __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_addr, float p_scale, bool ok) {
   const int qd = c.pw & 3, hc = c.pw >> 2;
   const int rr = 32 * qd + c.lane;
@@ -163,6 +208,16 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
   const int i = rr & 63;
   const float gi = c.cs->gam[s][i];
   const float glast = c.cs->gam[s][j0 + 31];
+  if (kNorm) {
+    const float4* r4 = reinterpret_cast<const float4*>(c.cs->rk[s] + j0);
+    const float rowf = rr < kChunk ? c.cs->rk[s][i] : c.cs->rq[s][i];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 t = r4[u];
+      vals[4 * u] *= rowf * t.x; vals[4 * u + 1] *= rowf * t.y;
+      vals[4 * u + 2] *= rowf * t.z; vals[4 * u + 3] *= rowf * t.w;
+    }
+  }
   float run = 1.f;
   if (rr < kChunk && !kWriteL) {
     // L not wanted
@@ -355,13 +410,16 @@ __device__ __forceinline__ void prep_solve_strip_h(const PrepCtx& c, float (&x)[
 }
 
 // A2 = A diag(beta) and (b2_addr != 0) B2 = A diag(beta exp(gam)) -> bf16 (128B-swizzled
-// rows at a2_addr, b2_addr) straight from a strip solve's fragments.
+// rows at a2_addr, b2_addr) straight from a strip solve's fragments. kNorm: B2 multiplies the raw
+// K tile, so its columns also take rk (B2 = A diag(beta exp(gam) rk)).
+template <bool kNorm = false>
 __device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const float (&x)[4][4], uint32_t a2_addr,
                                                  uint32_t b2_addr) {
   const int w = c.pw, gid = c.lane >> 2, tig = c.lane & 3;
   const int j = 8 * w + 2 * tig;
   const float b0 = c.cs->bet[s][j], b1 = c.cs->bet[s][j + 1];
-  const float e0 = b0 * c.cs->eg[s][j], e1 = b1 * c.cs->eg[s][j + 1];
+  const float* ek = kNorm ? c.cs->egk[s] : c.cs->eg[s];
+  const float e0 = b0 * ek[j], e1 = b1 * ek[j + 1];
 #pragma unroll
   for (int R = 0; R < 4; ++R) {
 #pragma unroll

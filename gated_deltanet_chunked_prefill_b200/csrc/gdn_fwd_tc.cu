@@ -90,6 +90,9 @@ constexpr uint32_t kIdE2 = idesc_bf16(128, 128, false, true);     // B MN-major
 
 }  // namespace
 
+// kNorm: q and k rows are L2-normalised in the kernel (their inverse norms folded into the
+// per-token factors; see ChunkScalars).
+template <bool kNorm>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
@@ -246,11 +249,12 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       named_bar_sync(kBarPrep, kNumPrep);
       if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
+      if (kNorm) row_inv_norms(st, st + kHalf, st + kOffQ, st + kHalf + kOffQ, ss->cs.rk[s], ss->cs.rq[s], pt);
       prep_scan(pc, s);
       // the bulk copies of earlier P tiles have read their slots (this chunk's masks rewrite one)
       if (pt == 0) bulk_wait_read();
       named_bar_sync(kBarPrep, kNumPrep);
-      prep_decays(pc, s, nv);
+      prep_decays<kNorm>(pc, s, nv);
     };
     if (nchunks > 0) {
       float gv0, bv0;
@@ -268,11 +272,12 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       pc.colG = gw_col;
-      prep_masks(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
+      prep_masks<true, kNorm>(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
       // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- diag(exp(gam)) Q
-      // in place (the Gram product has consumed Q); then one column strip of A per warp
+      // (times rq: the normalised rows) in place (the Gram product has consumed Q); then one
+      // column strip of A per warp
       if (warp < 4) prep_diag_inverse_h(pc);
-      else scale_rows_tile_part(st + kOffQ, kHalf, ss->cs.eg[s], 1.f, pt - 128, 128);
+      else scale_rows_tile_part(st + kOffQ, kHalf, kNorm ? ss->cs.egq[s] : ss->cs.eg[s], 1.f, pt - 128, 128);
       named_bar_sync(kBarPrep, kNumPrep);
       {
         float x[4][4];
@@ -286,7 +291,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           ok = ok && mbar_wait(&ss->wdone, (c - 1) & 1, abort_flag);
           ok = __all_sync(0xffffffffu, ok);
         }
-        prep_store_strip(pc, s, x, sbase + kOffA2, sbase + kOffB2);
+        prep_store_strip<kNorm>(pc, s, x, sbase + kOffA2, sbase + kOffB2);
       }
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
@@ -654,12 +659,12 @@ cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items,
     if (!make_tile_map(&ms, p.states, 1, slots * p.Hv * 128, 128)) return cudaErrorInvalidValue;
   }
   *what = "shared memory attribute";
-  cudaError_t err = cudaFuncSetAttribute(gdn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+  auto kernel = p.qk_l2norm ? gdn_fwd_tc_kernel<true> : gdn_fwd_tc_kernel<false>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (err != cudaSuccess) return err;
   *what = "tensor-core forward launch";
   trace_pre(kKernFwdTc, st);
-  gdn_fwd_tc_kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, ms, mo, p, plan);
+  kernel<<<num_items, kThreads, kSmemBytes, st>>>(mq, mk, mv, ms, mo, p, plan);
   err = cudaGetLastError();
   trace_post(st);
   return err;

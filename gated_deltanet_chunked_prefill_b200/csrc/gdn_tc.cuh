@@ -155,8 +155,9 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
 
 // Sum over the tokens [cs, cs + n) (n <= 64) of log(exp(g_t) max(1, |1 - beta_t |k_t|^2|)),
 // the log of the exact spectral norm of each token's state transition exp(g)(I - beta k k^T)
-// (eigenvalues exp(g) and exp(g)(1 - beta |k|^2)). All 512 threads of the CTA call it and
-// get the same value; wsum is 16 floats of shared scratch.
+// (eigenvalues exp(g) and exp(g)(1 - beta |k|^2)). Under the q/k normalisation k is the
+// normalised row, |k|^2 = s / (s + eps) for the raw squared norm s. All 512 threads of the CTA
+// call it and get the same value; wsum is 16 floats of shared scratch.
 __device__ __forceinline__ float chunk_log_bound(const FwdParams& p, const WorkItem& it, int cs, int n,
                                                  float* wsum) {
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(p.k);
@@ -180,6 +181,7 @@ __device__ __forceinline__ float chunk_log_bound(const FwdParams& p, const WorkI
   sq += __shfl_xor_sync(0xffffffffu, sq, 1);
   sq += __shfl_xor_sync(0xffffffffu, sq, 2);
   sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+  if (p.qk_l2norm) sq = sq / (sq + 1e-6f);
   float lt = 0.f;
   if (part == 0 && tok < n) {
     const size_t gi = row * p.Hv + it.j;

@@ -179,6 +179,10 @@ def test_states_option_checks():
     o = gdn.Options()
     o.states = FAKE
     assert _fwd(dtype=0, dk=64, dv=64, opt=o) == 2        # fp32 / CUDA-core path: unsupported
+    n = gdn.Options()
+    n.qk_l2norm = 1
+    assert _fwd(dtype=0, dk=64, dv=64, opt=n) == 2        # the normalisation: tensor-core path only
+    assert _fwd(dtype=1, dk=64, dv=64, opt=n) == 2
     o.states = MISALIGNED
     assert _fwd(opt=o) == 1
 
