@@ -191,10 +191,7 @@ struct BwdPlan {
 
 BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
   BwdPlan b;
-  gdn_options o{};
-  if (opt) o = *opt;
-  if (o.cp_exact) o.cp_segment_chunks = -1;   // exact: the sequential passes run unsplit
-  b.chain = plan_forward(GDN_BF16, s, &o);
+  b.chain = plan_forward(GDN_BF16, s, opt);     // the segments of both sequential passes
   const int nch = (s.T + kChunk - 1) / kChunk;
   b.total_chunks = s.packed ? (long long)nch + s.N : (long long)s.N * nch;
   b.grouped = s.Hv != s.Hqk;
@@ -498,35 +495,58 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   int items = s.N * s.Hv;
   cudaError_t err;
   const char* what = "";
+  int* first = nullptr;                          // packed sequences: first pair index of each sequence
   if (s.packed || f.kind != kPlanUnits) {
     int2* table = f.table ? reinterpret_cast<int2*>(ws + f.off_table) : nullptr;
     int* count = f.table ? reinterpret_cast<int*>(ws + f.off_count) : nullptr;
-    int* first = f.table ? reinterpret_cast<int*>(ws + f.off_first) : nullptr;
+    first = f.table ? reinterpret_cast<int*>(ws + f.off_first) : nullptr;
     if (s.packed) {
       err = launch_cp_plan(p, f.seg_chunks > 0 ? f.seg_chunks : 1, f.max_pairs, table, count, first,
                            const_cast<int*>(p.chunk_off), stream);
       if (err != cudaSuccess) return cuda_fail("backward plan", err);
     }
     if (f.kind != kPlanUnits) {
-      plan.kind = kPlanGate;
+      plan.kind = f.exact ? kPlanCpP3 : kPlanGate;
       plan.table = table;
       plan.table_count = count;
       items = f.max_pairs * s.Hv;
     }
   }
-  // 1) forward recompute: the bf16 start state of every chunk (unless the caller cached them)
+  if (f.exact) {
+    plan.seg_state = reinterpret_cast<float*>(ws + f.off_state);
+    plan.seg_trans = reinterpret_cast<float*>(ws + f.off_trans);
+  }
+  TcPlan map_plan = plan;                        // exact stitch, phase 1: two roles per segment
+  map_plan.kind = kPlanCpP1;
+  map_plan.roles = 2;
+  // 1) forward recompute: the bf16 start state of every chunk (unless the caller cached them).
+  //    Exact stitch: the segment maps, their chain, then the final pass that stores the states.
   if (!cached) {
+    if (f.exact) {
+      FwdParams p1 = p;
+      p1.states = nullptr;
+      err = launch_fwd_tc(p1, map_plan, f.max_pairs * 2 * s.Hv, stream, &what);
+      if (err != cudaSuccess) return cuda_fail(what, err);
+      err = launch_cp_stitch(p, plan, first, stream);
+      if (err != cudaSuccess) return cuda_fail("segment stitch", err);
+    }
     err = launch_fwd_tc(p, plan, items, stream, &what);
     if (err != cudaSuccess) return cuda_fail(what, err);
   }
-  // 2) reverse chain: the state gradient at every chunk end, and dh0
+  // 2) reverse chain: the state gradient at every chunk end, and dh0. Exact stitch: the mirror of
+  //    the forward's, from the sequence end (the segments' maps of the state gradient, their chain
+  //    in reverse, then the final pass that stores dS').
   FwdParams pc = p;
   pc.v = dO;
   pc.h0 = dhT;
   pc.hT = dh0;
   pc.states = dstates;
-
-
+  if (f.exact) {
+    err = launch_bwd_chain(pc, map_plan, f.max_pairs * 2 * s.Hv, stream, &what);
+    if (err != cudaSuccess) return cuda_fail(what, err);
+    err = launch_cp_stitch(pc, plan, first, stream, /*reverse=*/true);
+    if (err != cudaSuccess) return cuda_fail("segment stitch (reverse)", err);
+  }
   err = launch_bwd_chain(pc, plan, items, stream, &what);
   if (err != cudaSuccess) return cuda_fail(what, err);
   // 3) per-chunk gradients

@@ -89,14 +89,19 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (threadIdx.x == 0) report_error(p, kDevMisaligned);
     return;
   }
-  // decode the work item with h0/hT hidden: dhT / dh0 belong to the other ends here
+  // Decode the work item. Exact stitch (phases 1 and 3): the reverse item gives the end gradient
+  // (init) and where the start gradient goes (fin). Otherwise decode with h0/hT hidden (dhT / dh0
+  // belong to the other ends here) and take them below.
+  const bool exact = plan.kind == kPlanCpP1 || plan.kind == kPlanCpP3;
   FwdParams pd = p;
   pd.h0 = nullptr;
   pd.hT = nullptr;
   WorkItem it;
-  if (!get_work_item(pd, plan, blockIdx.x, it)) return;
+  if (!get_work_item(exact ? p : pd, plan, blockIdx.x, it, exact)) return;
   const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
   const bool is_first = it.s == it.seq_s, is_last = it.e == it.seq_e;
+  const bool zero_do = exact && it.zero_v;             // transition role: dO = 0
+  const bool store_ds = plan.kind != kPlanCpP1;        // phase 1 only maps the segment
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -117,6 +122,11 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_do);
+  }
+  if (zero_do) {                                      // both stages' dO tiles: 2 x 16 KB of zeros
+    for (int idx = threadIdx.x; idx < 2 * 1024; idx += kThreads)
+      *reinterpret_cast<uint4*>(sm + (idx >> 10) * kStageBytes + kOffDO + (idx & 1023) * 16) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -139,8 +149,20 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int we = ss->we;
   const int nchunks = (we - it.s + kChunk - 1) / kChunk;   // chunk c covers [s + 64c, min(s + 64c + 64, we))
   const bool from_seq_end = we == it.seq_e;
-  const float* init_ptr = (from_seq_end && p.h0) ? p.h0 + ((size_t)it.n * p.Hv + it.j) * (size_t)(128 * 128) : nullptr;
-  float* dh0 = (is_first && p.hT) ? p.hT + ((size_t)it.n * p.Hv + it.j) * (size_t)(128 * 128) : nullptr;
+  int init_mode = kInitZero;
+  const float* init_ptr = nullptr;
+  float* dh0 = nullptr;                                    // destination of the start gradient
+  if (exact) {
+    init_mode = it.init_mode;
+    init_ptr = it.init;
+    dh0 = it.fin;
+  } else {
+    if (from_seq_end && p.h0) {
+      init_mode = kInitPtr;
+      init_ptr = p.h0 + ((size_t)it.n * p.Hv + it.j) * (size_t)(128 * 128);
+    }
+    if (is_first && p.hT) dh0 = p.hT + ((size_t)it.n * p.Hv + it.j) * (size_t)(128 * 128);
+  }
 
   const uint32_t tmem = ss->tmem_base;
   volatile int* abort_flag = &ss->abort_flag;
@@ -152,13 +174,15 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int s = k & 1;
     const int row = it.b * p.T + it.s + chunk_of(k) * kChunk;
     uint8_t* st = sm + s * kStageBytes;
-    mbar_arrive_expect_tx(&ss->full[s], kStageBytes);
+    mbar_arrive_expect_tx(&ss->full[s], zero_do ? kOffDO : kStageBytes);
     tma_load_3d(st + 0, &tm_k, &ss->full[s], 0, it.hq, row);
     tma_load_3d(st + 8192, &tm_q, &ss->full[s], 0, it.hq, row);
     tma_load_3d(st + 16384, &tm_k, &ss->full[s], 64, it.hq, row);
     tma_load_3d(st + 24576, &tm_q, &ss->full[s], 64, it.hq, row);
-    tma_load_3d(st + kOffDO, &tm_do, &ss->full[s], 0, it.j, row);
-    tma_load_3d(st + kOffDO + 8192, &tm_do, &ss->full[s], 64, it.j, row);
+    if (!zero_do) {                                   // dO = 0: its tiles stay zero (cleared at the start)
+      tma_load_3d(st + kOffDO, &tm_do, &ss->full[s], 0, it.j, row);
+      tma_load_3d(st + kOffDO + 8192, &tm_do, &ss->full[s], 64, it.j, row);
+    }
   };
 
   if (warp < kEpiWarp0) {
@@ -242,7 +266,9 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
       for (int d = 0; d < 32; ++d) {
         const int col = hh * 64 + h2 * 32 + d;
-        v[d] = init_ptr ? init_ptr[(size_t)col * 128 + r] : 0.f;
+        if (init_mode == kInitPtr) v[d] = init_ptr[(size_t)col * 128 + r];
+        else if (init_mode == kInitIdentity) v[d] = (col == r) ? 1.f : 0.f;
+        else v[d] = 0.f;
       }
       tmem_st32_sync(s_addr + h2 * 32, v);
       write_sb(v, h2);
@@ -301,7 +327,7 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int c = chunk_of(k);
       const int t0 = it.s + c * kChunk;
       wait_mma();
-      if (et == 0 && t0 < it.e && ok) {
+      if (et == 0 && t0 < it.e && ok && store_ds) {
         // dS' of this chunk (its end gradient) for the gradient kernel: two TMA tile stores
         // from the swizzled bf16 copy, waited for (reads) before the copy is rewritten
         const int srow = (int)((chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) * 128);

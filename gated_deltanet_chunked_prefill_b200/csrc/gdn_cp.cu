@@ -92,11 +92,16 @@ gdn_cp_plan_kernel(const FwdParams p, int seg_chunks, int max_pairs, int2* table
 //   slot[s] <- M_{s-1} slot[s-1] + slot[s]
 // where slot[s] holds b_{s-1} from phase 1 (slot[1] already holds the exact start of
 // segment 1, phase 1 having run segment 0 from h0) and M is stored row-major [dk][dk].
+// reverse (the backward's state gradient dh = dS^T, carried from the sequence end): slot[s] is the
+// gradient at the end of segment s; for s = nseg - 3 .. 0,
+//   slot[s] <- M_{s+1} slot[s+1] + slot[s]
+// where slot[s] holds c_{s+1} (segment s + 1 run from a zero end gradient) and slot[nseg - 2]
+// already holds the exact value (the last segment ran from dhT).
 constexpr int kStitchCols = 8;
 constexpr int kStitchThreads = 256;
 
 __global__ void __launch_bounds__(kStitchThreads)
-gdn_cp_stitch_kernel(const FwdParams p, const TcPlan plan, const int* first_pair) {
+gdn_cp_stitch_kernel(const FwdParams p, const TcPlan plan, const int* first_pair, int reverse) {
   __shared__ float hcur[128 * kStitchCols];
   const int groups = 128 / kStitchCols;
   const int cg = blockIdx.x % groups;
@@ -112,12 +117,15 @@ gdn_cp_stitch_kernel(const FwdParams p, const TcPlan plan, const int* first_pair
   const int tid = threadIdx.x;
   const int row = tid >> 1, c4 = (tid & 1) * 4;      // 4 outputs: h[row][c0 + c4 .. +3]
   const int c0 = cg * kStitchCols;
-  float* slot1 = plan.seg_state + ((size_t)(pi0 + 1) * p.Hv + j) * hsz;
+  // forward: the known slot is 1 and the chain runs s = 2 .. nseg - 1 with M_{s-1};
+  // reverse: the known slot is nseg - 2 and the chain runs s = nseg - 3 .. 0 with M_{s+1}
+  float* slot1 = plan.seg_state + ((size_t)(pi0 + (reverse ? nseg - 2 : 1)) * p.Hv + j) * hsz;
   for (int idx = tid; idx < 128 * kStitchCols; idx += kStitchThreads)
     hcur[idx] = slot1[(size_t)(idx / kStitchCols) * 128 + c0 + idx % kStitchCols];
   __syncthreads();
-  for (int sg = 2; sg < nseg; ++sg) {
-    const float* M = plan.seg_trans + ((size_t)(pi0 + sg - 1) * p.Hv + j) * hsz;
+  for (int step = 0; step < nseg - 2; ++step) {
+    const int sg = reverse ? nseg - 3 - step : 2 + step;
+    const float* M = plan.seg_trans + ((size_t)(pi0 + (reverse ? sg + 1 : sg - 1)) * p.Hv + j) * hsz;
     float* dst = plan.seg_state + ((size_t)(pi0 + sg) * p.Hv + j) * hsz;
     float acc[4];
 #pragma unroll
@@ -152,10 +160,11 @@ cudaError_t launch_cp_plan(const FwdParams& p, int seg_chunks, int max_pairs, in
   return err;
 }
 
-cudaError_t launch_cp_stitch(const FwdParams& p, const TcPlan& plan, const int* first_pair, cudaStream_t st) {
+cudaError_t launch_cp_stitch(const FwdParams& p, const TcPlan& plan, const int* first_pair, cudaStream_t st,
+                             bool reverse) {
   const int grid = p.N * p.Hv * (128 / kStitchCols);
   trace_pre(kKernCpStitch, st);
-  gdn_cp_stitch_kernel<<<grid, kStitchThreads, 0, st>>>(p, plan, first_pair);
+  gdn_cp_stitch_kernel<<<grid, kStitchThreads, 0, st>>>(p, plan, first_pair, reverse ? 1 : 0);
   cudaError_t err = cudaGetLastError();
   trace_post(st);
   return err;

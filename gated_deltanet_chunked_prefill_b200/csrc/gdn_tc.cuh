@@ -76,7 +76,17 @@ struct WorkItem {
   bool zero_v;            // run with v = 0 (transition role)
 };
 
-__device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& plan, int item, WorkItem& w) {
+// reverse: the item of the backward's reverse chain under the exact stitch (kPlanCpP1 / kPlanCpP3),
+// where the state gradient runs from a segment's end to its start. There p.h0 is dhT and p.hT is
+// dh0 (the chain's parameter mapping), `init` is the gradient at the segment end and `fin` receives
+// the gradient at its start:
+//   kPlanCpP1, segment seg >= 1: role 0 runs from a zero end gradient (the last segment: from dhT)
+//     and stores its start gradient in the end slot of segment seg - 1 (pair pi - 1); role 1
+//     (seg <= nseg - 2) runs from the identity with dO = 0 and stores the segment's transition.
+//   kPlanCpP3: every segment runs from its stitched end gradient (the last: dhT), segment 0 writes
+//     dh0.
+__device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& plan, int item, WorkItem& w,
+                                              bool reverse = false) {
   const size_t hsz = (size_t)p.dk * p.dv;
   w.write_o = false;
   w.zero_v = false;
@@ -126,6 +136,28 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
   w.s = s + seg * plan.seg_chunks * kChunk;
   w.e = min(e, w.s + plan.seg_chunks * kChunk);
   const float* h0u = p.h0 ? p.h0 + ((size_t)w.n * p.Hv + w.j) * hsz : nullptr;
+  if (reverse) {
+    const bool last = seg + 1 == segs_used;
+    if (plan.kind == kPlanCpP1) {
+      if (seg == 0) return false;                           // its start gradient comes from phase 3
+      if (role == 0) {
+        if (last && h0u) { w.init_mode = kInitPtr; w.init = h0u; }
+        w.fin = plan.seg_state + ((size_t)(pi - 1) * p.Hv + w.j) * hsz;
+      } else {
+        if (last) return false;                             // the last segment ends at dhT
+        w.init_mode = kInitIdentity;
+        w.zero_v = true;
+        w.fin = plan.seg_trans + ((size_t)pi * p.Hv + w.j) * (size_t)p.dk * p.dk;
+      }
+      return true;
+    }
+    if (role != 0) return false;
+    if (!last) { w.init_mode = kInitPtr; w.init = plan.seg_state + ((size_t)pi * p.Hv + w.j) * hsz; }
+    else if (h0u) { w.init_mode = kInitPtr; w.init = h0u; }
+    if (seg == 0 && p.hT) w.fin = p.hT + ((size_t)w.n * p.Hv + w.j) * hsz;
+    w.write_o = true;
+    return true;
+  }
   if (plan.kind == kPlanCpP1) {
     if (seg + 1 >= segs_used) return false;                 // last segment: no map needed
     if (role == 0) {
@@ -207,7 +239,9 @@ cudaError_t launch_bwd_chain(const FwdParams& p, const TcPlan& plan, int num_ite
 // Packed sequences: build the (sequence, segment) table of a segmented plan.
 cudaError_t launch_cp_plan(const FwdParams& p, int seg_chunks, int max_pairs, int2* table, int* count,
                            int* first_pair, int* chunk_off, cudaStream_t st);
-// Exact stitch, phase 2: chain the segment maps h_{s+1} = M_s h_s + b_s in place.
-cudaError_t launch_cp_stitch(const FwdParams& p, const TcPlan& plan, const int* first_pair, cudaStream_t st);
+// Exact stitch, phase 2: chain the segment maps h_{s+1} = M_s h_s + b_s in place; reverse (the
+// backward's state gradient): dh_end(s) = M_{s+1} dh_end(s + 1) + c_{s+1}, from the sequence end.
+cudaError_t launch_cp_stitch(const FwdParams& p, const TcPlan& plan, const int* first_pair, cudaStream_t st,
+                             bool reverse = false);
 
 }  // namespace gdn

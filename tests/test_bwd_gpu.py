@@ -50,25 +50,44 @@ def test_bwd_small_parity(name):
         assert_close(gr[n], ref[n], "bf16", f"{name} {n}")
 
 
+@pytest.mark.parametrize("exact", [False, True])
 @pytest.mark.parametrize("cp", [1, 2, 5])
-def test_bwd_context_parallel(cp):
-    """Forced segments for the state pass and the reverse chain (gate-driven windows)."""
+def test_bwd_context_parallel(cp, exact):
+    """Forced segments for the state pass and the reverse chain: gate-driven windows, or the exact
+    affine stitch of both (the reverse one carries the state gradient from the sequence end);
+    packed sequences put the segment boundaries at odd token positions."""
     x = make_inputs(1, 0, 2, 2, 128, 128, "bf16", seed=31, h0_std=0.1, backward=True,
                     lengths=[700, 64, 1, 333, 129])
-    gr = run_gpu_bwd(x, cp_segment_chunks=cp)
+    gr = run_gpu_bwd(x, cp_segment_chunks=cp, cp_exact=exact)
     ref = oracle_bwd(x)
     for n in GRADS:
-        assert_close(gr[n], ref[n], "bf16", f"cp={cp} {n}")
+        assert_close(gr[n], ref[n], "bf16", f"cp={cp} exact={exact} {n}")
 
 
-def test_bwd_weak_decay_cp():
-    x = make_inputs(1, 1000, 1, 1, 128, 128, "bf16", seed=32, h0_std=0.1, backward=True)
+@pytest.mark.parametrize("exact", [False, True])
+def test_bwd_weak_decay_cp(exact):
+    """g close to 0 (x 0.02): the state and its gradient remember across many segments."""
+    x = make_inputs(1, 1000, 1, 2, 128, 128, "bf16", seed=32, h0_std=0.1, backward=True)
     x["g"] = (x["g"] * 0.02).contiguous()
+    ref = oracle_bwd(x)
     for cp in (-1, 3):
-        gr = run_gpu_bwd(x, cp_segment_chunks=cp)
-        ref = oracle_bwd(x)
+        gr = run_gpu_bwd(x, cp_segment_chunks=cp, cp_exact=exact)
         for n in GRADS:
-            assert_close(gr[n], ref[n], "bf16", f"weak decay cp={cp} {n}")
+            assert_close(gr[n], ref[n], "bf16", f"weak decay cp={cp} exact={exact} {n}")
+
+
+def test_bwd_exact_stitch_grouped_values_and_cache():
+    """Exact stitch in both passes with grouped values; the forward's cache (exact stitch too) gives
+    the same gradients, bit for bit, as the backward's own exact state pass."""
+    x = make_inputs(1, 1300, 2, 4, 128, 128, "bf16", seed=34, h0_std=0.1, backward=True)
+    d = to_dev(x)
+    states = _fwd_states(d, cp_segment_chunks=4, cp_exact=True)
+    cached = _bwd(d, cp_segment_chunks=4, cp_exact=True, states=states)
+    recomputed = _bwd(d, cp_segment_chunks=4, cp_exact=True)
+    ref = oracle_bwd(x)
+    for n in GRADS:
+        assert torch.equal(cached[n], recomputed[n]), n
+        assert_close(cached[n], ref[n], "bf16", f"exact gqa {n}")
 
 
 def test_bwd_no_cross_sequence_leakage():
