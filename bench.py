@@ -599,6 +599,38 @@ def measure_case(gdn, name, mode, args, dev, rank, world, dist, stream, pool, bu
     return res
 
 
+def measure_weak_decay(gdn, args, dev, rank, world, dist, stream):
+    """The long grouped-value forward with weakly decaying heads (g x 0.01: no gate window closes
+    within 16 chunks), unsplit and in each context-parallel mode: the restart fallback (default),
+    the exact stitch, and the gate-driven start with the exact stitch as fallback."""
+    name = "long_gqa_bf16"
+    w = CONFIGS[name]
+    x = make_inputs(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, rank_seed(w.seed, rank), h0_std=w.h0_std)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    d["g"] = (d["g"] * 0.01).contiguous()
+    o = torch.empty_like(d["v"])
+    hT = torch.empty((w.num_seqs, w.Hv, w.dk, w.dv), dtype=torch.float32, device=dev)
+    out = {"workload": w.description + "; g x 0.01 (weakly decaying heads)", "step": "fwd"}
+    for label, cp, cpx in (("unsplit", -1, 0), ("gate_restart", 0, 0), ("exact_stitch", 0, 1),
+                           ("gate_exact_fallback", 0, 2)):
+        ws = torch.zeros(gdn.fwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, cp, cpx),
+                         dtype=torch.uint8, device=dev)
+
+        def step():
+            gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"], None,
+                              cp_segment_chunks=cp, cp_exact=cpx, workspace=ws, o=o, hT=hT, check_status=False)
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        out[label + "_ms"] = max_over_ranks(time_steps(step, max(3, min(args.steps, 10)), stream), dist, dev)
+        del ws
+    out["speedup_vs_unsplit"] = {k[:-3]: out["unsplit_ms"] / out[k] for k in list(out) if k.endswith("_ms")}
+    del d
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_decode(gdn, args, dev, rank, world, dist, stream, pool, budget, c=DECODE):
     """One step = gdn_recurrent_step over every sequence of the batch (one token each)."""
     N, Hqk, Hv, dk, dv = c["N"], c["Hqk"], c["Hv"], c["dk"], c["dv"]
@@ -754,6 +786,7 @@ def main():
         for sname, smode in SUBS:
             per[f"{sname}:{smode}"] = measure_case(gdn, sname, smode, args, dev, rank, world, dist, stream, pool,
                                                    sub_budget, max(3, min(args.steps, 5)))
+        per["long_gqa_bf16:fwd:weak_decay"] = measure_weak_decay(gdn, args, dev, rank, world, dist, stream)
         per["decode"] = measure_decode(gdn, args, dev, rank, world, dist, stream, pool, sub_budget)
         per["decode_d256"] = measure_decode(gdn, args, dev, rank, world, dist, stream, pool, sub_budget / 2,
                                             DECODE_256)

@@ -119,7 +119,7 @@ def _opts(cp_segment_chunks: int = 0, cp_exact: bool = False, states=None, cp_mo
     o.cp_mode = int(cp_mode)
     o.deterministic = int(bool(deterministic))
     o.cp_segment_chunks = int(cp_segment_chunks)
-    o.cp_exact = int(bool(cp_exact))
+    o.cp_exact = int(cp_exact)       # 0 automatic, 1 exact stitch, 2 gate-driven restart (bool accepted)
     o.qk_l2norm = int(bool(qk_l2norm))
     o.test_stall = int(bool(test_stall))
     if states is not None:

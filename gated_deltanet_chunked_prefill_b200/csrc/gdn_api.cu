@@ -1,4 +1,5 @@
 // C-ABI entry points: argument validation, workspace layout, planning, launches.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 
@@ -77,6 +78,7 @@ gdn_status read_options(const gdn_options* opt, gdn_options& o) {
   if (o.qk_l2norm != 0 && o.qk_l2norm != 1) return GDN_ERR_INVALID_ARG;
   if (o.test_stall != 0 && o.test_stall != 1) return GDN_ERR_INVALID_ARG;
   if (o.cp_mode < -1) return GDN_ERR_INVALID_ARG;
+  if (o.cp_exact < 0 || o.cp_exact > 2) return GDN_ERR_INVALID_ARG;
   return GDN_OK;
 }
 
@@ -128,8 +130,12 @@ int auto_segment(const Shape& s, int nch) {
 struct FwdPlan {
   int kind = kPlanUnits;
   int seg_chunks = 0, max_segs = 0, max_pairs = 0;
-  bool table = false, exact = false;
-  size_t off_table = 0, off_count = 0, off_first = 0, off_state = 0, off_trans = 0, total = kStatusBytes;
+  bool table = false;
+  bool exact = false;      // exact affine stitch for every segment
+  bool fallback = false;   // gate-driven start, the exact stitch where a segment's window does not close
+  size_t off_table = 0, off_count = 0, off_first = 0, off_state = 0, off_trans = 0, off_ws = 0;
+  size_t total = kStatusBytes;
+  bool phased() const { return exact || fallback; }   // the three-phase launch sequence
   size_t off_chunk_off = 0;     // packed sequences: per-sequence first chunk slot (state cache)
 };
 
@@ -146,8 +152,13 @@ FwdPlan plan_forward(gdn_dtype dtype, const Shape& s, const gdn_options* opt) {
   const int seg = mode > 0 ? mode : auto_segment(s, nch);
   if (seg <= 0 || (!s.packed && seg >= nch)) return f;
   f.seg_chunks = seg;
-  f.exact = opt && opt->cp_exact;
-  f.kind = f.exact ? kPlanCpP3 : kPlanGate;
+  // cp_exact: 0 gate-driven start, restarting at the sequence start where a window does not close;
+  // 1 exact stitch; 2 gate-driven with the exact stitch as that fallback, once a sequence can have 3
+  // or more segments (with 2, the fallback's two phases take as long as the restart).
+  const int cpx = opt ? opt->cp_exact : 0;
+  f.exact = cpx == 1;
+  f.fallback = cpx == 2 && (nch + seg - 1) / seg >= 3;
+  f.kind = f.phased() ? kPlanCpP3 : kPlanGate;
   if (s.packed) {
     f.table = true;
     f.max_pairs = (nch + s.N + seg - 1) / seg + s.N;
@@ -161,10 +172,13 @@ FwdPlan plan_forward(gdn_dtype dtype, const Shape& s, const gdn_options* opt) {
     f.off_count = off; off = align256(off + sizeof(int));
     f.off_first = off; off = align256(off + (size_t)s.N * sizeof(int));
   }
-  if (f.exact) {
+  if (f.phased()) {
     const size_t per = (size_t)f.max_pairs * s.Hv * s.dk * s.dv * sizeof(float);
     f.off_state = off; off = align256(off + per);
     f.off_trans = off; off = align256(off + per);
+  }
+  if (f.fallback) {
+    f.off_ws = off; off = align256(off + (size_t)f.max_pairs * s.Hv * sizeof(int));
   }
   f.total = off;
   return f;
@@ -293,7 +307,8 @@ int gdn_trace_end(float* ms, int* kernel_ids) {
 const char* gdn_kernel_name(int kernel_id) {
   static const char* names[kKernCount] = {"gdn_fwd_tc_kernel",   "gdn_fwd_simt_kernel", "gdn_cp_stitch_kernel",
                                           "gdn_bwd_grad_kernel", "gdn_bwd_simt_kernel", "gdn_bwd_reduce_kernel",
-                                          "gdn_cp_plan_kernel",  "gdn_bwd_chain_kernel", "gdn_step_kernel"};
+                                          "gdn_cp_plan_kernel",  "gdn_bwd_chain_kernel", "gdn_step_kernel",
+                                          "gdn_cp_probe_kernel"};
   return (kernel_id >= 0 && kernel_id < kKernCount) ? names[kernel_id] : "unknown";
 }
 
@@ -319,11 +334,14 @@ const char* gdn_status_string(gdn_status s) {
 
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs,
                                     const gdn_options* opt) {
-  // sized for both the bf16 tensor-core plan (the larger) and the fp32 path
+  // sized for both the bf16 tensor-core plan (the larger) and the fp32 path. B == 1 with
+  // num_seqs >= 1 fits both a packed call and a call without cu_seqlens (whose num_seqs is ignored).
   Shape s;
-  const bool packed = num_seqs > 0 && B == 1;
-  if (check_shape(B, T, Hqk, Hv, dk, dv, packed ? num_seqs : 0, packed, s) != GDN_OK) return kStatusBytes;
-  return plan_forward(GDN_BF16, s, opt).total;
+  size_t total = kStatusBytes;
+  if (check_shape(B, T, Hqk, Hv, dk, dv, 0, false, s) == GDN_OK) total = plan_forward(GDN_BF16, s, opt).total;
+  if (num_seqs > 0 && B == 1 && check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, true, s) == GDN_OK)
+    total = std::max(total, plan_forward(GDN_BF16, s, opt).total);
+  return total;
 }
 
 gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
@@ -346,8 +364,8 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, o, hT, save_states};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
-  if (!workspace || !aligned16(workspace) ||
-      workspace_bytes < gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, num_seqs, opt))
+  // this call's own plan (the size query may also cover the other reading of B == 1)
+  if (!workspace || !aligned16(workspace) || workspace_bytes < plan_forward(dtype, s, opt).total)
     return GDN_ERR_WORKSPACE;
 
   FwdParams p{};
@@ -402,7 +420,7 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
                            const_cast<int*>(plan.table_count), first, chunk_off, stream);
       if (err != cudaSuccess) return cuda_fail("segment table", err);
     }
-    if (!f.exact) {
+    if (!f.phased()) {
       plan.kind = kPlanGate;
       err = launch_fwd_tc(pf, plan, f.max_pairs * s.Hv, stream, &what);
       if (err != cudaSuccess) return cuda_fail(what, err);
@@ -410,6 +428,11 @@ gdn_status gdn_chunk_fwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
     }
     plan.seg_state = reinterpret_cast<float*>(ws + f.off_state);
     plan.seg_trans = reinterpret_cast<float*>(ws + f.off_trans);
+    plan.seg_ws = f.fallback ? reinterpret_cast<int*>(ws + f.off_ws) : nullptr;
+    if (f.fallback) {                           // every segment's window, before phase 1
+      err = launch_cp_probe(p, plan, f.max_pairs * s.Hv, stream, false);
+      if (err != cudaSuccess) return cuda_fail("window probe", err);
+    }
     plan.kind = kPlanCpP1;
     plan.roles = 2;
     err = launch_fwd_tc(p, plan, f.max_pairs * 2 * s.Hv, stream, &what);
@@ -436,10 +459,13 @@ size_t gdn_chunk_states_size(int B, int T, int Hqk, int Hv, int dk, int dv, int 
 
 size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int dv, int num_seqs,
                                     const gdn_options* opt) {
+  // B == 1 with num_seqs >= 1 fits both a packed call and a call without cu_seqlens
   Shape s;
-  const bool packed = num_seqs > 0 && B == 1;
-  if (check_shape(B, T, Hqk, Hv, dk, dv, packed ? num_seqs : 0, packed, s) != GDN_OK) return kStatusBytes;
-  return plan_backward(s, opt).total;
+  size_t total = kStatusBytes;
+  if (check_shape(B, T, Hqk, Hv, dk, dv, 0, false, s) == GDN_OK) total = plan_backward(s, opt).total;
+  if (num_seqs > 0 && B == 1 && check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, true, s) == GDN_OK)
+    total = std::max(total, plan_backward(s, opt).total);
+  return total;
 }
 
 gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
@@ -506,15 +532,16 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
       if (err != cudaSuccess) return cuda_fail("backward plan", err);
     }
     if (f.kind != kPlanUnits) {
-      plan.kind = f.exact ? kPlanCpP3 : kPlanGate;
+      plan.kind = f.phased() ? kPlanCpP3 : kPlanGate;
       plan.table = table;
       plan.table_count = count;
       items = f.max_pairs * s.Hv;
     }
   }
-  if (f.exact) {
+  if (f.phased()) {
     plan.seg_state = reinterpret_cast<float*>(ws + f.off_state);
     plan.seg_trans = reinterpret_cast<float*>(ws + f.off_trans);
+    plan.seg_ws = f.fallback ? reinterpret_cast<int*>(ws + f.off_ws) : nullptr;
   }
   TcPlan map_plan = plan;                        // exact stitch, phase 1: two roles per segment
   map_plan.kind = kPlanCpP1;
@@ -522,9 +549,13 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   // 1) forward recompute: the bf16 start state of every chunk (unless the caller cached them).
   //    Exact stitch: the segment maps, their chain, then the final pass that stores the states.
   if (!cached) {
-    if (f.exact) {
+    if (f.phased()) {
       FwdParams p1 = p;
       p1.states = nullptr;
+      if (f.fallback) {
+        err = launch_cp_probe(p, plan, f.max_pairs * s.Hv, stream, false);
+        if (err != cudaSuccess) return cuda_fail("window probe", err);
+      }
       err = launch_fwd_tc(p1, map_plan, f.max_pairs * 2 * s.Hv, stream, &what);
       if (err != cudaSuccess) return cuda_fail(what, err);
       err = launch_cp_stitch(p, plan, first, stream);
@@ -541,7 +572,11 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   pc.h0 = dhT;
   pc.hT = dh0;
   pc.states = dstates;
-  if (f.exact) {
+  if (f.phased()) {
+    if (f.fallback) {
+      err = launch_cp_probe(pc, plan, f.max_pairs * s.Hv, stream, true);
+      if (err != cudaSuccess) return cuda_fail("window probe (reverse)", err);
+    }
     err = launch_bwd_chain(pc, map_plan, f.max_pairs * 2 * s.Hv, stream, &what);
     if (err != cudaSuccess) return cuda_fail(what, err);
     err = launch_cp_stitch(pc, plan, first, stream, /*reverse=*/true);

@@ -51,7 +51,6 @@ constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 struct Small {
   ChunkScalars cs;
   float wsum[16];
-  int we;                 // end of the processed range (warm-up window end)
   uint64_t full[2], prep_full[2], gdone, mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -96,12 +95,46 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   FwdParams pd = p;
   pd.h0 = nullptr;
   pd.hT = nullptr;
+  if (plan.seg_ws != nullptr && plan.kind == kPlanCpP1) {
+    // exact fallback, phase 1: item = (pi * 2 + role) * Hv + j. When the window after the
+    // predecessor's end closes (the probe's record, read first) no map is needed: leave at once.
+    const int j = blockIdx.x % p.Hv, pi = blockIdx.x / (2 * p.Hv);
+    if (pi >= 1 && plan.seg_ws[(size_t)(pi - 1) * p.Hv + j] >= 0) return;
+  }
   WorkItem it;
   if (!get_work_item(exact ? p : pd, plan, blockIdx.x, it, exact)) return;
   const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
   const bool is_first = it.s == it.seq_s, is_last = it.e == it.seq_e;
   const bool zero_do = exact && it.zero_v;             // transition role: dO = 0
   const bool store_ds = plan.kind != kPlanCpP1;        // phase 1 only maps the segment
+
+  // End (exclusive) of the processed range, decided before any setup. Gate-driven plan: a segment
+  // that ends inside the sequence starts from a zero gradient at the end of a window of later
+  // chunks whose decay bound is below 2^-64, else at the sequence end from dhT. With the exact
+  // stitch as fallback (plan.seg_ws, every segment's window after its end recorded by the probe
+  // kernel), the mirror of the forward: in phase 1, when the window after the predecessor's end (this
+  // segment's start) closes, the predecessor needs no end gradient and the CTA leaves; otherwise the
+  // segment's map is computed, or its start gradient straight from its own window (role 0). Phase 3
+  // starts from the window or from the stitched gradient.
+  int we = it.e;
+  if (it.gate) {
+    if (!is_last) {
+      const int w = gate_window_end(p, it, it.e, ss->wsum);
+      we = w >= 0 ? w : it.seq_e;
+    }
+  } else if (plan.seg_ws != nullptr && plan.kind == kPlanCpP1) {
+    if (plan.seg_ws[(size_t)(it.pi - 1) * p.Hv + it.j] >= 0) return;
+    if (it.seg + 1 < it.segs_used) {
+      const int w0 = plan.seg_ws[(size_t)it.pi * p.Hv + it.j];
+      if (w0 >= 0) {
+        if (it.role == 1) return;
+        we = w0;
+      }
+    }
+  } else if (plan.seg_ws != nullptr && plan.kind == kPlanCpP3 && it.seg + 1 < it.segs_used) {
+    const int w = plan.seg_ws[(size_t)it.pi * p.Hv + it.j];
+    if (w >= 0) we = w;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -111,7 +144,6 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&ss->gdone, 1);
     mbar_init(&ss->mma_done, 1);
     ss->abort_flag = 0;
-    ss->we = it.e;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -132,29 +164,19 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   __syncthreads();
   tc_fence_after();
 
-  // reverse warm-up window after the segment end
-  if (it.gate && !is_last) {
-    float logb = 0.f;
-    int end = it.seq_e;
-    for (int m = 0; m < kMaxWarm; ++m) {
-      const int cs = it.e + m * kChunk;
-      if (cs >= it.seq_e) break;
-      const int n = min(kChunk, it.seq_e - cs);
-      logb += chunk_log_bound(p, it, cs, n, ss->wsum);
-      if (logb <= kLogWarmBound) { end = cs + n; break; }
-    }
-    if (threadIdx.x == 0) ss->we = end;
-    __syncthreads();
-  }
-  const int we = ss->we;
   const int nchunks = (we - it.s + kChunk - 1) / kChunk;   // chunk c covers [s + 64c, min(s + 64c + 64, we))
   const bool from_seq_end = we == it.seq_e;
   int init_mode = kInitZero;
   const float* init_ptr = nullptr;
   float* dh0 = nullptr;                                    // destination of the start gradient
   if (exact) {
-    init_mode = it.init_mode;
-    init_ptr = it.init;
+    if (we == it.e) {                                    // from the item's end gradient
+      init_mode = it.init_mode;
+      init_ptr = it.init;
+    } else if (from_seq_end && p.h0) {                   // from a window that reaches the sequence end
+      init_mode = kInitPtr;
+      init_ptr = p.h0 + ((size_t)it.n * p.Hv + it.j) * (size_t)(128 * 128);
+    }
     dh0 = it.fin;
   } else {
     if (from_seq_end && p.h0) {

@@ -6,7 +6,7 @@
 //   gam = inclusive cumsum of g,  E_ij = exp(gam_i - gam_j)
 //   G = [K;Q] K^T   (one tcgen05 product, rows 0..63 = K K^T, rows 64..127 = Q K^T)
 //   L = strict_lower(diag(beta) K K^T * E)  -> fp16;  A = (I + L)^-1: 16 x 16 diagonal
-//       blocks by substitution, then one 8-column strip of A per warp (m16n8k16 products)
+//       blocks by substitution, then 2 x 2 blocking into 32 x 32 blocks (m16n8k16 products)
 //   P = lower_incl(Q K^T * E) * p_scale     -> bf16
 //   A2 = A diag(beta) -> bf16 (with B2 = A diag(beta exp(gam)), or A in bf16 and fp32)
 #pragma once
@@ -253,25 +253,6 @@ __device__ __forceinline__ void prep_masks(const PrepCtx& c, int s, uint32_t p_a
   tc::named_bar_sync(c.bar, kPrepThreads);
 }
 
-// Scale the 64 rows of a [64 x 128] bf16 tile held as two 8KB 128B-swizzled sub-tiles
-// (sub-tile 1 at +sub_stride) by f[row] * mult, in place.
-__device__ __forceinline__ void scale_rows_tile(const PrepCtx& c, uint8_t* tile, uint32_t sub_stride,
-                                                const float* f, float mult) {
-  uint4 qv[4];
-  uint8_t* qa[4];
-  float fs[4];
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int idx = c.pt + kPrepThreads * m;       // 0..1023
-    const int row = idx >> 4, half = (idx >> 3) & 1, ch = idx & 7;
-    qa[m] = tile + half * sub_stride + row * 128 + ch * 16;
-    fs[m] = f[row] * mult;
-    qv[m] = *reinterpret_cast<const uint4*>(qa[m]);
-  }
-#pragma unroll
-  for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(qa[m]) = scale_chunk(qv[m], fs[m]);
-}
-
 // Scale rows of a [64 x 128] bf16 tile (two 8KB 128B-swizzled sub-tiles, sub-tile 1 at
 // +sub_stride) by f[row] * mult, in place, with nt threads (t = this thread's index).
 __device__ __forceinline__ void scale_rows_tile_part(uint8_t* tile, uint32_t sub_stride, const float* f, float mult,
@@ -283,12 +264,13 @@ __device__ __forceinline__ void scale_rows_tile_part(uint8_t* tile, uint32_t sub
   }
 }
 
-// ---- fp16 variant of the inverse: L and the diagonal-block inverses D_R held as fp16
-// rows of stride kLdh (11-bit significand, as the tf32 products it replaces), the strip
-// products on m16n8k16 f16 tensor instructions (one per 16 x 16 block instead of two).
+// ---- the inverse: L and the diagonal-block inverses D_R held as fp16 rows of stride kLdh
+// (11-bit significand), the products below the diagonal on m16n8k16 f16 tensor instructions
+// with fp32 accumulation.
 
 // Diagonal 16 x 16 blocks, inverted in place (fp32 arithmetic, fp16 storage). Warps 0..3.
-__device__ __forceinline__ void prep_diag_inverse_h(const PrepCtx& c) {
+// af != nullptr: the blocks also go to af in fp32 (the stored-A layout, 64 x 64).
+__device__ __forceinline__ void prep_diag_inverse_h(const PrepCtx& c, float* af = nullptr) {
   __half* Lh = reinterpret_cast<__half*>(c.Lf);
   const int R = c.pw, col = c.lane & 15;
   float a[16];
@@ -319,6 +301,14 @@ __device__ __forceinline__ void prep_diag_inverse_h(const PrepCtx& c) {
   if (c.lane < 16) {
 #pragma unroll
     for (int ii = 0; ii < 16; ++ii) Lh[(16 * R + ii) * kLdh + 16 * R + col] = __float2half_rn(a[ii]);
+    if (af != nullptr) {
+      const int j = 16 * R + col;
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) {
+        const int i = 16 * R + ii;
+        af[i * kChunk + a_chunk(i, j >> 2) * 4 + (j & 3)] = a[ii];
+      }
+    }
   }
 }
 
@@ -352,86 +342,144 @@ __device__ __forceinline__ void acc_to_bfrag_h(const float* x, int lane, uint32_
   bf[1] = pack_h2(odd ? a3 : a2, odd ? b3 : b2);
 }
 
-// Column strip of A = (I + L)^-1 for warp w (columns 8w..8w+7, first block row R0 = w/2),
-// as prep_solve_strip_t, on the fp16 scratch.
-template <int R0>
-__device__ __forceinline__ void prep_solve_strip_h_t(const PrepCtx& c, float (&x)[4][4]) {
-  const __half* Lh = reinterpret_cast<const __half*>(c.Lf);
-  const int gid = c.lane >> 2, tig = c.lane & 3;
-  const int n0 = 8 * c.pw;
-  float t[4][4];
-#pragma unroll
-  for (int R = 0; R < 4; ++R)
-#pragma unroll
-    for (int u = 0; u < 4; ++u) t[R][u] = 0.f;
-#pragma unroll
-  for (int R = 0; R < R0; ++R)
-#pragma unroll
-    for (int u = 0; u < 4; ++u) x[R][u] = 0.f;
-  {
-    const __half2* d0 = reinterpret_cast<const __half2*>(Lh + (16 * R0 + gid) * kLdh + n0 + 2 * tig);
-    const __half2* d1 = reinterpret_cast<const __half2*>(Lh + (16 * R0 + gid + 8) * kLdh + n0 + 2 * tig);
-    const float2 f0 = __half22float2(*d0), f1 = __half22float2(*d1);
-    x[R0][0] = f0.x;
-    x[R0][1] = f0.y;
-    x[R0][2] = f1.x;
-    x[R0][3] = f1.y;
-  }
-#pragma unroll
-  for (int R = R0; R < 4; ++R) {
-    if (R > R0) {
-      uint32_t bt[2], af[4];
-      acc_to_bfrag_h(t[R], c.lane, bt);
-      lh_afrag(Lh, 16 * R, 16 * R, gid, tig, af);
-      float y[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_f16_16816(y, af, bt);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) x[R][u] = -y[u];
-    }
-    if (R < 3) {
-      uint32_t bx[2];
-      acc_to_bfrag_h(x[R], c.lane, bx);
-#pragma unroll
-      for (int R2 = R + 1; R2 < 4; ++R2) {
-        uint32_t af[4];
-        lh_afrag(Lh, 16 * R2, 16 * R, gid, tig, af);
-        mma_f16_16816(t[R2], af, bx);
-      }
-    }
-  }
+// B fragment (k16 x n8, the "col" operand of m16n8k16) of the fp16 scratch: B[k][n] at rows k0 + k,
+// columns n0 + n (b0 = rows 2 tig, 2 tig + 1; b1 = rows 2 tig + 8, 2 tig + 9; column gid)
+__device__ __forceinline__ void lh_bfrag(const __half* Lh, int k0, int n0, int gid, int tig, uint32_t* bf) {
+  const __half* p = Lh + (k0 + 2 * tig) * kLdh + n0 + gid;
+  __half2 h0 = __halves2half2(p[0], p[kLdh]);
+  __half2 h1 = __halves2half2(p[8 * kLdh], p[9 * kLdh]);
+  bf[0] = *reinterpret_cast<uint32_t*>(&h0);
+  bf[1] = *reinterpret_cast<uint32_t*>(&h1);
 }
-__device__ __forceinline__ void prep_solve_strip_h(const PrepCtx& c, float (&x)[4][4]) {
-  switch (c.pw >> 1) {                       // uniform over the warp
-    case 0: prep_solve_strip_h_t<0>(c, x); break;
-    case 1: prep_solve_strip_h_t<1>(c, x); break;
-    case 2: prep_solve_strip_h_t<2>(c, x); break;
-    default: prep_solve_strip_h_t<3>(c, x); break;
+
+// fp32 accumulator fragment (16 x 8) -> the fp16 scratch (rows r0 + gid (+8), columns n0 + 2 tig (+1))
+__device__ __forceinline__ void lh_store_acc(__half* Lh, int r0, int n0, int gid, int tig, const float* y) {
+  *reinterpret_cast<__half2*>(Lh + (r0 + gid) * kLdh + n0 + 2 * tig) = __floats2half2_rn(y[0], y[1]);
+  *reinterpret_cast<__half2*>(Lh + (r0 + gid + 8) * kLdh + n0 + 2 * tig) = __floats2half2_rn(y[2], y[3]);
+}
+
+// fp32 accumulator fragment (16 x 8) -> af (the stored-A layout), negated
+__device__ __forceinline__ void af_store_neg_acc(float* af, int r0, int n0, int gid, int tig, const float* y) {
+  const int j = n0 + 2 * tig;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = r0 + gid + 8 * h;
+    *reinterpret_cast<float2*>(af + i * kChunk + a_chunk(i, j >> 2) * 4 + (j & 3)) = make_float2(-y[2 * h], -y[2 * h + 1]);
   }
 }
 
-// A2 = A diag(beta) and (b2_addr != 0) B2 = A diag(beta exp(gam)) -> bf16 (128B-swizzled
-// rows at a2_addr, b2_addr) straight from a strip solve's fragments. kNorm: B2 multiplies the raw
-// K tile, so its columns also take rk (B2 = A diag(beta exp(gam) rk)).
-template <bool kNorm = false>
-__device__ __forceinline__ void prep_store_strip(const PrepCtx& c, int s, const float (&x)[4][4], uint32_t a2_addr,
-                                                 uint32_t b2_addr) {
-  const int w = c.pw, gid = c.lane >> 2, tig = c.lane & 3;
-  const int j = 8 * w + 2 * tig;
-  const float b0 = c.cs->bet[s][j], b1 = c.cs->bet[s][j + 1];
-  const float* ek = kNorm ? c.cs->egk[s] : c.cs->eg[s];
-  const float e0 = b0 * ek[j], e1 = b1 * ek[j + 1];
-#pragma unroll
-  for (int R = 0; R < 4; ++R) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = 16 * R + gid + 8 * h;
-      const uint32_t off = tc::sw128(i, w) + 4 * tig;
-      const float v0 = x[R][2 * h], v1 = x[R][2 * h + 1];
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2_addr + off), "r"(tc::pack_bf16(v0 * b0, v1 * b1)) : "memory");
-      if (b2_addr)
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(b2_addr + off), "r"(tc::pack_bf16(v0 * e0, v1 * e1)) : "memory");
-    }
+// Zero the strictly upper 16 x 16 blocks of af (the stored-A layout), with nt threads.
+__device__ __forceinline__ void af_zero_upper(float* af, int t, int nt) {
+  // blocks (R, C), C > R: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3); 16 rows x 4 16-byte pieces each
+  for (int idx = t; idx < 6 * 64; idx += nt) {
+    const int blk = idx >> 6, rem = idx & 63;
+    const int R = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+    const int C = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+    const int i = 16 * R + (rem >> 2), k = 4 * C + (rem & 3);
+    *reinterpret_cast<float4*>(af + i * kChunk + a_chunk(i, k) * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+
+// A = (I + L)^-1 below its 16 x 16 diagonal blocks D_R (already inverted in place in the fp16
+// scratch and written to af by prep_diag_inverse_h), by 2 x 2 blocking into 32 x 32 blocks:
+//   X10 = -D1 L10 D0,  X32 = -D3 L32 D2        (the 32 x 32 diagonal blocks A11, A22)
+//   T   = L21 A11 = [L21a D0 + L21b X10 | L21b D1]   (L21 = [L21a | L21b], rows 32..63, cols 0..31)
+//   A21 = -A22 T = -[D2 T_top ; X32 T_top + D3 T_bot]
+// on m16n8k16 f16 products with fp32 accumulation: X10 / X32 on warps 0..3 (one 8-column tile
+// each, two dependent products through shuffles), T on warps 4..7 (two tiles each), A21 on all
+// eight (one tile each). X10, X32 replace L10, L32 in the scratch; T goes to its unused upper
+// right 32 x 32 block (rows 0..31, columns 32..63). Every result goes to af in fp32. Three group
+// barriers inside; the caller separates the last af writes from their readers with a barrier.
+__device__ __forceinline__ void prep_inverse_blocked(const PrepCtx& c, float* af) {
+  __half* Lh = reinterpret_cast<__half*>(c.Lf);
+  const int w = c.pw, gid = c.lane >> 2, tig = c.lane & 3;
+  float x[4] = {0.f, 0.f, 0.f, 0.f};        // warps 0..3: the X tile
+  float ta[4] = {0.f, 0.f, 0.f, 0.f};       // warps 4..7: T tile in columns 0..15 (two terms)
+  float tb[4] = {0.f, 0.f, 0.f, 0.f};       // warps 4..7: T tile in columns 16..31
+  const int m = w & 3, tr = (m >> 1) * 16;  // warps 4..7: T rows tr .. tr + 15 (L rows 32 + tr ..)
+  const int na = 8 * (m & 1);               // T columns of ta: na .. na + 7; of tb: 16 + na ..
+  const int base = (w & 2) ? 32 : 0;        // warps 0..3: (D0, L10, D1) at 0, (D2, L32, D3) at 32
+  const int nx = base + 8 * (w & 1);        // X tile columns
+  if (w < 4) {
+    uint32_t af_[4], bf[2], bt[2];
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    lh_afrag(Lh, base + 16, base, gid, tig, af_);           // L10 / L32
+    lh_bfrag(Lh, base, nx, gid, tig, bf);                   // D0 / D2, columns nx ..
+    mma_f16_16816(y, af_, bf);
+    acc_to_bfrag_h(y, c.lane, bt);
+    lh_afrag(Lh, base + 16, base + 16, gid, tig, af_);      // D1 / D3
+    mma_f16_16816(x, af_, bt);                              // x = D1 L10 D0 (tile); X = -x
+  } else {
+    uint32_t af_[4], bf[2];
+    lh_afrag(Lh, 32 + tr, 0, gid, tig, af_);                // L21a
+    lh_bfrag(Lh, 0, na, gid, tig, bf);                      // D0
+    mma_f16_16816(ta, af_, bf);
+    lh_afrag(Lh, 32 + tr, 16, gid, tig, af_);               // L21b
+    lh_bfrag(Lh, 16, 16 + na, gid, tig, bf);                // D1
+    mma_f16_16816(tb, af_, bf);
+  }
+  tc::named_bar_sync(c.bar, kPrepThreads);                  // L10 and L32 are read
+  if (w < 4) {
+    const float nxv[4] = {-x[0], -x[1], -x[2], -x[3]};
+    lh_store_acc(Lh, base + 16, nx, gid, tig, nxv);
+    af_store_neg_acc(af, base + 16, nx, gid, tig, x);
+  }
+  tc::named_bar_sync(c.bar, kPrepThreads);                  // X10 (and X32) in the scratch
+  if (w >= 4) {
+    uint32_t af_[4], bf[2];
+    lh_afrag(Lh, 32 + tr, 16, gid, tig, af_);               // L21b
+    lh_bfrag(Lh, 16, na, gid, tig, bf);                     // X10, columns na ..
+    mma_f16_16816(ta, af_, bf);
+    lh_store_acc(Lh, tr, 32 + na, gid, tig, ta);            // T -> rows 0..31, columns 32..63
+    lh_store_acc(Lh, tr, 48 + na, gid, tig, tb);
+  }
+  tc::named_bar_sync(c.bar, kPrepThreads);                  // T in the scratch
+  {
+    const int rb = w >> 2, nt = w & 3;                      // A21 rows 32 + 16 rb .., columns 8 nt ..
+    uint32_t af_[4], bf[2];
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    lh_bfrag(Lh, 0, 32 + 8 * nt, gid, tig, bf);             // T_top
+    if (rb == 0) {
+      lh_afrag(Lh, 32, 32, gid, tig, af_);                  // D2
+      mma_f16_16816(y, af_, bf);
+    } else {
+      lh_afrag(Lh, 48, 32, gid, tig, af_);                  // X32
+      mma_f16_16816(y, af_, bf);
+      lh_bfrag(Lh, 16, 32 + 8 * nt, gid, tig, bf);          // T_bot
+      lh_afrag(Lh, 48, 48, gid, tig, af_);                  // D3
+      mma_f16_16816(y, af_, bf);
+    }
+    af_store_neg_acc(af, 32 + 16 * rb, 8 * nt, gid, tig, y);
+  }
+}
+
+// A2 = A diag(beta) and B2 = A diag(beta exp(gam)) -> bf16 (128B-swizzled rows at a2_addr,
+// b2_addr) from A in fp32 (af, the stored-A layout); thread: 16 columns of one row. kNorm: B2
+// multiplies the raw K tile, so its columns also take rk.
+template <bool kNorm = false>
+__device__ __forceinline__ void prep_store_a_f32(const PrepCtx& c, int s, const float* af, uint32_t a2_addr,
+                                                 uint32_t b2_addr) {
+  const int i = c.pt & 63, qq = c.pt >> 6;
+  const float* bet = c.cs->bet[s];
+  const float* ek = kNorm ? c.cs->egk[s] : c.cs->eg[s];
+  float a[16];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 t = *reinterpret_cast<const float4*>(af + i * kChunk + a_chunk(i, 4 * qq + u) * 4);
+    a[4 * u] = t.x; a[4 * u + 1] = t.y; a[4 * u + 2] = t.z; a[4 * u + 3] = t.w;
+  }
+  uint32_t w2[8], wb[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int j0 = qq * 16 + 2 * u;
+    const float b0 = bet[j0], b1 = bet[j0 + 1];
+    w2[u] = tc::pack_bf16(a[2 * u] * b0, a[2 * u + 1] * b1);
+    wb[u] = tc::pack_bf16(a[2 * u] * (b0 * ek[j0]), a[2 * u + 1] * (b1 * ek[j0 + 1]));
+  }
+  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq), w2[0], w2[1], w2[2], w2[3]);
+  st_shared_v4(a2_addr + tc::sw128(i, 2 * qq + 1), w2[4], w2[5], w2[6], w2[7]);
+  st_shared_v4(b2_addr + tc::sw128(i, 2 * qq), wb[0], wb[1], wb[2], wb[3]);
+  st_shared_v4(b2_addr + tc::sw128(i, 2 * qq + 1), wb[4], wb[5], wb[6], wb[7]);
 }
 
 // A2 = A diag(beta) and A -> bf16 (128B-swizzled rows at a2_addr, a_addr) from the fp32 rows
@@ -473,42 +521,6 @@ __device__ __forceinline__ void prep_fetch_a(const PrepCtx& c, const float* a_g)
     tc::cp_async_16(tc::smem_u32(c.Lf + ar * kLd + c16 * 4), a_g + ar * kChunk + a_chunk(ar, c16) * 4);
   }
   tc::cp_async_commit();
-}
-
-// A strip's fragments (prep_solve_strip_h) -> the stored-A layout at a_s (shared memory).
-__device__ __forceinline__ void prep_stage_strip_a(const PrepCtx& c, const float (&x)[4][4], float* a_s) {
-  const int gid = c.lane >> 2, tig = c.lane & 3;
-  const int j = 8 * c.pw + 2 * tig;
-#pragma unroll
-  for (int R = 0; R < 4; ++R)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = 16 * R + gid + 8 * h;
-      *reinterpret_cast<float2*>(a_s + i * kChunk + a_chunk(i, j >> 2) * 4 + (j & 3)) =
-          make_float2(x[R][2 * h], x[R][2 * h + 1]);
-    }
-}
-
-// A2 = A diag(beta) and A -> bf16 (128B-swizzled rows at a2_addr, a_addr), and A -> fp32
-// rows of stride kLd in the scratch, from prep_solve_strip_h's fragments. The caller
-// separates this from the solve with a group barrier (the fp32 rows overwrite the fp16 L).
-__device__ __forceinline__ void prep_store_strip_a(const PrepCtx& c, int s, const float (&x)[4][4], uint32_t a2_addr,
-                                                   uint32_t a_addr) {
-  const int w = c.pw, gid = c.lane >> 2, tig = c.lane & 3;
-  const int j = 8 * w + 2 * tig;
-  const float b0 = c.cs->bet[s][j], b1 = c.cs->bet[s][j + 1];
-#pragma unroll
-  for (int R = 0; R < 4; ++R) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = 16 * R + gid + 8 * h;
-      const uint32_t off = tc::sw128(i, w) + 4 * tig;
-      const float v0 = x[R][2 * h], v1 = x[R][2 * h + 1];
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2_addr + off), "r"(tc::pack_bf16(v0 * b0, v1 * b1)) : "memory");
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a_addr + off), "r"(tc::pack_bf16(v0, v1)) : "memory");
-      *reinterpret_cast<float2*>(c.Lf + i * kLd + j) = make_float2(v0, v1);
-    }
-  }
 }
 
 }  // namespace gdn

@@ -98,7 +98,7 @@ __device__ __forceinline__ bool seq_span(const FwdParams& p, int n, int& b, int&
 // ---- host-side launch instrumentation (gdn_api.cu)
 enum KernelId : int { kKernFwdTc = 0, kKernFwdSimt = 1, kKernCpStitch = 2, kKernBwdTc = 3,
                       kKernBwdSimt = 4, kKernBwdReduce = 5, kKernCpPlan = 6, kKernBwdChain = 7,
-                      kKernStep = 8, kKernCount = 9 };
+                      kKernStep = 8, kKernCpProbe = 9, kKernCount = 10 };
 void trace_pre(int kernel_id, cudaStream_t st);
 void set_last_error(const char* msg);   // text returned by gdn_last_error() on this thread
 void trace_post(cudaStream_t st);

@@ -56,13 +56,12 @@ constexpr uint32_t kOffSb = 128u * 1024u;       // 32KB     S in bf16 (two 64-co
 constexpr uint32_t kOffYt = 160u * 1024u;       // 16KB     Delta^T, bf16 [dv][token]
 constexpr uint32_t kOffDt = 176u * 1024u;       // 16KB     Delta~^T, then O staging (two swizzled 64-column halves)
 constexpr uint32_t kOffLf = 192u * 1024u;       // fp16 [64][kLdh] L, diagonal blocks inverted in place
-constexpr uint32_t kOffAst = kOffLf + 64u * kLdh * 2u;   // 16KB  A staged for its bulk copy (state-store mode)
+constexpr uint32_t kOffAst = kOffLf + 64u * kLdh * 2u;   // 16KB  A in fp32 (stored-A layout; bulk-copied for the backward)
 constexpr uint32_t kOffSmall = kOffAst + 16384u;
 
 struct Small {
   ChunkScalars cs;
   float wsum[16];         // warm-up window search: per-warp partial sums
-  int ws;                 // warm-up start token (context parallelism)
   uint64_t full_k[2], full_qv[2], prep_full[2], gdone, wdone, mma_done, dd_free;
   uint64_t stall;         // testing only: a barrier that nothing completes
   uint32_t tmem_base;
@@ -109,9 +108,47 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (threadIdx.x == 0) report_error(p, kDevMisaligned);
     return;
   }
+  if (plan.seg_ws != nullptr && plan.kind == kPlanCpP1) {
+    // exact fallback, phase 1: item = (pi * 2 + role) * Hv + j. When the successor's window closes
+    // (the probe's record, read before anything else) no map is needed: leave at once.
+    const int j = blockIdx.x % p.Hv, pi = blockIdx.x / (2 * p.Hv);
+    if ((pi + 1) * 2 * p.Hv < (int)gridDim.x && plan.seg_ws[(size_t)(pi + 1) * p.Hv + j] >= 0) return;
+  }
   WorkItem it;
   if (!get_work_item(p, plan, blockIdx.x, it)) return;   // uniform over the CTA
   const __nv_bfloat16* beta = static_cast<const __nv_bfloat16*>(p.beta);
+
+  // First token this CTA processes (ws), decided before any setup so that a phase-1 CTA with
+  // nothing to do leaves at once. Gate-driven warm-up (context parallelism): a segment that starts
+  // inside a sequence begins from a zero state at the start of a window of earlier chunks whose
+  // transition has spectral norm <= prod_t exp(g_t) max(1, |1 - beta_t |k_t|^2|) <= 2^-64: the
+  // state it drops is then below fp32 resolution. Each token's factor is the exact norm of
+  // exp(g)(I - beta k k^T); the window walks back chunk by chunk (at most kMaxWarm chunks).
+  //   gate-driven plan: without such a window the segment starts at the sequence start with h0.
+  //   with the exact stitch as fallback (plan.seg_ws, every segment's window recorded by the
+  //     probe kernel): in phase 1, when the successor's window closes it needs no map and the CTA
+  //     leaves; otherwise the segment's map is computed, or, when the segment's own window closes,
+  //     its end state straight from that window (role 0). Phase 3 starts from the window or from
+  //     the stitched state.
+  int ws = it.s;
+  if (it.gate) {
+    if (it.s > it.seq_s) {
+      const int w = gate_window_start(p, it, it.s, ss->wsum);
+      ws = w >= 0 ? w : it.seq_s;
+    }
+  } else if (plan.seg_ws != nullptr && plan.kind == kPlanCpP1) {
+    if (plan.seg_ws[(size_t)(it.pi + 1) * p.Hv + it.j] >= 0) return;
+    if (it.seg > 0) {
+      const int w0 = plan.seg_ws[(size_t)it.pi * p.Hv + it.j];
+      if (w0 >= 0) {
+        if (it.role == 1) return;
+        ws = w0;
+      }
+    }
+  } else if (plan.seg_ws != nullptr && plan.kind == kPlanCpP3 && it.seg > 0) {
+    const int w = plan.seg_ws[(size_t)it.pi * p.Hv + it.j];
+    if (w >= 0) ws = w;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -125,7 +162,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(&ss->mma_done, 1);
     mbar_init(&ss->stall, 1);
     ss->abort_flag = 0;
-    ss->ws = it.s;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -152,25 +188,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
   }
 
-  // Gate-driven warm-up (context parallelism): a segment that starts inside a sequence
-  // begins from a zero state at the start of a window of earlier chunks whose transition
-  // has spectral norm <= prod_t exp(g_t) max(1, |1 - beta_t |k_t|^2|) <= 2^-64: the state
-  // it drops is then below fp32 resolution. Each token's factor is the exact norm of
-  // exp(g)(I - beta k k^T); the window walks back chunk by chunk (at most kMaxWarm chunks,
-  // otherwise the segment starts at the sequence start with h0: the exact recurrence).
-  if (it.gate && it.s > it.seq_s) {
-    float logb = 0.f;
-    int start = it.seq_s;
-    for (int m = 1; m <= kMaxWarm; ++m) {
-      const int cs = it.s - m * kChunk;
-      if (cs < it.seq_s) break;
-      logb += chunk_log_bound(p, it, cs, kChunk, ss->wsum);
-      if (logb <= kLogWarmBound) { start = cs; break; }
-    }
-    if (threadIdx.x == 0) ss->ws = start;
-    __syncthreads();
-  }
-  const int ws = ss->ws;                          // first token processed (warm-up start)
   const int nchunks = (it.e - ws + kChunk - 1) / kChunk;
   const bool from_seq_start = (ws == it.seq_s);
   const int init_mode = (ws == it.s) ? it.init_mode : (from_seq_start && p.h0 ? (int)kInitPtr : (int)kInitZero);
@@ -273,26 +290,27 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_after();
       pc.colG = gw_col;
       prep_masks<true, kNorm>(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
-      // diagonal blocks of (I + L)^-1 (warps 0-3) while warps 4-7 form Q <- diag(exp(gam)) Q
-      // (times rq: the normalised rows) in place (the Gram product has consumed Q); then one
-      // column strip of A per warp
-      if (warp < 4) prep_diag_inverse_h(pc);
-      else scale_rows_tile_part(st + kOffQ, kHalf, kNorm ? ss->cs.egq[s] : ss->cs.eg[s], 1.f, pt - 128, 128);
-      named_bar_sync(kBarPrep, kNumPrep);
-      {
-        float x[4][4];
-        prep_solve_strip_h(pc, x);
-        const int t0 = ws + c * kChunk;
-        if (p.states != nullptr && p.chunk_a != nullptr && t0 >= it.s)   // A for the backward (copied below)
-          prep_stage_strip_a(pc, x, reinterpret_cast<float*>(sm + kOffAst));
-        // the previous chunk's U / W products have read A2, B2 (their completion is almost
-        // always past by now)
-        if (c > 0) {
-          ok = ok && mbar_wait(&ss->wdone, (c - 1) & 1, abort_flag);
-          ok = __all_sync(0xffffffffu, ok);
-        }
-        prep_store_strip<kNorm>(pc, s, x, sbase + kOffA2, sbase + kOffB2);
+      // A = (I + L)^-1 in fp32 into the A staging buffer (also the backward's copy): diagonal
+      // blocks on warps 0-3 while warps 4-7 form Q <- diag(exp(gam)) Q (times rq: the normalised
+      // rows) in place (the Gram product has consumed Q) and clear A's upper blocks; then the
+      // blocked inverse below the diagonal
+      float* af = reinterpret_cast<float*>(sm + kOffAst);
+      if (warp < 4) {
+        prep_diag_inverse_h(pc, af);
+      } else {
+        scale_rows_tile_part(st + kOffQ, kHalf, kNorm ? ss->cs.egq[s] : ss->cs.eg[s], 1.f, pt - 128, 128);
+        af_zero_upper(af, pt - 128, 128);
       }
+      named_bar_sync(kBarPrep, kNumPrep);
+      prep_inverse_blocked(pc, af);
+      // the previous chunk's U / W products have read A2, B2 (their completion is almost
+      // always past by now)
+      if (c > 0) {
+        ok = ok && mbar_wait(&ss->wdone, (c - 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      named_bar_sync(kBarPrep, kNumPrep);              // A complete in fp32
+      prep_store_a_f32<kNorm>(pc, s, af, sbase + kOffA2, sbase + kOffB2);
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && p.states != nullptr && p.chunk_p != nullptr && ws + c * kChunk >= it.s && ok) {

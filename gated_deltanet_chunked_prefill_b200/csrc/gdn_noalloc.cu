@@ -59,7 +59,15 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int H
                                              const void* beta, float scale, const float* h0,
                                              const int32_t* cu_seqlens, int num_seqs, void* o, float* hT,
                                              const gdn_options* opt, cudaStream_t stream) {
-  const size_t need = gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, cu_seqlens ? num_seqs : 0, opt);
+  gdn_options op{};
+  if (opt) op = *opt;
+  size_t need = gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, cu_seqlens ? num_seqs : 0, &op);
+  if (need > kNoAllocScratchBytes && op.cp_exact == 2) {
+    // the exact fallback of the gate-driven start keeps per-segment maps; with too little room, the
+    // other fallback (restart at the sequence start) needs only the segment table
+    op.cp_exact = 0;
+    need = gdn_chunk_fwd_workspace_size(B, T, Hqk, Hv, dk, dv, cu_seqlens ? num_seqs : 0, &op);
+  }
   if (need > kNoAllocScratchBytes) {                             // beyond the fixed array
     char msg[160];
     snprintf(msg, sizeof(msg), "gdn_chunk_fwd_noalloc: needs %zu bytes of scratch, the static array holds %zu",
@@ -79,5 +87,5 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int H
     return GDN_ERR_CUDA;
   }
   return gdn_chunk_fwd(dtype, B, T, Hqk, Hv, dk, dv, q, k, v, g, beta, scale, h0, cu_seqlens, num_seqs, o, hT,
-                       scratch, kNoAllocScratchBytes, opt, stream);
+                       scratch, kNoAllocScratchBytes, &op, stream);
 }

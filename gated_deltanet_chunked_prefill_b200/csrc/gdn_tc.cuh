@@ -63,11 +63,16 @@ struct TcPlan {
   const int* table_count;
   float* seg_state;      // [pairs][Hv][dk][dv] fp32: start state of segment pi (exact stitch)
   float* seg_trans;      // [pairs][Hv][dk][dk] fp32: transition of segment pi (exact stitch)
+  // Gate-driven start with the exact stitch as its fallback (nullable; phases 1 and 3 and the
+  // stitch): [pairs][Hv] the first token of segment pi's warm-up window when its window closes,
+  // else -1 (the segment then starts from its stitched state). Reverse chain: the window's end.
+  int* seg_ws;
 };
 
 struct WorkItem {
   int n, j, hq, b, s, e;  // sequence, v-head, q/k head, batch row, token range [s, e)
   int seq_s, seq_e;       // token range of the whole sequence
+  int seg, segs_used, pi, role;   // context-parallel plans: segment, segments of the sequence, pair, role
   bool gate;              // may start earlier than s with a warm-up window (kPlanGate)
   int init_mode;
   const float* init;      // [dk][dv] fp32 when init_mode == kInitPtr
@@ -94,6 +99,10 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
   w.init = nullptr;
   w.init_mode = kInitZero;
   w.gate = false;
+  w.seg = 0;
+  w.segs_used = 1;
+  w.pi = 0;
+  w.role = 0;
   if (plan.kind == kPlanUnits) {
     w.j = item % p.Hv;
     w.n = item / p.Hv;
@@ -135,6 +144,10 @@ __device__ __forceinline__ bool get_work_item(const FwdParams& p, const TcPlan& 
   w.hq = w.j / (p.Hv / p.Hqk);
   w.s = s + seg * plan.seg_chunks * kChunk;
   w.e = min(e, w.s + plan.seg_chunks * kChunk);
+  w.seg = seg;
+  w.segs_used = segs_used;
+  w.pi = pi;
+  w.role = role;
   const float* h0u = p.h0 ? p.h0 + ((size_t)w.n * p.Hv + w.j) * hsz : nullptr;
   if (reverse) {
     const bool last = seg + 1 == segs_used;
@@ -231,6 +244,34 @@ __device__ __forceinline__ float chunk_log_bound(const FwdParams& p, const WorkI
   return tot;
 }
 
+// First token of the shortest window of whole chunks before token `s` (at most kMaxWarm, within the
+// sequence) whose transition has spectral norm <= 2^-64, or -1 if there is none. CTA-wide.
+__device__ __forceinline__ int gate_window_start(const FwdParams& p, const WorkItem& it, int s, float* wsum) {
+  float logb = 0.f;
+  for (int m = 1; m <= kMaxWarm; ++m) {
+    const int cs = s - m * kChunk;
+    if (cs < it.seq_s) break;
+    logb += chunk_log_bound(p, it, cs, kChunk, wsum);
+    if (logb <= kLogWarmBound) return cs;
+  }
+  return -1;
+}
+
+// Reverse chain: the end (exclusive) of the shortest window of chunks after token `e` (at most
+// kMaxWarm, within the sequence) whose transition bound is <= 2^-64 (the adjoint's norm equals
+// the transition's), or -1. CTA-wide.
+__device__ __forceinline__ int gate_window_end(const FwdParams& p, const WorkItem& it, int e, float* wsum) {
+  float logb = 0.f;
+  for (int m = 0; m < kMaxWarm; ++m) {
+    const int cs = e + m * kChunk;
+    if (cs >= it.seq_e) break;
+    const int n = min(kChunk, it.seq_e - cs);
+    logb += chunk_log_bound(p, it, cs, n, wsum);
+    if (logb <= kLogWarmBound) return cs + n;
+  }
+  return -1;
+}
+
 cudaError_t launch_fwd_tc(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st,
                           const char** what);
 // Backward, reverse state-gradient chain (see gdn_bwd_chain.cu for the parameter mapping).
@@ -241,6 +282,12 @@ cudaError_t launch_cp_plan(const FwdParams& p, int seg_chunks, int max_pairs, in
                            int* first_pair, int* chunk_off, cudaStream_t st);
 // Exact stitch, phase 2: chain the segment maps h_{s+1} = M_s h_s + b_s in place; reverse (the
 // backward's state gradient): dh_end(s) = M_{s+1} dh_end(s + 1) + c_{s+1}, from the sequence end.
+// Gate-driven start with the exact fallback: the window of every segment and v-head into plan.seg_ws
+// (forward: before the segment's start; reverse: after its end), before phase 1.
+cudaError_t launch_cp_probe(const FwdParams& p, const TcPlan& plan, int num_items, cudaStream_t st, bool reverse);
+// With plan.seg_ws (gate-driven start with the exact fallback) only the segments whose window does
+// not close are chained; a segment whose predecessor's end state came straight from phase 1 (the
+// sequence start, or a window that closes) restarts the chain.
 cudaError_t launch_cp_stitch(const FwdParams& p, const TcPlan& plan, const int* first_pair, cudaStream_t st,
                              bool reverse = false);
 

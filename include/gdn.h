@@ -88,16 +88,23 @@ typedef struct {
   /* Finer control of the segment length, overriding cp_mode when nonzero: n > 0 = segments
    * of n chunks (64 tokens each), -1 = off. */
   int cp_segment_chunks;
-  /* How a segment obtains its start state.
-   * 0 (default): gate-driven. The segment's CTA runs, from a zero state, the
-   *   shortest window of preceding chunks whose transition has spectral norm
-   *   <= 2^-64 (each token's factor exp(g) max(1, |1 - beta |k|^2|) is exact), so
-   *   the dropped part is below fp32 resolution; with no such window within 16
-   *   chunks it starts at the sequence start (the plain recurrence).
-   * 1: exact affine stitch. Phase 1 computes every segment's map
-   *   h_end = M h_start + b, phase 2 chains the maps, phase 3 reruns each segment
-   *   from its stitched start state. The backward mirrors it on the state gradient:
-   *   dh_start = M'^T dh_end + c, chained from the sequence end. */
+  /* How a segment obtains its start state (0, 1 or 2; anything else GDN_ERR_INVALID_ARG).
+   * Gate-driven start: the segment's CTA runs, from a zero state, the shortest window of
+   *   preceding chunks whose transition has spectral norm <= 2^-64 (each token's factor
+   *   exp(g) max(1, |1 - beta |k|^2|) is exact), so the dropped part is below fp32
+   *   resolution. The backward's reverse chain does the same after a segment's end.
+   * Exact affine stitch: phase 1 computes a segment's map h_end = M h_start + b, phase 2
+   *   chains the maps, phase 3 reruns the segment from its stitched start state. The backward
+   *   mirrors it on the state gradient, dh_start = M' dh_end + c, chained from the sequence end.
+   * 0 (default): gate-driven; a segment without such a window within 16 chunks (weakly
+   *   decaying heads) restarts at the sequence start (the plain recurrence). The smallest
+   *   workspace: no per-segment maps.
+   * 1: the exact stitch for every segment.
+   * 2: gate-driven, with the exact stitch for the segments whose window does not close, once a
+   *   sequence can have 3 or more segments (with 2, as 0). A probe kernel records every
+   *   segment's window first and phase 1 maps only the segments that need it; the two extra
+   *   launches and phase 1's grid cost tens of microseconds even when every window closes, so
+   *   this pays off for long sequences with weakly decaying heads. */
   int cp_exact;
   /* Chunk start states cached between a forward and its backward (tensor-core path:
    * bf16, dk = dv = 128), device memory of gdn_chunk_states_size() bytes, 16-byte
@@ -209,7 +216,9 @@ gdn_status gdn_recurrent_step(gdn_dtype dtype, int N, int Hqk, int Hv, int dk, i
  * until the process exits; the call allocates nothing (no cudaMalloc, no library
  * allocator). Calls whose scratch need (gdn_chunk_fwd_workspace_size) exceeds 1 MiB,
  * e.g. the exact affine stitch (cp_exact) on large inputs, return GDN_ERR_WORKSPACE
- * with the sizes in gdn_last_error(). The first call on a device looks up the array's
+ * with the sizes in gdn_last_error(). With cp_exact = 2 and too little room for its
+ * per-segment maps, the call uses cp_exact = 0 (segments without a closing window restart
+ * at the sequence start). The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress, once per device); make that first call before
  * any stream capture. The address is kept for the life of the process: after a
  * cudaDeviceReset the array is reloaded elsewhere, so do not use this entry point on a

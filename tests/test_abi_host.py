@@ -76,7 +76,7 @@ def test_forward_rejects_reserved_options():
 
 
 @pytest.mark.parametrize("field,value", [("deterministic", 2), ("qk_l2norm", -1), ("test_stall", 3),
-                                         ("cp_mode", -2)])
+                                         ("cp_mode", -2), ("cp_exact", 3), ("cp_exact", -1)])
 def test_forward_rejects_option_values_out_of_range(field, value):
     o = gdn.Options()
     setattr(o, field, value)
@@ -104,6 +104,17 @@ def test_cp_mode_gives_the_segment_count():
     # cp_segment_chunks, when set, wins over cp_mode
     assert gdn.fwd_workspace_size(*dims, cp_mode=4, cp_segment_chunks=8, cp_exact=True) == \
         gdn.fwd_workspace_size(*dims, cp_segment_chunks=8, cp_exact=True)
+
+
+def test_context_parallel_modes_workspace():
+    """The exact fallback (mode 2) keeps per-segment maps and window records only once a sequence can
+    have 3 or more segments; the restart mode (0) needs none; the exact stitch (1) always has maps."""
+    dims = (1, 8192, 1, 8, 128, 128, 1)             # 128 chunks
+    ws = lambda **kw: gdn.fwd_workspace_size(*dims, **kw)
+    maps = 2 * 4 * 8 * 128 * 128 * 4               # 4 segments x 8 v-heads x (M, b), fp32
+    assert ws(cp_segment_chunks=32, cp_exact=0) + maps <= ws(cp_segment_chunks=32, cp_exact=2)
+    assert ws(cp_segment_chunks=32, cp_exact=1) + 4 * 8 * 4 <= ws(cp_segment_chunks=32, cp_exact=2) + 256
+    assert ws(cp_segment_chunks=64, cp_exact=2) == ws(cp_segment_chunks=64, cp_exact=0)   # 2 segments
 
 
 def test_interface_names():

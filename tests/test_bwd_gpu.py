@@ -76,6 +76,39 @@ def test_bwd_weak_decay_cp(exact):
             assert_close(gr[n], ref[n], "bf16", f"weak decay cp={cp} exact={exact} {n}")
 
 
+@pytest.mark.parametrize("pattern", ["weak", "weak_then_strong", "strong_then_weak", "mixed_heads"])
+@pytest.mark.parametrize("cp_exact", [2, 0])
+def test_bwd_gate_with_exact_fallback(pattern, cp_exact):
+    """Mode 2: the state pass and the reverse chain give segments whose window does not close the
+    exact stitch (each direction its own windows); mode 0 restarts them at the sequence end / start.
+    3-chunk segments; all six gradients. g x 0.02
+    over 1000 tokens: no window closes within 16 chunks, and the unsplit path still meets the bf16
+    bars (much longer weakly decaying memories make |dg| large enough that no path does)."""
+    from test_fwd_gpu import _decay_pattern
+    x = _decay_pattern(make_inputs(1, 1000, 1, 2, 128, 128, "bf16", seed=35, h0_std=0.1, backward=True),
+                       pattern, 0.02)
+    gr = run_gpu_bwd(x, cp_segment_chunks=3, cp_exact=cp_exact)
+    ref = oracle_bwd(x)
+    for n in GRADS:
+        assert_close(gr[n], ref[n], "bf16", f"{pattern} mode {cp_exact} {n}")
+
+
+def test_bwd_gate_fallback_packed_cache():
+    """Packed sequences with mixed decay per v-head, the exact fallback (mode 2), through the forward's
+    cache and through the backward's own state pass: bit-identical, and matching the oracle."""
+    from test_fwd_gpu import _decay_pattern
+    x = _decay_pattern(make_inputs(1, 0, 2, 4, 128, 128, "bf16", seed=36, h0_std=0.1, backward=True,
+                                   lengths=[900, 64, 1, 650, 300]), "mixed_heads", 0.02)
+    d = to_dev(x)
+    states = _fwd_states(d, cp_segment_chunks=2, cp_exact=2)
+    cached = _bwd(d, cp_segment_chunks=2, cp_exact=2, states=states)
+    recomputed = _bwd(d, cp_segment_chunks=2, cp_exact=2)
+    ref = oracle_bwd(x)
+    for n in GRADS:
+        assert torch.equal(cached[n], recomputed[n]), n
+        assert_close(cached[n], ref[n], "bf16", f"packed fallback {n}")
+
+
 def test_bwd_exact_stitch_grouped_values_and_cache():
     """Exact stitch in both passes with grouped values; the forward's cache (exact stitch too) gives
     the same gradients, bit for bit, as the backward's own exact state pass."""

@@ -73,6 +73,48 @@ def test_fwd_weak_decay_long_sequence():
         assert_close(hT, rh, "bf16", f"weak decay cp={cp} exact={exact} hT")
 
 
+def _decay_pattern(x, pattern, f=0.01):
+    """g scaled along the sequence (and per v-head): 'weak' x f everywhere; 'weak_then_strong'
+    / 'strong_then_weak' x f in one half of each sequence; 'mixed_heads' x f on even v-heads."""
+    g = x["g"].clone()
+    T = g.shape[1]
+    if pattern == "weak":
+        g *= f
+    elif pattern == "weak_then_strong":
+        g[:, : T // 2] *= f
+    elif pattern == "strong_then_weak":
+        g[:, T // 2:] *= f
+    elif pattern == "mixed_heads":
+        g[:, :, 0::2] *= f
+    x["g"] = g.contiguous()
+    return x
+
+
+@pytest.mark.parametrize("pattern", ["weak", "weak_then_strong", "strong_then_weak", "mixed_heads"])
+@pytest.mark.parametrize("cp_exact", [2, 0])
+def test_fwd_gate_with_exact_fallback(pattern, cp_exact):
+    """Segments whose gate window does not close: mode 2 gives them the exact stitch (only where
+    needed: a segment after a closing window gets its start straight from phase 1), the default mode
+    (0) restarts them at the sequence start; both match the oracle. 3-chunk segments, so a sequence
+    has many of them, some closing and some not."""
+    x = _decay_pattern(make_inputs(2, 2500, 1, 2, 128, 128, "bf16", seed=17, h0_std=0.1), pattern)
+    o, hT = run_gpu(x, cp_segment_chunks=3, cp_exact=cp_exact)
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"], None, chunk=64)
+    assert_close(o, ro, "bf16", f"{pattern} mode {cp_exact} o")
+    assert_close(hT, rh, "bf16", f"{pattern} mode {cp_exact} hT")
+
+
+def test_fwd_gate_fallback_packed_mixed_heads():
+    """Packed sequences of mixed lengths (segment boundaries at odd token positions) with weakly and
+    strongly decaying v-heads side by side, the exact fallback (mode 2), against the oracle."""
+    x = make_inputs(1, 0, 2, 4, 128, 128, "bf16", seed=19, h0_std=0.1, lengths=[1500, 64, 1, 777, 300])
+    x = _decay_pattern(x, "mixed_heads")
+    o, hT = run_gpu(x, cp_segment_chunks=2, cp_exact=2)
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"], x["cu_seqlens"], chunk=64)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(hT, rh, "bf16", "hT")
+
+
 @pytest.mark.parametrize("exact", [False, True])
 def test_fwd_context_parallel_dense_unit_norm_violation(exact):
     """Keys far from unit norm (beta |k|^2 > 2): the per-token bound grows instead of
