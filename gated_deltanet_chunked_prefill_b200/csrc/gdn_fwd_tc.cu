@@ -273,18 +273,16 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays<kNorm>(pc, s, nv);
     };
-    if (nchunks > 0) {
-      float gv0, bv0;
-      load_gb(0, gv0, bv0);
-      chunk_start(0, gv0, bv0);
-    }
-    for (int c = 0; c < nchunks; ++c) {
+    // Iteration c runs chunk c's prep, then chunk c + 1's start; iteration -1 only the first
+    // start (each phase has one call site: the kernel's code stays small for the instruction cache)
+    for (int c = -1; c < nchunks; ++c) {
+      float gv1 = 0.f, bv1 = 0.f;
+      if (c + 1 < nchunks) load_gb(c + 1, gv1, bv1);
+      if (c >= 0) {
       const int s = c & 1;
       uint8_t* st = sm + s * kStageBytes;
       const uint32_t st_addr = sbase + s * kStageBytes;
       const uint32_t gw_col = kColGW + 128u * s;
-      float gv1 = 0.f, bv1 = 0.f;
-      if (c + 1 < nchunks) load_gb(c + 1, gv1, bv1);
       ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
@@ -352,6 +350,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_before();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);
+      }
       // the next chunk's start (its Gram product goes to the other G/W buffer)
       if (c + 1 < nchunks) chunk_start(c + 1, gv1, bv1);
     }
@@ -464,23 +463,21 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       loaded_qv = loaded_k;
     }
-    if (nchunks > 0) {
-      ok = mbar_wait(&ss->prep_full[0], 0, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      store_w(0);
-      if (et == 0 && ok) issue_a(0);
-      if (ok) prescale(0);
-      tc_fence_before();
-    }
     auto wait_mma = [&]() {
       ok = ok && mbar_wait(&ss->mma_done, mph, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       mph ^= 1;
       tc_fence_after();
     };
-    for (int c = 0; c < nchunks; ++c) {
+    // Iteration c runs chunk c's chain, then hands over to chunk c + 1 (-W, its first product, the
+    // prescale); iteration -1 only the first hand-over (one call site per phase: the kernel's code
+    // stays small for the instruction cache)
+    for (int c = -1; c < nchunks; ++c) {
       const int s = c & 1;
       const int t0 = ws + c * kChunk;
+      bool write_o = false, o_tma = false;
+      int nv = 0;
+      if (c >= 0) {
       wait_mma();
       if (et == 0 && ok && c + 2 < nchunks) {     // Q~ and -W of stage s are consumed
         load_qv(c + 2);
@@ -543,7 +540,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       // (d) S -> bf16 copy for the next chunk's products;  O = scale * D_Q -> registers
       float oo[32];
-      const int nv = ss->cs.nv[s];
+      nv = ss->cs.nv[s];
       {
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -569,10 +566,9 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
-      const bool next = c + 1 < nchunks;
       // O staging (row j = token, 256 B per row) then coalesced 16-byte stores; the
       // prescale of S for the next chunk overlaps its first product
-      const bool write_o = it.write_o && t0 >= it.s && p.o != nullptr;
+      write_o = it.write_o && t0 >= it.s && p.o != nullptr;
       if (write_o) {
         // token rows, two 64-column halves, 128B-swizzled (the layout of the TMA tile store)
         uint8_t* stg = sm + kOffDt + (r >> 6) * 8192 + (r & 7) * 2;
@@ -586,7 +582,9 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // a full chunk's O leaves through two TMA tile stores as soon as the staging is fenced
       // (inside store_w when a chunk follows); their reads are waited for before this
       // iteration's last barrier, since the next chunk's step (b) rewrites the staging
-      const bool o_tma = write_o && nv == kChunk;
+      o_tma = write_o && nv == kChunk;
+      }
+      const bool next = c + 1 < nchunks;
       auto store_o = [&]() {
         tma_store_3d(&tm_o, sbase + kOffDt, 0, it.j, it.b * p.T + t0);
         tma_store_3d(&tm_o, sbase + kOffDt + 8192u, 64, it.j, it.b * p.T + t0);
@@ -600,6 +598,10 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (et == 0 && ok) issue_a(c + 1);
       }
       if (next && ok) prescale((c + 1) & 1);
+      if (c < 0) {
+        tc_fence_before();
+        continue;
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarEpi, kNumEpi);
