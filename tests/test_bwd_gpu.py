@@ -145,12 +145,40 @@ def test_bwd_no_cross_sequence_leakage():
         assert torch.equal(g1["dh0"][n], g2["dh0"][n])
 
 
+@pytest.mark.parametrize("cp_exact", [0, 1, 2])
+def test_bwd_no_cross_sequence_leakage_with_context_parallelism(cp_exact):
+    """Packed sequences in 2-chunk segments for both sequential passes: perturbing one sequence
+    leaves every other sequence's gradients bit for bit unchanged, in every context-parallel mode."""
+    lengths = [300, 451, 129, 520, 64]
+    x = make_inputs(1, 0, 1, 2, 128, 128, "bf16", seed=37, h0_std=0.1, lengths=lengths, backward=True)
+    g1 = run_gpu_bwd(x, cp_segment_chunks=2, cp_exact=cp_exact)
+    cu = x["cu_seqlens"].tolist()
+    m = 3
+    y = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    s, e = cu[m], cu[m + 1]
+    for name in ("q", "k", "v", "dO"):
+        y[name][:, s:e] = -y[name][:, s:e]
+    y["g"][:, s:e] *= 0.01
+    y["dhT"][m] = 1.0
+    g2 = run_gpu_bwd(y, cp_segment_chunks=2, cp_exact=cp_exact)
+    for n in range(len(lengths)):
+        if n == m:
+            continue
+        a, b = cu[n], cu[n + 1]
+        for name in ("dq", "dk", "dv", "dg", "dbeta"):
+            assert torch.equal(g1[name][:, a:b], g2[name][:, a:b]), (name, n)
+        assert torch.equal(g1["dh0"][n], g2["dh0"][n])
+    assert not torch.equal(g1["dv"][:, s:e], g2["dv"][:, s:e])
+
+
 def test_bwd_full_size_sampled_units():
+    """The backward workload at full size: all six gradients of 8 (sequence, v-head) units (first
+    and last head of both sequences among them) against the oracle's token adjoint."""
     x = config_inputs("bwd_bf16")
     gr = run_gpu_bwd(x)
     for name in GRADS:
         assert torch.isfinite(gr[name].float()).all(), name
-    for n, j in [(0, 0), (1, 9)]:
+    for n, j in [(0, 0), (1, 9), (0, 15), (1, 0), (1, 15), (0, 5), (1, 3), (0, 11)]:
         ref, (b, s, e) = oracle_unit_bwd(x, n, j)
         assert_close(gr["dq"][b, s:e, j], ref["dq"][0, :, 0], "bf16", f"unit ({n},{j}) dq")
         assert_close(gr["dk"][b, s:e, j], ref["dk"][0, :, 0], "bf16", f"unit ({n},{j}) dk")

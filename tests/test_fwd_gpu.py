@@ -162,6 +162,33 @@ def test_fwd_no_cross_sequence_leakage():
     assert not torch.equal(o1[:, s:e], o2[:, s:e])
 
 
+@pytest.mark.parametrize("cp_exact", [0, 1, 2])
+def test_fwd_no_cross_sequence_leakage_with_context_parallelism(cp_exact):
+    """Packed sequences split into 2-chunk segments (every mode of obtaining a segment's start):
+    perturbing one sequence, which spans several segments, leaves every other sequence's o and hT
+    bit for bit unchanged."""
+    lengths = [300, 451, 129, 520, 64]
+    x = make_inputs(1, 0, 2, 2, 128, 128, "bf16", seed=29, h0_std=0.1, lengths=lengths)
+    o1, h1 = run_gpu(x, cp_segment_chunks=2, cp_exact=cp_exact)
+    cu = x["cu_seqlens"].tolist()
+    m = 1
+    y = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    s, e = cu[m], cu[m + 1]
+    for name in ("q", "k", "v"):
+        y[name][:, s:e] = -y[name][:, s:e]
+    y["g"][:, s:e] = y["g"][:, s:e] * 0.01          # weak decay: its windows do not close
+    y["beta"][:, s:e] = 1 - y["beta"][:, s:e]
+    y["h0"][m] = 3.0
+    o2, h2 = run_gpu(y, cp_segment_chunks=2, cp_exact=cp_exact)
+    for n in range(len(lengths)):
+        if n == m:
+            continue
+        a, b = cu[n], cu[n + 1]
+        assert torch.equal(o1[:, a:b], o2[:, a:b]), n
+        assert torch.equal(h1[n], h2[n]), n
+    assert not torch.equal(o1[:, s:e], o2[:, s:e])
+
+
 def test_fwd_empty_and_zero_length_sequences():
     x = make_inputs(1, 0, 1, 1, 128, 128, "bf16", seed=3, h0_std=0.1, lengths=[0, 70, 0])
     o, hT = run_gpu(x)
@@ -226,9 +253,10 @@ def test_fwd_cp_mode_segments_and_deterministic_flag():
 
 # ---------------------------------------------------------------- full-size configurations
 FULL = {
-    "dense_bf16": [(0, 0), (3, 15), (1, 7)],
-    "long_gqa_bf16": [(0, 0), (0, 31), (0, 18)],
-    "varlen_bf16": None,   # sampled below: the longest, the shortest, a ragged one
+    # (sequence, v-head) units: first and last head, first and last sequence, others spread out
+    "dense_bf16": [(0, 0), (3, 15), (1, 7), (2, 3), (0, 12), (3, 0), (1, 15), (2, 9)],
+    "long_gqa_bf16": [(0, 0), (0, 31), (0, 18), (0, 1), (0, 7), (0, 14), (0, 23), (0, 30)],
+    "varlen_bf16": None,   # sampled below: the longest, the shortest, ragged ones, the last
 }
 
 
@@ -240,7 +268,9 @@ def test_fwd_full_size_sampled_units(name):
     units = FULL[name]
     if units is None:
         L = np.diff(x["cu_seqlens"].numpy())
-        units = [(int(np.argmax(L)), 3), (int(np.argmin(L)), 11), (5, 0)]
+        ragged = [n for n in range(len(L)) if L[n] % 64][:3]
+        units = [(int(np.argmax(L)), 3), (int(np.argmax(L)), 15), (int(np.argmin(L)), 11), (5, 0),
+                 (len(L) - 1, 15), (0, 8)] + [(n, (5 * n) % 16) for n in ragged]
     for n, j in units:
         ro, rh, (b, s, e) = oracle_unit_fwd(x, n, j)
         assert_close(o[b, s:e, j], ro, "bf16", f"{name} unit ({n},{j}) o")
