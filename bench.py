@@ -714,6 +714,26 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     name, mode = HEADLINE
+    if args.only in ("decode", "decode_d256"):
+        cfg = DECODE if args.only == "decode" else DECODE_256
+        if args.single:                          # warm-up steps plus one step, no report
+            x = make_inputs(cfg["N"], 1, cfg["Hqk"], cfg["Hv"], cfg["dk"], cfg["dv"], "bf16", 2000, h0_std=0.1)
+            tok = {n: x[n][:, 0].contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")}
+            state = x["h0"].to(dev)
+            for _ in range(max(args.warmup, 3) + 1):
+                gdn.gdn_recurrent_step(tok["q"], tok["k"], tok["v"], tok["g"], tok["beta"], state, x["scale"])
+            torch.cuda.synchronize()
+            return
+        line = measure_decode(gdn, args, dev, rank, world, dist, stream, pool, min(args.cpu_budget, 5.0), cfg)
+        line.update({"metric": "GDN recurrent decode step tokens/s on 1 B200; % of HBM roofline",
+                     "value": line["tokens_per_s"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                     "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                     "dtype": "bf16", "data": "synthetic"})
+        if pool is not None:
+            pool.terminate()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     if args.only:
         name, mode = args.only, args.mode or ("fwd" if args.only != "bwd_bf16" else "bwd")
     if args.single:
