@@ -43,6 +43,8 @@ constexpr int kEpiWarp0 = 8;              // warps 0-7: prep (TMEM lane quadrant
                                           // thread also issues the TMA loads and the chain MMAs
 constexpr int kNumPrep = 256, kNumEpi = 256;
 constexpr int kBarPrep = 1, kBarEpi = 2;  // named barrier ids
+constexpr int kBarScalars = 3;            // prep warps 0-1: the chunk's g, beta and decay scalars
+constexpr int kGramIssuer = 224;          // lane 0 of prep warp 7 (no part in the scalar scan)
 
 // shared memory layout (bytes from a 1024-aligned base)
 constexpr uint32_t kStageBytes = 48u * 1024u;   // [K0 Q0 V0 | K1 Q1 V1], 8KB 128B-swizzled sub-tiles
@@ -63,6 +65,7 @@ struct Small {
   ChunkScalars cs;
   float wsum[16];         // warm-up window search: per-warp partial sums
   uint64_t full_k[2], full_qv[2], prep_full[2], gdone, wdone, mma_done, dd_free;
+  uint64_t dec_ready[2];  // by stage: the chunk's decay scalars written and its Gram product done
   uint64_t stall;         // testing only: a barrier that nothing completes
   uint32_t tmem_base;
   int abort_flag;
@@ -155,6 +158,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(&ss->full_k[s], 1);
       mbar_init(&ss->full_qv[s], 1);
       mbar_init(&ss->prep_full[s], 1);
+      mbar_init(&ss->dec_ready[s], 1);
     }
     mbar_init(&ss->gdone, 1);
     mbar_init(&ss->wdone, 1);
@@ -250,8 +254,9 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       ok = ok && mbar_wait(&ss->full_k[s], (c >> 1) & 1, abort_flag);
       ok = ok && mbar_wait(&ss->full_qv[s], (c >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
-      // full chunk: the Gram product can start at once (a partial one waits for its zeroed rows)
-      if (nv == kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
+      // full chunk: the Gram product can start at once, issued by warp 7 while warps 0-1 form the
+      // scalars (a partial chunk waits for its zeroed rows)
+      if (nv == kChunk && pt == kGramIssuer && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
       prep_store_gb(pc, s, gv, bv);
       if (nv < kChunk) {
         // rows past the sequence end hold the next sequence's tokens: clear them
@@ -263,15 +268,20 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           *reinterpret_cast<uint4*>(st + toff + r * 128u + ch * 16u) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
+        named_bar_sync(kBarPrep, kNumPrep);
+        if (pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
+      } else if (pt < kChunk) {
+        named_bar_sync(kBarScalars, kChunk);      // g, beta of warps 0-1 -> the scan (warp 0)
       }
-      named_bar_sync(kBarPrep, kNumPrep);
-      if (nv < kChunk && pt == 0 && ok) issue_gram(tmem + kColGW + 128u * s, st_addr, &ss->gdone, kHalf);
       if (kNorm) row_inv_norms(st, st + kHalf, st + kOffQ, st + kHalf + kOffQ, ss->cs.rk[s], ss->cs.rq[s], pt);
       prep_scan(pc, s);
       // the bulk copies of earlier P tiles have read their slots (this chunk's masks rewrite one)
       if (pt == 0) bulk_wait_read();
       named_bar_sync(kBarPrep, kNumPrep);
       prep_decays<kNorm>(pc, s, nv);
+      // warps 0-1 wrote the decay scalars; thread 0 publishes them to the chain (dec_ready) once the
+      // Gram product is also done, at the top of this chunk's prep iteration
+      if (pt < kChunk) named_bar_sync(kBarScalars, kChunk);
     };
     // Iteration c runs chunk c's prep, then chunk c + 1's start; iteration -1 only the first
     // start (each phase has one call site: the kernel's code stays small for the instruction cache)
@@ -286,19 +296,16 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
+      // the Gram product has read Q and the decays are written: the chain may scale Q (Q~)
+      if (pt == 0 && ok) mbar_arrive(&ss->dec_ready[s]);
       pc.colG = gw_col;
       prep_masks<true, kNorm>(pc, s, sbase + kOffP + s * 8192u, 1.f, ok);
       // A = (I + L)^-1 in fp32 into the A staging buffer (also the backward's copy): diagonal
-      // blocks on warps 0-3 while warps 4-7 form Q <- diag(exp(gam)) Q (times rq: the normalised
-      // rows) in place (the Gram product has consumed Q) and clear A's upper blocks; then the
-      // blocked inverse below the diagonal
+      // blocks on warps 0-3 while warps 4-7 clear A's upper blocks; then the blocked inverse below
+      // the diagonal (Q~ is formed by the chain warps, see dec_ready)
       float* af = reinterpret_cast<float*>(sm + kOffAst);
-      if (warp < 4) {
-        prep_diag_inverse_h(pc, af);
-      } else {
-        scale_rows_tile_part(st + kOffQ, kHalf, kNorm ? ss->cs.egq[s] : ss->cs.eg[s], 1.f, pt - 128, 128);
-        af_zero_upper(af, pt - 128, 128);
-      }
+      if (warp < 4) prep_diag_inverse_h(pc, af);
+      else af_zero_upper(af, pt - 128, 128);
       named_bar_sync(kBarPrep, kNumPrep);
       prep_inverse_blocked(pc, af);
       // the previous chunk's U / W products have read A2, B2 (their completion is almost
@@ -591,7 +598,15 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bulk_commit();
       };
       if (next) {
-        ok = ok && mbar_wait(&ss->prep_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag);
+        // Q~ = diag(exp(gam)) Q of the next chunk (times rq under the normalisation), in place, while
+        // the chain would otherwise wait for the prep: its Gram product has read Q and its decays are
+        // written (dec_ready); store_w's fence and barrier order it before the first product
+        const int s1 = (c + 1) & 1;
+        ok = ok && mbar_wait(&ss->dec_ready[s1], ((c + 1) >> 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) scale_rows_tile_part(sm + s1 * kStageBytes + kOffQ, kHalf, kNorm ? ss->cs.egq[s1] : ss->cs.eg[s1], 1.f,
+                                     et, kNumEpi);
+        ok = ok && mbar_wait(&ss->prep_full[s1], ((c + 1) >> 1) & 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         store_w(c + 1);
         if (et == 0 && ok && o_tma) store_o();
