@@ -69,6 +69,8 @@ struct Small {
                                          // completion is implied by the next mma_bar phase)
   uint32_t tmem_base;
   int abort_flag;
+  int next[10];           // this CTA's next item, its position (n, c, j, b, s0, e0) and its tile rows
+                          // (row, hq, srow), from warp 3
 };
 constexpr uint32_t kSmemBytes = kOffSmall + sizeof(Small);
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the 227 KB a block can opt into");
@@ -177,27 +179,42 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     hq = q.j / (p.Hv / p.Hqk);
     srow = (int)((chunk_slot(p, q.n, q.c) * p.Hv + q.j) * 128);
   };
+  // decode() for one warp, scanning forward from sequence n0 (at most the item's own sequence: a
+  // CTA's items visit nondecreasing sequences): 32 chunk offsets per round instead of a binary
+  // search of dependent loads
+  auto decode_warp = [&](int item, int n0, Pos& q) -> bool {
+    q.j = item % p.Hv;
+    const int gc = item / p.Hv;
+    if (p.chunk_off) {                        // the last n with chunk_off[n] <= gc (offsets ascend)
+      int base = n0;
+      for (;;) {
+        const int cand = base + 1 + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, cand < p.N && p.chunk_off[cand] <= gc);
+        base += __popc(m);
+        if (m != 0xffffffffu) break;
+      }
+      q.n = base;
+      q.c = gc - p.chunk_off[base];
+    } else {
+      const int nch = (p.T + kChunk - 1) / kChunk;
+      q.n = gc / nch;
+      q.c = gc % nch;
+    }
+    if (q.n >= p.N || q.c < 0) return false;
+    if (!seq_span(p, q.n, q.b, q.s0, q.e0)) return false;
+    return q.s0 + q.c * kChunk < q.e0;
+  };
   uint32_t mph = 0, tph = 0;
-  // Persistent: this CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ... (setup and
-  // TMEM allocation once per CTA).
-  for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
-  Pos pos;
-  if (!decode(item, pos)) continue;           // uniform over the CTA
-  if (tid == 0) bulk_wait_read();             // the previous item's output tiles have been read
-  if (__syncthreads_or(*abort_flag)) break;
-  const int j = pos.j, n = pos.n, c = pos.c, b = pos.b, e0 = pos.e0;
-  int row, hq, srow;
-  item_rows(pos, row, hq, srow);
-  const int t0 = pos.s0 + c * kChunk;
-  const int nv = min(kChunk, e0 - t0);
-  (void)n;
-  (void)b;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&ss->tma_bar, 128u * 1024u);
+  // Persistent: this CTA takes the valid items among blockIdx.x, blockIdx.x + gridDim.x, ... (setup
+  // and TMEM allocation once per CTA). From the second item on, warp 3 has found the item and formed
+  // its gate scalars (in slot 1 of ChunkScalars, moved to slot 0 here) during the previous item.
+  auto load_kq = [&](int hq, int row) {
     tma_load_3d(sm + kOffKQ + 0, &tm_k, &ss->tma_bar, 0, hq, row);
     tma_load_3d(sm + kOffKQ + 8192, &tm_q, &ss->tma_bar, 0, hq, row);
     tma_load_3d(sm + kOffKQ + 16384, &tm_k, &ss->tma_bar, 64, hq, row);
     tma_load_3d(sm + kOffKQ + 24576, &tm_q, &ss->tma_bar, 64, hq, row);
+  };
+  auto load_rest = [&](int j, int row, int srow) {
     tma_load_3d(sm + kOffVDO + 0, &tm_v, &ss->tma_bar, 0, j, row);
     tma_load_3d(sm + kOffVDO + 8192, &tm_do, &ss->tma_bar, 0, j, row);
     tma_load_3d(sm + kOffVDO + 16384, &tm_v, &ss->tma_bar, 64, j, row);
@@ -206,17 +223,14 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_load_3d(sm + kOffS + 16384, &tm_s, &ss->tma_bar, 64, 0, srow);
     tma_load_3d(sm + kOffDS, &tm_ds, &ss->tma_bar, 0, 0, srow);
     tma_load_3d(sm + kOffDS + 16384, &tm_ds, &ss->tma_bar, 64, 0, srow);
-  }
-  PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColG, tid, warp, lane, kBar};
-  // A = (I + L)^-1 of this chunk, as the forward pass computed it: fp32 rows into the scratch
-  {
+  };
+  auto load_ap = [&](int srow) {
     const float* ag = out.chunk_a + (size_t)srow / 128 * (kChunk * kChunk);
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int idx = tid + kThreads * m, ar = idx >> 4, c16 = idx & 15;
       cp_async_16(sbase + kOffLf + (uint32_t)(ar * kLd + c16 * 4) * 4u, ag + ar * kChunk + a_chunk(ar, c16) * 4);
     }
-    // and P (the swizzled bf16 tile, byte for byte)
     const uint8_t* pg = out.chunk_p + (size_t)srow / 128 * 8192;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
@@ -224,19 +238,66 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       cp_async_16(sbase + kOffP + idx * 16u, pg + idx * 16);
     }
     cp_async_commit();
+  };
+  bool prefetched = false;
+  int item = blockIdx.x;
+  Pos pos;
+  while (item < num_items && !decode(item, pos)) item += gridDim.x;   // uniform over the CTA
+  bool scal_ready = false;
+  while (item < num_items) {
+  if (scal_ready && tid < kChunk) {
+    ChunkScalars& cs = ss->cs;
+    cs.gam[0][tid] = cs.gam[1][tid];
+    cs.egt[0][tid] = cs.egt[1][tid];
+    cs.eg[0][tid] = cs.eg[1][tid];
+    cs.egd[0][tid] = cs.egd[1][tid];
+    cs.bet[0][tid] = cs.bet[1][tid];
+    if (tid == 0) {
+      cs.egn[0] = cs.egn[1];
+      cs.nv[0] = cs.nv[1];
+    }
   }
-  float gv = 0.f, bv = 0.f;
-  if (tid < nv) {
-    const size_t gi = (size_t)row * p.Hv + j + (size_t)tid * p.Hv;
-    gv = p.g[gi];
-    bv = __bfloat162float(beta[gi]);
+  if (tid == 0) bulk_wait_read();             // the previous item's output tiles have been read
+  if (__syncthreads_or(*abort_flag)) break;
+  const int j = pos.j, n = pos.n, c = pos.c, b = pos.b, e0 = pos.e0;
+  int row, hq, srow;
+  if (scal_ready) {
+    row = ss->next[7];
+    hq = ss->next[8];
+    srow = ss->next[9];
+  } else {
+    item_rows(pos, row, hq, srow);
   }
-  prep_store_gb(pc, 0, gv, bv);
-  // gam and the decay factors need only g: they run while the tiles are in flight
-  __syncthreads();
-  prep_scan(pc, 0);
-  __syncthreads();
-  prep_decays(pc, 0, nv);
+  const int t0 = pos.s0 + c * kChunk;
+  const int nv = min(kChunk, e0 - t0);
+  (void)n;
+  (void)b;
+  if (!prefetched) {
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&ss->tma_bar, 128u * 1024u);
+      load_kq(hq, row);
+      load_rest(j, row, srow);
+    }
+    load_ap(srow);
+  } else if (kNorm && tid == 0) {
+    load_kq(hq, row);
+  }
+  prefetched = false;
+  PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColG, tid, warp, lane, kBar};
+  if (!scal_ready) {
+    float gv = 0.f, bv = 0.f;
+    if (tid < nv) {
+      const size_t gi = (size_t)row * p.Hv + j + (size_t)tid * p.Hv;
+      gv = p.g[gi];
+      bv = __bfloat162float(beta[gi]);
+    }
+    prep_store_gb(pc, 0, gv, bv);
+    // gam and the decay factors need only g: they run while the tiles are in flight
+    __syncthreads();
+    prep_scan(pc, 0);
+    __syncthreads();
+    prep_decays(pc, 0, nv);
+  }
   cp_async_wait_all();                        // A and P from the forward pass
   bool ok = mbar_wait(&ss->tma_bar, tph, abort_flag);
   tph ^= 1;
@@ -638,6 +699,65 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                1);
     }
   }
+  if (warp == 3) {
+    // warp 3 has no rows in the dL phase: it finds this CTA's next item and forms its gate scalars in
+    // slot 1 (the same arithmetic as prep_store_gb, prep_scan and prep_decays, two tokens per lane),
+    // so that the next item starts with its loads
+    int nx = item + gridDim.x;
+    Pos np;
+    while (nx < num_items && !decode_warp(nx, n, np)) nx += gridDim.x;
+    int nrow = 0, nhq = 0, nsrow = 0;
+    if (nx < num_items) {
+      item_rows(np, nrow, nhq, nsrow);
+      const int nnv = min(kChunk, np.e0 - (np.s0 + np.c * kChunk));
+      const int so = 1, i0 = 2 * lane, i1 = 2 * lane + 1;
+      float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+      const size_t gi = (size_t)nrow * p.Hv + np.j + (size_t)i0 * p.Hv;
+      if (i0 < nnv) {
+        a0 = p.g[gi];
+        b0 = __bfloat162float(beta[gi]);
+      }
+      if (i1 < nnv) {
+        a1 = p.g[gi + p.Hv];
+        b1 = __bfloat162float(beta[gi + p.Hv]);
+      }
+      ss->cs.bet[so][i0] = b0;
+      ss->cs.bet[so][i1] = b1;
+      ss->cs.egt[so][i0] = fast_exp(a0);
+      ss->cs.egt[so][i1] = fast_exp(a1);
+      const float pair = a0 + a1;
+      float run = pair;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, run, off);
+        if (lane >= off) run += y;
+      }
+      const float gam0 = run - pair + a0, gam1 = run;
+      const float gn = __shfl_sync(0xffffffffu, run, 31);
+      ss->cs.gam[so][i0] = gam0;
+      ss->cs.gam[so][i1] = gam1;
+      ss->cs.eg[so][i0] = fast_exp(gam0);
+      ss->cs.eg[so][i1] = fast_exp(gam1);
+      ss->cs.egd[so][i0] = fast_exp(gn - gam0);
+      ss->cs.egd[so][i1] = fast_exp(gn - gam1);
+      if (lane == 0) {
+        ss->cs.egn[so] = fast_exp(gn);
+        ss->cs.nv[so] = nnv;
+      }
+    }
+    if (lane == 0) {
+      ss->next[0] = min(nx, num_items);
+      ss->next[1] = np.n;
+      ss->next[2] = np.c;
+      ss->next[3] = np.j;
+      ss->next[4] = np.b;
+      ss->next[5] = np.s0;
+      ss->next[6] = np.e0;
+      ss->next[7] = nrow;
+      ss->next[8] = nhq;
+      ss->next[9] = nsrow;
+    }
+  }
   if (r < 64) {
     ok = ok && mbar_wait(&ss->mma_bar, mph, abort_flag);
     tc_fence_after();
@@ -733,6 +853,19 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       umma_f16(tmem + kColK, kdesc(sbase + kOffA + ks * 32), mdesc(sbase + kOffKQ + ks * 2048, 16384), idkm, 1);
   }
   commit_wait(kLateIssuer);
+  {
+    const int pnx = ss->next[0];
+    prefetched = ok && pnx < num_items;
+    if (prefetched) {
+      const int nrow = ss->next[7], nhq = ss->next[8], nsrow = ss->next[9];
+      if (tid == kLateIssuer) {
+        mbar_arrive_expect_tx(&ss->tma_bar, 128u * 1024u);
+        if (!kNorm) load_kq(nhq, nrow);
+        load_rest(ss->next[3], nrow, nsrow);
+      }
+      load_ap(nsrow);
+    }
+  }
   // ---- outputs: dq, dk (rows i < nv), dbeta, dg. A full chunk's bf16 dq, dk leave through TMA
   //      tile stores from staging (every operand tile is free now), otherwise per thread.
   const bool qk_tma = !out.qk_partial && nv == kChunk;
@@ -882,12 +1015,15 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
+  item = ss->next[0];
+  pos = Pos{ss->next[1], ss->next[2], ss->next[3], ss->next[4], ss->next[5], ss->next[6]};
+  scal_ready = true;
   }
   if (tid == 0) bulk_wait_all();
+  cp_async_wait_all();
   if (tid == 0 && *abort_flag) {
-    // aborted: do not leave the CTA with copies in flight (bounded wait, flag ignored)
     volatile int never = 0;
-    mbar_wait(&ss->tma_bar, tph ^ 1, &never);
+    mbar_wait(&ss->tma_bar, prefetched ? tph : (tph ^ 1), &never);
     report_error(p, kDevTimeout);
   }
   tc_fence_before();

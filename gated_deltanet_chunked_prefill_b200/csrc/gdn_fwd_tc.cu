@@ -290,7 +290,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (c + 1 < nchunks) load_gb(c + 1, gv1, bv1);
       if (c >= 0) {
       const int s = c & 1;
-      uint8_t* st = sm + s * kStageBytes;
       const uint32_t st_addr = sbase + s * kStageBytes;
       const uint32_t gw_col = kColGW + 128u * s;
       ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
