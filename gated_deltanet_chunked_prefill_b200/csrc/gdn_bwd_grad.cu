@@ -51,7 +51,7 @@ constexpr uint32_t kOffA2 = 160u * 1024;  // A diag(beta)
 constexpr uint32_t kOffP = 168u * 1024;   // P (from the forward pass); then dPm
 constexpr uint32_t kOffA = 176u * 1024;   // A; then dG + dG^T
 constexpr uint32_t kOffDA = 184u * 1024;  // dA; then X = dA A^T
-constexpr uint32_t kOffLf = 192u * 1024;  // fp32 64 x kLd: L -> A; then dG
+constexpr uint32_t kOffLf = 192u * 1024;  // A (fp32, the forward's swizzled 64 x 64 layout); then dG (64 x kLd)
 constexpr uint32_t kOffSmall = kOffLf + 64u * kLd * 4u;
 
 // Per-token partial sums, one slot per producer so that every slot entry is written exactly
@@ -224,21 +224,12 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_load_3d(sm + kOffDS, &tm_ds, &ss->tma_bar, 0, 0, srow);
     tma_load_3d(sm + kOffDS + 16384, &tm_ds, &ss->tma_bar, 64, 0, srow);
   };
+  // the forward's A (fp32, its swizzled 64 x 64 layout, kept as is) and P (the swizzled bf16 tile)
   auto load_ap = [&](int srow) {
-    const float* ag = out.chunk_a + (size_t)srow / 128 * (kChunk * kChunk);
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int idx = tid + kThreads * m, ar = idx >> 4, c16 = idx & 15;
-      cp_async_16(sbase + kOffLf + (uint32_t)(ar * kLd + c16 * 4) * 4u, ag + ar * kChunk + a_chunk(ar, c16) * 4);
-    }
-    const uint8_t* pg = out.chunk_p + (size_t)srow / 128 * 8192;
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const int idx = tid + kThreads * m;
-      cp_async_16(sbase + kOffP + idx * 16u, pg + idx * 16);
-    }
-    cp_async_commit();
+    bulk_load(sbase + kOffLf, out.chunk_a + (size_t)srow / 128 * (kChunk * kChunk), kChunk * kChunk * 4u, &ss->tma_bar);
+    bulk_load(sbase + kOffP, out.chunk_p + (size_t)srow / 128 * 8192, 8192u, &ss->tma_bar);
   };
+  constexpr uint32_t kItemBytes = 128u * 1024u + kChunk * kChunk * 4u + 8192u;   // tiles, A, P
   bool prefetched = false;
   int item = blockIdx.x;
   Pos pos;
@@ -274,11 +265,11 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   (void)b;
   if (!prefetched) {
     if (tid == 0) {
-      mbar_arrive_expect_tx(&ss->tma_bar, 128u * 1024u);
+      mbar_arrive_expect_tx(&ss->tma_bar, kItemBytes);
       load_kq(hq, row);
       load_rest(j, row, srow);
+      load_ap(srow);
     }
-    load_ap(srow);
   } else if (kNorm && tid == 0) {
     load_kq(hq, row);
   }
@@ -298,7 +289,6 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     prep_decays(pc, 0, nv);
   }
-  cp_async_wait_all();                        // A and P from the forward pass
   bool ok = mbar_wait(&ss->tma_bar, tph, abort_flag);
   tph ^= 1;
   if (nv < kChunk) {                          // rows past the sequence end: zero
@@ -308,7 +298,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       *reinterpret_cast<uint4*>(sm + tile * 8192u + rr * 128u + ch * 16u) = make_uint4(0, 0, 0, 0);
     }
   }
-  fence_proxy_async_smem();                   // zeroed rows and P (cp.async) are operands below
+  fence_proxy_async_smem();                   // zeroed rows are operands below
   ok = __syncthreads_and(ok);
   auto commit_wait = [&](int issuer = 0) {
     if (tid == issuer && ok) umma_commit(&ss->mma_bar);
@@ -339,7 +329,27 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                idmm, ks > 0);
   }
   // A (fp32 rows, from the forward pass) -> A diag(beta) and A in bf16
-  prep_write_a_rows(pc, 0, sbase + kOffA2, sbase + kOffA);
+  // A (fp32) -> A diag(beta) and A in bf16 (128B-swizzled K-major rows); thread: row i, 16 columns
+  {
+    const int i = tid & 63, qq = tid >> 6;
+    const float* af = reinterpret_cast<const float*>(sm + kOffLf);
+    const float* bet = ss->cs.bet[0];
+    float a[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 t = *reinterpret_cast<const float4*>(af + i * kChunk + a_chunk(i, qq * 4 + u) * 4);
+      a[4 * u] = t.x; a[4 * u + 1] = t.y; a[4 * u + 2] = t.z; a[4 * u + 3] = t.w;
+    }
+    uint32_t w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) w[u] = pack_bf16(a[2 * u] * bet[qq * 16 + 2 * u], a[2 * u + 1] * bet[qq * 16 + 2 * u + 1]);
+    st_shared_v4(sbase + kOffA2 + sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+    st_shared_v4(sbase + kOffA2 + sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) w[u] = pack_bf16(a[2 * u], a[2 * u + 1]);
+    st_shared_v4(sbase + kOffA + sw128(i, 2 * qq), w[0], w[1], w[2], w[3]);
+    st_shared_v4(sbase + kOffA + sw128(i, 2 * qq + 1), w[4], w[5], w[6], w[7]);
+  }
   if (kNorm) {
     // inverse row norms of K and Q, folded into the decay factors (egd, egk carry rk; egq rq)
     row_inv_norms(sm + kOffKQ, sm + kOffKQ + 16384, sm + kOffKQ + 8192, sm + kOffKQ + 24576, ss->cs.rk[0],
@@ -583,10 +593,9 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const float* bet = ss->cs.bet[0];
       uint32_t w[16];
       {
-        const float4* src = reinterpret_cast<const float4*>(Lf + i * kLd + j0);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const float4 t = src[u];
+          const float4 t = *reinterpret_cast<const float4*>(Lf + i * kChunk + a_chunk(i, (j0 >> 2) + u) * 4);
           colv[4 * u] = mvals[4 * u] * t.x;
           colv[4 * u + 1] = mvals[4 * u + 1] * t.y;
           colv[4 * u + 2] = mvals[4 * u + 2] * t.z;
@@ -859,11 +868,11 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (prefetched) {
       const int nrow = ss->next[7], nhq = ss->next[8], nsrow = ss->next[9];
       if (tid == kLateIssuer) {
-        mbar_arrive_expect_tx(&ss->tma_bar, 128u * 1024u);
+        mbar_arrive_expect_tx(&ss->tma_bar, kItemBytes);
         if (!kNorm) load_kq(nhq, nrow);
         load_rest(ss->next[3], nrow, nsrow);
+        load_ap(nsrow);
       }
-      load_ap(nsrow);
     }
   }
   // ---- outputs: dq, dk (rows i < nv), dbeta, dg. A full chunk's bf16 dq, dk leave through TMA
@@ -1020,7 +1029,6 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   scal_ready = true;
   }
   if (tid == 0) bulk_wait_all();
-  cp_async_wait_all();
   if (tid == 0 && *abort_flag) {
     volatile int never = 0;
     mbar_wait(&ss->tma_bar, prefetched ? tph : (tph ^ 1), &never);
