@@ -9,10 +9,11 @@
 //
 //   prep warps (state independent, overlap the previous chunk's chain):
 //     G  = [K;Q] K^T                               tcgen05, M=128 N=64 K=128
-//     L  = strict_lower(diag(beta) KK^T * E) (fp16),  A = (I + L)^-1: 16 x 16 diagonal blocks
-//          by substitution (CUDA cores), one column strip per warp on m16n8k16 f16 products
-//     A2 = A diag(beta), B2 = A diag(beta exp(gam)) -> bf16;  P = lower_incl(QK^T * E) -> bf16
-//     Q <- diag(exp(gam)) Q  (Q~)
+//     L  = strict_lower(diag(beta) KK^T * E) (fp16),  A = (I + L)^-1 (fp32): 16 x 16 diagonal
+//          blocks by substitution (CUDA cores), the blocks below by 2 x 2 blocking on m16n8k16 f16
+//          products;  P = lower_incl(QK^T * E) -> bf16
+//   epilogue warps, handing over to the chunk (in what would otherwise be a wait for the prep):
+//     Q <- diag(exp(gam)) Q  (Q~);  A2 = A diag(beta), B2 = A diag(beta exp(gam)) -> bf16
 //     U^T = V^T A2^T   into the chunk's Delta accumulator          tcgen05, M=128 N=64 K=64
 //     W   = B2 K       -> -W in bf16 over the V tile (token rows)   tcgen05, M=64 N=128 K=64
 //   epilogue warps (the sequential chain, two tensor-core round trips per chunk):
@@ -64,8 +65,10 @@ constexpr uint32_t kOffSmall = kOffAst + 16384u;
 struct Small {
   ChunkScalars cs;
   float wsum[16];         // warm-up window search: per-warp partial sums
-  uint64_t full_k[2], full_qv[2], prep_full[2], gdone, wdone, mma_done, dd_free;
+  uint64_t full_k[2], full_qv[2], prep_full[2], gdone, wdone, mma_done;
+  uint64_t dd_free[2];    // by stage: the chain has read the chunk's W and its scalars (step (c))
   uint64_t dec_ready[2];  // by stage: the chunk's decay scalars written and its Gram product done
+  uint64_t a_free;        // the chain has read the chunk's fp32 A (the prep may write the next one)
   uint64_t stall;         // testing only: a barrier that nothing completes
   uint32_t tmem_base;
   int abort_flag;
@@ -162,7 +165,9 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     mbar_init(&ss->gdone, 1);
     mbar_init(&ss->wdone, 1);
-    mbar_init(&ss->dd_free, 1);
+    mbar_init(&ss->dd_free[0], 1);
+    mbar_init(&ss->dd_free[1], 1);
+    mbar_init(&ss->a_free, 1);
     mbar_init(&ss->mma_done, 1);
     mbar_init(&ss->stall, 1);
     ss->abort_flag = 0;
@@ -232,7 +237,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int pt = threadIdx.x;            // 0..255
     PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColGW, pt, warp, lane, kBarPrep};
     bool ok = true;
-    const int qd = warp & 3, hc = warp >> 2;
     // g, beta of a chunk (0 past the sequence end), loaded one chunk ahead
     auto load_gb = [&](int c, float& gv, float& bv) {
       const int t0 = ws + c * kChunk;
@@ -249,6 +253,12 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto chunk_start = [&](int c, float gv, float bv) {
       const int s = c & 1;
       const int nv = min(kChunk, it.e - (ws + c * kChunk));
+      // chunk c - 2 (same slot) is done with: the chain has read its W and its scalars (each stage's
+      // barrier completes once per two chunks; chunk c's own phase cannot complete before its prep)
+      if (c >= 2) {
+        ok = ok && mbar_wait(&ss->dd_free[s], ((c - 2) >> 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+      }
       uint8_t* st = sm + s * kStageBytes;
       const uint32_t st_addr = sbase + s * kStageBytes;
       ok = ok && mbar_wait(&ss->full_k[s], (c >> 1) & 1, abort_flag);
@@ -290,7 +300,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (c + 1 < nchunks) load_gb(c + 1, gv1, bv1);
       if (c >= 0) {
       const int s = c & 1;
-      const uint32_t st_addr = sbase + s * kStageBytes;
       const uint32_t gw_col = kColGW + 128u * s;
       ok = ok && mbar_wait(&ss->gdone, c & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
@@ -303,18 +312,15 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // blocks on warps 0-3 while warps 4-7 clear A's upper blocks; then the blocked inverse below
       // the diagonal (Q~ is formed by the chain warps, see dec_ready)
       float* af = reinterpret_cast<float*>(sm + kOffAst);
+      if (c > 0) {                                     // the chain has read chunk c - 1's A
+        ok = ok && mbar_wait(&ss->a_free, (c - 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+      }
       if (warp < 4) prep_diag_inverse_h(pc, af);
       else af_zero_upper(af, pt - 128, 128);
       named_bar_sync(kBarPrep, kNumPrep);
       prep_inverse_blocked(pc, af);
-      // the previous chunk's U / W products have read A2, B2 (their completion is almost
-      // always past by now)
-      if (c > 0) {
-        ok = ok && mbar_wait(&ss->wdone, (c - 1) & 1, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-      }
-      named_bar_sync(kBarPrep, kNumPrep);              // A complete in fp32
-      prep_store_a_f32<kNorm>(pc, s, af, sbase + kOffA2, sbase + kOffB2);
+      // A complete in fp32 (the chain forms A2, B2 from it and issues the U^T, W products)
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && p.states != nullptr && p.chunk_p != nullptr && ws + c * kChunk >= it.s && ok) {
@@ -325,36 +331,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (p.chunk_a != nullptr) bulk_store(p.chunk_a + slot * (kChunk * kChunk), sbase + kOffAst, 16384u);
         bulk_commit();
       }
-      // the Delta accumulator is free once the chain has read chunk c - 1's
-      if (c > 0) {
-        ok = ok && mbar_wait(&ss->dd_free, (c - 1) & 1, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-      }
-      // U^T = V^T A2^T (A = the V tile read MN-major) into the Delta accumulator;
-      // W = B2 K (B = the K tile read MN-major, M = 64) over this chunk's G
-      if (pt == 0 && ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          if (!it.zero_v)
-            umma_f16(tmem + kColDd, sdesc_sw128(st_addr + kOffV + ks * 2048, kHalf, 1024),
-                     sdesc_sw128(sbase + kOffA2 + ks * 32, 16, 1024), kIdU, ks > 0);
-          umma_f16(tmem + gw_col, sdesc_sw128(sbase + kOffB2 + ks * 32, 16, 1024),
-                   sdesc_sw128(st_addr + ks * 2048, kHalf, 1024), kIdW, ks > 0);
-        }
-        umma_commit(&ss->wdone);
-      }
-      if (it.zero_v && ok) {                    // V = 0: the Delta accumulator starts from zero
-        tc_fence_after();
-        float z[32];
-#pragma unroll
-        for (int u = 0; u < 32; ++u) z[u] = 0.f;
-        tmem_st32_sync(tmem + ((uint32_t)(32 * qd) << 16) + kColDd + 32 * hc, z);
-      }
-      // the chain waits for these products and moves -W into the stage itself
-      fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(kBarPrep, kNumPrep);
       if (pt == 0 && ok) mbar_arrive(&ss->prep_full[s]);
       }
       // the next chunk's start (its Gram product goes to the other G/W buffer)
@@ -368,7 +345,9 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int qd = ew & 3, hh = ew >> 2;
     const int r = 32 * qd + lane;                 // dv row of S (= TMEM lane)
     const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-    const uint32_t s_addr = tmem + lane_base + kColS + hh * 64;   // this thread's 64 columns of S
+    const uint32_t s_addr = tmem + lane_base + kColS + hh * 64;
+    // for the A2 / B2 formation, which takes the group's thread index
+    const PrepCtx ec{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColGW, et, ew, lane, kBarEpi};   // this thread's 64 columns of S
     // initial state -> TMEM (fp32) and Sb (bf16)
     auto write_sb = [&](const float* v, int half32) {
       const uint32_t base = sbase + kOffSb + hh * 16384u;
@@ -484,6 +463,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       bool write_o = false, o_tma = false;
       int nv = 0;
       if (c >= 0) {
+      nv = ss->cs.nv[s];                            // read before step (c) releases the chunk's scalars
       wait_mma();
       if (et == 0 && ok && c + 2 < nchunks) {     // Q~ and -W of stage s are consumed
         load_qv(c + 2);
@@ -525,7 +505,7 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       named_bar_sync(kBarEpi, kNumEpi);
       // (c) D_Q += Delta^T P^T;  S += Delta~^T K   (S was pre-scaled by exp(gam_n))
       if (et == 0 && ok) {
-        mbar_arrive(&ss->dd_free);                // every Delta^T read is done: the prep may refill it
+        mbar_arrive(&ss->dd_free[s]);             // chunk c's scalars and W are read: the prep may reuse the slot
         tc_fence_after();
         const uint32_t ya = sbase + kOffYt, pb = sbase + kOffP + s * 8192u;
 #pragma unroll
@@ -546,7 +526,6 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       // (d) S -> bf16 copy for the next chunk's products;  O = scale * D_Q -> registers
       float oo[32];
-      nv = ss->cs.nv[s];
       {
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -607,6 +586,34 @@ gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                      et, kNumEpi);
         ok = ok && mbar_wait(&ss->prep_full[s1], ((c + 1) >> 1) & 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
+        // A2 = A diag(beta), B2 = A diag(beta exp(gam)) in bf16 from the prep's fp32 A, then
+        // U^T = V^T A2^T into the Delta accumulator (chunk c's Delta was read in step (b)) and
+        // W = B2 K into the chunk's G/W buffer (the previous U, W products completed before
+        // store_w(c), so A2 and B2 are free)
+        prep_store_a_f32<kNorm>(ec, s1, reinterpret_cast<const float*>(sm + kOffAst), sbase + kOffA2, sbase + kOffB2);
+        fence_proxy_async_smem();
+        named_bar_sync(kBarEpi, kNumEpi);
+        if (et == 0 && ok) {
+          mbar_arrive(&ss->a_free);
+          tc_fence_after();
+          const uint32_t st1 = sbase + s1 * kStageBytes;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            if (!it.zero_v)
+              umma_f16(tmem + kColDd, sdesc_sw128(st1 + kOffV + ks * 2048, kHalf, 1024),
+                       sdesc_sw128(sbase + kOffA2 + ks * 32, 16, 1024), kIdU, ks > 0);
+            umma_f16(tmem + kColGW + 128u * s1, sdesc_sw128(sbase + kOffB2 + ks * 32, 16, 1024),
+                     sdesc_sw128(st1 + ks * 2048, kHalf, 1024), kIdW, ks > 0);
+          }
+          umma_commit(&ss->wdone);
+        }
+        if (it.zero_v && ok) {                    // V = 0: the Delta accumulator starts from zero
+          tc_fence_after();
+          float z[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) z[u] = 0.f;
+          tmem_st32_sync(tmem + lane_base + kColDd + 32 * hh, z);
+        }
         store_w(c + 1);
         if (et == 0 && ok && o_tma) store_o();
         if (et == 0 && ok) issue_a(c + 1);
