@@ -494,59 +494,50 @@ class Case:
         return out
 
     def e2e(self, steps, stream, dist):
-        """The step through the public API from pinned host inputs, every output copied back to
-        pinned host memory, all inside the timed region. The backward-alone workload recomputes its
-        forward pass (the host holds no chunk-state cache)."""
-        mode = self.mode
-        need = ["q", "k", "v", "g", "beta", "h0", "cu_seqlens"] + (["dO", "dhT"] if mode != "fwd" else [])
-        host = {k: self.x[k].pin_memory() for k in need if self.x.get(k) is not None}
-        dev_in = {k: torch.empty_like(self.d[k]) for k in host}
-        dev_in["scale"] = self.d["scale"]
-        for k in ("h0", "dO", "dhT", "cu_seqlens"):
-            dev_in.setdefault(k, None)
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        out_host = {}
+        """The step through the public host-buffer entry point (gdn_chunk_host of the C ABI): inputs
+        from pinned host memory, every output back to pinned host memory, all inside the timed
+        region. Two scratch buffers and two output sets are used in turn on three streams (kernels,
+        copies in, copies out), so that one step's outputs go back while the next step's inputs
+        come in. The backward-alone workload recomputes its forward pass (the host holds no
+        chunk-state cache)."""
+        mode, w, x = self.mode, self.w, self.x
+        keys = ["q", "k", "v", "g", "beta", "h0", "cu_seqlens"] + (["dO", "dhT"] if mode != "fwd" else [])
+        host = {k: (x[k].contiguous().pin_memory() if isinstance(x.get(k), torch.Tensor) else None) for k in keys}
+        h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+        need = self.gdn.host_scratch_size(mode, host["q"].dtype, w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs,
+                                          self.cp)
+        scratch = [torch.empty(need, dtype=torch.uint8, device=self.dev) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
+        outs = [None, None]
 
-        def back(name, t):
-            if name not in out_host:
-                out_host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-            out_host[name].copy_(t, non_blocking=True)
-            return t.numel() * t.element_size()
+        def one(i):
+            outs[i % 2] = self.gdn.gdn_chunk_host(
+                host["q"], host["k"], host["v"], host["g"], host["beta"], x["scale"], host["h0"],
+                host["cu_seqlens"], dO=host.get("dO"), dhT=host.get("dhT"), mode=mode, scratch=scratch[i % 2],
+                outputs=outs[i % 2], stream=stream, h2d_stream=s_in, d2h_stream=s_out,
+                cp_segment_chunks=self.cp, synchronize=False)
 
-        def one():
-            for k, t in host.items():
-                dev_in[k].copy_(t, non_blocking=True)
-            nbytes = 0
-            if mode in ("fwd", "fwdbwd"):
-                self.fwd(dev_in)
-                nbytes += back("o", self.o) + back("hT", self.hT)
-            if mode != "fwd":
-                gr = self.bwd(dev_in, states=mode == "fwdbwd", ws=None if mode == "fwdbwd" else self._ws_recompute())
-                for k2, t2 in gr.items():
-                    if t2 is not None:
-                        nbytes += back(k2, t2)
-            return nbytes
-
-        for _ in range(2):
-            d2h = one()
+        for i in range(2):                       # also allocates the two output sets
+            one(i)
         torch.cuda.synchronize()
+        d2h = sum(t.numel() * t.element_size() for t in outs[0].values())
         if dist:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(steps):
-            one()
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(steps):
+            one(i)
+        for s_ in (s_in, s_out):                 # the timed region ends when all three streams have
+            ev = torch.cuda.Event()
+            ev.record(s_)
+            stream.wait_event(ev)
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, self.dev) / steps
         return e_ms, int(h2d), int(d2h)
 
-    def _ws_recompute(self):
-        if getattr(self, "_wsr", None) is None:
-            w = self.w
-            self._wsr = torch.zeros(self.gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs,
-                                                                self.cp), dtype=torch.uint8, device=self.dev)
-        return self._wsr
 
 
 def dominant_roofline(case, per_kernel, launches_one, step_label):

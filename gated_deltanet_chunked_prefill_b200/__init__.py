@@ -15,11 +15,13 @@ import torch
 
 __all__ = ["lib", "GdnError", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd", "fwd_workspace_size",
            "bwd_workspace_size", "chunk_states", "read_device_status", "check_device_error", "Options",
-           "LIB_PATH", "KernelTrace", "launch_count", "gdn_recurrent_step", "chunk_gated_delta_rule"]
+           "LIB_PATH", "KernelTrace", "launch_count", "gdn_recurrent_step", "chunk_gated_delta_rule",
+           "gdn_chunk_host", "host_scratch_size", "HOST_MODES"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
 GDN_F32, GDN_BF16 = 0, 1
+HOST_MODES = {"fwd": 1, "bwd": 2, "fwdbwd": 3}     # gdn_host_mode
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace",
           4: "CUDA runtime error", 5: "device timeout", 6: "inconsistent device input",
           7: "unusable kernel launch"}
@@ -77,6 +79,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_fwd_noalloc.argtypes = [i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp,
                                                             vp, vp]
         L.gdn_chunk_fwd_noalloc.restype = i
+        L.gdn_chunk_host_scratch_size.argtypes = [i, i] + dims + [vp]
+        L.gdn_chunk_host_scratch_size.restype = sz
+        L.gdn_chunk_host.argtypes = ([i, i] + [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, i, vp, vp, vp, vp,
+                                     vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp])
+        L.gdn_chunk_host.restype = i
         L.gdn_recurrent_step.argtypes = [i] * 6 + [vp, vp, vp, vp, vp, f, vp, vp, vp]
         L.gdn_recurrent_step.restype = i
         L.gdn_read_device_status.argtypes = [vp, vp]
@@ -331,6 +338,101 @@ def gdn_chunk_bwd(q, k, v, g, beta, dO, scale=None, h0=None, dhT=None, cu_seqlen
     if _check_default() if check_status is None else check_status:
         _status_after(ws, stream, "gdn_chunk_bwd")
     return dict(dq=dq, dk=dkk, dv=dvv, dg=dg, dbeta=db, dh0=dh0)
+
+
+def host_scratch_size(mode, dtype, B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks=0, cp_exact=False, cp_mode=0,
+                      qk_l2norm=False) -> int:
+    """Bytes of device scratch gdn_chunk_host needs (mode "fwd", "bwd" or "fwdbwd")."""
+    o = _opts(cp_segment_chunks, cp_exact, cp_mode=cp_mode, qk_l2norm=qk_l2norm)
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return int(lib().gdn_chunk_host_scratch_size(HOST_MODES[mode], code, B, T, Hqk, Hv, dk, dv, N, ctypes.byref(o)))
+
+
+def _check_host(t, name, dtype=None):
+    if t is None:
+        return
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a CPU tensor (host-buffer call)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def gdn_chunk_host(q, k, v, g, beta, scale=None, h0=None, cu_seqlens=None, dO=None, dhT=None, mode=None,
+                   scratch=None, outputs=None, output_final_state=True, want_dh0=True, stream=None,
+                   h2d_stream=None, d2h_stream=None, device=None, cp_segment_chunks=0, cp_exact=False, cp_mode=0,
+                   qk_l2norm=False, synchronize=True):
+    """Host-buffer call through the C ABI (gdn_chunk_host): CPU tensors in, CPU tensors out; the copies
+    and the kernels run on the current (or given) CUDA device. mode "fwd" (default without dO),
+    "bwd" (forward pass recomputed) or "fwdbwd" (default with dO). Page-locked inputs and outputs
+    (Tensor.pin_memory()) let the copies overlap; `outputs` (a dict from an earlier call) reuses
+    output buffers, `scratch` a device buffer of host_scratch_size() bytes. With synchronize=False
+    the call returns once everything is enqueued: the outputs are valid after d2h_stream (or stream)
+    synchronises. Returns a dict of the outputs (o, hT; dq, dk, dv, dg, dbeta, dh0)."""
+    mode = mode or ("fwd" if dO is None else "fwdbwd")
+    if mode not in HOST_MODES:
+        raise ValueError(f"mode must be one of {sorted(HOST_MODES)}")
+    fw, bw = mode in ("fwd", "fwdbwd"), mode in ("bwd", "fwdbwd")
+    if bw and dO is None:
+        raise ValueError(f"mode {mode!r} needs dO")
+    _check_shapes(q, k, v, g, beta, h0, cu_seqlens, dO=dO if bw else None, dhT=dhT if bw else None)
+    io = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check_host(t, n, io)
+    _check_host(g, "g", torch.float32)
+    _check_host(h0, "h0", torch.float32)
+    _check_host(cu_seqlens, "cu_seqlens", torch.int32)
+    if bw:
+        _check_host(dO, "dO", io)
+        _check_host(dhT, "dhT", torch.float32)
+    B, T, Hqk, Hv, dk, dv, N = _dims(q, v, cu_seqlens)
+    scale = dk ** -0.5 if scale is None else float(scale)
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    pin = q.is_pinned()
+    out = dict(outputs) if outputs is not None else {}
+
+    def buf(name, shape, dtype, want=True):
+        if not want:
+            return None
+        t = out.get(name)
+        if t is None:
+            t = torch.empty(shape, dtype=dtype, pin_memory=pin)
+            out[name] = t
+        _check_host(t, name, dtype)
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must be {tuple(shape)}, got {tuple(t.shape)}")
+        return t
+
+    o = buf("o", (B, T, Hv, dv), io, fw)
+    hT = buf("hT", (N, Hv, dk, dv), torch.float32, fw and output_final_state)
+    dq = buf("dq", tuple(q.shape), io, bw)
+    dkk = buf("dk", tuple(k.shape), io, bw)
+    dvv = buf("dv", tuple(v.shape), io, bw)
+    dg = buf("dg", tuple(g.shape), torch.float32, bw)
+    db = buf("dbeta", tuple(beta.shape), io, bw)
+    dh0 = buf("dh0", (N, Hv, dk, dv), torch.float32, bw and want_dh0)
+    need = host_scratch_size(mode, io, B, T, Hqk, Hv, dk, dv, N, cp_segment_chunks, cp_exact, cp_mode, qk_l2norm)
+    if scratch is None:
+        scratch = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    elif not scratch.is_cuda or scratch.numel() * scratch.element_size() < need:
+        raise ValueError(f"scratch must be a CUDA tensor of at least {need} bytes")
+    opt = _opts(cp_segment_chunks, cp_exact, cp_mode=cp_mode, qk_l2norm=qk_l2norm)
+    st_main = torch.cuda.current_stream(device) if stream is None else stream
+    with torch.cuda.device(device):
+        st = lib().gdn_chunk_host(HOST_MODES[mode], _dtype_code(q), B, T, Hqk, Hv, dk, dv, _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(g), _ptr(beta), scale, _ptr(h0), _ptr(cu_seqlens), N,
+                                  _ptr(dO if bw else None), _ptr(dhT if bw else None), _ptr(o), _ptr(hT),
+                                  _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db), _ptr(dh0), _ptr(scratch),
+                                  scratch.numel() * scratch.element_size(), ctypes.byref(opt),
+                                  ctypes.c_void_p(st_main.cuda_stream),
+                                  ctypes.c_void_p(h2d_stream.cuda_stream if h2d_stream is not None else 0),
+                                  ctypes.c_void_p(d2h_stream.cuda_stream if d2h_stream is not None else 0))
+    if st != 0:
+        raise GdnError(st, "gdn_chunk_host")
+    if synchronize:
+        (d2h_stream if d2h_stream is not None else st_main).synchronize()
+    return out
 
 
 def gdn_recurrent_step(q, k, v, g, beta, state, scale=None, o=None, stream=None):

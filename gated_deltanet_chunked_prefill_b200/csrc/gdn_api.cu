@@ -2,6 +2,8 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "gdn_common.cuh"
 #include "gdn_tc.cuh"
@@ -228,6 +230,93 @@ BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
   return b;
 }
 
+}  // namespace
+
+namespace {
+// ---- host-buffer calls (gdn_chunk_host)
+
+// Scratch layout: device copies of every input and output, then the chunk-state cache (forward +
+// backward) and the workspaces, each 256-byte aligned. Offsets in bytes from the scratch base;
+// n_* are array sizes in bytes.
+struct HostLayout {
+  size_t q = 0, k = 0, v = 0, g = 0, beta = 0, h0 = 0, cu = 0, dO = 0, dhT = 0;
+  size_t o = 0, hT = 0, dq = 0, dk = 0, dv = 0, dg = 0, dbeta = 0, dh0 = 0;
+  size_t states = 0, ws_f = 0, ws_b = 0;
+  size_t n_qk = 0, n_v = 0, n_g = 0, n_beta = 0, n_h = 0, n_cu = 0;
+  size_t ws_f_bytes = 0, ws_b_bytes = 0, total = 0;
+};
+
+HostLayout host_layout(gdn_dtype dtype, const Shape& s, bool fw, bool bw, const gdn_options& op) {
+  HostLayout L;
+  const size_t es = dtype == GDN_F32 ? 4 : 2;
+  const size_t tok = (size_t)s.B * s.T;
+  L.n_qk = tok * s.Hqk * s.dk * es;
+  L.n_v = tok * s.Hv * s.dv * es;
+  L.n_g = tok * s.Hv * sizeof(float);
+  L.n_beta = tok * s.Hv * es;
+  L.n_h = (size_t)s.N * s.Hv * s.dk * s.dv * sizeof(float);
+  L.n_cu = (size_t)(s.N + 1) * sizeof(int32_t);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.q = take(L.n_qk); L.k = take(L.n_qk); L.v = take(L.n_v); L.g = take(L.n_g); L.beta = take(L.n_beta);
+  L.h0 = take(L.n_h); L.cu = take(L.n_cu);
+  if (bw) { L.dO = take(L.n_v); L.dhT = take(L.n_h); }
+  if (fw) { L.o = take(L.n_v); L.hT = take(L.n_h); }
+  if (bw) {
+    L.dq = take(L.n_qk); L.dk = take(L.n_qk); L.dv = take(L.n_v); L.dg = take(L.n_g); L.dbeta = take(L.n_beta);
+    L.dh0 = take(L.n_h);
+  }
+  gdn_options plan_opt = op;
+  plan_opt.states = nullptr;
+  if (fw && bw) {
+    L.states = take(cache_states_bytes(s) + cache_a_bytes(s) + cache_p_bytes(s));
+    plan_opt.states = &L;           // the backward plans without its own state pass (only non-null matters)
+  }
+  if (fw) { L.ws_f_bytes = plan_forward(dtype, s, &plan_opt).total; L.ws_f = take(L.ws_f_bytes); }
+  if (bw) { L.ws_b_bytes = plan_backward(s, &plan_opt).total; L.ws_b = take(L.ws_b_bytes); }
+  L.total = off;
+  return L;
+}
+
+// Events that order calls sharing a scratch buffer, created on its first use on a device.
+struct HostEvents {
+  int device = -1;
+  bool used = false;                 // an earlier call recorded compute_done and out_done
+  cudaEvent_t in_fwd = nullptr, in_bwd = nullptr, fwd_done = nullptr, compute_done = nullptr, out_done = nullptr;
+};
+std::mutex g_host_mu;
+std::unordered_map<const void*, HostEvents>& host_event_map() {
+  static auto* m = new std::unordered_map<const void*, HostEvents>();   // lives as long as the process
+  return *m;
+}
+
+gdn_status host_events(const void* scratch, HostEvents*& out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail("gdn_chunk_host: cudaGetDevice", err);
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostEvents& e = host_event_map()[scratch];
+  if (e.device != dev) {             // first use, or the address now belongs to another device
+    cudaEvent_t* evs[] = {&e.in_fwd, &e.in_bwd, &e.fwd_done, &e.compute_done, &e.out_done};
+    for (cudaEvent_t* ev : evs) {
+      if (*ev) cudaEventDestroy(*ev);
+      *ev = nullptr;
+    }
+    e.device = -1;
+    e.used = false;
+    for (cudaEvent_t* ev : evs) {
+      err = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+      if (err != cudaSuccess) return cuda_fail("gdn_chunk_host: cudaEventCreate", err);
+    }
+    e.device = dev;
+  }
+  out = &e;
+  return GDN_OK;
+}
 }  // namespace
 
 // The library's per-device status word (gdn_check_device_error): kernels record their first
@@ -595,6 +684,132 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   out.dk_part = bp.grouped ? reinterpret_cast<float*>(ws + bp.off_dk) : nullptr;
   err = launch_bwd_grad(p, out, bp.total_chunks, stream, &what);
   if (err != cudaSuccess) return cuda_fail(what, err);
+  return GDN_OK;
+}
+
+size_t gdn_chunk_host_scratch_size(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int Hqk, int Hv,
+                                   int dk, int dv, int num_seqs, const gdn_options* opt) {
+  if (mode != GDN_HOST_FWD && mode != GDN_HOST_BWD && mode != GDN_HOST_FWD_BWD) return 0;
+  if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
+  gdn_options op;
+  if (read_options(opt, op) != GDN_OK) return 0;
+  const bool fw = (mode & GDN_HOST_FWD) != 0, bw = (mode & GDN_HOST_BWD) != 0;
+  Shape s;
+  size_t total = 0;
+  if (check_shape(B, T, Hqk, Hv, dk, dv, 0, false, s) == GDN_OK) total = host_layout(dtype, s, fw, bw, op).total;
+  if (num_seqs > 0 && B == 1 && check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, true, s) == GDN_OK)
+    total = std::max(total, host_layout(dtype, s, fw, bw, op).total);
+  return total;
+}
+
+gdn_status gdn_chunk_host(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
+                          const void* q, const void* k, const void* v, const float* g, const void* beta,
+                          float scale, const float* h0, const int32_t* cu_seqlens, int num_seqs,
+                          const void* dO, const float* dhT, void* o, float* hT, void* dq, void* dk_out,
+                          void* dv_out, float* dg, void* dbeta, float* dh0, void* scratch, size_t scratch_bytes,
+                          const gdn_options* opt, cudaStream_t stream, cudaStream_t h2d_stream,
+                          cudaStream_t d2h_stream) {
+  // every check that the device calls below make, before the first copy is enqueued
+  if (mode != GDN_HOST_FWD && mode != GDN_HOST_BWD && mode != GDN_HOST_FWD_BWD) return GDN_ERR_INVALID_ARG;
+  if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+  Shape s;
+  gdn_status st = check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, cu_seqlens != nullptr, s);
+  if (st != GDN_OK) return st;
+  gdn_options op;
+  st = read_options(opt, op);
+  if (st != GDN_OK) return st;
+  if (op.states) return GDN_ERR_INVALID_ARG;       // the call keeps its own cache in the scratch
+  const bool fw = (mode & GDN_HOST_FWD) != 0, bw = (mode & GDN_HOST_BWD) != 0;
+  if (T > 0) {
+    if (!q || !k || !v || !g || !beta) return GDN_ERR_INVALID_ARG;
+    if (fw && !o) return GDN_ERR_INVALID_ARG;
+    if (bw && (!dO || !dq || !dk_out || !dv_out || !dg || !dbeta)) return GDN_ERR_INVALID_ARG;
+  }
+  if (bw && (!uses_tc(dtype, s) || !state_rows_fit(state_slots(s), s.Hv))) return GDN_ERR_UNSUPPORTED;
+  if (fw && op.qk_l2norm && !uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;
+  const HostLayout L = host_layout(dtype, s, fw, bw, op);
+  if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u) != 0 || scratch_bytes < L.total)
+    return GDN_ERR_WORKSPACE;
+  if (s.T == 0) return GDN_OK;
+
+  HostEvents* ev = nullptr;
+  st = host_events(scratch, ev);
+  if (st != GDN_OK) return st;
+  uint8_t* sb = static_cast<uint8_t*>(scratch);
+  const cudaStream_t hs = h2d_stream ? h2d_stream : stream, ds = d2h_stream ? d2h_stream : stream;
+  cudaError_t err = cudaSuccess;
+  auto h2d = [&](size_t off, const void* src, size_t n) {
+    if (src && n && err == cudaSuccess) err = cudaMemcpyAsync(sb + off, src, n, cudaMemcpyHostToDevice, hs);
+  };
+  auto d2h = [&](void* dst, size_t off, size_t n) {
+    if (dst && n && err == cudaSuccess) err = cudaMemcpyAsync(dst, sb + off, n, cudaMemcpyDeviceToHost, ds);
+  };
+  auto record = [&](cudaEvent_t e, cudaStream_t on) {
+    if (err == cudaSuccess) err = cudaEventRecord(e, on);
+  };
+  auto wait = [&](cudaStream_t on, cudaEvent_t e) {
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(on, e, 0);
+  };
+  auto dev = [&](size_t off, const void* host_ptr) -> void* { return host_ptr ? sb + off : nullptr; };
+
+  // inputs in, once the previous call on this scratch has finished reading them; the forward's
+  // arrays first, so that it can start while dO, dhT are still coming in
+  if (ev->used) wait(hs, ev->compute_done);
+  h2d(L.q, q, L.n_qk);
+  h2d(L.k, k, L.n_qk);
+  h2d(L.v, v, L.n_v);
+  h2d(L.g, g, L.n_g);
+  h2d(L.beta, beta, L.n_beta);
+  h2d(L.h0, h0, L.n_h);
+  h2d(L.cu, cu_seqlens, s.packed ? L.n_cu : 0);
+  record(ev->in_fwd, hs);
+  if (bw) {
+    h2d(L.dO, dO, L.n_v);
+    h2d(L.dhT, dhT, L.n_h);
+    record(ev->in_bwd, hs);
+  }
+  // the kernels, once the previous call's output copies from this scratch are done
+  if (ev->used) wait(stream, ev->out_done);
+  wait(stream, ev->in_fwd);
+  if (err != cudaSuccess) return cuda_fail("gdn_chunk_host: enqueue", err);
+  const float* d_h0 = static_cast<const float*>(dev(L.h0, h0));
+  const int32_t* d_cu = static_cast<const int32_t*>(dev(L.cu, cu_seqlens));
+  gdn_options od = op;
+  if (fw) {
+    od.states = bw ? sb + L.states : nullptr;
+    st = gdn_chunk_fwd(dtype, B, T, Hqk, Hv, dk, dv, sb + L.q, sb + L.k, sb + L.v,
+                       reinterpret_cast<const float*>(sb + L.g), sb + L.beta, scale, d_h0, d_cu, num_seqs,
+                       sb + L.o, static_cast<float*>(dev(L.hT, hT)), sb + L.ws_f, L.ws_f_bytes, &od, stream);
+    if (st != GDN_OK) return st;
+    record(ev->fwd_done, stream);
+    wait(ds, ev->fwd_done);                        // o, hT go back while the backward runs
+    d2h(o, L.o, L.n_v);
+    d2h(hT, L.hT, L.n_h);
+  }
+  if (bw) {
+    wait(stream, ev->in_bwd);
+    if (err != cudaSuccess) return cuda_fail("gdn_chunk_host: enqueue", err);
+    od.states = fw ? sb + L.states : nullptr;
+    st = gdn_chunk_bwd(dtype, B, T, Hqk, Hv, dk, dv, sb + L.q, sb + L.k, sb + L.v,
+                       reinterpret_cast<const float*>(sb + L.g), sb + L.beta, scale, d_h0, d_cu, num_seqs,
+                       sb + L.dO, static_cast<const float*>(dev(L.dhT, dhT)), sb + L.dq, sb + L.dk, sb + L.dv,
+                       reinterpret_cast<float*>(sb + L.dg), sb + L.dbeta, static_cast<float*>(dev(L.dh0, dh0)),
+                       sb + L.ws_b, L.ws_b_bytes, &od, stream);
+    if (st != GDN_OK) return st;
+  }
+  record(ev->compute_done, stream);
+  if (bw) {
+    wait(ds, ev->compute_done);
+    d2h(dq, L.dq, L.n_qk);
+    d2h(dk_out, L.dk, L.n_qk);
+    d2h(dv_out, L.dv, L.n_v);
+    d2h(dg, L.dg, L.n_g);
+    d2h(dbeta, L.dbeta, L.n_beta);
+    d2h(dh0, L.dh0, L.n_h);
+  }
+  record(ev->out_done, ds);
+  if (err != cudaSuccess) return cuda_fail("gdn_chunk_host: enqueue", err);
+  ev->used = true;
   return GDN_OK;
 }
 

@@ -234,6 +234,51 @@ gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int Hqk, int Hv,
                                  void* o, float* hT,
                                  const gdn_options* opt, cudaStream_t stream);
 
+/*
+ * Host-buffer calls: the forward and/or the backward on arrays in host memory, for callers
+ * whose data is not on the GPU (the pages' scenarios include on-device agentic inference,
+ * "FlashQLA resource", section 4). Every input is copied to the device, the same kernels as
+ * gdn_chunk_fwd / gdn_chunk_bwd run, and every output is copied back; the call enqueues all of
+ * it and returns (asynchronous to the calling thread).
+ *   mode GDN_HOST_FWD:     q k v g beta [h0] [cu_seqlens] -> o [hT]
+ *   mode GDN_HOST_BWD:     q k v g beta [h0] [cu_seqlens] dO [dhT] -> dq dk dv dg dbeta [dh0]
+ *                          (the forward pass is recomputed inside)
+ *   mode GDN_HOST_FWD_BWD: both, the backward reading the forward's chunk-state cache, which
+ *                          lives in the scratch.
+ * Arrays, shapes, dtypes and limits as in gdn_chunk_fwd / gdn_chunk_bwd; bracketed ones are
+ * nullable, unused ones are ignored. Host arrays need no alignment; page-locked memory
+ * (cudaHostAlloc, cudaHostRegister) lets the copies run asynchronously and overlap, pageable
+ * memory works but every copy then blocks the thread.
+ *   scratch  device memory of >= gdn_chunk_host_scratch_size() bytes, 256-byte aligned, owned
+ *            by the caller: the device copies of all arrays, the cache and the workspaces.
+ *   stream   the kernels.  h2d_stream / d2h_stream: the input / output copies (NULL: stream).
+ *            With three distinct streams and two scratch buffers used in turn, one call's
+ *            outputs go back while the next call's inputs come in.
+ * Ordering: a call's input copies wait for the kernels of the previous call on the same
+ * scratch, and its kernels wait for that call's output copies (the library keeps a few CUDA
+ * events per scratch address, created on its first use on the current device). The outputs are
+ * in host memory once d2h_stream (or stream) has passed the call. opt->states must be NULL
+ * (GDN_ERR_INVALID_ARG). Device-side findings go to the per-device status word
+ * (gdn_check_device_error). A failing CUDA call returns GDN_ERR_CUDA; copies already enqueued
+ * then still run.
+ */
+typedef enum { GDN_HOST_FWD = 1, GDN_HOST_BWD = 2, GDN_HOST_FWD_BWD = 3 } gdn_host_mode;
+
+/* Bytes of scratch gdn_chunk_host needs (0 for invalid sizes). With B == 1 and num_seqs >= 1 it
+ * covers both a packed call and a call without cu_seqlens. */
+size_t gdn_chunk_host_scratch_size(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int Hqk, int Hv,
+                                   int dk, int dv, int num_seqs, const gdn_options* opt);
+
+gdn_status gdn_chunk_host(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
+                          const void* q, const void* k, const void* v,
+                          const float* g, const void* beta, float scale,
+                          const float* h0, const int32_t* cu_seqlens, int num_seqs,
+                          const void* dO, const float* dhT,
+                          void* o, float* hT,
+                          void* dq, void* dk_out, void* dv_out, float* dg, void* dbeta, float* dh0,
+                          void* scratch, size_t scratch_bytes, const gdn_options* opt,
+                          cudaStream_t stream, cudaStream_t h2d_stream, cudaStream_t d2h_stream);
+
 /* Synchronises `stream`, then returns (and clears) the status word that the
  * kernels of earlier calls on this workspace recorded: GDN_OK,
  * GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_DEVICE_INPUT or GDN_ERR_DEVICE_LAUNCH.

@@ -257,3 +257,85 @@ def test_binding_refuses_mismatched_shapes():
     for name, bad_t in (("state", x["h0"][:, :1]), ("g", t["g"][:, :1]), ("k", t["k"][:1])):
         with pytest.raises(ValueError, match=name):
             step(**{name: bad_t})
+
+
+def _host(mode=3, dtype=1, B=1, T=64, Hqk=1, Hv=1, dk=128, dv=128, q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE,
+          h0=None, cu=None, N=1, dO=FAKE, dhT=None, o=FAKE, hT=None, dq=FAKE, dk_=FAKE, dv_=FAKE, dg=FAKE, db=FAKE,
+          dh0=None, scratch=FAKE, nbytes=1 << 40, opt=None):
+    L = gdn.lib()
+    o_ = gdn.Options() if opt is None else opt
+
+    def n(p):
+        return ctypes.c_void_p(p) if p else None
+    return L.gdn_chunk_host(mode, dtype, B, T, Hqk, Hv, dk, dv, n(q), n(k), n(v), n(g), n(beta), 0.1, n(h0), n(cu),
+                            N, n(dO), n(dhT), n(o), n(hT), n(dq), n(dk_), n(dv_), n(dg), n(db), n(dh0), n(scratch),
+                            nbytes, ctypes.byref(o_), None, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mode=0), 1), (dict(mode=4), 1), (dict(dtype=7), 1), (dict(B=0), 1), (dict(Hqk=3, Hv=4), 1),
+    (dict(dk=96), 2), (dict(q=None), 1), (dict(g=None), 1), (dict(mode=1, o=None), 1),
+    (dict(mode=2, dO=None), 1), (dict(mode=3, dq=None), 1), (dict(mode=2, dbeta_absent=True), 1),
+    (dict(mode=2, dtype=0), 2), (dict(mode=3, dk=64, dv=64), 2),
+    (dict(scratch=None), 3), (dict(scratch=FAKE + 16), 3), (dict(nbytes=1024), 3),
+    (dict(cu=FAKE, B=2, N=2), 1),
+])
+def test_host_call_rejects_invalid_arguments(kw, code):
+    """gdn_chunk_host validates everything before its first copy: these calls return at once
+    (a call that passed would need a GPU)."""
+    if kw.pop("dbeta_absent", False):
+        kw["db"] = None
+    assert _host(**kw) == code
+
+
+def test_host_call_refuses_a_states_option():
+    o = gdn.Options()
+    o.states = FAKE                  # the host call keeps its own chunk-state cache in the scratch
+    assert _host(opt=o) == 1
+    o = gdn.Options()
+    o.reserved[0] = 1
+    assert _host(opt=o) == 1
+
+
+def test_host_scratch_size():
+    """The scratch holds a device copy of every array of the mode (and, for forward + backward, the
+    chunk-state cache): it grows with the mode's arrays, covers the packed reading of B == 1, and is
+    0 for invalid sizes."""
+    L = gdn.lib()
+    opt = gdn.Options()
+
+    def size(mode, dims, dtype=1):
+        return int(L.gdn_chunk_host_scratch_size(mode, dtype, *dims, ctypes.byref(opt)))
+    dims = (2, 1024, 2, 4, 128, 128, 2)
+    B, T, Hqk, Hv, dk, dv, N = dims
+    inputs = 2 * B * T * Hqk * dk * 2 + B * T * Hv * dv * 2 + B * T * Hv * 6
+    f, b, fb = size(1, dims), size(2, dims), size(3, dims)
+    assert f >= inputs + B * T * Hv * dv * 2 and f % 256 == 0
+    assert b >= inputs + B * T * Hv * dv * 2 + inputs          # dO in, the gradients out
+    assert fb > f and fb > b - gdn.bwd_workspace_size(*dims)
+    states = int(L.gdn_chunk_states_size(*dims))
+    assert fb >= f + states
+    # B == 1 with num_seqs: covers 24 packed sequences as well as one unpacked one
+    packed = (1, 65536, 16, 16, 128, 128, 24)
+    assert size(3, packed) >= size(3, packed[:6] + (0,))
+    assert size(3, (0, 64, 1, 1, 128, 128, 1)) == 0
+    assert size(5, dims) == 0
+    assert size(1, dims, dtype=0) > 0 and size(2, dims, dtype=0) > 0
+
+
+def test_host_binding_checks():
+    """The binding refuses non-host, mistyped or misshapen arrays before calling the C ABI."""
+    q = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
+    v = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
+    g = torch.zeros(1, 64, 1)
+    beta = torch.zeros(1, 64, 1, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        gdn.gdn_chunk_host(q, q, v, g.double(), beta)
+    with pytest.raises(ValueError):
+        gdn.gdn_chunk_host(q, q, v, g, beta, mode="bwd")            # no dO
+    with pytest.raises(ValueError):
+        gdn.gdn_chunk_host(q, q, v, g, beta, mode="sideways")
+    with pytest.raises(ValueError):
+        gdn.gdn_chunk_host(q[:, ::2], q[:, ::2], v[:, ::2], g[:, ::2], beta[:, ::2])   # not contiguous
+    with pytest.raises(ValueError):
+        gdn.gdn_chunk_host(q, q, v, g, beta, dO=torch.zeros(1, 64, 2, 128, dtype=torch.bfloat16))
