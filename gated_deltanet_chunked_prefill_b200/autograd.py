@@ -23,7 +23,13 @@ __all__ = ["chunk_gated_delta_rule", "backward_supported"]
 
 
 def backward_supported(q: torch.Tensor, v: torch.Tensor) -> bool:
-    """The backward runs on the tensor-core path only: bf16 with dk = dv = 128."""
+    """The backward takes what the forward takes: bf16 or fp32 with dk, dv in {64, 128} (tensor cores
+    for bf16 with dk = dv = 128, CUDA cores otherwise)."""
+    return q.dtype in (torch.bfloat16, torch.float32) and q.shape[-1] in (64, 128) and v.shape[-1] in (64, 128)
+
+
+def _tensor_core_path(q: torch.Tensor, v: torch.Tensor) -> bool:
+    """bf16 with dk = dv = 128: the path whose forward can keep a chunk-state cache for its backward."""
     return q.dtype == torch.bfloat16 and q.shape[-1] == 128 and v.shape[-1] == 128
 
 
@@ -31,7 +37,7 @@ class _ChunkGatedDeltaRule(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, g, beta, scale, initial_state, output_final_state, cu_seqlens,
                 cp_segment_chunks, needs_grad, qk_l2norm):
-        states = chunk_states(q, v, cu_seqlens) if needs_grad else None
+        states = chunk_states(q, v, cu_seqlens) if needs_grad and _tensor_core_path(q, v) else None
         o, hT = gdn_chunk_fwd(q, k, v, g, beta, scale, initial_state, cu_seqlens,
                               output_final_state=output_final_state,
                               cp_segment_chunks=cp_segment_chunks, states=states, qk_l2norm=qk_l2norm)
@@ -81,8 +87,8 @@ def chunk_gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g:
     dk ** -0.5. Returns o [B,T,Hv,dv] and, if output_final_state, the final state
     [N,Hv,dk,dv] fp32, else None.
 
-    Gradients flow to q, k, v, g, beta and initial_state; the backward supports bf16 with
-    dk = dv = 128 (the forward supports dk, dv in {64, 128} in bf16 and fp32).
+    Gradients flow to q, k, v, g, beta and initial_state, for bf16 and fp32 with dk, dv in
+    {64, 128} (bf16 with dk = dv = 128 on tensor cores, the rest on CUDA cores).
     use_qk_l2norm_in_kernel: q and k rows are divided by sqrt(|x|^2 + 1e-6) inside the kernels
     (bf16, dk = dv = 128), and their gradients are taken through that normalisation. A cu_seqlens
     on the host is checked before it is copied to the device; one already on the device is not
@@ -105,7 +111,7 @@ def chunk_gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g:
         any(t.requires_grad for t in (q, k, v, g, beta))
         or (initial_state is not None and initial_state.requires_grad))
     if needs_grad and not backward_supported(q, v):
-        raise NotImplementedError("backward: bf16 with dk = dv = 128 only")
+        raise NotImplementedError("backward: bf16 or fp32 with dk, dv in {64, 128}")
     return _ChunkGatedDeltaRule.apply(q, k, v, g, beta, scale, initial_state, output_final_state,
                                       cu_seqlens, int(cp_segment_chunks), needs_grad,
                                       bool(use_qk_l2norm_in_kernel))

@@ -10,6 +10,10 @@
 
 namespace gdn {
 cudaError_t launch_fwd_simt(const FwdParams& p, bool bf16, cudaStream_t st);
+size_t bwd_simt_tok_bytes(int dk, int dv);
+cudaError_t launch_bwd_simt(const FwdParams& p, bool bf16, const void* dO, const float* dhT, void* dq, void* dk,
+                            float* dq_part, float* dk_part, void* dv, float* dg, void* dbeta, float* dh0,
+                            float* ckpt, float* tok, int grid, cudaStream_t st);
 }
 
 using namespace gdn;
@@ -197,6 +201,37 @@ size_t cache_a_bytes(const Shape& s) { return (size_t)state_slots(s) * s.Hv * kC
 // then the bf16 P = lower_incl(Q K^T * E) tile of every chunk slot (8 KB, swizzled as the operand)
 size_t cache_p_bytes(const Shape& s) { return (size_t)state_slots(s) * s.Hv * kChunk * kChunk * 2; }
 
+// The CUDA-core backward (fp32 I/O or head dims 64): fp32 state checkpoints every 64 tokens (the
+// cache's slot order), one 64-token block buffer per persistent CTA, and with grouped values the
+// per-v-head dq / dk partials.
+struct SimtBwdPlan {
+  int grid = 1;
+  size_t off_ckpt = 0, off_tok = 0, off_dq = 0, off_dk = 0, total = 0;
+};
+SimtBwdPlan plan_backward_simt(const Shape& s) {
+  SimtBwdPlan b;
+  const long long units = (long long)s.N * s.Hv;
+  b.grid = (int)std::max<long long>(1, std::min<long long>(units, num_sms()));
+  size_t off = kStatusBytes;
+  b.off_ckpt = off;
+  off = align256(off + (size_t)state_slots(s) * s.Hv * s.dk * s.dv * sizeof(float));
+  b.off_tok = off;
+  off = align256(off + (size_t)b.grid * bwd_simt_tok_bytes(s.dk, s.dv));
+  if (s.Hv != s.Hqk) {
+    const size_t part = (size_t)s.B * s.T * s.Hv * s.dk * sizeof(float);
+    b.off_dq = off;
+    off = align256(off + part);
+    b.off_dk = off;
+    off = align256(off + part);
+  }
+  b.total = off;
+  return b;
+}
+
+// Workspace of gdn_chunk_bwd for one reading of the shape: the tensor-core plan (bf16, dk = dv = 128)
+// and, without a chunk-state cache, the CUDA-core plan (the size query does not know the dtype).
+size_t bwd_workspace_for(const Shape& s, const gdn_options* opt);
+
 struct BwdPlan {
   FwdPlan chain;                 // gate-driven segments (or none) for the two sequential passes
   long long total_chunks = 0;    // chunk slots (upper bound for packed sequences)
@@ -228,6 +263,13 @@ BwdPlan plan_backward(const Shape& s, const gdn_options* opt) {
   }
   b.total = off;
   return b;
+}
+
+size_t bwd_workspace_for(const Shape& s, const gdn_options* opt) {
+  size_t total = kStatusBytes;
+  if (s.dk == 128 && s.dv == 128) total = plan_backward(s, opt).total;
+  if (!(opt && opt->states)) total = std::max(total, plan_backward_simt(s).total);
+  return total;
 }
 
 }  // namespace
@@ -551,9 +593,9 @@ size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int d
   // B == 1 with num_seqs >= 1 fits both a packed call and a call without cu_seqlens
   Shape s;
   size_t total = kStatusBytes;
-  if (check_shape(B, T, Hqk, Hv, dk, dv, 0, false, s) == GDN_OK) total = plan_backward(s, opt).total;
+  if (check_shape(B, T, Hqk, Hv, dk, dv, 0, false, s) == GDN_OK) total = bwd_workspace_for(s, opt);
   if (num_seqs > 0 && B == 1 && check_shape(B, T, Hqk, Hv, dk, dv, num_seqs, true, s) == GDN_OK)
-    total = std::max(total, plan_backward(s, opt).total);
+    total = std::max(total, bwd_workspace_for(s, opt));
   return total;
 }
 
@@ -577,7 +619,28 @@ gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk,
   const void* ptrs[] = {q, k, v, g, beta, h0, cu_seqlens, dO, dhT, dq, dk_out, dv_out, dg, dbeta, dh0, cached};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
-  if (!uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;   // backward: bf16, dk = dv = 128
+  if (!uses_tc(dtype, s)) {
+    // CUDA-core backward (fp32 I/O or head dims 64): no chunk-state cache, no in-kernel q/k
+    // normalisation on this path
+    if (cached || op.qk_l2norm) return GDN_ERR_UNSUPPORTED;
+    const SimtBwdPlan sp = plan_backward_simt(s);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < sp.total) return GDN_ERR_WORKSPACE;
+    if (s.T == 0) return GDN_OK;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    FwdParams p{};
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.h0 = h0; p.cu = cu_seqlens;
+    p.status = static_cast<int*>(workspace);
+    p.status_dev = device_status_word();
+    p.B = s.B; p.T = s.T; p.Hqk = s.Hqk; p.Hv = s.Hv; p.dk = s.dk; p.dv = s.dv; p.N = s.N;
+    p.scale = scale;
+    const bool grouped = s.Hv != s.Hqk;
+    const cudaError_t err = launch_bwd_simt(
+        p, dtype == GDN_BF16, dO, dhT, dq, dk_out, grouped ? reinterpret_cast<float*>(ws + sp.off_dq) : nullptr,
+        grouped ? reinterpret_cast<float*>(ws + sp.off_dk) : nullptr, dv_out, dg, dbeta, dh0,
+        reinterpret_cast<float*>(ws + sp.off_ckpt), reinterpret_cast<float*>(ws + sp.off_tok), sp.grid, stream);
+    if (err != cudaSuccess) return cuda_fail("gdn_chunk_bwd (CUDA-core path)", err);
+    return GDN_OK;
+  }
   if (!state_rows_fit(state_slots(s), s.Hv)) return GDN_ERR_UNSUPPORTED;
   const BwdPlan bp = plan_backward(s, opt);
   if (!workspace || !aligned16(workspace) || workspace_bytes < bp.total) return GDN_ERR_WORKSPACE;

@@ -1,0 +1,326 @@
+// CUDA-core backward of the GDN chunked prefill for the sizes the tensor-core kernels do not
+// take (fp32 I/O, head dims of 64): the exact token-level adjoint of the recurrence, per
+// (sequence, v-head), with the forward states recomputed from checkpoints.
+//
+//   forward, per token:  h~ = exp(g) h;  r = v - h~^T k;  h = h~ + beta k r^T   (h = S^T, dk x dv)
+//   adjoint, in reverse token order, with dh the adjoint of the state after the token:
+//     dh += scale q do^T;   dq = scale h do = scale (h~ do + beta k (r . do))
+//     dbeta = k^T dh r;     dr = beta dh^T k;   dv = dr
+//     dk = beta dh r - h~ dr;   dh~ = dh - k dr^T;   dg = <dh~, h~>;   dh <- exp(g) dh~
+// dh starts at dhT (or 0) and ends as dh0. This is the recurrence the pages' chunked kernels
+// evaluate ("Qwen's FlashQLA targets the expensive bit of long-context AI", "What happened";
+// "FlashQLA resource", section 3), differentiated token by token.
+//
+// A persistent CTA takes (sequence, v-head) units in turn. Phase 1 runs the sequence forward and
+// stores the state at every 64th token (fp32, one slot per 64-token block of every sequence, the
+// slot order of the chunk-state cache). Phase 2 walks the blocks backward: it recomputes the
+// block's h~ and r token by token into the CTA's own buffer, then runs the adjoint over them.
+// Shared memory holds h (or h~) and dh as [dk][dv + 1] (padded: conflict-free by column and by
+// row); threads take state columns (r < dv) in the column passes and rows (d < dk) in the row
+// passes. Every reduction runs in a fixed order (bit-reproducible).
+#include <algorithm>
+
+#include "gdn_common.cuh"
+
+namespace gdn {
+
+namespace {
+
+constexpr int kBwdSimtThreads = 128;
+constexpr int kBlk = 64;               // tokens between checkpoints
+
+struct BwdSimtArgs {
+  const void* dO;        // [B,T,Hv,dv] (IO)
+  const float* dhT;      // nullable [N,Hv,dk,dv]
+  void* dq;              // [B,T,Hqk,dk] (IO), written directly when Hv == Hqk
+  void* dk;
+  float* dq_part;        // [B,T,Hv,dk] fp32 per v-head when Hv > Hqk (summed afterwards), else null
+  float* dk_part;
+  void* dv;              // [B,T,Hv,dv] (IO)
+  float* dg;             // [B,T,Hv]
+  void* dbeta;           // [B,T,Hv] (IO)
+  float* dh0;            // nullable [N,Hv,dk,dv]
+  float* ckpt;           // [slots][Hv][dk][dv]: the state before every 64th token of each sequence
+  float* tok;            // per CTA: [64][dk][dv] h~ of the block's tokens, then [64][dv] their r
+};
+
+template <int DK, int DV>
+struct BwdSimtSmem {
+  static constexpr int kLd = DV + 1;
+  static constexpr int kFloats = 2 * DK * kLd + 2 * DK /*k, q*/ + 4 * DV /*v|do, r, dr, spare*/ +
+                                 2 * kBwdSimtThreads /*reductions*/ + 8;
+  static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+// sum of red[0 .. kBwdSimtThreads) in a fixed order (warp shuffles, then the warps' partials);
+// every thread returns the total. Called by all threads.
+__device__ __forceinline__ float block_sum(float x, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kBwdSimtThreads / 32; ++w) t += red[w];
+  __syncthreads();
+  return t;
+}
+
+__device__ __forceinline__ int block_sum_int(int x, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  int* ired = reinterpret_cast<int*>(red);
+  if (lane == 0) ired[warp] = x;
+  __syncthreads();
+  int t = 0;
+#pragma unroll
+  for (int w = 0; w < kBwdSimtThreads / 32; ++w) t += ired[w];
+  __syncthreads();
+  return t;
+}
+
+template <typename IO, int DK, int DV>
+__global__ void __launch_bounds__(kBwdSimtThreads)
+gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
+  constexpr int LD = BwdSimtSmem<DK, DV>::kLd;
+  extern __shared__ float sm[];
+  float* H = sm;                       // [DK][LD]  h, or h~ of the token being differentiated
+  float* DH = H + DK * LD;             // [DK][LD]  dh
+  float* ks = DH + DK * LD;            // [DK]
+  float* qs = ks + DK;                 // [DK]
+  float* vs = qs + DK;                 // [DV]  v (recompute) or do (adjoint)
+  float* rs = vs + DV;                 // [DV]  r
+  float* drs = rs + DV;                // [DV]  dr
+  float* red = drs + 2 * DV;           // reductions
+  float* scal = red + 2 * kBwdSimtThreads;   // g, beta of the token
+
+  const int tid = threadIdx.x;
+  const IO* q = static_cast<const IO*>(p.q);
+  const IO* k = static_cast<const IO*>(p.k);
+  const IO* v = static_cast<const IO*>(p.v);
+  const IO* dO = static_cast<const IO*>(a.dO);
+  const IO* beta = static_cast<const IO*>(p.beta);
+  const size_t S = (size_t)DK * DV;
+  float* tokh = a.tok + (size_t)blockIdx.x * (kBlk * S + kBlk * DV);   // this CTA's block buffer
+  float* tokr = tokh + kBlk * S;
+  const int units = p.N * p.Hv;
+  const int nblk_dense = (p.T + kBlk - 1) / kBlk;
+
+  for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    const int n = unit / p.Hv, j = unit % p.Hv;
+    const int hq = j / (p.Hv / p.Hqk);
+    int b, s, e;
+    if (!seq_span(p, n, b, s, e)) continue;          // uniform over the CTA
+    const int Tn = e - s;
+    // first checkpoint slot of sequence n (the chunk-state cache's slot order)
+    int slot0 = n * nblk_dense;
+    if (p.cu != nullptr) {
+      int part = 0;
+      for (int m = tid; m < n; m += kBwdSimtThreads) part += (p.cu[m + 1] - p.cu[m] + kBlk - 1) / kBlk;
+      slot0 = block_sum_int(part, red);
+    }
+    auto row_of = [&](int t) { return (size_t)b * p.T + s + t; };
+    auto load_token = [&](int t, bool adjoint) {
+      const size_t row = row_of(t);
+      for (int d = tid; d < DK; d += kBwdSimtThreads) {
+        ks[d] = to_f32(k[(row * p.Hqk + hq) * DK + d]);
+        if (adjoint) qs[d] = to_f32(q[(row * p.Hqk + hq) * DK + d]);
+      }
+      for (int r = tid; r < DV; r += kBwdSimtThreads)
+        vs[r] = to_f32(adjoint ? dO[(row * p.Hv + j) * DV + r] : v[(row * p.Hv + j) * DV + r]);
+      if (tid == 0) {
+        scal[0] = p.g[row * p.Hv + j];
+        scal[1] = to_f32(beta[row * p.Hv + j]);
+      }
+    };
+    // one forward token on H (column pass); with `keep`, h~ and r go to the block buffer at i
+    auto forward_token = [&](bool keep, int i) {
+      const float eg = __expf(scal[0]), bt = scal[1];
+      for (int r = tid; r < DV; r += kBwdSimtThreads) {
+        float u = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < DK; ++d) u = fmaf(H[d * LD + r], ks[d], u);
+        const float rr = vs[r] - eg * u;
+        if (keep) tokr[i * DV + r] = rr;
+#pragma unroll 8
+        for (int d = 0; d < DK; ++d) {
+          const float ht = eg * H[d * LD + r];
+          if (keep) tokh[(size_t)i * S + (size_t)d * DV + r] = ht;
+          H[d * LD + r] = fmaf(bt * ks[d], rr, ht);
+        }
+      }
+    };
+
+    // ---- phase 1: forward over the sequence, the state before every 64th token to its slot
+    for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads) {
+      const int d = idx / DV, r = idx % DV;
+      H[d * LD + r] = p.h0 ? p.h0[((size_t)unit * DK + d) * DV + r] : 0.f;
+    }
+    __syncthreads();
+    for (int t = 0; t < Tn; ++t) {
+      if (t % kBlk == 0) {
+        float* c = a.ckpt + ((size_t)(slot0 + t / kBlk) * p.Hv + j) * S;
+        for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads) c[idx] = H[(idx / DV) * LD + idx % DV];
+      }
+      load_token(t, false);
+      __syncthreads();
+      forward_token(false, 0);
+      __syncthreads();
+    }
+
+    // ---- phase 2: the adjoint, block by block from the end
+    for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads) {
+      const int d = idx / DV, r = idx % DV;
+      DH[d * LD + r] = a.dhT ? a.dhT[((size_t)unit * DK + d) * DV + r] : 0.f;
+    }
+    for (int blk = (Tn + kBlk - 1) / kBlk - 1; blk >= 0; --blk) {
+      const int t0 = blk * kBlk, nt = min(kBlk, Tn - t0);
+      __syncthreads();
+      const float* c = a.ckpt + ((size_t)(slot0 + blk) * p.Hv + j) * S;
+      for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads) H[(idx / DV) * LD + idx % DV] = c[idx];
+      __syncthreads();
+      for (int i = 0; i < nt; ++i) {               // recompute h~, r of the block's tokens
+        load_token(t0 + i, false);
+        __syncthreads();
+        forward_token(true, i);
+        __syncthreads();
+      }
+      for (int i = nt - 1; i >= 0; --i) {
+        const int t = t0 + i;
+        const size_t row = row_of(t);
+        load_token(t, true);
+        for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads)
+          H[(idx / DV) * LD + idx % DV] = tokh[(size_t)i * S + idx];
+        for (int r = tid; r < DV; r += kBwdSimtThreads) rs[r] = tokr[i * DV + r];
+        __syncthreads();
+        const float eg = __expf(scal[0]), bt = scal[1];
+        // dh += scale q do^T;  dr = beta dh^T k
+        for (int r = tid; r < DV; r += kBwdSimtThreads) {
+          const float dor = p.scale * vs[r];
+          float acc = 0.f;
+#pragma unroll 8
+          for (int d = 0; d < DK; ++d) {
+            const float x = fmaf(qs[d], dor, DH[d * LD + r]);
+            DH[d * LD + r] = x;
+            acc = fmaf(x, ks[d], acc);
+          }
+          drs[r] = bt * acc;
+        }
+        __syncthreads();
+        // rows: dq = scale (h~ do + beta k (r . do)), dk = beta dh r - h~ dr, dbeta = k^T dh r
+        float bpart = 0.f;
+        for (int d = tid; d < DK; d += kBwdSimtThreads) {
+          float w = 0.f, a1 = 0.f, a2 = 0.f, rd = 0.f;
+#pragma unroll 8
+          for (int r = 0; r < DV; ++r) {
+            const float hh = H[d * LD + r];
+            w = fmaf(DH[d * LD + r], rs[r], w);
+            a1 = fmaf(hh, vs[r], a1);
+            a2 = fmaf(hh, drs[r], a2);
+            rd = fmaf(rs[r], vs[r], rd);
+          }
+          const float dqv = p.scale * fmaf(bt * ks[d], rd, a1);
+          const float dkv = bt * w - a2;
+          bpart = fmaf(ks[d], w, bpart);
+          if (a.dq_part) {
+            a.dq_part[(row * p.Hv + j) * DK + d] = dqv;
+            a.dk_part[(row * p.Hv + j) * DK + d] = dkv;
+          } else {
+            static_cast<IO*>(a.dq)[(row * p.Hqk + hq) * DK + d] = from_f32<IO>(dqv);
+            static_cast<IO*>(a.dk)[(row * p.Hqk + hq) * DK + d] = from_f32<IO>(dkv);
+          }
+        }
+        const float dbeta = block_sum(bpart, red);
+        // columns: dh~ = dh - k dr^T;  dg = <dh~, h~>;  dh <- exp(g) dh~;  dv = dr
+        float gpart = 0.f;
+        for (int r = tid; r < DV; r += kBwdSimtThreads) {
+          const float drr = drs[r];
+#pragma unroll 8
+          for (int d = 0; d < DK; ++d) {
+            const float x = DH[d * LD + r] - ks[d] * drr;
+            gpart = fmaf(x, H[d * LD + r], gpart);
+            DH[d * LD + r] = eg * x;
+          }
+          static_cast<IO*>(a.dv)[(row * p.Hv + j) * DV + r] = from_f32<IO>(drr);
+        }
+        const float dg = block_sum(gpart, red);
+        if (tid == 0) {
+          a.dg[row * p.Hv + j] = dg;
+          static_cast<IO*>(a.dbeta)[row * p.Hv + j] = from_f32<IO>(dbeta);
+        }
+      }
+    }
+    __syncthreads();
+    if (a.dh0) {
+      for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads)
+        a.dh0[(size_t)unit * S + idx] = DH[(idx / DV) * LD + idx % DV];
+    }
+    __syncthreads();
+  }
+}
+
+// fp32 per-v-head partials of dq / dk -> the sum over the v-heads of each q/k head (fixed order)
+template <typename IO>
+__global__ void gdn_bwd_simt_reduce_kernel(const float* __restrict__ part, IO* __restrict__ out, long long rows,
+                                           int Hv, int Hqk, int dk) {
+  const int G = Hv / Hqk;
+  const long long total = rows * Hqk * dk;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int d = (int)(idx % dk);
+    const long long rh = idx / dk;
+    const int hq = (int)(rh % Hqk);
+    const long long row = rh / Hqk;
+    float acc = 0.f;
+    for (int jj = 0; jj < G; ++jj) acc += part[(row * Hv + hq * G + jj) * dk + d];
+    out[idx] = from_f32<IO>(acc);
+  }
+}
+
+template <typename IO, int DK, int DV>
+cudaError_t launch_typed(const FwdParams& p, const BwdSimtArgs& a, int grid, cudaStream_t st) {
+  constexpr size_t smem = BwdSimtSmem<DK, DV>::kBytes;
+  cudaError_t err = cudaFuncSetAttribute(gdn_bwd_simt_kernel<IO, DK, DV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  trace_pre(kKernBwdSimt, st);
+  gdn_bwd_simt_kernel<IO, DK, DV><<<grid, kBwdSimtThreads, smem, st>>>(p, a);
+  err = cudaGetLastError();
+  trace_post(st);
+  if (err != cudaSuccess || !a.dq_part) return err;
+  const long long rows = (long long)p.B * p.T;
+  const long long total = rows * p.Hqk * DK;
+  const int blocks = (int)std::min<long long>((total + 255) / 256, 4096);
+  trace_pre(kKernBwdReduce, st);
+  gdn_bwd_simt_reduce_kernel<IO><<<blocks, 256, 0, st>>>(a.dq_part, static_cast<IO*>(a.dq), rows, p.Hv, p.Hqk, DK);
+  gdn_bwd_simt_reduce_kernel<IO><<<blocks, 256, 0, st>>>(a.dk_part, static_cast<IO*>(a.dk), rows, p.Hv, p.Hqk, DK);
+  err = cudaGetLastError();
+  trace_post(st);
+  return err;
+}
+
+template <typename IO>
+cudaError_t launch_io(const FwdParams& p, const BwdSimtArgs& a, int grid, cudaStream_t st) {
+  if (p.dk == 64 && p.dv == 64) return launch_typed<IO, 64, 64>(p, a, grid, st);
+  if (p.dk == 64 && p.dv == 128) return launch_typed<IO, 64, 128>(p, a, grid, st);
+  if (p.dk == 128 && p.dv == 64) return launch_typed<IO, 128, 64>(p, a, grid, st);
+  return launch_typed<IO, 128, 128>(p, a, grid, st);
+}
+
+}  // namespace
+
+// Bytes of the per-CTA block buffer of the CUDA-core backward.
+size_t bwd_simt_tok_bytes(int dk, int dv) { return sizeof(float) * ((size_t)kBlk * dk * dv + (size_t)kBlk * dv); }
+
+// The CUDA-core backward: `grid` persistent CTAs (each with bwd_simt_tok_bytes of `tok`), then,
+// with grouped values, the dq / dk sums over the v-heads.
+cudaError_t launch_bwd_simt(const FwdParams& p, bool bf16, const void* dO, const float* dhT, void* dq, void* dk,
+                            float* dq_part, float* dk_part, void* dv, float* dg, void* dbeta, float* dh0,
+                            float* ckpt, float* tok, int grid, cudaStream_t st) {
+  BwdSimtArgs a{dO, dhT, dq, dk, dq_part, dk_part, dv, dg, dbeta, dh0, ckpt, tok};
+  return bf16 ? launch_io<__nv_bfloat16>(p, a, grid, st) : launch_io<float>(p, a, grid, st);
+}
+
+}  // namespace gdn

@@ -173,6 +173,10 @@ size_t gdn_chunk_bwd_workspace_size(int B, int T, int Hqk, int Hv, int dk, int d
  *   dbeta [B,T,Hv] (dtype), dh0 (nullable) [N,Hv,dk,dv] fp32.
  * Unless opt->states holds the chunk start states of the matching forward call
  * (see gdn_options.states), the forward pass is recomputed inside the call.
+ * bf16 with dk = dv = 128 runs on tensor cores. The other supported sizes (fp32, or a head
+ * dim of 64) run the exact token-level adjoint on CUDA cores, one (sequence, v-head) per CTA
+ * with the states recomputed from fp32 checkpoints every 64 tokens; that path takes neither
+ * opt->states nor opt->qk_l2norm (GDN_ERR_UNSUPPORTED).
  */
 gdn_status gdn_chunk_bwd(gdn_dtype dtype, int B, int T, int Hqk, int Hv, int dk, int dv,
                          const void* q, const void* k, const void* v,

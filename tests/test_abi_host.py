@@ -211,8 +211,10 @@ def test_autograd_entry_host_checks():
             _host_cu_seqlens(torch.tensor(bad), 10)
     from gated_deltanet_chunked_prefill_b200.autograd import backward_supported
     assert backward_supported(x.to(torch.bfloat16), x)
-    assert not backward_supported(x, x)                                   # fp32
-    assert not backward_supported(torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), x)   # dk = 64
+    assert backward_supported(x, x)                                       # fp32: CUDA-core backward
+    assert backward_supported(torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), x)       # dk = 64
+    assert not backward_supported(x.double(), x)
+    assert not backward_supported(torch.zeros(1, 64, 1, 96), x)           # dk = 96
 
 
 def test_recurrent_step_host_validation():
@@ -339,3 +341,31 @@ def test_host_binding_checks():
         gdn.gdn_chunk_host(q[:, ::2], q[:, ::2], v[:, ::2], g[:, ::2], beta[:, ::2])   # not contiguous
     with pytest.raises(ValueError):
         gdn.gdn_chunk_host(q, q, v, g, beta, dO=torch.zeros(1, 64, 2, 128, dtype=torch.bfloat16))
+
+
+def _bwd(dtype=1, B=1, T=64, Hqk=1, Hv=1, dk=128, dv=128, ws=FAKE, wsb=1 << 40, opt=None):
+    L = gdn.lib()
+    vp = ctypes.c_void_p
+    o_ = gdn.Options() if opt is None else opt
+    f = vp(FAKE)
+    return L.gdn_chunk_bwd(dtype, B, T, Hqk, Hv, dk, dv, f, f, f, f, f, 0.1, None, None, 1, f, None, f, f, f, f, f,
+                           None, vp(ws) if ws else None, wsb, ctypes.byref(o_), None)
+
+
+def test_backward_cuda_core_path_host_checks():
+    """fp32 or head dims 64 take the CUDA-core backward, which has neither the chunk-state cache nor
+    the in-kernel q/k normalisation; its workspace is checked against its own plan."""
+    o = gdn.Options()
+    o.states = FAKE
+    assert _bwd(dtype=0, opt=o) == 2
+    assert _bwd(dtype=1, dk=64, dv=64, opt=o) == 2
+    n = gdn.Options()
+    n.qk_l2norm = 1
+    assert _bwd(dtype=0, dk=64, dv=64, opt=n) == 2
+    assert _bwd(dtype=0, dk=64, dv=64, ws=None) == 3
+    assert _bwd(dtype=0, dk=64, dv=64, wsb=1024) == 3
+    assert _bwd(dtype=0, dk=96, dv=64) == 2
+    # the size query (no dtype) covers the CUDA-core plan: fp32 checkpoints every 64 tokens
+    per = 64 * 64 * 4
+    assert gdn.bwd_workspace_size(1, 256, 2, 2, 64, 64, 1) >= 4 * 2 * per
+    assert gdn.bwd_workspace_size(2, 8192, 16, 16, 128, 128, 2) >= 2 * 128 * 16 * 128 * 128 * 4

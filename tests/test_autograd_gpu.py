@@ -85,9 +85,10 @@ def test_autograd_without_final_state_or_h0_grad():
         assert torch.equal(gr[n], ref[r]), n
 
 
-def test_autograd_forward_only_paths():
-    """fp32 / head dim 64 run forward-only (no grad): equal to the C ABI; asking for grads is refused."""
-    x = make_inputs(1, 100, 1, 1, 64, 64, "f32", seed=74, h0_std=0.1)
+def test_autograd_cuda_core_paths():
+    """fp32 and head dim 64: the forward equals the C ABI, and the gradients (CUDA-core backward)
+    equal gdn_chunk_bwd's and match the oracle."""
+    x = make_inputs(1, 100, 1, 1, 64, 64, "f32", seed=74, h0_std=0.1, backward=True)
     d = to_dev(x)
     with torch.no_grad():
         o, hT = gdn.chunk_gated_delta_rule(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["h0"],
@@ -95,6 +96,13 @@ def test_autograd_forward_only_paths():
     o_ref, hT_ref = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, d["h0"])
     torch.cuda.synchronize()
     assert torch.equal(o, o_ref) and torch.equal(hT, hT_ref)
-    q = d["q"].clone().requires_grad_(True)
-    with pytest.raises(NotImplementedError):
-        gdn.chunk_gated_delta_rule(q, d["k"], d["v"], d["g"], d["beta"])
+    leaves = {n: d[n].clone().requires_grad_(True) for n in ("q", "k", "v", "g", "beta", "h0")}
+    o, hT = gdn.chunk_gated_delta_rule(leaves["q"], leaves["k"], leaves["v"], leaves["g"], leaves["beta"],
+                                       initial_state=leaves["h0"], output_final_state=True)
+    (o * d["dO"]).sum().add((hT * d["dhT"]).sum()).backward()
+    gr = gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], None, d["h0"], d["dhT"])
+    ref = bwd_token(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["dO"], x["h0"], x["dhT"])
+    torch.cuda.synchronize()
+    for n, gname in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("beta", "dbeta"), ("h0", "dh0")):
+        assert torch.equal(leaves[n].grad, gr[gname]), gname
+        assert_close(leaves[n].grad.cpu(), ref[gname], "f32", f"autograd fp32 {gname}")
