@@ -314,12 +314,15 @@ HostLayout host_layout(gdn_dtype dtype, const Shape& s, bool fw, bool bw, const 
   }
   gdn_options plan_opt = op;
   plan_opt.states = nullptr;
-  if (fw && bw) {
+  if (fw && bw && uses_tc(dtype, s)) {   // the cache exists on the tensor-core path only
     L.states = take(cache_states_bytes(s) + cache_a_bytes(s) + cache_p_bytes(s));
     plan_opt.states = &L;           // the backward plans without its own state pass (only non-null matters)
   }
   if (fw) { L.ws_f_bytes = plan_forward(dtype, s, &plan_opt).total; L.ws_f = take(L.ws_f_bytes); }
-  if (bw) { L.ws_b_bytes = plan_backward(s, &plan_opt).total; L.ws_b = take(L.ws_b_bytes); }
+  if (bw) {
+    L.ws_b_bytes = uses_tc(dtype, s) ? plan_backward(s, &plan_opt).total : plan_backward_simt(s).total;
+    L.ws_b = take(L.ws_b_bytes);
+  }
   L.total = off;
   return L;
 }
@@ -788,8 +791,8 @@ gdn_status gdn_chunk_host(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int
     if (fw && !o) return GDN_ERR_INVALID_ARG;
     if (bw && (!dO || !dq || !dk_out || !dv_out || !dg || !dbeta)) return GDN_ERR_INVALID_ARG;
   }
-  if (bw && (!uses_tc(dtype, s) || !state_rows_fit(state_slots(s), s.Hv))) return GDN_ERR_UNSUPPORTED;
-  if (fw && op.qk_l2norm && !uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;
+  if (bw && uses_tc(dtype, s) && !state_rows_fit(state_slots(s), s.Hv)) return GDN_ERR_UNSUPPORTED;
+  if (op.qk_l2norm && !uses_tc(dtype, s)) return GDN_ERR_UNSUPPORTED;
   const HostLayout L = host_layout(dtype, s, fw, bw, op);
   if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u) != 0 || scratch_bytes < L.total)
     return GDN_ERR_WORKSPACE;
@@ -838,8 +841,9 @@ gdn_status gdn_chunk_host(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int
   const float* d_h0 = static_cast<const float*>(dev(L.h0, h0));
   const int32_t* d_cu = static_cast<const int32_t*>(dev(L.cu, cu_seqlens));
   gdn_options od = op;
+  const bool cache = fw && bw && uses_tc(dtype, s);   // otherwise the backward recomputes its forward pass
   if (fw) {
-    od.states = bw ? sb + L.states : nullptr;
+    od.states = cache ? sb + L.states : nullptr;
     st = gdn_chunk_fwd(dtype, B, T, Hqk, Hv, dk, dv, sb + L.q, sb + L.k, sb + L.v,
                        reinterpret_cast<const float*>(sb + L.g), sb + L.beta, scale, d_h0, d_cu, num_seqs,
                        sb + L.o, static_cast<float*>(dev(L.hT, hT)), sb + L.ws_f, L.ws_f_bytes, &od, stream);
@@ -852,7 +856,7 @@ gdn_status gdn_chunk_host(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int
   if (bw) {
     wait(stream, ev->in_bwd);
     if (err != cudaSuccess) return cuda_fail("gdn_chunk_host: enqueue", err);
-    od.states = fw ? sb + L.states : nullptr;
+    od.states = cache ? sb + L.states : nullptr;
     st = gdn_chunk_bwd(dtype, B, T, Hqk, Hv, dk, dv, sb + L.q, sb + L.k, sb + L.v,
                        reinterpret_cast<const float*>(sb + L.g), sb + L.beta, scale, d_h0, d_cu, num_seqs,
                        sb + L.dO, static_cast<const float*>(dev(L.dhT, dhT)), sb + L.dq, sb + L.dk, sb + L.dv,

@@ -247,8 +247,9 @@ gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int Hqk, int Hv,
  *   mode GDN_HOST_FWD:     q k v g beta [h0] [cu_seqlens] -> o [hT]
  *   mode GDN_HOST_BWD:     q k v g beta [h0] [cu_seqlens] dO [dhT] -> dq dk dv dg dbeta [dh0]
  *                          (the forward pass is recomputed inside)
- *   mode GDN_HOST_FWD_BWD: both, the backward reading the forward's chunk-state cache, which
- *                          lives in the scratch.
+ *   mode GDN_HOST_FWD_BWD: both; on the tensor-core sizes (bf16, dk = dv = 128) the backward
+ *                          reads the forward's chunk-state cache, which lives in the scratch, and
+ *                          on the others it recomputes the forward pass.
  * Arrays, shapes, dtypes and limits as in gdn_chunk_fwd / gdn_chunk_bwd; bracketed ones are
  * nullable, unused ones are ignored. Host arrays need no alignment; page-locked memory
  * (cudaHostAlloc, cudaHostRegister) lets the copies run asynchronously and overlap, pageable

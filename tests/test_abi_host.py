@@ -278,7 +278,7 @@ def _host(mode=3, dtype=1, B=1, T=64, Hqk=1, Hv=1, dk=128, dv=128, q=FAKE, k=FAK
     (dict(mode=0), 1), (dict(mode=4), 1), (dict(dtype=7), 1), (dict(B=0), 1), (dict(Hqk=3, Hv=4), 1),
     (dict(dk=96), 2), (dict(q=None), 1), (dict(g=None), 1), (dict(mode=1, o=None), 1),
     (dict(mode=2, dO=None), 1), (dict(mode=3, dq=None), 1), (dict(mode=2, dbeta_absent=True), 1),
-    (dict(mode=2, dtype=0), 2), (dict(mode=3, dk=64, dv=64), 2),
+    (dict(mode=2, dtype=0, opt_l2=True), 2), (dict(mode=1, dk=64, dv=64, opt_l2=True), 2),
     (dict(scratch=None), 3), (dict(scratch=FAKE + 16), 3), (dict(nbytes=1024), 3),
     (dict(cu=FAKE, B=2, N=2), 1),
 ])
@@ -287,6 +287,9 @@ def test_host_call_rejects_invalid_arguments(kw, code):
     (a call that passed would need a GPU)."""
     if kw.pop("dbeta_absent", False):
         kw["db"] = None
+    if kw.pop("opt_l2", False):                # the normalisation: tensor-core sizes only
+        kw["opt"] = gdn.Options()
+        kw["opt"].qk_l2norm = 1
     assert _host(**kw) == code
 
 

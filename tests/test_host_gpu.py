@@ -120,3 +120,36 @@ def test_host_call_reuses_output_buffers():
     ref = _device_results(x2, "fwdbwd")
     for k, v in ref.items():
         assert torch.equal(out2[k], v), k
+
+
+def test_host_call_passes_options():
+    """Options reach the kernels unchanged: q/k normalisation and an explicit segment length give
+    the device calls' results bit for bit."""
+    x = make_inputs(1, 900, 2, 2, 128, 128, "bf16", seed=601, h0_std=0.1, backward=True, qk_unit=False)
+    h = _host_args(x)
+    got = _host_call(h, "fwdbwd", qk_l2norm=True, cp_segment_chunks=3)
+    d = to_dev(x)
+    states = gdn.chunk_states(d["q"], d["v"], d["cu_seqlens"])
+    o, hT = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"], d["cu_seqlens"],
+                              states=states, qk_l2norm=True, cp_segment_chunks=3)
+    gr = gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["scale"], d["h0"], d["dhT"],
+                           d["cu_seqlens"], states=states, qk_l2norm=True, cp_segment_chunks=3)
+    torch.cuda.synchronize()
+    ref = dict(o=o, hT=hT, **gr)
+    for k, v in ref.items():
+        if v is not None:
+            assert torch.equal(got[k], v.cpu()), k
+
+
+def test_host_call_cuda_core_sizes():
+    """fp32 with head dims 64 through the host entry: the CUDA-core forward and backward."""
+    x = make_inputs(1, 0, 1, 2, 64, 64, "f32", seed=611, h0_std=0.1, lengths=[100, 1, 64], backward=True)
+    got = _host_call(_host_args(x), "fwdbwd")
+    d = to_dev(x)
+    o, hT = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["scale"], d["h0"], d["cu_seqlens"])
+    gr = gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], d["scale"], d["h0"], d["dhT"],
+                           d["cu_seqlens"])
+    torch.cuda.synchronize()
+    ref = dict(o=o, hT=hT, **gr)
+    for k, v in ref.items():
+        assert torch.equal(got[k], v.cpu()), k
