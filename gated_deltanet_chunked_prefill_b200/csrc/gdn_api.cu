@@ -331,6 +331,7 @@ HostLayout host_layout(gdn_dtype dtype, const Shape& s, bool fw, bool bw, const 
 struct HostEvents {
   int device = -1;
   bool used = false;                 // an earlier call recorded compute_done and out_done
+  int in_use = 0;                    // calls enqueuing on these events right now (never swept then)
   cudaEvent_t in_fwd = nullptr, in_bwd = nullptr, fwd_done = nullptr, compute_done = nullptr, out_done = nullptr;
 };
 std::mutex g_host_mu;
@@ -339,11 +340,42 @@ std::unordered_map<const void*, HostEvents>& host_event_map() {
   return *m;
 }
 
+// A scratch address whose recorded work has all completed needs no ordering any more: its events
+// can go. Swept when the table grows past a few dozen addresses (a caller that allocates a new
+// scratch for every call would otherwise grow it without bound).
+bool host_events_idle(const HostEvents& e) {
+  cudaEvent_t evs[] = {e.in_fwd, e.in_bwd, e.fwd_done, e.compute_done, e.out_done};
+  for (cudaEvent_t ev : evs) {
+    const cudaError_t q = ev ? cudaEventQuery(ev) : cudaSuccess;
+    if (q != cudaSuccess) {
+      cudaGetLastError();            // not ready (or never recorded on this device): keep it
+      return false;
+    }
+  }
+  return true;
+}
+void host_events_sweep(const void* keep) {
+  auto& m = host_event_map();
+  if (m.size() <= 64) return;
+  for (auto it = m.begin(); it != m.end();) {
+    if (it->first != keep && it->second.in_use == 0 && host_events_idle(it->second)) {
+      cudaEvent_t evs[] = {it->second.in_fwd, it->second.in_bwd, it->second.fwd_done, it->second.compute_done,
+                           it->second.out_done};
+      for (cudaEvent_t ev : evs)
+        if (ev) cudaEventDestroy(ev);
+      it = m.erase(it);
+    } else {
+      ++it;
+    }
+  }
+}
+
 gdn_status host_events(const void* scratch, HostEvents*& out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return cuda_fail("gdn_chunk_host: cudaGetDevice", err);
   std::lock_guard<std::mutex> lock(g_host_mu);
+  host_events_sweep(scratch);
   HostEvents& e = host_event_map()[scratch];
   if (e.device != dev) {             // first use, or the address now belongs to another device
     cudaEvent_t* evs[] = {&e.in_fwd, &e.in_bwd, &e.fwd_done, &e.compute_done, &e.out_done};
@@ -359,9 +391,21 @@ gdn_status host_events(const void* scratch, HostEvents*& out) {
     }
     e.device = dev;
   }
+  ++e.in_use;
   out = &e;
   return GDN_OK;
 }
+
+// Releases a scratch address's events at the end of the call that took them (host_events).
+struct HostEventsHold {
+  HostEvents* e = nullptr;
+  ~HostEventsHold() {
+    if (e) {
+      std::lock_guard<std::mutex> lock(g_host_mu);
+      --e->in_use;
+    }
+  }
+};
 }  // namespace
 
 // The library's per-device status word (gdn_check_device_error): kernels record their first
@@ -801,6 +845,7 @@ gdn_status gdn_chunk_host(gdn_host_mode mode, gdn_dtype dtype, int B, int T, int
   HostEvents* ev = nullptr;
   st = host_events(scratch, ev);
   if (st != GDN_OK) return st;
+  HostEventsHold hold{ev};
   uint8_t* sb = static_cast<uint8_t*>(scratch);
   const cudaStream_t hs = h2d_stream ? h2d_stream : stream, ds = d2h_stream ? d2h_stream : stream;
   cudaError_t err = cudaSuccess;

@@ -261,7 +261,8 @@ gdn_status gdn_chunk_fwd_noalloc(gdn_dtype dtype, int B, int T, int Hqk, int Hv,
  *            outputs go back while the next call's inputs come in.
  * Ordering: a call's input copies wait for the kernels of the previous call on the same
  * scratch, and its kernels wait for that call's output copies (the library keeps a few CUDA
- * events per scratch address, created on its first use on the current device). The outputs are
+ * events per scratch address, created on its first use on the current device; beyond 64
+ * addresses, those whose recorded work has completed are released). The outputs are
  * in host memory once d2h_stream (or stream) has passed the call. opt->states must be NULL
  * (GDN_ERR_INVALID_ARG). Device-side findings go to the per-device status word
  * (gdn_check_device_error). A failing CUDA call returns GDN_ERR_CUDA; copies already enqueued

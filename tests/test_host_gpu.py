@@ -153,3 +153,19 @@ def test_host_call_cuda_core_sizes():
     ref = dict(o=o, hT=hT, **gr)
     for k, v in ref.items():
         assert torch.equal(got[k], v.cpu()), k
+
+
+def test_host_call_many_scratch_buffers():
+    """A new scratch buffer per call (80 of them, all kept alive so their addresses differ): the
+    library's event table releases the idle ones past 64 addresses, and calls keep giving the
+    device calls' results, including one reusing the first buffer."""
+    x = make_inputs(1, 64, 1, 1, 128, 128, "bf16", seed=701, backward=True)
+    h = _host_args(x)
+    need = gdn.host_scratch_size("fwdbwd", torch.bfloat16, 1, 64, 1, 1, 128, 128, 1)
+    bufs = [torch.empty(need, dtype=torch.uint8, device="cuda") for _ in range(80)]
+    outs = [_host_call(h, "fwdbwd", scratch=b) for b in bufs]
+    outs.append(_host_call(h, "fwdbwd", scratch=bufs[0]))
+    ref = _device_results(x, "fwdbwd")
+    for out in (outs[0], outs[70], outs[-1]):
+        for k, v in ref.items():
+            assert torch.equal(out[k], v), k
