@@ -212,6 +212,20 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int pt = threadIdx.x;
     PrepCtx pc{sbase, reinterpret_cast<float*>(sm + kOffLf), &ss->cs, tmem, kColG, pt, warp, lane, kBarPrep};
     bool ok = true;
+    // g, beta of chunk k (0 past the segment's end), loaded one chunk ahead
+    auto load_gb = [&](int k, float& gv, float& bv) {
+      gv = 0.f;
+      bv = 0.f;
+      if (k >= nchunks) return;
+      const int t0 = it.s + chunk_of(k) * kChunk;
+      if (pt < kChunk && pt < min(kChunk, we - t0)) {
+        const size_t gi = (size_t)(it.b * p.T + t0 + pt) * p.Hv + it.j;
+        gv = p.g[gi];
+        bv = __bfloat162float(beta[gi]);
+      }
+    };
+    float gv_next = 0.f, bv_next = 0.f;
+    load_gb(0, gv_next, bv_next);
     for (int k = 0; k < nchunks; ++k) {
       const int s = k & 1;
       const int t0 = it.s + chunk_of(k) * kChunk;
@@ -220,12 +234,8 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       // A = (I + L)^-1 of this chunk, as the forward pass computed it (same arithmetic)
       prep_fetch_a(pc, p.chunk_a + (chunk_slot(p, it.n, (t0 - it.seq_s) / kChunk) * p.Hv + it.j) *
                                        (size_t)(kChunk * kChunk));
-      float gv = 0.f, bv = 0.f;
-      if (pt < kChunk && pt < nv) {
-        const size_t gi = (size_t)(it.b * p.T + t0 + pt) * p.Hv + it.j;
-        gv = p.g[gi];
-        bv = __bfloat162float(beta[gi]);
-      }
+      const float gv = gv_next, bv = bv_next;
+      load_gb(k + 1, gv_next, bv_next);
       ok = ok && mbar_wait(&ss->full[s], (k >> 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       // P = lower_incl(Q K^T * E) of this chunk from the forward pass (bf16 operand tile); its
