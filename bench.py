@@ -43,8 +43,8 @@ from gated_deltanet_chunked_prefill_b200.workloads import CONFIGS, make_inputs  
 METRIC = "GDN chunk fwd/bwd tokens/s and TFLOP/s on 1 B200; % of roofline"
 HEADLINE = ("varlen_bf16", "fwdbwd")
 # (workload, step) of the per-configuration entries; "bwd" = backward alone with the cache
-SUBS = [("tiny_fp32", "fwd"), ("dense_bf16", "fwd"), ("long_gqa_bf16", "fwd"), ("varlen_bf16", "fwd"),
-        ("bwd_bf16", "bwd")]
+SUBS = [("tiny_fp32", "fwd"), ("tiny_fp32", "bwd"), ("dense_bf16", "fwd"), ("long_gqa_bf16", "fwd"),
+        ("varlen_bf16", "fwd"), ("bwd_bf16", "bwd")]
 C = 64
 L2_BYTES = 126 * 1024 * 1024
 # datasheet peaks of a B200 (HGX), reported beside the measured ones
@@ -95,6 +95,8 @@ def kernel_alg_bytes(w):
         "gdn_bwd_chain_kernel": [2 * qk + vv + gb + st + st],
         # gradients: q k v dO g beta -> dq dk dv dg dbeta
         "gdn_bwd_grad_kernel": [2 * qk + 2 * vv + gb + 2 * qk + vv + gb],
+        # CUDA-core backward (fp32, head dims 64), one launch: q k v g beta h0 dO dhT -> dq dk dv dg dbeta dh0
+        "gdn_bwd_simt_kernel": [2 * qk + 2 * vv + gb + h0 + st + 2 * qk + vv + gb + st],
     }
 
 
@@ -424,7 +426,9 @@ class Case:
         self.hT = torch.empty((w.num_seqs, w.Hv, w.dk, w.dv), dtype=torch.float32, device=dev)
         self.ws_f = torch.zeros(gdn.fwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, cp),
                                 dtype=torch.uint8, device=dev)
-        self.states = gdn.chunk_states(d["q"], d["v"], d["cu_seqlens"]) if mode != "fwd" else None
+        # the chunk-state cache exists on the tensor-core sizes (bf16, dk = dv = 128) only
+        tc = w.dtype == "bf16" and w.dk == 128 and w.dv == 128
+        self.states = gdn.chunk_states(d["q"], d["v"], d["cu_seqlens"]) if mode != "fwd" and tc else None
         self.ws_b = None
         if mode != "fwd":
             self.ws_b = torch.zeros(gdn.bwd_workspace_size(w.B, w.T, w.Hqk, w.Hv, w.dk, w.dv, w.num_seqs, cp,

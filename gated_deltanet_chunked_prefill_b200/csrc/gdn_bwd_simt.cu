@@ -122,27 +122,52 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
       slot0 = block_sum_int(part, red);
     }
     auto row_of = [&](int t) { return (size_t)b * p.T + s + t; };
-    auto load_token = [&](int t, bool adjoint) {
+    // A token's inputs travel through registers one token ahead (every thread holds at most one
+    // element of k, q and v or do: DK, DV <= kBwdSimtThreads), so that their load latency overlaps
+    // the previous token's passes; publish() puts them in shared memory (the caller then syncs).
+    struct Tok {
+      float k, q, v, g, b;
+    };
+    static_assert(DK <= kBwdSimtThreads && DV <= kBwdSimtThreads, "one element per thread");
+    auto fetch = [&](int t, bool adjoint) {
+      Tok x{0.f, 0.f, 0.f, 0.f, 0.f};
+      if (t < 0 || t >= Tn) return x;
       const size_t row = row_of(t);
-      for (int d = tid; d < DK; d += kBwdSimtThreads) {
-        ks[d] = to_f32(k[(row * p.Hqk + hq) * DK + d]);
-        if (adjoint) qs[d] = to_f32(q[(row * p.Hqk + hq) * DK + d]);
+      if (tid < DK) {
+        x.k = to_f32(k[(row * p.Hqk + hq) * DK + tid]);
+        if (adjoint) x.q = to_f32(q[(row * p.Hqk + hq) * DK + tid]);
       }
-      for (int r = tid; r < DV; r += kBwdSimtThreads)
-        vs[r] = to_f32(adjoint ? dO[(row * p.Hv + j) * DV + r] : v[(row * p.Hv + j) * DV + r]);
+      if (tid < DV) x.v = to_f32(adjoint ? dO[(row * p.Hv + j) * DV + tid] : v[(row * p.Hv + j) * DV + tid]);
       if (tid == 0) {
-        scal[0] = p.g[row * p.Hv + j];
-        scal[1] = to_f32(beta[row * p.Hv + j]);
+        x.g = p.g[row * p.Hv + j];
+        x.b = to_f32(beta[row * p.Hv + j]);
+      }
+      return x;
+    };
+    auto publish = [&](const Tok& x, bool adjoint) {
+      if (tid < DK) {
+        ks[tid] = x.k;
+        if (adjoint) qs[tid] = x.q;
+      }
+      if (tid < DV) vs[tid] = x.v;
+      if (tid == 0) {
+        scal[0] = x.g;
+        scal[1] = x.b;
       }
     };
     // one forward token on H (column pass); with `keep`, h~ and r go to the block buffer at i
     auto forward_token = [&](bool keep, int i) {
       const float eg = __expf(scal[0]), bt = scal[1];
       for (int r = tid; r < DV; r += kBwdSimtThreads) {
-        float u = 0.f;
-#pragma unroll 8
-        for (int d = 0; d < DK; ++d) u = fmaf(H[d * LD + r], ks[d], u);
-        const float rr = vs[r] - eg * u;
+        float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
+#pragma unroll 4
+        for (int d = 0; d < DK; d += 4) {
+          u0 = fmaf(H[d * LD + r], ks[d], u0);
+          u1 = fmaf(H[(d + 1) * LD + r], ks[d + 1], u1);
+          u2 = fmaf(H[(d + 2) * LD + r], ks[d + 2], u2);
+          u3 = fmaf(H[(d + 3) * LD + r], ks[d + 3], u3);
+        }
+        const float rr = vs[r] - eg * ((u0 + u1) + (u2 + u3));
         if (keep) tokr[i * DV + r] = rr;
 #pragma unroll 8
         for (int d = 0; d < DK; ++d) {
@@ -159,12 +184,14 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
       H[d * LD + r] = p.h0 ? p.h0[((size_t)unit * DK + d) * DV + r] : 0.f;
     }
     __syncthreads();
+    Tok nx = fetch(0, false);
     for (int t = 0; t < Tn; ++t) {
       if (t % kBlk == 0) {
         float* c = a.ckpt + ((size_t)(slot0 + t / kBlk) * p.Hv + j) * S;
         for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads) c[idx] = H[(idx / DV) * LD + idx % DV];
       }
-      load_token(t, false);
+      publish(nx, false);
+      nx = fetch(t + 1, false);
       __syncthreads();
       forward_token(false, 0);
       __syncthreads();
@@ -181,16 +208,20 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
       const float* c = a.ckpt + ((size_t)(slot0 + blk) * p.Hv + j) * S;
       for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads) H[(idx / DV) * LD + idx % DV] = c[idx];
       __syncthreads();
+      nx = fetch(t0, false);
       for (int i = 0; i < nt; ++i) {               // recompute h~, r of the block's tokens
-        load_token(t0 + i, false);
+        publish(nx, false);
+        nx = fetch(i + 1 < nt ? t0 + i + 1 : -1, false);
         __syncthreads();
         forward_token(true, i);
         __syncthreads();
       }
+      nx = fetch(t0 + nt - 1, true);
       for (int i = nt - 1; i >= 0; --i) {
         const int t = t0 + i;
         const size_t row = row_of(t);
-        load_token(t, true);
+        publish(nx, true);
+        nx = fetch(i > 0 ? t - 1 : -1, true);
         for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads)
           H[(idx / DV) * LD + idx % DV] = tokh[(size_t)i * S + idx];
         for (int r = tid; r < DV; r += kBwdSimtThreads) rs[r] = tokr[i * DV + r];
@@ -199,14 +230,17 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
         // dh += scale q do^T;  dr = beta dh^T k
         for (int r = tid; r < DV; r += kBwdSimtThreads) {
           const float dor = p.scale * vs[r];
-          float acc = 0.f;
+          float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll 8
-          for (int d = 0; d < DK; ++d) {
-            const float x = fmaf(qs[d], dor, DH[d * LD + r]);
-            DH[d * LD + r] = x;
-            acc = fmaf(x, ks[d], acc);
+          for (int d = 0; d < DK; d += 2) {
+            const float x0 = fmaf(qs[d], dor, DH[d * LD + r]);
+            const float x1 = fmaf(qs[d + 1], dor, DH[(d + 1) * LD + r]);
+            DH[d * LD + r] = x0;
+            DH[(d + 1) * LD + r] = x1;
+            acc0 = fmaf(x0, ks[d], acc0);
+            acc1 = fmaf(x1, ks[d + 1], acc1);
           }
-          drs[r] = bt * acc;
+          drs[r] = bt * (acc0 + acc1);
         }
         __syncthreads();
         // rows: dq = scale (h~ do + beta k (r . do)), dk = beta dh r - h~ dr, dbeta = k^T dh r
@@ -237,12 +271,17 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
         float gpart = 0.f;
         for (int r = tid; r < DV; r += kBwdSimtThreads) {
           const float drr = drs[r];
+          float g0 = 0.f, g1 = 0.f;
 #pragma unroll 8
-          for (int d = 0; d < DK; ++d) {
-            const float x = DH[d * LD + r] - ks[d] * drr;
-            gpart = fmaf(x, H[d * LD + r], gpart);
-            DH[d * LD + r] = eg * x;
+          for (int d = 0; d < DK; d += 2) {
+            const float x0 = DH[d * LD + r] - ks[d] * drr;
+            const float x1 = DH[(d + 1) * LD + r] - ks[d + 1] * drr;
+            g0 = fmaf(x0, H[d * LD + r], g0);
+            g1 = fmaf(x1, H[(d + 1) * LD + r], g1);
+            DH[d * LD + r] = eg * x0;
+            DH[(d + 1) * LD + r] = eg * x1;
           }
+          gpart = g0 + g1;
           static_cast<IO*>(a.dv)[(row * p.Hv + j) * DV + r] = from_f32<IO>(drr);
         }
         const float dg = block_sum(gpart, red);
