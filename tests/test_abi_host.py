@@ -372,3 +372,12 @@ def test_backward_cuda_core_path_host_checks():
     per = 64 * 64 * 4
     assert gdn.bwd_workspace_size(1, 256, 2, 2, 64, 64, 1) >= 4 * 2 * per
     assert gdn.bwd_workspace_size(2, 8192, 16, 16, 128, 128, 2) >= 2 * 128 * 16 * 128 * 128 * 4
+
+
+def test_empty_inputs_succeed_before_any_device_work():
+    """T = 0 is a valid call that does nothing: the host-buffer entry and the CUDA-core backward
+    return GDN_OK after validation, before any device query or launch (this runs without a GPU)."""
+    assert _host(T=0) == 0
+    assert _host(mode=1, T=0, dtype=0, dk=64, dv=64) == 0
+    assert _bwd(dtype=0, dk=64, dv=64, T=0) == 0
+    assert _bwd(dtype=0, dk=64, dv=64, T=0, ws=None) == 3      # the workspace is still checked
