@@ -27,7 +27,7 @@ struct SimtSmem {
   static constexpr int kKs = kChunk * (DK + 1);
   static constexpr int kFloats = 2 * kKs + kChunk * kSimtSlice /*V*/ + DK * kSimtSlice /*h*/ +
                                  2 * kChunk * (kChunk + 1) /*L,P*/ + kChunk * kSimtSlice /*D*/ +
-                                 3 * kChunk /*gam, beta, exp(gam)*/;
+                                 4 * kChunk /*gam, beta, exp(gam), exp(gam_n - gam)*/;
   static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
 
@@ -55,6 +55,7 @@ gdn_fwd_simt_kernel(FwdParams p) {
   float* gam = Ds + kChunk * S;                    // [64]
   float* bet = gam + kChunk;                       // [64]
   float* eg = bet + kChunk;                        // [64] exp(gam)
+  float* egd = eg + kChunk;                        // [64] exp(gam_n - gam)
 
   const IO* q = static_cast<const IO*>(p.q);
   const IO* k = static_cast<const IO*>(p.k);
@@ -106,7 +107,10 @@ gdn_fwd_simt_kernel(FwdParams p) {
       gam[2 * tid + 1] = excl + a0 + a1;
     }
     __syncthreads();
-    if (tid < kChunk) eg[tid] = expf(gam[tid]);
+    if (tid < kChunk) {
+      eg[tid] = expf(gam[tid]);
+      egd[tid] = expf(gam[nv - 1] - gam[tid]);     // the state update's per-token factor
+    }
     // ---- L (strictly lower) and P (lower incl. diagonal)
     for (int idx = tid; idx < kChunk * kChunk; idx += kSimtThreads) {
       const int i = idx / kChunk, jj = idx % kChunk;
@@ -159,12 +163,11 @@ gdn_fwd_simt_kernel(FwdParams p) {
     __syncthreads();
     // ---- h' = exp(gam_n) h + (diag(exp(gam_n - gam)) K)^T D
     {
-      const float gn = gam[nv - 1];
-      const float egn = expf(gn);
+      const float egn = expf(gam[nv - 1]);
       for (int idx = tid; idx < DK * S; idx += kSimtThreads) {
         const int d = idx / S, c = idx % S;
         float acc = 0.f;
-        for (int t = 0; t < nv; ++t) acc += expf(gn - gam[t]) * Ks[t * (DK + 1) + d] * Ds[t * S + c];
+        for (int t = 0; t < nv; ++t) acc += egd[t] * Ks[t * (DK + 1) + d] * Ds[t * S + c];
         Hs[idx] = egn * Hs[idx] + acc;
       }
     }
