@@ -137,7 +137,9 @@ gdn_fwd_simt_kernel(FwdParams p) {
       Ds[idx] = bet[i] * (Vs[idx] - eg[i] * acc);       // diag(beta) Y
     }
     __syncthreads();
-    // ---- forward substitution (I + L) D = diag(beta) Y, row by row; 8 partial sums per column
+    // ---- forward substitution (I + L) D = diag(beta) Y, row by row; 8 partial sums per column.
+    //      A column's 8 lanes sit in one warp and rows only read earlier rows of their own column,
+    //      so the warps run their columns independently (warp-level ordering per row)
     {
       const int c = tid >> 3, part = tid & 7;
       for (int i = 1; i < kChunk; ++i) {
@@ -147,9 +149,10 @@ gdn_fwd_simt_kernel(FwdParams p) {
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
         acc += __shfl_xor_sync(0xffffffffu, acc, 4);
         if (part == 0) Ds[i * S + c] -= acc;
-        __syncthreads();
+        __syncwarp();
       }
     }
+    __syncthreads();
     // ---- O = scale [diag(exp(gam)) Q h + P D]
     for (int idx = tid; idx < kChunk * S; idx += kSimtThreads) {
       const int i = idx / S, c = idx % S;
