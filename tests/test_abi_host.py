@@ -381,3 +381,33 @@ def test_empty_inputs_succeed_before_any_device_work():
     assert _host(mode=1, T=0, dtype=0, dk=64, dv=64) == 0
     assert _bwd(dtype=0, dk=64, dv=64, T=0) == 0
     assert _bwd(dtype=0, dk=64, dv=64, T=0, ws=None) == 3      # the workspace is still checked
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="the probe calls pass validation and would then run")
+@pytest.mark.parametrize("dims,packed", [((2, 300, 2, 4, 128, 128, 2), False), ((1, 700, 1, 2, 128, 128, 5), True),
+                                         ((1, 256, 2, 2, 64, 64, 1), False), ((1, 500, 1, 1, 64, 128, 3), True)])
+def test_size_queries_cover_their_calls(dims, packed):
+    """Every size query covers its call: given exactly the queried bytes, a call passes all of its
+    host checks and stops only at its first CUDA call (status GDN_ERR_CUDA here, on a machine
+    without a GPU), while one byte less is refused as GDN_ERR_WORKSPACE."""
+    L = gdn.lib()
+    B, T, Hqk, Hv, dk, dv, N = dims
+    cu = FAKE if packed else None
+    opt = gdn.Options()
+    for dtype in (0, 1):
+        for mode in (1, 2, 3):
+            need = int(L.gdn_chunk_host_scratch_size(mode, dtype, B, T, Hqk, Hv, dk, dv, N if packed else 0,
+                                                     ctypes.byref(opt)))
+            assert need > 0
+            assert _host(mode=mode, dtype=dtype, B=B, T=T, Hqk=Hqk, Hv=Hv, dk=dk, dv=dv, cu=cu, N=N,
+                         nbytes=need) == 4, (dtype, mode)
+            assert _host(mode=mode, dtype=dtype, B=B, T=T, Hqk=Hqk, Hv=Hv, dk=dk, dv=dv, cu=cu, N=N,
+                         nbytes=need - 1) == 3, (dtype, mode)
+        wsb = gdn.bwd_workspace_size(B, T, Hqk, Hv, dk, dv, N if packed else 0)
+        f = ctypes.c_void_p(FAKE)
+        args = lambda ws_bytes: (dtype, B, T, Hqk, Hv, dk, dv, f, f, f, f, f, 0.1, None, ctypes.c_void_p(cu) if cu else None,
+                                 N, f, None, f, f, f, f, f, None, f, ws_bytes, ctypes.byref(opt), None)
+        assert L.gdn_chunk_bwd(*args(wsb)) == 4, dtype
+        assert L.gdn_chunk_bwd(*args(16)) == 3, dtype
+        if dtype == 0 or dk != 128 or dv != 128:      # the query takes no dtype: it covers both backward plans
+            assert L.gdn_chunk_bwd(*args(wsb // 2)) == 3, dtype
