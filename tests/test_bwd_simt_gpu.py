@@ -44,6 +44,21 @@ def test_cuda_core_backward_parity(name):
         assert_close(got[n], ref[n], tol, f"{name} {n}")
 
 
+@pytest.mark.parametrize("name", ["fp32_d64", "bf16_d64_gqa", "fp32_d64_varlen"])
+def test_cuda_core_backward_weak_decay(name):
+    """g x 0.01: the adjoint carried back across many tokens keeps its weight (with the recipe's
+    decay it fades within a chunk), so every term of the reverse pass is exercised."""
+    B, T, Hqk, Hv, dk, dv, dtype, h0, lengths = CASES[name]
+    x = make_inputs(B, T, Hqk, Hv, dk, dv, dtype, seed=960 + len(name), h0_std=h0, lengths=lengths, backward=True)
+    x["g"] = x["g"] * 0.01
+    got = _run(x)
+    ref = bwd_token(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["dO"], x["h0"], x["dhT"],
+                    x["cu_seqlens"])
+    tol = "f32" if dtype == "f32" else "bf16"
+    for n in GRADS:
+        assert_close(got[n], ref[n], tol, f"{name} weak decay {n}")
+
+
 def test_cuda_core_backward_tiny_fp32_config_and_reproducible():
     """The tiny fp32 workload (B1 H2 T256 d64) end to end, twice: bit-identical results (every
     reduction in a fixed order)."""

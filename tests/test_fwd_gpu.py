@@ -45,6 +45,23 @@ def test_fwd_small_parity(name):
     assert_close(hT, rh, dt, f"{name} hT")
 
 
+@pytest.mark.parametrize("name", ["tiny_fp32_full", "f32_d128_ragged", "f32_d64_gqa_varlen", "bf16_d64"])
+def test_fwd_cuda_core_weak_decay(name):
+    """The CUDA-core sizes with g x 0.01. With the recipe's decay, entries of L and P more than a
+    dozen tokens below the diagonal fall under fp32 resolution, so a wrong long-range term would
+    go unseen; with mild decay every term of the chunk and the state carried across chunks
+    weigh in."""
+    B, T, Hqk, Hv, dk, dv, dt, h0, lengths = SMALL[name]
+    x = make_inputs(B, T, Hqk, Hv, dk, dv, dt, seed=zlib.crc32(name.encode()) % 1000 + 1, h0_std=h0,
+                    lengths=lengths)
+    x["g"] = x["g"] * 0.01
+    o, hT = run_gpu(x)
+    ro, rh = fwd_chunk(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"],
+                       x["cu_seqlens"], chunk=64)
+    assert_close(o, ro, dt, f"{name} weak decay o")
+    assert_close(hT, rh, dt, f"{name} weak decay hT")
+
+
 @pytest.mark.parametrize("exact", [False, True])
 @pytest.mark.parametrize("cp", [-1, 1, 2, 3])
 def test_fwd_context_parallel_matches_oracle(cp, exact):
