@@ -15,9 +15,11 @@
 // stores the state at every 64th token (fp32, one slot per 64-token block of every sequence, the
 // slot order of the chunk-state cache). Phase 2 walks the blocks backward: it recomputes the
 // block's h~ and r token by token into the CTA's own buffer, then runs the adjoint over them.
-// Shared memory holds h (or h~) and dh as [dk][dv + 1] (padded: conflict-free by column and by
-// row); threads take state columns (r < dv) in the column passes and rows (d < dk) in the row
-// passes. Every reduction runs in a fixed order (bit-reproducible).
+// Shared memory holds h (or h~) and dh as [dk][dv + 1] (padded). In the column passes four lanes
+// of a warp share each state column, each walking a quarter of its rows, and in the row passes
+// four lanes share each row; two xor shuffles combine the quarters. The block buffer keeps h~ in
+// thread order, so its writes are coalesced and each token's h~ is loaded into registers one
+// token ahead of its adjoint. Every reduction runs in a fixed order (bit-reproducible).
 #include <algorithm>
 
 #include "gdn_common.cuh"
@@ -26,7 +28,7 @@ namespace gdn {
 
 namespace {
 
-constexpr int kBwdSimtThreads = 128;
+constexpr int kBwdSimtThreads = 256;
 constexpr int kBlk = 64;               // tokens between checkpoints
 
 struct BwdSimtArgs {
@@ -81,10 +83,21 @@ __device__ __forceinline__ int block_sum_int(int x, float* red) {
   return t;
 }
 
+// Sum over the four lanes qg = lane >> 3 that share lane & 7 (two xor steps). Floating-point
+// addition is commutative, so all four lanes hold the same bits afterwards.
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 8);
+  x += __shfl_xor_sync(0xffffffffu, x, 16);
+  return x;
+}
+
 template <typename IO, int DK, int DV>
 __global__ void __launch_bounds__(kBwdSimtThreads)
 gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
   constexpr int LD = BwdSimtSmem<DK, DV>::kLd;
+  constexpr int NC = DV / 64;          // column sets of a thread in the column passes
+  constexpr int NR = DK / 64;          // row sets of a thread in the row passes
+  constexpr int NE = (DK / 4) * NC;    // state elements a thread owns in the column passes
   extern __shared__ float sm[];
   float* H = sm;                       // [DK][LD]  h, or h~ of the token being differentiated
   float* DH = H + DK * LD;             // [DK][LD]  dh
@@ -97,13 +110,22 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
   float* scal = red + 2 * kBwdSimtThreads;   // g, beta of the token
 
   const int tid = threadIdx.x;
+  // State-pass coordinates. Column passes: this thread's columns are cb + 64 cs (cs < NC) and
+  // its rows 4 i + qg (i < DK / 4); row passes swap the roles (rows cb + 64 s, s < NR; columns
+  // 4 i + qg). The four lanes qg of one column (row) are lanes (lane & 7) + 8 qg of one warp, and
+  // at every step the 32 lanes of a warp touch 32 distinct banks (LD = 1 mod 32).
+  const int lane = tid & 31, warp = tid >> 5;
+  const int qg = lane >> 3;
+  const int cb = (warp & 3) + 32 * (warp >> 2) + 4 * (lane & 7);
   const IO* q = static_cast<const IO*>(p.q);
   const IO* k = static_cast<const IO*>(p.k);
   const IO* v = static_cast<const IO*>(p.v);
   const IO* dO = static_cast<const IO*>(a.dO);
   const IO* beta = static_cast<const IO*>(p.beta);
   const size_t S = (size_t)DK * DV;
-  float* tokh = a.tok + (size_t)blockIdx.x * (kBlk * S + kBlk * DV);   // this CTA's block buffer
+  // this CTA's block buffer: h~ of each token in thread order (element e of thread tid at
+  // e * kBwdSimtThreads + tid, e = i * NC + cs for row 4 i + qg and column cb + 64 cs), then r
+  float* tokh = a.tok + (size_t)blockIdx.x * (kBlk * S + kBlk * DV);
   float* tokr = tokh + kBlk * S;
   const int units = p.N * p.Hv;
   const int nblk_dense = (p.T + kBlk - 1) / kBlk;
@@ -158,21 +180,22 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
     // one forward token on H (column pass); with `keep`, h~ and r go to the block buffer at i
     auto forward_token = [&](bool keep, int i) {
       const float eg = __expf(scal[0]), bt = scal[1];
-      for (int r = tid; r < DV; r += kBwdSimtThreads) {
-        float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
-#pragma unroll 4
-        for (int d = 0; d < DK; d += 4) {
-          u0 = fmaf(H[d * LD + r], ks[d], u0);
-          u1 = fmaf(H[(d + 1) * LD + r], ks[d + 1], u1);
-          u2 = fmaf(H[(d + 2) * LD + r], ks[d + 2], u2);
-          u3 = fmaf(H[(d + 3) * LD + r], ks[d + 3], u3);
+#pragma unroll
+      for (int cs = 0; cs < NC; ++cs) {
+        const int r = cb + 64 * cs;
+        float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+        for (int x = 0; x < DK / 4; x += 2) {
+          u0 = fmaf(H[(4 * x + qg) * LD + r], ks[4 * x + qg], u0);
+          u1 = fmaf(H[(4 * x + 4 + qg) * LD + r], ks[4 * x + 4 + qg], u1);
         }
-        const float rr = vs[r] - eg * ((u0 + u1) + (u2 + u3));
-        if (keep) tokr[i * DV + r] = rr;
-#pragma unroll 8
-        for (int d = 0; d < DK; ++d) {
+        const float rr = vs[r] - eg * quad_sum(u0 + u1);
+        if (keep && qg == 0) tokr[i * DV + r] = rr;
+#pragma unroll
+        for (int x = 0; x < DK / 4; ++x) {
+          const int d = 4 * x + qg;
           const float ht = eg * H[d * LD + r];
-          if (keep) tokh[(size_t)i * S + (size_t)d * DV + r] = ht;
+          if (keep) tokh[(size_t)i * S + (size_t)(x * NC + cs) * kBwdSimtThreads + tid] = ht;
           H[d * LD + r] = fmaf(bt * ks[d], rr, ht);
         }
       }
@@ -202,6 +225,13 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
       const int d = idx / DV, r = idx % DV;
       DH[d * LD + r] = a.dhT ? a.dhT[((size_t)unit * DK + d) * DV + r] : 0.f;
     }
+    float hnext[NE];                   // h~ of the next token to differentiate (own elements), and its r
+    float rnext = 0.f;
+    auto load_tok = [&](int i) {
+#pragma unroll
+      for (int x = 0; x < NE; ++x) hnext[x] = tokh[(size_t)i * S + (size_t)x * kBwdSimtThreads + tid];
+      if (tid < DV) rnext = tokr[i * DV + tid];
+    };
     for (int blk = (Tn + kBlk - 1) / kBlk - 1; blk >= 0; --blk) {
       const int t0 = blk * kBlk, nt = min(kBlk, Tn - t0);
       __syncthreads();
@@ -217,72 +247,93 @@ gdn_bwd_simt_kernel(const FwdParams p, const BwdSimtArgs a) {
         __syncthreads();
       }
       nx = fetch(t0 + nt - 1, true);
+      load_tok(nt - 1);
       for (int i = nt - 1; i >= 0; --i) {
         const int t = t0 + i;
         const size_t row = row_of(t);
         publish(nx, true);
         nx = fetch(i > 0 ? t - 1 : -1, true);
-        for (int idx = tid; idx < DK * DV; idx += kBwdSimtThreads)
-          H[(idx / DV) * LD + idx % DV] = tokh[(size_t)i * S + idx];
-        for (int r = tid; r < DV; r += kBwdSimtThreads) rs[r] = tokr[i * DV + r];
+#pragma unroll
+        for (int x = 0; x < NE; ++x) H[(4 * (x / NC) + qg) * LD + cb + 64 * (x % NC)] = hnext[x];
+        if (tid < DV) rs[tid] = rnext;
+        if (i > 0) load_tok(i - 1);                // in flight during this token's passes
         __syncthreads();
         const float eg = __expf(scal[0]), bt = scal[1];
-        // dh += scale q do^T;  dr = beta dh^T k
-        for (int r = tid; r < DV; r += kBwdSimtThreads) {
+        // columns: dh += scale q do^T;  dr = beta dh^T k
+#pragma unroll
+        for (int cs = 0; cs < NC; ++cs) {
+          const int r = cb + 64 * cs;
           const float dor = p.scale * vs[r];
           float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-          for (int d = 0; d < DK; d += 2) {
-            const float x0 = fmaf(qs[d], dor, DH[d * LD + r]);
-            const float x1 = fmaf(qs[d + 1], dor, DH[(d + 1) * LD + r]);
-            DH[d * LD + r] = x0;
-            DH[(d + 1) * LD + r] = x1;
-            acc0 = fmaf(x0, ks[d], acc0);
-            acc1 = fmaf(x1, ks[d + 1], acc1);
+#pragma unroll
+          for (int x = 0; x < DK / 4; x += 2) {
+            const int d0 = 4 * x + qg, d1 = d0 + 4;
+            const float x0 = fmaf(qs[d0], dor, DH[d0 * LD + r]);
+            const float x1 = fmaf(qs[d1], dor, DH[d1 * LD + r]);
+            DH[d0 * LD + r] = x0;
+            DH[d1 * LD + r] = x1;
+            acc0 = fmaf(x0, ks[d0], acc0);
+            acc1 = fmaf(x1, ks[d1], acc1);
           }
-          drs[r] = bt * (acc0 + acc1);
+          const float acc = quad_sum(acc0 + acc1);
+          if (qg == 0) drs[r] = bt * acc;
         }
         __syncthreads();
         // rows: dq = scale (h~ do + beta k (r . do)), dk = beta dh r - h~ dr, dbeta = k^T dh r
         float bpart = 0.f;
-        for (int d = tid; d < DK; d += kBwdSimtThreads) {
+#pragma unroll
+        for (int rsx = 0; rsx < NR; ++rsx) {
+          const int d = cb + 64 * rsx;
           float w = 0.f, a1 = 0.f, a2 = 0.f, rd = 0.f;
-#pragma unroll 8
-          for (int r = 0; r < DV; ++r) {
+#pragma unroll
+          for (int x = 0; x < DV / 4; ++x) {
+            const int r = 4 * x + qg;
             const float hh = H[d * LD + r];
             w = fmaf(DH[d * LD + r], rs[r], w);
             a1 = fmaf(hh, vs[r], a1);
             a2 = fmaf(hh, drs[r], a2);
             rd = fmaf(rs[r], vs[r], rd);
           }
-          const float dqv = p.scale * fmaf(bt * ks[d], rd, a1);
-          const float dkv = bt * w - a2;
-          bpart = fmaf(ks[d], w, bpart);
-          if (a.dq_part) {
-            a.dq_part[(row * p.Hv + j) * DK + d] = dqv;
-            a.dk_part[(row * p.Hv + j) * DK + d] = dkv;
-          } else {
-            static_cast<IO*>(a.dq)[(row * p.Hqk + hq) * DK + d] = from_f32<IO>(dqv);
-            static_cast<IO*>(a.dk)[(row * p.Hqk + hq) * DK + d] = from_f32<IO>(dkv);
+          w = quad_sum(w);
+          a1 = quad_sum(a1);
+          a2 = quad_sum(a2);
+          rd = quad_sum(rd);
+          if (qg == 0) {
+            const float dqv = p.scale * fmaf(bt * ks[d], rd, a1);
+            const float dkv = bt * w - a2;
+            bpart = fmaf(ks[d], w, bpart);
+            if (a.dq_part) {
+              a.dq_part[(row * p.Hv + j) * DK + d] = dqv;
+              a.dk_part[(row * p.Hv + j) * DK + d] = dkv;
+            } else {
+              static_cast<IO*>(a.dq)[(row * p.Hqk + hq) * DK + d] = from_f32<IO>(dqv);
+              static_cast<IO*>(a.dk)[(row * p.Hqk + hq) * DK + d] = from_f32<IO>(dkv);
+            }
           }
         }
         const float dbeta = block_sum(bpart, red);
         // columns: dh~ = dh - k dr^T;  dg = <dh~, h~>;  dh <- exp(g) dh~;  dv = dr
         float gpart = 0.f;
-        for (int r = tid; r < DV; r += kBwdSimtThreads) {
+#pragma unroll
+        for (int cs = 0; cs < NC; ++cs) {
+          const int r = cb + 64 * cs;
           const float drr = drs[r];
           float g0 = 0.f, g1 = 0.f;
-#pragma unroll 8
-          for (int d = 0; d < DK; d += 2) {
-            const float x0 = DH[d * LD + r] - ks[d] * drr;
-            const float x1 = DH[(d + 1) * LD + r] - ks[d + 1] * drr;
-            g0 = fmaf(x0, H[d * LD + r], g0);
-            g1 = fmaf(x1, H[(d + 1) * LD + r], g1);
-            DH[d * LD + r] = eg * x0;
-            DH[(d + 1) * LD + r] = eg * x1;
+#pragma unroll
+          for (int x = 0; x < DK / 4; x += 2) {
+            const int d0 = 4 * x + qg, d1 = d0 + 4;
+            const float x0 = DH[d0 * LD + r] - ks[d0] * drr;
+            const float x1 = DH[d1 * LD + r] - ks[d1] * drr;
+            g0 = fmaf(x0, H[d0 * LD + r], g0);
+            g1 = fmaf(x1, H[d1 * LD + r], g1);
+            DH[d0 * LD + r] = eg * x0;
+            DH[d1 * LD + r] = eg * x1;
           }
-          gpart = g0 + g1;
-          static_cast<IO*>(a.dv)[(row * p.Hv + j) * DV + r] = from_f32<IO>(drr);
+          const float gt = quad_sum(g0 + g1);
+          if (qg == 0) {
+            gpart += gt;
+            static_cast<IO*>(a.dv)[(row * p.Hv + j) * DV + r] = from_f32<IO>(drr);
+          }
         }
         const float dg = block_sum(gpart, red);
         if (tid == 0) {
