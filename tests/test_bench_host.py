@@ -62,3 +62,14 @@ def test_source_hash_ignores_comments(tmp_path, monkeypatch):
     assert bench.sources_sha(["k.cu"]) != h1
     assert bench.sources_sha(["missing.cu"]) is None
     assert os.path.exists(src)
+
+
+def test_cuda_core_kernel_bytes():
+    """The tiny fp32 workload (B1 H2 T256, dk = dv = 64, fp32, h0 = 0), by hand. Forward: q, k, v
+    and o at 256 x 2 x 64 x 4 = 131,072 B each, g and beta 256 x 2 x 8 = 4,096 B, hT 2 x 64 x 64 x 4
+    = 32,768 B: 561,152 B. Backward: q k v dO in, dq dk dv out (7 x 131,072), g beta in and dg dbeta
+    out (2 x 4,096), dhT in and dh0 out (2 x 32,768): 991,232 B."""
+    kb = bench.kernel_alg_bytes(CONFIGS["tiny_fp32"])
+    assert CONFIGS["tiny_fp32"].h0_std is None
+    assert kb["gdn_fwd_simt_kernel"] == [561152]
+    assert kb["gdn_bwd_simt_kernel"] == [991232]
