@@ -385,7 +385,9 @@ def test_empty_inputs_succeed_before_any_device_work():
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="the probe calls pass validation and would then run")
 @pytest.mark.parametrize("dims,packed", [((2, 300, 2, 4, 128, 128, 2), False), ((1, 700, 1, 2, 128, 128, 5), True),
-                                         ((1, 256, 2, 2, 64, 64, 1), False), ((1, 500, 1, 1, 64, 128, 3), True)])
+                                         ((1, 256, 2, 2, 64, 64, 1), False), ((1, 500, 1, 1, 64, 128, 3), True),
+                                         ((1, 1 << 20, 16, 16, 128, 128, 1), False),     # tens of GiB of scratch
+                                         ((1, 300000, 4, 8, 64, 128, 1000), True)])
 def test_size_queries_cover_their_calls(dims, packed):
     """Every size query covers its call: given exactly the queried bytes, a call passes all of its
     host checks and stops only at its first CUDA call (status GDN_ERR_CUDA here, on a machine
