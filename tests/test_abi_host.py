@@ -413,3 +413,18 @@ def test_size_queries_cover_their_calls(dims, packed):
         assert L.gdn_chunk_bwd(*args(16)) == 3, dtype
         if dtype == 0 or dk != 128 or dv != 128:      # the query takes no dtype: it covers both backward plans
             assert L.gdn_chunk_bwd(*args(wsb // 2)) == 3, dtype
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library every entry point raises: there is no CPU path to fall back to,
+    not even for the host-buffer entry, whose inputs are CPU tensors."""
+    from gated_deltanet_chunked_prefill_b200.workloads import make_inputs
+    monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "libgdn.so"))
+    monkeypatch.setattr(gdn, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        gdn.lib()
+    x = make_inputs(1, 64, 1, 1, 128, 128, "bf16", seed=1, backward=True)
+    with pytest.raises(RuntimeError, match="not built|NVIDIA driver"):   # whichever it meets first
+        gdn.gdn_chunk_host(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], None, None, mode="fwd")
+    with pytest.raises(Exception):
+        gdn.chunk_gated_delta_rule(x["q"], x["k"], x["v"], x["g"], x["beta"], scale=x["scale"])
