@@ -73,3 +73,31 @@ def test_cuda_core_kernel_bytes():
     assert CONFIGS["tiny_fp32"].h0_std is None
     assert kb["gdn_fwd_simt_kernel"] == [561152]
     assert kb["gdn_bwd_simt_kernel"] == [991232]
+
+
+def _bench(args, **env):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, cwd=root, capture_output=True,
+                       text=True, timeout=600, env={**os.environ, **env})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_line():
+    """`--impl reference` (the oracle on the host cores; no GPU needed) prints one line with the
+    GPU arm's metric, unit and direction, its own cpu_baseline and an e2e with no copies."""
+    (d,) = _bench(["--impl", "reference", "--steps", "1", "--warmup", "0"])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "tokens/s"
+    assert d["higher_is_better"] is True and d["value"] > 0 and d["steps"] == 1
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    """Under a multi-rank launch only rank 0 runs and prints the reference line."""
+    assert _bench(["--impl", "reference", "--steps", "1", "--warmup", "0"], RANK="1", WORLD_SIZE="2") == []
